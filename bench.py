@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""DF11 decode benchmark: decoded BF16 GB/s and fraction of the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl {b200,reference}]
+
+A step is one pass of the whole decode path over one workload: every tensor
+of it decoded from its resident compressed form into BF16 in HBM (one
+batched launch per 16 tensors).  The default workload is one Qwen3-8B-shaped
+transformer block (7 weights, 192,937,984 elements, one codebook each).
+Other workloads: single (1024x1024), adversarial (64M mix), fibonacci
+(32-bit codewords), embedding (151936x4096), stack (36 blocks + embedding +
+LM head, decoded block by block into one reused scratch buffer).
+
+Inputs are seeded synthetic tensors; every step's output is checked
+bit-exact against the original tensor before any number is printed.
+
+Multi-GPU (torchrun): every rank decodes its own copy of the workload (its
+own seed) -- the decode has no exchange step, so there is no collective on
+the data path; the timed region is bracketed by barriers and the time is the
+maximum over ranks.
+
+--impl reference times the CPU oracle (single-threaded C, bit-serial decode)
+on the host on the same workload and metric, as the comparison arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = ("decoded BF16 GB/s and % of HBM roofline (1×B200), "
+          "bit-exact vs CPU oracle")
+UNIT = "GB/s"
+KERNEL_SRC = os.path.join(ROOT, "huffman_decode_df11_b200", "csrc", "df11_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# workloads as lists of (name, thunk(device) -> int16 bits)
+
+def workload_units(config: str, seed: int):
+    if config == "single":
+        return [("w_1024x1024", lambda d: workloads.single_matrix(seed, d))]
+    if config == "block":
+        return [(name, (lambda d, i=i: workloads.block_tensor(seed, i, d)))
+                for i, (name, _, _) in enumerate(workloads.BLOCK_SHAPES)]
+    if config == "adversarial":
+        return [("adversarial_64M", lambda d: workloads.adversarial_mix(64 << 20, seed, d))]
+    if config == "fibonacci":
+        return [("fibonacci34", lambda d: workloads.fibonacci_exponents(seed, d))]
+    if config == "embedding":
+        return [("embed_151936x4096", lambda d: workloads.embedding(seed, d))]
+    if config == "stack":
+        return [(name, thunk) for name, _, thunk in workloads.stack_units(seed)]
+    raise ValueError(config)
+
+
+def block_groups(config: str, names):
+    """Groups of tensors decoded by one batched call (a layer at a time)."""
+    if config != "stack":
+        return [list(range(len(names)))]
+    groups, cur, layer = [], [], None
+    for i, n in enumerate(names):
+        key = n.split(".")[1] if n.startswith("layers.") else n
+        if key != layer and cur:
+            groups.append(cur)
+            cur = []
+        layer = key
+        cur.append(i)
+    groups.append(cur)
+    return groups
+
+
+def algorithmic_bytes(h) -> int:
+    """Bytes one decode of this tensor must move: compressed input (stream,
+    sign/mantissa, gaps, block positions, tables, code lengths) + 2 B/elem
+    of BF16 output."""
+    p = h.params
+    chunks = p.num_blocks * p.threads_per_block
+    return ((p.total_bits + 7) // 8 + p.n + (5 * chunks + 7) // 8 + 4 * (p.num_blocks + 1)
+            + 1024 * p.num_luts + 256 + 2 * p.n)
+
+
+def kernel_hash() -> str:
+    return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """Per-launch DRAM bytes from an ncu capture of the current kernel source
+    (profiles/dram_traffic.txt: '<kernel sha16> <workload> <bytes per launch>')."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    kh = kernel_hash()
+    for line in open(TRAFFIC_FILE):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == kh and parts[1] == workload:
+            return float(parts[2])
+    return None
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        try:
+            return float(json.load(open(path))["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+
+def setup_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def prepare(config: str, seed: int, device: str):
+    """Compress every unit on the host; keep compressed tensors resident in
+    HBM.  Originals are regenerated from the seed when checked."""
+    import huffman_decode_df11_b200 as df11
+    units = workload_units(config, seed)
+    hosts, devs = [], []
+    for name, thunk in units:
+        bits = thunk(device)
+        h = df11.compress(bits)
+        hosts.append(h)
+        devs.append(df11.to_device(h, device))
+        del bits
+    return units, hosts, devs
+
+
+def run_b200(args, world, rank, local):
+    import huffman_decode_df11_b200 as df11
+    device = f"cuda:{local}"
+    seed = args.seed + rank
+    units, hosts, devs = prepare(args.config, seed, device)
+    names = [u[0] for u in units]
+    groups = block_groups(args.config, names)
+    n_total = sum(h.n for h in hosts)
+    # one reused scratch buffer sized for the largest group
+    group_elems = [sum(hosts[i].n for i in g) for g in groups]
+    scratch = torch.empty(max(group_elems), dtype=torch.bfloat16, device=device)
+    outs_for = []
+    for g in groups:
+        off, outs = 0, []
+        for i in g:
+            outs.append(scratch[off:off + hosts[i].n])
+            off += hosts[i].n
+        outs_for.append(outs)
+    err = df11.new_error_word(device)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        for gi, g in enumerate(groups):
+            if events is not None:
+                events[gi][0].record(stream)
+            df11.decode_batched([devs[i] for i in g], outs_for[gi], err=err, stream=stream)
+            if events is not None:
+                events[gi][1].record(stream)
+
+    # parity: every group's output equals the original, bit for bit
+    for gi, g in enumerate(groups):
+        df11.decode_batched([devs[i] for i in g], outs_for[gi], err=err, stream=stream)
+        torch.cuda.synchronize()
+        for i, o in zip(g, outs_for[gi]):
+            ref = units[i][1](device)
+            if not torch.equal(o.view(torch.int16), ref):
+                raise SystemExit(f"parity failure on {names[i]}")
+            del ref
+    df11.check_device_error(err)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = sum((len(g) + 15) // 16 for g in groups)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in groups] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                      else local) as clocks:
+        # keep the GPU busy (untimed) while the sampler starts, so that the
+        # samples taken around a short timed region show clocks under load
+        t_busy = time.perf_counter()
+        while time.perf_counter() - t_busy < 0.4:
+            step()
+            torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for s in range(args.steps):
+            step(ev[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    df11.check_device_error(err)
+    ms_local = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    out_bytes_all = sum_over_ranks(2.0 * n_total, world)
+    value = out_bytes_all / (ms * 1e-3) / 1e9
+
+    # dominant kernel: per-launch durations from events on the launch stream
+    per_group_ms = [statistics.mean(ev[s][gi][0].elapsed_time(ev[s][gi][1])
+                                    for s in range(args.steps)) for gi in range(len(groups))]
+    alg = [sum(algorithmic_bytes(hosts[i]) for i in g) for g in groups]
+    achieved = sum(alg) / (sum(per_group_ms) * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = recorded_traffic(args.config)
+
+    # end to end through the public API: host (pinned) compressed tensors in,
+    # host BF16 out, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, units, hosts, groups, device, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(hosts, args.cpu_budget_s)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+            "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
+            "config": {
+                "workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
+                "elements": n_total, "chunk_bytes": 8, "threads_per_block": 256,
+                "compressed_bytes": sum(h.compressed_bytes() for h in hosts),
+                "bits_per_weight": round(8.0 * sum(h.compressed_bytes() for h in hosts)
+                                         / n_total, 3),
+                "l2": "inputs larger than L2 (no flush)" if sum(alg) > 126e6 else
+                      "inputs smaller than L2: numbers include L2 reuse",
+                "parallelism": f"replicas x{world} (no collective)",
+                "parity": "bit-exact vs original on every tensor before timing",
+            },
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "traffic": traffic, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_step": sum(alg)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "per_group_ms": [round(x, 4) for x in per_group_ms]
+            if len(groups) <= 8 else {"min": round(min(per_group_ms), 4),
+                                      "max": round(max(per_group_ms), 4),
+                                      "groups": len(groups)},
+        }
+        print(json.dumps(line), flush=True)
+
+
+def measure_e2e(args, units, hosts, groups, device, world):
+    import huffman_decode_df11_b200 as df11
+    # bounded host memory: the first groups up to ~2G elements
+    keep, elems = [], 0
+    for g in groups:
+        if keep and elems + sum(hosts[i].n for i in g) > 2_000_000_000:
+            break
+        keep.append(g)
+        elems += sum(hosts[i].n for i in g)
+    sampled = len(keep) < len(groups)
+    groups = keep
+    idx = [i for g in groups for i in g]
+    hosts = {i: hosts[i] for i in idx}
+    # pinned host copies of the compressed tensors; device staging; pinned out
+    pinned, staged, out_dev, out_host = {}, {}, {}, {}
+    for i, h in hosts.items():
+        pinned[i] = {k: torch.from_numpy(getattr(h, k).view(np.uint8)).pin_memory()
+                     for k in ("bitstream", "gaps", "block_out_pos", "luts",
+                               "code_lengths", "sign_mantissa")}
+        staged[i] = df11.to_device(h, device)
+        out_dev[i] = df11.empty_output(staged[i])
+        out_host[i] = torch.empty(h.n, dtype=torch.bfloat16).pin_memory()
+    err = df11.new_error_word(device)
+    stream = torch.cuda.current_stream()
+    h2d = sum(sum(t.numel() for t in p.values()) for p in pinned.values())
+    d2h = sum(2 * h.n for h in hosts.values())
+
+    def step():
+        for g in groups:
+            for i in g:
+                for k, t in pinned[i].items():
+                    dst = getattr(staged[i], k)
+                    dst.view(torch.uint8).copy_(t, non_blocking=True)
+            df11.decode_batched([staged[i] for i in g], [out_dev[i] for i in g],
+                                err=err, stream=stream)
+            for i in g:
+                out_host[i].copy_(out_dev[i], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    for i in idx:  # the host result is the original tensor, bit for bit
+        if not torch.equal(out_host[i].view(torch.int16), units[i][1](device).cpu()):
+            raise SystemExit(f"e2e parity failure on {units[i][0]}")
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 10))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    df11.check_device_error(err)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
+    out_bytes_all = sum_over_ranks(2.0 * sum(h.n for h in hosts.values()), world)
+    res = {"value": round(out_bytes_all / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+           "ms_per_step": round(ms, 3), "steps": steps,
+           "path": "pinned host compressed -> H2D -> df11_decode_batched -> D2H pinned"}
+    if sampled:
+        res["sample"] = f"first {len(groups)} decode groups ({len(idx)} tensors)"
+    return res
+
+
+def _oracle_sample(hosts, budget_s: float):
+    """Decode the workload's tensors with the oracle until the budget is
+    spent; returns (decoded elements, seconds, description)."""
+    import oracle
+    done, t_used, names = 0, 0.0, 0
+    for h in hosts:
+        if t_used >= budget_s:
+            break
+        count = h.n
+        # bound one call to what fits the remaining budget (~15 ns/element)
+        cap = int(max(1, (budget_s - t_used) / 15e-9))
+        count = min(count, cap)
+        t = time.perf_counter()
+        out, _, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, count)
+        t_used += time.perf_counter() - t
+        done += count
+        names += 1
+    return done, t_used, f"{done} elements from the first {names} tensor(s), decoded in order"
+
+
+def cpu_baseline(hosts, budget_s: float):
+    done, secs, what = _oracle_sample(hosts, budget_s)
+    return {"value": round(2.0 * done / secs / 1e9, 4), "unit": UNIT, "cores": 1,
+            "kind": "oracle", "sample": what + " (single-threaded bit-serial C decode)"}
+
+
+def run_reference(args, world, rank):
+    """The comparison arm: the CPU oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return
+    units = workload_units(args.config, args.seed)
+    import huffman_decode_df11_b200 as df11
+    hosts = [df11.compress(thunk("cpu")) for _, thunk in units]
+    n_total = sum(h.n for h in hosts)
+    budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        _oracle_sample(hosts, budget)
+    tot_done, tot_s, what = 0, 0.0, ""
+    for _ in range(args.steps):
+        d, s, what = _oracle_sample(hosts, budget)
+        tot_done += d
+        tot_s += s
+    value = 2.0 * tot_done / tot_s / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+        "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
+        "config": {"workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
+                   "elements": n_total, "chunk_bytes": 8, "threads_per_block": 256,
+                   "step": f"bounded sample of the workload, ~{budget:.1f} s of CPU work"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": what + " per step (single-threaded bit-serial C decode)"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+WORKLOAD_NAMES = {
+    "single": "single 1024x1024 N(0,0.02)",
+    "block": "Qwen3-8B-shaped block (q,k,v,o,gate,up,down), 192,937,984 elems",
+    "adversarial": "adversarial exponent mix, 64M elems",
+    "fibonacci": "Fibonacci exponent counts (32-bit codewords), 14,930,351 elems",
+    "embedding": "embedding 151936x4096 N(0,0.02), 622,329,856 elems",
+    "stack": "36-layer Qwen3-8B-shaped stack + embedding + LM head, 8,190,427,136 elems",
+}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="block", choices=sorted(WORKLOAD_NAMES))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = setup_dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("the b200 arm needs a CUDA device")
+            run_b200(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

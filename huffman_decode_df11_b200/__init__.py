@@ -1,0 +1,319 @@
+"""DF11 (DFloat11) lossless BF16 weight decode on B200 (sm_100a).
+
+Thin Python binding over ``libdf11.so`` (built from ``csrc/``; C ABI declared
+in ``include/df11.h``).  This module only marshals arguments: every step of
+the decode runs in the library's CUDA kernel, and the format builder runs in
+the library's host C++ code.  There is no fallback: if the library cannot be
+loaded, importing the binding's entry points raises.
+
+PyTorch is used for device memory and streams only.
+
+    >>> h = compress(bf16_weight)            # host, once ("compression")
+    >>> d = to_device(h, "cuda")             # compressed tensors in HBM
+    >>> w = decode(d)                        # BF16 in HBM, bit-identical
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+from typing import List, Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _build
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+
+# ---------------------------------------------------------------------------
+# ctypes mirror of include/df11.h
+
+DF11_MAX_BATCH = 16
+STATUS = {
+    0: "DF11_OK", 1: "DF11_ERR_NULL", 2: "DF11_ERR_ALIGN", 3: "DF11_ERR_FORMAT",
+    4: "DF11_ERR_UNSUPPORTED", 5: "DF11_ERR_CUDA", 6: "DF11_ERR_TOO_LARGE",
+    7: "DF11_ERR_INVALID", 8: "DF11_ERR_NOMEM",
+}
+DEV_ERRORS = {
+    0: "DF11_DEV_OK", 1: "DF11_DEV_ERR_COUNT", 2: "DF11_DEV_ERR_OVERRUN",
+    3: "DF11_DEV_ERR_TABLE", 4: "DF11_DEV_ERR_TIMEOUT", 5: "DF11_DEV_ERR_CAPACITY",
+}
+
+
+class Params(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_uint64),
+        ("total_bits", ctypes.c_uint64),
+        ("chunk_bytes", ctypes.c_uint32),
+        ("threads_per_block", ctypes.c_uint32),
+        ("num_blocks", ctypes.c_uint32),
+        ("num_luts", ctypes.c_uint32),
+        ("max_block_elems", ctypes.c_uint32),
+        ("max_len", ctypes.c_uint32),
+    ]
+
+
+class TensorDesc(ctypes.Structure):
+    _fields_ = [
+        ("bitstream", ctypes.c_void_p),
+        ("gaps", ctypes.c_void_p),
+        ("block_out_pos", ctypes.c_void_p),
+        ("luts", ctypes.c_void_p),
+        ("code_lengths", ctypes.c_void_p),
+        ("sign_mantissa", ctypes.c_void_p),
+        ("out_bf16", ctypes.c_void_p),
+        ("params", Params),
+    ]
+
+
+class HostTensor(ctypes.Structure):
+    _fields_ = [
+        ("params", Params),
+        ("code_lengths", ctypes.c_uint8 * 256),
+        ("bitstream", ctypes.POINTER(ctypes.c_uint8)),
+        ("bitstream_bytes", ctypes.c_uint64),
+        ("gaps", ctypes.POINTER(ctypes.c_uint8)),
+        ("gaps_bytes", ctypes.c_uint64),
+        ("block_out_pos", ctypes.POINTER(ctypes.c_uint32)),
+        ("luts", ctypes.POINTER(ctypes.c_uint32)),
+        ("sign_mantissa", ctypes.POINTER(ctypes.c_uint8)),
+        ("sign_mantissa_bytes", ctypes.c_uint64),
+    ]
+
+
+class Df11Error(RuntimeError):
+    pass
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libdf11.so (built in-tree on first use if stale or missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.LIB
+    if _build._stale() and os.path.exists(_build.NVCC):
+        path = _build.build()
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing and nvcc is not available to build it; the DF11 "
+            "decode path has no CPU fallback")
+    L = ctypes.CDLL(path)
+    vp, u64, u32, i32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int32
+    L.df11_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, u64, ctypes.POINTER(Params), vp, vp]
+    L.df11_decode.restype = ctypes.c_int
+    L.df11_decode_batched.argtypes = [ctypes.POINTER(TensorDesc), ctypes.c_int, vp, vp]
+    L.df11_decode_batched.restype = ctypes.c_int
+    L.df11_shared_bytes.argtypes = [ctypes.POINTER(Params)]
+    L.df11_shared_bytes.restype = ctypes.c_size_t
+    L.df11_supported.argtypes = [u32, u32]
+    L.df11_supported.restype = ctypes.c_int
+    L.df11_status_string.argtypes = [ctypes.c_int]
+    L.df11_status_string.restype = ctypes.c_char_p
+    L.df11_device_error_string.argtypes = [i32]
+    L.df11_device_error_string.restype = ctypes.c_char_p
+    L.df11_build.argtypes = [vp, u64, u32, u32, ctypes.c_int, ctypes.POINTER(HostTensor)]
+    L.df11_build.restype = ctypes.c_int
+    L.df11_host_tensor_free.argtypes = [ctypes.POINTER(HostTensor)]
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = lib().df11_status_string(status).decode()
+        raise Df11Error(f"{what}: {STATUS.get(status, status)} ({msg})")
+
+
+def supported(chunk_bytes: int, threads_per_block: int) -> bool:
+    return bool(lib().df11_supported(chunk_bytes, threads_per_block))
+
+
+# ---------------------------------------------------------------------------
+# host side: the format builder
+
+@dataclass
+class Df11Host:
+    """One compressed tensor in host memory (numpy arrays)."""
+    params: Params
+    code_lengths: np.ndarray   # uint8[256]
+    bitstream: np.ndarray      # uint8
+    gaps: np.ndarray           # uint8 (5-bit fields)
+    block_out_pos: np.ndarray  # uint32[num_blocks + 1]
+    luts: np.ndarray           # uint32[num_luts * 256]
+    sign_mantissa: np.ndarray  # uint8 (n rounded up to 16)
+    shape: tuple = ()
+
+    @property
+    def n(self) -> int:
+        return int(self.params.n)
+
+    def compressed_bytes(self) -> int:
+        """Bytes a decode reads: bitstream + gaps + positions + tables +
+        code lengths + sign/mantissa, as stored."""
+        return (self.bitstream.nbytes + self.gaps.nbytes + self.block_out_pos.nbytes
+                + self.luts.nbytes + 256 + self.sign_mantissa.nbytes)
+
+
+def _as_u16_numpy(w) -> np.ndarray:
+    if isinstance(w, torch.Tensor):
+        t = w.detach()
+        if t.dtype in (torch.bfloat16, torch.float16, torch.uint16):
+            t = t.view(torch.int16)
+        if t.dtype != torch.int16:
+            raise TypeError("expected a 2-byte tensor of BF16 bit patterns")
+        return t.cpu().contiguous().reshape(-1).numpy().view(np.uint16)
+    a = np.ascontiguousarray(w).reshape(-1)
+    if a.dtype.itemsize != 2:
+        raise TypeError("expected 2-byte BF16 bit patterns")
+    return a.view(np.uint16)
+
+
+def _np_copy(ptr, count, dtype):
+    if count == 0:
+        return np.zeros(0, dtype)
+    ctype = np.ctypeslib.as_ctypes_type(dtype)
+    buf = ctypes.cast(ptr, ctypes.POINTER(ctype * count)).contents
+    return np.frombuffer(buf, dtype=dtype, count=count).copy()
+
+
+def compress(w, chunk_bytes: int = 8, threads_per_block: int = 256,
+             threads: int = 0) -> Df11Host:
+    """Encode a BF16 tensor (host or device; copied to host) into DF11."""
+    shape = tuple(w.shape) if hasattr(w, "shape") else ()
+    a = _as_u16_numpy(w)
+    h = HostTensor()
+    L = lib()
+    _check(L.df11_build(a.ctypes.data if a.size else None, a.size, chunk_bytes,
+                        threads_per_block, threads, ctypes.byref(h)), "df11_build")
+    try:
+        p = Params.from_buffer_copy(h.params)
+        out = Df11Host(
+            params=p,
+            code_lengths=np.frombuffer(bytes(h.code_lengths), np.uint8).copy(),
+            bitstream=_np_copy(h.bitstream, h.bitstream_bytes, np.uint8),
+            gaps=_np_copy(h.gaps, h.gaps_bytes, np.uint8),
+            block_out_pos=_np_copy(h.block_out_pos, p.num_blocks + 1, np.uint32),
+            luts=_np_copy(h.luts, p.num_luts * 256, np.uint32),
+            sign_mantissa=_np_copy(h.sign_mantissa, h.sign_mantissa_bytes, np.uint8),
+            shape=shape,
+        )
+    finally:
+        L.df11_host_tensor_free(ctypes.byref(h))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# device side
+
+@dataclass
+class Df11Device:
+    """One compressed tensor resident in device memory (torch tensors)."""
+    params: Params
+    bitstream: torch.Tensor
+    gaps: torch.Tensor
+    block_out_pos: torch.Tensor
+    luts: torch.Tensor
+    code_lengths: torch.Tensor
+    sign_mantissa: torch.Tensor
+    shape: tuple = ()
+
+    @property
+    def n(self) -> int:
+        return int(self.params.n)
+
+    @property
+    def device(self):
+        return self.bitstream.device
+
+    def compressed_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.bitstream, self.gaps, self.block_out_pos, self.luts,
+                    self.code_lengths, self.sign_mantissa))
+
+    def desc(self, out: torch.Tensor) -> TensorDesc:
+        return TensorDesc(self.bitstream.data_ptr(), self.gaps.data_ptr(),
+                          self.block_out_pos.data_ptr(), self.luts.data_ptr(),
+                          self.code_lengths.data_ptr(), self.sign_mantissa.data_ptr(),
+                          out.data_ptr(), self.params)
+
+
+def _np_to(t: np.ndarray, device, pin: bool = False) -> torch.Tensor:
+    x = torch.from_numpy(t)
+    if pin:
+        x = x.pin_memory()
+    return x.to(device, non_blocking=pin)
+
+
+def to_device(h: Df11Host, device="cuda") -> Df11Device:
+    """Copy a compressed tensor into device memory (16-byte aligned buffers)."""
+    return Df11Device(
+        params=Params.from_buffer_copy(h.params),
+        bitstream=_np_to(h.bitstream, device),
+        gaps=_np_to(h.gaps, device),
+        block_out_pos=_np_to(h.block_out_pos.view(np.int32), device),
+        luts=_np_to(h.luts.view(np.int32), device),
+        code_lengths=_np_to(h.code_lengths, device),
+        sign_mantissa=_np_to(h.sign_mantissa, device),
+        shape=h.shape,
+    )
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def empty_output(d: Df11Device) -> torch.Tensor:
+    return torch.empty(max(d.n, 1), dtype=torch.bfloat16, device=d.device)[: d.n]
+
+
+def decode(d: Df11Device, out: Optional[torch.Tensor] = None,
+           err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode into `out` (a flat BF16/int16 device tensor of n elements,
+    allocated if None).  Asynchronous on `stream` (default: current stream).
+    `err` is an optional int32 device tensor the kernel writes error codes
+    into (see check_device_error)."""
+    if out is None:
+        out = empty_output(d)
+    if out.numel() != d.n or not out.is_contiguous() or out.element_size() != 2:
+        raise ValueError("out must be a contiguous 2-byte tensor with n elements")
+    p = Params.from_buffer_copy(d.params)
+    _check(lib().df11_decode(
+        d.bitstream.data_ptr(), d.gaps.data_ptr(), d.block_out_pos.data_ptr(),
+        d.luts.data_ptr(), d.code_lengths.data_ptr(), d.sign_mantissa.data_ptr(),
+        out.data_ptr(), d.n, ctypes.byref(p),
+        err.data_ptr() if err is not None else None, _stream_handle(stream)),
+        "df11_decode")
+    return out
+
+
+def decode_batched(ds: Sequence[Df11Device], outs: Sequence[torch.Tensor],
+                   err: Optional[torch.Tensor] = None, stream=None):
+    """Decode several tensors with one launch per 16 tensors."""
+    if len(ds) != len(outs):
+        raise ValueError("one output per tensor")
+    for d, o in zip(ds, outs):
+        if o.numel() != d.n or not o.is_contiguous() or o.element_size() != 2:
+            raise ValueError("each out must be a contiguous 2-byte tensor with n elements")
+    arr = (TensorDesc * max(len(ds), 1))(*[d.desc(o) for d, o in zip(ds, outs)])
+    _check(lib().df11_decode_batched(arr, len(ds),
+                                     err.data_ptr() if err is not None else None,
+                                     _stream_handle(stream)), "df11_decode_batched")
+    return outs
+
+
+def new_error_word(device="cuda") -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check_device_error(err: torch.Tensor):
+    """Raise if the kernel flagged inconsistent data (synchronises)."""
+    code = int(err.item())
+    if code != 0:
+        msg = lib().df11_device_error_string(code).decode()
+        raise Df11Error(f"decode reported {DEV_ERRORS.get(code, code)}: {msg}")

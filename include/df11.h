@@ -1,0 +1,185 @@
+/*
+ * df11.h -- C ABI of the DF11 (DFloat11) decode library, libdf11.so.
+ *
+ * DF11 stores a BF16 weight tensor as
+ *   - its 8-bit exponents, Huffman coded with a canonical code of at most
+ *     32-bit codewords and packed into one MSB-first bitstream, and
+ *   - its sign and 7 mantissa bits, kept as they are, one byte per element
+ *     (sign in bit 7, mantissa in bits 0-6).
+ * Sources: "DFloat11无损压缩技术：基于哈夫曼编码的BFloat16大模型显存优化方案"
+ * (jsqmd.com), §2.1 (BF16 fields) and §2.2 items 1-3 (Huffman-coded
+ * exponents, sign/mantissa kept, aligned blocks, decode on the GPU right
+ * before the matmul, no CPU decompression, discard after use);
+ * "DFloat11：用于高效 GPU 推理的 LLM 和扩散模型无损压缩" (gittoolsai.com),
+ * section "工作原理" (bit-identical output, weights stay compressed in GPU
+ * memory); "DFloat11重新定义LLM无损压缩的技术边界" (ocdem.com), §2.2
+ * (multi-level lookup tables in shared memory, two-phase locate /
+ * reconstruct, parallel prefix sum).
+ *
+ * Layout of one encoded tensor (written by df11_build):
+ *   bitstream      the codewords of elements 0..n-1, one after another,
+ *                  first bit = bit 7 of byte 0.  Cut into chunks of C bytes
+ *                  (one per decoding thread) and blocks of T chunks (one per
+ *                  thread block).  num_blocks*T*C bytes + 16 zero bytes.
+ *   gaps           per chunk, the distance in bits (0..31) from the chunk's
+ *                  first bit to the first codeword that starts at or after
+ *                  it (to the end of the stream if none does; 0 for chunks
+ *                  past the end).  5-bit fields packed MSB-first;
+ *                  num_blocks*T*5/8 + 16 bytes.
+ *   block_out_pos  num_blocks+1 uint32: index of the first element whose
+ *                  codeword starts in each block; the last entry is n.
+ *   luts           num_luts tables of 256 uint32, table 0 first:
+ *                  table 0, indexed by the next 8 bits: up to three whole
+ *                  codewords in those bits -- bits 0-23 their exponents
+ *                  (first in bits 0-7, unused bytes 0), bits 24-27 the bits
+ *                  they use (1..8), bits 28-29 how many (1..3); or, when the
+ *                  first codeword is longer than 8 bits, bits 0-23 the number
+ *                  of the next-level table and bits 24-31 zero.
+ *                  tables 1.. (levels 1..3), indexed by the following 8
+ *                  bits: bits 0-7 the exponent and bits 28-29 = 1, or a
+ *                  pointer as above.  0 marks a bit pattern no codeword
+ *                  starts with.  Tables are numbered level by level and by
+ *                  prefix value within a level.
+ *   code_lengths   256 bytes, codeword length of each exponent (0 = absent).
+ *   sign_mantissa  n bytes, readable up to a multiple of 16 bytes.
+ *
+ * Every decode call is asynchronous on the given stream, allocates nothing,
+ * never synchronises the host and has no CPU fallback.  Argument errors are
+ * returned at once; errors the GPU finds in the data are written to the
+ * optional device word d_err (first error wins) and never trap.
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *df11_stream_t;
+
+typedef enum df11_status {
+  DF11_OK = 0,
+  DF11_ERR_NULL = 1,        /* a required pointer is NULL */
+  DF11_ERR_ALIGN = 2,       /* a pointer misses its required alignment */
+  DF11_ERR_FORMAT = 3,      /* parameters inconsistent with each other */
+  DF11_ERR_UNSUPPORTED = 4, /* (chunk_bytes, threads_per_block) not built */
+  DF11_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+  DF11_ERR_TOO_LARGE = 6,   /* n >= 2^32, or a batch over DF11_MAX_BATCH */
+  DF11_ERR_INVALID = 7,     /* other invalid argument */
+  DF11_ERR_NOMEM = 8        /* host allocation failed (df11_build) */
+} df11_status;
+
+/* Values the GPU writes to *d_err.  A device word that is not 0 means the
+ * output of the call is not to be trusted. */
+#define DF11_DEV_OK 0
+#define DF11_DEV_ERR_COUNT 1    /* a block decoded a different element count
+                                   than block_out_pos says */
+#define DF11_DEV_ERR_OVERRUN 2  /* a thread's last codeword ran past the
+                                   start of the next thread's first one */
+#define DF11_DEV_ERR_TABLE 3    /* the stream reached an invalid table entry
+                                   or a zero code length */
+#define DF11_DEV_ERR_TIMEOUT 4  /* an asynchronous copy into shared memory
+                                   did not complete in time */
+#define DF11_DEV_ERR_CAPACITY 5 /* a block holds more elements than
+                                   max_block_elems */
+
+/* Largest number of tensors one df11_decode_batched launch takes. */
+#define DF11_MAX_BATCH 16
+
+/* Per-tensor format parameters, written by df11_build. */
+typedef struct df11_params {
+  uint64_t n;                 /* elements (< 2^32) */
+  uint64_t total_bits;        /* meaningful bits of the bitstream */
+  uint32_t chunk_bytes;       /* C: bitstream bytes per thread */
+  uint32_t threads_per_block; /* T: threads (chunks) per block */
+  uint32_t num_blocks;        /* ceil(total_bits / (8*C*T)) */
+  uint32_t num_luts;          /* 256-entry tables (>= 1) */
+  uint32_t max_block_elems;   /* max over blocks of elements per block */
+  uint32_t max_len;           /* longest codeword in bits (<= 32) */
+} df11_params;
+
+/* One tensor to decode: device pointers plus its parameters. */
+typedef struct df11_tensor {
+  const uint8_t *bitstream;      /* 16-byte aligned */
+  const uint8_t *gaps;           /* 16-byte aligned */
+  const uint32_t *block_out_pos; /* 4-byte aligned */
+  const uint32_t *luts;          /* 16-byte aligned */
+  const uint8_t *code_lengths;   /* any alignment */
+  const uint8_t *sign_mantissa;  /* 16-byte aligned */
+  uint16_t *out_bf16;            /* 16-byte aligned, n elements, caller-owned */
+  df11_params params;
+} df11_tensor;
+
+/*
+ * Decode one tensor into out_bf16 (bit-identical to the BF16 tensor that was
+ * encoded).  All pointers are device pointers owned by the caller and laid
+ * out as described at the top of this file; `params` is a host pointer.
+ * n must equal params->n.  d_err is a device int32 (may be NULL) that the
+ * caller zeroes; the kernel writes a DF11_DEV_ERR_* code into it when the
+ * data are inconsistent.  Returns DF11_OK once the work is queued on
+ * `stream`.  n == 0 queues nothing.
+ */
+df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
+                        const uint32_t *block_out_pos, const uint32_t *luts,
+                        const uint8_t *code_lengths,
+                        const uint8_t *sign_mantissa, uint16_t *out_bf16,
+                        uint64_t n, const df11_params *params, int32_t *d_err,
+                        df11_stream_t stream);
+
+/*
+ * Decode `count` tensors (a layer's weights, say) with one kernel launch per
+ * DF11_MAX_BATCH tensors.  `tensors` is a host array; every tensor must use
+ * the same chunk_bytes and threads_per_block.  Same conventions as
+ * df11_decode.
+ */
+df11_status df11_decode_batched(const df11_tensor *tensors, int count,
+                                int32_t *d_err, df11_stream_t stream);
+
+/* Bytes of dynamic shared memory one block of the decode kernel uses for
+ * these parameters (for occupancy planning); 0 if unsupported. */
+size_t df11_shared_bytes(const df11_params *params);
+
+/* 1 if the library has a kernel for this (chunk_bytes, threads_per_block). */
+int df11_supported(uint32_t chunk_bytes, uint32_t threads_per_block);
+
+const char *df11_status_string(df11_status status);
+const char *df11_device_error_string(int32_t code);
+
+/* ---------------------------------------------------------------------- */
+/* Host-side format builder ("compression"; offline, host memory only).   */
+
+typedef struct df11_host_tensor {
+  df11_params params;
+  uint8_t code_lengths[256];
+  uint8_t *bitstream;
+  uint64_t bitstream_bytes;   /* num_blocks*T*C + 16 */
+  uint8_t *gaps;
+  uint64_t gaps_bytes;        /* num_blocks*T*5/8 + 16 */
+  uint32_t *block_out_pos;    /* num_blocks + 1 */
+  uint32_t *luts;             /* num_luts * 256 */
+  uint8_t *sign_mantissa;
+  uint64_t sign_mantissa_bytes; /* n rounded up to 16 */
+} df11_host_tensor;
+
+/*
+ * Encode n BF16 words (host memory) with chunk_bytes C (a multiple of 4,
+ * 4..64) and threads_per_block T (a multiple of 128, 128..1024), using up
+ * to num_threads host threads (<= 0: all cores).  The exponent code is the
+ * Huffman code of the exponent histogram, limited to 32-bit codewords by
+ * package-merge when needed, in canonical form; ties are broken by symbol
+ * value so the output is deterministic.  On success the buffers in *out
+ * belong to the caller and are released with df11_host_tensor_free.
+ */
+df11_status df11_build(const uint16_t *bf16, uint64_t n, uint32_t chunk_bytes,
+                       uint32_t threads_per_block, int num_threads,
+                       df11_host_tensor *out);
+void df11_host_tensor_free(df11_host_tensor *t);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DF11_H */

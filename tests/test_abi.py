@@ -1,0 +1,106 @@
+"""The C ABI: libdf11.so loads, exports every function include/df11.h
+declares, and rejects bad arguments on the host before touching the GPU.
+No call here launches a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import huffman_decode_df11_b200 as df11
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b(df11_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_function():
+    lib = df11.lib()
+    declared = _declared_functions()
+    assert {"df11_decode", "df11_decode_batched", "df11_build"} <= declared
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._name],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = declared - exported
+    assert not missing, missing
+    for name in declared:
+        getattr(lib, name)  # resolvable through ctypes
+
+
+def test_struct_layouts_match_header():
+    assert ctypes.sizeof(df11.Params) == 40
+    assert ctypes.sizeof(df11.TensorDesc) == 7 * 8 + 40
+
+
+def _params(**kw):
+    p = df11.Params(n=1000, total_bits=2600, chunk_bytes=8, threads_per_block=256,
+                    num_blocks=1, num_luts=1, max_block_elems=1000, max_len=10)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null address; never dereferenced
+
+
+def _call(p, n=None, ptrs=None, err=None):
+    ptrs = ptrs or [FAKE] * 7
+    return df11.lib().df11_decode(*ptrs, p.n if n is None else n, ctypes.byref(p), err, None)
+
+
+def test_host_validation_errors():
+    L = df11.lib()
+    assert L.df11_decode(*[FAKE] * 7, 10, None, None, None) == 1           # NULL params
+    assert _call(_params(), n=999) == 7                                      # n mismatch
+    assert _call(_params(n=0, total_bits=0, num_blocks=0)) == 0             # empty: no-op
+    assert _call(_params(), ptrs=[FAKE] * 6 + [0]) == 1                      # NULL out
+    assert _call(_params(), ptrs=[FAKE + 8] + [FAKE] * 6) == 2               # misaligned
+    assert _call(_params(), err=FAKE + 2) == 2                               # misaligned err
+    assert _call(_params(chunk_bytes=12)) == 4                               # unsupported C
+    assert _call(_params(threads_per_block=384)) == 4                        # unsupported T
+    assert _call(_params(num_blocks=2)) == 3                                 # wrong block count
+    assert _call(_params(total_bits=999)) == 3                               # < 1 bit/element
+    assert _call(_params(total_bits=40000)) == 3                             # > 32 bits/element
+    assert _call(_params(num_luts=0)) == 3
+    assert _call(_params(max_block_elems=20000)) == 3
+    assert _call(_params(n=1 << 32, total_bits=1 << 34, num_blocks=1 << 20)) == 6
+
+
+def test_batched_host_validation():
+    L = df11.lib()
+    assert L.df11_decode_batched(None, 0, None, None) == 0
+    assert L.df11_decode_batched(None, -1, None, None) == 7
+    assert L.df11_decode_batched(None, 1, None, None) == 1
+    a = df11.TensorDesc(*[FAKE] * 7, _params())
+    b = df11.TensorDesc(*[FAKE] * 7, _params(chunk_bytes=4, total_bits=2600,
+                                                num_blocks=1))
+    arr = (df11.TensorDesc * 2)(a, b)
+    assert L.df11_decode_batched(arr, 2, None, None) == 7  # mixed (C, T)
+
+
+def test_supported_shapes_and_shared_bytes():
+    assert df11.supported(8, 256) and df11.supported(4, 256) and df11.supported(16, 256)
+    assert df11.supported(8, 128) and df11.supported(8, 512)
+    assert not df11.supported(12, 256)
+    p = _params(max_block_elems=6400, num_luts=4)
+    sb = df11.lib().df11_shared_bytes(ctypes.byref(p))
+    assert 16_000 < sb < 24_000
+
+
+def test_status_strings():
+    L = df11.lib()
+    for code in range(9):
+        assert L.df11_status_string(code)
+    for code in range(6):
+        assert L.df11_device_error_string(code)

@@ -66,16 +66,22 @@ class NamedTensor:
     bits: torch.Tensor  # int16 BF16 bit patterns, flattened
 
 
+def block_tensor(seed: int, index: int, device="cpu", scale: int = 1) -> torch.Tensor:
+    """Weight `index` (order of BLOCK_SHAPES) of one Qwen3-8B-shaped block,
+    N(0, 1/sqrt(fan_in)) with fan_in = in_features.  `scale` > 1 divides the
+    out-features (rows) for small CPU-sized variants."""
+    name, rows, cols = BLOCK_SHAPES[index]
+    r = max(1, rows // scale)
+    return gaussian_bf16(r * cols, 1.0 / math.sqrt(cols), seed * 131 + index, device)
+
+
 def block_tensors(seed: int = 0, device="cpu", scale: int = 1):
-    """The seven weights of one Qwen3-8B-shaped block, each N(0, 1/sqrt(fan_in))
-    with fan_in = in_features.  `scale` > 1 divides the out-features (rows)
-    for small CPU-sized variants; 1 gives the full 193M-element block."""
+    """The seven weights of one Qwen3-8B-shaped block (see block_tensor);
+    scale 1 gives the full 192,937,984-element block."""
     out = []
     for i, (name, rows, cols) in enumerate(BLOCK_SHAPES):
         r = max(1, rows // scale)
-        bits = gaussian_bf16(r * cols, 1.0 / math.sqrt(cols), seed * 131 + i,
-                             device)
-        out.append(NamedTensor(name, (r, cols), bits))
+        out.append(NamedTensor(name, (r, cols), block_tensor(seed, i, device, scale)))
     return out
 
 
