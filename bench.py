@@ -293,7 +293,7 @@ def run_b200(args, world, rank, local):
         # keep the GPU busy (untimed) while the sampler starts, so that the
         # samples taken around a short timed region show clocks under load
         t_busy = time.perf_counter()
-        while time.perf_counter() - t_busy < 0.4:
+        while not args.no_clock_window and time.perf_counter() - t_busy < 0.4:
             step()
             torch.cuda.synchronize()
         barrier(world)
@@ -513,6 +513,9 @@ def main(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clock-window", action="store_true",
+                    help="skip the busy untimed loop before the timed region "
+                         "(for profiler runs)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -51,6 +51,8 @@ class Params(ctypes.Structure):
         ("num_luts", ctypes.c_uint32),
         ("max_block_elems", ctypes.c_uint32),
         ("max_len", ctypes.c_uint32),
+        ("max_chunk_elems", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
     ]
 
 

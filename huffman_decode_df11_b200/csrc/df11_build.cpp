@@ -328,6 +328,8 @@ extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
   out->gaps = (uint8_t *)std::calloc(out->gaps_bytes, 1);
   out->block_out_pos = (uint32_t *)std::calloc((size_t)p.num_blocks + 1, 4);
   std::vector<uint8_t> gap(chunks ? chunks : 1, 0);
+  // index of the first element whose codeword starts at or after each chunk
+  std::vector<uint32_t> first_elem(chunks + 1, (uint32_t)n);
   if (!out->bitstream || !out->gaps || !out->block_out_pos) {
     df11_host_tensor_free(out);
     return DF11_ERR_NOMEM;
@@ -349,8 +351,10 @@ extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
         int sym = (w[i] >> 7) & 0xFF;
         // chunks and blocks whose first codeword start is this one
         for (uint64_t c = prev < 0 ? 0 : (uint64_t)prev / chunk_bits + 1;
-             c * chunk_bits <= bit && c < chunks; ++c)
+             c * chunk_bits <= bit && c < chunks; ++c) {
           gap[c] = (uint8_t)(bit - c * chunk_bits);
+          first_elem[c] = (uint32_t)i;
+        }
         for (uint64_t b = prev < 0 ? 0 : (uint64_t)prev / block_bits + 1;
              b * block_bits <= bit && b < p.num_blocks; ++b)
           bpos[b] = (uint32_t)i;
@@ -397,6 +401,9 @@ extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
   uint32_t mx = 0;
   for (uint32_t b = 0; b < p.num_blocks; ++b) mx = std::max(mx, bpos[b + 1] - bpos[b]);
   p.max_block_elems = mx;
+  uint32_t mc = 0;
+  for (uint64_t c = 0; c < chunks; ++c) mc = std::max(mc, first_elem[c + 1] - first_elem[c]);
+  p.max_chunk_elems = mc;
   return DF11_OK;
 }
 

@@ -1,31 +1,50 @@
 // df11_decode.cu -- DF11 decode on sm_100a (B200) and the C ABI around it.
 //
-// One thread block decodes one block of T chunks of C bitstream bytes:
+// Persistent thread blocks.  Every thread block is assigned to one tensor of
+// the launch and walks that tensor's format blocks (T chunks of C bitstream
+// bytes each) with a stride.  Per thread block, once:
+//
+//   tables   table 0 of the format (256 entries, up to three codewords per
+//            8-bit index) and the code lengths are copied into shared memory
+//            with every exponent byte rotated right by one bit; a wide table
+//            of 2^WB entries, each holding up to four whole codewords of the
+//            next WB bits, is derived from them in shared memory.  Deeper
+//            format tables (codewords longer than 8 bits) are read from shared
+//            memory when few, from global memory otherwise.
+//
+// Per format block, software-pipelined with a two-slot stage:
 //
 //   stage    one thread issues bulk asynchronous copies (cp.async.bulk, no
-//            multicast) of the block's bitstream slice and gap fields, and of
-//            its sign/mantissa bytes, into shared memory; meanwhile all
-//            threads copy table 0 and the code lengths into shared memory.
-//   phase 1  "locate" ("DFloat11重新定义LLM无损压缩的技术边界" (ocdem.com)
-//            §2.2): each thread walks its chunk from its gap with the
-//            table and counts the codewords that start in it.
-//   scan     exclusive prefix sum of the counts (warp shuffles, then across
-//            warps) gives every thread its first output index; the block's
-//            total must equal its block_out_pos difference.
-//   phase 2  "reconstruct": each thread decodes its chunk again and writes
-//            its exponents to their final places in a shared-memory array.
-//   output   every thread fuses 16 exponents with 16 sign/mantissa bytes
-//            into 16 BF16 words with byte permutes and writes them with two
-//            16-byte stores; the block's ragged ends use 2-byte stores.
+//            multicast) of the NEXT block's bitstream slice, gap fields and
+//            sign/mantissa bytes into the free stage slot, completing on that
+//            slot's mbarrier, while the block in the other slot is decoded.
+//   decode   each thread walks its chunk from its gap ("locate" and
+//            "reconstruct" of "DFloat11重新定义LLM无损压缩的技术边界"
+//            (ocdem.com) §2.2, done in one pass): every lookup of the wide
+//            table yields up to four exponents, appended to a 64-bit
+//            accumulator and flushed as aligned 32-bit words into the
+//            thread's private slot (word j of thread t at j*T+t: one bank per
+//            thread, no conflicts).  Bits past the thread's region are set to
+//            one, so no lookup can accept a codeword beyond it (valid when the
+//            longest codeword is longer than WB bits; other codes take a loop
+//            that checks the region end on every lookup).
+//   scan     exclusive prefix sum of the per-thread counts (warp shuffles,
+//            then across warps) gives every thread its first output index;
+//            the total must equal the block's block_out_pos difference.
+//   compact  every thread moves its exponents from its slot to their final
+//            places in a block-wide byte array (funnel shifts, 32-bit stores).
+//   output   every thread fuses 16 exponents with 16 sign/mantissa bytes into
+//            16 BF16 words with byte permutes and writes them with two 16-byte
+//            stores; the block's ragged ends use 2-byte stores.
 //
-// Tables: table 0 lives in shared memory with its exponent bytes rotated
-// right by one bit (e>>1 | (e&1)<<7), which turns the BF16 rebuild into two
-// byte permutes and one bitwise select per output word.  Deeper tables (only
-// codewords longer than 8 bits reach them) are read from shared memory when
-// few, from global memory otherwise.
+// Why the rotation: with e' = e>>1 | (e&1)<<7, the high byte of a BF16 word
+// is (sm & 0x80) | (e' & 0x7F) and the low byte (e' & 0x80) | (sm & 0x7F), so
+// four output words cost two byte permutes and one bitwise select each.
 //
-// Nothing here waits on another block, so nothing can hang: the only waits
-// are on this block's own copies, bounded, reporting DF11_DEV_ERR_TIMEOUT.
+// Nothing here waits on another thread block, so nothing can hang: the only
+// waits are on this block's own copies, bounded, reporting
+// DF11_DEV_ERR_TIMEOUT.  Every data-dependent access is bounds-checked;
+// inconsistent data are reported through the error word, never by a trap.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -35,9 +54,11 @@
 
 namespace {
 
-constexpr int kSubTablesInSmem = 8;     // deeper tables kept in shared memory
+constexpr int kSubTablesInSmem = 8;        // deeper tables kept in shared memory
 constexpr uint32_t kSpinLimit = 1u << 20;  // x ~1 us suspend hint: ~1 s
 constexpr uint32_t kSuspendHintNs = 1000;
+constexpr int kWideBits = 10;              // index bits of the derived table
+constexpr int kWideSyms = 4;               // codewords per derived entry
 
 struct KTensor {
   const uint8_t *bitstream;
@@ -52,7 +73,9 @@ struct KTensor {
   uint32_t num_blocks;
   uint32_t num_luts;
   uint32_t max_block_elems;
-  uint32_t block_begin;  // first grid block of this tensor
+  uint32_t max_chunk_elems;
+  uint32_t masked;     // longest codeword > kWideBits: bits past a region may be set
+  uint32_t cta_begin;  // first thread block of this tensor
   uint32_t pad;
 };
 
@@ -60,25 +83,43 @@ struct KBatch {
   KTensor t[DF11_MAX_BATCH];
   int32_t *err;
   int count;
-  uint32_t stage_bytes;  // bytes of each of the sign/mantissa and exponent stages
-  uint32_t sub_in_smem;  // deeper tables copied to shared memory
+  uint32_t cta_end;      // total thread blocks
+  uint32_t stage_bytes;  // sign/mantissa bytes per stage slot (and exponent array)
+  uint32_t slot_words;   // 32-bit words of each thread's private slot
+  uint32_t sub_words;    // deeper-table words kept in shared memory (0: global)
+  uint32_t pad;
 };
 
-// shared memory layout (bytes); every buffer starts on a 16-byte boundary
-constexpr uint32_t kOffMbar = 0;      // 2 mbarriers
-constexpr uint32_t kOffScan = 16;     // 36 ints
-constexpr uint32_t kOffLens = 160;    // 256 code lengths, by rotated exponent
-constexpr uint32_t kOffLut0 = 416;    // 256 x u32
-constexpr uint32_t kOffBits = 1440;   // T*C + 16 bitstream bytes, then gaps ...
+// ---- shared memory layout --------------------------------------------------
+// [0,16)       2 mbarriers (one per stage slot)
+// [16,48)      2 x {P0, P1, ok, 0}: block positions of the block in each slot
+// [48,192)     36 ints of scan scratch
+// [192,448)    code lengths by rotated exponent
+// [448,1472)   table 0 (rotated)
+// [1472, ...)  wide table (2^WB x 8 bytes)
+// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16), sign/mantissa
+// then         exponent array (stage_bytes), private slots (slot_words*T*4),
+//              deeper tables (sub_words*4)
+constexpr uint32_t kOffMbar = 0;
+constexpr uint32_t kOffMeta = 16;
+constexpr uint32_t kOffScan = 48;
+constexpr uint32_t kOffLens = 192;
+constexpr uint32_t kOffLut0 = 448;
+constexpr uint32_t kOffWide = 1472;
+constexpr uint32_t kWideBytes = 8u << kWideBits;
+constexpr uint32_t kOffStages = kOffWide + kWideBytes;
 
 template <int T, int C>
 struct Layout {
   static constexpr uint32_t bits_bytes = T * C + 16;
   static constexpr uint32_t gaps_bytes = T * 5 / 8 + 16;
-  static constexpr uint32_t off_gaps = kOffBits + bits_bytes;
-  static constexpr uint32_t off_sm = off_gaps + gaps_bytes;
+  static constexpr uint32_t head_bytes = bits_bytes + gaps_bytes;  // per slot, before sm
   static_assert(bits_bytes % 16 == 0 && gaps_bytes % 16 == 0, "alignment");
 };
+
+__host__ __device__ constexpr uint32_t slot_stride(uint32_t head, uint32_t stage) {
+  return head + stage;
+}
 
 __device__ __forceinline__ uint32_t rot8x3(uint32_t v) {
   // rotate each of the low three bytes right by one bit
@@ -133,70 +174,123 @@ __device__ __forceinline__ int read_gap(const uint8_t *g, int k) {
   return (int)((v >> (11 - (bit & 7))) & 31u);
 }
 
+// One codeword at the start of a 32-bit window through the format's tables:
+// the (rotated) exponent and the codeword length; false for an invalid one.
+__device__ __forceinline__ bool decode_one(uint32_t win, const uint32_t *__restrict__ lut0,
+                                           const uint8_t *__restrict__ lens,
+                                           const uint32_t *sub, uint32_t num_luts,
+                                           uint32_t &sym, uint32_t &len) {
+  const uint32_t e = lut0[win >> 24];
+  if ((e >> 24) & 15u) {
+    sym = e & 0xFFu;
+  } else {
+    uint32_t t = e & 0xFFFFFFu, f = 0;
+#pragma unroll 1
+    for (int level = 1; level <= 3; ++level) {
+      if (t == 0 || t >= num_luts) break;
+      const uint32_t e2 = sub[(t - 1) * 256 + ((win >> (24 - 8 * level)) & 0xFFu)];
+      if (e2 >> 28) {
+        f = e2;
+        break;
+      }
+      t = e2 & 0xFFFFFFu;
+    }
+    if (f == 0) return false;
+    sym = rot8x3(f & 0xFFu);
+  }
+  len = lens[sym];
+  return len != 0;
+}
+
+// Derived table: entry i holds the codewords that lie wholly inside the WB
+// bits i (at most kWideSyms): x = exponents (first in bits 0-7),
+// y = bits used << 8 | count << 12.  y == 0: the first codeword is longer
+// than WB bits (or invalid) and takes the slow path.
+template <int T>
+__device__ void build_wide(uint2 *wide, const uint32_t *lut0, const uint8_t *lens,
+                           const uint32_t *sub, uint32_t num_luts) {
+  for (uint32_t i = threadIdx.x; i < (1u << kWideBits); i += T) {
+    const uint32_t bits = i << (32 - kWideBits);
+    uint32_t used = 0, n = 0, syms = 0;
+    while (n < kWideSyms) {
+      const uint32_t win = bits << used;
+      const uint32_t e = lut0[win >> 24];
+      const uint32_t ns = e >> 28;
+      if (((e >> 24) & 15u) == 0) {
+        uint32_t s, l;
+        if (!decode_one(win, lut0, lens, sub, num_luts, s, l) || used + l > kWideBits) break;
+        syms |= s << (8 * n);
+        ++n;
+        used += l;
+        continue;
+      }
+      bool stop = ns == 0;
+      for (uint32_t j = 0; j < ns && n < kWideSyms; ++j) {
+        const uint32_t s = (e >> (8 * j)) & 0xFFu, l = lens[s];
+        if (l == 0 || used + l > kWideBits) {
+          stop = true;
+          break;
+        }
+        syms |= s << (8 * n);
+        ++n;
+        used += l;
+      }
+      if (stop || used >= kWideBits) break;
+    }
+    wide[i] = n ? make_uint2(syms, (used << 8) | (n << 12)) : make_uint2(0, 0);
+  }
+}
+
 // Walk one thread's codewords [pos, end) (bit positions relative to its
-// chunk's first bit) through the tables; count them and, when EMIT, write
-// their (rotated) exponents to dst.  w holds the chunk and the 8 bytes after
-// it as big-endian 32-bit words.  Sets *bad on inconsistent data.
-template <int C, bool EMIT>
-__device__ __forceinline__ int decode_run(const uint32_t (&w)[C / 4 + 2], int pos,
-                                          const int end, const uint32_t *__restrict__ lut0,
-                                          const uint8_t *__restrict__ lens,
-                                          const uint32_t *sub, uint32_t num_luts,
-                                          uint8_t *dst, int &bad) {
+// chunk's first bit) and append their exponents to its private slot (word j
+// at slot[j*T]).  w: the chunk and the 8 bytes after it, big-endian words.
+// Returns the number of codewords; sets `bad` on inconsistent data.
+template <int T, int C, bool MASKED>
+__device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 2], int pos,
+                                                 const int end, const uint2 *__restrict__ wide,
+                                                 const uint32_t *__restrict__ lut0,
+                                                 const uint8_t *__restrict__ lens,
+                                                 const uint32_t *sub, uint32_t num_luts,
+                                                 uint32_t *slot, uint32_t slot_words, int &bad) {
   constexpr int NW = C / 4 + 2;
-  int count = 0;
+  uint32_t a0 = 0, a1 = 0, sh = 0, words = 0;
 #pragma unroll
   for (int k = 0; k < NW - 1; ++k) {
     const int lim = min(32 * (k + 1), end);
     const uint32_t hi = w[k], lo = w[k + 1];
     while (pos < lim) {
       const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)pos);  // bits [pos, pos+32)
-      uint32_t e = lut0[win >> 24];
-      uint32_t nbits = (e >> 24) & 15u;
-      if (nbits - 1u >= (uint32_t)(end - pos)) {
-        // rare: a codeword longer than 8 bits (nbits == 0: pointer), or the
-        // entry's codewords run past the end of this thread's region
-        uint32_t sym;
-        if (nbits == 0) {
-          uint32_t t = e & 0xFFFFFFu, f = 0;
-#pragma unroll 1
-          for (int level = 1; level <= 3; ++level) {
-            if (t == 0 || t >= num_luts) break;
-            const uint32_t e2 = sub[(t - 1) * 256 + ((win >> (24 - 8 * level)) & 0xFFu)];
-            if (e2 >> 28) {
-              f = e2;
-              break;
-            }
-            t = e2 & 0xFFFFFFu;
-          }
-          if (f == 0) {
-            bad = DF11_DEV_ERR_TABLE;
-            return count;
-          }
-          sym = rot8x3(f & 0xFFu);
-        } else {
-          sym = e & 0xFFu;
-        }
-        nbits = lens[sym];
-        if (nbits == 0) {
+      const uint2 e = wide[win >> (32 - kWideBits)];
+      uint32_t syms = e.x, nbits = (e.y >> 8) & 15u, nsym = e.y >> 12;
+      const bool slow = MASKED ? nbits == 0 : (nbits == 0 || (int)nbits > end - pos);
+      if (slow) {
+        uint32_t s, l;
+        if (!decode_one(win, lut0, lens, sub, num_luts, s, l)) {
           bad = DF11_DEV_ERR_TABLE;
-          return count;
+          return 0;
         }
-        e = sym | (1u << 28);
+        syms = s;
+        nbits = l;
+        nsym = 1;
       }
-      const uint32_t nsym = e >> 28;
-      if (EMIT) {
-        dst[0] = (uint8_t)e;
-        if (nsym >= 2) dst[1] = (uint8_t)(e >> 8);
-        if (nsym >= 3) dst[2] = (uint8_t)(e >> 16);
-        dst += nsym;
+      a0 |= syms << sh;
+      a1 |= __funnelshift_l(syms, 0u, sh);  // bytes pushed past the low word
+      sh += nsym << 3;
+      if (sh >= 32) {
+        if (words < slot_words) slot[words * T] = a0;
+        ++words;
+        a0 = a1;
+        a1 = 0;
+        sh -= 32;
       }
-      count += (int)nsym;
       pos += (int)nbits;
     }
   }
+  if (sh) {
+    if (words < slot_words) slot[words * T] = a0;
+  }
   if (pos != end) bad = DF11_DEV_ERR_OVERRUN;
-  return count;
+  return words * 4 + (sh >> 3);
 }
 
 // four sign/mantissa bytes and four rotated exponents -> four BF16 words
@@ -211,49 +305,74 @@ __device__ __forceinline__ uint16_t fuse1(uint32_t sm, uint32_t er) {
   return (uint16_t)(((sm & 0x80u) << 8) | ((er & 0x7Fu) << 8) | (er & 0x80u) | (sm & 0x7Fu));
 }
 
+// Thread 0: queue the copies of block b into stage slot `slot` (or, for
+// inconsistent block positions, an empty completion flagged not ok).
+template <int T, int C>
+__device__ __forceinline__ void issue_block(const KTensor &tk, uint32_t b, uint32_t P0,
+                                            uint32_t P1, uint8_t *stage, uint4 *meta,
+                                            uint32_t bar, uint32_t stage_bytes) {
+  using L = Layout<T, C>;
+  const uint32_t expected = P1 - P0;
+  const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems &&
+                  expected + 32 <= stage_bytes;
+  *meta = make_uint4(P0, P1, ok ? 1u : 0u, 0u);
+  if (!ok) {
+    mbar_arrive_expect_tx(bar, 0);
+    return;
+  }
+  const uint32_t sm_begin = P0 & ~15u;
+  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
+  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes + sm_bytes);
+  bulk_g2s(smem_addr(stage), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, bar);
+  bulk_g2s(smem_addr(stage + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
+           bar);
+  if (sm_bytes)
+    bulk_g2s(smem_addr(stage + L::head_bytes), tk.sign_mantissa + sm_begin, sm_bytes, bar);
+}
+
 template <int T, int C>
 __global__ void __launch_bounds__(T) df11_decode_kernel(const __grid_constant__ KBatch kb) {
   using L = Layout<T, C>;
   constexpr int NW = C / 4 + 2;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + kOffMbar);
+  uint4 *meta = reinterpret_cast<uint4 *>(smem + kOffMeta);
   int *scan = reinterpret_cast<int *>(smem + kOffScan);
   uint8_t *lens_s = smem + kOffLens;
   uint32_t *lut0_s = reinterpret_cast<uint32_t *>(smem + kOffLut0);
-  uint8_t *bits_s = smem + kOffBits;
-  uint8_t *gaps_s = smem + L::off_gaps;
-  uint8_t *sm_s = smem + L::off_sm;
-  uint8_t *ex_s = sm_s + kb.stage_bytes;
-  uint32_t *sub_s = reinterpret_cast<uint32_t *>(ex_s + kb.stage_bytes);
+  uint2 *wide_s = reinterpret_cast<uint2 *>(smem + kOffWide);
+  uint8_t *stages = smem + kOffStages;
+  const uint32_t stride_bytes = slot_stride(L::head_bytes, kb.stage_bytes);
+  uint8_t *ex_s = stages + 2 * stride_bytes;
+  uint32_t *slots = reinterpret_cast<uint32_t *>(ex_s + kb.stage_bytes);
+  uint32_t *sub_s = slots + kb.slot_words * T;
 
   int ti = 0;
   for (int i = 1; i < kb.count; ++i)
-    if (blockIdx.x >= kb.t[i].block_begin) ti = i;
+    if (blockIdx.x >= kb.t[i].cta_begin) ti = i;
   const KTensor &tk = kb.t[ti];
-  const uint32_t b = blockIdx.x - tk.block_begin;
+  const uint32_t ctas = (ti + 1 < kb.count ? kb.t[ti + 1].cta_begin : kb.cta_end) - tk.cta_begin;
+  const uint32_t first = blockIdx.x - tk.cta_begin;
   const int tid = threadIdx.x;
+  if (first >= tk.num_blocks) return;  // uniform: never issued anything
 
-  const uint32_t P0 = tk.block_out_pos[b], P1 = tk.block_out_pos[b + 1];
-  const uint32_t expected = P1 - P0;
-  if (P1 < P0 || P1 > tk.n || expected > tk.max_block_elems || expected + 32 > kb.stage_bytes) {
-    if (tid == 0) report(kb.err, DF11_DEV_ERR_CAPACITY);
-    return;
-  }
-  const uint32_t bar_in = smem_addr(&mbar[0]), bar_sm = smem_addr(&mbar[1]);
-  const uint32_t sm_begin = P0 & ~15u;
-  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
+  const uint32_t bar0 = smem_addr(&mbar[0]), bar1 = smem_addr(&mbar[1]);
+  uint32_t nP0 = 0, nP1 = 0;  // thread 0: positions of the next block to issue
   if (tid == 0) {
-    mbar_init(bar_in, 1);
-    mbar_init(bar_sm, 1);
+    mbar_init(bar0, 1);
+    mbar_init(bar1, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    mbar_arrive_expect_tx(bar_in, L::bits_bytes + L::gaps_bytes);
-    bulk_g2s(smem_addr(bits_s), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, bar_in);
-    bulk_g2s(smem_addr(gaps_s), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes, bar_in);
-    mbar_arrive_expect_tx(bar_sm, sm_bytes);
-    if (sm_bytes) bulk_g2s(smem_addr(sm_s), tk.sign_mantissa + sm_begin, sm_bytes, bar_sm);
+    issue_block<T, C>(tk, first, tk.block_out_pos[first], tk.block_out_pos[first + 1], stages,
+                      &meta[0], bar0, kb.stage_bytes);
+    const uint32_t nb = first + ctas;
+    if (nb < tk.num_blocks) {
+      nP0 = tk.block_out_pos[nb];
+      nP1 = tk.block_out_pos[nb + 1];
+    }
   }
-  // tables: level 0 with rotated exponent bytes, code lengths by rotated
-  // exponent, deeper tables verbatim
+
+  // tables (once per thread block): table 0 and lengths rotated, deeper
+  // tables verbatim, then the derived wide table
   for (int i = tid; i < 256; i += T) {
     uint32_t e = tk.luts[i] & 0x3FFFFFFFu;
     if ((e >> 24) & 15u) e = (e & 0xFF000000u) | rot8x3(e);
@@ -261,92 +380,152 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const __grid_constant__ 
     lens_s[((uint32_t)i >> 1) | (((uint32_t)i & 1u) << 7)] = tk.code_lengths[i];
   }
   const uint32_t *sub = tk.luts + 256;
-  if (kb.sub_in_smem) {
-    const uint32_t words = (tk.num_luts - 1) * 256;
-    for (uint32_t i = tid; i < words; i += T) sub_s[i] = sub[i];
+  const uint32_t sub_words = (tk.num_luts - 1) * 256;
+  if (sub_words && sub_words <= kb.sub_words) {
+    for (uint32_t i = tid; i < sub_words; i += T) sub_s[i] = sub[i];
     sub = sub_s;
   }
-  __syncthreads();  // tables and barrier initialisation visible to all
-
-  int bad = 0;
-  if (!mbar_wait(bar_in, 0)) bad = DF11_DEV_ERR_TIMEOUT;
-
-  // this thread's region of the stream, relative to its chunk's first bit
-  const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
-  int start = read_gap(gaps_s, tid);
-  int end = C * 8 + read_gap(gaps_s, tid + 1);
-  if (chunk_bit >= tk.total_bits) {
-    start = end = 0;
-  } else if ((uint64_t)end > tk.total_bits - chunk_bit) {
-    end = (int)(tk.total_bits - chunk_bit);
-  }
-  uint32_t w[NW];
-#pragma unroll
-  for (int k = 0; k < NW; ++k)
-    w[k] = __byte_perm(*reinterpret_cast<const uint32_t *>(bits_s + tid * C + 4 * k), 0, 0x0123);
-
-  // phase 1: count
-  int cnt = 0;
-  if (!bad) cnt = decode_run<C, false>(w, start, end, lut0_s, lens_s, sub, tk.num_luts, nullptr, bad);
-
-  // block exclusive scan of the counts
-  const int lane = tid & 31, warp = tid >> 5;
-  int incl = cnt;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-    if (lane >= d) incl += v;
-  }
-  if (lane == 31) scan[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    const int v = lane < T / 32 ? scan[lane] : 0;
-    int s = v;
+  build_wide<T>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
+  __syncthreads();
+
+  const int lane = tid & 31, warp = tid >> 5;
+  uint32_t k = 0;
+  for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
+    const uint32_t s = k & 1;
+    uint8_t *stage = stages + s * stride_bytes;
+    // queue the next block into the other slot (freed by the barrier that
+    // ended the previous iteration)
+    if (tid == 0 && b + ctas < tk.num_blocks) {
+      issue_block<T, C>(tk, b + ctas, nP0, nP1, stages + (s ^ 1) * stride_bytes, &meta[s ^ 1],
+                        s ? bar0 : bar1, kb.stage_bytes);
+      const uint32_t nb = b + 2 * ctas;
+      if (nb < tk.num_blocks) {
+        nP0 = tk.block_out_pos[nb];
+        nP1 = tk.block_out_pos[nb + 1];
+      }
+    }
+    int bad = 0;
+    if (!mbar_wait(s ? bar1 : bar0, (k >> 1) & 1)) bad = DF11_DEV_ERR_TIMEOUT;
+    const uint4 m = meta[s];
+    const uint32_t P0 = m.x, P1 = m.y, expected = P1 - P0;
+    if (!m.z) {
+      if (tid == 0) report(kb.err, DF11_DEV_ERR_CAPACITY);
+      __syncthreads();
+      continue;
+    }
+    const uint8_t *bits_s = stage;
+    const uint8_t *gaps_s = stage + L::bits_bytes;
+    const uint8_t *sm_s = stage + L::head_bytes;
+
+    // this thread's region, relative to its chunk's first bit
+    const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
+    int start = read_gap(gaps_s, tid);
+    int end = C * 8 + read_gap(gaps_s, tid + 1);
+    if (chunk_bit >= tk.total_bits) {
+      start = end = 0;
+    } else if ((uint64_t)end > tk.total_bits - chunk_bit) {
+      end = (int)(tk.total_bits - chunk_bit);
+    }
+    uint32_t w[NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j) {
+      w[j] = __byte_perm(*reinterpret_cast<const uint32_t *>(bits_s + tid * C + 4 * j), 0, 0x0123);
+      if (tk.masked) {  // ones from bit `end` on
+        const int lo = end - 32 * j;
+        if (lo <= 0) w[j] = 0xFFFFFFFFu;
+        else if (lo < 32) w[j] |= 0xFFFFFFFFu >> lo;
+      }
+    }
+
+    uint32_t cnt = 0;
+    if (!bad) {
+      if (tk.masked)
+        cnt = decode_chunk<T, C, true>(w, start, end, wide_s, lut0_s, lens_s, sub, tk.num_luts,
+                                       slots + tid, kb.slot_words, bad);
+      else
+        cnt = decode_chunk<T, C, false>(w, start, end, wide_s, lut0_s, lens_s, sub, tk.num_luts,
+                                        slots + tid, kb.slot_words, bad);
+      if (!bad && cnt > tk.max_chunk_elems) bad = DF11_DEV_ERR_CAPACITY;
+    }
+
+    // block exclusive scan of the counts
+    uint32_t incl = cnt;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const int u = __shfl_up_sync(0xFFFFFFFFu, s, d);
-      if (lane >= d) s += u;
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += v;
     }
-    if (lane < T / 32) scan[lane] = s - v;
-    if (lane == 31) scan[32] = s;
-  }
-  const int any_bad = __syncthreads_or(bad);
-  const int excl = scan[warp] + incl - cnt;
-  const uint32_t total = (uint32_t)scan[32];
-  if (any_bad || total != expected) {
-    if (bad) report(kb.err, bad);
-    else if (tid == 0 && !any_bad) report(kb.err, DF11_DEV_ERR_COUNT);
-    mbar_wait(bar_sm, 0);  // never leave with a copy in flight
-    return;
-  }
-
-  // phase 2: exponents to their final places (index i <-> element sm_begin+i)
-  const uint32_t head = P0 & 15u;
-  decode_run<C, true>(w, start, end, lut0_s, lens_s, sub, tk.num_luts, ex_s + head + excl, bad);
-  __syncthreads();
-  if (!mbar_wait(bar_sm, 0)) {
-    if (tid == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
-    return;
-  }
-
-  // output: fuse and store, 16 elements per thread per step
-  uint16_t *out = tk.out + sm_begin;
-  const uint32_t span = head + expected;
-  const uint32_t groups = (span + 15u) >> 4;
-  for (uint32_t g = tid; g < groups; g += T) {
-    const uint32_t i0 = g << 4;
-    if (i0 >= head && i0 + 16u <= span) {
-      const uint4 s = *reinterpret_cast<const uint4 *>(sm_s + i0);
-      const uint4 r = *reinterpret_cast<const uint4 *>(ex_s + i0);
-      const uint2 a = fuse4(s.x, r.x), c = fuse4(s.y, r.y);
-      const uint2 d = fuse4(s.z, r.z), f = fuse4(s.w, r.w);
-      uint4 *o = reinterpret_cast<uint4 *>(out + i0);
-      o[0] = make_uint4(a.x, a.y, c.x, c.y);
-      o[1] = make_uint4(d.x, d.y, f.x, f.y);
-    } else {
-      const uint32_t lo = i0 > head ? i0 : head, hi = i0 + 16u < span ? i0 + 16u : span;
-      for (uint32_t i = lo; i < hi; ++i) out[i] = fuse1(sm_s[i], ex_s[i]);
+    if (lane == 31) scan[warp] = (int)incl;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t v = lane < T / 32 ? (uint32_t)scan[lane] : 0u;
+      uint32_t sc = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, sc, d);
+        if (lane >= d) sc += u;
+      }
+      if (lane < T / 32) scan[lane] = (int)(sc - v);
+      if (lane == 31) scan[32] = (int)sc;
     }
+    const int any_bad = __syncthreads_or(bad);
+    const uint32_t excl = (uint32_t)scan[warp] + incl - cnt;
+    const uint32_t total = (uint32_t)scan[32];
+    if (any_bad || total != expected) {
+      if (bad) report(kb.err, bad);
+      else if (tid == 0 && !any_bad) report(kb.err, DF11_DEV_ERR_COUNT);
+      __syncthreads();
+      continue;
+    }
+
+    // compact: slot bytes [0, cnt) -> ex_s[d, d+cnt); exponent i of the
+    // array belongs to element (P0 & ~15) + i
+    {
+      const uint32_t d = (P0 & 15u) + excl;
+      const uint32_t *sl = slots + tid;
+      const uint32_t h = (4u - (d & 3u)) & 3u;  // bytes before the first aligned word
+      uint32_t cur = cnt ? sl[0] : 0u;
+      const uint32_t nh = cnt < h ? cnt : h;
+      for (uint32_t i = 0; i < nh; ++i) ex_s[d + i] = (uint8_t)(cur >> (8 * i));
+      if (cnt > h) {
+        // aligned words: source bytes h+4j .. h+4j+3 = words j, j+1 shifted by h bytes
+        const uint32_t full = (cnt - h) >> 2;
+        uint32_t *dst = reinterpret_cast<uint32_t *>(ex_s + d + h);
+        for (uint32_t j = 0; j < full; ++j) {
+          const uint32_t nxt = sl[(j + 1) * T];  // within the slot: j+1 <= cnt/4
+          dst[j] = __funnelshift_r(cur, nxt, 8 * h);
+          cur = nxt;
+        }
+        for (uint32_t i = h + 4 * full; i < cnt; ++i)
+          ex_s[d + i] = (uint8_t)(sl[(i >> 2) * T] >> (8 * (i & 3)));
+      }
+    }
+    __syncthreads();
+
+    // output: fuse and store, 16 elements per thread per step
+    {
+      const uint32_t head = P0 & 15u;
+      uint16_t *out = tk.out + (P0 & ~15u);
+      const uint32_t span = head + expected;
+      const uint32_t groups = (span + 15u) >> 4;
+      for (uint32_t g = tid; g < groups; g += T) {
+        const uint32_t i0 = g << 4;
+        if (i0 >= head && i0 + 16u <= span) {
+          const uint4 sv = *reinterpret_cast<const uint4 *>(sm_s + i0);
+          const uint4 rv = *reinterpret_cast<const uint4 *>(ex_s + i0);
+          const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
+          const uint2 dd = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+          uint4 *o = reinterpret_cast<uint4 *>(out + i0);
+          o[0] = make_uint4(a.x, a.y, c.x, c.y);
+          o[1] = make_uint4(dd.x, dd.y, f.x, f.y);
+        } else {
+          const uint32_t lo = i0 > head ? i0 : head, hi = i0 + 16u < span ? i0 + 16u : span;
+          for (uint32_t i = lo; i < hi; ++i) out[i] = fuse1(sm_s[i], ex_s[i]);
+        }
+      }
+    }
+    __syncthreads();  // stage slot, exponent array and private slots free again
   }
 }
 
@@ -363,9 +542,13 @@ uint32_t stage_bytes_for(uint32_t max_block_elems) {
   return (max_block_elems + 32u + 15u) & ~15u;
 }
 
-size_t shared_bytes(uint32_t C, uint32_t T, uint32_t stage, uint32_t sub_tables) {
-  return (size_t)kOffBits + (T * C + 16) + (T * 5 / 8 + 16) + 2 * (size_t)stage +
-         (size_t)sub_tables * 1024;
+uint32_t slot_words_for(uint32_t max_chunk_elems) { return (max_chunk_elems + 3u) / 4u + 1u; }
+
+size_t shared_bytes(uint32_t C, uint32_t T, uint32_t stage, uint32_t slot_words,
+                    uint32_t sub_words) {
+  const size_t head = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16;
+  return (size_t)kOffStages + 2 * (head + stage) + stage + (size_t)slot_words * T * 4 +
+         (size_t)sub_words * 4;
 }
 
 bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -385,35 +568,72 @@ df11_status validate(const df11_tensor &t) {
   if (p.total_bits < p.n || p.total_bits > 32ull * p.n) return DF11_ERR_FORMAT;
   if ((uint64_t)p.num_blocks != (p.total_bits + block_bits - 1) / block_bits) return DF11_ERR_FORMAT;
   if (p.num_luts < 1 || p.num_luts >= (1u << 24)) return DF11_ERR_FORMAT;
-  if (p.max_block_elems > 8ull * p.chunk_bytes * p.threads_per_block) return DF11_ERR_FORMAT;
-  if (p.max_block_elems == 0) return DF11_ERR_FORMAT;
+  if (p.max_block_elems == 0 || p.max_block_elems > 8ull * p.chunk_bytes * p.threads_per_block)
+    return DF11_ERR_FORMAT;
+  if (p.max_chunk_elems == 0 || p.max_chunk_elems > 8ull * p.chunk_bytes) return DF11_ERR_FORMAT;
+  if (p.max_len < 1 || p.max_len > 32) return DF11_ERR_FORMAT;
   return DF11_OK;
 }
 
+struct DeviceInfo {
+  int sms = 0;
+  std::atomic<size_t> configured[5];
+};
+
+DeviceInfo &device_info(int dev) {
+  static DeviceInfo info[64];
+  DeviceInfo &d = info[dev & 63];
+  if (d.sms == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    d.sms = v > 0 ? v : 1;
+  }
+  return d;
+}
+
 template <int T, int C>
-df11_status launch(const KBatch &kb, uint32_t grid, size_t smem, cudaStream_t s) {
-  static std::atomic<size_t> configured[64];
+df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t s,
+                   int instance) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
+  DeviceInfo &di = device_info(dev);
   auto kern = df11_decode_kernel<T, C>;
-  if (smem > 48 * 1024 && dev < 64 && configured[dev].load() < smem) {
+  if (smem > 48 * 1024 && di.configured[instance].load() < smem) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return DF11_ERR_CUDA;
-    configured[dev].store(smem);
+    di.configured[instance].store(smem);
   }
-  kern<<<grid, T, smem, s>>>(kb);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, smem) != cudaSuccess)
+    return DF11_ERR_CUDA;
+  if (per_sm < 1) return DF11_ERR_TOO_LARGE;
+  // thread blocks per tensor in proportion to its format blocks
+  const uint64_t budget = (uint64_t)di.sms * per_sm;
+  uint64_t total = 0;
+  for (int i = 0; i < kb.count; ++i) total += blocks[i];
+  uint32_t begin = 0;
+  for (int i = 0; i < kb.count; ++i) {
+    uint64_t c = (budget * blocks[i] + total / 2) / total;
+    if (c < 1) c = 1;
+    if (c > blocks[i]) c = blocks[i];
+    kb.t[i].cta_begin = begin;
+    begin += (uint32_t)c;
+  }
+  kb.cta_end = begin;
+  kern<<<begin, T, smem, s>>>(kb);
   return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
 df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaStream_t s) {
   KBatch kb{};
   kb.err = d_err;
-  uint32_t grid = 0, max_elems = 0, max_luts = 1, C = 0, T = 0;
+  uint32_t blocks[DF11_MAX_BATCH];
+  uint32_t max_elems = 0, max_chunk = 0, max_luts = 1, C = 0, T = 0;
   for (int i = 0; i < count; ++i) {
     const df11_params &p = ts[i].params;
     if (p.n == 0) continue;
-    KTensor &k = kb.t[kb.count++];
+    KTensor &k = kb.t[kb.count];
     k.bitstream = ts[i].bitstream;
     k.gaps = ts[i].gaps;
     k.block_out_pos = ts[i].block_out_pos;
@@ -426,24 +646,31 @@ df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     k.num_blocks = p.num_blocks;
     k.num_luts = p.num_luts;
     k.max_block_elems = p.max_block_elems;
-    k.block_begin = grid;
-    if ((uint64_t)grid + p.num_blocks > 0x7FFFFFFFu) return DF11_ERR_TOO_LARGE;
-    grid += p.num_blocks;
+    k.max_chunk_elems = p.max_chunk_elems;
+    k.masked = p.max_len > (uint32_t)kWideBits ? 1u : 0u;
+    blocks[kb.count] = p.num_blocks;
+    ++kb.count;
     max_elems = max_elems > p.max_block_elems ? max_elems : p.max_block_elems;
+    max_chunk = max_chunk > p.max_chunk_elems ? max_chunk : p.max_chunk_elems;
     max_luts = max_luts > p.num_luts ? max_luts : p.num_luts;
     C = p.chunk_bytes;
     T = p.threads_per_block;
   }
-  if (kb.count == 0 || grid == 0) return DF11_OK;
+  if (kb.count == 0) return DF11_OK;
   kb.stage_bytes = stage_bytes_for(max_elems);
-  kb.sub_in_smem = (max_luts - 1) <= (uint32_t)kSubTablesInSmem ? 1u : 0u;
-  const size_t smem = shared_bytes(C, T, kb.stage_bytes, kb.sub_in_smem ? max_luts - 1 : 0);
+  kb.slot_words = slot_words_for(max_chunk);
+  kb.sub_words = (max_luts - 1) <= (uint32_t)kSubTablesInSmem ? (max_luts - 1) * 256 : 0;
+  size_t smem = shared_bytes(C, T, kb.stage_bytes, kb.slot_words, kb.sub_words);
+  if (smem > 227 * 1024 && kb.sub_words) {  // drop the deeper tables to global memory
+    kb.sub_words = 0;
+    smem = shared_bytes(C, T, kb.stage_bytes, kb.slot_words, 0);
+  }
   if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
-  if (T == 256 && C == 8) return launch<256, 8>(kb, grid, smem, s);
-  if (T == 256 && C == 4) return launch<256, 4>(kb, grid, smem, s);
-  if (T == 256 && C == 16) return launch<256, 16>(kb, grid, smem, s);
-  if (T == 128 && C == 8) return launch<128, 8>(kb, grid, smem, s);
-  if (T == 512 && C == 8) return launch<512, 8>(kb, grid, smem, s);
+  if (T == 256 && C == 8) return launch<256, 8>(kb, blocks, smem, s, 0);
+  if (T == 256 && C == 4) return launch<256, 4>(kb, blocks, smem, s, 1);
+  if (T == 256 && C == 16) return launch<256, 16>(kb, blocks, smem, s, 2);
+  if (T == 128 && C == 8) return launch<128, 8>(kb, blocks, smem, s, 3);
+  if (T == 512 && C == 8) return launch<512, 8>(kb, blocks, smem, s, 4);
   return DF11_ERR_UNSUPPORTED;
 }
 
@@ -493,9 +720,10 @@ df11_status df11_decode_batched(const df11_tensor *tensors, int count, int32_t *
 
 size_t df11_shared_bytes(const df11_params *p) {
   if (!p || !supported(p->chunk_bytes, p->threads_per_block)) return 0;
-  const uint32_t subs = p->num_luts - 1 <= (uint32_t)kSubTablesInSmem ? p->num_luts - 1 : 0;
+  const uint32_t subs =
+      p->num_luts - 1 <= (uint32_t)kSubTablesInSmem ? (p->num_luts - 1) * 256 : 0;
   return shared_bytes(p->chunk_bytes, p->threads_per_block, stage_bytes_for(p->max_block_elems),
-                      subs);
+                      slot_words_for(p->max_chunk_elems), subs);
 }
 
 int df11_supported(uint32_t chunk_bytes, uint32_t threads_per_block) {
@@ -524,7 +752,7 @@ const char *df11_device_error_string(int32_t code) {
     case DF11_DEV_ERR_OVERRUN: return "a codeword ran past the next chunk's first codeword";
     case DF11_DEV_ERR_TABLE: return "invalid lookup-table entry or zero code length";
     case DF11_DEV_ERR_TIMEOUT: return "shared-memory copy did not complete in time";
-    case DF11_DEV_ERR_CAPACITY: return "block holds more elements than max_block_elems";
+    case DF11_DEV_ERR_CAPACITY: return "block or chunk holds more elements than its parameters allow";
   }
   return "unknown device error";
 }

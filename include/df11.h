@@ -100,6 +100,8 @@ typedef struct df11_params {
   uint32_t num_luts;          /* 256-entry tables (>= 1) */
   uint32_t max_block_elems;   /* max over blocks of elements per block */
   uint32_t max_len;           /* longest codeword in bits (<= 32) */
+  uint32_t max_chunk_elems;   /* max over chunks of codewords starting in it */
+  uint32_t reserved;          /* 0 */
 } df11_params;
 
 /* One tensor to decode: device pointers plus its parameters. */

@@ -415,6 +415,16 @@ int oracle_encode(const uint16_t *w, uint64_t n, uint32_t chunk_bytes,
   f->gaps_packed = (uint8_t *)calloc(f->gaps_bytes, 1);
   oracle_pack_gaps(f->gaps, chunks, f->gaps_packed);
 
+  /* codewords starting in each chunk, counted one start at a time */
+  f->max_chunk_elems = 0;
+  if (chunks) {
+    uint32_t *per_chunk = (uint32_t *)calloc(chunks, 4);
+    for (uint64_t i = 0; i < n; i++) per_chunk[starts[i] / (8ull * chunk_bytes)]++;
+    for (uint64_t c = 0; c < chunks; c++)
+      if (per_chunk[c] > f->max_chunk_elems) f->max_chunk_elems = per_chunk[c];
+    free(per_chunk);
+  }
+
   f->max_block_elems = 0;
   for (uint32_t b = 0; b < f->num_blocks; b++) {
     uint32_t e = f->block_out_pos[b + 1] - f->block_out_pos[b];

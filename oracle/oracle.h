@@ -49,6 +49,7 @@ typedef struct oracle_format {
   uint32_t num_luts;          /* 256-entry tables, level 0 first */
   uint32_t max_block_elems;   /* max over blocks of its element count */
   uint32_t max_len;           /* longest codeword */
+  uint32_t max_chunk_elems;   /* max over chunks of codewords starting in it */
   uint8_t code_lengths[256];  /* 0 = exponent absent */
   uint32_t codes[256];        /* canonical codeword, right-aligned */
   uint8_t *bitstream;         /* num_blocks*T*C + 16 bytes, MSB-first */

@@ -39,13 +39,14 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layouts_match_header():
-    assert ctypes.sizeof(df11.Params) == 40
-    assert ctypes.sizeof(df11.TensorDesc) == 7 * 8 + 40
+    assert ctypes.sizeof(df11.Params) == 48
+    assert ctypes.sizeof(df11.TensorDesc) == 7 * 8 + 48
 
 
 def _params(**kw):
     p = df11.Params(n=1000, total_bits=2600, chunk_bytes=8, threads_per_block=256,
-                    num_blocks=1, num_luts=1, max_block_elems=1000, max_len=10)
+                    num_blocks=1, num_luts=1, max_block_elems=1000, max_len=10,
+                    max_chunk_elems=40)
     for k, v in kw.items():
         setattr(p, k, v)
     return p
@@ -74,6 +75,8 @@ def test_host_validation_errors():
     assert _call(_params(total_bits=40000)) == 3                             # > 32 bits/element
     assert _call(_params(num_luts=0)) == 3
     assert _call(_params(max_block_elems=20000)) == 3
+    assert _call(_params(max_chunk_elems=65)) == 3                           # > 8*C
+    assert _call(_params(max_len=33)) == 3
     assert _call(_params(n=1 << 32, total_bits=1 << 34, num_blocks=1 << 20)) == 6
 
 
@@ -84,7 +87,7 @@ def test_batched_host_validation():
     assert L.df11_decode_batched(None, 1, None, None) == 1
     a = df11.TensorDesc(*[FAKE] * 7, _params())
     b = df11.TensorDesc(*[FAKE] * 7, _params(chunk_bytes=4, total_bits=2600,
-                                                num_blocks=1))
+                                                num_blocks=1, max_chunk_elems=30))
     arr = (df11.TensorDesc * 2)(a, b)
     assert L.df11_decode_batched(arr, 2, None, None) == 7  # mixed (C, T)
 
@@ -95,7 +98,7 @@ def test_supported_shapes_and_shared_bytes():
     assert not df11.supported(12, 256)
     p = _params(max_block_elems=6400, num_luts=4)
     sb = df11.lib().df11_shared_bytes(ctypes.byref(p))
-    assert 16_000 < sb < 24_000
+    assert 40_000 < sb < 56_000  # tables + two stage slots + slots
 
 
 def test_status_strings():

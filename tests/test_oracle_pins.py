@@ -353,6 +353,10 @@ def test_gaps_and_block_positions_brute_force(C, T):
     for b in range(f.num_blocks + 1):
         want = sum(1 for s in st if s < b * chunk_bits * T) if b < f.num_blocks else f.n
         assert f.block_out_pos[b] == want
+    per_chunk = [0] * (f.num_blocks * T)
+    for s in st:
+        per_chunk[s // chunk_bits] += 1
+    assert f.max_chunk_elems == max(per_chunk)
     # packed gaps: 5-bit fields, MSB first
     bits = np.unpackbits(f.gaps_packed)
     for c in range(f.num_blocks * T):
