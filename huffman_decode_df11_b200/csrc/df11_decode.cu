@@ -15,9 +15,10 @@
 // Per format block, software-pipelined with a two-slot stage:
 //
 //   stage    one thread issues bulk asynchronous copies (cp.async.bulk, no
-//            multicast) of the NEXT block's bitstream slice, gap fields and
-//            sign/mantissa bytes into the free stage slot, completing on that
-//            slot's mbarrier, while the block in the other slot is decoded.
+//            multicast) of the NEXT block's bitstream slice and gap fields
+//            into the free stage slot, completing on that slot's mbarrier,
+//            and a bulk L2 prefetch of its sign/mantissa bytes, while the
+//            block in the other slot is decoded.
 //   decode   each thread walks its chunk from its gap ("locate" and
 //            "reconstruct" of "DFloat11重新定义LLM无损压缩的技术边界"
 //            (ocdem.com) §2.2, done in one pass): every lookup of the wide
@@ -32,10 +33,12 @@
 //            then across warps) gives every thread its first output index;
 //            the total must equal the block's block_out_pos difference.
 //   compact  every thread moves its exponents from its slot to their final
-//            places in a block-wide byte array (funnel shifts, 32-bit stores).
-//   output   every thread fuses 16 exponents with 16 sign/mantissa bytes into
-//            16 BF16 words with byte permutes and writes them with two 16-byte
-//            stores; the block's ragged ends use 2-byte stores.
+//            places in a block-wide byte array: funnel-shifted 32-bit stores,
+//            shared atomic OR for the two words it shares with neighbours.
+//   output   every thread loads 16 sign/mantissa bytes (16-byte global load),
+//            fuses them with 16 exponents into 16 BF16 words with byte
+//            permutes and writes them with two 16-byte stores; the block's
+//            two ragged 16-element groups are written one element per lane.
 //
 // Why the rotation: with e' = e>>1 | (e&1)<<7, the high byte of a BF16 word
 // is (sm & 0x80) | (e' & 0x7F) and the low byte (e' & 0x80) | (sm & 0x7F), so
@@ -84,7 +87,7 @@ struct KBatch {
   int32_t *err;
   int count;
   uint32_t cta_end;      // total thread blocks
-  uint32_t stage_bytes;  // sign/mantissa bytes per stage slot (and exponent array)
+  uint32_t stage_bytes;  // bytes of the exponent array
   uint32_t slot_words;   // 32-bit words of each thread's private slot
   uint32_t sub_words;    // deeper-table words kept in shared memory (0: global)
   uint32_t pad;
@@ -97,7 +100,7 @@ struct KBatch {
 // [192,448)    code lengths by rotated exponent
 // [448,1472)   table 0 (rotated)
 // [1472, ...)  wide table (2^WB x 8 bytes)
-// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16), sign/mantissa
+// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16)
 // then         exponent array (stage_bytes), private slots (slot_words*T*4),
 //              deeper tables (sub_words*4)
 constexpr uint32_t kOffMbar = 0;
@@ -113,13 +116,9 @@ template <int T, int C>
 struct Layout {
   static constexpr uint32_t bits_bytes = T * C + 16;
   static constexpr uint32_t gaps_bytes = T * 5 / 8 + 16;
-  static constexpr uint32_t head_bytes = bits_bytes + gaps_bytes;  // per slot, before sm
+  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes;  // one stage slot
   static_assert(bits_bytes % 16 == 0 && gaps_bytes % 16 == 0, "alignment");
 };
-
-__host__ __device__ constexpr uint32_t slot_stride(uint32_t head, uint32_t stage) {
-  return head + stage;
-}
 
 __device__ __forceinline__ uint32_t rot8x3(uint32_t v) {
   // rotate each of the low three bytes right by one bit
@@ -204,8 +203,10 @@ __device__ __forceinline__ bool decode_one(uint32_t win, const uint32_t *__restr
 
 // Derived table: entry i holds the codewords that lie wholly inside the WB
 // bits i (at most kWideSyms): x = exponents (first in bits 0-7),
-// y = bits used << 8 | count << 12.  y == 0: the first codeword is longer
-// than WB bits (or invalid) and takes the slow path.
+// y = bits used | (8 * count) << 16, so that one add moves both the bit
+// position and the byte count of a packed (position, count) register.
+// y == 0: the first codeword is longer than WB bits (or invalid) and takes
+// the slow path.
 template <int T>
 __device__ void build_wide(uint2 *wide, const uint32_t *lut0, const uint8_t *lens,
                            const uint32_t *sub, uint32_t num_luts) {
@@ -237,60 +238,78 @@ __device__ void build_wide(uint2 *wide, const uint32_t *lut0, const uint8_t *len
       }
       if (stop || used >= kWideBits) break;
     }
-    wide[i] = n ? make_uint2(syms, (used << 8) | (n << 12)) : make_uint2(0, 0);
+    wide[i] = n ? make_uint2(syms, used | ((8u * n) << 16)) : make_uint2(0, 0);
   }
 }
 
-// Walk one thread's codewords [pos, end) (bit positions relative to its
+// 32 stream bits starting at bit `pos` of a chunk held as big-endian words.
+// Codeword starts lie below 8*C (the next chunk's gap covers the rest), so
+// for C = 8 the window comes from words (0,1) or (1,2).
+template <int C>
+__device__ __forceinline__ uint32_t window(const uint32_t (&w)[C / 4 + 2], uint32_t pos) {
+  if (C == 4) return __funnelshift_l(w[1], w[0], pos);
+  if (C == 8) {
+    const bool up = pos & 32u;
+    return __funnelshift_l(up ? w[2] : w[1], up ? w[1] : w[0], pos);
+  }
+  const uint32_t k = pos >> 5;
+  uint32_t hi = w[0], lo = w[1];
+#pragma unroll
+  for (int j = 1; j < C / 4; ++j)
+    if (k == (uint32_t)j) {
+      hi = w[j];
+      lo = w[j + 1];
+    }
+  return __funnelshift_l(lo, hi, pos);
+}
+
+// Walk one thread's codewords [start, end) (bit positions relative to its
 // chunk's first bit) and append their exponents to its private slot (word j
-// at slot[j*T]).  w: the chunk and the 8 bytes after it, big-endian words.
-// Returns the number of codewords; sets `bad` on inconsistent data.
+// at slot[j*T]).  `pk` packs the bit position (bits 0-15) with 8x the
+// bytes waiting in the 64-bit accumulator a1:a0 (bits 16-23).  Returns the
+// number of codewords; sets `bad` on inconsistent data.
 template <int T, int C, bool MASKED>
-__device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 2], int pos,
+__device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 2], int start,
                                                  const int end, const uint2 *__restrict__ wide,
                                                  const uint32_t *__restrict__ lut0,
                                                  const uint8_t *__restrict__ lens,
                                                  const uint32_t *sub, uint32_t num_luts,
                                                  uint32_t *slot, uint32_t slot_words, int &bad) {
-  constexpr int NW = C / 4 + 2;
-  uint32_t a0 = 0, a1 = 0, sh = 0, words = 0;
-#pragma unroll
-  for (int k = 0; k < NW - 1; ++k) {
-    const int lim = min(32 * (k + 1), end);
-    const uint32_t hi = w[k], lo = w[k + 1];
-    while (pos < lim) {
-      const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)pos);  // bits [pos, pos+32)
-      const uint2 e = wide[win >> (32 - kWideBits)];
-      uint32_t syms = e.x, nbits = (e.y >> 8) & 15u, nsym = e.y >> 12;
-      const bool slow = MASKED ? nbits == 0 : (nbits == 0 || (int)nbits > end - pos);
-      if (slow) {
-        uint32_t s, l;
-        if (!decode_one(win, lut0, lens, sub, num_luts, s, l)) {
-          bad = DF11_DEV_ERR_TABLE;
-          return 0;
-        }
-        syms = s;
-        nbits = l;
-        nsym = 1;
+  uint32_t a0 = 0, a1 = 0, pk = (uint32_t)start;
+  uint32_t *sp = slot;
+  uint32_t *const sp_end = slot + slot_words * T;
+  while ((int)(pk & 0xFFFFu) < end) {
+    const uint32_t pos = pk & 0xFFFFu;
+    const uint32_t win = window<C>(w, pos);
+    const uint2 e = wide[win >> (32 - kWideBits)];
+    uint32_t ex = e.x, ey = e.y;
+    if (ey == 0 || (!MASKED && (int)(ey & 0xFFFFu) > end - (int)pos)) {
+      // rare: a codeword longer than WB bits, or (unmasked streams) an
+      // entry running past the region's end: one codeword via the format's
+      // own tables
+      uint32_t sym, len;
+      if (!decode_one(win, lut0, lens, sub, num_luts, sym, len)) {
+        bad = DF11_DEV_ERR_TABLE;
+        return 0;
       }
-      a0 |= syms << sh;
-      a1 |= __funnelshift_l(syms, 0u, sh);  // bytes pushed past the low word
-      sh += nsym << 3;
-      if (sh >= 32) {
-        if (words < slot_words) slot[words * T] = a0;
-        ++words;
-        a0 = a1;
-        a1 = 0;
-        sh -= 32;
-      }
-      pos += (int)nbits;
+      ex = sym;
+      ey = len | (8u << 16);
+    }
+    const uint32_t sh = pk >> 16;
+    a0 |= ex << sh;
+    a1 |= __funnelshift_l(ex, 0u, sh);  // bytes pushed past the low word
+    pk += ey;
+    if (pk >= (32u << 16)) {  // a full word: flush it
+      if (sp < sp_end) *sp = a0;
+      sp += T;
+      a0 = a1;
+      a1 = 0;
+      pk -= 32u << 16;
     }
   }
-  if (sh) {
-    if (words < slot_words) slot[words * T] = a0;
-  }
-  if (pos != end) bad = DF11_DEV_ERR_OVERRUN;
-  return words * 4 + (sh >> 3);
+  if ((pk >> 16) && sp < sp_end) *sp = a0;
+  if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
+  return (uint32_t)(sp - slot) / T * 4u + (pk >> 19);
 }
 
 // four sign/mantissa bytes and four rotated exponents -> four BF16 words
@@ -305,8 +324,13 @@ __device__ __forceinline__ uint16_t fuse1(uint32_t sm, uint32_t er) {
   return (uint16_t)(((sm & 0x80u) << 8) | ((er & 0x7Fu) << 8) | (er & 0x80u) | (sm & 0x7Fu));
 }
 
-// Thread 0: queue the copies of block b into stage slot `slot` (or, for
-// inconsistent block positions, an empty completion flagged not ok).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Thread 0: queue the copies of block b into stage slot `stage` (or, for
+// inconsistent block positions, an empty completion flagged not ok) and an
+// L2 prefetch of its sign/mantissa bytes.
 template <int T, int C>
 __device__ __forceinline__ void issue_block(const KTensor &tk, uint32_t b, uint32_t P0,
                                             uint32_t P1, uint8_t *stage, uint4 *meta,
@@ -320,18 +344,17 @@ __device__ __forceinline__ void issue_block(const KTensor &tk, uint32_t b, uint3
     mbar_arrive_expect_tx(bar, 0);
     return;
   }
-  const uint32_t sm_begin = P0 & ~15u;
-  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
-  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes + sm_bytes);
+  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes);
   bulk_g2s(smem_addr(stage), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, bar);
   bulk_g2s(smem_addr(stage + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
            bar);
-  if (sm_bytes)
-    bulk_g2s(smem_addr(stage + L::head_bytes), tk.sign_mantissa + sm_begin, sm_bytes, bar);
+  const uint32_t sm_begin = P0 & ~15u;
+  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
+  if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
 }
 
 template <int T, int C>
-__global__ void __launch_bounds__(T) df11_decode_kernel(const __grid_constant__ KBatch kb) {
+__global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_constant__ KBatch kb) {
   using L = Layout<T, C>;
   constexpr int NW = C / 4 + 2;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -342,8 +365,7 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const __grid_constant__ 
   uint32_t *lut0_s = reinterpret_cast<uint32_t *>(smem + kOffLut0);
   uint2 *wide_s = reinterpret_cast<uint2 *>(smem + kOffWide);
   uint8_t *stages = smem + kOffStages;
-  const uint32_t stride_bytes = slot_stride(L::head_bytes, kb.stage_bytes);
-  uint8_t *ex_s = stages + 2 * stride_bytes;
+  uint8_t *ex_s = stages + 2 * L::slot_bytes;
   uint32_t *slots = reinterpret_cast<uint32_t *>(ex_s + kb.stage_bytes);
   uint32_t *sub_s = slots + kb.slot_words * T;
 
@@ -393,11 +415,11 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const __grid_constant__ 
   uint32_t k = 0;
   for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
     const uint32_t s = k & 1;
-    uint8_t *stage = stages + s * stride_bytes;
+    const uint8_t *stage = stages + s * L::slot_bytes;
     // queue the next block into the other slot (freed by the barrier that
     // ended the previous iteration)
     if (tid == 0 && b + ctas < tk.num_blocks) {
-      issue_block<T, C>(tk, b + ctas, nP0, nP1, stages + (s ^ 1) * stride_bytes, &meta[s ^ 1],
+      issue_block<T, C>(tk, b + ctas, nP0, nP1, stages + (s ^ 1) * L::slot_bytes, &meta[s ^ 1],
                         s ? bar0 : bar1, kb.stage_bytes);
       const uint32_t nb = b + 2 * ctas;
       if (nb < tk.num_blocks) {
@@ -414,10 +436,13 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const __grid_constant__ 
       __syncthreads();
       continue;
     }
+    const uint32_t head = P0 & 15u, span = head + expected;
+    // exponent array to zero: its boundary words are assembled with atomic OR
+    for (uint32_t i = tid; i < (span + 15u) >> 4; i += T)
+      reinterpret_cast<uint4 *>(ex_s)[i] = make_uint4(0, 0, 0, 0);
+
     const uint8_t *bits_s = stage;
     const uint8_t *gaps_s = stage + L::bits_bytes;
-    const uint8_t *sm_s = stage + L::head_bytes;
-
     // this thread's region, relative to its chunk's first bit
     const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
     int start = read_gap(gaps_s, tid);
@@ -480,49 +505,57 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const __grid_constant__ 
     }
 
     // compact: slot bytes [0, cnt) -> ex_s[d, d+cnt); exponent i of the
-    // array belongs to element (P0 & ~15) + i
-    {
-      const uint32_t d = (P0 & 15u) + excl;
+    // array belongs to element (P0 & ~15) + i.  Destination word k holds
+    // slot bytes 4k-s .. 4k-s+3 (s = d & 3): a funnel shift of slot words
+    // k-1 and k.  The first and last words are shared with the neighbours.
+    if (cnt) {
+      const uint32_t d = head + excl, e_end = d + cnt;
+      const uint32_t q0 = d >> 2, last = ((e_end - 1) >> 2) - q0;
+      const uint32_t s8 = (d & 3u) * 8u, r = e_end & 3u;
+      const uint32_t mlast = r ? 0xFFFFFFFFu >> (32u - 8u * r) : 0xFFFFFFFFu;
       const uint32_t *sl = slots + tid;
-      const uint32_t h = (4u - (d & 3u)) & 3u;  // bytes before the first aligned word
-      uint32_t cur = cnt ? sl[0] : 0u;
-      const uint32_t nh = cnt < h ? cnt : h;
-      for (uint32_t i = 0; i < nh; ++i) ex_s[d + i] = (uint8_t)(cur >> (8 * i));
-      if (cnt > h) {
-        // aligned words: source bytes h+4j .. h+4j+3 = words j, j+1 shifted by h bytes
-        const uint32_t full = (cnt - h) >> 2;
-        uint32_t *dst = reinterpret_cast<uint32_t *>(ex_s + d + h);
-        for (uint32_t j = 0; j < full; ++j) {
-          const uint32_t nxt = sl[(j + 1) * T];  // within the slot: j+1 <= cnt/4
-          dst[j] = __funnelshift_r(cur, nxt, 8 * h);
-          cur = nxt;
+      uint32_t *ex32 = reinterpret_cast<uint32_t *>(ex_s) + q0;
+      uint32_t prev = sl[0];
+      uint32_t v = __funnelshift_l(0u, prev, s8) & (0xFFFFFFFFu << s8);
+      if (last == 0) {
+        atomicOr(ex32, v & mlast);
+      } else {
+        atomicOr(ex32, v);
+        for (uint32_t j = 1; j < last; ++j) {  // slot word j <= cnt/4: inside the slot
+          const uint32_t cur = sl[j * T];
+          ex32[j] = __funnelshift_l(prev, cur, s8);
+          prev = cur;
         }
-        for (uint32_t i = h + 4 * full; i < cnt; ++i)
-          ex_s[d + i] = (uint8_t)(sl[(i >> 2) * T] >> (8 * (i & 3)));
+        const uint32_t cur = sl[last * T];
+        atomicOr(ex32 + last, __funnelshift_l(prev, cur, s8) & mlast);
       }
     }
     __syncthreads();
 
-    // output: fuse and store, 16 elements per thread per step
+    // output: fuse and store, 16 elements per thread per step; the ragged
+    // first and last groups one element per lane
     {
-      const uint32_t head = P0 & 15u;
-      uint16_t *out = tk.out + (P0 & ~15u);
-      const uint32_t span = head + expected;
-      const uint32_t groups = (span + 15u) >> 4;
-      for (uint32_t g = tid; g < groups; g += T) {
+      const uint32_t sm_begin = P0 & ~15u;
+      uint16_t *out = tk.out + sm_begin;
+      const uint8_t *smg = tk.sign_mantissa + sm_begin;
+      const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
+      for (uint32_t g = g_begin + tid; g < g_end; g += T) {
         const uint32_t i0 = g << 4;
-        if (i0 >= head && i0 + 16u <= span) {
-          const uint4 sv = *reinterpret_cast<const uint4 *>(sm_s + i0);
-          const uint4 rv = *reinterpret_cast<const uint4 *>(ex_s + i0);
-          const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
-          const uint2 dd = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
-          uint4 *o = reinterpret_cast<uint4 *>(out + i0);
-          o[0] = make_uint4(a.x, a.y, c.x, c.y);
-          o[1] = make_uint4(dd.x, dd.y, f.x, f.y);
-        } else {
-          const uint32_t lo = i0 > head ? i0 : head, hi = i0 + 16u < span ? i0 + 16u : span;
-          for (uint32_t i = lo; i < hi; ++i) out[i] = fuse1(sm_s[i], ex_s[i]);
-        }
+        const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(smg + i0));
+        const uint4 rv = *reinterpret_cast<const uint4 *>(ex_s + i0);
+        const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
+        const uint2 dd = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+        uint4 *o = reinterpret_cast<uint4 *>(out + i0);
+        o[0] = make_uint4(a.x, a.y, c.x, c.y);
+        o[1] = make_uint4(dd.x, dd.y, f.x, f.y);
+      }
+      if (warp == T / 32 - 1) {  // lanes 0-15: first group, 16-31: last group
+        const uint32_t gl = (span - 1) >> 4;
+        const bool first_partial = head != 0 || span < 16;
+        const bool last_partial = (span & 15u) != 0 && gl != 0;
+        const uint32_t i = lane < 16 ? (uint32_t)lane : (gl << 4) + (uint32_t)(lane - 16);
+        const bool mine = lane < 16 ? first_partial : last_partial;
+        if (mine && i >= head && i < span) out[i] = fuse1(smg[i], ex_s[i]);
       }
     }
     __syncthreads();  // stage slot, exponent array and private slots free again
@@ -546,8 +579,8 @@ uint32_t slot_words_for(uint32_t max_chunk_elems) { return (max_chunk_elems + 3u
 
 size_t shared_bytes(uint32_t C, uint32_t T, uint32_t stage, uint32_t slot_words,
                     uint32_t sub_words) {
-  const size_t head = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16;
-  return (size_t)kOffStages + 2 * (head + stage) + stage + (size_t)slot_words * T * 4 +
+  const size_t slot = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16;
+  return (size_t)kOffStages + 2 * slot + stage + (size_t)slot_words * T * 4 +
          (size_t)sub_words * 4;
 }
 
