@@ -96,19 +96,19 @@ struct KBatch {
 // ---- shared memory layout --------------------------------------------------
 // [0,16)       2 mbarriers (one per stage slot)
 // [16,48)      2 x {P0, P1, ok, 0}: block positions of the block in each slot
-// [48,192)     36 ints of scan scratch
-// [192,448)    code lengths by rotated exponent
-// [448,1472)   table 0 (rotated)
-// [1472, ...)  wide table (2^WB x 8 bytes)
+// [48,304)     2 x 32 ints of scan scratch (alternating between blocks)
+// [304,560)    code lengths by rotated exponent
+// [560,1584)   table 0 (rotated)
+// [1584, ...)  wide table (2^WB x 8 bytes)
 // then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16)
 // then         exponent array (stage_bytes), private slots (slot_words*T*4),
 //              deeper tables (sub_words*4)
 constexpr uint32_t kOffMbar = 0;
 constexpr uint32_t kOffMeta = 16;
 constexpr uint32_t kOffScan = 48;
-constexpr uint32_t kOffLens = 192;
-constexpr uint32_t kOffLut0 = 448;
-constexpr uint32_t kOffWide = 1472;
+constexpr uint32_t kOffLens = 304;
+constexpr uint32_t kOffLut0 = 560;
+constexpr uint32_t kOffWide = 1584;
 constexpr uint32_t kWideBytes = 8u << kWideBits;
 constexpr uint32_t kOffStages = kOffWide + kWideBytes;
 
@@ -131,6 +131,21 @@ __device__ __forceinline__ void report(int32_t *err, int32_t code) {
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// Shared-memory accesses through 32-bit shared-window addresses.
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -242,11 +257,12 @@ __device__ void build_wide(uint2 *wide, const uint32_t *lut0, const uint8_t *len
   }
 }
 
-// 32 stream bits starting at bit `pos` of a chunk held as big-endian words.
-// Codeword starts lie below 8*C (the next chunk's gap covers the rest), so
-// for C = 8 the window comes from words (0,1) or (1,2).
+// 32 stream bits starting at bit `pos` of a chunk held as big-endian words
+// (the chunk and the 4 bytes after it).  Codeword starts lie below 8*C (the
+// next chunk's gap covers the rest), so for C = 8 the window comes from words
+// (0,1) or (1,2).
 template <int C>
-__device__ __forceinline__ uint32_t window(const uint32_t (&w)[C / 4 + 2], uint32_t pos) {
+__device__ __forceinline__ uint32_t window(const uint32_t (&w)[C / 4 + 1], uint32_t pos) {
   if (C == 4) return __funnelshift_l(w[1], w[0], pos);
   if (C == 8) {
     const bool up = pos & 32u;
@@ -264,26 +280,25 @@ __device__ __forceinline__ uint32_t window(const uint32_t (&w)[C / 4 + 2], uint3
 }
 
 // Walk one thread's codewords [start, end) (bit positions relative to its
-// chunk's first bit) and append their exponents to its private slot (word j
-// at slot[j*T]).  `pk` packs the bit position (bits 0-15) with 8x the
-// bytes waiting in the 64-bit accumulator a1:a0 (bits 16-23).  Returns the
-// number of codewords; sets `bad` on inconsistent data.
+// chunk's first bit) and append their exponents to its private slot: word j
+// at shared address slot + 4*T*j.  `pk` packs the bit position (bits 0-15)
+// with 8x the bytes waiting in the 64-bit accumulator a1:a0 (bits 16-23).
+// The current word is stored after every lookup and the slot address moves
+// on when it is full, so no branch but the loop's and the rare slow path's.
+// Returns the number of codewords; sets `bad` on inconsistent data.
 template <int T, int C, bool MASKED>
-__device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 2], int start,
-                                                 const int end, const uint2 *__restrict__ wide,
+__device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1], int start,
+                                                 const int end, uint32_t wide,
                                                  const uint32_t *__restrict__ lut0,
                                                  const uint8_t *__restrict__ lens,
                                                  const uint32_t *sub, uint32_t num_luts,
-                                                 uint32_t *slot, uint32_t slot_words, int &bad) {
-  uint32_t a0 = 0, a1 = 0, pk = (uint32_t)start;
-  uint32_t *sp = slot;
-  uint32_t *const sp_end = slot + slot_words * T;
+                                                 uint32_t slot, uint32_t slot_words, int &bad) {
+  uint32_t a0 = 0, a1 = 0, pk = (uint32_t)start, sa = slot, words = 0;
+  const uint32_t sa_last = slot + (slot_words - 1) * (4u * T);
   while ((int)(pk & 0xFFFFu) < end) {
-    const uint32_t pos = pk & 0xFFFFu;
-    const uint32_t win = window<C>(w, pos);
-    const uint2 e = wide[win >> (32 - kWideBits)];
-    uint32_t ex = e.x, ey = e.y;
-    if (ey == 0 || (!MASKED && (int)(ey & 0xFFFFu) > end - (int)pos)) {
+    const uint32_t win = window<C>(w, pk & 0xFFFFu);
+    uint2 e = lds64(wide + ((win >> (32 - kWideBits)) << 3));
+    if (e.y == 0 || (!MASKED && (int)(e.y & 0xFFFFu) > end - (int)(pk & 0xFFFFu))) {
       // rare: a codeword longer than WB bits, or (unmasked streams) an
       // entry running past the region's end: one codeword via the format's
       // own tables
@@ -292,24 +307,24 @@ __device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 2],
         bad = DF11_DEV_ERR_TABLE;
         return 0;
       }
-      ex = sym;
-      ey = len | (8u << 16);
+      e = make_uint2(sym, len | (8u << 16));
     }
     const uint32_t sh = pk >> 16;
-    a0 |= ex << sh;
-    a1 |= __funnelshift_l(ex, 0u, sh);  // bytes pushed past the low word
-    pk += ey;
-    if (pk >= (32u << 16)) {  // a full word: flush it
-      if (sp < sp_end) *sp = a0;
-      sp += T;
+    a0 |= e.x << sh;
+    a1 |= __funnelshift_l(e.x, 0u, sh);  // bytes pushed past the low word
+    pk += e.y;
+    sts32(sa, a0);
+    if (pk >= (32u << 16)) {  // the word is complete: move on
+      sa = min(sa + 4u * T, sa_last);
+      ++words;
       a0 = a1;
       a1 = 0;
       pk -= 32u << 16;
     }
   }
-  if ((pk >> 16) && sp < sp_end) *sp = a0;
+  if (pk >> 16) sts32(sa, a0);
   if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
-  return (uint32_t)(sp - slot) / T * 4u + (pk >> 19);
+  return words * 4u + (pk >> 19);
 }
 
 // four sign/mantissa bytes and four rotated exponents -> four BF16 words
@@ -356,7 +371,7 @@ __device__ __forceinline__ void issue_block(const KTensor &tk, uint32_t b, uint3
 template <int T, int C>
 __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_constant__ KBatch kb) {
   using L = Layout<T, C>;
-  constexpr int NW = C / 4 + 2;
+  constexpr int NW = C / 4 + 1;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + kOffMbar);
   uint4 *meta = reinterpret_cast<uint4 *>(smem + kOffMeta);
@@ -407,6 +422,8 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
     for (uint32_t i = tid; i < sub_words; i += T) sub_s[i] = sub[i];
     sub = sub_s;
   }
+  for (uint32_t i = tid; i < kb.stage_bytes / 16; i += T)  // zeroed once; each
+    reinterpret_cast<uint4 *>(ex_s)[i] = make_uint4(0, 0, 0, 0);  // output re-zeroes
   __syncthreads();
   build_wide<T>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
   __syncthreads();
@@ -437,9 +454,6 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
       continue;
     }
     const uint32_t head = P0 & 15u, span = head + expected;
-    // exponent array to zero: its boundary words are assembled with atomic OR
-    for (uint32_t i = tid; i < (span + 15u) >> 4; i += T)
-      reinterpret_cast<uint4 *>(ex_s)[i] = make_uint4(0, 0, 0, 0);
 
     const uint8_t *bits_s = stage;
     const uint8_t *gaps_s = stage + L::bits_bytes;
@@ -456,51 +470,46 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
 #pragma unroll
     for (int j = 0; j < NW; ++j) {
       w[j] = __byte_perm(*reinterpret_cast<const uint32_t *>(bits_s + tid * C + 4 * j), 0, 0x0123);
-      if (tk.masked) {  // ones from bit `end` on
-        const int lo = end - 32 * j;
-        if (lo <= 0) w[j] = 0xFFFFFFFFu;
-        else if (lo < 32) w[j] |= 0xFFFFFFFFu >> lo;
-      }
+      if (tk.masked)  // ones from bit `end` on
+        w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
     }
 
     uint32_t cnt = 0;
     if (!bad) {
+      const uint32_t slot = smem_addr(slots + tid);
       if (tk.masked)
-        cnt = decode_chunk<T, C, true>(w, start, end, wide_s, lut0_s, lens_s, sub, tk.num_luts,
-                                       slots + tid, kb.slot_words, bad);
+        cnt = decode_chunk<T, C, true>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
+                                       tk.num_luts, slot, kb.slot_words, bad);
       else
-        cnt = decode_chunk<T, C, false>(w, start, end, wide_s, lut0_s, lens_s, sub, tk.num_luts,
-                                        slots + tid, kb.slot_words, bad);
+        cnt = decode_chunk<T, C, false>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
+                                        tk.num_luts, slot, kb.slot_words, bad);
       if (!bad && cnt > tk.max_chunk_elems) bad = DF11_DEV_ERR_CAPACITY;
     }
 
-    // block exclusive scan of the counts
+    // block exclusive scan of the counts: warp totals (bit 31: a thread of
+    // the warp found bad data) to shared memory, one barrier, then every
+    // warp adds up the totals of the warps before it
     uint32_t incl = cnt;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
       if (lane >= d) incl += v;
     }
-    if (lane == 31) scan[warp] = (int)incl;
+    const uint32_t warp_bad = __any_sync(0xFFFFFFFFu, bad != 0) ? 0x80000000u : 0u;
+    if (lane == 31) scan[(s << 5) + warp] = (int)(incl | warp_bad);
     __syncthreads();
-    if (warp == 0) {
-      const uint32_t v = lane < T / 32 ? (uint32_t)scan[lane] : 0u;
-      uint32_t sc = v;
+    uint32_t before = 0, total = 0, any_bad = 0;
 #pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, sc, d);
-        if (lane >= d) sc += u;
-      }
-      if (lane < T / 32) scan[lane] = (int)(sc - v);
-      if (lane == 31) scan[32] = (int)sc;
+    for (int j = 0; j < T / 32; ++j) {
+      const uint32_t v = (uint32_t)scan[(s << 5) + j];
+      any_bad |= v;
+      before += j < warp ? (v & 0x7FFFFFFFu) : 0u;
+      total += v & 0x7FFFFFFFu;
     }
-    const int any_bad = __syncthreads_or(bad);
-    const uint32_t excl = (uint32_t)scan[warp] + incl - cnt;
-    const uint32_t total = (uint32_t)scan[32];
-    if (any_bad || total != expected) {
+    const uint32_t excl = before + incl - cnt;
+    if ((any_bad >> 31) || total != expected) {
       if (bad) report(kb.err, bad);
-      else if (tid == 0 && !any_bad) report(kb.err, DF11_DEV_ERR_COUNT);
-      __syncthreads();
+      else if (tid == 0 && !(any_bad >> 31)) report(kb.err, DF11_DEV_ERR_COUNT);
       continue;
     }
 
@@ -513,20 +522,20 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
       const uint32_t q0 = d >> 2, last = ((e_end - 1) >> 2) - q0;
       const uint32_t s8 = (d & 3u) * 8u, r = e_end & 3u;
       const uint32_t mlast = r ? 0xFFFFFFFFu >> (32u - 8u * r) : 0xFFFFFFFFu;
-      const uint32_t *sl = slots + tid;
+      const uint32_t sl = smem_addr(slots + tid);
       uint32_t *ex32 = reinterpret_cast<uint32_t *>(ex_s) + q0;
-      uint32_t prev = sl[0];
-      uint32_t v = __funnelshift_l(0u, prev, s8) & (0xFFFFFFFFu << s8);
+      uint32_t prev = lds32(sl);
+      const uint32_t v = prev << s8;
       if (last == 0) {
         atomicOr(ex32, v & mlast);
       } else {
         atomicOr(ex32, v);
         for (uint32_t j = 1; j < last; ++j) {  // slot word j <= cnt/4: inside the slot
-          const uint32_t cur = sl[j * T];
-          ex32[j] = __funnelshift_l(prev, cur, s8);
+          const uint32_t cur = lds32(sl + j * (4u * T));
+          sts32(smem_addr(ex32 + j), __funnelshift_l(prev, cur, s8));
           prev = cur;
         }
-        const uint32_t cur = sl[last * T];
+        const uint32_t cur = lds32(sl + last * (4u * T));
         atomicOr(ex32 + last, __funnelshift_l(prev, cur, s8) & mlast);
       }
     }
@@ -542,7 +551,9 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
       for (uint32_t g = g_begin + tid; g < g_end; g += T) {
         const uint32_t i0 = g << 4;
         const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(smg + i0));
-        const uint4 rv = *reinterpret_cast<const uint4 *>(ex_s + i0);
+        uint4 *rp = reinterpret_cast<uint4 *>(ex_s + i0);
+        const uint4 rv = *rp;
+        *rp = make_uint4(0, 0, 0, 0);  // leave the array zeroed for the next block
         const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
         const uint2 dd = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
         uint4 *o = reinterpret_cast<uint4 *>(out + i0);
@@ -556,9 +567,14 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
         const uint32_t i = lane < 16 ? (uint32_t)lane : (gl << 4) + (uint32_t)(lane - 16);
         const bool mine = lane < 16 ? first_partial : last_partial;
         if (mine && i >= head && i < span) out[i] = fuse1(smg[i], ex_s[i]);
+        if (mine) ex_s[i] = 0;
       }
     }
-    __syncthreads();  // stage slot, exponent array and private slots free again
+    // No barrier here: the next block's decode writes only private slots
+    // (last read before the barrier above), its compaction writes the
+    // exponent array only after its scan barrier, which every thread reaches
+    // after finishing this output, and the stage slot refilled next was
+    // last read before this block's scan barrier.
   }
 }
 
