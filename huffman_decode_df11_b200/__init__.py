@@ -60,6 +60,7 @@ class TensorDesc(ctypes.Structure):
     _fields_ = [
         ("bitstream", ctypes.c_void_p),
         ("gaps", ctypes.c_void_p),
+        ("chunk_counts", ctypes.c_void_p),
         ("block_out_pos", ctypes.c_void_p),
         ("luts", ctypes.c_void_p),
         ("code_lengths", ctypes.c_void_p),
@@ -81,6 +82,8 @@ class HostTensor(ctypes.Structure):
         ("luts", ctypes.POINTER(ctypes.c_uint32)),
         ("sign_mantissa", ctypes.POINTER(ctypes.c_uint8)),
         ("sign_mantissa_bytes", ctypes.c_uint64),
+        ("chunk_counts", ctypes.POINTER(ctypes.c_uint8)),
+        ("chunk_counts_bytes", ctypes.c_uint64),
     ]
 
 
@@ -147,6 +150,7 @@ class Df11Host:
     block_out_pos: np.ndarray  # uint32[num_blocks + 1]
     luts: np.ndarray           # uint32[num_luts * 256]
     sign_mantissa: np.ndarray  # uint8 (n rounded up to 16)
+    chunk_counts: np.ndarray   # uint8, codewords starting in each chunk
     shape: tuple = ()
 
     @property
@@ -154,10 +158,11 @@ class Df11Host:
         return int(self.params.n)
 
     def compressed_bytes(self) -> int:
-        """Bytes a decode reads: bitstream + gaps + positions + tables +
-        code lengths + sign/mantissa, as stored."""
+        """Bytes stored: bitstream + gaps + positions + tables + code lengths
+        + sign/mantissa + chunk counts."""
         return (self.bitstream.nbytes + self.gaps.nbytes + self.block_out_pos.nbytes
-                + self.luts.nbytes + 256 + self.sign_mantissa.nbytes)
+                + self.luts.nbytes + 256 + self.sign_mantissa.nbytes
+                + self.chunk_counts.nbytes)
 
 
 def _as_u16_numpy(w) -> np.ndarray:
@@ -201,6 +206,7 @@ def compress(w, chunk_bytes: int = 8, threads_per_block: int = 256,
             block_out_pos=_np_copy(h.block_out_pos, p.num_blocks + 1, np.uint32),
             luts=_np_copy(h.luts, p.num_luts * 256, np.uint32),
             sign_mantissa=_np_copy(h.sign_mantissa, h.sign_mantissa_bytes, np.uint8),
+            chunk_counts=_np_copy(h.chunk_counts, h.chunk_counts_bytes, np.uint8),
             shape=shape,
         )
     finally:
@@ -221,6 +227,7 @@ class Df11Device:
     luts: torch.Tensor
     code_lengths: torch.Tensor
     sign_mantissa: torch.Tensor
+    chunk_counts: Optional[torch.Tensor] = None
     shape: tuple = ()
 
     @property
@@ -234,10 +241,12 @@ class Df11Device:
     def compressed_bytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
                    (self.bitstream, self.gaps, self.block_out_pos, self.luts,
-                    self.code_lengths, self.sign_mantissa))
+                    self.code_lengths, self.sign_mantissa)
+                   + ((self.chunk_counts,) if self.chunk_counts is not None else ()))
 
-    def desc(self, out: torch.Tensor) -> TensorDesc:
-        return TensorDesc(self.bitstream.data_ptr(), self.gaps.data_ptr(),
+    def desc(self, out: torch.Tensor, counts: bool = True) -> TensorDesc:
+        cc = self.chunk_counts.data_ptr() if (counts and self.chunk_counts is not None) else None
+        return TensorDesc(self.bitstream.data_ptr(), self.gaps.data_ptr(), cc,
                           self.block_out_pos.data_ptr(), self.luts.data_ptr(),
                           self.code_lengths.data_ptr(), self.sign_mantissa.data_ptr(),
                           out.data_ptr(), self.params)
@@ -260,6 +269,7 @@ def to_device(h: Df11Host, device="cuda") -> Df11Device:
         luts=_np_to(h.luts.view(np.int32), device),
         code_lengths=_np_to(h.code_lengths, device),
         sign_mantissa=_np_to(h.sign_mantissa, device),
+        chunk_counts=_np_to(h.chunk_counts, device),
         shape=h.shape,
     )
 
@@ -275,15 +285,19 @@ def empty_output(d: Df11Device) -> torch.Tensor:
 
 
 def decode(d: Df11Device, out: Optional[torch.Tensor] = None,
-           err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+           err: Optional[torch.Tensor] = None, stream=None,
+           counts: bool = True) -> torch.Tensor:
     """Decode into `out` (a flat BF16/int16 device tensor of n elements,
     allocated if None).  Asynchronous on `stream` (default: current stream).
     `err` is an optional int32 device tensor the kernel writes error codes
-    into (see check_device_error)."""
+    into (see check_device_error).  With counts (the default, when the tensor
+    carries chunk counts) the one-pass decode is used; counts=False runs the
+    format the pages describe through df11_decode (count by decoding)."""
     if out is None:
         out = empty_output(d)
-    if out.numel() != d.n or not out.is_contiguous() or out.element_size() != 2:
-        raise ValueError("out must be a contiguous 2-byte tensor with n elements")
+    _check_out(d, out)
+    if counts and d.chunk_counts is not None:
+        return decode_batched([d], [out], err=err, stream=stream)[0]
     p = Params.from_buffer_copy(d.params)
     _check(lib().df11_decode(
         d.bitstream.data_ptr(), d.gaps.data_ptr(), d.block_out_pos.data_ptr(),
@@ -294,15 +308,20 @@ def decode(d: Df11Device, out: Optional[torch.Tensor] = None,
     return out
 
 
+def _check_out(d: Df11Device, out: torch.Tensor):
+    if out.numel() != d.n or not out.is_contiguous() or out.element_size() != 2:
+        raise ValueError("out must be a contiguous 2-byte tensor with n elements")
+
+
 def decode_batched(ds: Sequence[Df11Device], outs: Sequence[torch.Tensor],
-                   err: Optional[torch.Tensor] = None, stream=None):
+                   err: Optional[torch.Tensor] = None, stream=None,
+                   counts: bool = True):
     """Decode several tensors with one launch per 16 tensors."""
     if len(ds) != len(outs):
         raise ValueError("one output per tensor")
     for d, o in zip(ds, outs):
-        if o.numel() != d.n or not o.is_contiguous() or o.element_size() != 2:
-            raise ValueError("each out must be a contiguous 2-byte tensor with n elements")
-    arr = (TensorDesc * max(len(ds), 1))(*[d.desc(o) for d, o in zip(ds, outs)])
+        _check_out(d, o)
+    arr = (TensorDesc * max(len(ds), 1))(*[d.desc(o, counts) for d, o in zip(ds, outs)])
     _check(lib().df11_decode_batched(arr, len(ds),
                                      err.data_ptr() if err is not None else None,
                                      _stream_handle(stream)), "df11_decode_batched")

@@ -257,7 +257,7 @@ extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
                                   df11_host_tensor *out) {
   if (!out || (n && !w)) return DF11_ERR_NULL;
   std::memset(out, 0, sizeof(*out));
-  if (C < 4 || C > 64 || C % 4) return DF11_ERR_INVALID;
+  if (C < 4 || C > 28 || C % 4) return DF11_ERR_INVALID;  // counts fit a byte
   if (T < 128 || T > 1024 || T % 128) return DF11_ERR_INVALID;
   if (n >= (1ull << 32)) return DF11_ERR_TOO_LARGE;
   int workers = num_threads > 0 ? num_threads : (int)std::thread::hardware_concurrency();
@@ -401,8 +401,18 @@ extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
   uint32_t mx = 0;
   for (uint32_t b = 0; b < p.num_blocks; ++b) mx = std::max(mx, bpos[b + 1] - bpos[b]);
   p.max_block_elems = mx;
+  out->chunk_counts_bytes = chunks + 16;
+  out->chunk_counts = (uint8_t *)std::calloc(out->chunk_counts_bytes, 1);
+  if (!out->chunk_counts) {
+    df11_host_tensor_free(out);
+    return DF11_ERR_NOMEM;
+  }
   uint32_t mc = 0;
-  for (uint64_t c = 0; c < chunks; ++c) mc = std::max(mc, first_elem[c + 1] - first_elem[c]);
+  for (uint64_t c = 0; c < chunks; ++c) {
+    const uint32_t k = first_elem[c + 1] - first_elem[c];
+    out->chunk_counts[c] = (uint8_t)k;
+    mc = std::max(mc, k);
+  }
   p.max_chunk_elems = mc;
   return DF11_OK;
 }
@@ -414,5 +424,6 @@ extern "C" void df11_host_tensor_free(df11_host_tensor *t) {
   std::free(t->block_out_pos);
   std::free(t->luts);
   std::free(t->sign_mantissa);
+  std::free(t->chunk_counts);
   std::memset(t, 0, sizeof(*t));
 }

@@ -66,6 +66,7 @@ constexpr int kWideSyms = 4;               // codewords per derived entry
 struct KTensor {
   const uint8_t *bitstream;
   const uint8_t *gaps;
+  const uint8_t *chunk_counts;  // NULL: count by decoding
   const uint32_t *block_out_pos;
   const uint32_t *luts;
   const uint8_t *code_lengths;
@@ -100,7 +101,7 @@ struct KBatch {
 // [304,560)    code lengths by rotated exponent
 // [560,1584)   table 0 (rotated)
 // [1584, ...)  wide table (2^WB x 8 bytes)
-// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16)
+// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16), counts (T)
 // then         exponent array (stage_bytes), private slots (slot_words*T*4),
 //              deeper tables (sub_words*4)
 constexpr uint32_t kOffMbar = 0;
@@ -116,8 +117,9 @@ template <int T, int C>
 struct Layout {
   static constexpr uint32_t bits_bytes = T * C + 16;
   static constexpr uint32_t gaps_bytes = T * 5 / 8 + 16;
-  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes;  // one stage slot
-  static_assert(bits_bytes % 16 == 0 && gaps_bytes % 16 == 0, "alignment");
+  static constexpr uint32_t counts_bytes = T;
+  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes + counts_bytes;  // one slot
+  static_assert(bits_bytes % 16 == 0 && gaps_bytes % 16 == 0 && T % 16 == 0, "alignment");
 };
 
 __device__ __forceinline__ uint32_t rot8x3(uint32_t v) {
@@ -146,6 +148,9 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
 }
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_or32(uint32_t a, uint32_t v) {
+  asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -179,13 +184,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (done) return true;
   }
   return false;
-}
-
-// 5-bit gap field k of a block's gap bytes (MSB-first packing)
-__device__ __forceinline__ int read_gap(const uint8_t *g, int k) {
-  const int bit = 5 * k;
-  const uint32_t v = ((uint32_t)g[bit >> 3] << 8) | g[(bit >> 3) + 1];
-  return (int)((v >> (11 - (bit & 7))) & 31u);
 }
 
 // One codeword at the start of a 32-bit window through the format's tables:
@@ -327,6 +325,52 @@ __device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1],
   return words * 4u + (pk >> 19);
 }
 
+// The same walk when the thread's output place is known before it decodes
+// (the format's chunk count): exponents go straight into the block's
+// exponent array at byte d onwards, as whole 32-bit words OR-ed into the
+// (zeroed) array, which also merges the words shared with neighbours.  The
+// accumulator starts d & 3 bytes in; `limit` is the last word the thread may
+// touch.  Returns the number of codewords decoded.
+template <int T, int C, bool MASKED>
+__device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1], int start,
+                                                  const int end, uint32_t wide,
+                                                  const uint32_t *__restrict__ lut0,
+                                                  const uint8_t *__restrict__ lens,
+                                                  const uint32_t *sub, uint32_t num_luts,
+                                                  uint32_t ex, uint32_t d, uint32_t limit,
+                                                  int &bad) {
+  uint32_t a0 = 0, a1 = 0, words = 0;
+  uint32_t pk = (uint32_t)start | (((d & 3u) * 8u) << 16);
+  uint32_t sa = ex + (d & ~3u);
+  while ((int)(pk & 0xFFFFu) < end) {
+    const uint32_t win = window<C>(w, pk & 0xFFFFu);
+    uint2 e = lds64(wide + ((win >> (32 - kWideBits)) << 3));
+    if (e.y == 0 || (!MASKED && (int)(e.y & 0xFFFFu) > end - (int)(pk & 0xFFFFu))) {
+      uint32_t sym, len;
+      if (!decode_one(win, lut0, lens, sub, num_luts, sym, len)) {
+        bad = DF11_DEV_ERR_TABLE;
+        return 0;
+      }
+      e = make_uint2(sym, len | (8u << 16));
+    }
+    const uint32_t sh = pk >> 16;
+    a0 |= e.x << sh;
+    a1 |= __funnelshift_l(e.x, 0u, sh);
+    pk += e.y;
+    if (pk >= (32u << 16)) {
+      red_or32(sa, a0);
+      sa = min(sa + 4u, limit);
+      ++words;
+      a0 = a1;
+      a1 = 0;
+      pk -= 32u << 16;
+    }
+  }
+  if (pk >> 16) red_or32(sa, a0);
+  if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
+  return words * 4u + (pk >> 19) - (d & 3u);
+}
+
 // four sign/mantissa bytes and four rotated exponents -> four BF16 words
 __device__ __forceinline__ uint2 fuse4(uint32_t sm4, uint32_t er4) {
   const uint32_t p0 = __byte_perm(sm4, er4, 0x5140), q0 = __byte_perm(sm4, er4, 0x1504);
@@ -359,10 +403,14 @@ __device__ __forceinline__ void issue_block(const KTensor &tk, uint32_t b, uint3
     mbar_arrive_expect_tx(bar, 0);
     return;
   }
-  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes);
+  const bool counts = tk.chunk_counts != nullptr;
+  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes + (counts ? L::counts_bytes : 0u));
   bulk_g2s(smem_addr(stage), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, bar);
   bulk_g2s(smem_addr(stage + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
            bar);
+  if (counts)
+    bulk_g2s(smem_addr(stage + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
+             L::counts_bytes, bar);
   const uint32_t sm_begin = P0 & ~15u;
   const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
   if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
@@ -457,10 +505,18 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
 
     const uint8_t *bits_s = stage;
     const uint8_t *gaps_s = stage + L::bits_bytes;
-    // this thread's region, relative to its chunk's first bit
+    // this thread's region, relative to its chunk's first bit: gaps of this
+    // chunk and the next, 10 bits at bit 5*tid of the big-endian gap words
     const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
-    int start = read_gap(gaps_s, tid);
-    int end = C * 8 + read_gap(gaps_s, tid + 1);
+    int start, end;
+    {
+      const uint32_t bit = 5u * (uint32_t)tid;
+      const uint32_t *g32 = reinterpret_cast<const uint32_t *>(gaps_s) + (bit >> 5);
+      const uint32_t v = __funnelshift_l(__byte_perm(g32[1], 0, 0x0123),
+                                         __byte_perm(g32[0], 0, 0x0123), bit);
+      start = (int)(v >> 27);
+      end = C * 8 + (int)((v >> 22) & 31u);
+    }
     if (chunk_bit >= tk.total_bits) {
       start = end = 0;
     } else if ((uint64_t)end > tk.total_bits - chunk_bit) {
@@ -473,9 +529,14 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
       if (tk.masked)  // ones from bit `end` on
         w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
     }
+    const bool direct = tk.chunk_counts != nullptr;  // uniform in the thread block
+    const uint32_t ex_addr = smem_addr(ex_s);
 
+    // counts: stored (direct) or by decoding into the private slot
     uint32_t cnt = 0;
-    if (!bad) {
+    if (direct) {
+      cnt = stage[L::bits_bytes + L::gaps_bytes + tid];
+    } else if (!bad) {
       const uint32_t slot = smem_addr(slots + tid);
       if (tk.masked)
         cnt = decode_chunk<T, C, true>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
@@ -483,8 +544,8 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
       else
         cnt = decode_chunk<T, C, false>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
                                         tk.num_luts, slot, kb.slot_words, bad);
-      if (!bad && cnt > tk.max_chunk_elems) bad = DF11_DEV_ERR_CAPACITY;
     }
+    if (!bad && cnt > tk.max_chunk_elems) bad = DF11_DEV_ERR_CAPACITY;
 
     // block exclusive scan of the counts: warp totals (bit 31: a thread of
     // the warp found bad data) to shared memory, one barrier, then every
@@ -510,36 +571,53 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
     if ((any_bad >> 31) || total != expected) {
       if (bad) report(kb.err, bad);
       else if (tid == 0 && !(any_bad >> 31)) report(kb.err, DF11_DEV_ERR_COUNT);
-      continue;
+      continue;  // nothing was written to the exponent array yet
     }
 
-    // compact: slot bytes [0, cnt) -> ex_s[d, d+cnt); exponent i of the
-    // array belongs to element (P0 & ~15) + i.  Destination word k holds
-    // slot bytes 4k-s .. 4k-s+3 (s = d & 3): a funnel shift of slot words
-    // k-1 and k.  The first and last words are shared with the neighbours.
-    if (cnt) {
-      const uint32_t d = head + excl, e_end = d + cnt;
-      const uint32_t q0 = d >> 2, last = ((e_end - 1) >> 2) - q0;
+    const uint32_t d = head + excl;  // my first byte in the exponent array
+    if (direct) {
+      // one pass straight to the exponent array, then check the count
+      const uint32_t limit = ex_addr + ((d + (cnt ? cnt : 1u) - 1u) & ~3u);
+      uint32_t got;
+      if (tk.masked)
+        got = decode_direct<T, C, true>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
+                                        tk.num_luts, ex_addr, d, limit, bad);
+      else
+        got = decode_direct<T, C, false>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
+                                         tk.num_luts, ex_addr, d, limit, bad);
+      if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
+    } else if (cnt) {
+      // compact: slot bytes [0, cnt) -> ex_s[d, d+cnt).  Destination word k
+      // holds slot bytes 4k-s .. 4k-s+3 (s = d & 3): a funnel shift of slot
+      // words k-1 and k.  The first and last words are shared with the
+      // neighbours and merged with OR into the zeroed array.
+      const uint32_t e_end = d + cnt;
+      const uint32_t last = ((e_end - 1) >> 2) - (d >> 2);
       const uint32_t s8 = (d & 3u) * 8u, r = e_end & 3u;
       const uint32_t mlast = r ? 0xFFFFFFFFu >> (32u - 8u * r) : 0xFFFFFFFFu;
       const uint32_t sl = smem_addr(slots + tid);
-      uint32_t *ex32 = reinterpret_cast<uint32_t *>(ex_s) + q0;
+      const uint32_t dst = ex_addr + (d & ~3u);
       uint32_t prev = lds32(sl);
-      const uint32_t v = prev << s8;
       if (last == 0) {
-        atomicOr(ex32, v & mlast);
+        red_or32(dst, (prev << s8) & mlast);
       } else {
-        atomicOr(ex32, v);
+        red_or32(dst, prev << s8);
         for (uint32_t j = 1; j < last; ++j) {  // slot word j <= cnt/4: inside the slot
           const uint32_t cur = lds32(sl + j * (4u * T));
-          sts32(smem_addr(ex32 + j), __funnelshift_l(prev, cur, s8));
+          sts32(dst + 4u * j, __funnelshift_l(prev, cur, s8));
           prev = cur;
         }
         const uint32_t cur = lds32(sl + last * (4u * T));
-        atomicOr(ex32 + last, __funnelshift_l(prev, cur, s8) & mlast);
+        red_or32(dst + 4u * last, __funnelshift_l(prev, cur, s8) & mlast);
       }
     }
-    __syncthreads();
+    if (__syncthreads_or(bad)) {
+      if (bad) report(kb.err, bad);
+      // leave the exponent array zeroed for the next block
+      for (uint32_t i = tid; i < (span + 15u) >> 4; i += T)
+        reinterpret_cast<uint4 *>(ex_s)[i] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
 
     // output: fuse and store, 16 elements per thread per step; the ragged
     // first and last groups one element per lane
@@ -570,11 +648,10 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
         if (mine) ex_s[i] = 0;
       }
     }
-    // No barrier here: the next block's decode writes only private slots
-    // (last read before the barrier above), its compaction writes the
-    // exponent array only after its scan barrier, which every thread reaches
-    // after finishing this output, and the stage slot refilled next was
-    // last read before this block's scan barrier.
+    // No barrier here: the next block's decode writes only private slots or,
+    // for direct decoding, the exponent array after the next scan barrier,
+    // which every thread reaches after finishing this output; the stage slot
+    // refilled next was last read before this block's scan barrier.
   }
 }
 
@@ -593,11 +670,15 @@ uint32_t stage_bytes_for(uint32_t max_block_elems) {
 
 uint32_t slot_words_for(uint32_t max_chunk_elems) { return (max_chunk_elems + 3u) / 4u + 1u; }
 
+// Must match the device layout: Layout<T, C>::slot_bytes per stage slot.
+size_t stage_slot_bytes(uint32_t C, uint32_t T) {
+  return (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16 + T;
+}
+
 size_t shared_bytes(uint32_t C, uint32_t T, uint32_t stage, uint32_t slot_words,
                     uint32_t sub_words) {
-  const size_t slot = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16;
-  return (size_t)kOffStages + 2 * slot + stage + (size_t)slot_words * T * 4 +
-         (size_t)sub_words * 4;
+  return (size_t)kOffStages + 2 * stage_slot_bytes(C, T) + stage +
+         (size_t)slot_words * T * 4 + (size_t)sub_words * 4;
 }
 
 bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -610,6 +691,7 @@ df11_status validate(const df11_tensor &t) {
       !t.sign_mantissa || !t.out_bf16)
     return DF11_ERR_NULL;
   if (!aligned(t.bitstream, 16) || !aligned(t.gaps, 16) || !aligned(t.luts, 16) ||
+      !aligned(t.chunk_counts, 16) ||
       !aligned(t.sign_mantissa, 16) || !aligned(t.out_bf16, 16) || !aligned(t.block_out_pos, 4))
     return DF11_ERR_ALIGN;
   if (!supported(p.chunk_bytes, p.threads_per_block)) return DF11_ERR_UNSUPPORTED;
@@ -620,6 +702,7 @@ df11_status validate(const df11_tensor &t) {
   if (p.max_block_elems == 0 || p.max_block_elems > 8ull * p.chunk_bytes * p.threads_per_block)
     return DF11_ERR_FORMAT;
   if (p.max_chunk_elems == 0 || p.max_chunk_elems > 8ull * p.chunk_bytes) return DF11_ERR_FORMAT;
+  if (t.chunk_counts && 8ull * p.chunk_bytes > 255) return DF11_ERR_FORMAT;
   if (p.max_len < 1 || p.max_len > 32) return DF11_ERR_FORMAT;
   return DF11_OK;
 }
@@ -643,6 +726,7 @@ DeviceInfo &device_info(int dev) {
 template <int T, int C>
 df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t s,
                    int instance) {
+  if (stage_slot_bytes(C, T) != Layout<T, C>::slot_bytes) return DF11_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
   DeviceInfo &di = device_info(dev);
@@ -685,6 +769,7 @@ df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     KTensor &k = kb.t[kb.count];
     k.bitstream = ts[i].bitstream;
     k.gaps = ts[i].gaps;
+    k.chunk_counts = ts[i].chunk_counts;
     k.block_out_pos = ts[i].block_out_pos;
     k.luts = ts[i].luts;
     k.code_lengths = ts[i].code_lengths;
@@ -700,14 +785,15 @@ df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     blocks[kb.count] = p.num_blocks;
     ++kb.count;
     max_elems = max_elems > p.max_block_elems ? max_elems : p.max_block_elems;
-    max_chunk = max_chunk > p.max_chunk_elems ? max_chunk : p.max_chunk_elems;
+    if (!ts[i].chunk_counts)  // only decoding without counts needs private slots
+      max_chunk = max_chunk > p.max_chunk_elems ? max_chunk : p.max_chunk_elems;
     max_luts = max_luts > p.num_luts ? max_luts : p.num_luts;
     C = p.chunk_bytes;
     T = p.threads_per_block;
   }
   if (kb.count == 0) return DF11_OK;
   kb.stage_bytes = stage_bytes_for(max_elems);
-  kb.slot_words = slot_words_for(max_chunk);
+  kb.slot_words = max_chunk ? slot_words_for(max_chunk) : 0u;
   kb.sub_words = (max_luts - 1) <= (uint32_t)kSubTablesInSmem ? (max_luts - 1) * 256 : 0;
   size_t smem = shared_bytes(C, T, kb.stage_bytes, kb.slot_words, kb.sub_words);
   if (smem > 227 * 1024 && kb.sub_words) {  // drop the deeper tables to global memory
@@ -735,7 +821,8 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
   if (!params) return DF11_ERR_NULL;
   if (params->n != n) return DF11_ERR_INVALID;
   if (d_err && !aligned(d_err, 4)) return DF11_ERR_ALIGN;
-  df11_tensor t{bitstream, gaps, block_out_pos, luts, code_lengths, sign_mantissa, out_bf16, *params};
+  df11_tensor t{bitstream, gaps, nullptr, block_out_pos, luts, code_lengths, sign_mantissa,
+                out_bf16, *params};
   df11_status st = validate(t);
   if (st != DF11_OK || n == 0) return st;
   return launch_batch(&t, 1, d_err, (cudaStream_t)stream);

@@ -28,6 +28,11 @@
  *                  num_blocks*T*5/8 + 16 bytes.
  *   block_out_pos  num_blocks+1 uint32: index of the first element whose
  *                  codeword starts in each block; the last entry is n.
+ *   chunk_counts   per chunk, the number of codewords that start in it
+ *                  (uint8; num_blocks*T + 16 bytes).  Derived metadata the
+ *                  pages do not have: with it a decoding thread knows where
+ *                  its output goes before it decodes; without it (NULL) the
+ *                  thread counts by decoding first.
  *   luts           num_luts tables of 256 uint32, table 0 first:
  *                  table 0, indexed by the next 8 bits: up to three whole
  *                  codewords in those bits -- bits 0-23 their exponents
@@ -108,6 +113,7 @@ typedef struct df11_params {
 typedef struct df11_tensor {
   const uint8_t *bitstream;      /* 16-byte aligned */
   const uint8_t *gaps;           /* 16-byte aligned */
+  const uint8_t *chunk_counts;   /* 16-byte aligned, or NULL */
   const uint32_t *block_out_pos; /* 4-byte aligned */
   const uint32_t *luts;          /* 16-byte aligned */
   const uint8_t *code_lengths;   /* any alignment */
@@ -118,8 +124,10 @@ typedef struct df11_tensor {
 
 /*
  * Decode one tensor into out_bf16 (bit-identical to the BF16 tensor that was
- * encoded).  All pointers are device pointers owned by the caller and laid
- * out as described at the top of this file; `params` is a host pointer.
+ * encoded), from the format the pages describe (no chunk counts: every
+ * thread counts its codewords by decoding, then places them after the scan).
+ * All pointers are device pointers owned by the caller and laid out as
+ * described at the top of this file; `params` is a host pointer.
  * n must equal params->n.  d_err is a device int32 (may be NULL) that the
  * caller zeroes; the kernel writes a DF11_DEV_ERR_* code into it when the
  * data are inconsistent.  Returns DF11_OK once the work is queued on
@@ -135,8 +143,9 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
 /*
  * Decode `count` tensors (a layer's weights, say) with one kernel launch per
  * DF11_MAX_BATCH tensors.  `tensors` is a host array; every tensor must use
- * the same chunk_bytes and threads_per_block.  Same conventions as
- * df11_decode.
+ * the same chunk_bytes and threads_per_block.  A tensor whose chunk_counts is
+ * not NULL is decoded in one pass straight to its output places; the others
+ * as in df11_decode.  Same conventions as df11_decode.
  */
 df11_status df11_decode_batched(const df11_tensor *tensors, int count,
                                 int32_t *d_err, df11_stream_t stream);
@@ -165,11 +174,13 @@ typedef struct df11_host_tensor {
   uint32_t *luts;             /* num_luts * 256 */
   uint8_t *sign_mantissa;
   uint64_t sign_mantissa_bytes; /* n rounded up to 16 */
+  uint8_t *chunk_counts;
+  uint64_t chunk_counts_bytes;  /* num_blocks*T + 16 */
 } df11_host_tensor;
 
 /*
  * Encode n BF16 words (host memory) with chunk_bytes C (a multiple of 4,
- * 4..64) and threads_per_block T (a multiple of 128, 128..1024), using up
+ * 4..28) and threads_per_block T (a multiple of 128, 128..1024), using up
  * to num_threads host threads (<= 0: all cores).  The exponent code is the
  * Huffman code of the exponent histogram, limited to 32-bit codewords by
  * package-merge when needed, in canonical form; ties are broken by symbol

@@ -76,6 +76,8 @@ class _Format(ctypes.Structure):
         ("luts", ctypes.POINTER(ctypes.c_uint32)),
         ("sign_mantissa", ctypes.POINTER(ctypes.c_uint8)),
         ("sm_bytes", ctypes.c_uint64),
+        ("chunk_counts", ctypes.POINTER(ctypes.c_uint8)),
+        ("chunk_counts_bytes", ctypes.c_uint64),
     ]
 
 
@@ -147,6 +149,7 @@ class OracleFormat:
     block_out_pos: np.ndarray  # uint32[num_blocks + 1]
     luts: np.ndarray           # uint32[num_luts*256]
     sign_mantissa: np.ndarray  # uint8[roundup(n, 16)]
+    chunk_counts: np.ndarray   # uint8[num_blocks*T + 16]
 
 
 def split(w):
@@ -256,6 +259,7 @@ def encode(w, chunk_bytes: int = 8, threads_per_block: int = 256) -> OracleForma
             block_out_pos=_copy(f.block_out_pos, f.num_blocks + 1, np.uint32),
             luts=_copy(f.luts, f.num_luts * 256, np.uint32),
             sign_mantissa=_copy(f.sign_mantissa, f.sm_bytes, np.uint8),
+            chunk_counts=_copy(f.chunk_counts, f.chunk_counts_bytes, np.uint8),
         )
     finally:
         lib.oracle_format_free(ctypes.byref(f))

@@ -370,7 +370,7 @@ void oracle_pack_gaps(const uint8_t *gaps, uint64_t count, uint8_t *packed) {
 int oracle_encode(const uint16_t *w, uint64_t n, uint32_t chunk_bytes,
                   uint32_t threads_per_block, oracle_format *f) {
   memset(f, 0, sizeof(*f));
-  if (chunk_bytes < 4 || chunk_bytes % 4 != 0) return 1;
+  if (chunk_bytes < 4 || chunk_bytes > 28 || chunk_bytes % 4 != 0) return 1;
   if (threads_per_block == 0 || threads_per_block % 128 != 0) return 1;
   if (n >= (1ull << 32)) return 1;
   f->n = n;
@@ -417,11 +417,15 @@ int oracle_encode(const uint16_t *w, uint64_t n, uint32_t chunk_bytes,
 
   /* codewords starting in each chunk, counted one start at a time */
   f->max_chunk_elems = 0;
+  f->chunk_counts_bytes = chunks + 16;
+  f->chunk_counts = (uint8_t *)calloc(f->chunk_counts_bytes, 1);
   if (chunks) {
     uint32_t *per_chunk = (uint32_t *)calloc(chunks, 4);
     for (uint64_t i = 0; i < n; i++) per_chunk[starts[i] / (8ull * chunk_bytes)]++;
-    for (uint64_t c = 0; c < chunks; c++)
+    for (uint64_t c = 0; c < chunks; c++) {
       if (per_chunk[c] > f->max_chunk_elems) f->max_chunk_elems = per_chunk[c];
+      f->chunk_counts[c] = (uint8_t)per_chunk[c];
+    }
     free(per_chunk);
   }
 
@@ -448,6 +452,7 @@ void oracle_format_free(oracle_format *f) {
   free(f->block_out_pos);
   free(f->luts);
   free(f->sign_mantissa);
+  free(f->chunk_counts);
   memset(f, 0, sizeof(*f));
 }
 

@@ -61,6 +61,8 @@ typedef struct oracle_format {
   uint32_t *luts;             /* num_luts * 256 entries */
   uint8_t *sign_mantissa;     /* n bytes, buffer padded to a multiple of 16 */
   uint64_t sm_bytes;
+  uint8_t *chunk_counts;      /* codewords starting in each chunk; chunks+16 */
+  uint64_t chunk_counts_bytes;
 } oracle_format;
 
 /* Field split of one BF16 word. */

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layouts_match_header():
     assert ctypes.sizeof(df11.Params) == 48
-    assert ctypes.sizeof(df11.TensorDesc) == 7 * 8 + 48
+    assert ctypes.sizeof(df11.TensorDesc) == 8 * 8 + 48
 
 
 def _params(**kw):
@@ -85,8 +85,8 @@ def test_batched_host_validation():
     assert L.df11_decode_batched(None, 0, None, None) == 0
     assert L.df11_decode_batched(None, -1, None, None) == 7
     assert L.df11_decode_batched(None, 1, None, None) == 1
-    a = df11.TensorDesc(*[FAKE] * 7, _params())
-    b = df11.TensorDesc(*[FAKE] * 7, _params(chunk_bytes=4, total_bits=2600,
+    a = df11.TensorDesc(*[FAKE] * 8, _params())
+    b = df11.TensorDesc(*[FAKE] * 8, _params(chunk_bytes=4, total_bits=2600,
                                                 num_blocks=1, max_chunk_elems=30))
     arr = (df11.TensorDesc * 2)(a, b)
     assert L.df11_decode_batched(arr, 2, None, None) == 7  # mixed (C, T)

@@ -28,6 +28,7 @@ def _compare(w, C, T, threads=4):
     assert np.array_equal(h.block_out_pos, f.block_out_pos)
     assert np.array_equal(h.luts, f.luts)
     assert np.array_equal(h.sign_mantissa, f.sign_mantissa)
+    assert np.array_equal(h.chunk_counts, f.chunk_counts)
     return h
 
 
@@ -82,6 +83,6 @@ def test_oracle_decodes_builder_stream():
 
 def test_builder_rejects_bad_parameters():
     w = np.zeros(10, np.uint16)
-    for C, T in [(3, 256), (6, 256), (8, 100), (8, 2048), (0, 256), (68, 256)]:
+    for C, T in [(3, 256), (6, 256), (8, 100), (8, 2048), (0, 256), (32, 256), (68, 256)]:
         with pytest.raises(df11.Df11Error):
             df11.compress(w, C, T)

@@ -25,18 +25,21 @@ def _cuda():
     torch.cuda.init()
 
 
-def _decode(h, stream=None):
+def _decode(h, stream=None, counts=True):
     d = df11.to_device(h, "cuda")
     err = df11.new_error_word()
-    out = df11.decode(d, err=err, stream=stream)
+    out = df11.decode(d, err=err, stream=stream, counts=counts)
     torch.cuda.synchronize()
     df11.check_device_error(err)
     return out
 
 
-def _gpu_vs_oracle_full(w_np, C=8, T=256):
+COUNTS = pytest.mark.parametrize("counts", [True, False], ids=["counts", "no_counts"])
+
+
+def _gpu_vs_oracle_full(w_np, C=8, T=256, counts=True):
     h = df11.compress(w_np, C, T)
-    out = _decode(h).view(torch.int16).cpu().numpy().view(np.uint16)
+    out = _decode(h, counts=counts).view(torch.int16).cpu().numpy().view(np.uint16)
     ref, end, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, h.n)
     assert end == h.params.total_bits
     assert np.array_equal(out, ref)       # GPU == oracle, element by element
@@ -46,51 +49,69 @@ def _gpu_vs_oracle_full(w_np, C=8, T=256):
 
 # --- oracle-sized cases, compared in full ---------------------------------
 
+@COUNTS
 @pytest.mark.parametrize("C,T", [(8, 256), (4, 256), (16, 256), (8, 128), (8, 512)])
-def test_single_matrix_all_kernel_shapes(C, T):
+def test_single_matrix_all_kernel_shapes(C, T, counts):
     w = workloads.as_numpy_u16(workloads.single_matrix(0))
-    _gpu_vs_oracle_full(w, C, T)
+    _gpu_vs_oracle_full(w, C, T, counts)
 
 
+@COUNTS
 @pytest.mark.parametrize("n", [1, 2, 7, 31, 32, 33, 255, 256, 257, 4095, 6399,
                                6400, 6401, 65537, 1_000_003])
-def test_ragged_sizes(n):
+def test_ragged_sizes(n, counts):
     w = workloads.as_numpy_u16(workloads.gaussian_bf16(n, 0.02, 100 + n))
-    _gpu_vs_oracle_full(w)
+    _gpu_vs_oracle_full(w, counts=counts)
 
 
-def test_every_bf16_pattern():
+@COUNTS
+def test_every_bf16_pattern(counts):
     w = workloads.as_numpy_u16(workloads.all_bf16_patterns())
-    _gpu_vs_oracle_full(w)
+    _gpu_vs_oracle_full(w, counts=counts)
     # shuffled, so that every block holds many exponents
     rng = np.random.default_rng(0)
-    _gpu_vs_oracle_full(rng.permutation(w))
+    _gpu_vs_oracle_full(rng.permutation(w), counts=counts)
 
 
-def test_single_symbol_streams():
-    _gpu_vs_oracle_full(np.zeros(300_001, np.uint16))           # +0.0 only
-    _gpu_vs_oracle_full(np.full(300_001, 0x8000, np.uint16))    # -0.0 only
+@COUNTS
+def test_single_symbol_streams(counts):
+    _gpu_vs_oracle_full(np.zeros(300_001, np.uint16), counts=counts)         # +0.0 only
+    _gpu_vs_oracle_full(np.full(300_001, 0x8000, np.uint16), counts=counts)  # -0.0 only
     # one exponent, random sign/mantissa: a 1-bit code, 16384 per block
     rng = np.random.default_rng(1)
     sm = rng.integers(0, 256, 500_000)
     w = (((sm & 0x80) << 8) | (120 << 7) | (sm & 0x7F)).astype(np.uint16)
-    h = _gpu_vs_oracle_full(w)
+    h = _gpu_vs_oracle_full(w, counts=counts)
     assert h.params.max_block_elems == 8 * 8 * 256
 
 
-def test_adversarial_mix_multilevel_tables():
+@COUNTS
+def test_adversarial_mix_multilevel_tables(counts):
     w = workloads.as_numpy_u16(workloads.adversarial_mix(1 << 22, 4))
-    h = _gpu_vs_oracle_full(w)
+    h = _gpu_vs_oracle_full(w, counts=counts)
     assert h.params.num_luts > 1
 
 
-def test_fibonacci_32_bit_codewords():
+@COUNTS
+def test_fibonacci_32_bit_codewords(counts):
     w = workloads.as_numpy_u16(workloads.fibonacci_exponents(0))
-    h = _gpu_vs_oracle_full(w)
+    h = _gpu_vs_oracle_full(w, counts=counts)
     assert h.params.max_len == 32
 
 
-def test_many_deep_tables_read_from_global_memory():
+@COUNTS
+def test_few_codewords_no_masking(counts):
+    # longest codeword <= 10 bits: the kernel checks region ends per lookup
+    rng = np.random.default_rng(11)
+    e = rng.choice(np.arange(120, 126), size=400_003, p=[.4, .25, .15, .1, .06, .04])
+    sm = rng.integers(0, 256, e.size)
+    w = (((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)).astype(np.uint16)
+    h = _gpu_vs_oracle_full(w, counts=counts)
+    assert h.params.max_len <= 10
+
+
+@COUNTS
+def test_many_deep_tables_read_from_global_memory(counts):
     # near-uniform exponents over a wide range with a heavy head: many
     # sub-tables, more than the kernel keeps in shared memory
     rng = np.random.default_rng(7)
@@ -99,17 +120,18 @@ def test_many_deep_tables_read_from_global_memory():
     rng.shuffle(e)
     sm = rng.integers(0, 256, e.size)
     w = (((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)).astype(np.uint16)
-    h = _gpu_vs_oracle_full(w)
+    h = _gpu_vs_oracle_full(w, counts=counts)
     assert h.params.num_luts > 9
 
 
-def test_block_scaled_batched_against_oracle():
+@COUNTS
+def test_block_scaled_batched_against_oracle(counts):
     ts = workloads.block_tensors(5, scale=8)
     hs = [df11.compress(workloads.as_numpy_u16(t.bits)) for t in ts]
     ds = [df11.to_device(h) for h in hs]
     outs = [df11.empty_output(d) for d in ds]
     err = df11.new_error_word()
-    df11.decode_batched(ds, outs, err=err)
+    df11.decode_batched(ds, outs, err=err, counts=counts)
     torch.cuda.synchronize()
     df11.check_device_error(err)
     for t, h, o in zip(ts, hs, outs):
@@ -124,6 +146,9 @@ def test_batched_more_than_one_launch_and_empty_tensors():
           [0, 5000, 1, 70000, 0, 123457] + [20000 + 37 * i for i in range(15)]]
     hs = [df11.compress(w) for w in ws]
     ds = [df11.to_device(h) for h in hs]
+    for i, d in enumerate(ds):  # mix: every third tensor without its counts
+        if i % 3 == 2:
+            d.chunk_counts = None
     outs = [df11.empty_output(d) for d in ds]
     err = df11.new_error_word()
     df11.decode_batched(ds, outs, err=err)
@@ -163,11 +188,11 @@ def _sampled_blocks_vs_oracle(h, out_cpu_u16, samples=12):
         assert np.array_equal(out_cpu_u16[lo:hi], ref), b
 
 
-def _full_size(bits_dev: torch.Tensor):
+def _full_size(bits_dev: torch.Tensor, counts=True):
     h = df11.compress(bits_dev)
     d = df11.to_device(h)
     err = df11.new_error_word()
-    out = df11.decode(d, err=err)
+    out = df11.decode(d, err=err, counts=counts)
     torch.cuda.synchronize()
     df11.check_device_error(err)
     assert torch.equal(out.view(torch.int16), bits_dev)   # round trip, on device
@@ -194,46 +219,66 @@ def test_full_adversarial_64m():
     assert h.params.num_luts >= 4
 
 
-def test_full_embedding_622m():
-    _full_size(workloads.embedding(0, device="cuda"))
+@COUNTS
+def test_full_embedding_622m(counts):
+    _full_size(workloads.embedding(0, device="cuda"), counts)
 
 
 # --- corrupted inputs: flagged, never a fault ------------------------------
 
-def _decode_with_err(d):
+def _decode_with_err(d, counts=True):
     err = df11.new_error_word()
-    out = df11.decode(d, err=err)
+    out = df11.decode(d, err=err, counts=counts)
     torch.cuda.synchronize()
     return out, int(err.item())
 
 
-def test_corrupt_block_positions_are_flagged():
+@COUNTS
+def test_corrupt_block_positions_are_flagged(counts):
     w = workloads.single_matrix(1)
     h = df11.compress(w)
     d = df11.to_device(h)
     d.block_out_pos[1] += 1
-    _, code = _decode_with_err(d)
+    _, code = _decode_with_err(d, counts)
     assert code in (1, 5)  # COUNT or CAPACITY
     d = df11.to_device(h)
     d.block_out_pos[-1] += 1000  # past n
-    _, code = _decode_with_err(d)
+    _, code = _decode_with_err(d, counts)
     assert code == 5
 
 
-def test_corrupt_tables_are_flagged():
+@COUNTS
+def test_corrupt_tables_are_flagged(counts):
     w = workloads.adversarial_mix(1 << 20, 2)
     h = df11.compress(w)
     d = df11.to_device(h)
     d.luts[: 256].zero_()      # every level-0 entry invalid
-    _, code = _decode_with_err(d)
+    _, code = _decode_with_err(d, counts)
     assert code == 3
     d = df11.to_device(h)
     d.code_lengths.zero_()     # no codeword can be consumed on the slow path
-    _, code = _decode_with_err(d)
+    _, code = _decode_with_err(d, counts)
     assert code in (1, 2, 3)
 
 
-def test_corrupt_bitstream_never_faults():
+def test_corrupt_chunk_counts_are_flagged():
+    w = workloads.single_matrix(4)
+    h = df11.compress(w)
+    d = df11.to_device(h)
+    d.chunk_counts[10] += 1
+    d.chunk_counts[11] -= 1      # block total unchanged: caught per thread
+    out, code = _decode_with_err(d)
+    assert code == 1
+    d = df11.to_device(h)
+    d.chunk_counts[300] += 3     # block total changed: caught by the scan
+    _, code = _decode_with_err(d)
+    assert code == 1
+    out = _decode(h)             # the context is still healthy
+    assert torch.equal(out.view(torch.int16).cpu(), w)
+
+
+@COUNTS
+def test_corrupt_bitstream_never_faults(counts):
     w = workloads.single_matrix(2)
     h = df11.compress(w)
     rng = np.random.default_rng(3)
@@ -244,7 +289,7 @@ def test_corrupt_bitstream_never_faults():
                                             device="cuda")
         # Huffman streams carry no checksum: a flip is flagged or decodes to
         # other values; either way the call completes inside its buffers
-        _, code = _decode_with_err(d)
+        _, code = _decode_with_err(d, counts)
         assert code in (0, 1, 2, 3)
     out = _decode(h)
     assert torch.equal(out.view(torch.int16).cpu(), w)  # context still healthy

@@ -357,6 +357,8 @@ def test_gaps_and_block_positions_brute_force(C, T):
     for s in st:
         per_chunk[s // chunk_bits] += 1
     assert f.max_chunk_elems == max(per_chunk)
+    assert f.chunk_counts[: len(per_chunk)].tolist() == per_chunk
+    assert not f.chunk_counts[len(per_chunk):].any()
     # packed gaps: 5-bit fields, MSB first
     bits = np.unpackbits(f.gaps_packed)
     for c in range(f.num_blocks * T):
