@@ -87,14 +87,14 @@ def block_groups(config: str, names):
     return groups
 
 
-def algorithmic_bytes(h) -> int:
+def algorithmic_bytes(h, counts: bool = True) -> int:
     """Bytes one decode of this tensor must move: compressed input (stream,
-    sign/mantissa, gaps, block positions, tables, code lengths) + 2 B/elem
-    of BF16 output."""
+    sign/mantissa, gaps, chunk counts when used, block positions, tables,
+    code lengths) + 2 B/elem of BF16 output."""
     p = h.params
     chunks = p.num_blocks * p.threads_per_block
     return ((p.total_bits + 7) // 8 + p.n + (5 * chunks + 7) // 8 + 4 * (p.num_blocks + 1)
-            + 1024 * p.num_luts + 256 + 2 * p.n)
+            + (chunks if counts else 0) + 1024 * p.num_luts + 256 + 2 * p.n)
 
 
 def kernel_hash() -> str:
@@ -262,17 +262,21 @@ def run_b200(args, world, rank, local):
     err = df11.new_error_word(device)
     stream = torch.cuda.current_stream()
 
+    counts = not args.no_counts
+
     def step(events=None):
         for gi, g in enumerate(groups):
             if events is not None:
                 events[gi][0].record(stream)
-            df11.decode_batched([devs[i] for i in g], outs_for[gi], err=err, stream=stream)
+            df11.decode_batched([devs[i] for i in g], outs_for[gi], err=err, stream=stream,
+                                counts=counts)
             if events is not None:
                 events[gi][1].record(stream)
 
     # parity: every group's output equals the original, bit for bit
     for gi, g in enumerate(groups):
-        df11.decode_batched([devs[i] for i in g], outs_for[gi], err=err, stream=stream)
+        df11.decode_batched([devs[i] for i in g], outs_for[gi], err=err, stream=stream,
+                            counts=not args.no_counts)
         torch.cuda.synchronize()
         for i, o in zip(g, outs_for[gi]):
             ref = units[i][1](device)
@@ -313,7 +317,7 @@ def run_b200(args, world, rank, local):
     # dominant kernel: per-launch durations from events on the launch stream
     per_group_ms = [statistics.mean(ev[s][gi][0].elapsed_time(ev[s][gi][1])
                                     for s in range(args.steps)) for gi in range(len(groups))]
-    alg = [sum(algorithmic_bytes(hosts[i]) for i in g) for g in groups]
+    alg = [sum(algorithmic_bytes(hosts[i], counts) for i in g) for g in groups]
     achieved = sum(alg) / (sum(per_group_ms) * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     traffic = recorded_traffic(args.config)
@@ -345,6 +349,7 @@ def run_b200(args, world, rank, local):
                       "inputs smaller than L2: numbers include L2 reuse",
                 "parallelism": f"replicas x{world} (no collective)",
                 "parity": "bit-exact vs original on every tensor before timing",
+                "chunk_counts": not args.no_counts,
             },
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s",
@@ -381,7 +386,7 @@ def measure_e2e(args, units, hosts, groups, device, world):
     for i, h in hosts.items():
         pinned[i] = {k: torch.from_numpy(getattr(h, k).view(np.uint8)).pin_memory()
                      for k in ("bitstream", "gaps", "block_out_pos", "luts",
-                               "code_lengths", "sign_mantissa")}
+                               "code_lengths", "sign_mantissa", "chunk_counts")}
         staged[i] = df11.to_device(h, device)
         out_dev[i] = df11.empty_output(staged[i])
         out_host[i] = torch.empty(h.n, dtype=torch.bfloat16).pin_memory()
@@ -397,7 +402,7 @@ def measure_e2e(args, units, hosts, groups, device, world):
                     dst = getattr(staged[i], k)
                     dst.view(torch.uint8).copy_(t, non_blocking=True)
             df11.decode_batched([staged[i] for i in g], [out_dev[i] for i in g],
-                                err=err, stream=stream)
+                                err=err, stream=stream, counts=not args.no_counts)
             for i in g:
                 out_host[i].copy_(out_dev[i], non_blocking=True)
 
@@ -513,6 +518,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-counts", action="store_true",
+                    help="decode without the format's chunk counts (count by decoding)")
     ap.add_argument("--no-clock-window", action="store_true",
                     help="skip the busy untimed loop before the timed region "
                          "(for profiler runs)")
