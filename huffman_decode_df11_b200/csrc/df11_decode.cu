@@ -656,6 +656,259 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
 }
 
 // ---------------------------------------------------------------------------
+// Warp-specialised decode for tensors that carry chunk counts.
+//
+// With the counts in shared memory every warp can work out where its output
+// goes on its own, so the thread block needs no block-wide barrier per format
+// block.  One producer warp (one lane) keeps kWsStages stage slots filled,
+// each guarded by a "full" mbarrier (completed by the bulk copies) and an
+// "empty" mbarrier (one arrival per consumer warp once it holds the slot's
+// data in registers).  Each of the T/32 consumer warps, per format block:
+//   - sums the block's chunk counts before its own chunks and over the whole
+//     block (two warp reductions over T bytes) and scans its lanes' counts;
+//   - releases the slot;
+//   - decodes straight into its private exponent region (zeroed; words shared
+//     by two lanes merged with OR) and checks every count;
+//   - writes its own output range: whole 16-element groups with 16-byte
+//     stores, the two ragged edge groups one element per lane.
+constexpr int kWsStages = 4;
+
+template <int T, int C>
+struct WsLayout {
+  static constexpr uint32_t bits_bytes = T * C + 16;
+  static constexpr uint32_t gaps_bytes = T * 5 / 8 + 16;
+  static constexpr uint32_t counts_bytes = T;
+  static constexpr uint32_t meta_bytes = 16;
+  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes + counts_bytes + meta_bytes;
+  static_assert(slot_bytes % 16 == 0, "alignment");
+};
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+template <int T, int C>
+__device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t *slot,
+                                         uint32_t full, uint32_t region_bytes) {
+  using L = WsLayout<T, C>;
+  const uint32_t P0 = tk.block_out_pos[b], P1 = tk.block_out_pos[b + 1];
+  const uint32_t expected = P1 - P0;
+  // a warp's exponents fit its region whatever the block: every chunk count
+  // is checked against max_chunk_elems before decoding
+  const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems;
+  *reinterpret_cast<uint4 *>(slot + L::bits_bytes + L::gaps_bytes + L::counts_bytes) =
+      make_uint4(P0, P1, ok ? 1u : 0u, b);
+  if (!ok) {
+    mbar_arrive_expect_tx(full, 0);
+    return;
+  }
+  mbar_arrive_expect_tx(full, L::bits_bytes + L::gaps_bytes + L::counts_bytes);
+  bulk_g2s(smem_addr(slot), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, full);
+  bulk_g2s(smem_addr(slot + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
+           full);
+  bulk_g2s(smem_addr(slot + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
+           L::counts_bytes, full);
+  const uint32_t sm_begin = P0 & ~15u;
+  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
+  if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
+}
+
+// Sum of the byte counts a lane holds (T/32 of them).
+template <int T>
+__device__ __forceinline__ uint32_t lane_count_sum(const uint8_t *counts, int lane) {
+  if (T == 128) {
+    return __dp4a(*reinterpret_cast<const uint32_t *>(counts + 4 * lane), 0x01010101u, 0u);
+  } else if (T == 256) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(counts + 8 * lane);
+    return __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u, 0u));
+  } else {
+    const uint4 v = *reinterpret_cast<const uint4 *>(counts + 16 * lane);
+    return __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u,
+                  __dp4a(v.z, 0x01010101u, __dp4a(v.w, 0x01010101u, 0u))));
+  }
+}
+
+template <int T, int C>
+__global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
+    df11_decode_ws_kernel(const __grid_constant__ KBatch kb) {
+  using L = WsLayout<T, C>;
+  constexpr int NW = C / 4 + 1;
+  constexpr int CONSUMERS = T / 32;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);  // full[S], empty[S]
+  uint8_t *lens_s = smem + kOffLens;
+  uint32_t *lut0_s = reinterpret_cast<uint32_t *>(smem + kOffLut0);
+  uint2 *wide_s = reinterpret_cast<uint2 *>(smem + kOffWide);
+  uint8_t *stages = smem + kOffStages;
+  uint8_t *regions = stages + kWsStages * L::slot_bytes;
+  uint32_t *sub_s = reinterpret_cast<uint32_t *>(regions + CONSUMERS * kb.stage_bytes);
+
+  int ti = 0;
+  for (int i = 1; i < kb.count; ++i)
+    if (blockIdx.x >= kb.t[i].cta_begin) ti = i;
+  const KTensor &tk = kb.t[ti];
+  const uint32_t ctas = (ti + 1 < kb.count ? kb.t[ti + 1].cta_begin : kb.cta_end) - tk.cta_begin;
+  const uint32_t first = blockIdx.x - tk.cta_begin;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (first >= tk.num_blocks) return;
+
+  if (tid == 0) {
+    for (int i = 0; i < kWsStages; ++i) {
+      mbar_init(smem_addr(&bars[i]), 1);
+      mbar_init(smem_addr(&bars[kWsStages + i]), CONSUMERS);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // tables, as in the other kernel
+  for (int i = tid; i < 256; i += T + 32) {
+    uint32_t e = tk.luts[i] & 0x3FFFFFFFu;
+    if ((e >> 24) & 15u) e = (e & 0xFF000000u) | rot8x3(e);
+    lut0_s[i] = e;
+    lens_s[((uint32_t)i >> 1) | (((uint32_t)i & 1u) << 7)] = tk.code_lengths[i];
+  }
+  const uint32_t *sub = tk.luts + 256;
+  const uint32_t sub_words = (tk.num_luts - 1) * 256;
+  if (sub_words && sub_words <= kb.sub_words) {
+    for (uint32_t i = tid; i < sub_words; i += T + 32) sub_s[i] = sub[i];
+    sub = sub_s;
+  }
+  for (uint32_t i = tid; i < CONSUMERS * kb.stage_bytes / 16; i += T + 32)
+    reinterpret_cast<uint4 *>(regions)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  build_wide<T + 32>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
+  __syncthreads();
+
+  if (warp == CONSUMERS) {  // producer
+    if (lane == 0) {
+      uint32_t k = 0;
+      for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
+        const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
+        if (!mbar_wait(smem_addr(&bars[kWsStages + s]), par ^ 1u)) {
+          report(kb.err, DF11_DEV_ERR_TIMEOUT);
+          break;
+        }
+        ws_issue<T, C>(tk, b, stages + s * L::slot_bytes, smem_addr(&bars[s]), kb.stage_bytes);
+      }
+    }
+    return;
+  }
+
+  const uint32_t region = smem_addr(regions + warp * kb.stage_bytes);
+  uint8_t *region_p = regions + warp * kb.stage_bytes;
+  const uint32_t wide = smem_addr(wide_s);
+  uint32_t k = 0;
+  for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
+    const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
+    const uint8_t *slot = stages + s * L::slot_bytes;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_addr(&bars[s]), par))) {
+      if (lane == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
+      return;  // whole warp
+    }
+    const uint4 m = *reinterpret_cast<const uint4 *>(slot + L::bits_bytes + L::gaps_bytes +
+                                                     L::counts_bytes);
+    const uint32_t P0 = m.x, P1 = m.y, expected = P1 - P0;
+    const uint8_t *counts = slot + L::bits_bytes + L::gaps_bytes;
+    // everything this warp needs from the slot, into registers
+    const uint32_t lsum = lane_count_sum<T>(counts, lane);
+    const uint32_t cnt = counts[tid];
+    const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
+    int start, end;
+    {
+      const uint32_t bit = 5u * (uint32_t)tid;
+      const uint32_t *g32 = reinterpret_cast<const uint32_t *>(slot + L::bits_bytes) + (bit >> 5);
+      const uint32_t v = __funnelshift_l(__byte_perm(g32[1], 0, 0x0123),
+                                         __byte_perm(g32[0], 0, 0x0123), bit);
+      start = (int)(v >> 27);
+      end = C * 8 + (int)((v >> 22) & 31u);
+    }
+    uint32_t w[NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j)
+      w[j] = __byte_perm(*reinterpret_cast<const uint32_t *>(slot + tid * C + 4 * j), 0, 0x0123);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&bars[kWsStages + s]));  // slot free for refill
+
+    const uint32_t before = __reduce_add_sync(0xFFFFFFFFu,
+                                              lane < warp * 32 / (T / 32) ? lsum : 0u);
+    const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, lsum);
+    if (!m.z || total != expected ||
+        __any_sync(0xFFFFFFFFu, cnt > tk.max_chunk_elems)) {
+      if (warp == 0 && lane == 0) report(kb.err, m.z ? (total != expected ? DF11_DEV_ERR_COUNT
+                                                                          : DF11_DEV_ERR_CAPACITY)
+                                                     : DF11_DEV_ERR_CAPACITY);
+      continue;
+    }
+    if (chunk_bit >= tk.total_bits) {
+      start = end = 0;
+    } else if ((uint64_t)end > tk.total_bits - chunk_bit) {
+      end = (int)(tk.total_bits - chunk_bit);
+    }
+    if (tk.masked) {
+#pragma unroll
+      for (int j = 0; j < NW; ++j)
+        w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
+    }
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int dd = 1; dd < 32; dd <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, dd);
+      if (lane >= dd) incl += v;
+    }
+    const uint32_t warp_total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    const uint32_t G0 = P0 + before;            // first element of this warp
+    const uint32_t head = G0 & 15u, span = head + warp_total;
+    const uint32_t d = head + incl - cnt;       // my first byte in the region
+    const uint32_t limit = region + ((d + (cnt ? cnt : 1u) - 1u) & ~3u);
+    int bad = 0;
+    uint32_t got;
+    if (tk.masked)
+      got = decode_direct<T, C, true>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts,
+                                      region, d, limit, bad);
+    else
+      got = decode_direct<T, C, false>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts,
+                                       region, d, limit, bad);
+    if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
+    if (__any_sync(0xFFFFFFFFu, bad != 0)) {
+      if (bad) report(kb.err, bad);
+      __syncwarp();
+      for (uint32_t i = lane; i < (span + 15u) >> 4; i += 32)
+        reinterpret_cast<uint4 *>(region_p)[i] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+      continue;
+    }
+    __syncwarp();
+
+    // output of this warp's elements [G0, G0 + warp_total)
+    const uint32_t base = G0 & ~15u;
+    uint16_t *out = tk.out + base;
+    const uint8_t *smg = tk.sign_mantissa + base;
+    const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
+    for (uint32_t g = g_begin + lane; g < g_end; g += 32) {
+      const uint32_t i0 = g << 4;
+      const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(smg + i0));
+      uint4 *rp = reinterpret_cast<uint4 *>(region_p + i0);
+      const uint4 rv = *rp;
+      *rp = make_uint4(0, 0, 0, 0);
+      const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
+      const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+      uint4 *o = reinterpret_cast<uint4 *>(out + i0);
+      o[0] = make_uint4(a.x, a.y, c.x, c.y);
+      o[1] = make_uint4(e2.x, e2.y, f.x, f.y);
+    }
+    if (span) {  // lanes 0-15: first group, 16-31: last group
+      const uint32_t gl = (span - 1) >> 4;
+      const bool first_partial = head != 0 || span < 16;
+      const bool last_partial = (span & 15u) != 0 && gl != 0;
+      const uint32_t i = lane < 16 ? (uint32_t)lane : (gl << 4) + (uint32_t)(lane - 16);
+      const bool mine = lane < 16 ? first_partial : last_partial;
+      if (mine && i >= head && i < span) out[i] = fuse1(smg[i], region_p[i]);
+      if (mine) region_p[i] = 0;
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 
 bool supported(uint32_t C, uint32_t T) {
@@ -709,7 +962,7 @@ df11_status validate(const df11_tensor &t) {
 
 struct DeviceInfo {
   int sms = 0;
-  std::atomic<size_t> configured[5];
+  std::atomic<size_t> configured[10];
 };
 
 DeviceInfo &device_info(int dev) {
@@ -723,26 +976,8 @@ DeviceInfo &device_info(int dev) {
   return d;
 }
 
-template <int T, int C>
-df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t s,
-                   int instance) {
-  if (stage_slot_bytes(C, T) != Layout<T, C>::slot_bytes) return DF11_ERR_UNSUPPORTED;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
-  DeviceInfo &di = device_info(dev);
-  auto kern = df11_decode_kernel<T, C>;
-  if (smem > 48 * 1024 && di.configured[instance].load() < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return DF11_ERR_CUDA;
-    di.configured[instance].store(smem);
-  }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, smem) != cudaSuccess)
-    return DF11_ERR_CUDA;
-  if (per_sm < 1) return DF11_ERR_TOO_LARGE;
-  // thread blocks per tensor in proportion to its format blocks
-  const uint64_t budget = (uint64_t)di.sms * per_sm;
+// thread blocks per tensor in proportion to its format blocks
+uint32_t split_grid(KBatch &kb, const uint32_t *blocks, uint64_t budget) {
   uint64_t total = 0;
   for (int i = 0; i < kb.count; ++i) total += blocks[i];
   uint32_t begin = 0;
@@ -754,11 +989,67 @@ df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t
     begin += (uint32_t)c;
   }
   kb.cta_end = begin;
-  kern<<<begin, T, smem, s>>>(kb);
+  return begin;
+}
+
+template <typename K>
+df11_status prepare(K kern, int threads, size_t smem, int instance, uint64_t &budget) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
+  DeviceInfo &di = device_info(dev);
+  if (smem > 48 * 1024 && di.configured[instance].load() < smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return DF11_ERR_CUDA;
+    di.configured[instance].store(smem);
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess)
+    return DF11_ERR_CUDA;
+  if (per_sm < 1) return DF11_ERR_TOO_LARGE;
+  budget = (uint64_t)di.sms * per_sm;
+  return DF11_OK;
+}
+
+template <int T, int C>
+df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t s,
+                   int instance) {
+  if (stage_slot_bytes(C, T) != Layout<T, C>::slot_bytes) return DF11_ERR_UNSUPPORTED;
+  auto kern = df11_decode_kernel<T, C>;
+  uint64_t budget = 0;
+  df11_status st = prepare(kern, T, smem, instance, budget);
+  if (st != DF11_OK) return st;
+  const uint32_t grid = split_grid(kb, blocks, budget);
+  kern<<<grid, T, smem, s>>>(kb);
   return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
-df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaStream_t s) {
+template <int T, int C>
+df11_status launch_ws(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t s,
+                      int instance) {
+  auto kern = df11_decode_ws_kernel<T, C>;
+  uint64_t budget = 0;
+  df11_status st = prepare(kern, T + 32, smem, instance, budget);
+  if (st != DF11_OK) return st;
+  const uint32_t grid = split_grid(kb, blocks, budget);
+  kern<<<grid, T + 32, smem, s>>>(kb);
+  return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+// Per-warp exponent region of the warp-specialised kernel: the warp's head
+// (< 16), up to 32 chunks of max_chunk_elems exponents, a word of slack.
+uint32_t region_bytes_for(uint32_t max_chunk_elems) {
+  return (15u + 32u * max_chunk_elems + 4u + 15u) & ~15u;
+}
+
+size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t region, uint32_t sub_words) {
+  const size_t slot = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16 + T + 16;
+  return (size_t)kOffStages + kWsStages * slot + (size_t)(T / 32) * region +
+         (size_t)sub_words * 4;
+}
+
+df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaStream_t s,
+                         bool ws) {
   KBatch kb{};
   kb.err = d_err;
   uint32_t blocks[DF11_MAX_BATCH];
@@ -785,16 +1076,31 @@ df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     blocks[kb.count] = p.num_blocks;
     ++kb.count;
     max_elems = max_elems > p.max_block_elems ? max_elems : p.max_block_elems;
-    if (!ts[i].chunk_counts)  // only decoding without counts needs private slots
-      max_chunk = max_chunk > p.max_chunk_elems ? max_chunk : p.max_chunk_elems;
+    max_chunk = max_chunk > p.max_chunk_elems ? max_chunk : p.max_chunk_elems;
     max_luts = max_luts > p.num_luts ? max_luts : p.num_luts;
     C = p.chunk_bytes;
     T = p.threads_per_block;
   }
   if (kb.count == 0) return DF11_OK;
-  kb.stage_bytes = stage_bytes_for(max_elems);
-  kb.slot_words = max_chunk ? slot_words_for(max_chunk) : 0u;
   kb.sub_words = (max_luts - 1) <= (uint32_t)kSubTablesInSmem ? (max_luts - 1) * 256 : 0;
+  if (ws) {
+    kb.stage_bytes = region_bytes_for(max_chunk);  // bytes of each warp's region
+    kb.slot_words = 0;
+    size_t smem = ws_shared_bytes(C, T, kb.stage_bytes, kb.sub_words);
+    if (smem > 227 * 1024 && kb.sub_words) {
+      kb.sub_words = 0;
+      smem = ws_shared_bytes(C, T, kb.stage_bytes, 0);
+    }
+    if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
+    if (T == 256 && C == 8) return launch_ws<256, 8>(kb, blocks, smem, s, 5);
+    if (T == 256 && C == 4) return launch_ws<256, 4>(kb, blocks, smem, s, 6);
+    if (T == 256 && C == 16) return launch_ws<256, 16>(kb, blocks, smem, s, 7);
+    if (T == 128 && C == 8) return launch_ws<128, 8>(kb, blocks, smem, s, 8);
+    if (T == 512 && C == 8) return launch_ws<512, 8>(kb, blocks, smem, s, 9);
+    return DF11_ERR_UNSUPPORTED;
+  }
+  kb.stage_bytes = stage_bytes_for(max_elems);
+  kb.slot_words = slot_words_for(max_chunk);
   size_t smem = shared_bytes(C, T, kb.stage_bytes, kb.slot_words, kb.sub_words);
   if (smem > 227 * 1024 && kb.sub_words) {  // drop the deeper tables to global memory
     kb.sub_words = 0;
@@ -807,6 +1113,21 @@ df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   if (T == 128 && C == 8) return launch<128, 8>(kb, blocks, smem, s, 3);
   if (T == 512 && C == 8) return launch<512, 8>(kb, blocks, smem, s, 4);
   return DF11_ERR_UNSUPPORTED;
+}
+
+// Tensors with chunk counts go to the warp-specialised kernel, the others to
+// the count-by-decoding kernel (one launch each, same stream).
+df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaStream_t s) {
+  df11_tensor with[DF11_MAX_BATCH], without[DF11_MAX_BATCH];
+  int nw = 0, nwo = 0;
+  for (int i = 0; i < count; ++i) {
+    if (ts[i].chunk_counts) with[nw++] = ts[i];
+    else without[nwo++] = ts[i];
+  }
+  df11_status st = DF11_OK;
+  if (nwo) st = launch_group(without, nwo, d_err, s, false);
+  if (st == DF11_OK && nw) st = launch_group(with, nw, d_err, s, true);
+  return st;
 }
 
 }  // namespace
