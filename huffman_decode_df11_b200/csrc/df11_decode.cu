@@ -91,7 +91,7 @@ struct KBatch {
   uint32_t stage_bytes;  // bytes of the exponent array
   uint32_t slot_words;   // 32-bit words of each thread's private slot
   uint32_t sub_words;    // deeper-table words kept in shared memory (0: global)
-  uint32_t pad;
+  uint32_t sm_bytes;     // sign/mantissa bytes per stage slot (warp-specialised kernel)
 };
 
 // ---- shared memory layout --------------------------------------------------
@@ -660,18 +660,19 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
 //
 // With the counts in shared memory every warp can work out where its output
 // goes on its own, so the thread block needs no block-wide barrier per format
-// block.  One producer warp (one lane) keeps kWsStages stage slots filled,
-// each guarded by a "full" mbarrier (completed by the bulk copies) and an
-// "empty" mbarrier (one arrival per consumer warp once it holds the slot's
-// data in registers).  Each of the T/32 consumer warps, per format block:
+// block.  One producer warp (one lane) keeps kWsStages stage slots filled
+// (bitstream slice, gap fields, chunk counts, positions and the block's
+// sign/mantissa bytes), each guarded by a "full" mbarrier (completed by the
+// bulk copies) and an "empty" mbarrier (one arrival per consumer warp when it
+// is done with the block).  Each of the T/32 consumer warps, per format block:
 //   - sums the block's chunk counts before its own chunks and over the whole
 //     block (two warp reductions over T bytes) and scans its lanes' counts;
-//   - releases the slot;
 //   - decodes straight into its private exponent region (zeroed; words shared
 //     by two lanes merged with OR) and checks every count;
-//   - writes its own output range: whole 16-element groups with 16-byte
-//     stores, the two ragged edge groups one element per lane.
-constexpr int kWsStages = 4;
+//   - writes its own output range from shared memory: whole 16-element
+//     groups with 16-byte stores, the two ragged edge groups one element per
+//     lane; then releases the slot.
+constexpr int kWsStages = 2;
 
 template <int T, int C>
 struct WsLayout {
@@ -679,8 +680,9 @@ struct WsLayout {
   static constexpr uint32_t gaps_bytes = T * 5 / 8 + 16;
   static constexpr uint32_t counts_bytes = T;
   static constexpr uint32_t meta_bytes = 16;
-  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes + counts_bytes + meta_bytes;
-  static_assert(slot_bytes % 16 == 0, "alignment");
+  // the block's sign/mantissa bytes follow (KBatch::sm_bytes of them)
+  static constexpr uint32_t head_bytes = bits_bytes + gaps_bytes + counts_bytes + meta_bytes;
+  static_assert(head_bytes % 16 == 0, "alignment");
 };
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -689,28 +691,30 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 
 template <int T, int C>
 __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t *slot,
-                                         uint32_t full, uint32_t region_bytes) {
+                                         uint32_t full, uint32_t sm_capacity) {
   using L = WsLayout<T, C>;
   const uint32_t P0 = tk.block_out_pos[b], P1 = tk.block_out_pos[b + 1];
   const uint32_t expected = P1 - P0;
   // a warp's exponents fit its region whatever the block: every chunk count
   // is checked against max_chunk_elems before decoding
-  const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems;
+  const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems &&
+                  expected + 32 <= sm_capacity;
   *reinterpret_cast<uint4 *>(slot + L::bits_bytes + L::gaps_bytes + L::counts_bytes) =
       make_uint4(P0, P1, ok ? 1u : 0u, b);
   if (!ok) {
     mbar_arrive_expect_tx(full, 0);
     return;
   }
-  mbar_arrive_expect_tx(full, L::bits_bytes + L::gaps_bytes + L::counts_bytes);
+  const uint32_t sm_begin = P0 & ~15u;
+  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
+  mbar_arrive_expect_tx(full, L::bits_bytes + L::gaps_bytes + L::counts_bytes + sm_bytes);
   bulk_g2s(smem_addr(slot), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, full);
   bulk_g2s(smem_addr(slot + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
            full);
   bulk_g2s(smem_addr(slot + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
            L::counts_bytes, full);
-  const uint32_t sm_begin = P0 & ~15u;
-  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
-  if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
+  if (sm_bytes)
+    bulk_g2s(smem_addr(slot + L::head_bytes), tk.sign_mantissa + sm_begin, sm_bytes, full);
 }
 
 // Sum of the byte counts a lane holds (T/32 of them).
@@ -740,7 +744,8 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
   uint32_t *lut0_s = reinterpret_cast<uint32_t *>(smem + kOffLut0);
   uint2 *wide_s = reinterpret_cast<uint2 *>(smem + kOffWide);
   uint8_t *stages = smem + kOffStages;
-  uint8_t *regions = stages + kWsStages * L::slot_bytes;
+  const uint32_t slot_bytes = L::head_bytes + kb.sm_bytes;
+  uint8_t *regions = stages + kWsStages * slot_bytes;
   uint32_t *sub_s = reinterpret_cast<uint32_t *>(regions + CONSUMERS * kb.stage_bytes);
 
   int ti = 0;
@@ -787,7 +792,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
           report(kb.err, DF11_DEV_ERR_TIMEOUT);
           break;
         }
-        ws_issue<T, C>(tk, b, stages + s * L::slot_bytes, smem_addr(&bars[s]), kb.stage_bytes);
+        ws_issue<T, C>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
       }
     }
     return;
@@ -799,7 +804,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
   uint32_t k = 0;
   for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
     const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
-    const uint8_t *slot = stages + s * L::slot_bytes;
+    const uint8_t *slot = stages + s * slot_bytes;
     if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_addr(&bars[s]), par))) {
       if (lane == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
       return;  // whole warp
@@ -825,17 +830,18 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
 #pragma unroll
     for (int j = 0; j < NW; ++j)
       w[j] = __byte_perm(*reinterpret_cast<const uint32_t *>(slot + tid * C + 4 * j), 0, 0x0123);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&bars[kWsStages + s]));  // slot free for refill
 
     const uint32_t before = __reduce_add_sync(0xFFFFFFFFu,
                                               lane < warp * 32 / (T / 32) ? lsum : 0u);
     const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, lsum);
+    const uint32_t release = smem_addr(&bars[kWsStages + s]);
     if (!m.z || total != expected ||
         __any_sync(0xFFFFFFFFu, cnt > tk.max_chunk_elems)) {
       if (warp == 0 && lane == 0) report(kb.err, m.z ? (total != expected ? DF11_DEV_ERR_COUNT
                                                                           : DF11_DEV_ERR_CAPACITY)
                                                      : DF11_DEV_ERR_CAPACITY);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(release);
       continue;
     }
     if (chunk_bit >= tk.total_bits) {
@@ -874,18 +880,20 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
       for (uint32_t i = lane; i < (span + 15u) >> 4; i += 32)
         reinterpret_cast<uint4 *>(region_p)[i] = make_uint4(0, 0, 0, 0);
       __syncwarp();
+      if (lane == 0) mbar_arrive(release);
       continue;
     }
     __syncwarp();
 
-    // output of this warp's elements [G0, G0 + warp_total)
+    // output of this warp's elements [G0, G0 + warp_total); its sign/mantissa
+    // bytes are in the slot, which starts at element P0 & ~15
     const uint32_t base = G0 & ~15u;
     uint16_t *out = tk.out + base;
-    const uint8_t *smg = tk.sign_mantissa + base;
+    const uint8_t *smg = slot + L::head_bytes + (base - (P0 & ~15u));
     const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
     for (uint32_t g = g_begin + lane; g < g_end; g += 32) {
       const uint32_t i0 = g << 4;
-      const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(smg + i0));
+      const uint4 sv = *reinterpret_cast<const uint4 *>(smg + i0);
       uint4 *rp = reinterpret_cast<uint4 *>(region_p + i0);
       const uint4 rv = *rp;
       *rp = make_uint4(0, 0, 0, 0);
@@ -905,6 +913,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
       if (mine) region_p[i] = 0;
     }
     __syncwarp();
+    if (lane == 0) mbar_arrive(release);  // slot free for refill
   }
 }
 
@@ -1042,8 +1051,9 @@ uint32_t region_bytes_for(uint32_t max_chunk_elems) {
   return (15u + 32u * max_chunk_elems + 4u + 15u) & ~15u;
 }
 
-size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t region, uint32_t sub_words) {
-  const size_t slot = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16 + T + 16;
+size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
+                       uint32_t sub_words) {
+  const size_t slot = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16 + T + 16 + sm_bytes;
   return (size_t)kOffStages + kWsStages * slot + (size_t)(T / 32) * region +
          (size_t)sub_words * 4;
 }
@@ -1086,10 +1096,11 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   if (ws) {
     kb.stage_bytes = region_bytes_for(max_chunk);  // bytes of each warp's region
     kb.slot_words = 0;
-    size_t smem = ws_shared_bytes(C, T, kb.stage_bytes, kb.sub_words);
+    kb.sm_bytes = stage_bytes_for(max_elems);
+    size_t smem = ws_shared_bytes(C, T, kb.sm_bytes, kb.stage_bytes, kb.sub_words);
     if (smem > 227 * 1024 && kb.sub_words) {
       kb.sub_words = 0;
-      smem = ws_shared_bytes(C, T, kb.stage_bytes, 0);
+      smem = ws_shared_bytes(C, T, kb.sm_bytes, kb.stage_bytes, 0);
     }
     if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
     if (T == 256 && C == 8) return launch_ws<256, 8>(kb, blocks, smem, s, 5);
