@@ -60,7 +60,7 @@ namespace {
 constexpr int kSubTablesInSmem = 8;        // deeper tables kept in shared memory
 constexpr uint32_t kSpinLimit = 1u << 20;  // x ~1 us suspend hint: ~1 s
 constexpr uint32_t kSuspendHintNs = 1000;
-constexpr int kWideBits = 10;              // index bits of the derived table
+constexpr int kWideBits = 11;              // index bits of the derived table
 constexpr int kWideSyms = 4;               // codewords per derived entry
 
 struct KTensor {
