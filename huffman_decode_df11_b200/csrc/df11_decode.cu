@@ -149,6 +149,25 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts128_zero(uint32_t a) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts8_zero(uint32_t a) {
+  asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "h"((unsigned short)0) : "memory");
+}
 __device__ __forceinline__ void red_or32(uint32_t a, uint32_t v) {
   asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
@@ -886,22 +905,26 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
     __syncwarp();
 
     // output of this warp's elements [G0, G0 + warp_total); its sign/mantissa
-    // bytes are in the slot, which starts at element P0 & ~15
+    // bytes are in the slot, which starts at element P0 & ~15.  Group g (16
+    // elements) is at byte 16g of the region and of `sm` and at element 16g of
+    // `out`.
     const uint32_t base = G0 & ~15u;
     uint16_t *out = tk.out + base;
-    const uint8_t *smg = slot + L::head_bytes + (base - (P0 & ~15u));
+    const uint32_t sm = smem_addr(slot + L::head_bytes) + (base - (P0 & ~15u));
     const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
-    for (uint32_t g = g_begin + lane; g < g_end; g += 32) {
-      const uint32_t i0 = g << 4;
-      const uint4 sv = *reinterpret_cast<const uint4 *>(smg + i0);
-      uint4 *rp = reinterpret_cast<uint4 *>(region_p + i0);
-      const uint4 rv = *rp;
-      *rp = make_uint4(0, 0, 0, 0);
-      const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
-      const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
-      uint4 *o = reinterpret_cast<uint4 *>(out + i0);
-      o[0] = make_uint4(a.x, a.y, c.x, c.y);
-      o[1] = make_uint4(e2.x, e2.y, f.x, f.y);
+    {
+      uint32_t g = g_begin + (uint32_t)lane;
+      uint32_t sa_sm = sm + 16u * g, sa_rg = region + 16u * g;
+      uint4 *o = reinterpret_cast<uint4 *>(out) + 2u * g;
+      for (; g < g_end; g += 32, sa_sm += 512u, sa_rg += 512u, o += 64) {
+        const uint4 sv = lds128(sa_sm);
+        const uint4 rv = lds128(sa_rg);
+        sts128_zero(sa_rg);  // leave the region zeroed for the next block
+        const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
+        const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+        o[0] = make_uint4(a.x, a.y, c.x, c.y);
+        o[1] = make_uint4(e2.x, e2.y, f.x, f.y);
+      }
     }
     if (span) {  // lanes 0-15: first group, 16-31: last group
       const uint32_t gl = (span - 1) >> 4;
@@ -909,8 +932,10 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
       const bool last_partial = (span & 15u) != 0 && gl != 0;
       const uint32_t i = lane < 16 ? (uint32_t)lane : (gl << 4) + (uint32_t)(lane - 16);
       const bool mine = lane < 16 ? first_partial : last_partial;
-      if (mine && i >= head && i < span) out[i] = fuse1(smg[i], region_p[i]);
-      if (mine) region_p[i] = 0;
+      if (mine) {
+        if (i >= head && i < span) out[i] = fuse1(lds8(sm + i), lds8(region + i));
+        sts8_zero(region + i);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(release);  // slot free for refill
