@@ -736,21 +736,6 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
     bulk_g2s(smem_addr(slot + L::head_bytes), tk.sign_mantissa + sm_begin, sm_bytes, full);
 }
 
-// Sum of the byte counts a lane holds (T/32 of them).
-template <int T>
-__device__ __forceinline__ uint32_t lane_count_sum(const uint8_t *counts, int lane) {
-  if (T == 128) {
-    return __dp4a(*reinterpret_cast<const uint32_t *>(counts + 4 * lane), 0x01010101u, 0u);
-  } else if (T == 256) {
-    const uint2 v = *reinterpret_cast<const uint2 *>(counts + 8 * lane);
-    return __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u, 0u));
-  } else {
-    const uint4 v = *reinterpret_cast<const uint4 *>(counts + 16 * lane);
-    return __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u,
-                  __dp4a(v.z, 0x01010101u, __dp4a(v.w, 0x01010101u, 0u))));
-  }
-}
-
 template <int T, int C>
 __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
     df11_decode_ws_kernel(const __grid_constant__ KBatch kb) {
@@ -828,27 +813,38 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
       if (lane == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
       return;  // whole warp
     }
-    const uint4 m = *reinterpret_cast<const uint4 *>(slot + L::bits_bytes + L::gaps_bytes +
-                                                     L::counts_bytes);
+    // everything this warp needs from the slot, into registers (32-bit
+    // shared-window addresses throughout)
+    const uint32_t slot_sa = smem_addr(slot);
+    const uint32_t counts_sa = slot_sa + L::bits_bytes + L::gaps_bytes;
+    const uint4 m = lds128(counts_sa + L::counts_bytes);
     const uint32_t P0 = m.x, P1 = m.y, expected = P1 - P0;
-    const uint8_t *counts = slot + L::bits_bytes + L::gaps_bytes;
-    // everything this warp needs from the slot, into registers
-    const uint32_t lsum = lane_count_sum<T>(counts, lane);
-    const uint32_t cnt = counts[tid];
+    uint32_t lsum;
+    if (T == 128) {
+      lsum = __dp4a(lds32(counts_sa + 4u * lane), 0x01010101u, 0u);
+    } else if (T == 256) {
+      const uint2 v = lds64(counts_sa + 8u * lane);
+      lsum = __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u, 0u));
+    } else {
+      const uint4 v = lds128(counts_sa + 16u * lane);
+      lsum = __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u,
+                    __dp4a(v.z, 0x01010101u, __dp4a(v.w, 0x01010101u, 0u))));
+    }
+    const uint32_t cnt = lds8(counts_sa + tid);
     const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
     int start, end;
     {
       const uint32_t bit = 5u * (uint32_t)tid;
-      const uint32_t *g32 = reinterpret_cast<const uint32_t *>(slot + L::bits_bytes) + (bit >> 5);
-      const uint32_t v = __funnelshift_l(__byte_perm(g32[1], 0, 0x0123),
-                                         __byte_perm(g32[0], 0, 0x0123), bit);
+      const uint32_t ga = slot_sa + L::bits_bytes + 4u * (bit >> 5);
+      const uint32_t v = __funnelshift_l(__byte_perm(lds32(ga + 4u), 0, 0x0123),
+                                         __byte_perm(lds32(ga), 0, 0x0123), bit);
       start = (int)(v >> 27);
       end = C * 8 + (int)((v >> 22) & 31u);
     }
     uint32_t w[NW];
 #pragma unroll
     for (int j = 0; j < NW; ++j)
-      w[j] = __byte_perm(*reinterpret_cast<const uint32_t *>(slot + tid * C + 4 * j), 0, 0x0123);
+      w[j] = __byte_perm(lds32(slot_sa + (uint32_t)tid * C + 4u * j), 0, 0x0123);
 
     const uint32_t before = __reduce_add_sync(0xFFFFFFFFu,
                                               lane < warp * 32 / (T / 32) ? lsum : 0u);
