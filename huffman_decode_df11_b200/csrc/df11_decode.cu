@@ -235,8 +235,8 @@ __device__ __forceinline__ bool decode_one(uint32_t win, const uint32_t *__restr
 
 // Derived table: entry i holds the codewords that lie wholly inside the WB
 // bits i (at most kWideSyms): x = exponents (first in bits 0-7),
-// y = bits used | (8 * count) << 16, so that one add moves both the bit
-// position and the byte count of a packed (position, count) register.
+// y = bits used | count << 16, so that one add moves both the bit position
+// and the output byte position of a packed (bit, byte) register.
 // y == 0: the first codeword is longer than WB bits (or invalid) and takes
 // the slow path.
 template <int T>
@@ -270,7 +270,7 @@ __device__ void build_wide(uint2 *wide, const uint32_t *lut0, const uint8_t *len
       }
       if (stop || used >= kWideBits) break;
     }
-    wide[i] = n ? make_uint2(syms, used | ((8u * n) << 16)) : make_uint2(0, 0);
+    wide[i] = n ? make_uint2(syms, used | (n << 16)) : make_uint2(0, 0);
   }
 }
 
@@ -299,10 +299,11 @@ __device__ __forceinline__ uint32_t window(const uint32_t (&w)[C / 4 + 1], uint3
 // Walk one thread's codewords [start, end) (bit positions relative to its
 // chunk's first bit) and append their exponents to its private slot: word j
 // at shared address slot + 4*T*j.  `pk` packs the bit position (bits 0-15)
-// with 8x the bytes waiting in the 64-bit accumulator a1:a0 (bits 16-23).
-// The current word is stored after every lookup and the slot address moves
-// on when it is full, so no branch but the loop's and the rare slow path's.
-// Returns the number of codewords; sets `bad` on inconsistent data.
+// with the number of bytes waiting in the 64-bit accumulator a1:a0 (bits
+// 16-23).  The current word is stored after every lookup and the slot
+// address moves on when it is full, so no branch but the loop's and the rare
+// slow path's.  Returns the number of codewords; sets `bad` on inconsistent
+// data.
 template <int T, int C, bool MASKED>
 __device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1], int start,
                                                  const int end, uint32_t wide,
@@ -324,32 +325,34 @@ __device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1],
         bad = DF11_DEV_ERR_TABLE;
         return 0;
       }
-      e = make_uint2(sym, len | (8u << 16));
+      e = make_uint2(sym, len | (1u << 16));
     }
-    const uint32_t sh = pk >> 16;
+    const uint32_t sh = (pk >> 16) << 3;
     a0 |= e.x << sh;
     a1 |= __funnelshift_l(e.x, 0u, sh);  // bytes pushed past the low word
     pk += e.y;
     sts32(sa, a0);
-    if (pk >= (32u << 16)) {  // the word is complete: move on
+    if (pk >= (4u << 16)) {  // the word is complete: move on
       sa = min(sa + 4u * T, sa_last);
       ++words;
       a0 = a1;
       a1 = 0;
-      pk -= 32u << 16;
+      pk -= 4u << 16;
     }
   }
   if (pk >> 16) sts32(sa, a0);
   if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
-  return words * 4u + (pk >> 19);
+  return words * 4u + (pk >> 16);
 }
 
 // The same walk when the thread's output place is known before it decodes
 // (the format's chunk count): exponents go straight into the block's
-// exponent array at byte d onwards, as whole 32-bit words OR-ed into the
-// (zeroed) array, which also merges the words shared with neighbours.  The
-// accumulator starts d & 3 bytes in; `limit` is the last word the thread may
-// touch.  Returns the number of codewords decoded.
+// (zeroed) exponent array from byte d on.  Every lookup ORs its up to four
+// bytes into the word that holds the next byte and the word after it (the
+// part that spills over; zero when nothing does), which also merges the
+// words a thread shares with its neighbours.  `pk` packs the bit position
+// (bits 0-15) with the next byte (bits 16-31); `limit` is the last word the
+// thread may touch.  Returns the number of codewords decoded.
 template <int T, int C, bool MASKED>
 __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1], int start,
                                                   const int end, uint32_t wide,
@@ -358,9 +361,7 @@ __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1]
                                                   const uint32_t *sub, uint32_t num_luts,
                                                   uint32_t ex, uint32_t d, uint32_t limit,
                                                   int &bad) {
-  uint32_t a0 = 0, a1 = 0, words = 0;
-  uint32_t pk = (uint32_t)start | (((d & 3u) * 8u) << 16);
-  uint32_t sa = ex + (d & ~3u);
+  uint32_t pk = (uint32_t)start | (d << 16);
   while ((int)(pk & 0xFFFFu) < end) {
     const uint32_t win = window<C>(w, pk & 0xFFFFu);
     uint2 e = lds64(wide + ((win >> (32 - kWideBits)) << 3));
@@ -370,24 +371,17 @@ __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1]
         bad = DF11_DEV_ERR_TABLE;
         return 0;
       }
-      e = make_uint2(sym, len | (8u << 16));
+      e = make_uint2(sym, len | (1u << 16));
     }
-    const uint32_t sh = pk >> 16;
-    a0 |= e.x << sh;
-    a1 |= __funnelshift_l(e.x, 0u, sh);
+    const uint32_t bp = pk >> 16;
+    const uint32_t sh = (bp & 3u) << 3;
+    const uint32_t a = min(ex + (bp & ~3u), limit);
+    red_or32(a, e.x << sh);
+    red_or32(a + 4u, __funnelshift_l(e.x, 0u, sh));
     pk += e.y;
-    if (pk >= (32u << 16)) {
-      red_or32(sa, a0);
-      sa = min(sa + 4u, limit);
-      ++words;
-      a0 = a1;
-      a1 = 0;
-      pk -= 32u << 16;
-    }
   }
-  if (pk >> 16) red_or32(sa, a0);
   if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
-  return words * 4u + (pk >> 19) - (d & 3u);
+  return (pk >> 16) - d;
 }
 
 // four sign/mantissa bytes and four rotated exponents -> four BF16 words
@@ -1067,9 +1061,10 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStrea
 }
 
 // Per-warp exponent region of the warp-specialised kernel: the warp's head
-// (< 16), up to 32 chunks of max_chunk_elems exponents, a word of slack.
+// (< 16), up to 32 chunks of max_chunk_elems exponents, two words of slack
+// (a lookup ORs into the word after the one it fills).
 uint32_t region_bytes_for(uint32_t max_chunk_elems) {
-  return (15u + 32u * max_chunk_elems + 4u + 15u) & ~15u;
+  return (15u + 32u * max_chunk_elems + 8u + 15u) & ~15u;
 }
 
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
