@@ -1113,6 +1113,10 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     kb.stage_bytes = region_bytes_for(max_chunk);  // bytes of each warp's region
     kb.slot_words = 0;
     kb.sm_bytes = stage_bytes_for(max_elems);
+    // deeper tables only serve codewords longer than the derived table's
+    // index (about one lookup in a thousand): read them from global memory
+    // and spend the shared memory on one more resident thread block
+    kb.sub_words = 0;
     size_t smem = ws_shared_bytes(C, T, kb.sm_bytes, kb.stage_bytes, kb.sub_words);
     if (smem > 227 * 1024 && kb.sub_words) {
       kb.sub_words = 0;
