@@ -320,7 +320,8 @@ def run_b200(args, world, rank, local):
     alg = [sum(algorithmic_bytes(hosts[i], counts) for i in g) for g in groups]
     achieved = sum(alg) / (sum(per_group_ms) * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
-    traffic = recorded_traffic(args.config)
+    # the capture covers the chunk-count kernel; the page-layout kernel has none
+    traffic = recorded_traffic(args.config) if counts else None
 
     # end to end through the public API: host (pinned) compressed tensors in,
     # host BF16 out, copies inside the timed region

@@ -101,7 +101,7 @@ struct KBatch {
 // [304,560)    code lengths by rotated exponent
 // [560,1584)   table 0 (rotated)
 // [1584, ...)  wide table (2^WB x 8 bytes)
-// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16), counts (T)
+// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16)
 // then         exponent array (stage_bytes), private slots (slot_words*T*4),
 //              deeper tables (sub_words*4)
 constexpr uint32_t kOffMbar = 0;
@@ -117,9 +117,8 @@ template <int T, int C>
 struct Layout {
   static constexpr uint32_t bits_bytes = T * C + 16;
   static constexpr uint32_t gaps_bytes = T * 5 / 8 + 16;
-  static constexpr uint32_t counts_bytes = T;
-  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes + counts_bytes;  // one slot
-  static_assert(bits_bytes % 16 == 0 && gaps_bytes % 16 == 0 && T % 16 == 0, "alignment");
+  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes;  // one slot
+  static_assert(bits_bytes % 16 == 0 && gaps_bytes % 16 == 0, "alignment");
 };
 
 __device__ __forceinline__ uint32_t rot8x3(uint32_t v) {
@@ -235,8 +234,8 @@ __device__ __forceinline__ bool decode_one(uint32_t win, const uint32_t *__restr
 
 // Derived table: entry i holds the codewords that lie wholly inside the WB
 // bits i (at most kWideSyms): x = exponents (first in bits 0-7),
-// y = bits used | count << 16, so that one add moves both the bit position
-// and the output byte position of a packed (bit, byte) register.
+// y = bits used | 8 * count << 16, so that one add moves both the bit
+// position and the output bit offset of a packed (bit, output bit) register.
 // y == 0: the first codeword is longer than WB bits (or invalid) and takes
 // the slow path.
 template <int T>
@@ -270,7 +269,7 @@ __device__ void build_wide(uint2 *wide, const uint32_t *lut0, const uint8_t *len
       }
       if (stop || used >= kWideBits) break;
     }
-    wide[i] = n ? make_uint2(syms, used | (n << 16)) : make_uint2(0, 0);
+    wide[i] = n ? make_uint2(syms, used | (n << 19)) : make_uint2(0, 0);
   }
 }
 
@@ -299,8 +298,8 @@ __device__ __forceinline__ uint32_t window(const uint32_t (&w)[C / 4 + 1], uint3
 // Walk one thread's codewords [start, end) (bit positions relative to its
 // chunk's first bit) and append their exponents to its private slot: word j
 // at shared address slot + 4*T*j.  `pk` packs the bit position (bits 0-15)
-// with the number of bytes waiting in the 64-bit accumulator a1:a0 (bits
-// 16-23).  The current word is stored after every lookup and the slot
+// with the number of bits waiting in the 64-bit accumulator a1:a0 (bits
+// 16-31, a multiple of 8).  The current word is stored after every lookup and the slot
 // address moves on when it is full, so no branch but the loop's and the rare
 // slow path's.  Returns the number of codewords; sets `bad` on inconsistent
 // data.
@@ -325,24 +324,24 @@ __device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1],
         bad = DF11_DEV_ERR_TABLE;
         return 0;
       }
-      e = make_uint2(sym, len | (1u << 16));
+      e = make_uint2(sym, len | (8u << 16));
     }
-    const uint32_t sh = (pk >> 16) << 3;
+    const uint32_t sh = pk >> 16;
     a0 |= e.x << sh;
     a1 |= __funnelshift_l(e.x, 0u, sh);  // bytes pushed past the low word
     pk += e.y;
     sts32(sa, a0);
-    if (pk >= (4u << 16)) {  // the word is complete: move on
+    if (pk >= (32u << 16)) {  // the word is complete: move on
       sa = min(sa + 4u * T, sa_last);
       ++words;
       a0 = a1;
       a1 = 0;
-      pk -= 4u << 16;
+      pk -= 32u << 16;
     }
   }
   if (pk >> 16) sts32(sa, a0);
   if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
-  return words * 4u + (pk >> 16);
+  return words * 4u + (pk >> 19);
 }
 
 // The same walk when the thread's output place is known before it decodes
@@ -351,8 +350,9 @@ __device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1],
 // bytes into the word that holds the next byte and the word after it (the
 // part that spills over; zero when nothing does), which also merges the
 // words a thread shares with its neighbours.  `pk` packs the bit position
-// (bits 0-15) with the next byte (bits 16-31); `limit` is the last word the
-// thread may touch.  Returns the number of codewords decoded.
+// (bits 0-15) with the bit offset of the next byte (bits 16-31, so d stays
+// below 8192); `limit` is the last word the thread may touch.  Returns the
+// number of codewords decoded.
 template <int T, int C, bool MASKED>
 __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1], int start,
                                                   const int end, uint32_t wide,
@@ -361,7 +361,7 @@ __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1]
                                                   const uint32_t *sub, uint32_t num_luts,
                                                   uint32_t ex, uint32_t d, uint32_t limit,
                                                   int &bad) {
-  uint32_t pk = (uint32_t)start | (d << 16);
+  uint32_t pk = (uint32_t)start | (d << 19);
   while ((int)(pk & 0xFFFFu) < end) {
     const uint32_t win = window<C>(w, pk & 0xFFFFu);
     uint2 e = lds64(wide + ((win >> (32 - kWideBits)) << 3));
@@ -371,17 +371,80 @@ __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1]
         bad = DF11_DEV_ERR_TABLE;
         return 0;
       }
-      e = make_uint2(sym, len | (1u << 16));
+      e = make_uint2(sym, len | (8u << 16));
     }
-    const uint32_t bp = pk >> 16;
-    const uint32_t sh = (bp & 3u) << 3;
-    const uint32_t a = min(ex + (bp & ~3u), limit);
+    const uint32_t sh = (pk >> 16) & 24u;
+    const uint32_t a = min(ex + ((pk >> 21) << 2), limit);
     red_or32(a, e.x << sh);
     red_or32(a + 4u, __funnelshift_l(e.x, 0u, sh));
     pk += e.y;
   }
   if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
-  return (pk >> 16) - d;
+  return (pk >> 19) - d;
+}
+
+// The direct walk for masked streams when the chunk's count is known, with
+// fewer operations per lookup:
+//   - the chunk's bits sit in a shifting window of NW words (next bit at the
+//     top of s[0]), moved on by funnel shifts whose amount is the entry's
+//     second word itself: funnel shifts use only its low five bits, which
+//     hold the bits used (at most kWideBits here), and ones come in from the
+//     right, so the stream stays masked past its last word;
+//   - the loop ends on the element count, not the bit position: it runs
+//     while the output bit offset (bits 16-31 of `pk`, bit position in bits
+//     0-15) is below 8*(d+cnt).  Every iteration emits at least one element,
+//     so a corrupt stream stops within cnt lookups and writes at most three
+//     bytes (plus the spill word) past the thread's range, which the region's
+//     slack absorbs: no clamp on the address.  Bits past `end` are ones, so
+//     on valid data the last lookup stops exactly at `end` (checked after).
+// Returns the number of elements written.
+template <int C>
+__device__ __forceinline__ uint32_t decode_counted(const uint32_t (&w)[C / 4 + 1], int start,
+                                                   const int end, uint32_t wide,
+                                                   const uint32_t *__restrict__ lut0,
+                                                   const uint8_t *__restrict__ lens,
+                                                   const uint32_t *sub, uint32_t num_luts,
+                                                   uint32_t ex, uint32_t d, uint32_t cnt,
+                                                   int &bad) {
+  constexpr int NW = C / 4 + 1;
+  uint32_t s[NW];
+#pragma unroll
+  for (int j = 0; j < NW - 1; ++j) s[j] = __funnelshift_l(w[j + 1], w[j], (uint32_t)start);
+  s[NW - 1] = __funnelshift_l(0xFFFFFFFFu, w[NW - 1], (uint32_t)start);
+  uint32_t pk = (uint32_t)start | ((8u * d) << 16);
+  const uint32_t lim = (8u * (d + cnt)) << 16;
+  while (pk < lim) {
+    uint2 e = lds64(wide + ((s[0] >> (32 - kWideBits)) << 3));
+    if (e.y == 0) {
+      // rare: a codeword longer than the derived table's index.  Shift by
+      // half its length here and the rest below (both at most 16 bits, in
+      // the funnel shifts' range).
+      uint32_t sym, len;
+      if (!decode_one(s[0], lut0, lens, sub, num_luts, sym, len)) {
+        bad = DF11_DEV_ERR_TABLE;
+        return 0;
+      }
+      const uint32_t half = len >> 1;
+#pragma unroll
+      for (int j = 0; j < NW - 1; ++j) s[j] = __funnelshift_l(s[j + 1], s[j], half);
+      s[NW - 1] = __funnelshift_l(0xFFFFFFFFu, s[NW - 1], half);
+      pk += half;
+      e = make_uint2(sym, (len - half) | (8u << 16));
+    }
+    const uint32_t sh = pk >> 16;  // funnel shifts use sh & 31: the bit offset in the word
+    const uint32_t a = ex + ((pk >> 21) << 2);
+    red_or32(a, __funnelshift_l(0u, e.x, sh));
+    red_or32(a + 4u, __funnelshift_l(e.x, 0u, sh));
+#pragma unroll
+    for (int j = 0; j < NW - 1; ++j) s[j] = __funnelshift_l(s[j + 1], s[j], e.y);
+    s[NW - 1] = __funnelshift_l(0xFFFFFFFFu, s[NW - 1], e.y);
+    pk += e.y;
+  }
+  // a count that disagrees with the stream ends the walk short of `end`
+  // (too small) or past it (too large, or a corrupt stream)
+  const int pos = (int)(pk & 0xFFFFu);
+  if (pos != end) bad = pos < end ? DF11_DEV_ERR_COUNT : DF11_DEV_ERR_OVERRUN;
+  return (pk >> 19) - d;
 }
 
 // four sign/mantissa bytes and four rotated exponents -> four BF16 words
@@ -416,14 +479,10 @@ __device__ __forceinline__ void issue_block(const KTensor &tk, uint32_t b, uint3
     mbar_arrive_expect_tx(bar, 0);
     return;
   }
-  const bool counts = tk.chunk_counts != nullptr;
-  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes + (counts ? L::counts_bytes : 0u));
+  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes);
   bulk_g2s(smem_addr(stage), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, bar);
   bulk_g2s(smem_addr(stage + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
            bar);
-  if (counts)
-    bulk_g2s(smem_addr(stage + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
-             L::counts_bytes, bar);
   const uint32_t sm_begin = P0 & ~15u;
   const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
   if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
@@ -542,14 +601,11 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
       if (tk.masked)  // ones from bit `end` on
         w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
     }
-    const bool direct = tk.chunk_counts != nullptr;  // uniform in the thread block
     const uint32_t ex_addr = smem_addr(ex_s);
 
-    // counts: stored (direct) or by decoding into the private slot
+    // count by decoding into the private slot
     uint32_t cnt = 0;
-    if (direct) {
-      cnt = stage[L::bits_bytes + L::gaps_bytes + tid];
-    } else if (!bad) {
+    if (!bad) {
       const uint32_t slot = smem_addr(slots + tid);
       if (tk.masked)
         cnt = decode_chunk<T, C, true>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
@@ -588,18 +644,7 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
     }
 
     const uint32_t d = head + excl;  // my first byte in the exponent array
-    if (direct) {
-      // one pass straight to the exponent array, then check the count
-      const uint32_t limit = ex_addr + ((d + (cnt ? cnt : 1u) - 1u) & ~3u);
-      uint32_t got;
-      if (tk.masked)
-        got = decode_direct<T, C, true>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
-                                        tk.num_luts, ex_addr, d, limit, bad);
-      else
-        got = decode_direct<T, C, false>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
-                                         tk.num_luts, ex_addr, d, limit, bad);
-      if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
-    } else if (cnt) {
+    if (cnt) {
       // compact: slot bytes [0, cnt) -> ex_s[d, d+cnt).  Destination word k
       // holds slot bytes 4k-s .. 4k-s+3 (s = d & 3): a funnel shift of slot
       // words k-1 and k.  The first and last words are shared with the
@@ -661,10 +706,10 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
         if (mine) ex_s[i] = 0;
       }
     }
-    // No barrier here: the next block's decode writes only private slots or,
-    // for direct decoding, the exponent array after the next scan barrier,
-    // which every thread reaches after finishing this output; the stage slot
-    // refilled next was last read before this block's scan barrier.
+    // No barrier here: the next block's decode writes only private slots,
+    // and the exponent array only after the next scan barrier, which every
+    // thread reaches after finishing this output; the stage slot refilled
+    // next was last read before this block's scan barrier.
   }
 }
 
@@ -712,8 +757,13 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   // is checked against max_chunk_elems before decoding
   const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems &&
                   expected + 32 <= sm_capacity;
+  // bits of the stream inside this block: all of them but in the last block
+  const uint64_t bit0 = (uint64_t)b * (T * C * 8);
+  const uint32_t valid_bits = tk.total_bits - bit0 < (uint64_t)(T * C * 8)
+                                  ? (uint32_t)(tk.total_bits - bit0)
+                                  : 0xFFFFFFFFu;
   *reinterpret_cast<uint4 *>(slot + L::bits_bytes + L::gaps_bytes + L::counts_bytes) =
-      make_uint4(P0, P1, ok ? 1u : 0u, b);
+      make_uint4(P0, P1, ok ? 1u : 0u, valid_bits);
   if (!ok) {
     mbar_arrive_expect_tx(full, 0);
     return;
@@ -825,7 +875,6 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
                     __dp4a(v.z, 0x01010101u, __dp4a(v.w, 0x01010101u, 0u))));
     }
     const uint32_t cnt = lds8(counts_sa + tid);
-    const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
     int start, end;
     {
       const uint32_t bit = 5u * (uint32_t)tid;
@@ -853,15 +902,19 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
       if (lane == 0) mbar_arrive(release);
       continue;
     }
-    if (chunk_bit >= tk.total_bits) {
-      start = end = 0;
-    } else if ((uint64_t)end > tk.total_bits - chunk_bit) {
-      end = (int)(tk.total_bits - chunk_bit);
+    if (m.w != 0xFFFFFFFFu) {  // the block that holds the end of the stream
+      const uint32_t b0 = (uint32_t)tid * (C * 8);
+      if (b0 >= m.w) start = end = 0;
+      else if ((uint32_t)end > m.w - b0) end = (int)(m.w - b0);
     }
-    if (tk.masked) {
+    if (tk.masked) {  // ones from bit `end` on; mostly only the last word has any
+      if (end >= C * 8) {
+        w[NW - 1] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)(end - C * 8));
+      } else {
 #pragma unroll
-      for (int j = 0; j < NW; ++j)
-        w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
+        for (int j = 0; j < NW; ++j)
+          w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
+      }
     }
     uint32_t incl = cnt;
 #pragma unroll
@@ -873,20 +926,22 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
     const uint32_t G0 = P0 + before;            // first element of this warp
     const uint32_t head = G0 & 15u, span = head + warp_total;
     const uint32_t d = head + incl - cnt;       // my first byte in the region
-    const uint32_t limit = region + ((d + (cnt ? cnt : 1u) - 1u) & ~3u);
     int bad = 0;
     uint32_t got;
-    if (tk.masked)
-      got = decode_direct<T, C, true>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts,
-                                      region, d, limit, bad);
-    else
+    if (tk.masked) {
+      got = decode_counted<C>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts, region, d,
+                              cnt, bad);
+    } else {
+      const uint32_t limit = region + ((d + (cnt ? cnt : 1u) - 1u) & ~3u);
       got = decode_direct<T, C, false>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts,
                                        region, d, limit, bad);
+    }
     if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
     if (__any_sync(0xFFFFFFFFu, bad != 0)) {
       if (bad) report(kb.err, bad);
       __syncwarp();
-      for (uint32_t i = lane; i < (span + 15u) >> 4; i += 32)
+      // a counted walk over corrupt data may write up to 7 bytes past `span`
+      for (uint32_t i = lane; i < (span + 8u + 15u) >> 4; i += 32)
         reinterpret_cast<uint4 *>(region_p)[i] = make_uint4(0, 0, 0, 0);
       __syncwarp();
       if (lane == 0) mbar_arrive(release);
@@ -949,7 +1004,7 @@ uint32_t slot_words_for(uint32_t max_chunk_elems) { return (max_chunk_elems + 3u
 
 // Must match the device layout: Layout<T, C>::slot_bytes per stage slot.
 size_t stage_slot_bytes(uint32_t C, uint32_t T) {
-  return (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16 + T;
+  return (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16;
 }
 
 size_t shared_bytes(uint32_t C, uint32_t T, uint32_t stage, uint32_t slot_words,
@@ -1061,8 +1116,9 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStrea
 }
 
 // Per-warp exponent region of the warp-specialised kernel: the warp's head
-// (< 16), up to 32 chunks of max_chunk_elems exponents, two words of slack
-// (a lookup ORs into the word after the one it fills).
+// (< 16), up to 32 chunks of max_chunk_elems exponents, and slack for the
+// last lookup: it touches bytes up to 6 past the warp's last element (the
+// spill word, or up to three extra exponents of a corrupt stream).
 uint32_t region_bytes_for(uint32_t max_chunk_elems) {
   return (15u + 32u * max_chunk_elems + 8u + 15u) & ~15u;
 }
@@ -1210,8 +1266,13 @@ size_t df11_shared_bytes(const df11_params *p) {
   if (!p || !supported(p->chunk_bytes, p->threads_per_block)) return 0;
   const uint32_t subs =
       p->num_luts - 1 <= (uint32_t)kSubTablesInSmem ? (p->num_luts - 1) * 256 : 0;
-  return shared_bytes(p->chunk_bytes, p->threads_per_block, stage_bytes_for(p->max_block_elems),
-                      slot_words_for(p->max_chunk_elems), subs);
+  const size_t page = shared_bytes(p->chunk_bytes, p->threads_per_block,
+                                   stage_bytes_for(p->max_block_elems),
+                                   slot_words_for(p->max_chunk_elems), subs);
+  const size_t ws = ws_shared_bytes(p->chunk_bytes, p->threads_per_block,
+                                    stage_bytes_for(p->max_block_elems),
+                                    region_bytes_for(p->max_chunk_elems), 0);
+  return page > ws ? page : ws;
 }
 
 int df11_supported(uint32_t chunk_bytes, uint32_t threads_per_block) {

@@ -150,8 +150,9 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
 df11_status df11_decode_batched(const df11_tensor *tensors, int count,
                                 int32_t *d_err, df11_stream_t stream);
 
-/* Bytes of dynamic shared memory one block of the decode kernel uses for
- * these parameters (for occupancy planning); 0 if unsupported. */
+/* Bytes of dynamic shared memory one thread block of a decode launch for
+ * these parameters may use: the larger of the two kernels' needs (with and
+ * without chunk counts), for occupancy planning; 0 if unsupported. */
 size_t df11_shared_bytes(const df11_params *params);
 
 /* 1 if the library has a kernel for this (chunk_bytes, threads_per_block). */

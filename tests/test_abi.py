@@ -98,7 +98,11 @@ def test_supported_shapes_and_shared_bytes():
     assert not df11.supported(12, 256)
     p = _params(max_block_elems=6400, num_luts=4)
     sb = df11.lib().df11_shared_bytes(ctypes.byref(p))
-    assert 25_000 < sb < 40_000  # tables + two stage slots + exponents + slots
+    # tables (16 KB derived table) + two stage slots + exponents + slots
+    assert 30_000 < sb < 60_000
+    bigger = _params(max_block_elems=12800, num_luts=4)
+    assert df11.lib().df11_shared_bytes(ctypes.byref(bigger)) > sb
+    assert df11.lib().df11_shared_bytes(ctypes.byref(_params(chunk_bytes=12))) == 0
 
 
 def test_status_strings():

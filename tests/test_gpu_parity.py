@@ -268,7 +268,9 @@ def test_corrupt_chunk_counts_are_flagged():
     d.chunk_counts[10] += 1
     d.chunk_counts[11] -= 1      # block total unchanged: caught per thread
     out, code = _decode_with_err(d)
-    assert code == 1
+    # the walk counted by chunk 11 stops short of its last bit (count error),
+    # the one counted by chunk 10 runs past it (overrun): either comes first
+    assert code in (1, 2)
     d = df11.to_device(h)
     d.chunk_counts[300] += 3     # block total changed: caught by the scan
     _, code = _decode_with_err(d)
