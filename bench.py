@@ -226,7 +226,8 @@ def barrier(world: int):
         dist.barrier()
 
 
-def prepare(config: str, seed: int, device: str):
+def prepare(config: str, seed: int, device: str, chunk_bytes: int = 8,
+            threads_per_block: int = 256):
     """Compress every unit on the host; keep compressed tensors resident in
     HBM.  Originals are regenerated from the seed when checked."""
     import huffman_decode_df11_b200 as df11
@@ -234,7 +235,7 @@ def prepare(config: str, seed: int, device: str):
     hosts, devs = [], []
     for name, thunk in units:
         bits = thunk(device)
-        h = df11.compress(bits)
+        h = df11.compress(bits, chunk_bytes=chunk_bytes, threads_per_block=threads_per_block)
         hosts.append(h)
         devs.append(df11.to_device(h, device))
         del bits
@@ -245,7 +246,8 @@ def run_b200(args, world, rank, local):
     import huffman_decode_df11_b200 as df11
     device = f"cuda:{local}"
     seed = args.seed + rank
-    units, hosts, devs = prepare(args.config, seed, device)
+    units, hosts, devs = prepare(args.config, seed, device, args.chunk_bytes,
+                                 args.threads_per_block)
     names = [u[0] for u in units]
     groups = block_groups(args.config, names)
     n_total = sum(h.n for h in hosts)
@@ -342,7 +344,7 @@ def run_b200(args, world, rank, local):
             "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
             "config": {
                 "workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
-                "elements": n_total, "chunk_bytes": 8, "threads_per_block": 256,
+                "elements": n_total, "chunk_bytes": args.chunk_bytes, "threads_per_block": args.threads_per_block,
                 "compressed_bytes": sum(h.compressed_bytes() for h in hosts),
                 "bits_per_weight": round(8.0 * sum(h.compressed_bytes() for h in hosts)
                                          / n_total, 3),
@@ -469,7 +471,8 @@ def run_reference(args, world, rank):
         return
     units = workload_units(args.config, args.seed)
     import huffman_decode_df11_b200 as df11
-    hosts = [df11.compress(thunk("cpu")) for _, thunk in units]
+    hosts = [df11.compress(thunk("cpu"), chunk_bytes=args.chunk_bytes,
+                           threads_per_block=args.threads_per_block) for _, thunk in units]
     n_total = sum(h.n for h in hosts)
     budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
     for _ in range(args.warmup):
@@ -487,7 +490,7 @@ def run_reference(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "u32",
         "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
         "config": {"workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
-                   "elements": n_total, "chunk_bytes": 8, "threads_per_block": 256,
+                   "elements": n_total, "chunk_bytes": args.chunk_bytes, "threads_per_block": args.threads_per_block,
                    "step": f"bounded sample of the workload, ~{budget:.1f} s of CPU work"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": what + " per step (single-threaded bit-serial C decode)"},
@@ -516,6 +519,10 @@ def main(argv=None):
     ap.add_argument("--config", default="block", choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--chunk-bytes", type=int, default=8, choices=[4, 8, 16],
+                    help="bitstream bytes per chunk (C) of the compressed format")
+    ap.add_argument("--threads-per-block", type=int, default=256, choices=[128, 256, 512],
+                    help="chunks per format block (T) of the compressed format")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

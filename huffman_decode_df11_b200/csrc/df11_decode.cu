@@ -42,7 +42,7 @@
 //
 // Why the rotation: with e' = e>>1 | (e&1)<<7, the high byte of a BF16 word
 // is (sm & 0x80) | (e' & 0x7F) and the low byte (e' & 0x80) | (sm & 0x7F), so
-// four output words cost two byte permutes and one bitwise select each.
+// four output words cost two bitwise selects and two byte permutes.
 //
 // Nothing here waits on another thread block, so nothing can hang: the only
 // waits are on this block's own copies, bounded, reporting
@@ -91,7 +91,8 @@ struct KBatch {
   uint32_t stage_bytes;  // bytes of the exponent array
   uint32_t slot_words;   // 32-bit words of each thread's private slot
   uint32_t sub_words;    // deeper-table words kept in shared memory (0: global)
-  uint32_t sm_bytes;     // sign/mantissa bytes per stage slot (warp-specialised kernel)
+  uint32_t sm_bytes;     // sign/mantissa bytes per stage slot (warp-specialised kernel;
+                         // 0: read from global memory)
 };
 
 // ---- shared memory layout --------------------------------------------------
@@ -447,16 +448,18 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t (&w)[C / 4 + 1
   return (pk >> 19) - d;
 }
 
-// four sign/mantissa bytes and four rotated exponents -> four BF16 words
+// four sign/mantissa bytes and four rotated exponents -> four BF16 words:
+// the four low bytes (E0 | mantissa) and the four high bytes (sign | E7..E1)
+// are two bitwise selects, then two byte permutes interleave them
 __device__ __forceinline__ uint2 fuse4(uint32_t sm4, uint32_t er4) {
-  const uint32_t p0 = __byte_perm(sm4, er4, 0x5140), q0 = __byte_perm(sm4, er4, 0x1504);
-  const uint32_t p1 = __byte_perm(sm4, er4, 0x7362), q1 = __byte_perm(sm4, er4, 0x3726);
-  return make_uint2((p0 & 0x7F7F7F7Fu) | (q0 & 0x80808080u),
-                    (p1 & 0x7F7F7F7Fu) | (q1 & 0x80808080u));
+  const uint32_t lo = (sm4 & 0x7F7F7F7Fu) | (er4 & 0x80808080u);
+  const uint32_t hi = (er4 & 0x7F7F7F7Fu) | (sm4 & 0x80808080u);
+  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
 __device__ __forceinline__ uint16_t fuse1(uint32_t sm, uint32_t er) {
-  return (uint16_t)(((sm & 0x80u) << 8) | ((er & 0x7Fu) << 8) | (er & 0x80u) | (sm & 0x7Fu));
+  const uint32_t lo = (sm & 0x7Fu) | (er & 0x80u), hi = (er & 0x7Fu) | (sm & 0x80u);
+  return (uint16_t)__byte_perm(lo, hi, 0x3340);
 }
 
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
@@ -747,7 +750,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-template <int T, int C>
+template <int T, int C, bool SMG>
 __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t *slot,
                                          uint32_t full, uint32_t sm_capacity) {
   using L = WsLayout<T, C>;
@@ -756,7 +759,7 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   // a warp's exponents fit its region whatever the block: every chunk count
   // is checked against max_chunk_elems before decoding
   const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems &&
-                  expected + 32 <= sm_capacity;
+                  (SMG || expected + 32 <= sm_capacity);
   // bits of the stream inside this block: all of them but in the last block
   const uint64_t bit0 = (uint64_t)b * (T * C * 8);
   const uint32_t valid_bits = tk.total_bits - bit0 < (uint64_t)(T * C * 8)
@@ -770,18 +773,25 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   }
   const uint32_t sm_begin = P0 & ~15u;
   const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
-  mbar_arrive_expect_tx(full, L::bits_bytes + L::gaps_bytes + L::counts_bytes + sm_bytes);
+  mbar_arrive_expect_tx(full,
+                        L::bits_bytes + L::gaps_bytes + L::counts_bytes + (SMG ? 0u : sm_bytes));
   bulk_g2s(smem_addr(slot), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, full);
   bulk_g2s(smem_addr(slot + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
            full);
   bulk_g2s(smem_addr(slot + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
            L::counts_bytes, full);
-  if (sm_bytes)
+  if (SMG) {
+    if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
+  } else if (sm_bytes) {
     bulk_g2s(smem_addr(slot + L::head_bytes), tk.sign_mantissa + sm_begin, sm_bytes, full);
+  }
 }
 
-template <int T, int C>
-__global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
+// SMG: the output reads the sign/mantissa bytes from global memory (L2-
+// prefetched by the producer) instead of the stage slot, for formats whose
+// blocks are too large to stage without losing resident thread blocks.
+template <int T, int C, bool SMG>
+__global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
     df11_decode_ws_kernel(const __grid_constant__ KBatch kb) {
   using L = WsLayout<T, C>;
   constexpr int NW = C / 4 + 1;
@@ -840,7 +850,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
           report(kb.err, DF11_DEV_ERR_TIMEOUT);
           break;
         }
-        ws_issue<T, C>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
+        ws_issue<T, C, SMG>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
       }
     }
     return;
@@ -955,14 +965,16 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
     // `out`.
     const uint32_t base = G0 & ~15u;
     uint16_t *out = tk.out + base;
-    const uint32_t sm = smem_addr(slot + L::head_bytes) + (base - (P0 & ~15u));
+    const uint8_t *smg = tk.sign_mantissa + base;  // SMG
+    const uint32_t sm = SMG ? 0u : smem_addr(slot + L::head_bytes) + (base - (P0 & ~15u));
     const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
     {
       uint32_t g = g_begin + (uint32_t)lane;
       uint32_t sa_sm = sm + 16u * g, sa_rg = region + 16u * g;
       uint4 *o = reinterpret_cast<uint4 *>(out) + 2u * g;
-      for (; g < g_end; g += 32, sa_sm += 512u, sa_rg += 512u, o += 64) {
-        const uint4 sv = lds128(sa_sm);
+      const uint4 *sp = reinterpret_cast<const uint4 *>(smg) + g;
+      for (; g < g_end; g += 32, sa_sm += 512u, sa_rg += 512u, o += 64, sp += 32) {
+        const uint4 sv = SMG ? __ldg(sp) : lds128(sa_sm);
         const uint4 rv = lds128(sa_rg);
         sts128_zero(sa_rg);  // leave the region zeroed for the next block
         const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
@@ -971,16 +983,14 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
         o[1] = make_uint4(e2.x, e2.y, f.x, f.y);
       }
     }
-    if (span) {  // lanes 0-15: first group, 16-31: last group
-      const uint32_t gl = (span - 1) >> 4;
-      const bool first_partial = head != 0 || span < 16;
-      const bool last_partial = (span & 15u) != 0 && gl != 0;
-      const uint32_t i = lane < 16 ? (uint32_t)lane : (gl << 4) + (uint32_t)(lane - 16);
-      const bool mine = lane < 16 ? first_partial : last_partial;
-      if (mine) {
-        if (i >= head && i < span) out[i] = fuse1(lds8(sm + i), lds8(region + i));
-        sts8_zero(region + i);
-      }
+    if (span) {
+      // the elements outside whole groups [g_begin, g_end), one per lane:
+      // lanes 0-15 take the first group, 16-31 the last one (the same group
+      // when there is only one: both lanes then write the same value)
+      const uint32_t i = ((uint32_t)lane & 15u) + (lane >> 4 ? ((span - 1) >> 4) << 4 : 0u);
+      if (i >= head && i < span && (i < (g_begin << 4) || i >= (g_end << 4)))
+        out[i] = fuse1(SMG ? (uint32_t)__ldg(smg + i) : lds8(sm + i), lds8(region + i));
+      sts8_zero(region + i);  // the loop zeroed whole groups; this does the rest
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(release);  // slot free for refill
@@ -1041,7 +1051,7 @@ df11_status validate(const df11_tensor &t) {
 
 struct DeviceInfo {
   int sms = 0;
-  std::atomic<size_t> configured[10];
+  std::atomic<size_t> configured[16];
 };
 
 DeviceInfo &device_info(int dev) {
@@ -1103,15 +1113,36 @@ df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t
   return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
+size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
+                       uint32_t sub_words);
+
+// Stage the blocks' sign/mantissa bytes in shared memory (one bulk copy per
+// block, 16-byte shared loads in the output) unless that costs resident
+// thread blocks; then the output reads them from global memory instead.
 template <int T, int C>
-df11_status launch_ws(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t s,
+df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
-  auto kern = df11_decode_ws_kernel<T, C>;
-  uint64_t budget = 0;
-  df11_status st = prepare(kern, T + 32, smem, instance, budget);
+  auto staged = df11_decode_ws_kernel<T, C, false>;
+  auto direct = df11_decode_ws_kernel<T, C, true>;
+  const size_t smem_st = ws_shared_bytes(C, T, sm_stage, kb.stage_bytes, kb.sub_words);
+  const size_t smem_gl = ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words);
+  if (smem_gl > 227 * 1024) return DF11_ERR_TOO_LARGE;
+  uint64_t budget_gl = 0, budget_st = 0;
+  df11_status st = prepare(direct, T + 32, smem_gl, 2 * instance + 1, budget_gl);
   if (st != DF11_OK) return st;
-  const uint32_t grid = split_grid(kb, blocks, budget);
-  kern<<<grid, T + 32, smem, s>>>(kb);
+  if (smem_st <= 227 * 1024) {
+    st = prepare(staged, T + 32, smem_st, 2 * instance, budget_st);
+    if (st != DF11_OK && st != DF11_ERR_TOO_LARGE) return st;
+  }
+  if (budget_st >= budget_gl) {
+    kb.sm_bytes = sm_stage;
+    const uint32_t grid = split_grid(kb, blocks, budget_st);
+    staged<<<grid, T + 32, smem_st, s>>>(kb);
+  } else {
+    kb.sm_bytes = 0;
+    const uint32_t grid = split_grid(kb, blocks, budget_gl);
+    direct<<<grid, T + 32, smem_gl, s>>>(kb);
+  }
   return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
@@ -1168,22 +1199,16 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   if (ws) {
     kb.stage_bytes = region_bytes_for(max_chunk);  // bytes of each warp's region
     kb.slot_words = 0;
-    kb.sm_bytes = stage_bytes_for(max_elems);
     // deeper tables only serve codewords longer than the derived table's
     // index (about one lookup in a thousand): read them from global memory
-    // and spend the shared memory on one more resident thread block
+    // and spend the shared memory on resident thread blocks
     kb.sub_words = 0;
-    size_t smem = ws_shared_bytes(C, T, kb.sm_bytes, kb.stage_bytes, kb.sub_words);
-    if (smem > 227 * 1024 && kb.sub_words) {
-      kb.sub_words = 0;
-      smem = ws_shared_bytes(C, T, kb.sm_bytes, kb.stage_bytes, 0);
-    }
-    if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
-    if (T == 256 && C == 8) return launch_ws<256, 8>(kb, blocks, smem, s, 5);
-    if (T == 256 && C == 4) return launch_ws<256, 4>(kb, blocks, smem, s, 6);
-    if (T == 256 && C == 16) return launch_ws<256, 16>(kb, blocks, smem, s, 7);
-    if (T == 128 && C == 8) return launch_ws<128, 8>(kb, blocks, smem, s, 8);
-    if (T == 512 && C == 8) return launch_ws<512, 8>(kb, blocks, smem, s, 9);
+    const uint32_t sm_stage = stage_bytes_for(max_elems);
+    if (T == 256 && C == 8) return launch_ws<256, 8>(kb, blocks, sm_stage, s, 3);
+    if (T == 256 && C == 4) return launch_ws<256, 4>(kb, blocks, sm_stage, s, 4);
+    if (T == 256 && C == 16) return launch_ws<256, 16>(kb, blocks, sm_stage, s, 5);
+    if (T == 128 && C == 8) return launch_ws<128, 8>(kb, blocks, sm_stage, s, 6);
+    if (T == 512 && C == 8) return launch_ws<512, 8>(kb, blocks, sm_stage, s, 7);
     return DF11_ERR_UNSUPPORTED;
   }
   kb.stage_bytes = stage_bytes_for(max_elems);
