@@ -30,6 +30,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 # ctypes mirror of include/df11.h
 
 DF11_MAX_BATCH = 16
+DF11_DECODE_TABLE_BYTES = 17664
 STATUS = {
     0: "DF11_OK", 1: "DF11_ERR_NULL", 2: "DF11_ERR_ALIGN", 3: "DF11_ERR_FORMAT",
     4: "DF11_ERR_UNSUPPORTED", 5: "DF11_ERR_CUDA", 6: "DF11_ERR_TOO_LARGE",
@@ -66,6 +67,7 @@ class TensorDesc(ctypes.Structure):
         ("code_lengths", ctypes.c_void_p),
         ("sign_mantissa", ctypes.c_void_p),
         ("out_bf16", ctypes.c_void_p),
+        ("decode_table", ctypes.c_void_p),
         ("params", Params),
     ]
 
@@ -123,6 +125,8 @@ def lib():
     L.df11_build.argtypes = [vp, u64, u32, u32, ctypes.c_int, ctypes.POINTER(HostTensor)]
     L.df11_build.restype = ctypes.c_int
     L.df11_host_tensor_free.argtypes = [ctypes.POINTER(HostTensor)]
+    L.df11_build_decode_table.argtypes = [vp, vp, u32, vp, vp]
+    L.df11_build_decode_table.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -229,6 +233,7 @@ class Df11Device:
     sign_mantissa: torch.Tensor
     chunk_counts: Optional[torch.Tensor] = None
     shape: tuple = ()
+    decode_table: Optional[torch.Tensor] = None  # df11_build_decode_table output
 
     @property
     def n(self) -> int:
@@ -246,10 +251,11 @@ class Df11Device:
 
     def desc(self, out: torch.Tensor, counts: bool = True) -> TensorDesc:
         cc = self.chunk_counts.data_ptr() if (counts and self.chunk_counts is not None) else None
+        dt = self.decode_table.data_ptr() if self.decode_table is not None else None
         return TensorDesc(self.bitstream.data_ptr(), self.gaps.data_ptr(), cc,
                           self.block_out_pos.data_ptr(), self.luts.data_ptr(),
                           self.code_lengths.data_ptr(), self.sign_mantissa.data_ptr(),
-                          out.data_ptr(), self.params)
+                          out.data_ptr(), dt, self.params)
 
 
 def _np_to(t: np.ndarray, device, pin: bool = False) -> torch.Tensor:
@@ -259,9 +265,11 @@ def _np_to(t: np.ndarray, device, pin: bool = False) -> torch.Tensor:
     return x.to(device, non_blocking=pin)
 
 
-def to_device(h: Df11Host, device="cuda") -> Df11Device:
-    """Copy a compressed tensor into device memory (16-byte aligned buffers)."""
-    return Df11Device(
+def to_device(h: Df11Host, device="cuda", decode_table: bool = True) -> Df11Device:
+    """Copy a compressed tensor into device memory (16-byte aligned buffers)
+    and, unless decode_table=False, derive its decode table there once
+    (df11_build_decode_table) so that decode calls need not."""
+    d = Df11Device(
         params=Params.from_buffer_copy(h.params),
         bitstream=_np_to(h.bitstream, device),
         gaps=_np_to(h.gaps, device),
@@ -272,6 +280,18 @@ def to_device(h: Df11Host, device="cuda") -> Df11Device:
         chunk_counts=_np_to(h.chunk_counts, device),
         shape=h.shape,
     )
+    if decode_table:
+        d.decode_table = build_decode_table(d)
+    return d
+
+
+def build_decode_table(d: Df11Device, stream=None) -> torch.Tensor:
+    """The decode table of a device tensor (df11_build_decode_table)."""
+    t = torch.empty(DF11_DECODE_TABLE_BYTES, dtype=torch.uint8, device=d.device)
+    _check(lib().df11_build_decode_table(d.luts.data_ptr(), d.code_lengths.data_ptr(),
+                                         int(d.params.num_luts), t.data_ptr(),
+                                         _stream_handle(stream)), "df11_build_decode_table")
+    return t
 
 
 def _stream_handle(stream) -> Optional[int]:

@@ -72,6 +72,7 @@ struct KTensor {
   const uint8_t *code_lengths;
   const uint8_t *sign_mantissa;
   uint16_t *out;
+  const void *decode_table;  // NULL: derived by every thread block
   uint64_t total_bits;
   uint32_t n;
   uint32_t num_blocks;
@@ -113,6 +114,9 @@ constexpr uint32_t kOffLut0 = 560;
 constexpr uint32_t kOffWide = 1584;
 constexpr uint32_t kWideBytes = 8u << kWideBits;
 constexpr uint32_t kOffStages = kOffWide + kWideBytes;
+// a decode table (df11_build_decode_table) is the image of [kOffLens, kOffStages)
+static_assert(kOffStages - kOffLens == DF11_DECODE_TABLE_BYTES, "decode table layout");
+static_assert(kOffLut0 - kOffLens == 256 && kOffWide - kOffLut0 == 1024, "decode table layout");
 
 template <int T, int C>
 struct Layout {
@@ -231,6 +235,20 @@ __device__ __forceinline__ bool decode_one(uint32_t win, const uint32_t *__restr
   }
   len = lens[sym];
   return len != 0;
+}
+
+// Table 0 of the format and the code lengths into shared memory, every
+// exponent byte rotated right by one bit (code lengths indexed by the
+// rotated exponent).
+__device__ __forceinline__ void load_tables(int tid, int nthreads, const uint32_t *luts,
+                                            const uint8_t *code_lengths, uint32_t *lut0_s,
+                                            uint8_t *lens_s) {
+  for (int i = tid; i < 256; i += nthreads) {
+    uint32_t e = luts[i] & 0x3FFFFFFFu;
+    if ((e >> 24) & 15u) e = (e & 0xFF000000u) | rot8x3(e);
+    lut0_s[i] = e;
+    lens_s[((uint32_t)i >> 1) | (((uint32_t)i & 1u) << 7)] = code_lengths[i];
+  }
 }
 
 // Derived table: entry i holds the codewords that lie wholly inside the WB
@@ -533,12 +551,7 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
 
   // tables (once per thread block): table 0 and lengths rotated, deeper
   // tables verbatim, then the derived wide table
-  for (int i = tid; i < 256; i += T) {
-    uint32_t e = tk.luts[i] & 0x3FFFFFFFu;
-    if ((e >> 24) & 15u) e = (e & 0xFF000000u) | rot8x3(e);
-    lut0_s[i] = e;
-    lens_s[((uint32_t)i >> 1) | (((uint32_t)i & 1u) << 7)] = tk.code_lengths[i];
-  }
+  load_tables(tid, T, tk.luts, tk.code_lengths, lut0_s, lens_s);
   const uint32_t *sub = tk.luts + 256;
   const uint32_t sub_words = (tk.num_luts - 1) * 256;
   if (sub_words && sub_words <= kb.sub_words) {
@@ -735,6 +748,14 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
 //     lane; then releases the slot.
 constexpr int kWsStages = 2;
 
+// Where the output of the warp-specialised kernel finds a block's sign/
+// mantissa bytes: in the stage slot (one bulk copy per block by the
+// producer), in global memory (L2-prefetched by the producer), or in a
+// buffer of the warp's own, filled by one bulk copy of the warp's output
+// range that the warp issues before it decodes.  The host takes the first
+// that keeps the most thread blocks resident.
+enum SmMode { kSmSlot = 0, kSmGlobal = 1, kSmWarp = 2 };
+
 template <int T, int C>
 struct WsLayout {
   static constexpr uint32_t bits_bytes = T * C + 16;
@@ -750,7 +771,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-template <int T, int C, bool SMG>
+template <int T, int C, int SM>
 __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t *slot,
                                          uint32_t full, uint32_t sm_capacity) {
   using L = WsLayout<T, C>;
@@ -759,7 +780,7 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   // a warp's exponents fit its region whatever the block: every chunk count
   // is checked against max_chunk_elems before decoding
   const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems &&
-                  (SMG || expected + 32 <= sm_capacity);
+                  (SM != kSmSlot || expected + 32 <= sm_capacity);
   // bits of the stream inside this block: all of them but in the last block
   const uint64_t bit0 = (uint64_t)b * (T * C * 8);
   const uint32_t valid_bits = tk.total_bits - bit0 < (uint64_t)(T * C * 8)
@@ -773,25 +794,22 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   }
   const uint32_t sm_begin = P0 & ~15u;
   const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
-  mbar_arrive_expect_tx(full,
-                        L::bits_bytes + L::gaps_bytes + L::counts_bytes + (SMG ? 0u : sm_bytes));
+  mbar_arrive_expect_tx(full, L::bits_bytes + L::gaps_bytes + L::counts_bytes +
+                                  (SM == kSmSlot ? sm_bytes : 0u));
   bulk_g2s(smem_addr(slot), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, full);
   bulk_g2s(smem_addr(slot + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
            full);
   bulk_g2s(smem_addr(slot + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
            L::counts_bytes, full);
-  if (SMG) {
+  if (SM == kSmGlobal) {
     if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
-  } else if (sm_bytes) {
+  } else if (SM == kSmSlot && sm_bytes) {
     bulk_g2s(smem_addr(slot + L::head_bytes), tk.sign_mantissa + sm_begin, sm_bytes, full);
   }
 }
 
-// SMG: the output reads the sign/mantissa bytes from global memory (L2-
-// prefetched by the producer) instead of the stage slot, for formats whose
-// blocks are too large to stage without losing resident thread blocks.
-template <int T, int C, bool SMG>
-__global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
+template <int T, int C, int SM>
+__global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
     df11_decode_ws_kernel(const __grid_constant__ KBatch kb) {
   using L = WsLayout<T, C>;
   constexpr int NW = C / 4 + 1;
@@ -804,7 +822,8 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
   uint8_t *stages = smem + kOffStages;
   const uint32_t slot_bytes = L::head_bytes + kb.sm_bytes;
   uint8_t *regions = stages + kWsStages * slot_bytes;
-  uint32_t *sub_s = reinterpret_cast<uint32_t *>(regions + CONSUMERS * kb.stage_bytes);
+  // kSmWarp: each warp's sign/mantissa buffer (region-sized) follows the regions
+  uint8_t *warp_sm = regions + CONSUMERS * kb.stage_bytes;
 
   int ti = 0;
   for (int i = 1; i < kb.count; ++i)
@@ -815,42 +834,58 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (first >= tk.num_blocks) return;
 
+  // barriers: full[S], empty[S], per-warp (kSmWarp), tables
+  const uint32_t tbar = smem_addr(&bars[2 * kWsStages + 16]);
   if (tid == 0) {
     for (int i = 0; i < kWsStages; ++i) {
       mbar_init(smem_addr(&bars[i]), 1);
       mbar_init(smem_addr(&bars[kWsStages + i]), CONSUMERS);
     }
+    if (SM == kSmWarp)
+      for (int i = 0; i < CONSUMERS; ++i) mbar_init(smem_addr(&bars[2 * kWsStages + i]), 1);
+    mbar_init(tbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // tables, as in the other kernel
-  for (int i = tid; i < 256; i += T + 32) {
-    uint32_t e = tk.luts[i] & 0x3FFFFFFFu;
-    if ((e >> 24) & 15u) e = (e & 0xFF000000u) | rot8x3(e);
-    lut0_s[i] = e;
-    lens_s[((uint32_t)i >> 1) | (((uint32_t)i & 1u) << 7)] = tk.code_lengths[i];
+  __syncthreads();
+  // the producer queues the decode table and the first blocks before
+  // anything else, so that they arrive while the tables are set up
+  const bool have_table = tk.decode_table != nullptr;
+  uint32_t issued = 0;
+  if (warp == CONSUMERS && lane == 0) {
+    if (have_table) {
+      mbar_arrive_expect_tx(tbar, DF11_DECODE_TABLE_BYTES);
+      bulk_g2s(smem_addr(lens_s), tk.decode_table, DF11_DECODE_TABLE_BYTES, tbar);
+    }
+    for (uint32_t b = first; b < tk.num_blocks && issued < kWsStages; b += ctas, ++issued)
+      ws_issue<T, C, SM>(tk, b, stages + issued * slot_bytes, smem_addr(&bars[issued]),
+                         kb.sm_bytes);
   }
-  const uint32_t *sub = tk.luts + 256;
-  const uint32_t sub_words = (tk.num_luts - 1) * 256;
-  if (sub_words && sub_words <= kb.sub_words) {
-    for (uint32_t i = tid; i < sub_words; i += T + 32) sub_s[i] = sub[i];
-    sub = sub_s;
-  }
+  const uint32_t *sub = tk.luts + 256;  // deeper tables: global memory
   for (uint32_t i = tid; i < CONSUMERS * kb.stage_bytes / 16; i += T + 32)
     reinterpret_cast<uint4 *>(regions)[i] = make_uint4(0, 0, 0, 0);
-  __syncthreads();
-  build_wide<T + 32>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
-  __syncthreads();
+  bool tables_ok = true;
+  if (have_table) {
+    tables_ok = mbar_wait(tbar, 0);
+  } else {
+    load_tables(tid, T + 32, tk.luts, tk.code_lengths, lut0_s, lens_s);
+    __syncthreads();
+    build_wide<T + 32>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
+  }
+  if (!__syncthreads_and(tables_ok)) {
+    if (tid == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
+    return;
+  }
 
   if (warp == CONSUMERS) {  // producer
     if (lane == 0) {
-      uint32_t k = 0;
-      for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
+      uint32_t k = issued;
+      for (uint32_t b = first + issued * ctas; b < tk.num_blocks; b += ctas, ++k) {
         const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
         if (!mbar_wait(smem_addr(&bars[kWsStages + s]), par ^ 1u)) {
           report(kb.err, DF11_DEV_ERR_TIMEOUT);
           break;
         }
-        ws_issue<T, C, SMG>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
+        ws_issue<T, C, SM>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
       }
     }
     return;
@@ -859,6 +894,9 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
   const uint32_t region = smem_addr(regions + warp * kb.stage_bytes);
   uint8_t *region_p = regions + warp * kb.stage_bytes;
   const uint32_t wide = smem_addr(wide_s);
+  const uint32_t wsm = smem_addr(warp_sm + warp * kb.stage_bytes);  // kSmWarp
+  const uint32_t wbar = smem_addr(&bars[2 * kWsStages + warp]);     // kSmWarp
+  uint32_t wph = 0;  // kSmWarp: copies issued so far (phase parity)
   uint32_t k = 0;
   for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
     const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
@@ -936,6 +974,14 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
     const uint32_t G0 = P0 + before;            // first element of this warp
     const uint32_t head = G0 & 15u, span = head + warp_total;
     const uint32_t d = head + incl - cnt;       // my first byte in the region
+    // kSmWarp: the warp's sign/mantissa bytes, elements [G0 & ~15,
+    // round16(G0 + warp_total)), inside the block's range, copied while it
+    // decodes; every path below waits for the copy before going on
+    const uint32_t wsm_bytes = SM == kSmWarp ? (span + 15u) & ~15u : 0u;
+    if (SM == kSmWarp && wsm_bytes && lane == 0) {
+      mbar_arrive_expect_tx(wbar, wsm_bytes);
+      bulk_g2s(wsm, tk.sign_mantissa + (G0 & ~15u), wsm_bytes, wbar);
+    }
     int bad = 0;
     uint32_t got;
     if (tk.masked) {
@@ -947,6 +993,14 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
                                        region, d, limit, bad);
     }
     if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
+    if (SM == kSmWarp && wsm_bytes) {
+      const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(wbar, wph & 1u));
+      ++wph;
+      if (!landed) {
+        if (lane == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
+        return;  // whole warp; the buffer may still be written
+      }
+    }
     if (__any_sync(0xFFFFFFFFu, bad != 0)) {
       if (bad) report(kb.err, bad);
       __syncwarp();
@@ -965,8 +1019,10 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
     // `out`.
     const uint32_t base = G0 & ~15u;
     uint16_t *out = tk.out + base;
-    const uint8_t *smg = tk.sign_mantissa + base;  // SMG
-    const uint32_t sm = SMG ? 0u : smem_addr(slot + L::head_bytes) + (base - (P0 & ~15u));
+    const uint8_t *smg = tk.sign_mantissa + base;  // kSmGlobal
+    const uint32_t sm = SM == kSmWarp   ? wsm
+                        : SM == kSmSlot ? smem_addr(slot + L::head_bytes) + (base - (P0 & ~15u))
+                                        : 0u;
     const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
     {
       uint32_t g = g_begin + (uint32_t)lane;
@@ -974,7 +1030,7 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
       uint4 *o = reinterpret_cast<uint4 *>(out) + 2u * g;
       const uint4 *sp = reinterpret_cast<const uint4 *>(smg) + g;
       for (; g < g_end; g += 32, sa_sm += 512u, sa_rg += 512u, o += 64, sp += 32) {
-        const uint4 sv = SMG ? __ldg(sp) : lds128(sa_sm);
+        const uint4 sv = SM == kSmGlobal ? __ldg(sp) : lds128(sa_sm);
         const uint4 rv = lds128(sa_rg);
         sts128_zero(sa_rg);  // leave the region zeroed for the next block
         const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
@@ -989,12 +1045,32 @@ __global__ void __launch_bounds__(T + 32, T == 128 ? 8 : (T == 256 ? 5 : 3))
       // when there is only one: both lanes then write the same value)
       const uint32_t i = ((uint32_t)lane & 15u) + (lane >> 4 ? ((span - 1) >> 4) << 4 : 0u);
       if (i >= head && i < span && (i < (g_begin << 4) || i >= (g_end << 4)))
-        out[i] = fuse1(SMG ? (uint32_t)__ldg(smg + i) : lds8(sm + i), lds8(region + i));
+        out[i] = fuse1(SM == kSmGlobal ? (uint32_t)__ldg(smg + i) : lds8(sm + i),
+                       lds8(region + i));
       sts8_zero(region + i);  // the loop zeroed whole groups; this does the rest
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(release);  // slot free for refill
   }
+}
+
+// ---------------------------------------------------------------------------
+// The decode table of one tensor (df11_build_decode_table): the shared-memory
+// image of table 0, the code lengths and the derived table, as the decode
+// kernels set them up, written to global memory once.
+__global__ void __launch_bounds__(256) df11_table_kernel(const uint32_t *luts,
+                                                         const uint8_t *code_lengths,
+                                                         uint32_t num_luts, uint4 *out) {
+  __shared__ __align__(16) uint8_t t[DF11_DECODE_TABLE_BYTES];
+  uint8_t *lens_s = t;
+  uint32_t *lut0_s = reinterpret_cast<uint32_t *>(t + (kOffLut0 - kOffLens));
+  uint2 *wide_s = reinterpret_cast<uint2 *>(t + (kOffWide - kOffLens));
+  load_tables(threadIdx.x, 256, luts, code_lengths, lut0_s, lens_s);
+  __syncthreads();
+  build_wide<256>(wide_s, lut0_s, lens_s, luts + 256, num_luts);
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < DF11_DECODE_TABLE_BYTES / 16; i += 256)
+    out[i] = reinterpret_cast<const uint4 *>(t)[i];
 }
 
 // ---------------------------------------------------------------------------
@@ -1033,7 +1109,7 @@ df11_status validate(const df11_tensor &t) {
       !t.sign_mantissa || !t.out_bf16)
     return DF11_ERR_NULL;
   if (!aligned(t.bitstream, 16) || !aligned(t.gaps, 16) || !aligned(t.luts, 16) ||
-      !aligned(t.chunk_counts, 16) ||
+      !aligned(t.chunk_counts, 16) || !aligned(t.decode_table, 16) ||
       !aligned(t.sign_mantissa, 16) || !aligned(t.out_bf16, 16) || !aligned(t.block_out_pos, 4))
     return DF11_ERR_ALIGN;
   if (!supported(p.chunk_bytes, p.threads_per_block)) return DF11_ERR_UNSUPPORTED;
@@ -1051,7 +1127,7 @@ df11_status validate(const df11_tensor &t) {
 
 struct DeviceInfo {
   int sms = 0;
-  std::atomic<size_t> configured[16];
+  std::atomic<size_t> configured[32];
 };
 
 DeviceInfo &device_info(int dev) {
@@ -1114,35 +1190,38 @@ df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t
 }
 
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
-                       uint32_t sub_words);
+                       uint32_t sub_words, bool warp_sm);
 
-// Stage the blocks' sign/mantissa bytes in shared memory (one bulk copy per
-// block, 16-byte shared loads in the output) unless that costs resident
-// thread blocks; then the output reads them from global memory instead.
+// Sign/mantissa bytes staged per block in the stage slot, per warp in the
+// warp's own buffer, or read from global memory: the first of these that
+// keeps the most thread blocks resident (16-byte shared loads in the output
+// beat L2 loads at equal residency).
 template <int T, int C>
 df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
-  auto staged = df11_decode_ws_kernel<T, C, false>;
-  auto direct = df11_decode_ws_kernel<T, C, true>;
-  const size_t smem_st = ws_shared_bytes(C, T, sm_stage, kb.stage_bytes, kb.sub_words);
-  const size_t smem_gl = ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words);
-  if (smem_gl > 227 * 1024) return DF11_ERR_TOO_LARGE;
-  uint64_t budget_gl = 0, budget_st = 0;
-  df11_status st = prepare(direct, T + 32, smem_gl, 2 * instance + 1, budget_gl);
-  if (st != DF11_OK) return st;
-  if (smem_st <= 227 * 1024) {
-    st = prepare(staged, T + 32, smem_st, 2 * instance, budget_st);
+  void (*kern[3])(KBatch) = {df11_decode_ws_kernel<T, C, kSmSlot>,
+                             df11_decode_ws_kernel<T, C, kSmGlobal>,
+                             df11_decode_ws_kernel<T, C, kSmWarp>};
+  const size_t smem[3] = {ws_shared_bytes(C, T, sm_stage, kb.stage_bytes, kb.sub_words, false),
+                          ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, false),
+                          ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, true)};
+  const int order[3] = {kSmSlot, kSmWarp, kSmGlobal};
+  uint64_t best = 0;
+  int pick = -1;
+  for (int m : order) {
+    if (smem[m] > 227 * 1024) continue;
+    uint64_t budget = 0;
+    const df11_status st = prepare(kern[m], T + 32, smem[m], 3 * instance + m, budget);
     if (st != DF11_OK && st != DF11_ERR_TOO_LARGE) return st;
+    if (budget > best) {
+      best = budget;
+      pick = m;
+    }
   }
-  if (budget_st >= budget_gl) {
-    kb.sm_bytes = sm_stage;
-    const uint32_t grid = split_grid(kb, blocks, budget_st);
-    staged<<<grid, T + 32, smem_st, s>>>(kb);
-  } else {
-    kb.sm_bytes = 0;
-    const uint32_t grid = split_grid(kb, blocks, budget_gl);
-    direct<<<grid, T + 32, smem_gl, s>>>(kb);
-  }
+  if (pick < 0) return DF11_ERR_TOO_LARGE;
+  kb.sm_bytes = pick == kSmSlot ? sm_stage : 0u;
+  const uint32_t grid = split_grid(kb, blocks, best);
+  kern[pick]<<<grid, T + 32, smem[pick], s>>>(kb);
   return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
@@ -1155,9 +1234,9 @@ uint32_t region_bytes_for(uint32_t max_chunk_elems) {
 }
 
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
-                       uint32_t sub_words) {
+                       uint32_t sub_words, bool warp_sm) {
   const size_t slot = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16 + T + 16 + sm_bytes;
-  return (size_t)kOffStages + kWsStages * slot + (size_t)(T / 32) * region +
+  return (size_t)kOffStages + kWsStages * slot + (size_t)(T / 32) * region * (warp_sm ? 2 : 1) +
          (size_t)sub_words * 4;
 }
 
@@ -1179,6 +1258,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     k.code_lengths = ts[i].code_lengths;
     k.sign_mantissa = ts[i].sign_mantissa;
     k.out = ts[i].out_bf16;
+    k.decode_table = ts[i].decode_table;
     k.total_bits = p.total_bits;
     k.n = (uint32_t)p.n;
     k.num_blocks = p.num_blocks;
@@ -1255,7 +1335,7 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
   if (params->n != n) return DF11_ERR_INVALID;
   if (d_err && !aligned(d_err, 4)) return DF11_ERR_ALIGN;
   df11_tensor t{bitstream, gaps, nullptr, block_out_pos, luts, code_lengths, sign_mantissa,
-                out_bf16, *params};
+                out_bf16, nullptr, *params};
   df11_status st = validate(t);
   if (st != DF11_OK || n == 0) return st;
   return launch_batch(&t, 1, d_err, (cudaStream_t)stream);
@@ -1287,6 +1367,16 @@ df11_status df11_decode_batched(const df11_tensor *tensors, int count, int32_t *
   return DF11_OK;
 }
 
+df11_status df11_build_decode_table(const uint32_t *luts, const uint8_t *code_lengths,
+                                    uint32_t num_luts, void *out, df11_stream_t stream) {
+  if (!luts || !code_lengths || !out) return DF11_ERR_NULL;
+  if (!aligned(luts, 16) || !aligned(out, 16)) return DF11_ERR_ALIGN;
+  if (num_luts < 1 || num_luts >= (1u << 24)) return DF11_ERR_FORMAT;
+  df11_table_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(luts, code_lengths, num_luts,
+                                                           reinterpret_cast<uint4 *>(out));
+  return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
 size_t df11_shared_bytes(const df11_params *p) {
   if (!p || !supported(p->chunk_bytes, p->threads_per_block)) return 0;
   const uint32_t subs =
@@ -1296,7 +1386,7 @@ size_t df11_shared_bytes(const df11_params *p) {
                                    slot_words_for(p->max_chunk_elems), subs);
   const size_t ws = ws_shared_bytes(p->chunk_bytes, p->threads_per_block,
                                     stage_bytes_for(p->max_block_elems),
-                                    region_bytes_for(p->max_chunk_elems), 0);
+                                    region_bytes_for(p->max_chunk_elems), 0, false);
   return page > ws ? page : ws;
 }
 

@@ -109,6 +109,9 @@ typedef struct df11_params {
   uint32_t reserved;          /* 0 */
 } df11_params;
 
+/* Bytes of the decode table that df11_build_decode_table writes. */
+#define DF11_DECODE_TABLE_BYTES 17664
+
 /* One tensor to decode: device pointers plus its parameters. */
 typedef struct df11_tensor {
   const uint8_t *bitstream;      /* 16-byte aligned */
@@ -119,6 +122,10 @@ typedef struct df11_tensor {
   const uint8_t *code_lengths;   /* any alignment */
   const uint8_t *sign_mantissa;  /* 16-byte aligned */
   uint16_t *out_bf16;            /* 16-byte aligned, n elements, caller-owned */
+  const void *decode_table;      /* 16-byte aligned, DF11_DECODE_TABLE_BYTES
+                                    written by df11_build_decode_table from
+                                    this tensor's luts and code_lengths; or
+                                    NULL: every thread block derives it */
   df11_params params;
 } df11_tensor;
 
@@ -149,6 +156,22 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
  */
 df11_status df11_decode_batched(const df11_tensor *tensors, int count,
                                 int32_t *d_err, df11_stream_t stream);
+
+/*
+ * Derive, on the device, the decode table of one tensor from its luts and
+ * code_lengths (device pointers, as in df11_tensor) into `out` (device,
+ * 16-byte aligned, DF11_DECODE_TABLE_BYTES, caller-owned).  The table is an
+ * acceleration structure of this library (no counterpart in the format the
+ * pages describe): the format's first table and code lengths with every
+ * exponent byte rotated right by one bit, and a table of 2^11 entries each
+ * holding the codewords that lie wholly inside an 11-bit window.  Passing it
+ * in df11_tensor.decode_table saves every thread block of every decode call
+ * from deriving it.  Asynchronous on `stream`; DF11_ERR_NULL / _ALIGN /
+ * _FORMAT (num_luts outside 1 .. 2^24-1) are returned before anything is
+ * queued.
+ */
+df11_status df11_build_decode_table(const uint32_t *luts, const uint8_t *code_lengths,
+                                    uint32_t num_luts, void *out, df11_stream_t stream);
 
 /* Bytes of dynamic shared memory one thread block of a decode launch for
  * these parameters may use: the larger of the two kernels' needs (with and

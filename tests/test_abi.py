@@ -40,7 +40,7 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layouts_match_header():
     assert ctypes.sizeof(df11.Params) == 48
-    assert ctypes.sizeof(df11.TensorDesc) == 8 * 8 + 48
+    assert ctypes.sizeof(df11.TensorDesc) == 9 * 8 + 48
 
 
 def _params(**kw):
@@ -85,11 +85,23 @@ def test_batched_host_validation():
     assert L.df11_decode_batched(None, 0, None, None) == 0
     assert L.df11_decode_batched(None, -1, None, None) == 7
     assert L.df11_decode_batched(None, 1, None, None) == 1
-    a = df11.TensorDesc(*[FAKE] * 8, _params())
-    b = df11.TensorDesc(*[FAKE] * 8, _params(chunk_bytes=4, total_bits=2600,
-                                                num_blocks=1, max_chunk_elems=30))
+    a = df11.TensorDesc(*[FAKE] * 8, None, _params())
+    b = df11.TensorDesc(*[FAKE] * 8, None, _params(chunk_bytes=4, total_bits=2600,
+                                                      num_blocks=1, max_chunk_elems=30))
     arr = (df11.TensorDesc * 2)(a, b)
     assert L.df11_decode_batched(arr, 2, None, None) == 7  # mixed (C, T)
+    c = df11.TensorDesc(*[FAKE] * 8, FAKE + 8, _params())  # misaligned decode table
+    assert L.df11_decode_batched(ctypes.byref(c), 1, None, None) == 2
+
+
+def test_decode_table_host_validation():
+    L = df11.lib()
+    assert L.df11_build_decode_table(None, FAKE, 1, FAKE, None) == 1
+    assert L.df11_build_decode_table(FAKE, FAKE, 1, None, None) == 1
+    assert L.df11_build_decode_table(FAKE + 4, FAKE, 1, FAKE, None) == 2
+    assert L.df11_build_decode_table(FAKE, FAKE, 1, FAKE + 8, None) == 2
+    assert L.df11_build_decode_table(FAKE, FAKE, 0, FAKE, None) == 3
+    assert L.df11_build_decode_table(FAKE, FAKE, 1 << 24, FAKE, None) == 3
 
 
 def test_supported_shapes_and_shared_bytes():

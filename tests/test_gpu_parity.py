@@ -25,8 +25,8 @@ def _cuda():
     torch.cuda.init()
 
 
-def _decode(h, stream=None, counts=True):
-    d = df11.to_device(h, "cuda")
+def _decode(h, stream=None, counts=True, table=True):
+    d = df11.to_device(h, "cuda", decode_table=table)
     err = df11.new_error_word()
     out = df11.decode(d, err=err, stream=stream, counts=counts)
     torch.cuda.synchronize()
@@ -37,9 +37,9 @@ def _decode(h, stream=None, counts=True):
 COUNTS = pytest.mark.parametrize("counts", [True, False], ids=["counts", "no_counts"])
 
 
-def _gpu_vs_oracle_full(w_np, C=8, T=256, counts=True):
+def _gpu_vs_oracle_full(w_np, C=8, T=256, counts=True, table=True):
     h = df11.compress(w_np, C, T)
-    out = _decode(h, counts=counts).view(torch.int16).cpu().numpy().view(np.uint16)
+    out = _decode(h, counts=counts, table=table).view(torch.int16).cpu().numpy().view(np.uint16)
     ref, end, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, h.n)
     assert end == h.params.total_bits
     assert np.array_equal(out, ref)       # GPU == oracle, element by element
@@ -48,6 +48,47 @@ def _gpu_vs_oracle_full(w_np, C=8, T=256, counts=True):
 
 
 # --- oracle-sized cases, compared in full ---------------------------------
+
+@pytest.mark.parametrize("case", ["gaussian", "adversarial", "fibonacci", "patterns", "few"])
+@pytest.mark.parametrize("C", [8, 16])
+def test_without_decode_table(case, C):
+    """Every thread block derives the decode table itself (no
+    df11_build_decode_table): same output as with it."""
+    if case == "gaussian":
+        w = workloads.as_numpy_u16(workloads.gaussian_bf16(1_000_003, 0.02, 7))
+    elif case == "adversarial":
+        w = workloads.as_numpy_u16(workloads.adversarial_mix(1 << 20, 3))
+    elif case == "fibonacci":
+        w = workloads.as_numpy_u16(workloads.fibonacci_exponents(1, symbols=26))
+    elif case == "patterns":
+        w = np.random.default_rng(1).permutation(
+            workloads.as_numpy_u16(workloads.all_bf16_patterns()))
+    else:  # three exponents: codewords of at most 2 bits (unmasked walk)
+        rng = np.random.default_rng(2)
+        w = ((rng.integers(120, 123, 200_001) << 7) | rng.integers(0, 128, 200_001)).astype(np.uint16)
+    _gpu_vs_oracle_full(w, C=C, table=False)
+    _gpu_vs_oracle_full(w, C=C, table=True)
+
+
+def test_decode_table_holds_the_rotated_format_tables():
+    """The first 1280 bytes of the decode table are the code lengths indexed
+    by rotated exponent and table 0 with rotated exponent bytes."""
+    w = workloads.as_numpy_u16(workloads.adversarial_mix(1 << 18, 4))
+    h = df11.compress(w)
+    d = df11.to_device(h, "cuda")
+    t = d.decode_table.cpu().numpy()
+    assert t.size == df11.DF11_DECODE_TABLE_BYTES
+    rot = lambda e: ((e >> 1) | ((e & 1) << 7)) & 0xFF
+    lens = np.zeros(256, np.uint8)
+    for e in range(256):
+        lens[rot(e)] = h.code_lengths[e]
+    assert np.array_equal(t[:256], lens)
+    lut0 = t[256:1280].view(np.uint32)
+    for i, e in enumerate(h.luts[:256]):
+        e = int(e) & 0x3FFFFFFF
+        if (e >> 24) & 15:
+            e = (e & 0xFF000000) | rot(e & 0xFF) | (rot((e >> 8) & 0xFF) << 8) | (rot((e >> 16) & 0xFF) << 16)
+        assert int(lut0[i]) == e
 
 @COUNTS
 @pytest.mark.parametrize("C,T", [(8, 256), (4, 256), (16, 256), (8, 128), (8, 512)])
@@ -248,17 +289,33 @@ def test_corrupt_block_positions_are_flagged(counts):
 
 
 @COUNTS
-def test_corrupt_tables_are_flagged(counts):
+@pytest.mark.parametrize("table", [True, False], ids=["table", "no_table"])
+def test_corrupt_tables_are_flagged(counts, table):
+    # the decode table is derived from the format's tables: corrupt those,
+    # then derive it again (or let every thread block derive it)
     w = workloads.adversarial_mix(1 << 20, 2)
     h = df11.compress(w)
-    d = df11.to_device(h)
+    d = df11.to_device(h, decode_table=False)
     d.luts[: 256].zero_()      # every level-0 entry invalid
+    if table:
+        d.decode_table = df11.build_decode_table(d)
     _, code = _decode_with_err(d, counts)
     assert code == 3
-    d = df11.to_device(h)
+    d = df11.to_device(h, decode_table=False)
     d.code_lengths.zero_()     # no codeword can be consumed on the slow path
+    if table:
+        d.decode_table = df11.build_decode_table(d)
     _, code = _decode_with_err(d, counts)
     assert code in (1, 2, 3)
+
+
+def test_corrupt_decode_table_is_flagged():
+    w = workloads.adversarial_mix(1 << 20, 5)
+    h = df11.compress(w)
+    d = df11.to_device(h)
+    d.decode_table.zero_()     # no codeword resolves
+    _, code = _decode_with_err(d, True)
+    assert code == 3
 
 
 def test_corrupt_chunk_counts_are_flagged():
