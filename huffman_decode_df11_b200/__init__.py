@@ -348,6 +348,34 @@ def decode_batched(ds: Sequence[Df11Device], outs: Sequence[torch.Tensor],
     return outs
 
 
+class DecodePlan:
+    """A decode of fixed compressed tensors into fixed outputs (one layer's
+    weights into its scratch buffers, say), prepared once: the descriptor
+    array is built here, and every run() is one library call (one launch per
+    16 tensors), as a layer-by-layer decode loop wants."""
+
+    def __init__(self, ds: Sequence[Df11Device], outs: Sequence[torch.Tensor],
+                 counts: bool = True):
+        if len(ds) != len(outs):
+            raise ValueError("one output per tensor")
+        for d, o in zip(ds, outs):
+            _check_out(d, o)
+        self._keep = (list(ds), list(outs))  # the buffers the descriptors point to
+        self._n = len(ds)
+        self._arr = (TensorDesc * max(self._n, 1))(*[d.desc(o, counts) for d, o in zip(ds, outs)])
+        self._lib = lib()
+
+    @property
+    def outs(self):
+        return self._keep[1]
+
+    def run(self, err: Optional[torch.Tensor] = None, stream=None):
+        _check(self._lib.df11_decode_batched(self._arr, self._n,
+                                             err.data_ptr() if err is not None else None,
+                                             _stream_handle(stream)), "df11_decode_batched")
+        return self._keep[1]
+
+
 def new_error_word(device="cuda") -> torch.Tensor:
     return torch.zeros(1, dtype=torch.int32, device=device)
 

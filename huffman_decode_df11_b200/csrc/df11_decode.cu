@@ -51,6 +51,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstdlib>
 #include <cstdint>
 
 #include "df11.h"
@@ -175,6 +176,22 @@ __device__ __forceinline__ void sts8_zero(uint32_t a) {
 __device__ __forceinline__ void red_or32(uint32_t a, uint32_t v) {
   asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
+
+// Programmatic dependent launch: a launch of this library may start while
+// the previous kernel in the stream is still running.  Each thread block
+// lets the next launch start once it has queued its last block
+// (launch_dependents; the next grid starts when every block has, so its
+// thread blocks take the places of this grid's as they finish, and set up
+// their tables and first blocks meanwhile), and waits for the previous grid
+// to finish, and its writes to be visible, only before its first store to
+// the output (wait): the output buffer may be one that the previous kernel
+// wrote or still reads, while the compressed inputs are read-only.  Letting
+// the next grid start at once measured slower on sequences of different
+// launches.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -533,6 +550,7 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
   const uint32_t first = blockIdx.x - tk.cta_begin;
   const int tid = threadIdx.x;
   if (first >= tk.num_blocks) return;  // uniform: never issued anything
+  bool waited = false;  // for the previous grid (programmatic dependent launch)
 
   const uint32_t bar0 = smem_addr(&mbar[0]), bar1 = smem_addr(&mbar[1]);
   uint32_t nP0 = 0, nP1 = 0;  // thread 0: positions of the next block to issue
@@ -580,6 +598,7 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
         nP1 = tk.block_out_pos[nb + 1];
       }
     }
+    if (tid == 0 && b + ctas >= tk.num_blocks) pdl_launch_dependents();  // last block
     int bad = 0;
     if (!mbar_wait(s ? bar1 : bar0, (k >> 1) & 1)) bad = DF11_DEV_ERR_TIMEOUT;
     const uint4 m = meta[s];
@@ -695,6 +714,10 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
 
     // output: fuse and store, 16 elements per thread per step; the ragged
     // first and last groups one element per lane
+    if (!waited) {
+      pdl_wait();
+      waited = true;
+    }
     {
       const uint32_t sm_begin = P0 & ~15u;
       uint16_t *out = tk.out + sm_begin;
@@ -887,6 +910,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
         }
         ws_issue<T, C, SM>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
       }
+      pdl_launch_dependents();  // every block of this thread block is queued
     }
     return;
   }
@@ -897,6 +921,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
   const uint32_t wsm = smem_addr(warp_sm + warp * kb.stage_bytes);  // kSmWarp
   const uint32_t wbar = smem_addr(&bars[2 * kWsStages + warp]);     // kSmWarp
   uint32_t wph = 0;  // kSmWarp: copies issued so far (phase parity)
+  bool waited = false;  // for the previous grid (programmatic dependent launch)
   uint32_t k = 0;
   for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
     const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
@@ -1012,6 +1037,10 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
       continue;
     }
     __syncwarp();
+    if (!waited) {
+      pdl_wait();
+      waited = true;
+    }
 
     // output of this warp's elements [G0, G0 + warp_total); its sign/mantissa
     // bytes are in the slot, which starts at element P0 & ~15.  Group g (16
@@ -1127,7 +1156,8 @@ df11_status validate(const df11_tensor &t) {
 
 struct DeviceInfo {
   int sms = 0;
-  std::atomic<size_t> configured[32];
+  std::atomic<size_t> configured[32];  // shared-memory limit set, per kernel instance
+  std::atomic<uint64_t> occupancy[32]; // last (smem << 8 | blocks per SM), per instance
 };
 
 DeviceInfo &device_info(int dev) {
@@ -1157,6 +1187,33 @@ uint32_t split_grid(KBatch &kb, const uint32_t *blocks, uint64_t budget) {
   return begin;
 }
 
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous one in the stream finishes (see pdl_wait).  DF11_PDL=0 in the
+// environment launches without it.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char *v = std::getenv("DF11_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
+template <typename... Args>
+df11_status launch_pdl(void (*kern)(Args...), uint32_t grid, uint32_t threads, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
 template <typename K>
 df11_status prepare(K kern, int threads, size_t smem, int instance, uint64_t &budget) {
   int dev = 0;
@@ -1168,9 +1225,18 @@ df11_status prepare(K kern, int threads, size_t smem, int instance, uint64_t &bu
       return DF11_ERR_CUDA;
     di.configured[instance].store(smem);
   }
+  // occupancy queries cost microseconds of host time: one per instance and
+  // shared-memory size (a layer-by-layer decode loop repeats the sizes)
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess)
-    return DF11_ERR_CUDA;
+  const uint64_t cached = di.occupancy[instance].load();
+  if (cached && (cached >> 8) == (uint64_t)smem) {
+    per_sm = (int)(cached & 0xFF);
+  } else {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) !=
+        cudaSuccess)
+      return DF11_ERR_CUDA;
+    di.occupancy[instance].store(((uint64_t)smem << 8) | (uint64_t)(per_sm & 0xFF));
+  }
   if (per_sm < 1) return DF11_ERR_TOO_LARGE;
   budget = (uint64_t)di.sms * per_sm;
   return DF11_OK;
@@ -1185,8 +1251,7 @@ df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t
   df11_status st = prepare(kern, T, smem, instance, budget);
   if (st != DF11_OK) return st;
   const uint32_t grid = split_grid(kb, blocks, budget);
-  kern<<<grid, T, smem, s>>>(kb);
-  return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+  return launch_pdl(kern, grid, T, smem, s, kb);
 }
 
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
@@ -1221,8 +1286,7 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
   if (pick < 0) return DF11_ERR_TOO_LARGE;
   kb.sm_bytes = pick == kSmSlot ? sm_stage : 0u;
   const uint32_t grid = split_grid(kb, blocks, best);
-  kern[pick]<<<grid, T + 32, smem[pick], s>>>(kb);
-  return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+  return launch_pdl(kern[pick], grid, T + 32, smem[pick], s, kb);
 }
 
 // Per-warp exponent region of the warp-specialised kernel: the warp's head

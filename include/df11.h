@@ -148,6 +148,14 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
                         df11_stream_t stream);
 
 /*
+ * Launches use programmatic dependent launch: a decode kernel may start
+ * while the previous kernel in the stream finishes, and waits for it to
+ * complete before its first store to out_bf16 (which that kernel may still
+ * read or write); the compressed inputs must not be written by it.  Setting
+ * DF11_PDL=0 in the environment before the first call launches plainly.
+ */
+
+/*
  * Decode `count` tensors (a layer's weights, say) with one kernel launch per
  * DF11_MAX_BATCH tensors.  `tensors` is a host array; every tensor must use
  * the same chunk_bytes and threads_per_block.  A tensor whose chunk_counts is
