@@ -1171,17 +1171,44 @@ DeviceInfo &device_info(int dev) {
   return d;
 }
 
-// thread blocks per tensor in proportion to its format blocks
+// Thread blocks per tensor: one wave (at most `budget`, the resident
+// count), at least one per tensor, and as few format blocks per thread block
+// as possible, since a launch lasts as long as its busiest thread block.
+// Shares in proportion to the format blocks, rounded down, then thread
+// blocks moved to where the most format blocks per thread block remain.
 uint32_t split_grid(KBatch &kb, const uint32_t *blocks, uint64_t budget) {
+  const int n = kb.count;
   uint64_t total = 0;
-  for (int i = 0; i < kb.count; ++i) total += blocks[i];
+  for (int i = 0; i < n; ++i) total += blocks[i];
+  if (budget < (uint64_t)n) budget = n;
+  uint64_t c[DF11_MAX_BATCH], sum = 0;
+  for (int i = 0; i < n; ++i) {
+    c[i] = budget * blocks[i] / total;
+    if (c[i] < 1) c[i] = 1;
+    if (c[i] > blocks[i]) c[i] = blocks[i];
+    sum += c[i];
+  }
+  auto per = [&](int i, uint64_t ci) { return (blocks[i] + ci - 1) / ci; };
+  while (sum > budget) {  // only from the at-least-one rule: take from the idlest
+    int best = -1;
+    for (int i = 0; i < n; ++i)
+      if (c[i] > 1 && (best < 0 || per(i, c[i] - 1) < per(best, c[best] - 1))) best = i;
+    if (best < 0) break;
+    --c[best];
+    --sum;
+  }
+  while (sum < budget) {  // the rest to the busiest tensor that can use one
+    int best = -1;
+    for (int i = 0; i < n; ++i)
+      if (c[i] < blocks[i] && (best < 0 || per(i, c[i]) > per(best, c[best]))) best = i;
+    if (best < 0) break;
+    ++c[best];
+    ++sum;
+  }
   uint32_t begin = 0;
-  for (int i = 0; i < kb.count; ++i) {
-    uint64_t c = (budget * blocks[i] + total / 2) / total;
-    if (c < 1) c = 1;
-    if (c > blocks[i]) c = blocks[i];
+  for (int i = 0; i < n; ++i) {
     kb.t[i].cta_begin = begin;
-    begin += (uint32_t)c;
+    begin += (uint32_t)c[i];
   }
   kb.cta_end = begin;
   return begin;
@@ -1258,9 +1285,9 @@ size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t regio
                        uint32_t sub_words, bool warp_sm);
 
 // Sign/mantissa bytes staged per block in the stage slot, per warp in the
-// warp's own buffer, or read from global memory: the first of these that
-// keeps the most thread blocks resident (16-byte shared loads in the output
-// beat L2 loads at equal residency).
+// warp's own buffer, or read from global memory, in this order of speed as
+// measured: the first that keeps at least 24 consumer warps resident per SM,
+// else the one that keeps the most.
 template <int T, int C>
 df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
@@ -1271,6 +1298,13 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
                           ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, false),
                           ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, true)};
   const int order[3] = {kSmSlot, kSmWarp, kSmGlobal};
+  constexpr uint64_t kEnoughWarps = 24;  // consumer warps per SM
+  int dev_sms = 0;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
+    dev_sms = device_info(dev).sms;
+  }
   uint64_t best = 0;
   int pick = -1;
   for (int m : order) {
@@ -1281,6 +1315,11 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
     if (budget > best) {
       best = budget;
       pick = m;
+    }
+    if (budget * (T / 32) >= kEnoughWarps * (uint64_t)dev_sms) {
+      best = budget;
+      pick = m;
+      break;
     }
   }
   if (pick < 0) return DF11_ERR_TOO_LARGE;
