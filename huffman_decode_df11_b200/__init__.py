@@ -53,7 +53,7 @@ class Params(ctypes.Structure):
         ("max_block_elems", ctypes.c_uint32),
         ("max_len", ctypes.c_uint32),
         ("max_chunk_elems", ctypes.c_uint32),
-        ("reserved", ctypes.c_uint32),
+        ("max_warp_elems", ctypes.c_uint32),
     ]
 
 

@@ -407,13 +407,18 @@ extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
     df11_host_tensor_free(out);
     return DF11_ERR_NOMEM;
   }
-  uint32_t mc = 0;
+  uint32_t mc = 0, mw = 0;
   for (uint64_t c = 0; c < chunks; ++c) {
     const uint32_t k = first_elem[c + 1] - first_elem[c];
     out->chunk_counts[c] = (uint8_t)k;
     mc = std::max(mc, k);
   }
+  for (uint64_t g = 0; g < chunks; g += 32) {  // groups of 32 consecutive chunks
+    const uint64_t e = std::min<uint64_t>(g + 32, chunks);
+    mw = std::max(mw, first_elem[e] - first_elem[g]);
+  }
   p.max_chunk_elems = mc;
+  p.max_warp_elems = mw;
   return DF11_OK;
 }
 

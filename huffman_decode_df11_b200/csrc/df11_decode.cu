@@ -80,6 +80,7 @@ struct KTensor {
   uint32_t num_luts;
   uint32_t max_block_elems;
   uint32_t max_chunk_elems;
+  uint32_t max_warp_elems;   // sizes the per-warp regions of the warp-specialised kernel
   uint32_t masked;     // longest codeword > kWideBits: bits past a region may be set
   uint32_t cta_begin;  // first thread block of this tensor
   uint32_t pad;
@@ -996,6 +997,12 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : 1280 / T)
       if (lane >= dd) incl += v;
     }
     const uint32_t warp_total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if (warp_total > tk.max_warp_elems) {  // would not fit the region (uniform)
+      if (lane == 0) report(kb.err, DF11_DEV_ERR_CAPACITY);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(release);
+      continue;
+    }
     const uint32_t G0 = P0 + before;            // first element of this warp
     const uint32_t head = G0 & 15u, span = head + warp_total;
     const uint32_t d = head + incl - cnt;       // my first byte in the region
@@ -1149,6 +1156,8 @@ df11_status validate(const df11_tensor &t) {
   if (p.max_block_elems == 0 || p.max_block_elems > 8ull * p.chunk_bytes * p.threads_per_block)
     return DF11_ERR_FORMAT;
   if (p.max_chunk_elems == 0 || p.max_chunk_elems > 8ull * p.chunk_bytes) return DF11_ERR_FORMAT;
+  if (p.max_warp_elems == 0 || p.max_warp_elems > 32ull * p.max_chunk_elems)
+    return DF11_ERR_FORMAT;
   if (t.chunk_counts && 8ull * p.chunk_bytes > 255) return DF11_ERR_FORMAT;
   if (p.max_len < 1 || p.max_len > 32) return DF11_ERR_FORMAT;
   return DF11_OK;
@@ -1284,10 +1293,10 @@ df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
                        uint32_t sub_words, bool warp_sm);
 
-// Sign/mantissa bytes staged per block in the stage slot, per warp in the
-// warp's own buffer, or read from global memory, in this order of speed as
-// measured: the first that keeps at least 24 consumer warps resident per SM,
-// else the one that keeps the most.
+// Sign/mantissa bytes staged per block in the stage slot or per warp in the
+// warp's own buffer, whichever keeps more thread blocks resident (the slot
+// on a tie); read from global memory only when neither fits.  Measured: at
+// equal residency the slot beats the warp buffer, which beats global reads.
 template <int T, int C>
 df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
@@ -1298,16 +1307,10 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
                           ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, false),
                           ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, true)};
   const int order[3] = {kSmSlot, kSmWarp, kSmGlobal};
-  constexpr uint64_t kEnoughWarps = 24;  // consumer warps per SM
-  int dev_sms = 0;
-  {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
-    dev_sms = device_info(dev).sms;
-  }
   uint64_t best = 0;
   int pick = -1;
   for (int m : order) {
+    if (m == kSmGlobal && pick >= 0) break;
     if (smem[m] > 227 * 1024) continue;
     uint64_t budget = 0;
     const df11_status st = prepare(kern[m], T + 32, smem[m], 3 * instance + m, budget);
@@ -1315,11 +1318,6 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
     if (budget > best) {
       best = budget;
       pick = m;
-    }
-    if (budget * (T / 32) >= kEnoughWarps * (uint64_t)dev_sms) {
-      best = budget;
-      pick = m;
-      break;
     }
   }
   if (pick < 0) return DF11_ERR_TOO_LARGE;
@@ -1329,11 +1327,12 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
 }
 
 // Per-warp exponent region of the warp-specialised kernel: the warp's head
-// (< 16), up to 32 chunks of max_chunk_elems exponents, and slack for the
-// last lookup: it touches bytes up to 6 past the warp's last element (the
-// spill word, or up to three extra exponents of a corrupt stream).
-uint32_t region_bytes_for(uint32_t max_chunk_elems) {
-  return (15u + 32u * max_chunk_elems + 8u + 15u) & ~15u;
+// (< 16), up to max_warp_elems exponents (checked per block before
+// decoding), and slack for the last lookup: it touches bytes up to 6 past
+// the warp's last element (the spill word, or up to three extra exponents of
+// a corrupt stream).
+uint32_t region_bytes_for(uint32_t max_warp_elems) {
+  return (15u + max_warp_elems + 8u + 15u) & ~15u;
 }
 
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
@@ -1348,7 +1347,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   KBatch kb{};
   kb.err = d_err;
   uint32_t blocks[DF11_MAX_BATCH];
-  uint32_t max_elems = 0, max_chunk = 0, max_luts = 1, C = 0, T = 0;
+  uint32_t max_elems = 0, max_chunk = 0, max_warp = 0, max_luts = 1, C = 0, T = 0;
   for (int i = 0; i < count; ++i) {
     const df11_params &p = ts[i].params;
     if (p.n == 0) continue;
@@ -1368,11 +1367,13 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     k.num_luts = p.num_luts;
     k.max_block_elems = p.max_block_elems;
     k.max_chunk_elems = p.max_chunk_elems;
+    k.max_warp_elems = p.max_warp_elems;
     k.masked = p.max_len > (uint32_t)kWideBits ? 1u : 0u;
     blocks[kb.count] = p.num_blocks;
     ++kb.count;
     max_elems = max_elems > p.max_block_elems ? max_elems : p.max_block_elems;
     max_chunk = max_chunk > p.max_chunk_elems ? max_chunk : p.max_chunk_elems;
+    max_warp = max_warp > p.max_warp_elems ? max_warp : p.max_warp_elems;
     max_luts = max_luts > p.num_luts ? max_luts : p.num_luts;
     C = p.chunk_bytes;
     T = p.threads_per_block;
@@ -1380,7 +1381,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   if (kb.count == 0) return DF11_OK;
   kb.sub_words = (max_luts - 1) <= (uint32_t)kSubTablesInSmem ? (max_luts - 1) * 256 : 0;
   if (ws) {
-    kb.stage_bytes = region_bytes_for(max_chunk);  // bytes of each warp's region
+    kb.stage_bytes = region_bytes_for(max_warp);  // bytes of each warp's region
     kb.slot_words = 0;
     // deeper tables only serve codewords longer than the derived table's
     // index (about one lookup in a thousand): read them from global memory
@@ -1489,7 +1490,7 @@ size_t df11_shared_bytes(const df11_params *p) {
                                    slot_words_for(p->max_chunk_elems), subs);
   const size_t ws = ws_shared_bytes(p->chunk_bytes, p->threads_per_block,
                                     stage_bytes_for(p->max_block_elems),
-                                    region_bytes_for(p->max_chunk_elems), 0, false);
+                                    region_bytes_for(p->max_warp_elems), 0, false);
   return page > ws ? page : ws;
 }
 

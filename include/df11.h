@@ -106,7 +106,10 @@ typedef struct df11_params {
   uint32_t max_block_elems;   /* max over blocks of elements per block */
   uint32_t max_len;           /* longest codeword in bits (<= 32) */
   uint32_t max_chunk_elems;   /* max over chunks of codewords starting in it */
-  uint32_t reserved;          /* 0 */
+  uint32_t max_warp_elems;    /* max over groups of 32 consecutive chunks of
+                                 the codewords starting in them (one warp's
+                                 share of a block in the decode kernel;
+                                 sizes its shared-memory buffers) */
 } df11_params;
 
 /* Bytes of the decode table that df11_build_decode_table writes. */

@@ -65,6 +65,7 @@ class _Format(ctypes.Structure):
         ("max_block_elems", ctypes.c_uint32),
         ("max_len", ctypes.c_uint32),
         ("max_chunk_elems", ctypes.c_uint32),
+        ("max_warp_elems", ctypes.c_uint32),
         ("code_lengths", ctypes.c_uint8 * 256),
         ("codes", ctypes.c_uint32 * 256),
         ("bitstream", ctypes.POINTER(ctypes.c_uint8)),
@@ -141,6 +142,7 @@ class OracleFormat:
     max_block_elems: int
     max_len: int
     max_chunk_elems: int
+    max_warp_elems: int
     code_lengths: np.ndarray   # uint8[256]
     codes: np.ndarray          # uint32[256]
     bitstream: np.ndarray      # uint8[num_blocks*T*C + 16]
@@ -251,6 +253,7 @@ def encode(w, chunk_bytes: int = 8, threads_per_block: int = 256) -> OracleForma
             threads_per_block=f.threads_per_block, num_blocks=f.num_blocks,
             num_luts=f.num_luts, max_block_elems=f.max_block_elems,
             max_len=f.max_len, max_chunk_elems=f.max_chunk_elems,
+            max_warp_elems=f.max_warp_elems,
             code_lengths=np.frombuffer(bytes(f.code_lengths), np.uint8).copy(),
             codes=np.array(list(f.codes), dtype=np.uint32),
             bitstream=_copy(f.bitstream, f.bitstream_bytes, np.uint8),

@@ -415,8 +415,10 @@ int oracle_encode(const uint16_t *w, uint64_t n, uint32_t chunk_bytes,
   f->gaps_packed = (uint8_t *)calloc(f->gaps_bytes, 1);
   oracle_pack_gaps(f->gaps, chunks, f->gaps_packed);
 
-  /* codewords starting in each chunk, counted one start at a time */
+  /* codewords starting in each chunk, counted one start at a time, and in
+     each group of 32 consecutive chunks */
   f->max_chunk_elems = 0;
+  f->max_warp_elems = 0;
   f->chunk_counts_bytes = chunks + 16;
   f->chunk_counts = (uint8_t *)calloc(f->chunk_counts_bytes, 1);
   if (chunks) {
@@ -425,6 +427,11 @@ int oracle_encode(const uint16_t *w, uint64_t n, uint32_t chunk_bytes,
     for (uint64_t c = 0; c < chunks; c++) {
       if (per_chunk[c] > f->max_chunk_elems) f->max_chunk_elems = per_chunk[c];
       f->chunk_counts[c] = (uint8_t)per_chunk[c];
+    }
+    for (uint64_t g = 0; g < chunks; g += 32) {
+      uint32_t sum = 0;
+      for (uint64_t c = g; c < g + 32 && c < chunks; c++) sum += per_chunk[c];
+      if (sum > f->max_warp_elems) f->max_warp_elems = sum;
     }
     free(per_chunk);
   }

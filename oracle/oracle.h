@@ -50,6 +50,8 @@ typedef struct oracle_format {
   uint32_t max_block_elems;   /* max over blocks of its element count */
   uint32_t max_len;           /* longest codeword */
   uint32_t max_chunk_elems;   /* max over chunks of codewords starting in it */
+  uint32_t max_warp_elems;    /* max over groups of 32 consecutive chunks of
+                                 the codewords starting in them */
   uint8_t code_lengths[256];  /* 0 = exponent absent */
   uint32_t codes[256];        /* canonical codeword, right-aligned */
   uint8_t *bitstream;         /* num_blocks*T*C + 16 bytes, MSB-first */

@@ -46,7 +46,7 @@ def test_struct_layouts_match_header():
 def _params(**kw):
     p = df11.Params(n=1000, total_bits=2600, chunk_bytes=8, threads_per_block=256,
                     num_blocks=1, num_luts=1, max_block_elems=1000, max_len=10,
-                    max_chunk_elems=40)
+                    max_chunk_elems=40, max_warp_elems=1000)
     for k, v in kw.items():
         setattr(p, k, v)
     return p
@@ -76,6 +76,8 @@ def test_host_validation_errors():
     assert _call(_params(num_luts=0)) == 3
     assert _call(_params(max_block_elems=20000)) == 3
     assert _call(_params(max_chunk_elems=65)) == 3                           # > 8*C
+    assert _call(_params(max_warp_elems=0)) == 3
+    assert _call(_params(max_warp_elems=32 * 40 + 1)) == 3                   # > 32*max_chunk
     assert _call(_params(max_len=33)) == 3
     assert _call(_params(n=1 << 32, total_bits=1 << 34, num_blocks=1 << 20)) == 6
 
@@ -87,7 +89,8 @@ def test_batched_host_validation():
     assert L.df11_decode_batched(None, 1, None, None) == 1
     a = df11.TensorDesc(*[FAKE] * 8, None, _params())
     b = df11.TensorDesc(*[FAKE] * 8, None, _params(chunk_bytes=4, total_bits=2600,
-                                                      num_blocks=1, max_chunk_elems=30))
+                                                      num_blocks=1, max_chunk_elems=30,
+                                                      max_warp_elems=900))
     arr = (df11.TensorDesc * 2)(a, b)
     assert L.df11_decode_batched(arr, 2, None, None) == 7  # mixed (C, T)
     c = df11.TensorDesc(*[FAKE] * 8, FAKE + 8, _params())  # misaligned decode table

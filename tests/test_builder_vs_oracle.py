@@ -22,6 +22,7 @@ def _compare(w, C, T, threads=4):
     assert p.max_block_elems == f.max_block_elems
     assert p.max_len == f.max_len
     assert p.max_chunk_elems == f.max_chunk_elems
+    assert p.max_warp_elems == f.max_warp_elems
     assert np.array_equal(h.code_lengths, f.code_lengths)
     assert np.array_equal(h.bitstream, f.bitstream)
     assert np.array_equal(h.gaps, f.gaps_packed)

@@ -357,6 +357,7 @@ def test_gaps_and_block_positions_brute_force(C, T):
     for s in st:
         per_chunk[s // chunk_bits] += 1
     assert f.max_chunk_elems == max(per_chunk)
+    assert f.max_warp_elems == max(sum(per_chunk[g:g + 32]) for g in range(0, len(per_chunk), 32))
     assert f.chunk_counts[: len(per_chunk)].tolist() == per_chunk
     assert not f.chunk_counts[len(per_chunk):].any()
     # packed gaps: 5-bit fields, MSB first
