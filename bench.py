@@ -103,7 +103,8 @@ def kernel_hash() -> str:
 
 def recorded_traffic(workload: str):
     """Per-launch DRAM bytes from an ncu capture of the current kernel source
-    (profiles/dram_traffic.txt: '<kernel sha16> <workload> <bytes per launch>')."""
+    (profiles/dram_traffic.txt: '<kernel sha16> <workload>/c<C>/t<T> <bytes
+    per launch>')."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     kh = kernel_hash()
@@ -335,7 +336,8 @@ def run_b200(args, world, rank, local):
     achieved = sum(alg) / (ms_local * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     # the capture covers the chunk-count kernel; the page-layout kernel has none
-    traffic = recorded_traffic(args.config) if counts else None
+    traffic = (recorded_traffic(f"{args.config}/c{args.chunk_bytes}/t{args.threads_per_block}")
+               if counts else None)
 
     # end to end through the public API: host (pinned) compressed tensors in,
     # host BF16 out, copies inside the timed region

@@ -1,52 +1,51 @@
 // df11_decode.cu -- DF11 decode on sm_100a (B200) and the C ABI around it.
 //
-// Persistent thread blocks.  Every thread block is assigned to one tensor of
-// the launch and walks that tensor's format blocks (T chunks of C bitstream
-// bytes each) with a stride.  Per thread block, once:
+// Two kernels, both with persistent thread blocks: every thread block is
+// assigned to one tensor of the launch (one wave, split by format blocks)
+// and walks that tensor's format blocks (T chunks of C bitstream bytes) with
+// a stride.  Both use the same decode table in shared memory: table 0 of
+// the format and the code lengths with every exponent byte rotated right by
+// one bit, and a derived table of 2^11 entries, each holding up to four
+// whole codewords of the next 11 bits (built once per tensor by
+// df11_table_kernel, or by every thread block when none is passed).
+// Deeper format tables (codewords longer than 8 bits) are read from global
+// memory.
 //
-//   tables   table 0 of the format (256 entries, up to three codewords per
-//            8-bit index) and the code lengths are copied into shared memory
-//            with every exponent byte rotated right by one bit; a wide table
-//            of 2^WB entries, each holding up to four whole codewords of the
-//            next WB bits, is derived from them in shared memory.  Deeper
-//            format tables (codewords longer than 8 bits) are read from shared
-//            memory when few, from global memory otherwise.
+// df11_decode_ws_kernel, for tensors with chunk counts (the default path).
+// Warp-specialised: one producer warp and T/32 consumer warps per thread
+// block, no block-wide barrier per format block.
+//   stage    the producer's lane 0 keeps two stage slots filled with bulk
+//            copies (cp.async.bulk, no multicast) of a block's bitstream
+//            slice, gap fields and chunk counts, and its sign/mantissa bytes
+//            (or those go to per-warp buffers, or stay in L2), each slot
+//            guarded by a full and an empty mbarrier.
+//   locate   every consumer warp sums the stored chunk counts before its 32
+//            chunks (warp reductions) and scans its lanes' counts: each lane
+//            knows where its exponents go before it decodes.
+//   decode   each lane walks its chunk once ("locate" and "reconstruct" of
+//            "DFloat11重新定义LLM无损压缩的技术边界" (ocdem.com) §2.2 in one
+//            pass) with a shifting bit window, stopping on its element
+//            count; every lookup ORs its up to four exponents into the
+//            warp's zeroed exponent region (two shared reductions).
+//   output   the warp fuses 16 exponents with 16 sign/mantissa bytes per
+//            lane and step (two selects, two byte permutes per four
+//            elements), writes two 16-byte stores, re-zeroes what it read,
+//            and writes the two ragged 16-element groups one element per
+//            lane; then releases the slot.
 //
-// Per format block, software-pipelined with a two-slot stage:
-//
-//   stage    one thread issues bulk asynchronous copies (cp.async.bulk, no
-//            multicast) of the NEXT block's bitstream slice and gap fields
-//            into the free stage slot, completing on that slot's mbarrier,
-//            and a bulk L2 prefetch of its sign/mantissa bytes, while the
-//            block in the other slot is decoded.
-//   decode   each thread walks its chunk from its gap ("locate" and
-//            "reconstruct" of "DFloat11重新定义LLM无损压缩的技术边界"
-//            (ocdem.com) §2.2, done in one pass): every lookup of the wide
-//            table yields up to four exponents, appended to a 64-bit
-//            accumulator and flushed as aligned 32-bit words into the
-//            thread's private slot (word j of thread t at j*T+t: one bank per
-//            thread, no conflicts).  Bits past the thread's region are set to
-//            one, so no lookup can accept a codeword beyond it (valid when the
-//            longest codeword is longer than WB bits; other codes take a loop
-//            that checks the region end on every lookup).
-//   scan     exclusive prefix sum of the per-thread counts (warp shuffles,
-//            then across warps) gives every thread its first output index;
-//            the total must equal the block's block_out_pos difference.
-//   compact  every thread moves its exponents from its slot to their final
-//            places in a block-wide byte array: funnel-shifted 32-bit stores,
-//            shared atomic OR for the two words it shares with neighbours.
-//   output   every thread loads 16 sign/mantissa bytes (16-byte global load),
-//            fuses them with 16 exponents into 16 BF16 words with byte
-//            permutes and writes them with two 16-byte stores; the block's
-//            two ragged 16-element groups are written one element per lane.
+// df11_decode_kernel, for the format as the pages state it (no chunk
+// counts): every thread decodes its chunk into a private slot, counting
+// ("locate"), a block-wide scan places the slots, they are compacted into a
+// block-wide exponent array, and the block writes its output range.
 //
 // Why the rotation: with e' = e>>1 | (e&1)<<7, the high byte of a BF16 word
 // is (sm & 0x80) | (e' & 0x7F) and the low byte (e' & 0x80) | (sm & 0x7F), so
 // four output words cost two bitwise selects and two byte permutes.
 //
-// Nothing here waits on another thread block, so nothing can hang: the only
-// waits are on this block's own copies, bounded, reporting
-// DF11_DEV_ERR_TIMEOUT.  Every data-dependent access is bounds-checked;
+// Nothing here waits on another thread block of the same grid, so nothing
+// can hang: the waits are on this block's own copies and barriers, bounded,
+// reporting DF11_DEV_ERR_TIMEOUT, and (programmatic dependent launch) for
+// the previous grid in the stream to complete.  Every data-dependent access is bounds-checked;
 // inconsistent data are reported through the error word, never by a trap.
 #include <cuda_runtime.h>
 
