@@ -227,7 +227,7 @@ def barrier(world: int):
         dist.barrier()
 
 
-def prepare(config: str, seed: int, device: str, chunk_bytes: int = 16,
+def prepare(config: str, seed: int, device: str, chunk_bytes: int = 24,
             threads_per_block: int = 256):
     """Compress every unit on the host; keep compressed tensors resident in
     HBM.  Originals are regenerated from the seed when checked."""
@@ -533,7 +533,7 @@ def main(argv=None):
     ap.add_argument("--config", default="block", choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--chunk-bytes", type=int, default=16, choices=[4, 8, 16],
+    ap.add_argument("--chunk-bytes", type=int, default=24, choices=[4, 8, 16, 24],
                     help="bitstream bytes per chunk (C) of the compressed format")
     ap.add_argument("--threads-per-block", type=int, default=256, choices=[128, 256, 512],
                     help="chunks per format block (T) of the compressed format")

@@ -1112,7 +1112,7 @@ __global__ void __launch_bounds__(256) df11_table_kernel(const uint32_t *luts,
 // host side
 
 bool supported(uint32_t C, uint32_t T) {
-  if (T == 256) return C == 4 || C == 8 || C == 16;
+  if (T == 256) return C == 4 || C == 8 || C == 16 || C == 24;
   if (T == 128 || T == 512) return C == 8;
   return false;
 }
@@ -1164,8 +1164,8 @@ df11_status validate(const df11_tensor &t) {
 
 struct DeviceInfo {
   int sms = 0;
-  std::atomic<size_t> configured[32];  // shared-memory limit set, per kernel instance
-  std::atomic<uint64_t> occupancy[32]; // last (smem << 8 | blocks per SM), per instance
+  std::atomic<size_t> configured[40];  // shared-memory limit set, per kernel instance
+  std::atomic<uint64_t> occupancy[40]; // last (smem << 8 | blocks per SM), per instance
 };
 
 DeviceInfo &device_info(int dev) {
@@ -1390,6 +1390,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     if (T == 256 && C == 8) return launch_ws<256, 8>(kb, blocks, sm_stage, s, 3);
     if (T == 256 && C == 4) return launch_ws<256, 4>(kb, blocks, sm_stage, s, 4);
     if (T == 256 && C == 16) return launch_ws<256, 16>(kb, blocks, sm_stage, s, 5);
+    if (T == 256 && C == 24) return launch_ws<256, 24>(kb, blocks, sm_stage, s, 8);
     if (T == 128 && C == 8) return launch_ws<128, 8>(kb, blocks, sm_stage, s, 6);
     if (T == 512 && C == 8) return launch_ws<512, 8>(kb, blocks, sm_stage, s, 7);
     return DF11_ERR_UNSUPPORTED;
@@ -1405,6 +1406,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   if (T == 256 && C == 8) return launch<256, 8>(kb, blocks, smem, s, 0);
   if (T == 256 && C == 4) return launch<256, 4>(kb, blocks, smem, s, 1);
   if (T == 256 && C == 16) return launch<256, 16>(kb, blocks, smem, s, 2);
+  if (T == 256 && C == 24) return launch<256, 24>(kb, blocks, smem, s, 33);
   if (T == 128 && C == 8) return launch<128, 8>(kb, blocks, smem, s, 3);
   if (T == 512 && C == 8) return launch<512, 8>(kb, blocks, smem, s, 4);
   return DF11_ERR_UNSUPPORTED;

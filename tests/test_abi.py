@@ -109,6 +109,7 @@ def test_decode_table_host_validation():
 
 def test_supported_shapes_and_shared_bytes():
     assert df11.supported(8, 256) and df11.supported(4, 256) and df11.supported(16, 256)
+    assert df11.supported(24, 256) and not df11.supported(20, 256)
     assert df11.supported(8, 128) and df11.supported(8, 512)
     assert not df11.supported(12, 256)
     p = _params(max_block_elems=6400, num_luts=4)

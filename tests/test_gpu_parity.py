@@ -50,7 +50,7 @@ def _gpu_vs_oracle_full(w_np, C=8, T=256, counts=True, table=True):
 # --- oracle-sized cases, compared in full ---------------------------------
 
 @pytest.mark.parametrize("case", ["gaussian", "adversarial", "fibonacci", "patterns", "few"])
-@pytest.mark.parametrize("C", [8, 16])
+@pytest.mark.parametrize("C", [8, 16, 24])
 def test_without_decode_table(case, C):
     """Every thread block derives the decode table itself (no
     df11_build_decode_table): same output as with it."""
@@ -91,7 +91,7 @@ def test_decode_table_holds_the_rotated_format_tables():
         assert int(lut0[i]) == e
 
 @COUNTS
-@pytest.mark.parametrize("C,T", [(8, 256), (4, 256), (16, 256), (8, 128), (8, 512)])
+@pytest.mark.parametrize("C,T", [(8, 256), (4, 256), (16, 256), (24, 256), (8, 128), (8, 512)])
 def test_single_matrix_all_kernel_shapes(C, T, counts):
     w = workloads.as_numpy_u16(workloads.single_matrix(0))
     _gpu_vs_oracle_full(w, C, T, counts)
