@@ -3,11 +3,12 @@
 // Two kernels, both with persistent thread blocks: every thread block is
 // assigned to one tensor of the launch (one wave, split by format blocks)
 // and walks that tensor's format blocks (T chunks of C bitstream bytes) with
-// a stride.  Both use the same decode table in shared memory: table 0 of
-// the format and the code lengths with every exponent byte rotated right by
-// one bit, and a derived table of 2^11 entries, each holding up to four
-// whole codewords of the next 11 bits (built once per tensor by
-// df11_table_kernel, or by every thread block when none is passed).
+// a stride.  Both use a decode table in shared memory: table 0 of the format
+// and the code lengths with every exponent byte rotated right by one bit,
+// and a derived table of 2^11 entries, each holding up to five whole
+// codewords of the next 11 bits (built once per tensor by df11_table_kernel,
+// or by every thread block when none is passed; the page-layout kernel
+// derives its own with up to four, which its accumulator takes).
 // Deeper format tables (codewords longer than 8 bits) are read from global
 // memory.
 //
@@ -25,7 +26,7 @@
 //   decode   each lane walks its chunk once ("locate" and "reconstruct" of
 //            "DFloat11重新定义LLM无损压缩的技术边界" (ocdem.com) §2.2 in one
 //            pass) with a shifting bit window, stopping on its element
-//            count; every lookup ORs its up to four exponents into the
+//            count; every lookup ORs its up to five exponents into the
 //            warp's zeroed exponent region (two shared reductions).
 //   output   the warp fuses 16 exponents with 16 sign/mantissa bytes per
 //            lane and step (two selects, two byte permutes per four
@@ -61,7 +62,6 @@ constexpr int kSubTablesInSmem = 8;        // deeper tables kept in shared memor
 constexpr uint32_t kSpinLimit = 1u << 20;  // x ~1 us suspend hint: ~1 s
 constexpr uint32_t kSuspendHintNs = 1000;
 constexpr int kWideBits = 11;              // index bits of the derived table
-constexpr int kWideSyms = 4;               // codewords per derived entry
 
 struct KTensor {
   const uint8_t *bitstream;
@@ -269,43 +269,48 @@ __device__ __forceinline__ void load_tables(int tid, int nthreads, const uint32_
 }
 
 // Derived table: entry i holds the codewords that lie wholly inside the WB
-// bits i (at most kWideSyms): x = exponents (first in bits 0-7),
-// y = bits used | 8 * count << 16, so that one add moves both the bit
-// position and the output bit offset of a packed (bit, output bit) register.
+// bits i, at most MS of them: x = the first four exponents (first in bits
+// 0-7), y = bits used | 8 * count << 16 | fifth exponent << 24, so that one
+// add of y's low 24 bits moves both the bit position and the output bit
+// offset of a packed (bit, output bit) register, and the five exponent
+// bytes shift into two words with two funnel shifts.
 // y == 0: the first codeword is longer than WB bits (or invalid) and takes
 // the slow path.
-template <int T>
+template <int T, int MS>
 __device__ void build_wide(uint2 *wide, const uint32_t *lut0, const uint8_t *lens,
                            const uint32_t *sub, uint32_t num_luts) {
+  static_assert(MS >= 1 && MS <= 5, "at most five exponent bytes per entry");
   for (uint32_t i = threadIdx.x; i < (1u << kWideBits); i += T) {
     const uint32_t bits = i << (32 - kWideBits);
-    uint32_t used = 0, n = 0, syms = 0;
-    while (n < kWideSyms) {
+    uint32_t used = 0, n = 0;
+    uint64_t syms = 0;
+    while (n < MS) {
       const uint32_t win = bits << used;
       const uint32_t e = lut0[win >> 24];
       const uint32_t ns = e >> 28;
       if (((e >> 24) & 15u) == 0) {
         uint32_t s, l;
         if (!decode_one(win, lut0, lens, sub, num_luts, s, l) || used + l > kWideBits) break;
-        syms |= s << (8 * n);
+        syms |= (uint64_t)s << (8 * n);
         ++n;
         used += l;
         continue;
       }
       bool stop = ns == 0;
-      for (uint32_t j = 0; j < ns && n < kWideSyms; ++j) {
+      for (uint32_t j = 0; j < ns && n < MS; ++j) {
         const uint32_t s = (e >> (8 * j)) & 0xFFu, l = lens[s];
         if (l == 0 || used + l > kWideBits) {
           stop = true;
           break;
         }
-        syms |= s << (8 * n);
+        syms |= (uint64_t)s << (8 * n);
         ++n;
         used += l;
       }
       if (stop || used >= kWideBits) break;
     }
-    wide[i] = n ? make_uint2(syms, used | (n << 19)) : make_uint2(0, 0);
+    wide[i] = n ? make_uint2((uint32_t)syms, used | (n << 19) | ((uint32_t)(syms >> 32) << 24))
+                : make_uint2(0, 0);
   }
 }
 
@@ -382,7 +387,7 @@ __device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1],
 
 // The same walk when the thread's output place is known before it decodes
 // (the format's chunk count): exponents go straight into the block's
-// (zeroed) exponent array from byte d on.  Every lookup ORs its up to four
+// (zeroed) exponent array from byte d on.  Every lookup ORs its up to five
 // bytes into the word that holds the next byte and the word after it (the
 // part that spills over; zero when nothing does), which also merges the
 // words a thread shares with its neighbours.  `pk` packs the bit position
@@ -412,8 +417,8 @@ __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1]
     const uint32_t sh = (pk >> 16) & 24u;
     const uint32_t a = min(ex + ((pk >> 21) << 2), limit);
     red_or32(a, e.x << sh);
-    red_or32(a + 4u, __funnelshift_l(e.x, 0u, sh));
-    pk += e.y;
+    red_or32(a + 4u, __funnelshift_l(e.x, e.y >> 24, sh));  // with the fifth exponent
+    pk += e.y & 0x00FFFFFFu;
   }
   if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
   return (pk >> 19) - d;
@@ -429,9 +434,9 @@ __device__ __forceinline__ uint32_t decode_direct(const uint32_t (&w)[C / 4 + 1]
 //   - the loop ends on the element count, not the bit position: it runs
 //     while the output bit offset (bits 16-31 of `pk`, bit position in bits
 //     0-15) is below 8*(d+cnt).  Every iteration emits at least one element,
-//     so a corrupt stream stops within cnt lookups and writes at most three
-//     bytes (plus the spill word) past the thread's range, which the region's
-//     slack absorbs: no clamp on the address.  Bits past `end` are ones, so
+//     so a corrupt stream stops within cnt lookups and writes at most four
+//     bytes past the thread's range (the last lookup's five bytes stay in two
+//     words), which the region's slack absorbs: no clamp on the address.  Bits past `end` are ones, so
 //     on valid data the last lookup stops exactly at `end` (checked after).
 // Returns the number of elements written.
 template <int C>
@@ -470,11 +475,11 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t (&w)[C / 4 + 1
     const uint32_t sh = pk >> 16;  // funnel shifts use sh & 31: the bit offset in the word
     const uint32_t a = ex + ((pk >> 21) << 2);
     red_or32(a, __funnelshift_l(0u, e.x, sh));
-    red_or32(a + 4u, __funnelshift_l(e.x, 0u, sh));
+    red_or32(a + 4u, __funnelshift_l(e.x, e.y >> 24, sh));  // with the fifth exponent
 #pragma unroll
     for (int j = 0; j < NW - 1; ++j) s[j] = __funnelshift_l(s[j + 1], s[j], e.y);
     s[NW - 1] = __funnelshift_l(0xFFFFFFFFu, s[NW - 1], e.y);
-    pk += e.y;
+    pk += e.y & 0x00FFFFFFu;
   }
   // a count that disagrees with the stream ends the walk short of `end`
   // (too small) or past it (too large, or a corrupt stream)
@@ -579,7 +584,7 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
   for (uint32_t i = tid; i < kb.stage_bytes / 16; i += T)  // zeroed once; each
     reinterpret_cast<uint4 *>(ex_s)[i] = make_uint4(0, 0, 0, 0);  // output re-zeroes
   __syncthreads();
-  build_wide<T>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
+  build_wide<T, 4>(wide_s, lut0_s, lens_s, sub, tk.num_luts);  // its accumulator takes 4
   __syncthreads();
 
   const int lane = tid & 31, warp = tid >> 5;
@@ -895,7 +900,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : (C >= 16 && T ==
   } else {
     load_tables(tid, T + 32, tk.luts, tk.code_lengths, lut0_s, lens_s);
     __syncthreads();
-    build_wide<T + 32>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
+    build_wide<T + 32, 5>(wide_s, lut0_s, lens_s, sub, tk.num_luts);
   }
   if (!__syncthreads_and(tables_ok)) {
     if (tid == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
@@ -1105,7 +1110,7 @@ __global__ void __launch_bounds__(256) df11_table_kernel(const uint32_t *luts,
   uint2 *wide_s = reinterpret_cast<uint2 *>(t + (kOffWide - kOffLens));
   load_tables(threadIdx.x, 256, luts, code_lengths, lut0_s, lens_s);
   __syncthreads();
-  build_wide<256>(wide_s, lut0_s, lens_s, luts + 256, num_luts);
+  build_wide<256, 5>(wide_s, lut0_s, lens_s, luts + 256, num_luts);
   __syncthreads();
   for (uint32_t i = threadIdx.x; i < DF11_DECODE_TABLE_BYTES / 16; i += 256)
     out[i] = reinterpret_cast<const uint4 *>(t)[i];
