@@ -363,3 +363,14 @@ def test_host_side_argument_errors():
         df11.decode(d, out=big[1:])
     with pytest.raises(ValueError):
         df11.decode(d, out=out[:-1])
+
+
+def test_tensors_loaded_from_a_file_decode_bit_exact(tmp_path):
+    from huffman_decode_df11_b200 import serialization as ser
+    ws = {"a": workloads.as_numpy_u16(workloads.adversarial_mix(1 << 20, 11)),
+          "b": workloads.as_numpy_u16(workloads.gaussian_bf16(777_777, 0.02, 12))}
+    path = str(tmp_path / "w.df11")
+    ser.save(path, {k: df11.compress(v) for k, v in ws.items()})
+    for k, h in ser.load(path).items():
+        out = _decode(h).view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(out, ws[k])
