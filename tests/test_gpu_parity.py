@@ -374,3 +374,46 @@ def test_tensors_loaded_from_a_file_decode_bit_exact(tmp_path):
     for k, h in ser.load(path).items():
         out = _decode(h).view(torch.int16).cpu().numpy().view(np.uint16)
         assert np.array_equal(out, ws[k])
+
+
+def test_offload_pipeline_decodes_every_layer_bit_exact():
+    """Layers packed in pinned host memory, copied and decoded through two
+    device slots; every layer's output checked right after its decode, and
+    a second run of the same pipeline."""
+    from huffman_decode_df11_b200 import offload
+    rng = np.random.default_rng(5)
+    layers = []
+    for i in range(5):  # sizes differ, so the slots are reused at several offsets
+        ws = [workloads.as_numpy_u16(workloads.gaussian_bf16(int(rng.integers(1, 400_000)),
+                                                             0.02, 20 + 3 * i + j))
+              for j in range(3)]
+        if i == 2:
+            ws.append(workloads.as_numpy_u16(workloads.adversarial_mix(1 << 18, 7)))
+        layers.append(ws)
+    packed = [offload.pack_layer([df11.compress(w) for w in ws]) for ws in layers]
+    # one scratch buffer for every layer; outputs start 16-byte aligned
+    scratch = torch.empty(max(sum(len(w) + 8 for w in ws) for ws in layers),
+                          dtype=torch.int16, device="cuda")
+    outs = []
+    for ws in layers:
+        off, o = 0, []
+        for w in ws:
+            o.append(scratch[off:off + len(w)])
+            off = (off + len(w) + 7) // 8 * 8
+        outs.append(o)
+    pipe = offload.OffloadPipeline(packed, outs)
+    err = df11.new_error_word()
+    got = {}
+
+    def check(i):  # copies the layer's output before the next decode overwrites it
+        got[i] = [o.clone() for o in outs[i]]
+
+    for _ in range(2):
+        got.clear()
+        pipe.run(err=err, after_layer=check)
+        torch.cuda.synchronize()
+        df11.check_device_error(err)
+        for i, ws in enumerate(layers):
+            for o, w in zip(got[i], ws):
+                assert np.array_equal(o.cpu().numpy().view(np.uint16), w)
+    assert pipe.h2d_bytes == sum(p.nbytes for p in packed)
