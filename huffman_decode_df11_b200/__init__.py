@@ -127,6 +127,14 @@ def lib():
     L.df11_host_tensor_free.argtypes = [ctypes.POINTER(HostTensor)]
     L.df11_build_decode_table.argtypes = [vp, vp, u32, vp, vp]
     L.df11_build_decode_table.restype = ctypes.c_int
+    L.df11_gpu_build_begin.argtypes = [vp, u64, u32, u32, vp, ctypes.POINTER(Params), vp,
+                                       ctypes.POINTER(vp)]
+    L.df11_gpu_build_begin.restype = ctypes.c_int
+    L.df11_gpu_build_finish.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                        ctypes.POINTER(Params), vp]
+    L.df11_gpu_build_finish.restype = ctypes.c_int
+    L.df11_gpu_build_free.argtypes = [vp]
+    L.df11_gpu_build_free.restype = None
     _lib = L
     return L
 
@@ -286,6 +294,58 @@ def to_device(h: Df11Host, device="cuda", decode_table: bool = True) -> Df11Devi
     )
     if decode_table:
         d.decode_table = build_decode_table(d)
+    return d
+
+
+def compress_on_device(w: torch.Tensor, chunk_bytes: int = 24, threads_per_block: int = 256,
+                       stream=None, decode_table: bool = True) -> Df11Device:
+    """Encode a BF16 tensor that is in device memory into DF11 on the device
+    (df11_gpu_build_begin / df11_gpu_build_finish): the same bytes and
+    parameters as compress() of the same words, written straight into
+    device buffers.  Synchronises the stream."""
+    if not w.is_cuda:
+        raise ValueError("compress_on_device takes a CUDA tensor; use compress() for host data")
+    if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected BF16 words (bfloat16, int16 or uint16), got {w.dtype}")
+    shape = tuple(w.shape)
+    flat = w.contiguous().reshape(-1)
+    n = flat.numel()
+    ptr = flat.data_ptr() if n else None
+    L = lib()
+    sh = _stream_handle(stream)
+    p = Params()
+    lens = (ctypes.c_uint8 * 256)()
+    handle = ctypes.c_void_p()
+    _check(L.df11_gpu_build_begin(ptr, n, chunk_bytes, threads_per_block, sh, ctypes.byref(p),
+                                  ctypes.cast(lens, ctypes.c_void_p), ctypes.byref(handle)),
+           "df11_gpu_build_begin")
+    try:
+        chunks = int(p.num_blocks) * threads_per_block
+        dev = w.device
+
+        def buf(count, dtype=torch.uint8):
+            # at least 16 bytes so that no pointer is NULL; the view has `count`
+            t = torch.empty(max(count, 16), dtype=dtype, device=dev)
+            return t, t[:count]
+
+        bs, bs_v = buf(chunks * chunk_bytes + 16)
+        gp, gp_v = buf(chunks * 5 // 8 + 16)
+        cc, cc_v = buf(chunks + 16)
+        bp, bp_v = buf(int(p.num_blocks) + 1, torch.int32)
+        lu, lu_v = buf(int(p.num_luts) * 256, torch.int32)
+        cl, cl_v = buf(256)
+        sm, sm_v = buf((n + 15) // 16 * 16)
+    except BaseException:
+        L.df11_gpu_build_free(handle)
+        raise
+    st = L.df11_gpu_build_finish(handle, ptr, bs.data_ptr(), gp.data_ptr(), cc.data_ptr(),
+                                 bp.data_ptr(), lu.data_ptr(), cl.data_ptr(), sm.data_ptr(),
+                                 ctypes.byref(p), sh)
+    _check(st, "df11_gpu_build_finish")
+    d = Df11Device(params=p, bitstream=bs_v, gaps=gp_v, block_out_pos=bp_v, luts=lu_v,
+                   code_lengths=cl_v, sign_mantissa=sm_v, chunk_counts=cc_v, shape=shape)
+    if decode_table:
+        d.decode_table = build_decode_table(d, stream)
     return d
 
 

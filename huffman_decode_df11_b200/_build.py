@@ -1,5 +1,5 @@
-"""Build step for libdf11.so: the sm_100a decode kernel, its C ABI and the host
-format builder, compiled in-tree with nvcc (no GPU needed to build).
+"""Build step for libdf11.so: the sm_100a decode kernels, their C ABI, and the
+host and device format builders, compiled in-tree with nvcc (no GPU needed to build).
 
     python -m huffman_decode_df11_b200._build [--force]
 """
@@ -14,8 +14,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdf11.so")
-SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_build.cpp")]
-HEADERS = [os.path.join(INCLUDE, "df11.h")]
+SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_gpu_build.cu"),
+           os.path.join(CSRC, "df11_build.cpp")]
+HEADERS = [os.path.join(INCLUDE, "df11.h"), os.path.join(CSRC, "df11_codebook.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

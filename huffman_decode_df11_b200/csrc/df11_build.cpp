@@ -28,6 +28,7 @@
 #include <vector>
 
 #include "df11.h"
+#include "df11_codebook.h"
 
 namespace {
 
@@ -252,6 +253,15 @@ std::vector<uint32_t> build_tables(const uint8_t len[256], const uint32_t code[2
 
 }  // namespace
 
+int df11_internal::codebook(const uint64_t hist[256], uint8_t len[256], uint32_t code[256],
+                            std::vector<uint32_t> &luts) {
+  int longest = huffman_depths(hist, len);
+  if (longest > kMaxLen) longest = package_merge(hist, kMaxLen, len);
+  canonical(len, code);
+  luts = build_tables(len, code);
+  return longest;
+}
+
 extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
                                   uint32_t T, int num_threads,
                                   df11_host_tensor *out) {
@@ -281,16 +291,12 @@ extern "C" df11_status df11_build(const uint16_t *w, uint64_t n, uint32_t C,
   for (auto &p : part)
     for (int s = 0; s < 256; ++s) hist[s] += p[s];
 
-  // 3-4. code
+  // 3-5. code and tables
   uint8_t len[256];
-  int longest = huffman_depths(hist, len);
-  if (longest > kMaxLen) longest = package_merge(hist, kMaxLen, len);
   uint32_t code[256];
-  canonical(len, code);
+  std::vector<uint32_t> luts;
+  const int longest = df11_internal::codebook(hist, len, code, luts);
   std::memcpy(out->code_lengths, len, 256);
-
-  // 5. tables
-  std::vector<uint32_t> luts = build_tables(len, code);
   df11_params &p = out->params;
   p.n = n;
   p.chunk_bytes = C;

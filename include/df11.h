@@ -227,6 +227,58 @@ df11_status df11_build(const uint16_t *bf16, uint64_t n, uint32_t chunk_bytes,
                        df11_host_tensor *out);
 void df11_host_tensor_free(df11_host_tensor *t);
 
+/* ---------------------------------------------------------------------- */
+/* Device-side format builder: the same encoding, byte for byte, of BF16  */
+/* words already in device memory.                                        */
+/*                                                                        */
+/* The pages build the format offline on the host ("DFloat11无损压缩技术"  */
+/* (jsqmd.com) §2.2 items 1-2).  Here histogram, bit offsets, packing,    */
+/* gaps, block positions and counts run on the device; the codebook (256  */
+/* symbols) on the host.  Two calls, so that the caller allocates the     */
+/* output buffers once their sizes are known.                             */
+
+typedef struct df11_gpu_build df11_gpu_build;
+
+/*
+ * Phase 1.  d_bf16: n BF16 words in device memory (2-byte aligned; 16-byte
+ * alignment lets the kernels load 8 words at a time and must then hold in
+ * phase 2 too).  Same chunk_bytes / threads_per_block rules as df11_build.
+ * Computes the histogram and the code, synchronises `stream`, and on
+ * success fills *params (n, total_bits, chunk_bytes, threads_per_block,
+ * num_blocks, num_luts, max_len; the max_* counts are filled by phase 2),
+ * code_lengths (host, 256 bytes) and *handle, which holds device scratch
+ * until phase 2 or df11_gpu_build_free.  The buffers phase 2 writes, with
+ * C = chunk_bytes, T = threads_per_block, B = num_blocks:
+ *   bitstream      B*T*C + 16 bytes       gaps           B*T*5/8 + 16 bytes
+ *   chunk_counts   B*T + 16 bytes         block_out_pos  (B + 1) uint32
+ *   luts           num_luts*256 uint32    code_lengths   256 bytes
+ *   sign_mantissa  n rounded up to 16 bytes
+ * Errors: DF11_ERR_NULL, _INVALID, _TOO_LARGE, _ALIGN, _NOMEM before any
+ * device work; DF11_ERR_CUDA if a CUDA call fails.  *handle is NULL on
+ * every error.
+ */
+df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t chunk_bytes,
+                                 uint32_t threads_per_block, df11_stream_t stream,
+                                 df11_params *params, uint8_t code_lengths[256],
+                                 df11_gpu_build **handle);
+
+/*
+ * Phase 2.  Writes the encoded tensor into caller-owned device buffers of
+ * the sizes above (bitstream, gaps, chunk_counts, luts, sign_mantissa
+ * 16-byte aligned; block_out_pos 4-byte aligned), from the same d_bf16,
+ * on `stream`, and synchronises it.  On success *params is complete and
+ * equal to what df11_build returns for the same words.  Releases the
+ * handle in every case (success or error).
+ */
+df11_status df11_gpu_build_finish(df11_gpu_build *handle, const uint16_t *d_bf16,
+                                  uint8_t *bitstream, uint8_t *gaps, uint8_t *chunk_counts,
+                                  uint32_t *block_out_pos, uint32_t *luts,
+                                  uint8_t *code_lengths, uint8_t *sign_mantissa,
+                                  df11_params *params, df11_stream_t stream);
+
+/* Release a phase-1 handle without running phase 2 (NULL is a no-op). */
+void df11_gpu_build_free(df11_gpu_build *handle);
+
 #ifdef __cplusplus
 }
 #endif

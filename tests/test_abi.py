@@ -107,6 +107,34 @@ def test_decode_table_host_validation():
     assert L.df11_build_decode_table(FAKE, FAKE, 1 << 24, FAKE, None) == 3
 
 
+def test_device_builder_host_validation():
+    """Phase 1 rejects bad arguments before any CUDA call; phase 2 rejects a
+    NULL handle; freeing NULL is a no-op."""
+    L = df11.lib()
+    p = df11.Params()
+    lens = (ctypes.c_uint8 * 256)()
+    lp = ctypes.cast(lens, ctypes.c_void_p)
+    h = ctypes.c_void_p(123)
+    assert L.df11_gpu_build_begin(None, 10, 24, 256, None, ctypes.byref(p), lp,
+                                  ctypes.byref(h)) == 1
+    assert h.value is None  # cleared even on error
+    assert L.df11_gpu_build_begin(FAKE, 10, 24, 256, None, None, lp, ctypes.byref(h)) == 1
+    assert L.df11_gpu_build_begin(FAKE, 10, 6, 256, None, ctypes.byref(p), lp,
+                                  ctypes.byref(h)) == 7   # C not a multiple of 4
+    assert L.df11_gpu_build_begin(FAKE, 10, 32, 256, None, ctypes.byref(p), lp,
+                                  ctypes.byref(h)) == 7   # counts would not fit a byte
+    assert L.df11_gpu_build_begin(FAKE, 10, 24, 200, None, ctypes.byref(p), lp,
+                                  ctypes.byref(h)) == 7
+    assert L.df11_gpu_build_begin(FAKE, 1 << 32, 24, 256, None, ctypes.byref(p), lp,
+                                  ctypes.byref(h)) == 6
+    assert L.df11_gpu_build_begin(FAKE + 1, 10, 24, 256, None, ctypes.byref(p), lp,
+                                  ctypes.byref(h)) == 2
+    assert L.df11_gpu_build_finish(None, *[FAKE] * 8, ctypes.byref(p), None) == 1
+    L.df11_gpu_build_free(None)
+    with pytest.raises(ValueError):
+        df11.compress_on_device(df11.torch.zeros(4, dtype=df11.torch.int16))
+
+
 def test_supported_shapes_and_shared_bytes():
     assert df11.supported(8, 256) and df11.supported(4, 256) and df11.supported(16, 256)
     assert df11.supported(24, 256) and not df11.supported(20, 256)

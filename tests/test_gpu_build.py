@@ -1,0 +1,139 @@
+"""Device-side format builder (df11_gpu_build_begin / _finish) against the
+host builder and the oracle.
+
+Byte identity is the bar: every buffer and every parameter the device
+builder writes must equal what the host builder writes for the same words
+(the host builder is itself pinned to the oracle's encoder in
+test_builder_vs_oracle.py), and the result must decode to the original
+words.  Cases cover several pack blocks with a ragged tail, the empty and
+one-element tensors, one exponent only, 8-bit codes, the multi-level tables
+of the adversarial mix, 32-bit codewords, every chunk size the format
+allows, and input that is not 16-byte aligned (the scalar load path).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+df11 = pytest.importorskip("huffman_decode_df11_b200")
+
+_BUFFERS = ("bitstream", "gaps", "chunk_counts", "block_out_pos", "luts", "code_lengths",
+            "sign_mantissa")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def _host_bytes(h, f):
+    return np.ascontiguousarray(getattr(h, f)).view(np.uint8)
+
+
+def _same_as_host(bits: torch.Tensor, C=24, T=256):
+    """Build on the device from `bits` (a CUDA tensor of BF16 words) and
+    compare with the host builder; returns the device tensor."""
+    w_np = workloads.as_numpy_u16(bits.cpu())
+    h = df11.compress(w_np, C, T)
+    d = df11.compress_on_device(bits, C, T)
+    torch.cuda.synchronize()
+    for f, _ in df11.Params._fields_:
+        assert getattr(d.params, f) == getattr(h.params, f), f
+    for f in _BUFFERS:
+        got = getattr(d, f).cpu().numpy().view(np.uint8)
+        want = _host_bytes(h, f)
+        assert got.shape == want.shape, f
+        assert np.array_equal(got, want), f
+    assert d.shape == tuple(bits.shape)
+    return d, h, w_np
+
+
+def _decodes_to(d, w_np):
+    err = df11.new_error_word()
+    out = df11.decode(d, err=err)
+    torch.cuda.synchronize()
+    df11.check_device_error(err)
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), w_np)
+
+
+@pytest.mark.parametrize("n", [0, 1, 2, 7, 8, 9, 2047, 2048, 2049, 3 * 2048 + 77, 1_000_003])
+def test_gaussian_sizes(n):
+    bits = workloads.gaussian_bf16(n, 0.02, 500 + n, device="cuda")
+    d, h, w = _same_as_host(bits)
+    if n:
+        _decodes_to(d, w)
+
+
+@pytest.mark.parametrize("C,T", [(4, 128), (8, 256), (16, 256), (24, 256), (28, 1024),
+                                 (8, 512)])
+def test_chunk_and_block_sizes(C, T):
+    bits = workloads.gaussian_bf16(777_777, 0.02, C * 1000 + T, device="cuda")
+    d, h, w = _same_as_host(bits, C, T)
+    if df11.supported(C, T):
+        _decodes_to(d, w)
+
+
+def test_matches_the_oracle_encoder():
+    bits = workloads.adversarial_mix(1 << 18, 21, device="cuda")
+    d, h, w = _same_as_host(bits, 8, 256)
+    o = oracle.encode(w, 8, 256)
+    assert np.array_equal(d.bitstream.cpu().numpy(), o.bitstream)
+    assert np.array_equal(d.code_lengths.cpu().numpy(), o.code_lengths)
+
+
+def test_adversarial_multilevel_tables():
+    bits = workloads.adversarial_mix(1 << 22, 4, device="cuda")
+    d, h, w = _same_as_host(bits)
+    assert d.params.num_luts > 1
+    _decodes_to(d, w)
+
+
+def test_fibonacci_32_bit_codewords():
+    bits = workloads.fibonacci_exponents(0, device="cuda")
+    d, h, w = _same_as_host(bits)
+    assert d.params.max_len == 32
+    _decodes_to(d, w)
+
+
+def test_every_bf16_pattern_and_one_exponent():
+    d, h, w = _same_as_host(workloads.all_bf16_patterns(device="cuda"))
+    _decodes_to(d, w)
+    one = torch.full((12345,), 0x3F80, dtype=torch.int16, device="cuda")
+    d, h, w = _same_as_host(one)
+    assert d.params.max_len == 1
+    _decodes_to(d, w)
+
+
+def test_unaligned_input_takes_the_scalar_loads():
+    base = workloads.gaussian_bf16(300_001, 0.02, 9, device="cuda")
+    view = base[3:]  # 6 bytes past a 16-byte boundary
+    assert view.data_ptr() % 16
+    d, h, w = _same_as_host(view)
+    _decodes_to(d, w)
+
+
+def test_bf16_dtype_and_shape_kept():
+    x = torch.randn(333, 517, device="cuda", dtype=torch.float32).mul_(0.02).to(torch.bfloat16)
+    d = df11.compress_on_device(x)
+    assert d.shape == (333, 517)
+    out = df11.decode(d)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16).view(333, 517), x.view(torch.int16))
+
+
+def test_argument_errors():
+    x = workloads.gaussian_bf16(1000, 0.02, 1, device="cuda")
+    with pytest.raises(df11.Df11Error):
+        df11.compress_on_device(x, chunk_bytes=6)
+    with pytest.raises(df11.Df11Error):
+        df11.compress_on_device(x, threads_per_block=200)
+    with pytest.raises(ValueError):
+        df11.compress_on_device(x.cpu())
+    with pytest.raises(TypeError):
+        df11.compress_on_device(x.float())
