@@ -6,24 +6,34 @@
 // §2.2 items 1-2 give the recipe; "DFloat11重新定义LLM无损压缩的技术边界"
 // (ocdem.com) §2.2 the lookup tables).  Here every step that touches the n
 // elements runs on the device; only the codebook, a function of 256 counts,
-// is computed on the host (df11_codebook.h, shared with the host builder):
-//   histogram  exponent counts: per-warp shared counters, lanes holding the
-//              same exponent combined with a match before one atomic add;
-//   sums       the code-length total of every pack block (2048 elements);
-//              their exclusive scan on the host gives each pack block its
-//              first bit;
-//   pack       a pack block scans its threads' bit counts, ORs every
-//              codeword into a shared-memory image of its words, then
-//              writes the words out coalesced: plain stores for the words
-//              wholly its own, atomic OR for its first and last word, which
-//              the neighbouring pack blocks share.  Each thread also writes
-//              its 8 sign/mantissa bytes and, for every chunk and block
-//              whose first codeword start is one of its elements, the gap,
-//              the first element and the block position;
+// is computed on the host (df11_codebook.h, shared with the host builder).
+// The elements are cut into pack blocks of 2048 (8 per thread of a
+// 256-thread block); the kernels, in stream order:
+//   histogram  exponent counts, one pass: counters in registers for a
+//              window of 16 exponents around the mode of a first sample,
+//              summed over the warp now and then; shared counters for the
+//              rest;
+//   sums       the code-length total of every pack block.  Each thread
+//              block walks a contiguous range of pack blocks and keeps a
+//              running total, so it writes every pack block's first bit
+//              relative to its range, and the range's total;
+//   scan       the ranges' first bits (one thread block; at most a few
+//              thousand ranges) and the stream's total, which the host
+//              reads to size the outputs;
+//   prepare    chunk first elements preset to n, gaps and maxima cleared,
+//              the bitstream words two pack blocks share cleared;
+//   pack       persistent: per pack block, a block scan of the threads' bit
+//              counts, every codeword ORed into a shared-memory image of the
+//              block's words, the words written out coalesced (atomic OR
+//              for the first and last word when a neighbour owns part of
+//              it), the sign/mantissa bytes, and for every chunk and block
+//              whose first codeword start is one of the thread's elements
+//              the gap, first element and block position; the next pack
+//              block's words are loaded while this one is packed;
 //   finish     the chunks and blocks after the last codeword start, chunk
-//              counts from first-element differences, the gaps packed eight
-//              to five bytes, and the largest block, chunk and group of 32
-//              chunks.
+//              counts from first-element differences, the gaps packed
+//              eight to five bytes, and the largest block, chunk and group
+//              of 32 chunks.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -45,23 +55,79 @@ constexpr int kPerCta = kThreads * kPerThread;  // elements per pack block
 constexpr int kCtaWords = kPerCta + 1;
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
-__device__ __forceinline__ uint32_t exponent(uint16_t x) { return (x >> 7) & 0xFFu; }
+__device__ __forceinline__ uint32_t exponent(uint32_t x) { return (x >> 7) & 0xFFu; }
 
-// the 8 words of elements i0 .. i0+7 (zero past n)
-__device__ __forceinline__ void load8(const uint16_t *w, uint64_t n, uint64_t i0, bool vec,
-                                      uint16_t x[kPerThread]) {
-  if (vec && i0 + kPerThread <= n) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(w + i0);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+// The 8 words of elements i0 .. i0+7, two per 32-bit lane (element i0+2k in
+// the low half of the k-th of .x .y .z .w); zero past n.
+__device__ __forceinline__ uint4 load8(const uint16_t *w, uint64_t n, uint64_t i0, bool vec) {
+  if (vec && i0 + kPerThread <= n) return __ldg(reinterpret_cast<const uint4 *>(w + i0));
+  uint32_t u[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      x[2 * k] = (uint16_t)(u[k] & 0xFFFFu);
-      x[2 * k + 1] = (uint16_t)(u[k] >> 16);
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < kPerThread; ++k) x[k] = i0 + k < n ? w[i0 + k] : 0;
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t a = i0 + 2 * k < n ? w[i0 + 2 * k] : 0u;
+    const uint32_t b = i0 + 2 * k + 1 < n ? w[i0 + 2 * k + 1] : 0u;
+    u[k] = a | (b << 16);
   }
+  return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+__device__ __forceinline__ uint32_t exponent_of(const uint4 &v, int k) {
+  const uint32_t u = (k >> 1) == 0 ? v.x : (k >> 1) == 1 ? v.y : (k >> 1) == 2 ? v.z : v.w;
+  return (u >> ((k & 1) ? 23 : 7)) & 0xFFu;
+}
+
+// how many of elements i0 .. i0+7 exist (0..8)
+__device__ __forceinline__ uint32_t live_of(uint64_t i0, uint64_t n) {
+  return i0 >= n ? 0u : (n - i0 >= (uint64_t)kPerThread ? (uint32_t)kPerThread : (uint32_t)(n - i0));
+}
+
+// ---- histogram -----------------------------------------------------------
+// Per lane, 16 four-bit counters in one 64-bit register take the 8 elements
+// of a tile whose exponent falls in the warp's window (mode - 11 .. mode + 4);
+// after each tile they are spread into byte counters (four registers), and
+// those are summed over the warp into shared counters every 31 tiles
+// (at most 248 counts per byte).  Exponents outside the window go to the
+// shared counters at once.
+constexpr int kWindow = 16;
+constexpr int kWindowBelow = 11;
+constexpr int kFlushTiles = 31;
+
+// byte j of counter register r holds window bin (r >> 1) * 8 + 2 j + (r & 1)
+__device__ __forceinline__ void flush_window(uint32_t (&c)[4], int lo, uint32_t *h, int lane) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    // two 16-bit sums per word: 32 lanes x 248 < 2^16
+    const uint32_t even = __reduce_add_sync(0xFFFFFFFFu, c[r] & 0x00FF00FFu);
+    const uint32_t odd = __reduce_add_sync(0xFFFFFFFFu, (c[r] >> 8) & 0x00FF00FFu);
+    if (lane == 0) {
+      const uint32_t v[4] = {even & 0xFFFFu, odd & 0xFFFFu, even >> 16, odd >> 16};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = lo + (r >> 1) * 8 + 2 * j + (r & 1);
+        if (v[j] && e >= 0 && e < 256) atomicAdd(&h[e], v[j]);
+      }
+    }
+    c[r] = 0;
+  }
+}
+
+__device__ __forceinline__ void count8(const uint4 &v, uint32_t live, int lo, uint32_t (&c)[4],
+                                       uint32_t *h) {
+  unsigned long long nib = 0;
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    if ((uint32_t)k < live) {
+      const uint32_t e = exponent_of(v, k);
+      const uint32_t d = (uint32_t)((int)e - lo);
+      if (d < (uint32_t)kWindow) nib += 1ull << (4 * d);
+      else atomicAdd(&h[e], 1u);
+    }
+  }
+  const uint32_t n_lo = (uint32_t)nib, n_hi = (uint32_t)(nib >> 32);
+  c[0] += n_lo & 0x0F0F0F0Fu;
+  c[1] += (n_lo >> 4) & 0x0F0F0F0Fu;
+  c[2] += n_hi & 0x0F0F0F0Fu;
+  c[3] += (n_hi >> 4) & 0x0F0F0F0Fu;
 }
 
 __global__ void __launch_bounds__(kThreads) hist_kernel(const uint16_t *w, uint64_t n, bool vec,
@@ -69,175 +135,364 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const uint16_t *w, uint6
   __shared__ uint32_t h[kThreads / 32][256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int j = threadIdx.x; j < (kThreads / 32) * 256; j += kThreads) (&h[0][0])[j] = 0;
-  __syncthreads();
   const uint64_t stride = (uint64_t)gridDim.x * kPerCta;
+  uint64_t base = (uint64_t)blockIdx.x * kPerCta;
+  const uint64_t me = (uint64_t)threadIdx.x * kPerThread;
+  uint4 next = load8(w, n, base + me, vec);
+  // the window: around the most frequent exponent among the warp's lanes'
+  // first elements
+  int lo;
+  {
+    const uint32_t key = base + me < n ? exponent(next.x & 0xFFFFu) : 256u;
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
+    const uint32_t best = __reduce_max_sync(0xFFFFFFFFu, ((uint32_t)__popc(peers) << 16) | key);
+    lo = (int)(best & 0x1FFu) - kWindowBelow;
+  }
+  __syncthreads();
+  uint32_t c[4] = {0, 0, 0, 0};
+  int tiles = 0;
   // `base` is the same for every thread of the block: whole warps iterate
-  for (uint64_t base = (uint64_t)blockIdx.x * kPerCta; base < n; base += stride) {
-    const uint64_t i0 = base + (uint64_t)threadIdx.x * kPerThread;
-    uint16_t x[kPerThread];
-    load8(w, n, i0, vec, x);
-#pragma unroll
-    for (int k = 0; k < kPerThread; ++k) {
-      const bool live = i0 + k < n;
-      // 256 matches no exponent: lanes past the end group apart
-      const uint32_t key = live ? exponent(x[k]) : 256u;
-      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
-      if (live && lane == __ffs(peers) - 1) atomicAdd(&h[warp][key], (uint32_t)__popc(peers));
+  for (; base < n; base += stride) {
+    const uint4 v = next;
+    if (base + stride < n) next = load8(w, n, base + stride + me, vec);
+    count8(v, live_of(base + me, n), lo, c, h[warp]);
+    if (++tiles == kFlushTiles) {
+      flush_window(c, lo, h[warp], lane);
+      tiles = 0;
     }
   }
+  flush_window(c, lo, h[warp], lane);
   __syncthreads();
   uint32_t s = 0;
   for (int j = 0; j < kThreads / 32; ++j) s += h[j][threadIdx.x];
   if (s) atomicAdd(&hist[threadIdx.x], (unsigned long long)s);
 }
 
-// code-length total of each pack block's elements
-__global__ void __launch_bounds__(kThreads) sums_kernel(const uint16_t *w, uint64_t n, bool vec,
-                                                        const uint2 *tab,
-                                                        unsigned long long *cta_bits) {
+// ---- bit offsets ---------------------------------------------------------
+constexpr int kSumsBlocks = 4;  // pack blocks per iteration of the sums kernel
+
+struct Ranges {
+  uint64_t pack_ctas;  // pack blocks
+  uint64_t per;        // pack blocks per range (one range per sums thread block)
+  uint32_t *local;     // first bit of each pack block within its range
+  unsigned long long *range_start;  // first bit of each range; the total after the last
+};
+
+// pack blocks and ranges number below 2^21: 32-bit division
+__device__ __forceinline__ unsigned long long pack_start(const Ranges &r, uint64_t pb) {
+  return r.range_start[(uint32_t)pb / (uint32_t)r.per] + r.local[pb];
+}
+
+__global__ void __launch_bounds__(kThreads, 4) sums_kernel(const uint16_t *w, uint64_t n, bool vec,
+                                                        const uint2 *tab, const Ranges r,
+                                                        unsigned long long *range_total) {
   __shared__ uint8_t len[256];
-  __shared__ uint32_t part[kThreads / 32];
+  __shared__ uint32_t part[kSumsBlocks][kThreads / 32];
   len[threadIdx.x] = (uint8_t)tab[threadIdx.x].y;
-  __syncthreads();
-  const uint64_t i0 = (uint64_t)blockIdx.x * kPerCta + (uint64_t)threadIdx.x * kPerThread;
-  uint16_t x[kPerThread];
-  load8(w, n, i0, vec, x);
-  uint32_t s = 0;
+  const uint64_t pb_begin = (uint64_t)blockIdx.x * r.per;
+  const uint64_t pb_end = pb_begin + r.per < r.pack_ctas ? pb_begin + r.per : r.pack_ctas;
+  const uint64_t me = (uint64_t)threadIdx.x * kPerThread;
+  uint4 next[kSumsBlocks];
 #pragma unroll
-  for (int k = 0; k < kPerThread; ++k)
-    if (i0 + k < n) s += len[exponent(x[k])];
-  s = __reduce_add_sync(0xFFFFFFFFu, s);
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  for (int j = 0; j < kSumsBlocks; ++j)
+    next[j] = pb_begin + j < pb_end ? load8(w, n, (pb_begin + j) * kPerCta + me, vec)
+                                    : make_uint4(0, 0, 0, 0);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned long long t = 0;
-    for (int j = 0; j < kThreads / 32; ++j) t += part[j];
-    cta_bits[blockIdx.x] = t;
+  uint32_t running = 0;  // thread 0: bits of the range so far
+  for (uint64_t pb = pb_begin; pb < pb_end; pb += kSumsBlocks) {
+    uint4 v[kSumsBlocks];
+#pragma unroll
+    for (int j = 0; j < kSumsBlocks; ++j) {
+      v[j] = next[j];
+      const uint64_t q = pb + kSumsBlocks + j;
+      if (q < pb_end) next[j] = load8(w, n, q * kPerCta + me, vec);
+    }
+#pragma unroll
+    for (int j = 0; j < kSumsBlocks; ++j) {
+      const uint32_t live = pb + j < pb_end ? live_of((pb + j) * kPerCta + me, n) : 0u;
+      uint32_t s = 0;
+#pragma unroll
+      for (int k = 0; k < kPerThread; ++k)
+        if ((uint32_t)k < live) s += len[exponent_of(v[j], k)];
+      s = __reduce_add_sync(0xFFFFFFFFu, s);
+      if ((threadIdx.x & 31) == 0) part[j][threadIdx.x >> 5] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int j = 0; j < kSumsBlocks && pb + j < pb_end; ++j) {
+        uint32_t t = 0;
+        for (int k = 0; k < kThreads / 32; ++k) t += part[j][k];
+        r.local[pb + j] = running;
+        running += t;
+      }
+    }
+    __syncthreads();  // part is rewritten next iteration
+  }
+  if (threadIdx.x == 0) range_total[blockIdx.x] = running;
+}
+
+// Exclusive scan of the range totals into the ranges' first bits, the total
+// at starts[count]; one thread block, each thread a contiguous run.
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const unsigned long long *totals,
+                                                            uint64_t count,
+                                                            unsigned long long *starts) {
+  __shared__ unsigned long long warp_tot[kScanThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint64_t per = (count + kScanThreads - 1) / kScanThreads;
+  const uint64_t b = threadIdx.x * per;
+  const uint64_t e = b + per < count ? b + per : count;
+  unsigned long long mine = 0;
+  for (uint64_t i = b; i < e; ++i) mine += totals[i];
+  unsigned long long incl = mine;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  unsigned long long run = incl - mine;
+  for (int j = 0; j < warp; ++j) run += warp_tot[j];
+  for (uint64_t i = b; i < e; ++i) {
+    starts[i] = run;
+    run += totals[i];
+  }
+  if (threadIdx.x == kScanThreads - 1) starts[count] = run;
+}
+
+// Before packing: first elements preset to n, gaps cleared, the bitstream
+// words that two pack blocks share cleared (they are ORed into), maxima
+// cleared.
+__global__ void prepare_kernel(uint32_t *first_elem, uint8_t *gap, uint64_t chunks, uint32_t n,
+                               const Ranges r, uint32_t *bs32, unsigned int *maxima) {
+  const uint64_t all = chunks + 1 > r.pack_ctas ? chunks + 1 : r.pack_ctas;
+  for (uint64_t i = blockIdx.x * 256ull + threadIdx.x; i < all; i += (uint64_t)gridDim.x * 256) {
+    if (i <= chunks) {
+      first_elem[i] = n;
+      gap[i] = 0;
+    }
+    if (i >= 1 && i < r.pack_ctas) {
+      const unsigned long long s = pack_start(r, i);
+      if (s & 31u) bs32[s >> 5] = 0;
+    }
+    if (i < 3) maxima[i] = 0;
   }
 }
 
-__global__ void fill_u32(uint32_t *p, uint64_t count, uint32_t v) {
-  for (uint64_t i = blockIdx.x * 256ull + threadIdx.x; i < count; i += (uint64_t)gridDim.x * 256)
-    p[i] = v;
-}
-
+// ---- pack ----------------------------------------------------------------
 struct PackArgs {
   const uint16_t *w;
   uint64_t n;
-  bool vec;                            // w is 16-byte aligned
-  const uint2 *tab;                    // {codeword, length} per exponent
-  const unsigned long long *cta_bits;  // first bit of each pack block
-  uint32_t *bs32;                      // bitstream as 32-bit words, zeroed
-  uint8_t *sm;                         // 16-byte aligned
-  uint8_t *gap;                        // one byte per chunk
-  uint32_t *first_elem;                // chunks + 1, preset to n
+  bool vec;             // w is 16-byte aligned
+  const uint2 *tab;     // {codeword, length} per exponent
+  Ranges r;
+  uint32_t *bs32;       // bitstream as 32-bit words
+  uint8_t *sm;          // 16-byte aligned
+  uint8_t *gap;         // one byte per chunk
+  uint32_t *first_elem; // chunks + 1, preset to n
   uint32_t *bpos;
-  uint64_t chunk_bits, chunks, block_bits;
+  uint64_t chunks;
   uint32_t num_blocks;
+  uint32_t chunk_bits, block_bits;    // 8 C and 8 C T
+  uint32_t chunk_words, block_words;  // chunk_bits / 32, block_bits / 32
+  float inv_chunk, inv_block;         // 1 / chunk_bits, 1 / block_bits
 };
+
+// floor(x / d) for |x| < 2^20 from a float estimate, corrected to exact
+__device__ __forceinline__ int floor_div(int x, int d, float inv) {
+  int j = __float2int_rd((float)x * inv);
+  if (j * d > x) --j;
+  if ((j + 1) * d <= x) ++j;
+  return j;
+}
 
 __global__ void __launch_bounds__(kThreads) pack_kernel(const PackArgs a) {
   __shared__ uint32_t code[256];
   __shared__ uint8_t len[256];
   __shared__ uint32_t warp_sum[kThreads / 32];
+  __shared__ uint8_t last_len[kThreads];  // length of each thread's last codeword
+  __shared__ long long bound[4];          // first chunk and block at or before the origin
   __shared__ uint32_t words[kCtaWords];
   const uint2 t = a.tab[threadIdx.x];
   code[threadIdx.x] = t.x;
   len[threadIdx.x] = (uint8_t)t.y;
   for (int j = threadIdx.x; j < kCtaWords; j += kThreads) words[j] = 0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint64_t i0 = (uint64_t)blockIdx.x * kPerCta + (uint64_t)threadIdx.x * kPerThread;
-  uint16_t x[kPerThread];
-  load8(a.w, a.n, i0, a.vec, x);
-  __syncthreads();
-  uint32_t mine = 0;
-#pragma unroll
-  for (int k = 0; k < kPerThread; ++k)
-    if (i0 + k < a.n) mine += len[exponent(x[k])];
-  uint32_t incl = mine;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-    if (lane >= d) incl += v;
+  const uint64_t me = (uint64_t)threadIdx.x * kPerThread;
+  const uint64_t pack_ctas = a.r.pack_ctas;
+  uint64_t pb = blockIdx.x;
+  // pack block pb's words, first bit and previous element (thread 0)
+  uint4 nx = make_uint4(0, 0, 0, 0);
+  unsigned long long nstart = 0;
+  uint32_t nprev = 0;
+  if (pb < pack_ctas) {
+    nx = load8(a.w, a.n, pb * kPerCta + me, a.vec);
+    nstart = pack_start(a.r, pb);
+    if (threadIdx.x == 0 && pb) nprev = a.w[pb * kPerCta - 1];
   }
-  if (lane == 31) warp_sum[warp] = incl;
   __syncthreads();
-  uint32_t before = 0, cta_total = 0;
+  for (; pb < pack_ctas; pb += gridDim.x) {
+    const uint4 v = nx;
+    const unsigned long long cta_start = nstart;
+    const uint32_t prev_word = nprev;
+    const uint64_t pn = pb + gridDim.x;
+    if (pn < pack_ctas) {
+      nx = load8(a.w, a.n, pn * kPerCta + me, a.vec);
+      nstart = pack_start(a.r, pn);
+      if (threadIdx.x == 0) nprev = a.w[pn * kPerCta - 1];
+    }
+    // bit positions below are relative to `origin`, the first bit of the
+    // word this pack block begins in
+    const unsigned long long origin = cta_start & ~31ull;
+    if (threadIdx.x == 0) {
+      const uint32_t ow = (uint32_t)(origin >> 5);  // < 2^32: bit offsets stay below 2^37
+      const uint64_t c0 = ow / a.chunk_words, q0 = ow / a.block_words;
+      bound[0] = (long long)c0;
+      bound[1] = (long long)(c0 * a.chunk_bits) - (long long)origin;
+      bound[2] = (long long)q0;
+      bound[3] = (long long)(q0 * a.block_bits) - (long long)origin;
+    }
+    const uint64_t i0 = pb * kPerCta + me;
+    const uint32_t live = live_of(i0, a.n);
+    uint32_t e[kPerThread], l[kPerThread];
+    uint32_t mine = 0, last = 0;
 #pragma unroll
-  for (int j = 0; j < kThreads / 32; ++j) {
-    const uint32_t v = warp_sum[j];
-    before += j < warp ? v : 0u;
-    cta_total += v;
-  }
-  const unsigned long long cta_start = a.cta_bits[blockIdx.x];
-  const uint32_t lead = (uint32_t)(cta_start & 31u);  // bits of the first word before the block
-  const uint32_t rel = lead + before + incl - mine;   // this thread's first bit in `words`
+    for (int k = 0; k < kPerThread; ++k) {
+      e[k] = exponent_of(v, k);
+      l[k] = (uint32_t)k < live ? (uint32_t)len[e[k]] : 0u;
+      mine += l[k];
+      last = (uint32_t)k < live ? l[k] : last;
+    }
+    uint32_t incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += u;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    last_len[threadIdx.x] = (uint8_t)last;
+    __syncthreads();
+    uint32_t before = 0, cta_total = 0;
+#pragma unroll
+    for (int j = 0; j < kThreads / 32; ++j) {
+      const uint32_t u = warp_sum[j];
+      before += j < warp ? u : 0u;
+      cta_total += u;
+    }
+    // length of element i0 - 1's codeword
+    const uint32_t prev_len = threadIdx.x ? last_len[threadIdx.x - 1]
+                                          : (pb ? len[exponent(prev_word)] : 0u);
+    const uint64_t c_org = (uint64_t)bound[0], q_org = (uint64_t)bound[2];
+    const int cr0 = (int)bound[1], qr0 = (int)bound[3];
+    const uint32_t lead = (uint32_t)(cta_start & 31u);  // bits of the first word before the block
+    const uint32_t rel = lead + before + incl - mine;   // this thread's first bit
 
-  // codewords, MSB first, into the shared image of the block's words
-  uint32_t wk = rel >> 5, nbits = rel & 31u;
-  unsigned long long acc = 0;
-  bool first = true;
+    // codewords, MSB first, ORed into the shared image of the block's words.
+    // Up to 64 bits (the usual case) are gathered in one register first and
+    // placed with at most three ORs; longer runs go word by word.
+    if (mine <= 64) {
+      unsigned long long acc = 0;
 #pragma unroll
-  for (int k = 0; k < kPerThread; ++k) {
-    if (i0 + k < a.n) {
-      const uint32_t s = exponent(x[k]), l = len[s];
-      acc = (acc << l) | code[s];
-      nbits += l;
-      while (nbits >= 32) {
-        const uint32_t v = (uint32_t)(acc >> (nbits - 32));
-        if (first) atomicOr(&words[wk], v);  // the previous thread may own its first bits
-        else words[wk] = v;
-        first = false;
-        ++wk;
-        nbits -= 32;
-        acc &= (1ull << nbits) - 1;
+      for (int k = 0; k < kPerThread; ++k)
+        acc = (acc << l[k]) | (l[k] ? code[e[k]] : 0u);
+      if (mine) {
+        const uint32_t o = rel & 31u, wk = rel >> 5;
+        const unsigned long long left = acc << (64 - mine);  // first bit at bit 63
+        const uint32_t hi = (uint32_t)(left >> 32), lo = (uint32_t)left;
+        atomicOr(&words[wk], hi >> o);
+        if (o + mine > 32) atomicOr(&words[wk + 1], __funnelshift_r(lo, hi, o));
+        if (o + mine > 64) atomicOr(&words[wk + 2], __funnelshift_lc(0u, lo, 32 - o));
+      }
+    } else {
+      // `cur` holds the pending bits left-aligned, `nb` of them
+      uint32_t wk = rel >> 5, nb = rel & 31u, cur = 0;
+      bool first = true;
+#pragma unroll
+      for (int k = 0; k < kPerThread; ++k) {
+        if (l[k]) {
+          const uint32_t cw = code[e[k]], tot = nb + l[k];
+          if (tot >= 32) {
+            const uint32_t u = cur | (cw >> (tot - 32));
+            if (first) atomicOr(&words[wk], u);  // the previous thread may own its first bits
+            else words[wk] = u;
+            first = false;
+            ++wk;
+            nb = tot - 32;
+            cur = __funnelshift_lc(0u, cw, 32 - nb);  // 0 when nb == 0
+          } else {
+            cur |= cw << (32 - tot);
+            nb = tot;
+          }
+        }
+      }
+      if (nb) atomicOr(&words[wk], cur);  // the last, partial word, which the next thread may share
+    }
+    __syncthreads();
+    // words out, and cleared for the next pack block: ORed where a
+    // neighbouring pack block owns part of the word (cleared beforehand),
+    // stored otherwise
+    const uint64_t base = origin >> 5;
+    const uint32_t end_bits = lead + cta_total;
+    const uint32_t nwords = (end_bits + 31) >> 5;
+    const bool shared_last = (end_bits & 31u) && pb + 1 < pack_ctas;
+    for (uint32_t j = threadIdx.x; j < nwords; j += kThreads) {
+      const uint32_t u = bswap32(words[j]);
+      words[j] = 0;
+      if ((j == 0 && lead) || (j == nwords - 1 && shared_last)) atomicOr(&a.bs32[base + j], u);
+      else a.bs32[base + j] = u;
+    }
+    if (!live) continue;
+
+    // sign/mantissa bytes: bit 15 -> bit 7, bits 0-6 kept; two per word
+    uint32_t sm2[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const uint32_t u = r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
+      sm2[r] = (u & 0x007F007Fu) | ((u >> 8) & 0x00800080u);  // bytes 0 and 2
+    }
+    const uint2 smv = make_uint2(__byte_perm(sm2[0], sm2[1], 0x6420),
+                                 __byte_perm(sm2[2], sm2[3], 0x6420));
+    if (live == kPerThread) {
+      *reinterpret_cast<uint2 *>(a.sm + i0) = smv;
+    } else {
+      for (uint32_t k = 0; k < live; ++k)
+        a.sm[i0 + k] = (uint8_t)((k < 4 ? smv.x : smv.y) >> (8 * (k & 3)));
+    }
+
+    // chunks and blocks whose first codeword start is one of these
+    // elements: those that begin after element i0 - 1's codeword start and
+    // at or before element i0 + live - 1's.  cb and qb run over their
+    // positions in order.
+    const int p0 = (int)rel;
+    const int prev = i0 == 0 ? -1 : p0 - (int)prev_len;
+    const int p_last = p0 + (int)(mine - last);
+    const int jc = floor_div(prev - cr0, (int)a.chunk_bits, a.inv_chunk) + 1;
+    const int jq = floor_div(prev - qr0, (int)a.block_bits, a.inv_block) + 1;
+    int cb = cr0 + jc * (int)a.chunk_bits, qb = qr0 + jq * (int)a.block_bits;
+    if (cb <= p_last || qb <= p_last) {
+      uint64_t c = c_org + jc, q = q_org + jq;
+      int pk = p0;
+#pragma unroll
+      for (int k = 0; k < kPerThread; ++k) {
+        if (l[k]) {
+          for (; cb <= pk; cb += (int)a.chunk_bits, ++c) {
+            if (c < a.chunks) {
+              a.gap[c] = (uint8_t)(pk - cb);
+              a.first_elem[c] = (uint32_t)(i0 + k);
+            }
+          }
+          for (; qb <= pk; qb += (int)a.block_bits, ++q)
+            if (q < a.num_blocks) a.bpos[q] = (uint32_t)(i0 + k);
+          pk += (int)l[k];
+        }
       }
     }
   }
-  // the last, partial word, which the next thread may share
-  if (nbits > (rel & 31u) || (!first && nbits))
-    atomicOr(&words[wk], (uint32_t)(acc << (32 - nbits)));
-  __syncthreads();
-  const uint64_t base = cta_start >> 5;
-  const uint32_t nwords = (lead + cta_total + 31) >> 5;
-  for (uint32_t j = threadIdx.x; j < nwords; j += kThreads) {
-    const uint32_t v = bswap32(words[j]);
-    if (j == 0 || j == nwords - 1) atomicOr(&a.bs32[base + j], v);  // shared with a neighbour
-    else a.bs32[base + j] = v;
-  }
-  if (i0 >= a.n) return;
-
-  // sign/mantissa bytes
-  uint32_t b[kPerThread];
-#pragma unroll
-  for (int k = 0; k < kPerThread; ++k) b[k] = ((x[k] >> 8) & 0x80u) | (x[k] & 0x7Fu);
-  if (i0 + kPerThread <= a.n) {
-    const uint2 v = make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
-                               b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
-    *reinterpret_cast<uint2 *>(a.sm + i0) = v;
-  } else {
-    for (int k = 0; k < kPerThread && i0 + k < a.n; ++k) a.sm[i0 + k] = (uint8_t)b[k];
-  }
-
-  // chunks and blocks whose first codeword start is one of these elements:
-  // those that begin after the previous codeword start and at or before
-  // this one
-  unsigned long long bit = cta_start + before + incl - mine;
-  long long prev = i0 == 0 ? -1 : (long long)(bit - len[exponent(a.w[i0 - 1])]);
-  for (int k = 0; k < kPerThread && i0 + k < a.n; ++k) {
-    const uint64_t c_lo = prev < 0 ? 0 : (uint64_t)prev / a.chunk_bits + 1;
-    for (uint64_t c = c_lo; c * a.chunk_bits <= bit && c < a.chunks; ++c) {
-      a.gap[c] = (uint8_t)(bit - c * a.chunk_bits);
-      a.first_elem[c] = (uint32_t)(i0 + k);
-    }
-    const uint64_t b_lo = prev < 0 ? 0 : (uint64_t)prev / a.block_bits + 1;
-    for (uint64_t q = b_lo; q * a.block_bits <= bit && q < a.num_blocks; ++q)
-      a.bpos[q] = (uint32_t)(i0 + k);
-    prev = (long long)bit;
-    bit += len[exponent(x[k])];
-  }
 }
 
+// ---- finish --------------------------------------------------------------
 struct FinishArgs {
   const uint8_t *gap;
   const uint32_t *first_elem;
@@ -302,6 +557,21 @@ bool grid_for(uint64_t items, uint64_t per_cta, unsigned *grid) {
   return true;
 }
 
+uint64_t round256(uint64_t x) { return (x + 255) & ~255ull; }
+
+// resident thread blocks of kThreads on the current device (at least 1)
+template <class K>
+uint64_t resident(K kernel) {
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    sms = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  return (uint64_t)sms * per_sm;
+}
+
 }  // namespace
 
 struct df11_gpu_build {
@@ -311,15 +581,20 @@ struct df11_gpu_build {
   uint8_t len[256];
   uint32_t code[256];
   std::vector<uint32_t> luts;
-  uint64_t total = 0, last_start = 0, num_blocks = 0, chunks = 0, pack_ctas = 0;
+  uint64_t total = 0, last_start = 0, num_blocks = 0, chunks = 0;
   bool vec = false;
-  // device scratch: pack-block first bits, {codeword, length} per exponent
-  unsigned long long *d_cta_bits = nullptr;
+  Ranges r{};
+  uint64_t ranges = 0;
+  // device scratch, phase 1: histogram, {codeword, length} per exponent,
+  // range totals and first bits, pack-block first bits within their range
+  void *scratch1 = nullptr;
+  unsigned long long *d_hist = nullptr, *d_range_total = nullptr;
   uint2 *d_tab = nullptr;
-  // device scratch: per-chunk gap and first element, the three maxima
-  uint8_t *d_gap = nullptr;
+  // device scratch, phase 2: per-chunk first element and gap, the maxima
+  void *scratch2 = nullptr;
   uint32_t *d_first = nullptr;
   unsigned int *d_max = nullptr;
+  uint8_t *d_gap = nullptr;
 };
 
 namespace {
@@ -341,11 +616,8 @@ extern "C" {
 
 void df11_gpu_build_free(df11_gpu_build *h) {
   if (!h) return;
-  cudaFree(h->d_cta_bits);
-  cudaFree(h->d_tab);
-  cudaFree(h->d_gap);
-  cudaFree(h->d_first);
-  cudaFree(h->d_max);
+  cudaFree(h->scratch1);
+  cudaFree(h->scratch2);
   delete h;
 }
 
@@ -365,34 +637,47 @@ df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t C,
   h->C = C;
   h->T = T;
   h->vec = ((uintptr_t)d_bf16 & 15) == 0;
-  h->pack_ctas = (n + kPerCta - 1) / kPerCta;
-  unsigned long long *d_hist = nullptr;
+  // contiguous ranges of pack blocks, one per resident sums thread block.
+  // A range's bits fit 32 bits: at most 2^21 pack blocks over at least
+  // min(pack blocks, SMs) ranges, at most 65536 bits per pack block.
+  h->r.pack_ctas = (n + kPerCta - 1) / kPerCta;
+  const uint64_t slots = resident(sums_kernel);
+  h->ranges = h->r.pack_ctas < slots ? h->r.pack_ctas : slots;
+  h->r.per = h->ranges ? (h->r.pack_ctas + h->ranges - 1) / h->ranges : 1;
+  if (h->ranges) h->ranges = (h->r.pack_ctas + h->r.per - 1) / h->r.per;
   auto fail = [&](df11_status st) {
-    cudaFree(d_hist);
+    cudaStreamSynchronize(s);  // nothing queued may outlive the scratch
     df11_gpu_build_free(h);
     return st;
   };
-  if (cudaMalloc(&d_hist, 256 * sizeof(unsigned long long)) != cudaSuccess ||
-      cudaMalloc(&h->d_tab, 256 * sizeof(uint2)) != cudaSuccess ||
-      cudaMalloc(&h->d_cta_bits, (h->pack_ctas + 1) * sizeof(unsigned long long)) != cudaSuccess)
-    return fail(DF11_ERR_CUDA);
+  const uint64_t o_tab = round256(256 * sizeof(unsigned long long));
+  const uint64_t o_tot = o_tab + round256(256 * sizeof(uint2));
+  const uint64_t o_rs = o_tot + round256(h->ranges * sizeof(unsigned long long) + 8);
+  const uint64_t o_loc = o_rs + round256((h->ranges + 1) * sizeof(unsigned long long));
+  const uint64_t bytes1 = o_loc + round256(h->r.pack_ctas * sizeof(uint32_t) + 4);
+  if (cudaMalloc(&h->scratch1, bytes1) != cudaSuccess) return fail(DF11_ERR_CUDA);
+  char *base1 = static_cast<char *>(h->scratch1);
+  h->d_hist = reinterpret_cast<unsigned long long *>(base1);
+  h->d_tab = reinterpret_cast<uint2 *>(base1 + o_tab);
+  h->d_range_total = reinterpret_cast<unsigned long long *>(base1 + o_tot);
+  h->r.range_start = reinterpret_cast<unsigned long long *>(base1 + o_rs);
+  h->r.local = reinterpret_cast<uint32_t *>(base1 + o_loc);
 
   // histogram, and the last element (its codeword ends the stream)
   unsigned long long hist[256];
   uint16_t last = 0;
-  bool ok = cudaMemsetAsync(d_hist, 0, 256 * sizeof(unsigned long long), s) == cudaSuccess;
+  bool ok = cudaMemsetAsync(h->d_hist, 0, 256 * sizeof(unsigned long long), s) == cudaSuccess;
   if (ok && n) {
-    const uint64_t want = (n + kPerCta - 1) / kPerCta;
-    const unsigned grid = (unsigned)(want < 148 * 8 ? want : 148 * 8);
-    hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16, n, h->vec, d_hist);
+    const uint64_t want = resident(hist_kernel);
+    const unsigned grid = (unsigned)(h->r.pack_ctas < want ? h->r.pack_ctas : want);
+    hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16, n, h->vec, h->d_hist);
     ok = cudaGetLastError() == cudaSuccess &&
          cudaMemcpyAsync(&last, d_bf16 + (n - 1), 2, cudaMemcpyDeviceToHost, s) == cudaSuccess;
   }
-  ok = ok && cudaMemcpyAsync(hist, d_hist, sizeof(hist), cudaMemcpyDeviceToHost, s) == cudaSuccess &&
+  ok = ok &&
+       cudaMemcpyAsync(hist, h->d_hist, sizeof(hist), cudaMemcpyDeviceToHost, s) == cudaSuccess &&
        cudaStreamSynchronize(s) == cudaSuccess;
   if (!ok) return fail(DF11_ERR_CUDA);
-  cudaFree(d_hist);
-  d_hist = nullptr;
 
   // codebook (host: 256 symbols)
   uint64_t hist64[256];
@@ -400,42 +685,35 @@ df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t C,
   h->longest = df11_internal::codebook(hist64, h->len, h->code, h->luts);
   uint2 tab[256];
   for (int i = 0; i < 256; ++i) tab[i] = make_uint2(h->code[i], h->len[i]);
+
+  // first bit of every range and pack block, and the total
+  unsigned long long total = 0;
   if (cudaMemcpyAsync(h->d_tab, tab, sizeof(tab), cudaMemcpyHostToDevice, s) != cudaSuccess)
     return fail(DF11_ERR_CUDA);
-
-  // first bit of every pack block
-  std::vector<unsigned long long> bits(h->pack_ctas + 1, 0);
-  if (h->pack_ctas) {
-    unsigned grid;
-    if (!grid_for(n, kPerCta, &grid)) return fail(DF11_ERR_TOO_LARGE);
-    sums_kernel<<<grid, kThreads, 0, s>>>(d_bf16, n, h->vec, h->d_tab, h->d_cta_bits);
+  if (h->ranges) {
+    sums_kernel<<<(unsigned)h->ranges, kThreads, 0, s>>>(d_bf16, n, h->vec, h->d_tab, h->r,
+                                                         h->d_range_total);
+    scan_kernel<<<1, kScanThreads, 0, s>>>(h->d_range_total, h->ranges, h->r.range_start);
     if (cudaGetLastError() != cudaSuccess ||
-        cudaMemcpyAsync(bits.data(), h->d_cta_bits, h->pack_ctas * sizeof(unsigned long long),
-                        cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
+        cudaMemcpyAsync(&total, h->r.range_start + h->ranges, sizeof(total),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
   }
-  unsigned long long run = 0;
-  for (uint64_t i = 0; i < h->pack_ctas; ++i) {
-    const unsigned long long v = bits[i];
-    bits[i] = run;
-    run += v;
-  }
-  h->total = run;
-  if (h->pack_ctas &&
-      cudaMemcpyAsync(h->d_cta_bits, bits.data(), h->pack_ctas * sizeof(unsigned long long),
-                      cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return fail(DF11_ERR_CUDA);
+  // the table copy reads `tab` until it is done
+  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(DF11_ERR_CUDA);
+  h->total = total;
   if (n) h->last_start = h->total - h->len[(last >> 7) & 0xFF];
   const uint64_t block_bits = 8ull * C * T;
   h->num_blocks = (h->total + block_bits - 1) / block_bits;
   h->chunks = h->num_blocks * T;
-  if (cudaMalloc(&h->d_gap, h->chunks + 1) != cudaSuccess ||
-      cudaMalloc(&h->d_first, (h->chunks + 1) * sizeof(uint32_t)) != cudaSuccess ||
-      cudaMalloc(&h->d_max, 3 * sizeof(unsigned int)) != cudaSuccess)
+  const uint64_t o_max = round256((h->chunks + 1) * sizeof(uint32_t));
+  const uint64_t o_gap = o_max + 256;
+  if (cudaMalloc(&h->scratch2, o_gap + round256(h->chunks + 1)) != cudaSuccess)
     return fail(DF11_ERR_CUDA);
-  // the copy out of `bits` must be done before `bits` goes away
-  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(DF11_ERR_CUDA);
+  char *base2 = static_cast<char *>(h->scratch2);
+  h->d_first = reinterpret_cast<uint32_t *>(base2);
+  h->d_max = reinterpret_cast<unsigned int *>(base2 + o_max);
+  h->d_gap = reinterpret_cast<uint8_t *>(base2 + o_gap);
   fill_params(h, params);
   std::memcpy(code_lengths, h->len, 256);
   *handle = h;
@@ -449,28 +727,28 @@ df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uin
   if (!h) return DF11_ERR_NULL;
   df11_status st = DF11_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  const uint64_t chunks = h->chunks;
+  const uint64_t chunks = h->chunks, n = h->n;
   const uint64_t bs_bytes = chunks * h->C + 16, gaps_bytes = chunks * 5 / 8 + 16;
-  const uint64_t sm_bytes = (h->n + 15) / 16 * 16;
+  const uint64_t sm_bytes = (n + 15) / 16 * 16;
+  const uint64_t bs_written = (h->total + 31) / 32 * 4;  // the pack blocks' words
   do {
     if (!params || !bitstream || !gaps || !chunk_counts || !block_out_pos || !luts ||
-        !code_lengths || !sign_mantissa || (h->n && !d_bf16)) {
+        !code_lengths || !sign_mantissa || (n && !d_bf16)) {
       st = DF11_ERR_NULL;
       break;
     }
     if (((uintptr_t)bitstream & 15) || ((uintptr_t)gaps & 15) || ((uintptr_t)luts & 15) ||
         ((uintptr_t)chunk_counts & 15) || ((uintptr_t)sign_mantissa & 15) ||
-        ((uintptr_t)block_out_pos & 3) || (h->n && h->vec != (((uintptr_t)d_bf16 & 15) == 0))) {
+        ((uintptr_t)block_out_pos & 3) || (n && h->vec != (((uintptr_t)d_bf16 & 15) == 0))) {
       st = DF11_ERR_ALIGN;
       break;
     }
+    // every byte the kernels do not write: the padding after each buffer
     const bool ok =
-        cudaMemsetAsync(bitstream, 0, bs_bytes, s) == cudaSuccess &&
-        cudaMemsetAsync(gaps, 0, gaps_bytes, s) == cudaSuccess &&
-        cudaMemsetAsync(chunk_counts, 0, chunks + 16, s) == cudaSuccess &&
-        (sm_bytes == 0 || cudaMemsetAsync(sign_mantissa, 0, sm_bytes, s) == cudaSuccess) &&
-        cudaMemsetAsync(h->d_gap, 0, chunks + 1, s) == cudaSuccess &&
-        cudaMemsetAsync(h->d_max, 0, 3 * sizeof(unsigned int), s) == cudaSuccess &&
+        cudaMemsetAsync(bitstream + bs_written, 0, bs_bytes - bs_written, s) == cudaSuccess &&
+        cudaMemsetAsync(gaps + chunks * 5 / 8, 0, gaps_bytes - chunks * 5 / 8, s) == cudaSuccess &&
+        cudaMemsetAsync(chunk_counts + chunks, 0, 16, s) == cudaSuccess &&
+        (sm_bytes == n || cudaMemsetAsync(sign_mantissa + n, 0, sm_bytes - n, s) == cudaSuccess) &&
         cudaMemcpyAsync(luts, h->luts.data(), h->luts.size() * 4, cudaMemcpyHostToDevice, s) ==
             cudaSuccess &&
         cudaMemcpyAsync(code_lengths, h->len, 256, cudaMemcpyHostToDevice, s) == cudaSuccess;
@@ -478,15 +756,22 @@ df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uin
       st = DF11_ERR_CUDA;
       break;
     }
-    fill_u32<<<148 * 4, 256, 0, s>>>(h->d_first, chunks + 1, (uint32_t)h->n);
-    const PackArgs pa{d_bf16, h->n, h->vec, h->d_tab, h->d_cta_bits,
-                      reinterpret_cast<uint32_t *>(bitstream), sign_mantissa, h->d_gap,
-                      h->d_first, block_out_pos, 8ull * h->C, chunks, 8ull * h->C * h->T,
-                      (uint32_t)h->num_blocks};
-    if (h->pack_ctas) pack_kernel<<<(unsigned)h->pack_ctas, kThreads, 0, s>>>(pa);
+    uint32_t *bs32 = reinterpret_cast<uint32_t *>(bitstream);
+    prepare_kernel<<<148 * 4, 256, 0, s>>>(h->d_first, h->d_gap, chunks, (uint32_t)n, h->r, bs32,
+                                           h->d_max);
+    const uint32_t chunk_bits = 8 * h->C, block_bits = 8 * h->C * h->T;
+    const PackArgs pa{d_bf16, n, h->vec, h->d_tab, h->r, bs32, sign_mantissa, h->d_gap,
+                      h->d_first, block_out_pos, chunks, (uint32_t)h->num_blocks,
+                      chunk_bits, block_bits, h->C / 4, h->C / 4 * h->T,
+                      1.0f / (float)chunk_bits, 1.0f / (float)block_bits};
+    if (h->r.pack_ctas) {
+      const uint64_t want = resident(pack_kernel);
+      const unsigned grid = (unsigned)(h->r.pack_ctas < want ? h->r.pack_ctas : want);
+      pack_kernel<<<grid, kThreads, 0, s>>>(pa);
+    }
     const FinishArgs fa{h->d_gap, h->d_first, gaps, chunk_counts, block_out_pos, h->d_max,
                         8ull * h->C, chunks, 8ull * h->C * h->T, h->total, h->last_start,
-                        (uint32_t)h->num_blocks, (uint32_t)h->n};
+                        (uint32_t)h->num_blocks, (uint32_t)n};
     unsigned grid;
     if (chunks) {
       if (!grid_for(chunks / 8, 256, &grid)) {

@@ -137,3 +137,17 @@ def test_argument_errors():
         df11.compress_on_device(x.cpu())
     with pytest.raises(TypeError):
         df11.compress_on_device(x.float())
+
+
+def test_runs_of_long_codewords():
+    """A thread's 8 codewords longer than 64 bits in total (a run of rare
+    exponents among one common one) take the word-by-word packing path."""
+    common = np.full(300_000, 240 << 7, np.uint16)
+    rare = ((np.arange(2000) % 200 + 20) << 7).astype(np.uint16)
+    w = np.concatenate([common[:150_001], rare, common[150_001:]])
+    bits = torch.from_numpy(w.view(np.int16)).cuda()
+    d, h, w = _same_as_host(bits)
+    lens = h.code_lengths.astype(np.int64)[(w.astype(np.int64) >> 7) & 0xFF]
+    per_thread = np.add.reduceat(lens, np.arange(0, len(lens), 8))
+    assert per_thread.max() > 64  # the case this test is for
+    _decodes_to(d, w)
