@@ -36,9 +36,11 @@
 //              of 32 chunks.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -559,17 +561,61 @@ bool grid_for(uint64_t items, uint64_t per_cta, unsigned *grid) {
 
 uint64_t round256(uint64_t x) { return (x + 255) & ~255ull; }
 
-// resident thread blocks of kThreads on the current device (at least 1)
+constexpr int kMaxDevices = 64;
+
+// resident thread blocks of kThreads on the current device (at least 1),
+// queried once per kernel and device
 template <class K>
 uint64_t resident(K kernel) {
-  int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+  static std::atomic<uint64_t> known[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = -1;
+  if (dev >= 0) {
+    const uint64_t v = known[dev].load(std::memory_order_relaxed);
+    if (v) return v;
+  }
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev < 0 ? 0 : dev) !=
+          cudaSuccess ||
+      sms < 1)
     sms = 1;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
-  return (uint64_t)sms * per_sm;
+  const uint64_t v = (uint64_t)sms * per_sm;
+  if (dev >= 0) known[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+// The builder's device scratch comes from a memory pool of the library's
+// own per device, allocated and freed in stream order; the pool keeps what
+// it has reserved, so repeated builds neither map memory nor synchronise
+// the device to release it.
+cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t s) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaMalloc(p, bytes);
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      if ((e = cudaMemPoolCreate(&pools[dev], &props)) != cudaSuccess) {
+        pools[dev] = nullptr;
+        return e;
+      }
+      uint64_t keep = UINT64_MAX;
+      cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+    pool = pools[dev];
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, s);
 }
 
 }  // namespace
@@ -587,6 +633,7 @@ struct df11_gpu_build {
   uint64_t ranges = 0;
   // device scratch, phase 1: histogram, {codeword, length} per exponent,
   // range totals and first bits, pack-block first bits within their range
+  cudaStream_t stream = nullptr;  // the stream the scratch was allocated on
   void *scratch1 = nullptr;
   unsigned long long *d_hist = nullptr, *d_range_total = nullptr;
   uint2 *d_tab = nullptr;
@@ -616,8 +663,9 @@ extern "C" {
 
 void df11_gpu_build_free(df11_gpu_build *h) {
   if (!h) return;
-  cudaFree(h->scratch1);
-  cudaFree(h->scratch2);
+  // after the work queued on the handle's stream, which may read the scratch
+  if (h->scratch1) cudaFreeAsync(h->scratch1, h->stream);
+  if (h->scratch2) cudaFreeAsync(h->scratch2, h->stream);
   delete h;
 }
 
@@ -645,8 +693,8 @@ df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t C,
   h->ranges = h->r.pack_ctas < slots ? h->r.pack_ctas : slots;
   h->r.per = h->ranges ? (h->r.pack_ctas + h->ranges - 1) / h->ranges : 1;
   if (h->ranges) h->ranges = (h->r.pack_ctas + h->r.per - 1) / h->r.per;
+  h->stream = s;
   auto fail = [&](df11_status st) {
-    cudaStreamSynchronize(s);  // nothing queued may outlive the scratch
     df11_gpu_build_free(h);
     return st;
   };
@@ -655,7 +703,7 @@ df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t C,
   const uint64_t o_rs = o_tot + round256(h->ranges * sizeof(unsigned long long) + 8);
   const uint64_t o_loc = o_rs + round256((h->ranges + 1) * sizeof(unsigned long long));
   const uint64_t bytes1 = o_loc + round256(h->r.pack_ctas * sizeof(uint32_t) + 4);
-  if (cudaMalloc(&h->scratch1, bytes1) != cudaSuccess) return fail(DF11_ERR_CUDA);
+  if (scratch_alloc(&h->scratch1, bytes1, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
   char *base1 = static_cast<char *>(h->scratch1);
   h->d_hist = reinterpret_cast<unsigned long long *>(base1);
   h->d_tab = reinterpret_cast<uint2 *>(base1 + o_tab);
@@ -708,7 +756,7 @@ df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t C,
   h->chunks = h->num_blocks * T;
   const uint64_t o_max = round256((h->chunks + 1) * sizeof(uint32_t));
   const uint64_t o_gap = o_max + 256;
-  if (cudaMalloc(&h->scratch2, o_gap + round256(h->chunks + 1)) != cudaSuccess)
+  if (scratch_alloc(&h->scratch2, o_gap + round256(h->chunks + 1), s) != cudaSuccess)
     return fail(DF11_ERR_CUDA);
   char *base2 = static_cast<char *>(h->scratch2);
   h->d_first = reinterpret_cast<uint32_t *>(base2);
@@ -794,7 +842,7 @@ df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uin
     params->max_chunk_elems = mx[1];
     params->max_warp_elems = mx[2];
   } while (false);
-  if (st != DF11_OK) cudaStreamSynchronize(s);  // nothing queued may outlive the scratch
+  h->stream = s;  // frees follow this call's work
   df11_gpu_build_free(h);
   return st;
 }

@@ -247,7 +247,10 @@ typedef struct df11_gpu_build df11_gpu_build;
  * success fills *params (n, total_bits, chunk_bytes, threads_per_block,
  * num_blocks, num_luts, max_len; the max_* counts are filled by phase 2),
  * code_lengths (host, 256 bytes) and *handle, which holds device scratch
- * until phase 2 or df11_gpu_build_free.  The buffers phase 2 writes, with
+ * until phase 2 or df11_gpu_build_free.  The scratch comes from a memory
+ * pool the library keeps per device (allocated and freed in stream order;
+ * what the pool has reserved stays reserved for the process, so repeated
+ * builds allocate nothing new).  The buffers phase 2 writes, with
  * C = chunk_bytes, T = threads_per_block, B = num_blocks:
  *   bitstream      B*T*C + 16 bytes       gaps           B*T*5/8 + 16 bytes
  *   chunk_counts   B*T + 16 bytes         block_out_pos  (B + 1) uint32
@@ -276,7 +279,9 @@ df11_status df11_gpu_build_finish(df11_gpu_build *handle, const uint16_t *d_bf16
                                   uint8_t *code_lengths, uint8_t *sign_mantissa,
                                   df11_params *params, df11_stream_t stream);
 
-/* Release a phase-1 handle without running phase 2 (NULL is a no-op). */
+/* Release a phase-1 handle without running phase 2 (NULL is a no-op); its
+ * scratch is freed in order on the stream phase 1 ran on, which must still
+ * exist. */
 void df11_gpu_build_free(df11_gpu_build *handle);
 
 #ifdef __cplusplus
