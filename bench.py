@@ -46,7 +46,13 @@ import workloads  # noqa: E402
 METRIC = ("decoded BF16 GB/s and % of HBM roofline (1×B200), "
           "bit-exact vs CPU oracle")
 UNIT = "GB/s"
+BUILD_METRIC = ("compressed BF16 GB/s (device-side format builder, 1×B200), "
+                "byte-identical to the host builder")
+# launches of the library's own kernels per device build: histogram, sums,
+# scan, prepare, pack, and two finishing kernels
+BUILD_LAUNCHES = 7
 KERNEL_SRC = os.path.join(ROOT, "huffman_decode_df11_b200", "csrc", "df11_decode.cu")
+BUILD_SRC = os.path.join(ROOT, "huffman_decode_df11_b200", "csrc", "df11_gpu_build.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 FALLBACK_HBM_GBS = 6650.0
 
@@ -68,6 +74,8 @@ def workload_units(config: str, seed: int):
         return [("embed_151936x4096", lambda d: workloads.embedding(seed, d))]
     if config == "stack":
         return [(name, thunk) for name, _, thunk in workloads.stack_units(seed)]
+    if config == "build":  # the block's tensors, compressed on the device
+        return workload_units("block", seed)
     if config == "offload":  # the stack's first layers, without embedding and LM head
         return [(name, thunk) for name, _, thunk
                 in workloads.stack_units(seed, OFFLOAD_LAYERS)[1:-1]]
@@ -100,17 +108,17 @@ def algorithmic_bytes(h, counts: bool = True) -> int:
             + (chunks if counts else 0) + 1024 * p.num_luts + 256 + 2 * p.n)
 
 
-def kernel_hash() -> str:
-    return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+def kernel_hash(src: str = KERNEL_SRC) -> str:
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """Per-launch DRAM bytes from an ncu capture of the current kernel source
-    (profiles/dram_traffic.txt: '<kernel sha16> <workload>/c<C>/t<T> <bytes
-    per launch>')."""
+def recorded_traffic(workload: str, src: str = KERNEL_SRC):
+    """Per-launch (per-step for the builder) DRAM bytes from an ncu capture
+    of the current kernel source (profiles/dram_traffic.txt: '<source sha16>
+    <workload>/c<C>/t<T> <bytes>')."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
-    kh = kernel_hash()
+    kh = kernel_hash(src)
     for line in open(TRAFFIC_FILE):
         parts = line.split()
         if len(parts) >= 3 and not line.startswith("#") and parts[0] == kh and parts[1] == workload:
@@ -523,6 +531,169 @@ def run_offload(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def build_algorithmic_bytes(h) -> int:
+    """Bytes a build of this tensor must move: the BF16 input read twice (the
+    code depends on the whole histogram, so the codewords can only be
+    written in a second pass; the input is larger than L2) and the
+    compressed tensor written once."""
+    return 4 * h.n + h.compressed_bytes()
+
+
+def _same_bytes(d, h) -> bool:
+    for f in ("bitstream", "gaps", "chunk_counts", "block_out_pos", "luts", "code_lengths",
+              "sign_mantissa"):
+        got = getattr(d, f).cpu().numpy().view(np.uint8)
+        want = np.ascontiguousarray(getattr(h, f)).view(np.uint8)
+        if got.shape != want.shape or not np.array_equal(got, want):
+            return False
+    return all(getattr(d.params, f) == getattr(h.params, f) for f, _ in d.params._fields_)
+
+
+def run_build(args, world, rank, local):
+    """The format builder on the device: every tensor of the workload
+    compressed from BF16 already in HBM (df11_gpu_build_begin / _finish via
+    compress_on_device).  Parity: byte-identical buffers and parameters to
+    the host builder, and a decode back to the original words, before any
+    timing.  A step builds every tensor once; each build reads the counts
+    and the stream's length back to the host (that is in the timed region)."""
+    import huffman_decode_df11_b200 as df11
+    device = f"cuda:{local}"
+    seed = args.seed + rank
+    units = workload_units(args.config, seed)
+    C, T = args.chunk_bytes, args.threads_per_block
+    ws = [thunk(device) for _, thunk in units]
+    hosts = []
+    for (name, _), w in zip(units, ws):
+        h = df11.compress(w, chunk_bytes=C, threads_per_block=T)
+        d = df11.compress_on_device(w, C, T)
+        if not _same_bytes(d, h):
+            raise SystemExit(f"device build differs from the host build on {name}")
+        out = df11.decode(d)
+        torch.cuda.synchronize()
+        if not torch.equal(out.view(torch.int16).view(w.shape), w):
+            raise SystemExit(f"device build does not decode to the original on {name}")
+        hosts.append(h)
+        del d, out
+    n_total = sum(h.n for h in hosts)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for w in ws:
+            df11.compress_on_device(w, C, T, decode_table=False)
+
+    for _ in range(args.warmup):
+        step()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_local = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    value = sum_over_ranks(2.0 * n_total, world) / (ms * 1e-3) / 1e9
+    alg = sum(build_algorithmic_bytes(h) for h in hosts)
+    achieved = alg / (ms_local * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = recorded_traffic(f"build/c{C}/t{T}", BUILD_SRC)
+
+    # end to end: BF16 in pinned host memory, copied in, built, and the
+    # compressed buffers copied back to pinned host memory, every step
+    e2e = None
+    if not args.no_e2e:
+        pins = [w.cpu().pin_memory() for w in ws]
+        devs = [torch.empty_like(w) for w in ws]
+        backs = [{f: torch.empty(getattr(h, f).nbytes, dtype=torch.uint8).pin_memory()
+                  for f in ("bitstream", "gaps", "chunk_counts", "block_out_pos", "luts",
+                            "code_lengths", "sign_mantissa")} for h in hosts]
+
+        def e2e_step():
+            for pin, dev, back in zip(pins, devs, backs):
+                dev.copy_(pin, non_blocking=True)
+                d = df11.compress_on_device(dev, C, T, decode_table=False)
+                for f, b in back.items():
+                    b.copy_(getattr(d, f).view(torch.uint8).view(-1), non_blocking=True)
+            torch.cuda.synchronize()
+
+        for _ in range(2):
+            e2e_step()
+        e_steps = max(3, min(args.steps, 20))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(a.elapsed_time(b) / e_steps, world)
+        e2e = {"value": round(sum_over_ranks(2.0 * n_total, world) / (e_ms * 1e-3) / 1e9, 2),
+               "unit": UNIT, "h2d_bytes_per_step": 2 * n_total,
+               "d2h_bytes_per_step": sum(h.compressed_bytes() for h in hosts),
+               "ms_per_step": round(e_ms, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_build_baseline(ws, args.cpu_budget_s)
+    if rank == 0:
+        line = {
+            "metric": BUILD_METRIC, "value": round(value, 2), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+            "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
+            "config": {
+                "workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
+                "elements": n_total, "chunk_bytes": C, "threads_per_block": T,
+                "compressed_bytes": sum(h.compressed_bytes() for h in hosts),
+                "l2": "inputs larger than L2 (no flush)",
+                "parallelism": f"replicas x{world} (no collective)",
+                "parity": "byte-identical to the host builder and bit-exact decode, "
+                          "every tensor, before timing",
+            },
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": traffic, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_step": alg,
+                         "kernel": "the whole build (7 launches and 3 host round trips "
+                                   "per tensor), timed as one"},
+            "gpu_launches": BUILD_LAUNCHES * len(ws) * args.steps,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def _oracle_encode_sample(ws, budget_s: float):
+    """Encode leading slices of the workload's tensors with the oracle until
+    the budget is spent; returns (elements, seconds, description)."""
+    import oracle
+    done, t_used, names = 0, 0.0, 0
+    for w in ws:
+        if t_used >= budget_s:
+            break
+        # bound one call to what fits the remaining budget (~40 ns/element)
+        count = int(min(w.numel(), max(2048, (budget_s - t_used) / 40e-9)))
+        a = workloads.as_numpy_u16(w.reshape(-1)[:count])
+        t = time.perf_counter()
+        oracle.encode(a, 24, 256)
+        t_used += time.perf_counter() - t
+        done += count
+        names += 1
+    return done, t_used, f"{done} elements from the first {names} tensor(s), encoded in order"
+
+
+def cpu_build_baseline(ws, budget_s: float):
+    done, secs, what = _oracle_encode_sample(ws, budget_s)
+    return {"value": round(2.0 * done / secs / 1e9, 4), "unit": UNIT, "cores": 1,
+            "kind": "oracle", "sample": what + " (single-threaded C encoder)"}
+
+
 def measure_e2e(args, units, hosts, groups, device, world):
     import huffman_decode_df11_b200 as df11
     # bounded host memory: the first groups up to ~2G elements
@@ -622,6 +793,8 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     units = workload_units(args.config, args.seed)
+    if args.config == "build":
+        return run_reference_build(args, world, units)
     import huffman_decode_df11_b200 as df11
     hosts = [df11.compress(thunk("cpu"), chunk_bytes=args.chunk_bytes,
                            threads_per_block=args.threads_per_block) for _, thunk in units]
@@ -653,6 +826,38 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_build(args, world, units):
+    """The comparison arm for the builder: the oracle's encoder, as it
+    stands, on bounded samples of the workload."""
+    ws = [thunk("cpu") for _, thunk in units]
+    n_total = sum(w.numel() for w in ws)
+    budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        _oracle_encode_sample(ws, budget)
+    tot_done, tot_s, what = 0, 0.0, ""
+    for _ in range(args.steps):
+        d, s_, what = _oracle_encode_sample(ws, budget)
+        tot_done += d
+        tot_s += s_
+    value = 2.0 * tot_done / tot_s / 1e9
+    line = {
+        "impl": "reference", "metric": BUILD_METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+        "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
+        "config": {"workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
+                   "elements": n_total, "chunk_bytes": 24, "threads_per_block": 256,
+                   "step": f"bounded sample of the workload, ~{budget:.1f} s of CPU work"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": what + " per step (single-threaded C encoder)"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
 OFFLOAD_LAYERS = 8
 
 WORKLOAD_NAMES = {
@@ -662,6 +867,8 @@ WORKLOAD_NAMES = {
     "fibonacci": "Fibonacci exponent counts (32-bit codewords), 14,930,351 elems",
     "embedding": "embedding 151936x4096 N(0,0.02), 622,329,856 elems",
     "stack": "36-layer Qwen3-8B-shaped stack + embedding + LM head, 8,190,427,136 elems",
+    "build": "format builder on the GPU: Qwen3-8B-shaped block (q,k,v,o,gate,up,down) "
+             "compressed from BF16 in HBM, 192,937,984 elems",
     "offload": f"{OFFLOAD_LAYERS} Qwen3-8B-shaped layers streamed from pinned host memory "
                f"(compressed, one host-to-device copy per layer), "
                f"{OFFLOAD_LAYERS * 192_937_984:,} elems",
@@ -700,6 +907,8 @@ def main(argv=None):
                 raise SystemExit("the b200 arm needs a CUDA device")
             if args.config == "offload":
                 run_offload(args, world, rank, local)
+            elif args.config == "build":
+                run_build(args, world, rank, local)
             else:
                 run_b200(args, world, rank, local)
     finally:
