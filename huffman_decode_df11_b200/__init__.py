@@ -135,6 +135,8 @@ def lib():
     L.df11_gpu_build_finish.restype = ctypes.c_int
     L.df11_gpu_build_free.argtypes = [vp]
     L.df11_gpu_build_free.restype = None
+    L.df11_exponent_histogram.argtypes = [vp, u64, vp, vp]
+    L.df11_exponent_histogram.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -347,6 +349,22 @@ def compress_on_device(w: torch.Tensor, chunk_bytes: int = 24, threads_per_block
     if decode_table:
         d.decode_table = build_decode_table(d, stream)
     return d
+
+
+def exponent_histogram(w: torch.Tensor, stream=None) -> np.ndarray:
+    """Counts of the 256 exponent values of a BF16 tensor in device memory
+    (df11_exponent_histogram; allocates nothing on the device)."""
+    if not w.is_cuda:
+        raise ValueError("exponent_histogram takes a CUDA tensor")
+    if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected BF16 words (bfloat16, int16 or uint16), got {w.dtype}")
+    flat = w.contiguous().reshape(-1)
+    n = flat.numel()
+    hist = np.zeros(256, dtype=np.uint64)
+    _check(lib().df11_exponent_histogram(flat.data_ptr() if n else None, n,
+                                         hist.ctypes.data, _stream_handle(stream)),
+           "df11_exponent_histogram")
+    return hist
 
 
 def build_decode_table(d: Df11Device, stream=None) -> torch.Tensor:

@@ -848,3 +848,37 @@ df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uin
 }
 
 }  // extern "C"
+
+// ---- exponent histogram into a static device buffer ----------------------
+namespace {
+// The histogram entry point's device counters: a module global, so the call
+// needs no allocation.  One copy per device; calls are serialised.
+__device__ __align__(256) unsigned long long g_exponent_hist[256];
+std::mutex g_exponent_hist_mutex;
+}  // namespace
+
+extern "C" df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t n,
+                                               uint64_t hist[256], df11_stream_t stream) {
+  if (!hist || (n && !d_bf16)) return DF11_ERR_NULL;
+  if (n >= (1ull << 32)) return DF11_ERR_TOO_LARGE;
+  if ((uintptr_t)d_bf16 & 1) return DF11_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_exponent_hist_mutex);
+  void *sym = nullptr;
+  if (cudaGetSymbolAddress(&sym, g_exponent_hist) != cudaSuccess) return DF11_ERR_CUDA;
+  unsigned long long *d = static_cast<unsigned long long *>(sym);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(d, 0, 256 * sizeof(unsigned long long), s) != cudaSuccess)
+    return DF11_ERR_CUDA;
+  if (n) {
+    const uint64_t tiles = (n + kPerCta - 1) / kPerCta, slots = resident(hist_kernel);
+    const bool vec = ((uintptr_t)d_bf16 & 15) == 0;
+    hist_kernel<<<(unsigned)(tiles < slots ? tiles : slots), kThreads, 0, s>>>(d_bf16, n, vec, d);
+  }
+  unsigned long long counts[256];
+  if (cudaGetLastError() != cudaSuccess ||
+      cudaMemcpyAsync(counts, d, sizeof(counts), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return DF11_ERR_CUDA;
+  for (int i = 0; i < 256; ++i) hist[i] = counts[i];
+  return DF11_OK;
+}

@@ -279,6 +279,22 @@ df11_status df11_gpu_build_finish(df11_gpu_build *handle, const uint16_t *d_bf16
                                   uint8_t *code_lengths, uint8_t *sign_mantissa,
                                   df11_params *params, df11_stream_t stream);
 
+/*
+ * Exponent histogram of n BF16 words in device memory: hist[e] (host array
+ * of 256) = how many words have exponent field e (bits 7-14).  The paper has
+ * no counterpart to this entry point: it is the builder's first step on its
+ * own, for callers that want the exponent statistics (entropy, the size a
+ * tensor will compress to) without building.  It allocates nothing: the
+ * device counters are a static buffer of the library (one per device), so
+ * concurrent calls are serialised inside the library.  Queues its work on
+ * `stream` and synchronises it.  d_bf16 must be 2-byte aligned (16-byte
+ * alignment lets the kernel load 8 words at a time).  Errors:
+ * DF11_ERR_NULL, _TOO_LARGE (n >= 2^32), _ALIGN before any device work;
+ * DF11_ERR_CUDA if a CUDA call fails.
+ */
+df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t n, uint64_t hist[256],
+                                    df11_stream_t stream);
+
 /* Release a phase-1 handle without running phase 2 (NULL is a no-op); its
  * scratch is freed in order on the stream phase 1 ran on, which must still
  * exist. */
