@@ -72,6 +72,14 @@ class TensorDesc(ctypes.Structure):
     ]
 
 
+class GemvOp(ctypes.Structure):
+    """df11_gemv: the matrix-vector product applied to one decoded tensor."""
+    _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("cols", ctypes.c_uint32),
+                ("batch", ctypes.c_uint32), ("x_stride", ctypes.c_uint32),
+                ("y_stride", ctypes.c_uint32), ("accumulate", ctypes.c_int32),
+                ("pad", ctypes.c_uint32)]
+
+
 class HostTensor(ctypes.Structure):
     _fields_ = [
         ("params", Params),
@@ -135,6 +143,9 @@ def lib():
     L.df11_gpu_build_finish.restype = ctypes.c_int
     L.df11_gpu_build_free.argtypes = [vp]
     L.df11_gpu_build_free.restype = None
+    L.df11_decode_gemv.argtypes = [ctypes.POINTER(TensorDesc), ctypes.POINTER(GemvOp),
+                                   ctypes.c_int, vp, vp]
+    L.df11_decode_gemv.restype = ctypes.c_int
     L.df11_exponent_histogram.argtypes = [vp, u64, vp, vp]
     L.df11_exponent_histogram.restype = ctypes.c_int
     _lib = L
@@ -456,6 +467,45 @@ class DecodePlan:
                                              err.data_ptr() if err is not None else None,
                                              _stream_handle(stream)), "df11_decode_batched")
         return self._keep[1]
+
+
+def _gemv_op(d: "Df11Device", x: torch.Tensor, y: torch.Tensor, accumulate: bool) -> GemvOp:
+    """Check one (tensor, activations, outputs) triple and describe it."""
+    if len(d.shape) != 2:
+        raise ValueError("decode_gemv needs a 2-D weight (rows x cols)")
+    rows, cols = d.shape
+    if x.dtype not in (torch.bfloat16, torch.int16) or y.dtype != torch.float32:
+        raise TypeError("x must be BF16 and y float32")
+    x2 = x if x.dim() == 2 else x.view(1, -1)
+    y2 = y if y.dim() == 2 else y.view(1, -1)
+    if x2.shape[1] != cols or y2.shape[1] != rows or x2.shape[0] != y2.shape[0]:
+        raise ValueError(f"shapes: W {rows}x{cols}, x {tuple(x.shape)}, y {tuple(y.shape)}")
+    if x2.stride(1) != 1 or y2.stride(1) != 1:
+        raise ValueError("x and y rows must be contiguous")
+    if x2.device != d.device or y2.device != d.device:
+        raise ValueError("x and y must be on the weight's device")
+    return GemvOp(x2.data_ptr(), y2.data_ptr(), cols, x2.shape[0], x2.stride(0),
+                  y2.stride(0), 1 if accumulate else 0, 0)
+
+
+def decode_gemv(ds: Sequence["Df11Device"], xs: Sequence[torch.Tensor],
+                ys: Sequence[torch.Tensor], accumulate: bool = False,
+                err: Optional[torch.Tensor] = None, stream=None):
+    """y = W x (or y += W x) for each compressed weight W (rows x cols) with
+    BF16 activations x (batch x cols, or cols) into float32 y (batch x
+    rows, or rows), decoding W inside the product (df11_decode_gemv): the
+    BF16 weights never reach memory.  One launch per 16 tensors."""
+    if not (len(ds) == len(xs) == len(ys)):
+        raise ValueError("one x and one y per tensor")
+    n = len(ds)
+    if n == 0:
+        return
+    descs = (TensorDesc * n)(*[d.desc(torch.empty(0, device=d.device)) for d in ds])
+    for i, d in enumerate(ds):
+        descs[i].out_bf16 = None
+    ops = (GemvOp * n)(*[_gemv_op(d, x, y, accumulate) for d, x, y in zip(ds, xs, ys)])
+    _check(lib().df11_decode_gemv(descs, ops, n, err.data_ptr() if err is not None else None,
+                                  _stream_handle(stream)), "df11_decode_gemv")
 
 
 def new_error_word(device="cuda") -> torch.Tensor:

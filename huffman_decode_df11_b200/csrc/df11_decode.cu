@@ -83,6 +83,11 @@ struct KTensor {
   uint32_t masked;     // longest codeword > kWideBits: bits past a region may be set
   uint32_t cta_begin;  // first thread block of this tensor
   uint32_t pad;
+  // fused matrix-vector product (df11_decode_gemv): y[b][r] += sum_c W[r][c] x[b][c]
+  // with W the decoded tensor as rows x cols, row-major
+  const uint16_t *x;  // BF16 activations, batch rows of x_stride elements
+  float *y;           // batch rows of y_stride floats
+  uint32_t cols, batch, x_stride, y_stride;
 };
 
 struct KBatch {
@@ -784,6 +789,54 @@ constexpr int kWsStages = 2;
 // that keeps the most thread blocks resident.
 enum SmMode { kSmSlot = 0, kSmGlobal = 1, kSmWarp = 2 };
 
+// ---- fused matrix-vector product -------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// sum over 16 elements of w * x, both BF16, two per word, fp32 arithmetic
+// (BF16 products are exact in fp32)
+__device__ __forceinline__ float dot16(const uint32_t (&w)[8], const uint4 &x0, const uint4 &x1) {
+  const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+  float a = 0.f, b = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    a = fmaf(bf16_lo(w[k]), bf16_lo(xv[k]), a);
+    b = fmaf(bf16_hi(w[k]), bf16_hi(xv[k]), b);
+  }
+  return a + b;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Add the warp's partial sums p (lane l: row `row`, only where `act`) into
+// y[row].  Active lanes hold consecutive 16-element groups, so rows do not
+// decrease across lanes; one or two rows take warp sums and one atomic add
+// each, more rows (matrices narrower than 512 columns) one add per lane.
+__device__ __forceinline__ void warp_row_add(float p, uint32_t row, bool act, float *y,
+                                             int lane) {
+  const uint32_t mask = __ballot_sync(0xFFFFFFFFu, act);
+  if (!mask) return;
+  const uint32_t r0 = __shfl_sync(0xFFFFFFFFu, row, __ffs(mask) - 1);
+  const uint32_t r1 = __shfl_sync(0xFFFFFFFFu, row, 31 - __clz(mask));
+  if (r0 == r1) {
+    const float s = warp_sum(act ? p : 0.f);
+    if (lane == 0) atomicAdd(y + r0, s);
+  } else if (__all_sync(0xFFFFFFFFu, !act || row == r0 || row == r1)) {
+    const float s0 = warp_sum(act && row == r0 ? p : 0.f);
+    const float s1 = warp_sum(act && row == r1 ? p : 0.f);
+    if (lane == 0) {
+      atomicAdd(y + r0, s0);
+      atomicAdd(y + r1, s1);
+    }
+  } else if (act) {
+    atomicAdd(y + row, p);
+  }
+}
+
 template <int T, int C>
 struct WsLayout {
   static constexpr uint32_t bits_bytes = T * C + 16;
@@ -838,9 +891,10 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
 
 // Register budget from the resident thread blocks the shared memory allows:
 // five at 8-byte chunks, at most four from 16 bytes on (more registers there
-// measured about 1% faster).
-template <int T, int C, int SM>
-__global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : (C >= 16 && T == 256 ? 4 : 1280 / T))
+// measured about 1% faster) and for the fused matrix-vector product.
+template <int T, int C, int SM, bool GEMV>
+__global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
+                                          : ((C >= 16 || GEMV) && T == 256 ? 4 : 1280 / T))
     df11_decode_ws_kernel(const __grid_constant__ KBatch kb) {
   using L = WsLayout<T, C>;
   constexpr int NW = C / 4 + 1;
@@ -1067,30 +1121,87 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8 : (C >= 16 && T ==
                         : SM == kSmSlot ? smem_addr(slot + L::head_bytes) + (base - (P0 & ~15u))
                                         : 0u;
     const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
-    {
-      uint32_t g = g_begin + (uint32_t)lane;
-      uint32_t sa_sm = sm + 16u * g, sa_rg = region + 16u * g;
-      uint4 *o = reinterpret_cast<uint4 *>(out) + 2u * g;
-      const uint4 *sp = reinterpret_cast<const uint4 *>(smg) + g;
-      for (; g < g_end; g += 32, sa_sm += 512u, sa_rg += 512u, o += 64, sp += 32) {
-        const uint4 sv = SM == kSmGlobal ? __ldg(sp) : lds128(sa_sm);
-        const uint4 rv = lds128(sa_rg);
-        sts128_zero(sa_rg);  // leave the region zeroed for the next block
-        const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
-        const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
-        o[0] = make_uint4(a.x, a.y, c.x, c.y);
-        o[1] = make_uint4(e2.x, e2.y, f.x, f.y);
+    if constexpr (GEMV) {
+      // the decoded weights go into y += W x instead of to memory: per
+      // 16-element group (within one row, since cols is a multiple of 16)
+      // one partial sum per batch row, summed over the warp per row
+      const uint32_t cols = tk.cols, nb = tk.batch;
+      uint32_t e = base + 16u * (g_begin + (uint32_t)lane);
+      uint32_t row = e / cols, col = e - row * cols;
+      for (uint32_t gg = g_begin; gg < g_end; gg += 32) {
+        const uint32_t g = gg + (uint32_t)lane;
+        const bool act = g < g_end;
+        uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (act) {
+          const uint4 sv = SM == kSmGlobal ? __ldg(reinterpret_cast<const uint4 *>(smg) + g)
+                                           : lds128(sm + 16u * g);
+          const uint4 rv = lds128(region + 16u * g);
+          sts128_zero(region + 16u * g);
+          const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
+          const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+          wv[0] = a.x, wv[1] = a.y, wv[2] = c.x, wv[3] = c.y;
+          wv[4] = e2.x, wv[5] = e2.y, wv[6] = f.x, wv[7] = f.y;
+        }
+        for (uint32_t bi = 0; bi < nb; ++bi) {
+          float p = 0.f;
+          if (act) {
+            const uint4 *xp = reinterpret_cast<const uint4 *>(tk.x + (size_t)bi * tk.x_stride + col);
+            p = dot16(wv, __ldg(xp), __ldg(xp + 1));
+          }
+          warp_row_add(p, row, act, tk.y + (size_t)bi * tk.y_stride, lane);
+        }
+        col += 512u;
+        while (col >= cols) {
+          col -= cols;
+          ++row;
+        }
       }
-    }
-    if (span) {
-      // the elements outside whole groups [g_begin, g_end), one per lane:
-      // lanes 0-15 take the first group, 16-31 the last one (the same group
-      // when there is only one: both lanes then write the same value)
-      const uint32_t i = ((uint32_t)lane & 15u) + (lane >> 4 ? ((span - 1) >> 4) << 4 : 0u);
-      if (i >= head && i < span && (i < (g_begin << 4) || i >= (g_end << 4)))
-        out[i] = fuse1(SM == kSmGlobal ? (uint32_t)__ldg(smg + i) : lds8(sm + i),
-                       lds8(region + i));
-      sts8_zero(region + i);  // the loop zeroed whole groups; this does the rest
+      if (span) {
+        // the elements outside whole groups, one per lane: lanes 0-15 the
+        // first group, 16-31 the last one when it is another group
+        const uint32_t last_g = (span - 1) >> 4;
+        const uint32_t i = ((uint32_t)lane & 15u) + (lane >> 4 ? last_g << 4 : 0u);
+        const bool act = i >= head && i < span && (i < (g_begin << 4) || i >= (g_end << 4)) &&
+                         (lane < 16 || last_g != 0);
+        const uint32_t wbits = act ? fuse1(SM == kSmGlobal ? (uint32_t)__ldg(smg + i) : lds8(sm + i),
+                                           lds8(region + i))
+                                   : 0u;
+        sts8_zero(region + i);  // the loop zeroed whole groups; this does the rest
+        const uint32_t ei = base + i, r = ei / cols, ci = ei - r * cols;
+        const uint32_t half = __ballot_sync(0xFFFFFFFFu, act) >> (lane & 16);
+        for (uint32_t bi = 0; bi < nb; ++bi) {
+          float p = act ? bf16_lo(wbits) * bf16_lo(tk.x[(size_t)bi * tk.x_stride + ci]) : 0.f;
+#pragma unroll
+          for (int o = 8; o; o >>= 1) p += __shfl_xor_sync(0xFFFFFFFFu, p, o);
+          if ((lane & 15) == 0 && (half & 0xFFFFu)) atomicAdd(tk.y + (size_t)bi * tk.y_stride + r, p);
+        }
+      }
+    } else {
+      {
+        uint32_t g = g_begin + (uint32_t)lane;
+        uint32_t sa_sm = sm + 16u * g, sa_rg = region + 16u * g;
+        uint4 *o = reinterpret_cast<uint4 *>(out) + 2u * g;
+        const uint4 *sp = reinterpret_cast<const uint4 *>(smg) + g;
+        for (; g < g_end; g += 32, sa_sm += 512u, sa_rg += 512u, o += 64, sp += 32) {
+          const uint4 sv = SM == kSmGlobal ? __ldg(sp) : lds128(sa_sm);
+          const uint4 rv = lds128(sa_rg);
+          sts128_zero(sa_rg);  // leave the region zeroed for the next block
+          const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
+          const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+          o[0] = make_uint4(a.x, a.y, c.x, c.y);
+          o[1] = make_uint4(e2.x, e2.y, f.x, f.y);
+        }
+      }
+      if (span) {
+        // the elements outside whole groups [g_begin, g_end), one per lane:
+        // lanes 0-15 take the first group, 16-31 the last one (the same group
+        // when there is only one: both lanes then write the same value)
+        const uint32_t i = ((uint32_t)lane & 15u) + (lane >> 4 ? ((span - 1) >> 4) << 4 : 0u);
+        if (i >= head && i < span && (i < (g_begin << 4) || i >= (g_end << 4)))
+          out[i] = fuse1(SM == kSmGlobal ? (uint32_t)__ldg(smg + i) : lds8(sm + i),
+                         lds8(region + i));
+        sts8_zero(region + i);  // the loop zeroed whole groups; this does the rest
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(release);  // slot free for refill
@@ -1170,10 +1281,13 @@ df11_status validate(const df11_tensor &t) {
   return DF11_OK;
 }
 
+// Per-device launch state, indexed by kernel instance: the page-layout
+// kernels use 0-5, the warp-specialised ones 3 * i + mode with i = 3-8
+// (decode) and 12-14 (fused matrix-vector product).
 struct DeviceInfo {
   int sms = 0;
-  std::atomic<size_t> configured[40];  // shared-memory limit set, per kernel instance
-  std::atomic<uint64_t> occupancy[40]; // last (smem << 8 | blocks per SM), per instance
+  std::atomic<size_t> configured[64];  // shared-memory limit set, per kernel instance
+  std::atomic<uint64_t> occupancy[64]; // last (smem << 8 | blocks per SM), per instance
 };
 
 DeviceInfo &device_info(int dev) {
@@ -1304,12 +1418,12 @@ size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t regio
 // warp's own buffer, whichever keeps more thread blocks resident (the slot
 // on a tie); read from global memory only when neither fits.  Measured: at
 // equal residency the slot beats the warp buffer, which beats global reads.
-template <int T, int C>
+template <int T, int C, bool GEMV = false>
 df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
-  void (*kern[3])(KBatch) = {df11_decode_ws_kernel<T, C, kSmSlot>,
-                             df11_decode_ws_kernel<T, C, kSmGlobal>,
-                             df11_decode_ws_kernel<T, C, kSmWarp>};
+  void (*kern[3])(KBatch) = {df11_decode_ws_kernel<T, C, kSmSlot, GEMV>,
+                             df11_decode_ws_kernel<T, C, kSmGlobal, GEMV>,
+                             df11_decode_ws_kernel<T, C, kSmWarp, GEMV>};
   const size_t smem[3] = {ws_shared_bytes(C, T, sm_stage, kb.stage_bytes, kb.sub_words, false),
                           ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, false),
                           ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, true)};
@@ -1350,7 +1464,7 @@ size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t regio
 }
 
 df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaStream_t s,
-                         bool ws) {
+                         bool ws, const df11_gemv *ops = nullptr) {
   KBatch kb{};
   kb.err = d_err;
   uint32_t blocks[DF11_MAX_BATCH];
@@ -1376,6 +1490,14 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     k.max_chunk_elems = p.max_chunk_elems;
     k.max_warp_elems = p.max_warp_elems;
     k.masked = p.max_len > (uint32_t)kWideBits ? 1u : 0u;
+    if (ops) {
+      k.x = ops[i].x;
+      k.y = ops[i].y;
+      k.cols = ops[i].cols;
+      k.batch = ops[i].batch;
+      k.x_stride = ops[i].x_stride;
+      k.y_stride = ops[i].y_stride;
+    }
     blocks[kb.count] = p.num_blocks;
     ++kb.count;
     max_elems = max_elems > p.max_block_elems ? max_elems : p.max_block_elems;
@@ -1395,6 +1517,12 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     // and spend the shared memory on resident thread blocks
     kb.sub_words = 0;
     const uint32_t sm_stage = stage_bytes_for(max_elems);
+    if (ops) {
+      if (T == 256 && C == 8) return launch_ws<256, 8, true>(kb, blocks, sm_stage, s, 12);
+      if (T == 256 && C == 16) return launch_ws<256, 16, true>(kb, blocks, sm_stage, s, 13);
+      if (T == 256 && C == 24) return launch_ws<256, 24, true>(kb, blocks, sm_stage, s, 14);
+      return DF11_ERR_UNSUPPORTED;
+    }
     if (T == 256 && C == 8) return launch_ws<256, 8>(kb, blocks, sm_stage, s, 3);
     if (T == 256 && C == 4) return launch_ws<256, 4>(kb, blocks, sm_stage, s, 4);
     if (T == 256 && C == 16) return launch_ws<256, 16>(kb, blocks, sm_stage, s, 5);
@@ -1414,7 +1542,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   if (T == 256 && C == 8) return launch<256, 8>(kb, blocks, smem, s, 0);
   if (T == 256 && C == 4) return launch<256, 4>(kb, blocks, smem, s, 1);
   if (T == 256 && C == 16) return launch<256, 16>(kb, blocks, smem, s, 2);
-  if (T == 256 && C == 24) return launch<256, 24>(kb, blocks, smem, s, 33);
+  if (T == 256 && C == 24) return launch<256, 24>(kb, blocks, smem, s, 5);
   if (T == 128 && C == 8) return launch<128, 8>(kb, blocks, smem, s, 3);
   if (T == 512 && C == 8) return launch<512, 8>(kb, blocks, smem, s, 4);
   return DF11_ERR_UNSUPPORTED;
@@ -1475,6 +1603,71 @@ df11_status df11_decode_batched(const df11_tensor *tensors, int count, int32_t *
   for (int i = 0; i < count; i += DF11_MAX_BATCH) {
     const int c = count - i < DF11_MAX_BATCH ? count - i : DF11_MAX_BATCH;
     df11_status st = launch_batch(tensors + i, c, d_err, (cudaStream_t)stream);
+    if (st != DF11_OK) return st;
+  }
+  return DF11_OK;
+}
+
+df11_status df11_decode_gemv(const df11_tensor *tensors, const df11_gemv *ops, int count,
+                             int32_t *d_err, df11_stream_t stream) {
+  if (count < 0) return DF11_ERR_INVALID;
+  if (count == 0) return DF11_OK;
+  if (!tensors || !ops) return DF11_ERR_NULL;
+  if (d_err && !aligned(d_err, 4)) return DF11_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t C = 0, T = 0;
+  for (int i = 0; i < count; ++i) {
+    const df11_tensor &t = tensors[i];
+    const df11_gemv &g = ops[i];
+    const df11_params &p = t.params;
+    if (!g.y || (p.n && !g.x)) return DF11_ERR_NULL;
+    if (g.cols == 0 || g.cols % 16 || p.n % g.cols) return DF11_ERR_INVALID;
+    const uint64_t rows = p.n / g.cols;
+    if (g.batch < 1 || g.batch > DF11_GEMV_MAX_BATCH) return DF11_ERR_INVALID;
+    if (g.x_stride < g.cols || g.x_stride % 8 || g.y_stride < rows) return DF11_ERR_INVALID;
+    if (!aligned(g.x, 16) || !aligned(g.y, 4)) return DF11_ERR_ALIGN;
+    df11_tensor v = t;
+    v.out_bf16 = reinterpret_cast<uint16_t *>(16);  // not written; passes the output checks
+    const df11_status st = validate(v);
+    if (st != DF11_OK) return st;
+    if (p.n == 0) continue;
+    if (!t.chunk_counts) return DF11_ERR_UNSUPPORTED;
+    if (C == 0) {
+      C = p.chunk_bytes;
+      T = p.threads_per_block;
+    } else if (C != p.chunk_bytes || T != p.threads_per_block) {
+      return DF11_ERR_INVALID;
+    }
+  }
+  if (C && !(T == 256 && (C == 8 || C == 16 || C == 24))) return DF11_ERR_UNSUPPORTED;
+  // y = W x: clear the outputs first, in stream order
+  for (int i = 0; i < count; ++i) {
+    const df11_gemv &g = ops[i];
+    if (g.accumulate) continue;
+    const uint64_t rows = tensors[i].params.n / g.cols;
+    if (g.y_stride == rows) {
+      if (cudaMemsetAsync(g.y, 0, (size_t)g.batch * rows * sizeof(float), s) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    } else {
+      for (uint32_t b = 0; b < g.batch; ++b)
+        if (cudaMemsetAsync(g.y + (size_t)b * g.y_stride, 0, rows * sizeof(float), s) !=
+            cudaSuccess)
+          return DF11_ERR_CUDA;
+    }
+  }
+  for (int i = 0; i < count; i += DF11_MAX_BATCH) {
+    const int c = count - i < DF11_MAX_BATCH ? count - i : DF11_MAX_BATCH;
+    df11_tensor ts[DF11_MAX_BATCH];
+    df11_gemv gs[DF11_MAX_BATCH];
+    int m = 0;
+    for (int j = 0; j < c; ++j) {
+      if (tensors[i + j].params.n == 0) continue;
+      ts[m] = tensors[i + j];
+      gs[m] = ops[i + j];
+      ++m;
+    }
+    if (!m) continue;
+    const df11_status st = launch_group(ts, m, d_err, s, true, gs);
     if (st != DF11_OK) return st;
   }
   return DF11_OK;

@@ -168,6 +168,46 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
 df11_status df11_decode_batched(const df11_tensor *tensors, int count,
                                 int32_t *d_err, df11_stream_t stream);
 
+/* Largest batch (activation rows) one df11_decode_gemv operation takes. */
+#define DF11_GEMV_MAX_BATCH 8
+
+/* The matrix-vector product applied to one decoded tensor. */
+typedef struct df11_gemv {
+  const uint16_t *x;   /* BF16 activations (device, 16-byte aligned): `batch` rows of
+                          `cols` elements, row b at x + b*x_stride */
+  float *y;            /* fp32 outputs (device, 4-byte aligned): `batch` rows of
+                          n/cols elements, row b at y + b*y_stride */
+  uint32_t cols;       /* in-features: the decoded tensor is (n/cols) x cols, row-major;
+                          a multiple of 16 that divides n */
+  uint32_t batch;      /* 1 .. DF11_GEMV_MAX_BATCH */
+  uint32_t x_stride;   /* elements between activation rows: >= cols, a multiple of 8 */
+  uint32_t y_stride;   /* elements between output rows: >= n/cols */
+  int32_t accumulate;  /* 0: y = W x (the call clears y first, in stream order);
+                          otherwise y += W x */
+  uint32_t pad;
+} df11_gemv;
+
+/*
+ * Decode-and-multiply without writing the decoded tensor anywhere: for each
+ * tensor W (rows x cols) and its df11_gemv op, y[b][r] (+)= sum over c of
+ * W[r][c] * x[b][c], the decoded BF16 weights taken straight from the decode
+ * kernel's registers into fp32 fused multiply-adds.  This is the pages'
+ * "decode just before the matmul" ("DFloat11无损压缩技术" (jsqmd.com) §2.2
+ * item 3; "DFloat11重新定义LLM无损压缩的技术边界" (ocdem.com) §2.2) for
+ * batch-1 and small-batch matrix-vector products, without the round trip of
+ * the BF16 weights through memory.  Needs chunk counts and T = 256 with
+ * C = 8, 16 or 24; out_bf16 is not used (may be NULL).  Every product
+ * w*x is exact in fp32; the sums run in fp32 in an order that depends on
+ * scheduling (atomic adds per row segment), so y may differ from run to
+ * run in the last bits, within the usual bound for an fp32 sum of cols
+ * terms.  Same conventions as df11_decode_batched otherwise (asynchronous,
+ * no allocation, device-detected errors in d_err); the activations may be
+ * written by the previous kernel in the stream.  DF11_ERR_INVALID for a
+ * cols, batch or stride outside the rules above.
+ */
+df11_status df11_decode_gemv(const df11_tensor *tensors, const df11_gemv *ops, int count,
+                             int32_t *d_err, df11_stream_t stream);
+
 /*
  * Derive, on the device, the decode table of one tensor from its luts and
  * code_lengths (device pointers, as in df11_tensor) into `out` (device,

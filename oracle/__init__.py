@@ -21,6 +21,12 @@ build_luts                  every entry re-derived by brute-force parsing
 encode / decode             round trip on every synthetic workload; decoded
                             hand-written bit strings in tests/golden/
 metadata_from_starts        brute-force gap / block position definitions
+bf16_to_f64                 hand-checked values (1, -2, the smallest subnormal,
+                            infinity); every finite pattern widens and narrows
+                            back exactly
+gemv                        exact rational sums (fractions.Fraction) of tiny
+                            products; one-hot activations return the decoded
+                            weight columns exactly
 ==========================  ==================================================
 
 No function is left "parity unpinned".
@@ -317,3 +323,27 @@ def roundtrip(w, chunk_bytes: int = 8, threads_per_block: int = 256):
     if end != f.total_bits:
         raise ValueError("decode did not end at the last encoded bit")
     return f, out
+
+
+def bf16_to_f64(words) -> np.ndarray:
+    """BF16 bit patterns (any 2-byte array) as float64: a BF16 word is the top
+    half of the float32 with the same bits, and float32 widens to float64
+    exactly."""
+    u = np.ascontiguousarray(words).view(np.uint16).astype(np.uint32) << 16
+    with np.errstate(invalid="ignore"):  # NaN patterns stay NaN
+        return u.view(np.float32).astype(np.float64)
+
+
+def gemv(bitstream, code_lengths, sign_mantissa, n: int, cols: int, x) -> np.ndarray:
+    """y = W x for the tensor W that the stream decodes to, taken as
+    (n / cols) x cols row-major (a weight applied right after its decode,
+    "DFloat11无损压缩技术" (jsqmd.com) §2.2 item 3), and BF16 activations x
+    (batch x cols, or cols).  Float64 throughout: the decoded weights and the
+    activations widen exactly, and the product is one library matmul.
+    Returns float64 of shape (batch, n / cols)."""
+    if cols <= 0 or n % cols:
+        raise ValueError("cols must divide n")
+    w, end, _ = decode(bitstream, code_lengths, sign_mantissa, n)
+    W = bf16_to_f64(w).reshape(n // cols, cols)
+    X = bf16_to_f64(np.ascontiguousarray(x)).reshape(-1, cols)
+    return X @ W.T

@@ -135,6 +135,27 @@ def test_device_builder_host_validation():
         df11.compress_on_device(df11.torch.zeros(4, dtype=df11.torch.int16))
 
 
+def test_gemv_host_validation():
+    """df11_decode_gemv rejects bad arguments before any CUDA call."""
+    L = df11.lib()
+    t = (df11.TensorDesc * 1)(df11.TensorDesc(*[FAKE] * 7, None, None,
+                                              _params(n=4096 * 64, chunk_bytes=24)))
+    def op(**kw):
+        f = dict(x=FAKE, y=FAKE, cols=4096, batch=1, x_stride=4096, y_stride=64, accumulate=0,
+                 pad=0)
+        f.update(kw)
+        return (df11.GemvOp * 1)(df11.GemvOp(**f))
+    assert L.df11_decode_gemv(t, op(), 0, None, None) == 0
+    assert L.df11_decode_gemv(None, op(), 1, None, None) == 1
+    assert L.df11_decode_gemv(t, None, 1, None, None) == 1
+    assert L.df11_decode_gemv(t, op(), -1, None, None) == 7
+    assert L.df11_decode_gemv(t, op(cols=4095), 1, None, None) == 7
+    assert L.df11_decode_gemv(t, op(batch=9), 1, None, None) == 7
+    assert L.df11_decode_gemv(t, op(y_stride=63), 1, None, None) == 7
+    assert L.df11_decode_gemv(t, op(x=FAKE + 2), 1, None, None) == 2
+    assert L.df11_decode_gemv(t, op(x=None), 1, None, None) == 1
+
+
 def test_supported_shapes_and_shared_bytes():
     assert df11.supported(8, 256) and df11.supported(4, 256) and df11.supported(16, 256)
     assert df11.supported(24, 256) and not df11.supported(20, 256)

@@ -429,3 +429,63 @@ def test_size_claim_about_eleven_bits_per_weight():
                  32 * (f.num_blocks + 1) + 32 * 256 * f.num_luts + 8 * 256)
         bpw = total / f.n
         assert 10.5 <= bpw <= 11.2, bpw
+
+
+# --- the matrix-vector product (oracle.gemv) --------------------------------
+
+def test_bf16_widening_hand_checked_values():
+    words = np.array([0x3F80, 0xC000, 0x0001, 0x7F80, 0x8000, 0x3E80], np.uint16)
+    got = oracle.bf16_to_f64(words)
+    assert got[0] == 1.0 and got[1] == -2.0
+    assert got[2] == 2.0 ** -133  # smallest positive subnormal: 2^-126 * 2^-7
+    assert math.isinf(got[3]) and got[3] > 0
+    assert got[4] == 0.0 and math.copysign(1.0, got[4]) == -1.0
+    assert got[5] == 0.25
+
+
+def test_bf16_widening_is_exact_on_every_finite_pattern():
+    w = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    f = oracle.bf16_to_f64(w)
+    fin = np.isfinite(f)
+    back = (f[fin].astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(back, w[fin])
+    assert np.all((f[fin].astype(np.float32).view(np.uint32) & 0xFFFF) == 0)
+
+
+def _exact_value(word: int):
+    """A finite BF16 word as an exact rational, from its fields."""
+    from fractions import Fraction
+    s, e, m = word >> 15, (word >> 7) & 0xFF, word & 0x7F
+    v = Fraction(m, 128) * Fraction(2) ** -126 if e == 0 else \
+        (1 + Fraction(m, 128)) * Fraction(2) ** (e - 127)
+    return -v if s else v
+
+
+@pytest.mark.parametrize("rows,cols,batch,seed", [(3, 16, 1, 0), (5, 32, 2, 1), (2, 48, 3, 2)])
+def test_gemv_matches_exact_rational_sums(rows, cols, batch, seed):
+    rng = np.random.default_rng(seed)
+    w = (np.float32(rng.normal(0, 0.05, rows * cols)).view(np.uint32) >> 16).astype(np.uint16)
+    x = (np.float32(rng.normal(0, 1.0, batch * cols)).view(np.uint32) >> 16).astype(np.uint16)
+    f = oracle.encode(w, 8, 128)
+    y = oracle.gemv(f.bitstream, f.code_lengths, f.sign_mantissa, f.n, cols, x)
+    assert y.shape == (batch, rows)
+    for b in range(batch):
+        for r in range(rows):
+            terms = [_exact_value(int(w[r * cols + c])) * _exact_value(int(x[b * cols + c]))
+                     for c in range(cols)]
+            exact = sum(terms)
+            bound = cols * 2.0 ** -53 * float(sum(abs(t) for t in terms))
+            assert abs(y[b, r] - float(exact)) <= bound + 1e-300
+
+
+def test_gemv_one_hot_activations_return_weight_columns():
+    rng = np.random.default_rng(7)
+    rows, cols = 6, 32
+    w = (np.float32(rng.normal(0, 0.02, rows * cols)).view(np.uint32) >> 16).astype(np.uint16)
+    f = oracle.encode(w, 8, 128)
+    W = oracle.bf16_to_f64(w).reshape(rows, cols)
+    for j in (0, 5, 31):
+        x = np.zeros(cols, np.uint16)
+        x[j] = 0x3F80  # 1.0
+        y = oracle.gemv(f.bitstream, f.code_lengths, f.sign_mantissa, f.n, cols, x)
+        assert np.array_equal(y[0], W[:, j])  # column j, row by row: no transpose slip
