@@ -46,6 +46,8 @@ import workloads  # noqa: E402
 METRIC = ("decoded BF16 GB/s and % of HBM roofline (1×B200), "
           "bit-exact vs CPU oracle")
 UNIT = "GB/s"
+GEMV_METRIC = ("BF16-equivalent weight GB/s through the fused decode and matrix-vector "
+               "product (1×B200), within the fp32 sum bound of the exact product")
 BUILD_METRIC = ("compressed BF16 GB/s (device-side format builder, 1×B200), "
                 "byte-identical to the host builder")
 # launches of the library's own kernels per device build: histogram, sums,
@@ -74,7 +76,7 @@ def workload_units(config: str, seed: int):
         return [("embed_151936x4096", lambda d: workloads.embedding(seed, d))]
     if config == "stack":
         return [(name, thunk) for name, _, thunk in workloads.stack_units(seed)]
-    if config == "build":  # the block's tensors, compressed on the device
+    if config in ("build", "gemv"):  # the block's tensors
         return workload_units("block", seed)
     if config == "offload":  # the stack's first layers, without embedding and LM head
         return [(name, thunk) for name, _, thunk
@@ -669,6 +671,132 @@ def run_build(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_gemv(args, world, rank, local):
+    """y = W x for each weight of the block, W decoded inside the product
+    (decode_gemv: one launch for the seven weights, the BF16 weights never
+    written), against the same product done in two steps (batched decode
+    into a BF16 scratch buffer, then a cuBLAS matrix-vector product per
+    weight) and against BF16 weights kept uncompressed (cuBLAS alone).
+    Parity: every output within the fp32 summation bound of the float64
+    product of the original weights, before timing."""
+    import huffman_decode_df11_b200 as df11
+    device = f"cuda:{local}"
+    seed = args.seed + rank
+    B = args.batch
+    if not 1 <= B <= 8:
+        raise SystemExit("--batch must be 1..8")
+    units = workload_units(args.config, seed)
+    shapes = [(r, c) for _, r, c in workloads.BLOCK_SHAPES]
+    hosts, ds, ws_bf16 = [], [], []
+    for (name, thunk), shape in zip(units, shapes):
+        bits = thunk(device)
+        h = df11.compress(bits, chunk_bytes=args.chunk_bytes,
+                          threads_per_block=args.threads_per_block)
+        h.shape = shape
+        hosts.append(h)
+        ds.append(df11.to_device(h, device))
+        ws_bf16.append(bits.view(shape).view(torch.bfloat16))
+    n_total = sum(h.n for h in hosts)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 77)
+    xs = [torch.randn(B, c, generator=g, device=device).to(torch.bfloat16) for _, c in shapes]
+    ys = [torch.empty(B, r, dtype=torch.float32, device=device) for r, _ in shapes]
+    err = df11.new_error_word(device)
+    stream = torch.cuda.current_stream()
+
+    # parity: within gamma_cols * |x||W|^T of the float64 product
+    df11.decode_gemv(ds, xs, ys, err=err)
+    torch.cuda.synchronize()
+    df11.check_device_error(err)
+    for (name, _), (r, c), x, y, w in zip(units, shapes, xs, ys, ws_bf16):
+        W = w.double()
+        ref = x.double() @ W.T
+        k = c * 2.0 ** -24
+        bound = (k / (1 - k)) * (x.double().abs() @ W.abs().T)
+        if not torch.all((y.double() - ref).abs() <= bound):
+            raise SystemExit(f"gemv outside the fp32 bound on {name}")
+        del W, ref, bound
+
+    scratch = torch.empty(max(h.n for h in hosts), dtype=torch.bfloat16, device=device)
+    plans = [df11.DecodePlan([d], [scratch[: d.n]]) for d in ds]
+
+    def fused():
+        df11.decode_gemv(ds, xs, ys, err=err, stream=stream)
+
+    ybs = [torch.empty(B, r, dtype=torch.bfloat16, device=device) for r, _ in shapes]
+
+    def two_step():  # decode each weight into the scratch buffer, then cuBLAS (BF16 out)
+        for plan, d, x, yb, (r, c) in zip(plans, ds, xs, ybs, shapes):
+            plan.run(err=err, stream=stream)
+            torch.matmul(x, scratch[: d.n].view(r, c).T, out=yb)
+
+    def bf16():  # uncompressed weights resident in HBM, cuBLAS (BF16 out)
+        for w, x, yb in zip(ws_bf16, xs, ybs):
+            torch.matmul(x, w.T, out=yb)
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return a.elapsed_time(b) / steps
+
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t_busy = time.perf_counter()
+        while time.perf_counter() - t_busy < 0.4:
+            fused()
+            torch.cuda.synchronize()
+        ms_local = timed(fused, args.steps)
+    df11.check_device_error(err)
+    ms_two = timed(two_step, max(3, args.steps // 4))
+    ms_bf16 = timed(bf16, max(3, args.steps // 4))
+    ms = max_over_ranks(ms_local, world)
+    value = sum_over_ranks(2.0 * n_total, world) / (ms * 1e-3) / 1e9
+    alg = sum(algorithmic_bytes(h) - 2 * h.n for h in hosts) + \
+        sum(x.numel() * 2 for x in xs) + sum(y.numel() * 4 for y in ys)
+    achieved = alg / (ms_local * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    if rank == 0:
+        line = {
+            "metric": GEMV_METRIC, "value": round(value, 2), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32",
+            "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
+            "config": {
+                "workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
+                "elements": n_total, "batch": B, "chunk_bytes": args.chunk_bytes,
+                "threads_per_block": args.threads_per_block,
+                "l2": "inputs larger than L2 (no flush)",
+                "parallelism": f"replicas x{world} (no collective)",
+                "parity": "every output within gamma_cols*|x||W|^T of the float64 product "
+                          "of the original weights, before timing",
+                "y": "y = W x (the call clears y first)",
+            },
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_step": alg,
+                         "kernel": "df11_decode_ws_kernel (fused product epilogue), one "
+                                   "launch per step for the seven weights"},
+            "decode_then_cublas": {"ms_per_step": round(ms_two, 4),
+                                   "value": round(2.0 * n_total / (ms_two * 1e-3) / 1e9, 2)},
+            "bf16_cublas": {"ms_per_step": round(ms_bf16, 4),
+                            "value": round(2.0 * n_total / (ms_bf16 * 1e-3) / 1e9, 2)},
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+            "e2e": None,
+            "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def _oracle_encode_sample(ws, budget_s: float):
     """Encode leading slices of the workload's tensors with the oracle until
     the budget is spent; returns (elements, seconds, description)."""
@@ -867,6 +995,8 @@ WORKLOAD_NAMES = {
     "fibonacci": "Fibonacci exponent counts (32-bit codewords), 14,930,351 elems",
     "embedding": "embedding 151936x4096 N(0,0.02), 622,329,856 elems",
     "stack": "36-layer Qwen3-8B-shaped stack + embedding + LM head, 8,190,427,136 elems",
+    "gemv": "fused decode and matrix-vector product: Qwen3-8B-shaped block "
+            "(q,k,v,o,gate,up,down), 192,937,984 weights, BF16 activations",
     "build": "format builder on the GPU: Qwen3-8B-shaped block (q,k,v,o,gate,up,down) "
              "compressed from BF16 in HBM, 192,937,984 elems",
     "offload": f"{OFFLOAD_LAYERS} Qwen3-8B-shaped layers streamed from pinned host memory "
@@ -887,6 +1017,8 @@ def main(argv=None):
                     help="bitstream bytes per chunk (C) of the compressed format")
     ap.add_argument("--threads-per-block", type=int, default=256, choices=[128, 256, 512],
                     help="chunks per format block (T) of the compressed format")
+    ap.add_argument("--batch", type=int, default=1,
+                    help="activation rows of the gemv workload (1-8)")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -909,6 +1041,8 @@ def main(argv=None):
                 run_offload(args, world, rank, local)
             elif args.config == "build":
                 run_build(args, world, rank, local)
+            elif args.config == "gemv":
+                run_gemv(args, world, rank, local)
             else:
                 run_b200(args, world, rank, local)
     finally:
