@@ -141,6 +141,10 @@ def lib():
     L.df11_gpu_build_finish.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                         ctypes.POINTER(Params), vp]
     L.df11_gpu_build_finish.restype = ctypes.c_int
+    L.df11_gpu_build_begin_batched.argtypes = [vp, vp, ctypes.c_int, u32, u32, vp, vp, vp, vp]
+    L.df11_gpu_build_begin_batched.restype = ctypes.c_int
+    L.df11_gpu_build_finish_batched.argtypes = [vp, ctypes.c_int, vp, vp, vp, vp]
+    L.df11_gpu_build_finish_batched.restype = ctypes.c_int
     L.df11_gpu_build_free.argtypes = [vp]
     L.df11_gpu_build_free.restype = None
     L.df11_decode_gemv.argtypes = [ctypes.POINTER(TensorDesc), ctypes.POINTER(GemvOp),
@@ -310,56 +314,89 @@ def to_device(h: Df11Host, device="cuda", decode_table: bool = True) -> Df11Devi
     return d
 
 
+class GpuBuildOut(ctypes.Structure):
+    """df11_gpu_build_out: one tensor's phase-2 output buffers."""
+    _fields_ = [(f, ctypes.c_void_p) for f in ("bitstream", "gaps", "chunk_counts",
+                                               "block_out_pos", "luts", "code_lengths",
+                                               "sign_mantissa")]
+
+
 def compress_on_device(w: torch.Tensor, chunk_bytes: int = 24, threads_per_block: int = 256,
                        stream=None, decode_table: bool = True) -> Df11Device:
     """Encode a BF16 tensor that is in device memory into DF11 on the device
     (df11_gpu_build_begin / df11_gpu_build_finish): the same bytes and
     parameters as compress() of the same words, written straight into
     device buffers.  Synchronises the stream."""
-    if not w.is_cuda:
-        raise ValueError("compress_on_device takes a CUDA tensor; use compress() for host data")
-    if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
-        raise TypeError(f"expected BF16 words (bfloat16, int16 or uint16), got {w.dtype}")
-    shape = tuple(w.shape)
-    flat = w.contiguous().reshape(-1)
-    n = flat.numel()
-    ptr = flat.data_ptr() if n else None
+    return compress_on_device_batched([w], chunk_bytes, threads_per_block, stream,
+                                      decode_table)[0]
+
+
+def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24,
+                               threads_per_block: int = 256, stream=None,
+                               decode_table: bool = True) -> List[Df11Device]:
+    """compress_on_device for several tensors, with one stream
+    synchronisation per phase for all of them
+    (df11_gpu_build_begin_batched / _finish_batched)."""
+    count = len(ws)
+    if count == 0:
+        return []
+    flats, shapes = [], []
+    for w in ws:
+        if not w.is_cuda:
+            raise ValueError("compress_on_device takes CUDA tensors; use compress() for host data")
+        if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+            raise TypeError(f"expected BF16 words (bfloat16, int16 or uint16), got {w.dtype}")
+        shapes.append(tuple(w.shape))
+        flats.append(w.contiguous().reshape(-1))
     L = lib()
     sh = _stream_handle(stream)
-    p = Params()
-    lens = (ctypes.c_uint8 * 256)()
-    handle = ctypes.c_void_p()
-    _check(L.df11_gpu_build_begin(ptr, n, chunk_bytes, threads_per_block, sh, ctypes.byref(p),
-                                  ctypes.cast(lens, ctypes.c_void_p), ctypes.byref(handle)),
-           "df11_gpu_build_begin")
+    vp = ctypes.c_void_p
+    ptrs = (vp * count)(*[f.data_ptr() if f.numel() else None for f in flats])
+    ns = (ctypes.c_uint64 * count)(*[f.numel() for f in flats])
+    params = (Params * count)()
+    lens = (ctypes.c_uint8 * (256 * count))()
+    handles = (vp * count)()
+    _check(L.df11_gpu_build_begin_batched(ptrs, ns, count, chunk_bytes, threads_per_block, sh,
+                                          params, ctypes.cast(lens, vp), handles),
+           "df11_gpu_build_begin_batched")
+    outs = (GpuBuildOut * count)()
+    views = []
     try:
-        chunks = int(p.num_blocks) * threads_per_block
-        dev = w.device
+        for i, (f, p) in enumerate(zip(flats, params)):
+            chunks = int(p.num_blocks) * threads_per_block
+            dev = f.device
 
-        def buf(count, dtype=torch.uint8):
-            # at least 16 bytes so that no pointer is NULL; the view has `count`
-            t = torch.empty(max(count, 16), dtype=dtype, device=dev)
-            return t, t[:count]
+            def buf(cnt, dtype=torch.uint8):
+                # at least 16 bytes so that no pointer is NULL; the view has `cnt`
+                t = torch.empty(max(cnt, 16), dtype=dtype, device=dev)
+                return t, t[:cnt]
 
-        bs, bs_v = buf(chunks * chunk_bytes + 16)
-        gp, gp_v = buf(chunks * 5 // 8 + 16)
-        cc, cc_v = buf(chunks + 16)
-        bp, bp_v = buf(int(p.num_blocks) + 1, torch.int32)
-        lu, lu_v = buf(int(p.num_luts) * 256, torch.int32)
-        cl, cl_v = buf(256)
-        sm, sm_v = buf((n + 15) // 16 * 16)
+            bs = buf(chunks * chunk_bytes + 16)
+            gp = buf(chunks * 5 // 8 + 16)
+            cc = buf(chunks + 16)
+            bp = buf(int(p.num_blocks) + 1, torch.int32)
+            lu = buf(int(p.num_luts) * 256, torch.int32)
+            cl = buf(256)
+            sm = buf((f.numel() + 15) // 16 * 16)
+            outs[i] = GpuBuildOut(bs[0].data_ptr(), gp[0].data_ptr(), cc[0].data_ptr(),
+                                  bp[0].data_ptr(), lu[0].data_ptr(), cl[0].data_ptr(),
+                                  sm[0].data_ptr())
+            views.append((bs[1], gp[1], cc[1], bp[1], lu[1], cl[1], sm[1]))
     except BaseException:
-        L.df11_gpu_build_free(handle)
+        for hnd in handles:
+            L.df11_gpu_build_free(hnd)
         raise
-    st = L.df11_gpu_build_finish(handle, ptr, bs.data_ptr(), gp.data_ptr(), cc.data_ptr(),
-                                 bp.data_ptr(), lu.data_ptr(), cl.data_ptr(), sm.data_ptr(),
-                                 ctypes.byref(p), sh)
-    _check(st, "df11_gpu_build_finish")
-    d = Df11Device(params=p, bitstream=bs_v, gaps=gp_v, block_out_pos=bp_v, luts=lu_v,
-                   code_lengths=cl_v, sign_mantissa=sm_v, chunk_counts=cc_v, shape=shape)
-    if decode_table:
-        d.decode_table = build_decode_table(d, stream)
-    return d
+    _check(L.df11_gpu_build_finish_batched(handles, count, ptrs, outs, params, sh),
+           "df11_gpu_build_finish_batched")
+    out = []
+    for p, v, shape in zip(params, views, shapes):
+        d = Df11Device(params=Params.from_buffer_copy(p), bitstream=v[0], gaps=v[1],
+                       chunk_counts=v[2], block_out_pos=v[3], luts=v[4], code_lengths=v[5],
+                       sign_mantissa=v[6], shape=shape)
+        if decode_table:
+            d.decode_table = build_decode_table(d, stream)
+        out.append(d)
+    return out
 
 
 def exponent_histogram(w: torch.Tensor, stream=None) -> np.ndarray:

@@ -52,9 +52,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kPerThread = 8;
 constexpr int kPerCta = kThreads * kPerThread;  // elements per pack block
-// words a pack block's codewords can touch: 2048 codewords of at most 32
-// bits after an offset of at most 31 bits
-constexpr int kCtaWords = kPerCta + 1;
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 __device__ __forceinline__ uint32_t exponent(uint32_t x) { return (x >> 7) & 0xFFu; }
@@ -171,62 +168,77 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const uint16_t *w, uint6
 }
 
 // ---- bit offsets ---------------------------------------------------------
-constexpr int kSumsBlocks = 4;  // pack blocks per iteration of the sums kernel
+// The pack kernel works in units of 256 elements (one warp, 8 per lane).  A
+// sums thread block walks a contiguous range of units, 32 per iteration
+// (four per warp), and keeps a running total, so it writes each unit's first
+// bit relative to its range, and the range's total.
+constexpr int kUnit = 32 * kPerThread;        // elements per unit
+constexpr int kUnitWords = kUnit + 1;         // words a unit's codewords can touch
+constexpr int kUnitsPerWarp = 4;              // per iteration of the sums kernel
+constexpr int kUnitsPerIter = (kThreads / 32) * kUnitsPerWarp;
+static_assert(kUnitsPerIter == 32, "one warp scans an iteration's units");
 
 struct Ranges {
-  uint64_t pack_ctas;  // pack blocks
-  uint64_t per;        // pack blocks per range (one range per sums thread block)
-  uint32_t *local;     // first bit of each pack block within its range
+  uint64_t units;  // units of the tensor
+  uint64_t per;    // units per range (one range per sums thread block)
+  uint32_t *local; // first bit of each unit within its range
   unsigned long long *range_start;  // first bit of each range; the total after the last
 };
 
-// pack blocks and ranges number below 2^21: 32-bit division
-__device__ __forceinline__ unsigned long long pack_start(const Ranges &r, uint64_t pb) {
-  return r.range_start[(uint32_t)pb / (uint32_t)r.per] + r.local[pb];
+// units and ranges number below 2^24: 32-bit division
+__device__ __forceinline__ unsigned long long unit_start(const Ranges &r, uint64_t u) {
+  return r.range_start[(uint32_t)u / (uint32_t)r.per] + r.local[u];
 }
 
 __global__ void __launch_bounds__(kThreads, 4) sums_kernel(const uint16_t *w, uint64_t n, bool vec,
-                                                        const uint2 *tab, const Ranges r,
-                                                        unsigned long long *range_total) {
+                                                           const uint2 *tab, const Ranges r,
+                                                           unsigned long long *range_total) {
   __shared__ uint8_t len[256];
-  __shared__ uint32_t part[kSumsBlocks][kThreads / 32];
+  __shared__ uint32_t part[kUnitsPerIter];
   len[threadIdx.x] = (uint8_t)tab[threadIdx.x].y;
-  const uint64_t pb_begin = (uint64_t)blockIdx.x * r.per;
-  const uint64_t pb_end = pb_begin + r.per < r.pack_ctas ? pb_begin + r.per : r.pack_ctas;
-  const uint64_t me = (uint64_t)threadIdx.x * kPerThread;
-  uint4 next[kSumsBlocks];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint64_t u_begin = (uint64_t)blockIdx.x * r.per;
+  const uint64_t u_end = u_begin + r.per < r.units ? u_begin + r.per : r.units;
+  const uint64_t me = (uint64_t)lane * kPerThread;
+  uint4 next[kUnitsPerWarp];
 #pragma unroll
-  for (int j = 0; j < kSumsBlocks; ++j)
-    next[j] = pb_begin + j < pb_end ? load8(w, n, (pb_begin + j) * kPerCta + me, vec)
-                                    : make_uint4(0, 0, 0, 0);
+  for (int j = 0; j < kUnitsPerWarp; ++j) {
+    const uint64_t u = u_begin + warp * kUnitsPerWarp + j;
+    next[j] = u < u_end ? load8(w, n, u * kUnit + me, vec) : make_uint4(0, 0, 0, 0);
+  }
   __syncthreads();
-  uint32_t running = 0;  // thread 0: bits of the range so far
-  for (uint64_t pb = pb_begin; pb < pb_end; pb += kSumsBlocks) {
-    uint4 v[kSumsBlocks];
+  unsigned long long running = 0;  // warp 0: bits of the range so far (uniform)
+  for (uint64_t u0 = u_begin; u0 < u_end; u0 += kUnitsPerIter) {
+    uint4 v[kUnitsPerWarp];
 #pragma unroll
-    for (int j = 0; j < kSumsBlocks; ++j) {
+    for (int j = 0; j < kUnitsPerWarp; ++j) {
       v[j] = next[j];
-      const uint64_t q = pb + kSumsBlocks + j;
-      if (q < pb_end) next[j] = load8(w, n, q * kPerCta + me, vec);
+      const uint64_t u = u0 + kUnitsPerIter + warp * kUnitsPerWarp + j;
+      if (u < u_end) next[j] = load8(w, n, u * kUnit + me, vec);
     }
 #pragma unroll
-    for (int j = 0; j < kSumsBlocks; ++j) {
-      const uint32_t live = pb + j < pb_end ? live_of((pb + j) * kPerCta + me, n) : 0u;
+    for (int j = 0; j < kUnitsPerWarp; ++j) {
+      const uint64_t u = u0 + warp * kUnitsPerWarp + j;
+      const uint32_t live = u < u_end ? live_of(u * kUnit + me, n) : 0u;
       uint32_t s = 0;
 #pragma unroll
       for (int k = 0; k < kPerThread; ++k)
         if ((uint32_t)k < live) s += len[exponent_of(v[j], k)];
       s = __reduce_add_sync(0xFFFFFFFFu, s);
-      if ((threadIdx.x & 31) == 0) part[j][threadIdx.x >> 5] = s;
+      if (lane == 0) part[warp * kUnitsPerWarp + j] = s;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      for (int j = 0; j < kSumsBlocks && pb + j < pb_end; ++j) {
-        uint32_t t = 0;
-        for (int k = 0; k < kThreads / 32; ++k) t += part[j][k];
-        r.local[pb + j] = running;
-        running += t;
+    if (warp == 0) {  // the iteration's 32 units in order, one per lane
+      const uint32_t mine = part[lane];
+      uint32_t incl = mine;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += t;
       }
+      const uint64_t u = u0 + lane;
+      if (u < u_end) r.local[u] = (uint32_t)(running + incl - mine);
+      running += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
     __syncthreads();  // part is rewritten next iteration
   }
@@ -265,18 +277,18 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const unsigned long 
 }
 
 // Before packing: first elements preset to n, gaps cleared, the bitstream
-// words that two pack blocks share cleared (they are ORed into), maxima
-// cleared.
+// words that two units share cleared (they are ORed into), maxima cleared.
 __global__ void prepare_kernel(uint32_t *first_elem, uint8_t *gap, uint64_t chunks, uint32_t n,
                                const Ranges r, uint32_t *bs32, unsigned int *maxima) {
-  const uint64_t all = chunks + 1 > r.pack_ctas ? chunks + 1 : r.pack_ctas;
+  uint64_t all = chunks + 1 > r.units ? chunks + 1 : r.units;
+  all = all > 3 ? all : 3;  // the maxima
   for (uint64_t i = blockIdx.x * 256ull + threadIdx.x; i < all; i += (uint64_t)gridDim.x * 256) {
     if (i <= chunks) {
       first_elem[i] = n;
       gap[i] = 0;
     }
-    if (i >= 1 && i < r.pack_ctas) {
-      const unsigned long long s = pack_start(r, i);
+    if (i >= 1 && i < r.units) {
+      const unsigned long long s = unit_start(r, i);
       if (s & 31u) bs32[s >> 5] = 0;
     }
     if (i < 3) maxima[i] = 0;
@@ -297,162 +309,166 @@ struct PackArgs {
   uint32_t *bpos;
   uint64_t chunks;
   uint32_t num_blocks;
-  uint32_t chunk_bits, block_bits;    // 8 C and 8 C T
+  uint32_t chunk_bits, block_bits;  // 8 C and 8 C T
   uint32_t chunk_words, block_words;  // chunk_bits / 32, block_bits / 32
-  float inv_chunk, inv_block;         // 1 / chunk_bits, 1 / block_bits
+  uint64_t chunk_magic, block_magic;  // ceil(2^64 / words) (words >= 2)
+  uint32_t chunk_m32;                 // ceil(2^32 / chunk_bits): floor(x / chunk_bits)
+                                      // = umulhi(x, chunk_m32) for x < 2^16
 };
 
-// floor(x / d) for |x| < 2^20 from a float estimate, corrected to exact
-__device__ __forceinline__ int floor_div(int x, int d, float inv) {
-  int j = __float2int_rd((float)x * inv);
-  if (j * d > x) --j;
-  if ((j + 1) * d <= x) ++j;
-  return j;
+// floor(x / d) for x < 2^32 by a multiply-high with ceil(2^64 / d): the
+// error, below x / 2^64 < 2^-32, never crosses an integer (d < 2^32)
+__device__ __forceinline__ uint64_t div_words(uint32_t x, uint32_t d, uint64_t magic) {
+  return d == 1 ? x : __umul64hi((uint64_t)x, magic);
 }
 
 __global__ void __launch_bounds__(kThreads) pack_kernel(const PackArgs a) {
-  __shared__ uint32_t code[256];
-  __shared__ uint8_t len[256];
-  __shared__ uint32_t warp_sum[kThreads / 32];
-  __shared__ uint8_t last_len[kThreads];  // length of each thread's last codeword
-  __shared__ long long bound[4];          // first chunk and block at or before the origin
-  __shared__ uint32_t words[kCtaWords];
-  const uint2 t = a.tab[threadIdx.x];
-  code[threadIdx.x] = t.x;
-  len[threadIdx.x] = (uint8_t)t.y;
-  for (int j = threadIdx.x; j < kCtaWords; j += kThreads) words[j] = 0;
+  __shared__ uint2 tab_s[256];
+  __shared__ uint32_t words_s[kThreads / 32][kUnitWords];
+  tab_s[threadIdx.x] = a.tab[threadIdx.x];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint64_t me = (uint64_t)threadIdx.x * kPerThread;
-  const uint64_t pack_ctas = a.r.pack_ctas;
-  uint64_t pb = blockIdx.x;
-  // pack block pb's words, first bit and previous element (thread 0)
+  uint32_t *words = words_s[warp];
+  for (int j = lane; j < kUnitWords; j += 32) words[j] = 0;
+  const uint64_t me = (uint64_t)lane * kPerThread;
+  const uint64_t units = a.r.units;
+  const uint64_t stride = (uint64_t)gridDim.x * (kThreads / 32);
+  uint64_t u = (uint64_t)blockIdx.x * (kThreads / 32) + warp;
+  // unit u's words, first bit and previous element (lane 0)
   uint4 nx = make_uint4(0, 0, 0, 0);
   unsigned long long nstart = 0;
   uint32_t nprev = 0;
-  if (pb < pack_ctas) {
-    nx = load8(a.w, a.n, pb * kPerCta + me, a.vec);
-    nstart = pack_start(a.r, pb);
-    if (threadIdx.x == 0 && pb) nprev = a.w[pb * kPerCta - 1];
+  if (u < units) {
+    nx = load8(a.w, a.n, u * kUnit + me, a.vec);
+    nstart = unit_start(a.r, u);
+    if (lane == 0 && u) nprev = a.w[u * kUnit - 1];
   }
-  __syncthreads();
-  for (; pb < pack_ctas; pb += gridDim.x) {
+  __syncthreads();  // the table
+  for (; u < units; u += stride) {
     const uint4 v = nx;
-    const unsigned long long cta_start = nstart;
+    const unsigned long long start = nstart;
     const uint32_t prev_word = nprev;
-    const uint64_t pn = pb + gridDim.x;
-    if (pn < pack_ctas) {
-      nx = load8(a.w, a.n, pn * kPerCta + me, a.vec);
-      nstart = pack_start(a.r, pn);
-      if (threadIdx.x == 0) nprev = a.w[pn * kPerCta - 1];
+    const uint64_t un = u + stride;
+    if (un < units) {
+      nx = load8(a.w, a.n, un * kUnit + me, a.vec);
+      nstart = unit_start(a.r, un);
+      if (lane == 0) nprev = a.w[un * kUnit - 1];
     }
-    // bit positions below are relative to `origin`, the first bit of the
-    // word this pack block begins in
-    const unsigned long long origin = cta_start & ~31ull;
-    if (threadIdx.x == 0) {
-      const uint32_t ow = (uint32_t)(origin >> 5);  // < 2^32: bit offsets stay below 2^37
-      const uint64_t c0 = ow / a.chunk_words, q0 = ow / a.block_words;
-      bound[0] = (long long)c0;
-      bound[1] = (long long)(c0 * a.chunk_bits) - (long long)origin;
-      bound[2] = (long long)q0;
-      bound[3] = (long long)(q0 * a.block_bits) - (long long)origin;
-    }
-    const uint64_t i0 = pb * kPerCta + me;
+    const uint64_t i0 = u * kUnit + me;
     const uint32_t live = live_of(i0, a.n);
-    uint32_t e[kPerThread], l[kPerThread];
+    uint32_t e[kPerThread], l[kPerThread], cw[kPerThread];
     uint32_t mine = 0, last = 0;
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k) {
       e[k] = exponent_of(v, k);
-      l[k] = (uint32_t)k < live ? (uint32_t)len[e[k]] : 0u;
+      const uint2 t = tab_s[e[k]];
+      const bool in = (uint32_t)k < live;
+      l[k] = in ? t.y : 0u;
+      cw[k] = in ? t.x : 0u;
       mine += l[k];
-      last = (uint32_t)k < live ? l[k] : last;
+      last = in ? l[k] : last;
     }
     uint32_t incl = mine;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-      if (lane >= d) incl += u;
+      const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += t;
     }
-    if (lane == 31) warp_sum[warp] = incl;
-    last_len[threadIdx.x] = (uint8_t)last;
-    __syncthreads();
-    uint32_t before = 0, cta_total = 0;
-#pragma unroll
-    for (int j = 0; j < kThreads / 32; ++j) {
-      const uint32_t u = warp_sum[j];
-      before += j < warp ? u : 0u;
-      cta_total += u;
-    }
-    // length of element i0 - 1's codeword
-    const uint32_t prev_len = threadIdx.x ? last_len[threadIdx.x - 1]
-                                          : (pb ? len[exponent(prev_word)] : 0u);
-    const uint64_t c_org = (uint64_t)bound[0], q_org = (uint64_t)bound[2];
-    const int cr0 = (int)bound[1], qr0 = (int)bound[3];
-    const uint32_t lead = (uint32_t)(cta_start & 31u);  // bits of the first word before the block
-    const uint32_t rel = lead + before + incl - mine;   // this thread's first bit
+    const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    // length of element i0 - 1's codeword: the previous lane's last, or
+    // for lane 0 the previous unit's last element (0 for element 0)
+    const uint32_t up = __shfl_up_sync(0xFFFFFFFFu, last, 1);
+    const uint32_t prev_len = lane ? up : (u ? tab_s[exponent(prev_word)].y : 0u);
+    // positions below are relative to `origin`, the first bit of the word
+    // this unit begins in
+    const unsigned long long origin = start & ~31ull;
+    const uint32_t lead = (uint32_t)(start & 31u);
+    const uint32_t rel = lead + incl - mine;  // this lane's first bit
 
-    // codewords, MSB first, ORed into the shared image of the block's words.
-    // Up to 64 bits (the usual case) are gathered in one register first and
-    // placed with at most three ORs; longer runs go word by word.
-    if (mine <= 64) {
-      unsigned long long acc = 0;
+    // codewords, MSB first, ORed into the warp's image of the unit's words:
+    // up to 32 bits (the usual case) gathered in one register and placed
+    // with one or two ORs, up to 64 in two registers, longer runs word by word
+    __syncwarp();  // the previous unit's words are written out and cleared
+    if (mine && mine <= 32) {
+      uint32_t acc = 0;
 #pragma unroll
-      for (int k = 0; k < kPerThread; ++k)
-        acc = (acc << l[k]) | (l[k] ? code[e[k]] : 0u);
-      if (mine) {
+      for (int k = 0; k < kPerThread; ++k) acc = (acc << l[k]) | cw[k];
+      const uint32_t o = rel & 31u, wk = rel >> 5;
+      const uint32_t left = acc << (32 - mine);  // first bit at bit 31
+      atomicOr(&words[wk], left >> o);
+      if (o + mine > 32) atomicOr(&words[wk + 1], left << (32 - o));
+    } else if (mine) {
+      if (mine <= 64) {
+        unsigned long long acc = 0;
+#pragma unroll
+        for (int k = 0; k < kPerThread; ++k) acc = (acc << l[k]) | cw[k];
         const uint32_t o = rel & 31u, wk = rel >> 5;
-        const unsigned long long left = acc << (64 - mine);  // first bit at bit 63
+        const unsigned long long left = acc << (64 - mine);
         const uint32_t hi = (uint32_t)(left >> 32), lo = (uint32_t)left;
         atomicOr(&words[wk], hi >> o);
-        if (o + mine > 32) atomicOr(&words[wk + 1], __funnelshift_r(lo, hi, o));
+        atomicOr(&words[wk + 1], __funnelshift_r(lo, hi, o));
         if (o + mine > 64) atomicOr(&words[wk + 2], __funnelshift_lc(0u, lo, 32 - o));
-      }
-    } else {
-      // `cur` holds the pending bits left-aligned, `nb` of them
-      uint32_t wk = rel >> 5, nb = rel & 31u, cur = 0;
-      bool first = true;
+      } else {
+        // `cur` holds the pending bits left-aligned, `nb` of them
+        uint32_t wk = rel >> 5, nb = rel & 31u, cur = 0;
+        bool first = true;
 #pragma unroll
-      for (int k = 0; k < kPerThread; ++k) {
-        if (l[k]) {
-          const uint32_t cw = code[e[k]], tot = nb + l[k];
-          if (tot >= 32) {
-            const uint32_t u = cur | (cw >> (tot - 32));
-            if (first) atomicOr(&words[wk], u);  // the previous thread may own its first bits
-            else words[wk] = u;
-            first = false;
-            ++wk;
-            nb = tot - 32;
-            cur = __funnelshift_lc(0u, cw, 32 - nb);  // 0 when nb == 0
-          } else {
-            cur |= cw << (32 - tot);
-            nb = tot;
+        for (int k = 0; k < kPerThread; ++k) {
+          if (l[k]) {
+            const uint32_t tot = nb + l[k];
+            if (tot >= 32) {
+              const uint32_t t = cur | (cw[k] >> (tot - 32));
+              if (first) atomicOr(&words[wk], t);  // the previous lane may own its first bits
+              else words[wk] = t;
+              first = false;
+              ++wk;
+              nb = tot - 32;
+              cur = __funnelshift_lc(0u, cw[k], 32 - nb);  // 0 when nb == 0
+            } else {
+              cur |= cw[k] << (32 - tot);
+              nb = tot;
+            }
           }
         }
+        if (nb) atomicOr(&words[wk], cur);  // the last, partial word, which the next lane may share
       }
-      if (nb) atomicOr(&words[wk], cur);  // the last, partial word, which the next thread may share
     }
-    __syncthreads();
-    // words out, and cleared for the next pack block: ORed where a
-    // neighbouring pack block owns part of the word (cleared beforehand),
-    // stored otherwise
+    __syncwarp();
+    // words out, and cleared for the next unit: ORed where a neighbouring
+    // unit owns part of the word (cleared beforehand), stored otherwise
     const uint64_t base = origin >> 5;
-    const uint32_t end_bits = lead + cta_total;
+    const uint32_t end_bits = lead + total;
     const uint32_t nwords = (end_bits + 31) >> 5;
-    const bool shared_last = (end_bits & 31u) && pb + 1 < pack_ctas;
-    for (uint32_t j = threadIdx.x; j < nwords; j += kThreads) {
-      const uint32_t u = bswap32(words[j]);
+    const bool shared_last = (end_bits & 31u) && u + 1 < units;
+    for (uint32_t j = lane; j < nwords; j += 32) {
+      const uint32_t t = bswap32(words[j]);
       words[j] = 0;
-      if ((j == 0 && lead) || (j == nwords - 1 && shared_last)) atomicOr(&a.bs32[base + j], u);
-      else a.bs32[base + j] = u;
+      if ((j == 0 && lead) || (j == nwords - 1 && shared_last)) atomicOr(&a.bs32[base + j], t);
+      else a.bs32[base + j] = t;
     }
+    // chunks and blocks whose first codeword start is one of these
+    // elements: those that begin after element i0 - 1's codeword start and
+    // at or before element i0 + live - 1's.  The first chunk (block) after
+    // that start is floor(start / chunk bits) + 1; bit offsets stay below
+    // 2^37, so offset / 32 fits 32 bits and floor(p / (32 m)) =
+    // floor(floor(p / 32) / m).  Blocks are skipped unless one begins
+    // inside this unit (warp-wide test, before any lane leaves).
+    const int p_last = (int)(rel + mine - last);
+    const uint32_t pw = (uint32_t)((origin + rel - prev_len) >> 5);  // element i0 - 1's start / 32
+    // chunk c_base begins o_c bits before `origin` (0 <= o_c < chunk bits)
+    const uint64_t c_base = div_words((uint32_t)(origin >> 5), a.chunk_words, a.chunk_magic);
+    const int o_c = (int)(origin - c_base * a.chunk_bits);
+    const uint32_t pw0 = __shfl_sync(0xFFFFFFFFu, pw, 0);
+    const int p_end = __shfl_sync(0xFFFFFFFFu, p_last, 31);
+    const uint64_t q0 = u ? div_words(pw0, a.block_words, a.block_magic) + 1 : 0;
+    const bool blocks_here = (long long)(q0 * a.block_bits) - (long long)origin <= p_end;
     if (!live) continue;
 
     // sign/mantissa bytes: bit 15 -> bit 7, bits 0-6 kept; two per word
     uint32_t sm2[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const uint32_t u = r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
-      sm2[r] = (u & 0x007F007Fu) | ((u >> 8) & 0x00800080u);  // bytes 0 and 2
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t t = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+      sm2[q] = (t & 0x007F007Fu) | ((t >> 8) & 0x00800080u);  // bytes 0 and 2
     }
     const uint2 smv = make_uint2(__byte_perm(sm2[0], sm2[1], 0x6420),
                                  __byte_perm(sm2[2], sm2[3], 0x6420));
@@ -463,28 +479,39 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const PackArgs a) {
         a.sm[i0 + k] = (uint8_t)((k < 4 ? smv.x : smv.y) >> (8 * (k & 3)));
     }
 
-    // chunks and blocks whose first codeword start is one of these
-    // elements: those that begin after element i0 - 1's codeword start and
-    // at or before element i0 + live - 1's.  cb and qb run over their
-    // positions in order.
-    const int p0 = (int)rel;
-    const int prev = i0 == 0 ? -1 : p0 - (int)prev_len;
-    const int p_last = p0 + (int)(mine - last);
-    const int jc = floor_div(prev - cr0, (int)a.chunk_bits, a.inv_chunk) + 1;
-    const int jq = floor_div(prev - qr0, (int)a.block_bits, a.inv_block) + 1;
-    int cb = cr0 + jc * (int)a.chunk_bits, qb = qr0 + jq * (int)a.block_bits;
-    if (cb <= p_last || qb <= p_last) {
-      uint64_t c = c_org + jc, q = q_org + jq;
-      int pk = p0;
+    // the first chunk boundary after element i0 - 1's start; then, while
+    // it lies at or before this lane's last start, the first element
+    // starting at or after it (counted without branches) takes it
+    const uint32_t x = (uint32_t)((int)rel - (int)prev_len + o_c + (int)a.chunk_bits);
+    const uint32_t jc = i0 ? __umulhi(x, a.chunk_m32) : 0u;  // floor(x / chunk_bits)
+    int cb = (int)(jc * a.chunk_bits) - o_c;
+    if (cb <= p_last) {
+      uint64_t c = c_base + jc;
+      do {
+        uint32_t k = 0, bits = 0;
+        int pj = (int)rel;
+#pragma unroll
+        for (int j = 0; j < kPerThread; ++j) {
+          const bool before = l[j] && pj < cb;
+          k += before ? 1u : 0u;
+          bits += before ? l[j] : 0u;
+          pj += (int)l[j];
+        }
+        if (c < a.chunks) {
+          a.gap[c] = (uint8_t)((int)(rel + bits) - cb);
+          a.first_elem[c] = (uint32_t)(i0 + k);
+        }
+        ++c;
+        cb += (int)a.chunk_bits;
+      } while (cb <= p_last);
+    }
+    if (blocks_here) {  // the same for block boundaries (about one unit in 25)
+      uint64_t q = i0 ? div_words(pw, a.block_words, a.block_magic) + 1 : 0;
+      int qb = (int)((long long)(q * a.block_bits) - (long long)origin);
+      int pk = (int)rel;
 #pragma unroll
       for (int k = 0; k < kPerThread; ++k) {
         if (l[k]) {
-          for (; cb <= pk; cb += (int)a.chunk_bits, ++c) {
-            if (c < a.chunks) {
-              a.gap[c] = (uint8_t)(pk - cb);
-              a.first_elem[c] = (uint32_t)(i0 + k);
-            }
-          }
           for (; qb <= pk; qb += (int)a.block_bits, ++q)
             if (q < a.num_blocks) a.bpos[q] = (uint32_t)(i0 + k);
           pk += (int)l[k];
@@ -657,6 +684,48 @@ void fill_params(const df11_gpu_build *h, df11_params *p) {
   p->max_len = (uint32_t)h->longest;
 }
 
+// Small host<->device transfers go through one pinned buffer of the
+// library's (grown on demand, kept for the process), so that they queue
+// without synchronising the stream the way pageable copies do.  A build call
+// holds it from its first copy to its last synchronisation.
+struct Staging {
+  std::mutex mu;
+  void *p = nullptr;
+  size_t bytes = 0;
+  // caller holds mu
+  void *get(size_t want) {
+    if (want <= bytes) return p;
+    if (p) cudaFreeHost(p);
+    p = nullptr;
+    bytes = 0;
+    if (cudaHostAlloc(&p, want, cudaHostAllocDefault) != cudaSuccess) {
+      p = nullptr;
+      return nullptr;
+    }
+    bytes = want;
+    return p;
+  }
+};
+Staging g_staging;
+
+// what one tensor's phase 1 reads back and sends
+struct BeginSlot {
+  unsigned long long hist[256];
+  uint2 tab[256];
+  unsigned long long total;
+  uint16_t last;
+  uint16_t pad[3];
+};
+
+df11_status check_begin_args(const uint16_t *d_bf16, uint64_t n, uint32_t C, uint32_t T) {
+  if (n && !d_bf16) return DF11_ERR_NULL;
+  if (C < 4 || C > 28 || C % 4) return DF11_ERR_INVALID;
+  if (T < 128 || T > 1024 || T % 128) return DF11_ERR_INVALID;
+  if (n >= (1ull << 32)) return DF11_ERR_TOO_LARGE;
+  if ((uintptr_t)d_bf16 & 1) return DF11_ERR_ALIGN;
+  return DF11_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -669,157 +738,213 @@ void df11_gpu_build_free(df11_gpu_build *h) {
   delete h;
 }
 
+df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const uint64_t *n,
+                                         int count, uint32_t C, uint32_t T,
+                                         df11_stream_t stream, df11_params *params,
+                                         uint8_t *code_lengths, df11_gpu_build **handles) {
+  if (count < 0) return DF11_ERR_INVALID;
+  if (count == 0) return DF11_OK;
+  if (!handles) return DF11_ERR_NULL;
+  for (int i = 0; i < count; ++i) handles[i] = nullptr;
+  if (!d_bf16 || !n || !params || !code_lengths) return DF11_ERR_NULL;
+  for (int i = 0; i < count; ++i) {
+    const df11_status st = check_begin_args(d_bf16[i], n[i], C, T);
+    if (st != DF11_OK) return st;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  std::vector<df11_gpu_build *> hs(count, nullptr);
+  auto fail = [&](df11_status st) {
+    for (auto *h : hs) df11_gpu_build_free(h);
+    return st;
+  };
+  const uint64_t slots = resident(sums_kernel), hist_slots = resident(hist_kernel);
+  std::lock_guard<std::mutex> lock(g_staging.mu);
+  BeginSlot *stage = static_cast<BeginSlot *>(g_staging.get(sizeof(BeginSlot) * count));
+  if (!stage) return DF11_ERR_NOMEM;
+
+  // histograms, and each tensor's last element (its codeword ends the stream)
+  for (int i = 0; i < count; ++i) {
+    df11_gpu_build *h = hs[i] = new (std::nothrow) df11_gpu_build();
+    if (!h) return fail(DF11_ERR_NOMEM);
+    h->n = n[i];
+    h->C = C;
+    h->T = T;
+    h->vec = ((uintptr_t)d_bf16[i] & 15) == 0;
+    h->stream = s;
+    // contiguous ranges of units, one per resident sums thread block.  A
+    // range's bits fit 32 bits: at most 2^24 units over at least
+    // min(units, SMs) ranges, at most 8192 bits per unit.
+    h->r.units = (h->n + kUnit - 1) / kUnit;
+    h->ranges = h->r.units < slots ? h->r.units : slots;
+    h->r.per = h->ranges ? (h->r.units + h->ranges - 1) / h->ranges : 1;
+    if (h->ranges) h->ranges = (h->r.units + h->r.per - 1) / h->r.per;
+    const uint64_t o_tab = round256(256 * sizeof(unsigned long long));
+    const uint64_t o_tot = o_tab + round256(256 * sizeof(uint2));
+    const uint64_t o_rs = o_tot + round256(h->ranges * sizeof(unsigned long long) + 8);
+    const uint64_t o_loc = o_rs + round256((h->ranges + 1) * sizeof(unsigned long long));
+    const uint64_t bytes1 = o_loc + round256(h->r.units * sizeof(uint32_t) + 4);
+    if (scratch_alloc(&h->scratch1, bytes1, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
+    char *base1 = static_cast<char *>(h->scratch1);
+    h->d_hist = reinterpret_cast<unsigned long long *>(base1);
+    h->d_tab = reinterpret_cast<uint2 *>(base1 + o_tab);
+    h->d_range_total = reinterpret_cast<unsigned long long *>(base1 + o_tot);
+    h->r.range_start = reinterpret_cast<unsigned long long *>(base1 + o_rs);
+    h->r.local = reinterpret_cast<uint32_t *>(base1 + o_loc);
+    stage[i].last = 0;
+    if (cudaMemsetAsync(h->d_hist, 0, 256 * sizeof(unsigned long long), s) != cudaSuccess)
+      return fail(DF11_ERR_CUDA);
+    if (h->n) {
+      const uint64_t tiles = (h->n + kPerCta - 1) / kPerCta;
+      const unsigned grid = (unsigned)(tiles < hist_slots ? tiles : hist_slots);
+      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_hist);
+      if (cudaGetLastError() != cudaSuccess ||
+          cudaMemcpyAsync(&stage[i].last, d_bf16[i] + (h->n - 1), 2, cudaMemcpyDeviceToHost,
+                          s) != cudaSuccess)
+        return fail(DF11_ERR_CUDA);
+    }
+    if (cudaMemcpyAsync(stage[i].hist, h->d_hist, sizeof(stage[i].hist), cudaMemcpyDeviceToHost,
+                        s) != cudaSuccess)
+      return fail(DF11_ERR_CUDA);
+  }
+  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(DF11_ERR_CUDA);
+
+  // codebooks (host: 256 symbols each), then every unit's first bit and the
+  // totals
+  for (int i = 0; i < count; ++i) {
+    df11_gpu_build *h = hs[i];
+    uint64_t hist64[256];
+    for (int k = 0; k < 256; ++k) hist64[k] = stage[i].hist[k];
+    h->longest = df11_internal::codebook(hist64, h->len, h->code, h->luts);
+    for (int k = 0; k < 256; ++k) stage[i].tab[k] = make_uint2(h->code[k], h->len[k]);
+    stage[i].total = 0;
+    if (cudaMemcpyAsync(h->d_tab, stage[i].tab, sizeof(stage[i].tab), cudaMemcpyHostToDevice,
+                        s) != cudaSuccess)
+      return fail(DF11_ERR_CUDA);
+    if (h->ranges) {
+      sums_kernel<<<(unsigned)h->ranges, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_tab,
+                                                           h->r, h->d_range_total);
+      scan_kernel<<<1, kScanThreads, 0, s>>>(h->d_range_total, h->ranges, h->r.range_start);
+      if (cudaGetLastError() != cudaSuccess ||
+          cudaMemcpyAsync(&stage[i].total, h->r.range_start + h->ranges,
+                          sizeof(stage[i].total), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return fail(DF11_ERR_CUDA);
+    }
+  }
+  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(DF11_ERR_CUDA);
+
+  for (int i = 0; i < count; ++i) {
+    df11_gpu_build *h = hs[i];
+    h->total = stage[i].total;
+    if (h->n) h->last_start = h->total - h->len[(stage[i].last >> 7) & 0xFF];
+    const uint64_t block_bits = 8ull * C * T;
+    h->num_blocks = (h->total + block_bits - 1) / block_bits;
+    h->chunks = h->num_blocks * T;
+    const uint64_t o_max = round256((h->chunks + 1) * sizeof(uint32_t));
+    const uint64_t o_gap = o_max + 256;
+    if (scratch_alloc(&h->scratch2, o_gap + round256(h->chunks + 1), s) != cudaSuccess)
+      return fail(DF11_ERR_CUDA);
+    char *base2 = static_cast<char *>(h->scratch2);
+    h->d_first = reinterpret_cast<uint32_t *>(base2);
+    h->d_max = reinterpret_cast<unsigned int *>(base2 + o_max);
+    h->d_gap = reinterpret_cast<uint8_t *>(base2 + o_gap);
+    fill_params(h, &params[i]);
+    std::memcpy(code_lengths + 256 * (size_t)i, h->len, 256);
+  }
+  for (int i = 0; i < count; ++i) handles[i] = hs[i];
+  return DF11_OK;
+}
+
 df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t C, uint32_t T,
                                  df11_stream_t stream, df11_params *params,
                                  uint8_t code_lengths[256], df11_gpu_build **handle) {
   if (handle) *handle = nullptr;
   if (!params || !code_lengths || !handle || (n && !d_bf16)) return DF11_ERR_NULL;
-  if (C < 4 || C > 28 || C % 4) return DF11_ERR_INVALID;
-  if (T < 128 || T > 1024 || T % 128) return DF11_ERR_INVALID;
-  if (n >= (1ull << 32)) return DF11_ERR_TOO_LARGE;
-  if ((uintptr_t)d_bf16 & 1) return DF11_ERR_ALIGN;
-  cudaStream_t s = (cudaStream_t)stream;
-  df11_gpu_build *h = new (std::nothrow) df11_gpu_build();
-  if (!h) return DF11_ERR_NOMEM;
-  h->n = n;
-  h->C = C;
-  h->T = T;
-  h->vec = ((uintptr_t)d_bf16 & 15) == 0;
-  // contiguous ranges of pack blocks, one per resident sums thread block.
-  // A range's bits fit 32 bits: at most 2^21 pack blocks over at least
-  // min(pack blocks, SMs) ranges, at most 65536 bits per pack block.
-  h->r.pack_ctas = (n + kPerCta - 1) / kPerCta;
-  const uint64_t slots = resident(sums_kernel);
-  h->ranges = h->r.pack_ctas < slots ? h->r.pack_ctas : slots;
-  h->r.per = h->ranges ? (h->r.pack_ctas + h->ranges - 1) / h->ranges : 1;
-  if (h->ranges) h->ranges = (h->r.pack_ctas + h->r.per - 1) / h->r.per;
-  h->stream = s;
-  auto fail = [&](df11_status st) {
-    df11_gpu_build_free(h);
-    return st;
-  };
-  const uint64_t o_tab = round256(256 * sizeof(unsigned long long));
-  const uint64_t o_tot = o_tab + round256(256 * sizeof(uint2));
-  const uint64_t o_rs = o_tot + round256(h->ranges * sizeof(unsigned long long) + 8);
-  const uint64_t o_loc = o_rs + round256((h->ranges + 1) * sizeof(unsigned long long));
-  const uint64_t bytes1 = o_loc + round256(h->r.pack_ctas * sizeof(uint32_t) + 4);
-  if (scratch_alloc(&h->scratch1, bytes1, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
-  char *base1 = static_cast<char *>(h->scratch1);
-  h->d_hist = reinterpret_cast<unsigned long long *>(base1);
-  h->d_tab = reinterpret_cast<uint2 *>(base1 + o_tab);
-  h->d_range_total = reinterpret_cast<unsigned long long *>(base1 + o_tot);
-  h->r.range_start = reinterpret_cast<unsigned long long *>(base1 + o_rs);
-  h->r.local = reinterpret_cast<uint32_t *>(base1 + o_loc);
-
-  // histogram, and the last element (its codeword ends the stream)
-  unsigned long long hist[256];
-  uint16_t last = 0;
-  bool ok = cudaMemsetAsync(h->d_hist, 0, 256 * sizeof(unsigned long long), s) == cudaSuccess;
-  if (ok && n) {
-    const uint64_t want = resident(hist_kernel);
-    const unsigned grid = (unsigned)(h->r.pack_ctas < want ? h->r.pack_ctas : want);
-    hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16, n, h->vec, h->d_hist);
-    ok = cudaGetLastError() == cudaSuccess &&
-         cudaMemcpyAsync(&last, d_bf16 + (n - 1), 2, cudaMemcpyDeviceToHost, s) == cudaSuccess;
-  }
-  ok = ok &&
-       cudaMemcpyAsync(hist, h->d_hist, sizeof(hist), cudaMemcpyDeviceToHost, s) == cudaSuccess &&
-       cudaStreamSynchronize(s) == cudaSuccess;
-  if (!ok) return fail(DF11_ERR_CUDA);
-
-  // codebook (host: 256 symbols)
-  uint64_t hist64[256];
-  for (int i = 0; i < 256; ++i) hist64[i] = hist[i];
-  h->longest = df11_internal::codebook(hist64, h->len, h->code, h->luts);
-  uint2 tab[256];
-  for (int i = 0; i < 256; ++i) tab[i] = make_uint2(h->code[i], h->len[i]);
-
-  // first bit of every range and pack block, and the total
-  unsigned long long total = 0;
-  if (cudaMemcpyAsync(h->d_tab, tab, sizeof(tab), cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return fail(DF11_ERR_CUDA);
-  if (h->ranges) {
-    sums_kernel<<<(unsigned)h->ranges, kThreads, 0, s>>>(d_bf16, n, h->vec, h->d_tab, h->r,
-                                                         h->d_range_total);
-    scan_kernel<<<1, kScanThreads, 0, s>>>(h->d_range_total, h->ranges, h->r.range_start);
-    if (cudaGetLastError() != cudaSuccess ||
-        cudaMemcpyAsync(&total, h->r.range_start + h->ranges, sizeof(total),
-                        cudaMemcpyDeviceToHost, s) != cudaSuccess)
-      return fail(DF11_ERR_CUDA);
-  }
-  // the table copy reads `tab` until it is done
-  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(DF11_ERR_CUDA);
-  h->total = total;
-  if (n) h->last_start = h->total - h->len[(last >> 7) & 0xFF];
-  const uint64_t block_bits = 8ull * C * T;
-  h->num_blocks = (h->total + block_bits - 1) / block_bits;
-  h->chunks = h->num_blocks * T;
-  const uint64_t o_max = round256((h->chunks + 1) * sizeof(uint32_t));
-  const uint64_t o_gap = o_max + 256;
-  if (scratch_alloc(&h->scratch2, o_gap + round256(h->chunks + 1), s) != cudaSuccess)
-    return fail(DF11_ERR_CUDA);
-  char *base2 = static_cast<char *>(h->scratch2);
-  h->d_first = reinterpret_cast<uint32_t *>(base2);
-  h->d_max = reinterpret_cast<unsigned int *>(base2 + o_max);
-  h->d_gap = reinterpret_cast<uint8_t *>(base2 + o_gap);
-  fill_params(h, params);
-  std::memcpy(code_lengths, h->len, 256);
-  *handle = h;
-  return DF11_OK;
+  return df11_gpu_build_begin_batched(&d_bf16, &n, 1, C, T, stream, params, code_lengths,
+                                      handle);
 }
 
-df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uint8_t *bitstream,
-                                  uint8_t *gaps, uint8_t *chunk_counts, uint32_t *block_out_pos,
-                                  uint32_t *luts, uint8_t *code_lengths, uint8_t *sign_mantissa,
-                                  df11_params *params, df11_stream_t stream) {
-  if (!h) return DF11_ERR_NULL;
+df11_status df11_gpu_build_finish_batched(df11_gpu_build *const *handles, int count,
+                                          const uint16_t *const *d_bf16,
+                                          const df11_gpu_build_out *outs, df11_params *params,
+                                          df11_stream_t stream) {
+  if (count < 0) return DF11_ERR_INVALID;
+  if (count == 0) return DF11_OK;
+  if (!handles) return DF11_ERR_NULL;
   df11_status st = DF11_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  const uint64_t chunks = h->chunks, n = h->n;
-  const uint64_t bs_bytes = chunks * h->C + 16, gaps_bytes = chunks * 5 / 8 + 16;
-  const uint64_t sm_bytes = (n + 15) / 16 * 16;
-  const uint64_t bs_written = (h->total + 31) / 32 * 4;  // the pack blocks' words
-  do {
-    if (!params || !bitstream || !gaps || !chunk_counts || !block_out_pos || !luts ||
-        !code_lengths || !sign_mantissa || (n && !d_bf16)) {
+  for (int i = 0; i < count && st == DF11_OK; ++i) {
+    const df11_gpu_build *h = handles[i];
+    if (!h || !d_bf16 || !outs || !params) {
       st = DF11_ERR_NULL;
       break;
     }
-    if (((uintptr_t)bitstream & 15) || ((uintptr_t)gaps & 15) || ((uintptr_t)luts & 15) ||
-        ((uintptr_t)chunk_counts & 15) || ((uintptr_t)sign_mantissa & 15) ||
-        ((uintptr_t)block_out_pos & 3) || (n && h->vec != (((uintptr_t)d_bf16 & 15) == 0))) {
+    const df11_gpu_build_out &o = outs[i];
+    if (!o.bitstream || !o.gaps || !o.chunk_counts || !o.block_out_pos || !o.luts ||
+        !o.code_lengths || !o.sign_mantissa || (h->n && !d_bf16[i])) {
+      st = DF11_ERR_NULL;
+    } else if (((uintptr_t)o.bitstream & 15) || ((uintptr_t)o.gaps & 15) ||
+               ((uintptr_t)o.luts & 15) || ((uintptr_t)o.chunk_counts & 15) ||
+               ((uintptr_t)o.sign_mantissa & 15) || ((uintptr_t)o.block_out_pos & 3) ||
+               (h->n && h->vec != (((uintptr_t)d_bf16[i] & 15) == 0))) {
       st = DF11_ERR_ALIGN;
-      break;
     }
+  }
+  std::unique_lock<std::mutex> lock(g_staging.mu, std::defer_lock);
+  size_t stage_bytes = 0;
+  std::vector<size_t> off(count > 0 ? count : 0);
+  if (st == DF11_OK) {
+    for (int i = 0; i < count; ++i) {
+      off[i] = stage_bytes;  // luts, code lengths, then the maxima read back
+      stage_bytes += (handles[i]->luts.size() * 4 + 256 + 16 + 15) & ~(size_t)15;
+    }
+    lock.lock();
+  }
+  uint8_t *stage = st == DF11_OK ? static_cast<uint8_t *>(g_staging.get(stage_bytes)) : nullptr;
+  if (st == DF11_OK && !stage) st = DF11_ERR_NOMEM;
+  for (int i = 0; i < count && st == DF11_OK; ++i) {
+    df11_gpu_build *h = handles[i];
+    const df11_gpu_build_out &o = outs[i];
+    const uint64_t chunks = h->chunks, n = h->n;
+    const uint64_t bs_bytes = chunks * h->C + 16, gaps_bytes = chunks * 5 / 8 + 16;
+    const uint64_t sm_bytes = (n + 15) / 16 * 16;
+    const uint64_t bs_written = (h->total + 31) / 32 * 4;  // the units' words
+    const size_t lut_bytes = h->luts.size() * 4;
+    uint8_t *st_luts = stage + off[i], *st_lens = st_luts + lut_bytes;
+    std::memcpy(st_luts, h->luts.data(), lut_bytes);
+    std::memcpy(st_lens, h->len, 256);
     // every byte the kernels do not write: the padding after each buffer
     const bool ok =
-        cudaMemsetAsync(bitstream + bs_written, 0, bs_bytes - bs_written, s) == cudaSuccess &&
-        cudaMemsetAsync(gaps + chunks * 5 / 8, 0, gaps_bytes - chunks * 5 / 8, s) == cudaSuccess &&
-        cudaMemsetAsync(chunk_counts + chunks, 0, 16, s) == cudaSuccess &&
-        (sm_bytes == n || cudaMemsetAsync(sign_mantissa + n, 0, sm_bytes - n, s) == cudaSuccess) &&
-        cudaMemcpyAsync(luts, h->luts.data(), h->luts.size() * 4, cudaMemcpyHostToDevice, s) ==
+        cudaMemsetAsync(o.bitstream + bs_written, 0, bs_bytes - bs_written, s) == cudaSuccess &&
+        cudaMemsetAsync(o.gaps + chunks * 5 / 8, 0, gaps_bytes - chunks * 5 / 8, s) ==
             cudaSuccess &&
-        cudaMemcpyAsync(code_lengths, h->len, 256, cudaMemcpyHostToDevice, s) == cudaSuccess;
+        cudaMemsetAsync(o.chunk_counts + chunks, 0, 16, s) == cudaSuccess &&
+        (sm_bytes == n ||
+         cudaMemsetAsync(o.sign_mantissa + n, 0, sm_bytes - n, s) == cudaSuccess) &&
+        cudaMemcpyAsync(o.luts, st_luts, lut_bytes, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+        cudaMemcpyAsync(o.code_lengths, st_lens, 256, cudaMemcpyHostToDevice, s) == cudaSuccess;
     if (!ok) {
       st = DF11_ERR_CUDA;
       break;
     }
-    uint32_t *bs32 = reinterpret_cast<uint32_t *>(bitstream);
+    uint32_t *bs32 = reinterpret_cast<uint32_t *>(o.bitstream);
     prepare_kernel<<<148 * 4, 256, 0, s>>>(h->d_first, h->d_gap, chunks, (uint32_t)n, h->r, bs32,
                                            h->d_max);
     const uint32_t chunk_bits = 8 * h->C, block_bits = 8 * h->C * h->T;
-    const PackArgs pa{d_bf16, n, h->vec, h->d_tab, h->r, bs32, sign_mantissa, h->d_gap,
-                      h->d_first, block_out_pos, chunks, (uint32_t)h->num_blocks,
-                      chunk_bits, block_bits, h->C / 4, h->C / 4 * h->T,
-                      1.0f / (float)chunk_bits, 1.0f / (float)block_bits};
-    if (h->r.pack_ctas) {
-      const uint64_t want = resident(pack_kernel);
-      const unsigned grid = (unsigned)(h->r.pack_ctas < want ? h->r.pack_ctas : want);
+    const uint32_t chunk_words = h->C / 4, block_words = h->C / 4 * h->T;
+    const PackArgs pa{d_bf16[i], n, h->vec, h->d_tab, h->r, bs32, o.sign_mantissa, h->d_gap,
+                      h->d_first, o.block_out_pos, chunks, (uint32_t)h->num_blocks,
+                      chunk_bits, block_bits, chunk_words, block_words,
+                      chunk_words > 1 ? UINT64_MAX / chunk_words + 1 : 0,
+                      block_words > 1 ? UINT64_MAX / block_words + 1 : 0,
+                      (uint32_t)(((1ull << 32) + chunk_bits - 1) / chunk_bits)};
+    if (h->r.units) {
+      const uint64_t want = resident(pack_kernel), ctas = (h->r.units + 7) / 8;
+      const unsigned grid = (unsigned)(ctas < want ? ctas : want);
       pack_kernel<<<grid, kThreads, 0, s>>>(pa);
     }
-    const FinishArgs fa{h->d_gap, h->d_first, gaps, chunk_counts, block_out_pos, h->d_max,
-                        8ull * h->C, chunks, 8ull * h->C * h->T, h->total, h->last_start,
-                        (uint32_t)h->num_blocks, (uint32_t)n};
+    const FinishArgs fa{h->d_gap, h->d_first, o.gaps, o.chunk_counts, o.block_out_pos,
+                        h->d_max, 8ull * h->C, chunks, 8ull * h->C * h->T, h->total,
+                        h->last_start, (uint32_t)h->num_blocks, (uint32_t)n};
     unsigned grid;
     if (chunks) {
       if (!grid_for(chunks / 8, 256, &grid)) {
@@ -830,21 +955,41 @@ df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uin
     }
     grid_for(h->num_blocks + 1, 256, &grid);
     finish_blocks<<<grid, 256, 0, s>>>(fa);
-    unsigned int mx[3];
     if (cudaGetLastError() != cudaSuccess ||
-        cudaMemcpyAsync(mx, h->d_max, sizeof(mx), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaMemcpyAsync(st_lens + 256, h->d_max, 3 * sizeof(unsigned int), cudaMemcpyDeviceToHost,
+                        s) != cudaSuccess) {
       st = DF11_ERR_CUDA;
       break;
     }
-    fill_params(h, params);
-    params->max_block_elems = mx[0];
-    params->max_chunk_elems = mx[1];
-    params->max_warp_elems = mx[2];
-  } while (false);
-  h->stream = s;  // frees follow this call's work
-  df11_gpu_build_free(h);
+  }
+  if (st == DF11_OK && cudaStreamSynchronize(s) != cudaSuccess) st = DF11_ERR_CUDA;
+  for (int i = 0; i < count && st == DF11_OK; ++i) {
+    const df11_gpu_build *h = handles[i];
+    unsigned int mx[3];
+    std::memcpy(mx, stage + off[i] + h->luts.size() * 4 + 256, sizeof(mx));
+    fill_params(h, &params[i]);
+    params[i].max_block_elems = mx[0];
+    params[i].max_chunk_elems = mx[1];
+    params[i].max_warp_elems = mx[2];
+  }
+  if (st != DF11_OK) cudaStreamSynchronize(s);  // the staging buffer is read until then
+  if (lock.owns_lock()) lock.unlock();
+  for (int i = 0; i < count; ++i) {
+    if (!handles[i]) continue;
+    handles[i]->stream = s;  // frees follow this call's work
+    df11_gpu_build_free(handles[i]);
+  }
   return st;
+}
+
+df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uint8_t *bitstream,
+                                  uint8_t *gaps, uint8_t *chunk_counts, uint32_t *block_out_pos,
+                                  uint32_t *luts, uint8_t *code_lengths, uint8_t *sign_mantissa,
+                                  df11_params *params, df11_stream_t stream) {
+  if (!h) return DF11_ERR_NULL;
+  const df11_gpu_build_out o{bitstream, gaps, chunk_counts, block_out_pos, luts, code_lengths,
+                             sign_mantissa};
+  return df11_gpu_build_finish_batched(&h, 1, &d_bf16, &o, params, stream);
 }
 
 }  // extern "C"

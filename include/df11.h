@@ -298,7 +298,8 @@ typedef struct df11_gpu_build df11_gpu_build;
  *   sign_mantissa  n rounded up to 16 bytes
  * Errors: DF11_ERR_NULL, _INVALID, _TOO_LARGE, _ALIGN, _NOMEM before any
  * device work; DF11_ERR_CUDA if a CUDA call fails.  *handle is NULL on
- * every error.
+ * every error.  Small transfers between host and device go through a pinned
+ * buffer the library keeps; concurrent build calls take turns on it.
  */
 df11_status df11_gpu_build_begin(const uint16_t *d_bf16, uint64_t n, uint32_t chunk_bytes,
                                  uint32_t threads_per_block, df11_stream_t stream,
@@ -334,6 +335,36 @@ df11_status df11_gpu_build_finish(df11_gpu_build *handle, const uint16_t *d_bf16
  */
 df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t n, uint64_t hist[256],
                                     df11_stream_t stream);
+
+/* The output buffers of one tensor's phase 2 (sizes and alignment as for
+ * df11_gpu_build_finish). */
+typedef struct df11_gpu_build_out {
+  uint8_t *bitstream;
+  uint8_t *gaps;
+  uint8_t *chunk_counts;
+  uint32_t *block_out_pos;
+  uint32_t *luts;
+  uint8_t *code_lengths;
+  uint8_t *sign_mantissa;
+} df11_gpu_build_out;
+
+/*
+ * Both phases for `count` tensors at once (d_bf16[i], n[i]; params and
+ * handles arrays of count, code_lengths count*256 bytes, all host arrays):
+ * each phase synchronises the stream once for all of them instead of once
+ * per tensor.  Same conventions as the single-tensor calls; on an error in
+ * phase 1 no handle is returned (all NULL), and phase 2 releases every
+ * handle in all cases.  The single-tensor calls are these with count 1.
+ */
+df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const uint64_t *n,
+                                         int count, uint32_t chunk_bytes,
+                                         uint32_t threads_per_block, df11_stream_t stream,
+                                         df11_params *params, uint8_t *code_lengths,
+                                         df11_gpu_build **handles);
+df11_status df11_gpu_build_finish_batched(df11_gpu_build *const *handles, int count,
+                                          const uint16_t *const *d_bf16,
+                                          const df11_gpu_build_out *outs, df11_params *params,
+                                          df11_stream_t stream);
 
 /* Release a phase-1 handle without running phase 2 (NULL is a no-op); its
  * scratch is freed in order on the stream phase 1 ran on, which must still

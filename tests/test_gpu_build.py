@@ -151,3 +151,27 @@ def test_runs_of_long_codewords():
     per_thread = np.add.reduceat(lens, np.arange(0, len(lens), 8))
     assert per_thread.max() > 64  # the case this test is for
     _decodes_to(d, w)
+
+
+def test_batched_builds_equal_single_builds():
+    """Several tensors in one begin/finish pair (one synchronisation per
+    phase): each byte-identical to the host builder, empty and unaligned
+    ones included."""
+    base = workloads.gaussian_bf16(300_001, 0.02, 31, device="cuda")
+    bits = [workloads.gaussian_bf16(1_000_003, 0.02, 30, device="cuda"),
+            torch.zeros(0, dtype=torch.int16, device="cuda"),
+            base[3:],
+            workloads.adversarial_mix(1 << 20, 32, device="cuda"),
+            workloads.gaussian_bf16(2049, 0.5, 33, device="cuda")]
+    ds = df11.compress_on_device_batched(bits, 24, 256)
+    torch.cuda.synchronize()
+    assert len(ds) == len(bits)
+    for b, d in zip(bits, ds):
+        w_np = workloads.as_numpy_u16(b.cpu())
+        h = df11.compress(w_np, 24, 256)
+        for f, _ in df11.Params._fields_:
+            assert getattr(d.params, f) == getattr(h.params, f), f
+        for f in _BUFFERS:
+            assert np.array_equal(getattr(d, f).cpu().numpy().view(np.uint8), _host_bytes(h, f)), f
+        if h.n:
+            _decodes_to(d, w_np)
