@@ -346,6 +346,8 @@ def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24
             raise ValueError("compress_on_device takes CUDA tensors; use compress() for host data")
         if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
             raise TypeError(f"expected BF16 words (bfloat16, int16 or uint16), got {w.dtype}")
+        if w.device != ws[0].device:
+            raise ValueError("all tensors of one batched build must be on one device")
         shapes.append(tuple(w.shape))
         flats.append(w.contiguous().reshape(-1))
     L = lib()
@@ -362,26 +364,28 @@ def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24
     outs = (GpuBuildOut * count)()
     views = []
     try:
-        for i, (f, p) in enumerate(zip(flats, params)):
+        # every output buffer of the call in one allocation, each at a
+        # 256-byte boundary (at least 16 bytes, so that no pointer is NULL)
+        layout, total = [], 0
+        for f, p in zip(flats, params):
             chunks = int(p.num_blocks) * threads_per_block
-            dev = f.device
-
-            def buf(cnt, dtype=torch.uint8):
-                # at least 16 bytes so that no pointer is NULL; the view has `cnt`
-                t = torch.empty(max(cnt, 16), dtype=dtype, device=dev)
-                return t, t[:cnt]
-
-            bs = buf(chunks * chunk_bytes + 16)
-            gp = buf(chunks * 5 // 8 + 16)
-            cc = buf(chunks + 16)
-            bp = buf(int(p.num_blocks) + 1, torch.int32)
-            lu = buf(int(p.num_luts) * 256, torch.int32)
-            cl = buf(256)
-            sm = buf((f.numel() + 15) // 16 * 16)
-            outs[i] = GpuBuildOut(bs[0].data_ptr(), gp[0].data_ptr(), cc[0].data_ptr(),
-                                  bp[0].data_ptr(), lu[0].data_ptr(), cl[0].data_ptr(),
-                                  sm[0].data_ptr())
-            views.append((bs[1], gp[1], cc[1], bp[1], lu[1], cl[1], sm[1]))
+            sizes = (chunks * chunk_bytes + 16, chunks * 5 // 8 + 16, chunks + 16,
+                     4 * (int(p.num_blocks) + 1), 4 * int(p.num_luts) * 256, 256,
+                     (f.numel() + 15) // 16 * 16)
+            offs = []
+            for nbytes in sizes:
+                offs.append(total)
+                total += (max(nbytes, 16) + 255) & ~255
+            layout.append((offs, sizes))
+        dev = flats[0].device
+        block = torch.empty(max(total, 256), dtype=torch.uint8, device=dev)
+        base = block.data_ptr()
+        for i, (offs, sizes) in enumerate(layout):
+            outs[i] = GpuBuildOut(*[base + o for o in offs])
+            v = [block[o:o + nbytes] for o, nbytes in zip(offs, sizes)]
+            v[3] = v[3].view(torch.int32)
+            v[4] = v[4].view(torch.int32)
+            views.append(v)
     except BaseException:
         for hnd in handles:
             L.df11_gpu_build_free(hnd)

@@ -761,6 +761,19 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
   std::lock_guard<std::mutex> lock(g_staging.mu);
   BeginSlot *stage = static_cast<BeginSlot *>(g_staging.get(sizeof(BeginSlot) * count));
   if (!stage) return DF11_ERR_NOMEM;
+  // one event per tensor: its counts are back
+  struct Events {
+    std::vector<cudaEvent_t> e;
+    ~Events() {
+      for (cudaEvent_t x : e)
+        if (x) cudaEventDestroy(x);
+    }
+  } ev;
+  ev.e.assign(count, nullptr);
+  for (int i = 0; i < count; ++i)
+    if (cudaEventCreateWithFlags(&ev.e[i], cudaEventDisableTiming) != cudaSuccess)
+      return DF11_ERR_CUDA;
+  const std::vector<cudaEvent_t> &events = ev.e;
 
   // histograms, and each tensor's last element (its codeword ends the stream)
   for (int i = 0; i < count; ++i) {
@@ -803,15 +816,17 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
         return fail(DF11_ERR_CUDA);
     }
     if (cudaMemcpyAsync(stage[i].hist, h->d_hist, sizeof(stage[i].hist), cudaMemcpyDeviceToHost,
-                        s) != cudaSuccess)
+                        s) != cudaSuccess ||
+        cudaEventRecord(events[i], s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
   }
-  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(DF11_ERR_CUDA);
 
-  // codebooks (host: 256 symbols each), then every unit's first bit and the
-  // totals
+  // codebooks (host: 256 symbols each), each as soon as its counts are
+  // back, while the device computes the previous tensors' bit offsets; then
+  // every unit's first bit and the totals
   for (int i = 0; i < count; ++i) {
     df11_gpu_build *h = hs[i];
+    if (cudaEventSynchronize(events[i]) != cudaSuccess) return fail(DF11_ERR_CUDA);
     uint64_t hist64[256];
     for (int k = 0; k < 256; ++k) hist64[k] = stage[i].hist[k];
     h->longest = df11_internal::codebook(hist64, h->len, h->code, h->luts);
