@@ -813,15 +813,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Add the warp's partial sums p (lane l: row `row`, only where `act`) into
-// y[row].  Active lanes hold consecutive 16-element groups, so rows do not
-// decrease across lanes; one or two rows take warp sums and one atomic add
-// each, more rows (matrices narrower than 512 columns) one add per lane.
+// y[row].  When the active lanes' rows take at most two values, each row
+// takes one warp sum and one atomic add; otherwise (matrices narrower than
+// 512 columns) every active lane adds its own.
 __device__ __forceinline__ void warp_row_add(float p, uint32_t row, bool act, float *y,
                                              int lane) {
-  const uint32_t mask = __ballot_sync(0xFFFFFFFFu, act);
-  if (!mask) return;
-  const uint32_t r0 = __shfl_sync(0xFFFFFFFFu, row, __ffs(mask) - 1);
-  const uint32_t r1 = __shfl_sync(0xFFFFFFFFu, row, 31 - __clz(mask));
+  if (!__any_sync(0xFFFFFFFFu, act)) return;
+  const uint32_t r0 = __reduce_min_sync(0xFFFFFFFFu, act ? row : 0xFFFFFFFFu);
+  const uint32_t r1 = __reduce_max_sync(0xFFFFFFFFu, act ? row : 0u);
   if (r0 == r1) {
     const float s = warp_sum(act ? p : 0.f);
     if (lane == 0) atomicAdd(y + r0, s);
@@ -834,6 +833,27 @@ __device__ __forceinline__ void warp_row_add(float p, uint32_t row, bool act, fl
     }
   } else if (act) {
     atomicAdd(y + row, p);
+  }
+}
+
+// y = W x: the outputs of a launch's products cleared by one small kernel
+// before it (the product kernel adds into them only after its
+// dependent-launch wait, which waits for this grid to complete)
+struct ClearArgs {
+  float *y[DF11_MAX_BATCH];
+  uint32_t rows[DF11_MAX_BATCH], batch[DF11_MAX_BATCH], stride[DF11_MAX_BATCH];
+  int count;
+};
+
+__global__ void __launch_bounds__(256) clear_rows_kernel(const __grid_constant__ ClearArgs c) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel may still read y
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  for (int t = 0; t < c.count; ++t) {
+    const uint64_t all = (uint64_t)c.rows[t] * c.batch[t];
+    for (uint64_t i = blockIdx.x * 256ull + threadIdx.x; i < all; i += (uint64_t)gridDim.x * 256) {
+      const uint64_t b = i / c.rows[t], r = i - b * c.rows[t];
+      c.y[t][b * c.stride[t] + r] = 0.f;
+    }
   }
 }
 
@@ -887,6 +907,64 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   } else if (SM == kSmSlot && sm_bytes) {
     bulk_g2s(smem_addr(slot + L::head_bytes), tk.sign_mantissa + sm_begin, sm_bytes, full);
   }
+}
+
+// The whole 16-element groups [g_begin, g_end) of a warp's range into
+// y += W x (batch rows nb <= NB): each lane sums its groups of one row in
+// registers and hands the sums over (warp sums per row, one atomic add each)
+// when it moves to the next row, and at the end.
+template <int SM, int NB>
+__device__ __forceinline__ void gemv_groups(const KTensor &tk, int lane, uint32_t base,
+                                            uint32_t g_begin, uint32_t g_end, uint32_t sm,
+                                            uint32_t region, const uint8_t *smg, uint32_t cols,
+                                            uint32_t nb) {
+  uint32_t e = base + 16u * (g_begin + (uint32_t)lane);
+  uint32_t row = e / cols, col = e - row * cols;
+  float acc[NB];
+#pragma unroll
+  for (int bi = 0; bi < NB; ++bi) acc[bi] = 0.f;
+  uint32_t acc_row = row;
+  bool has = false;
+  for (uint32_t gg = g_begin; gg < g_end; gg += 32) {
+    const uint32_t g = gg + (uint32_t)lane;
+    const bool act = g < g_end;
+    const bool moved = act && has && row != acc_row;
+    if (__any_sync(0xFFFFFFFFu, moved)) {
+#pragma unroll
+      for (int bi = 0; bi < NB; ++bi) {
+        if ((uint32_t)bi < nb) {
+          warp_row_add(acc[bi], acc_row, moved, tk.y + (size_t)bi * tk.y_stride, lane);
+          acc[bi] = moved ? 0.f : acc[bi];
+        }
+      }
+    }
+    if (act) {
+      const uint4 sv = SM == kSmGlobal ? __ldg(reinterpret_cast<const uint4 *>(smg) + g)
+                                       : lds128(sm + 16u * g);
+      const uint4 rv = lds128(region + 16u * g);
+      sts128_zero(region + 16u * g);
+      const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
+      const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+      const uint32_t wv[8] = {a.x, a.y, c.x, c.y, e2.x, e2.y, f.x, f.y};
+#pragma unroll
+      for (int bi = 0; bi < NB; ++bi) {
+        if ((uint32_t)bi < nb) {
+          const uint4 *xp = reinterpret_cast<const uint4 *>(tk.x + (size_t)bi * tk.x_stride + col);
+          acc[bi] += dot16(wv, __ldg(xp), __ldg(xp + 1));
+        }
+      }
+      acc_row = row;
+      has = true;
+    }
+    col += 512u;
+    while (col >= cols) {
+      col -= cols;
+      ++row;
+    }
+  }
+#pragma unroll
+  for (int bi = 0; bi < NB; ++bi)
+    if ((uint32_t)bi < nb) warp_row_add(acc[bi], acc_row, has, tk.y + (size_t)bi * tk.y_stride, lane);
 }
 
 // Register budget from the resident thread blocks the shared memory allows:
@@ -1126,36 +1204,11 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
       // 16-element group (within one row, since cols is a multiple of 16)
       // one partial sum per batch row, summed over the warp per row
       const uint32_t cols = tk.cols, nb = tk.batch;
-      uint32_t e = base + 16u * (g_begin + (uint32_t)lane);
-      uint32_t row = e / cols, col = e - row * cols;
-      for (uint32_t gg = g_begin; gg < g_end; gg += 32) {
-        const uint32_t g = gg + (uint32_t)lane;
-        const bool act = g < g_end;
-        uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (act) {
-          const uint4 sv = SM == kSmGlobal ? __ldg(reinterpret_cast<const uint4 *>(smg) + g)
-                                           : lds128(sm + 16u * g);
-          const uint4 rv = lds128(region + 16u * g);
-          sts128_zero(region + 16u * g);
-          const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
-          const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
-          wv[0] = a.x, wv[1] = a.y, wv[2] = c.x, wv[3] = c.y;
-          wv[4] = e2.x, wv[5] = e2.y, wv[6] = f.x, wv[7] = f.y;
-        }
-        for (uint32_t bi = 0; bi < nb; ++bi) {
-          float p = 0.f;
-          if (act) {
-            const uint4 *xp = reinterpret_cast<const uint4 *>(tk.x + (size_t)bi * tk.x_stride + col);
-            p = dot16(wv, __ldg(xp), __ldg(xp + 1));
-          }
-          warp_row_add(p, row, act, tk.y + (size_t)bi * tk.y_stride, lane);
-        }
-        col += 512u;
-        while (col >= cols) {
-          col -= cols;
-          ++row;
-        }
-      }
+      if (nb == 1)
+        gemv_groups<SM, 1>(tk, lane, base, g_begin, g_end, sm, region, smg, cols, nb);
+      else
+        gemv_groups<SM, DF11_GEMV_MAX_BATCH>(tk, lane, base, g_begin, g_end, sm, region, smg,
+                                             cols, nb);
       if (span) {
         // the elements outside whole groups, one per lane: lanes 0-15 the
         // first group, 16-31 the last one when it is another group
@@ -1640,20 +1693,20 @@ df11_status df11_decode_gemv(const df11_tensor *tensors, const df11_gemv *ops, i
     }
   }
   if (C && !(T == 256 && (C == 8 || C == 16 || C == 24))) return DF11_ERR_UNSUPPORTED;
-  // y = W x: clear the outputs first, in stream order
-  for (int i = 0; i < count; ++i) {
-    const df11_gemv &g = ops[i];
-    if (g.accumulate) continue;
-    const uint64_t rows = tensors[i].params.n / g.cols;
-    if (g.y_stride == rows) {
-      if (cudaMemsetAsync(g.y, 0, (size_t)g.batch * rows * sizeof(float), s) != cudaSuccess)
-        return DF11_ERR_CUDA;
-    } else {
-      for (uint32_t b = 0; b < g.batch; ++b)
-        if (cudaMemsetAsync(g.y + (size_t)b * g.y_stride, 0, rows * sizeof(float), s) !=
-            cudaSuccess)
-          return DF11_ERR_CUDA;
+  // y = W x: clear the outputs first, in stream order, one launch per 16
+  for (int i = 0; i < count; i += DF11_MAX_BATCH) {
+    ClearArgs ca{};
+    for (int j = i; j < count && j < i + DF11_MAX_BATCH; ++j) {
+      const df11_gemv &g = ops[j];
+      if (g.accumulate || tensors[j].params.n == 0) continue;
+      ca.y[ca.count] = g.y;
+      ca.rows[ca.count] = (uint32_t)(tensors[j].params.n / g.cols);
+      ca.batch[ca.count] = g.batch;
+      ca.stride[ca.count] = g.y_stride;
+      ++ca.count;
     }
+    if (ca.count && launch_pdl(clear_rows_kernel, 148u, 256u, 0, s, ca) != DF11_OK)
+      return DF11_ERR_CUDA;
   }
   for (int i = 0; i < count; i += DF11_MAX_BATCH) {
     const int c = count - i < DF11_MAX_BATCH ? count - i : DF11_MAX_BATCH;
