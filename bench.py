@@ -760,6 +760,12 @@ def run_gemv(args, world, rank, local):
     ms_bf16 = timed(bf16, max(3, args.steps // 4))
     ms = max_over_ranks(ms_local, world)
     value = sum_over_ranks(2.0 * n_total, world) / (ms * 1e-3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        x_host = [workloads.as_numpy_u16(x.view(torch.int16)) for x in xs]
+        done, secs, what = _oracle_gemv_sample(hosts, shapes, x_host, args.cpu_budget_s)
+        cpu = {"value": round(2.0 * done / secs / 1e9, 4), "unit": UNIT, "cores": 1,
+               "kind": "oracle", "sample": what + " (bit-serial C decode, float64 product)"}
     alg = sum(algorithmic_bytes(h) - 2 * h.n for h in hosts) + \
         sum(x.numel() * 2 for x in xs) + sum(y.numel() * 4 for y in ys)
     achieved = alg / (ms_local * 1e-3) / 1e9
@@ -793,7 +799,7 @@ def run_gemv(args, world, rank, local):
             "gpu_launches": args.steps,
             "clocks": clocks.summary(),
             "e2e": None,
-            "cpu_baseline": None,
+            "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
 
@@ -924,6 +930,8 @@ def run_reference(args, world, rank):
     units = workload_units(args.config, args.seed)
     if args.config == "build":
         return run_reference_build(args, world, units)
+    if args.config == "gemv":
+        return run_reference_gemv(args, world, units)
     import huffman_decode_df11_b200 as df11
     hosts = [df11.compress(thunk("cpu"), chunk_bytes=args.chunk_bytes,
                            threads_per_block=args.threads_per_block) for _, thunk in units]
@@ -948,6 +956,64 @@ def run_reference(args, world, rank):
                    "step": f"bounded sample of the workload, ~{budget:.1f} s of CPU work"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": what + " per step (single-threaded bit-serial C decode)"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _oracle_gemv_sample(hosts, shapes, x_rows, budget_s: float):
+    """The oracle's product (bit-serial decode, float64 matmul) on leading
+    rows of the workload's weights until the budget is spent; returns
+    (weights applied, seconds, description)."""
+    import oracle
+    done, t_used, names = 0, 0.0, 0
+    for h, (r, c), x in zip(hosts, shapes, x_rows):
+        if t_used >= budget_s:
+            break
+        rows = int(min(r, max(1, (budget_s - t_used) / 20e-9 / c)))
+        t = time.perf_counter()
+        w, _, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, rows * c)
+        W = oracle.bf16_to_f64(w).reshape(rows, c)
+        _ = oracle.bf16_to_f64(x).reshape(-1, c) @ W.T
+        t_used += time.perf_counter() - t
+        done += rows * c
+        names += 1
+    return done, t_used, f"{done} weights from the leading rows of {names} weight(s)"
+
+
+def run_reference_gemv(args, world, units):
+    """The comparison arm for the fused product: the oracle's decode and
+    float64 product, as they stand, on bounded samples of the workload."""
+    import huffman_decode_df11_b200 as df11
+    shapes = [(r, c) for _, r, c in workloads.BLOCK_SHAPES]
+    hosts = [df11.compress(thunk("cpu"), chunk_bytes=args.chunk_bytes,
+                           threads_per_block=args.threads_per_block) for _, thunk in units]
+    xs = [workloads.as_numpy_u16(workloads.gaussian_bf16(args.batch * c, 1.0, 77 + i))
+          for i, (_, c) in enumerate(shapes)]
+    n_total = sum(h.n for h in hosts)
+    budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        _oracle_gemv_sample(hosts, shapes, xs, budget)
+    tot_done, tot_s, what = 0, 0.0, ""
+    for _ in range(args.steps):
+        d, s_, what = _oracle_gemv_sample(hosts, shapes, xs, budget)
+        tot_done += d
+        tot_s += s_
+    value = 2.0 * tot_done / tot_s / 1e9
+    line = {
+        "impl": "reference", "metric": GEMV_METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32+f64",
+        "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
+        "config": {"workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
+                   "elements": n_total, "batch": args.batch, "chunk_bytes": args.chunk_bytes,
+                   "threads_per_block": args.threads_per_block,
+                   "step": f"bounded sample of the workload, ~{budget:.1f} s of CPU work"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": what + " per step (bit-serial C decode, float64 product)"},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
