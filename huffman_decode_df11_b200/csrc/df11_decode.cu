@@ -790,19 +790,23 @@ constexpr int kWsStages = 2;
 enum SmMode { kSmSlot = 0, kSmGlobal = 1, kSmWarp = 2 };
 
 // ---- fused matrix-vector product -------------------------------------------
+// a BF16 word (low 16 bits) widened to fp32, exactly
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
-// sum over 16 elements of w * x, both BF16, two per word, fp32 arithmetic
-// (BF16 products are exact in fp32)
+// sum over 16 elements of w * x, both BF16, two per word, in fp32: the
+// mixed-precision fused multiply-add of PTX takes the BF16 halves of a
+// register as they are (no widening instructions); its product is exact
+// and the sum rounds once, as fmaf on the widened values would
 __device__ __forceinline__ float dot16(const uint32_t (&w)[8], const uint4 &x0, const uint4 &x1) {
   const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
   float a = 0.f, b = 0.f;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    a = fmaf(bf16_lo(w[k]), bf16_lo(xv[k]), a);
-    b = fmaf(bf16_hi(w[k]), bf16_hi(xv[k]), b);
-  }
+  for (int k = 0; k < 8; ++k)
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\tfma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
+        : "+f"(a), "+f"(b)
+        : "r"(w[k]), "r"(xv[k]));
   return a + b;
 }
 
