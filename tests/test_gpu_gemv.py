@@ -170,3 +170,31 @@ def test_argument_errors():
     torch.cuda.synchronize()
     with pytest.raises(ValueError):
         df11.decode_gemv([d], [x[:, :128]], [y])
+
+
+def test_more_than_one_launch_and_both_modes():
+    """20 weights in one call: the descriptor array is split into launches
+    of at most 16 (product and clearing kernels alike); once adding into a
+    given y, once clearing it first."""
+    hs, ds, xs, y0s = [], [], [], []
+    for i in range(20):
+        rows, cols = 32 + 16 * i, 256 * (1 + i % 3)
+        w = _weights(rows, cols, 200 + i)
+        h = df11.compress(workloads.as_numpy_u16(w))
+        h.shape = (rows, cols)
+        hs.append(h)
+        ds.append(df11.to_device(h, "cuda"))
+        xs.append(_acts(2, cols, 300 + i))
+        y0s.append(torch.randn(2, rows, dtype=torch.float64))
+    xd = [x.cuda().view(torch.bfloat16) for x in xs]
+    err = df11.new_error_word()
+    ya = [y0.float().cuda() for y0 in y0s]
+    df11.decode_gemv(ds, xd, ya, accumulate=True, err=err)
+    yc = [torch.full_like(y, 7.0) for y in ya]
+    df11.decode_gemv(ds, xd, yc, accumulate=False, err=err)
+    torch.cuda.synchronize()
+    df11.check_device_error(err)
+    for h, x, y0, y_acc, y_clr in zip(hs, xs, y0s, ya, yc):
+        cols = h.shape[1]
+        _check(h, cols, x, y_acc, y0=y0.float().double().numpy())
+        _check(h, cols, x, y_clr)
