@@ -130,7 +130,10 @@ __device__ __forceinline__ void count8(const uint4 &v, uint32_t live, int lo, ui
 }
 
 __global__ void __launch_bounds__(kThreads) hist_kernel(const uint16_t *w, uint64_t n, bool vec,
-                                                        unsigned long long *hist) {
+                                                        unsigned long long *hist,
+                                                        unsigned long long *last) {
+  // the last element (its codeword ends the stream), for the builder
+  if (last && blockIdx.x == 0 && threadIdx.x == 0 && n) *last = w[n - 1];
   __shared__ uint32_t h[kThreads / 32][256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int j = threadIdx.x; j < (kThreads / 32) * 256; j += kThreads) (&h[0][0])[j] = 0;
@@ -277,22 +280,47 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const unsigned long 
 }
 
 // Before packing: first elements preset to n, gaps cleared, the bitstream
-// words that two units share cleared (they are ORed into), maxima cleared.
-__global__ void prepare_kernel(uint32_t *first_elem, uint8_t *gap, uint64_t chunks, uint32_t n,
-                               const Ranges r, uint32_t *bs32, unsigned int *maxima) {
-  uint64_t all = chunks + 1 > r.units ? chunks + 1 : r.units;
-  all = all > 3 ? all : 3;  // the maxima
+// words that two units share cleared (they are ORed into), maxima cleared;
+// also the output paddings no kernel writes cleared, and the tables copied
+// from the device staging area into the caller's buffers.
+struct PrepareArgs {
+  uint32_t *first_elem;
+  uint8_t *gap;
+  uint64_t chunks;
+  uint32_t n;
+  Ranges r;
+  uint32_t *bs32;
+  unsigned int *maxima;
+  uint8_t *zero[4];        // byte ranges to clear
+  uint32_t zero_bytes[4];
+  const uint4 *luts_src;   // num_luts * 1 KB
+  uint4 *luts_dst;         // 16-byte aligned
+  uint32_t luts_vec4;      // 16-byte words of the tables
+  const uint8_t *lens_src;
+  uint8_t *lens_dst;       // 256 bytes, any alignment
+};
+
+__global__ void prepare_kernel(const PrepareArgs a) {
+  uint64_t all = a.chunks + 1 > a.r.units ? a.chunks + 1 : a.r.units;
+  all = all > a.luts_vec4 ? all : a.luts_vec4;
+  all = all > 256 ? all : 256;  // the code lengths, the paddings, the maxima
   for (uint64_t i = blockIdx.x * 256ull + threadIdx.x; i < all; i += (uint64_t)gridDim.x * 256) {
-    if (i <= chunks) {
-      first_elem[i] = n;
-      gap[i] = 0;
+    if (i <= a.chunks) {
+      a.first_elem[i] = a.n;
+      a.gap[i] = 0;
     }
-    if (i >= 1 && i < r.units) {
-      const unsigned long long s = unit_start(r, i);
-      if (s & 31u) bs32[s >> 5] = 0;
+    if (i >= 1 && i < a.r.units) {
+      const unsigned long long st = unit_start(a.r, i);
+      if (st & 31u) a.bs32[st >> 5] = 0;
     }
-    if (i < 3) maxima[i] = 0;
+    if (i < 3) a.maxima[i] = 0;
+    if (i < a.luts_vec4) a.luts_dst[i] = a.luts_src[i];
+    if (i < 256) a.lens_dst[i] = a.lens_src[i];
   }
+  // paddings: each at most a block of the bitstream plus 16 bytes
+  for (int k = 0; k < 4; ++k)
+    for (uint32_t i = blockIdx.x * 256u + threadIdx.x; i < a.zero_bytes[k]; i += gridDim.x * 256u)
+      a.zero[k][i] = 0;
 }
 
 // ---- pack ----------------------------------------------------------------
@@ -669,6 +697,7 @@ struct df11_gpu_build {
   uint32_t *d_first = nullptr;
   unsigned int *d_max = nullptr;
   uint8_t *d_gap = nullptr;
+  uint8_t *d_tables = nullptr;  // the luts, then the code lengths, for the prepare kernel
 };
 
 namespace {
@@ -710,11 +739,9 @@ Staging g_staging;
 
 // what one tensor's phase 1 reads back and sends
 struct BeginSlot {
-  unsigned long long hist[256];
+  unsigned long long hist[257];  // the counts, then the last element
   uint2 tab[256];
   unsigned long long total;
-  uint16_t last;
-  uint16_t pad[3];
 };
 
 df11_status check_begin_args(const uint16_t *d_bf16, uint64_t n, uint32_t C, uint32_t T) {
@@ -791,7 +818,7 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     h->ranges = h->r.units < slots ? h->r.units : slots;
     h->r.per = h->ranges ? (h->r.units + h->ranges - 1) / h->ranges : 1;
     if (h->ranges) h->ranges = (h->r.units + h->r.per - 1) / h->r.per;
-    const uint64_t o_tab = round256(256 * sizeof(unsigned long long));
+    const uint64_t o_tab = round256(257 * sizeof(unsigned long long));
     const uint64_t o_tot = o_tab + round256(256 * sizeof(uint2));
     const uint64_t o_rs = o_tot + round256(h->ranges * sizeof(unsigned long long) + 8);
     const uint64_t o_loc = o_rs + round256((h->ranges + 1) * sizeof(unsigned long long));
@@ -803,17 +830,13 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     h->d_range_total = reinterpret_cast<unsigned long long *>(base1 + o_tot);
     h->r.range_start = reinterpret_cast<unsigned long long *>(base1 + o_rs);
     h->r.local = reinterpret_cast<uint32_t *>(base1 + o_loc);
-    stage[i].last = 0;
-    if (cudaMemsetAsync(h->d_hist, 0, 256 * sizeof(unsigned long long), s) != cudaSuccess)
+    if (cudaMemsetAsync(h->d_hist, 0, 257 * sizeof(unsigned long long), s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
     if (h->n) {
       const uint64_t tiles = (h->n + kPerCta - 1) / kPerCta;
       const unsigned grid = (unsigned)(tiles < hist_slots ? tiles : hist_slots);
-      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_hist);
-      if (cudaGetLastError() != cudaSuccess ||
-          cudaMemcpyAsync(&stage[i].last, d_bf16[i] + (h->n - 1), 2, cudaMemcpyDeviceToHost,
-                          s) != cudaSuccess)
-        return fail(DF11_ERR_CUDA);
+      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_hist, h->d_hist + 256);
+      if (cudaGetLastError() != cudaSuccess) return fail(DF11_ERR_CUDA);
     }
     if (cudaMemcpyAsync(stage[i].hist, h->d_hist, sizeof(stage[i].hist), cudaMemcpyDeviceToHost,
                         s) != cudaSuccess ||
@@ -850,18 +873,21 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
   for (int i = 0; i < count; ++i) {
     df11_gpu_build *h = hs[i];
     h->total = stage[i].total;
-    if (h->n) h->last_start = h->total - h->len[(stage[i].last >> 7) & 0xFF];
+    if (h->n) h->last_start = h->total - h->len[(stage[i].hist[256] >> 7) & 0xFF];
     const uint64_t block_bits = 8ull * C * T;
     h->num_blocks = (h->total + block_bits - 1) / block_bits;
     h->chunks = h->num_blocks * T;
     const uint64_t o_max = round256((h->chunks + 1) * sizeof(uint32_t));
     const uint64_t o_gap = o_max + 256;
-    if (scratch_alloc(&h->scratch2, o_gap + round256(h->chunks + 1), s) != cudaSuccess)
+    const uint64_t o_tables = o_gap + round256(h->chunks + 1);
+    const uint64_t table_bytes = h->luts.size() * 4 + 256;
+    if (scratch_alloc(&h->scratch2, o_tables + round256(table_bytes), s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
     char *base2 = static_cast<char *>(h->scratch2);
     h->d_first = reinterpret_cast<uint32_t *>(base2);
     h->d_max = reinterpret_cast<unsigned int *>(base2 + o_max);
     h->d_gap = reinterpret_cast<uint8_t *>(base2 + o_gap);
+    h->d_tables = reinterpret_cast<uint8_t *>(base2 + o_tables);
     fill_params(h, &params[i]);
     std::memcpy(code_lengths + 256 * (size_t)i, h->len, 256);
   }
@@ -927,23 +953,21 @@ df11_status df11_gpu_build_finish_batched(df11_gpu_build *const *handles, int co
     uint8_t *st_luts = stage + off[i], *st_lens = st_luts + lut_bytes;
     std::memcpy(st_luts, h->luts.data(), lut_bytes);
     std::memcpy(st_lens, h->len, 256);
-    // every byte the kernels do not write: the padding after each buffer
-    const bool ok =
-        cudaMemsetAsync(o.bitstream + bs_written, 0, bs_bytes - bs_written, s) == cudaSuccess &&
-        cudaMemsetAsync(o.gaps + chunks * 5 / 8, 0, gaps_bytes - chunks * 5 / 8, s) ==
-            cudaSuccess &&
-        cudaMemsetAsync(o.chunk_counts + chunks, 0, 16, s) == cudaSuccess &&
-        (sm_bytes == n ||
-         cudaMemsetAsync(o.sign_mantissa + n, 0, sm_bytes - n, s) == cudaSuccess) &&
-        cudaMemcpyAsync(o.luts, st_luts, lut_bytes, cudaMemcpyHostToDevice, s) == cudaSuccess &&
-        cudaMemcpyAsync(o.code_lengths, st_lens, 256, cudaMemcpyHostToDevice, s) == cudaSuccess;
-    if (!ok) {
+    if (cudaMemcpyAsync(h->d_tables, st_luts, lut_bytes + 256, cudaMemcpyHostToDevice, s) !=
+        cudaSuccess) {
       st = DF11_ERR_CUDA;
       break;
     }
     uint32_t *bs32 = reinterpret_cast<uint32_t *>(o.bitstream);
-    prepare_kernel<<<148 * 4, 256, 0, s>>>(h->d_first, h->d_gap, chunks, (uint32_t)n, h->r, bs32,
-                                           h->d_max);
+    // every byte the kernels do not write: the padding after each buffer
+    PrepareArgs pr{h->d_first, h->d_gap, chunks, (uint32_t)n, h->r, bs32, h->d_max,
+                   {o.bitstream + bs_written, o.gaps + chunks * 5 / 8, o.chunk_counts + chunks,
+                    o.sign_mantissa + n},
+                   {(uint32_t)(bs_bytes - bs_written), (uint32_t)(gaps_bytes - chunks * 5 / 8), 16u,
+                    (uint32_t)(sm_bytes - n)},
+                   reinterpret_cast<const uint4 *>(h->d_tables), reinterpret_cast<uint4 *>(o.luts),
+                   (uint32_t)(lut_bytes / 16), h->d_tables + lut_bytes, o.code_lengths};
+    prepare_kernel<<<148 * 4, 256, 0, s>>>(pr);
     const uint32_t chunk_bits = 8 * h->C, block_bits = 8 * h->C * h->T;
     const uint32_t chunk_words = h->C / 4, block_words = h->C / 4 * h->T;
     const PackArgs pa{d_bf16[i], n, h->vec, h->d_tab, h->r, bs32, o.sign_mantissa, h->d_gap,
@@ -1032,7 +1056,8 @@ extern "C" df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t 
   if (n) {
     const uint64_t tiles = (n + kPerCta - 1) / kPerCta, slots = resident(hist_kernel);
     const bool vec = ((uintptr_t)d_bf16 & 15) == 0;
-    hist_kernel<<<(unsigned)(tiles < slots ? tiles : slots), kThreads, 0, s>>>(d_bf16, n, vec, d);
+    hist_kernel<<<(unsigned)(tiles < slots ? tiles : slots), kThreads, 0, s>>>(d_bf16, n, vec, d,
+                                                                               nullptr);
   }
   unsigned long long counts[256];
   if (cudaGetLastError() != cudaSuccess ||
