@@ -781,6 +781,9 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
   cudaStream_t s = (cudaStream_t)stream;
   std::vector<df11_gpu_build *> hs(count, nullptr);
   auto fail = [&](df11_status st) {
+    // copies into the staging buffer may still be queued: let them land
+    // before the buffer is released to another call
+    cudaStreamSynchronize(s);
     for (auto *h : hs) df11_gpu_build_free(h);
     return st;
   };
