@@ -350,11 +350,13 @@ typedef struct df11_gpu_build_out {
 
 /*
  * Both phases for `count` tensors at once (d_bf16[i], n[i]; params and
- * handles arrays of count, code_lengths count*256 bytes, all host arrays):
- * each phase synchronises the stream once for all of them instead of once
- * per tensor.  Same conventions as the single-tensor calls; on an error in
- * phase 1 no handle is returned (all NULL), and phase 2 releases every
- * handle in all cases.  The single-tensor calls are these with count 1.
+ * handles arrays of count, code_lengths count*256 bytes, all host arrays).
+ * Phase 1 waits for each tensor's counts as they arrive (computing its
+ * code while the device works on the later tensors) and synchronises the
+ * stream once; phase 2 synchronises it once.  Same conventions as the
+ * single-tensor calls; on an error in phase 1 no handle is returned (all
+ * NULL), and phase 2 releases every handle in all cases.  The
+ * single-tensor calls are these with count 1.
  */
 df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const uint64_t *n,
                                          int count, uint32_t chunk_bytes,
