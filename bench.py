@@ -587,6 +587,11 @@ def run_build(args, world, rank, local):
         step()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clocks:
+        # keep the GPU busy (untimed) while the sampler starts, so that the
+        # samples taken around a short timed region show clocks under load
+        t_busy = time.perf_counter()
+        while time.perf_counter() - t_busy < 0.4:
+            step()
         barrier(world)
         torch.cuda.synchronize()
         t0.record(stream)
