@@ -693,7 +693,7 @@ def run_gemv(args, world, rank, local):
         raise SystemExit("--batch must be 1..8")
     units = workload_units(args.config, seed)
     shapes = [(r, c) for _, r, c in workloads.BLOCK_SHAPES]
-    hosts, ds, ws_bf16 = [], [], []
+    hosts, ds, ws_bf16, fused_ds = [], [], [], []
     for (name, thunk), shape in zip(units, shapes):
         bits = thunk(device)
         h = df11.compress(bits, chunk_bytes=args.chunk_bytes,
@@ -701,6 +701,11 @@ def run_gemv(args, world, rank, local):
         h.shape = shape
         hosts.append(h)
         ds.append(df11.to_device(h, device))
+        if args.interleave != 1:  # the fused path's weights, in the interleaved order
+            hi = df11.compress(bits.view(shape), chunk_bytes=args.chunk_bytes,
+                               threads_per_block=args.threads_per_block,
+                               interleave=args.interleave)
+            fused_ds.append(df11.to_device(hi, device))
         ws_bf16.append(bits.view(shape).view(torch.bfloat16))
     n_total = sum(h.n for h in hosts)
     g = torch.Generator(device=device)
@@ -710,8 +715,9 @@ def run_gemv(args, world, rank, local):
     err = df11.new_error_word(device)
     stream = torch.cuda.current_stream()
 
+    fds = fused_ds if args.interleave != 1 else ds
     # parity: within gamma_cols * |x||W|^T of the float64 product
-    df11.decode_gemv(ds, xs, ys, err=err)
+    df11.decode_gemv(fds, xs, ys, err=err)
     torch.cuda.synchronize()
     df11.check_device_error(err)
     for (name, _), (r, c), x, y, w in zip(units, shapes, xs, ys, ws_bf16):
@@ -727,7 +733,7 @@ def run_gemv(args, world, rank, local):
     plans = [df11.DecodePlan([d], [scratch[: d.n]]) for d in ds]
 
     def fused():
-        df11.decode_gemv(ds, xs, ys, err=err, stream=stream)
+        df11.decode_gemv(fds, xs, ys, err=err, stream=stream)
 
     ybs = [torch.empty(B, r, dtype=torch.bfloat16, device=device) for r, _ in shapes]
 
@@ -784,7 +790,8 @@ def run_gemv(args, world, rank, local):
             "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
             "config": {
                 "workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
-                "elements": n_total, "batch": B, "chunk_bytes": args.chunk_bytes,
+                "elements": n_total, "batch": B, "interleave": args.interleave,
+                "chunk_bytes": args.chunk_bytes,
                 "threads_per_block": args.threads_per_block,
                 "l2": "inputs larger than L2 (no flush)",
                 "parallelism": f"replicas x{world} (no collective)",
@@ -1106,6 +1113,9 @@ def main(argv=None):
                     help="chunks per format block (T) of the compressed format")
     ap.add_argument("--batch", type=int, default=1,
                     help="activation rows of the gemv workload (1-8)")
+    ap.add_argument("--interleave", type=int, default=1,
+                    help="gemv workload: rows interleaved per 16 columns in the fused "
+                         "path's compressed weights (1: row-major)")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -77,7 +77,7 @@ class GemvOp(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("cols", ctypes.c_uint32),
                 ("batch", ctypes.c_uint32), ("x_stride", ctypes.c_uint32),
                 ("y_stride", ctypes.c_uint32), ("accumulate", ctypes.c_int32),
-                ("pad", ctypes.c_uint32)]
+                ("interleave", ctypes.c_uint32)]
 
 
 class HostTensor(ctypes.Structure):
@@ -181,6 +181,7 @@ class Df11Host:
     sign_mantissa: np.ndarray  # uint8 (n rounded up to 16)
     chunk_counts: np.ndarray   # uint8, codewords starting in each chunk
     shape: tuple = ()
+    interleave: int = 1        # rows interleaved per 16 columns in the stream (1: row-major)
 
     @property
     def n(self) -> int:
@@ -216,8 +217,33 @@ def _np_copy(ptr, count, dtype):
     return np.frombuffer(buf, dtype=dtype, count=count).copy()
 
 
+def interleave_rows(w, rows_per_block: int):
+    """The element order df11_gemv calls R rows interleaved (R =
+    rows_per_block): for each block of R rows and each group of 16 columns,
+    the R rows' 16 elements one after another.  Takes a 2-D array or tensor
+    (rows a multiple of R, columns of 16) and returns it flattened in that
+    order."""
+    R = int(rows_per_block)
+    rows, cols = w.shape
+    if R < 1 or R > 32 or R & (R - 1) or rows % R or cols % 16:
+        raise ValueError(f"cannot interleave a {rows}x{cols} matrix by {R} rows")
+    v = w.reshape(rows // R, R, cols // 16, 16)
+    v = v.permute(0, 2, 1, 3) if isinstance(v, torch.Tensor) else v.transpose(0, 2, 1, 3)
+    return v.reshape(-1) if isinstance(v, torch.Tensor) else np.ascontiguousarray(v).reshape(-1)
+
+
+def deinterleave_rows(flat, shape, rows_per_block: int):
+    """The inverse of interleave_rows: a stream-ordered flat array or
+    tensor back to the rows x cols matrix."""
+    R = int(rows_per_block)
+    rows, cols = shape
+    v = flat.reshape(rows // R, cols // 16, R, 16)
+    v = v.permute(0, 2, 1, 3) if isinstance(v, torch.Tensor) else v.transpose(0, 2, 1, 3)
+    return v.reshape(rows, cols)
+
+
 def compress(w, chunk_bytes: int = 24, threads_per_block: int = 256,
-             threads: int = 0) -> Df11Host:
+             threads: int = 0, interleave: int = 1) -> Df11Host:
     """Encode a BF16 tensor (host or device; copied to host) into DF11.
     The default chunk of 24 bitstream bytes per thread decodes fastest on
     B200 of the built kernel shapes (fewer per-chunk setup steps per element
@@ -225,6 +251,8 @@ def compress(w, chunk_bytes: int = 24, threads_per_block: int = 256,
     a valid format."""
     shape = tuple(w.shape) if hasattr(w, "shape") else ()
     a = _as_u16_numpy(w)
+    if interleave != 1:
+        a = interleave_rows(a.reshape(shape), interleave)
     h = HostTensor()
     L = lib()
     _check(L.df11_build(a.ctypes.data if a.size else None, a.size, chunk_bytes,
@@ -241,6 +269,7 @@ def compress(w, chunk_bytes: int = 24, threads_per_block: int = 256,
             sign_mantissa=_np_copy(h.sign_mantissa, h.sign_mantissa_bytes, np.uint8),
             chunk_counts=_np_copy(h.chunk_counts, h.chunk_counts_bytes, np.uint8),
             shape=shape,
+            interleave=int(interleave),
         )
     finally:
         L.df11_host_tensor_free(ctypes.byref(h))
@@ -263,6 +292,7 @@ class Df11Device:
     chunk_counts: Optional[torch.Tensor] = None
     shape: tuple = ()
     decode_table: Optional[torch.Tensor] = None  # df11_build_decode_table output
+    interleave: int = 1  # rows interleaved per 16 columns in the stream (1: row-major)
 
     @property
     def n(self) -> int:
@@ -308,6 +338,7 @@ def to_device(h: Df11Host, device="cuda", decode_table: bool = True) -> Df11Devi
         sign_mantissa=_np_to(h.sign_mantissa, device),
         chunk_counts=_np_to(h.chunk_counts, device),
         shape=h.shape,
+        interleave=int(getattr(h, "interleave", 1)),
     )
     if decode_table:
         d.decode_table = build_decode_table(d)
@@ -322,18 +353,20 @@ class GpuBuildOut(ctypes.Structure):
 
 
 def compress_on_device(w: torch.Tensor, chunk_bytes: int = 24, threads_per_block: int = 256,
-                       stream=None, decode_table: bool = True) -> Df11Device:
+                       stream=None, decode_table: bool = True,
+                       interleave: int = 1) -> Df11Device:
     """Encode a BF16 tensor that is in device memory into DF11 on the device
     (df11_gpu_build_begin / df11_gpu_build_finish): the same bytes and
     parameters as compress() of the same words, written straight into
     device buffers.  Synchronises the stream."""
     return compress_on_device_batched([w], chunk_bytes, threads_per_block, stream,
-                                      decode_table)[0]
+                                      decode_table, interleave)[0]
 
 
 def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24,
                                threads_per_block: int = 256, stream=None,
-                               decode_table: bool = True) -> List[Df11Device]:
+                               decode_table: bool = True,
+                               interleave: int = 1) -> List[Df11Device]:
     """compress_on_device for several tensors, with one stream
     synchronisation per phase for all of them
     (df11_gpu_build_begin_batched / _finish_batched)."""
@@ -349,7 +382,8 @@ def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24
         if w.device != ws[0].device:
             raise ValueError("all tensors of one batched build must be on one device")
         shapes.append(tuple(w.shape))
-        flats.append(w.contiguous().reshape(-1))
+        flats.append(interleave_rows(w, interleave).contiguous() if interleave != 1
+                     else w.contiguous().reshape(-1))
     L = lib()
     sh = _stream_handle(stream)
     vp = ctypes.c_void_p
@@ -396,7 +430,7 @@ def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24
     for p, v, shape in zip(params, views, shapes):
         d = Df11Device(params=Params.from_buffer_copy(p), bitstream=v[0], gaps=v[1],
                        chunk_counts=v[2], block_out_pos=v[3], luts=v[4], code_lengths=v[5],
-                       sign_mantissa=v[6], shape=shape)
+                       sign_mantissa=v[6], shape=shape, interleave=int(interleave))
         if decode_table:
             d.decode_table = build_decode_table(d, stream)
         out.append(d)
@@ -526,7 +560,7 @@ def _gemv_op(d: "Df11Device", x: torch.Tensor, y: torch.Tensor, accumulate: bool
     if x2.device != d.device or y2.device != d.device:
         raise ValueError("x and y must be on the weight's device")
     return GemvOp(x2.data_ptr(), y2.data_ptr(), cols, x2.shape[0], x2.stride(0),
-                  y2.stride(0), 1 if accumulate else 0, 0)
+                  y2.stride(0), 1 if accumulate else 0, int(getattr(d, "interleave", 1)))
 
 
 def decode_gemv(ds: Sequence["Df11Device"], xs: Sequence[torch.Tensor],

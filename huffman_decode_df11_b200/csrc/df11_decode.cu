@@ -88,6 +88,8 @@ struct KTensor {
   const uint16_t *x;  // BF16 activations, batch rows of x_stride elements
   float *y;           // batch rows of y_stride floats
   uint32_t cols, batch, x_stride, y_stride;
+  uint32_t interleave_log2;  // rows interleaved per 16-column group: 2^this (0: row-major)
+  uint32_t pad2;
 };
 
 struct KBatch {
@@ -913,17 +915,33 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   }
 }
 
+// Where 16-element group q of the stream (q = element / 16) sits in the
+// rows x cols weight: with R = 2^s rows interleaved, the stream holds, per
+// block of R rows and per 16-column group, the R rows' 16 elements one after
+// another (R = 1: row-major).  Returns the row; *cg = the column group.
+__device__ __forceinline__ uint32_t group_row(uint32_t q, uint32_t groups_per_row, uint32_t s,
+                                              uint32_t *cg) {
+  const uint32_t t = q >> s, r = q & ((1u << s) - 1u);
+  const uint32_t rb = t / groups_per_row;
+  *cg = t - rb * groups_per_row;
+  return (rb << s) + r;
+}
+
 // The whole 16-element groups [g_begin, g_end) of a warp's range into
 // y += W x (batch rows nb <= NB): each lane sums its groups of one row in
 // registers and hands the sums over (warp sums per row, one atomic add each)
-// when it moves to the next row, and at the end.
+// when it moves to another row, and at the end.  With R rows interleaved
+// a lane keeps one row of each block of R rows and the lanes that share
+// a column group read the same activations.
 template <int SM, int NB>
 __device__ __forceinline__ void gemv_groups(const KTensor &tk, int lane, uint32_t base,
                                             uint32_t g_begin, uint32_t g_end, uint32_t sm,
                                             uint32_t region, const uint8_t *smg, uint32_t cols,
                                             uint32_t nb) {
-  uint32_t e = base + 16u * (g_begin + (uint32_t)lane);
-  uint32_t row = e / cols, col = e - row * cols;
+  const uint32_t s = tk.interleave_log2, gpr = cols >> 4;  // column groups per row
+  const uint32_t step = 32u >> s;                         // column groups per iteration
+  uint32_t cg;
+  uint32_t row = group_row((base >> 4) + g_begin + (uint32_t)lane, gpr, s, &cg);
   float acc[NB];
 #pragma unroll
   for (int bi = 0; bi < NB; ++bi) acc[bi] = 0.f;
@@ -953,17 +971,20 @@ __device__ __forceinline__ void gemv_groups(const KTensor &tk, int lane, uint32_
 #pragma unroll
       for (int bi = 0; bi < NB; ++bi) {
         if ((uint32_t)bi < nb) {
-          const uint4 *xp = reinterpret_cast<const uint4 *>(tk.x + (size_t)bi * tk.x_stride + col);
+          const uint4 *xp =
+              reinterpret_cast<const uint4 *>(tk.x + (size_t)bi * tk.x_stride + 16u * cg);
           acc[bi] += dot16(wv, __ldg(xp), __ldg(xp + 1));
         }
       }
       acc_row = row;
       has = true;
     }
-    col += 512u;
-    while (col >= cols) {
-      col -= cols;
-      ++row;
+    // the next group of this lane: `step` column groups on, in the same rows
+    // or, past the row's end, in the next block of rows
+    cg += step;
+    while (cg >= gpr) {
+      cg -= gpr;
+      row += 1u << s;
     }
   }
 #pragma unroll
@@ -1224,7 +1245,9 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
                                            lds8(region + i))
                                    : 0u;
         sts8_zero(region + i);  // the loop zeroed whole groups; this does the rest
-        const uint32_t ei = base + i, r = ei / cols, ci = ei - r * cols;
+        uint32_t cgi;
+        const uint32_t r = group_row((base + i) >> 4, cols >> 4, tk.interleave_log2, &cgi);
+        const uint32_t ci = 16u * cgi + (i & 15u);
         const uint32_t half = __ballot_sync(0xFFFFFFFFu, act) >> (lane & 16);
         for (uint32_t bi = 0; bi < nb; ++bi) {
           float p = act ? bf16_lo(wbits) * bf16_lo(tk.x[(size_t)bi * tk.x_stride + ci]) : 0.f;
@@ -1554,6 +1577,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
       k.batch = ops[i].batch;
       k.x_stride = ops[i].x_stride;
       k.y_stride = ops[i].y_stride;
+      k.interleave_log2 = ops[i].interleave > 1 ? (uint32_t)__builtin_ctz(ops[i].interleave) : 0u;
     }
     blocks[kb.count] = p.num_blocks;
     ++kb.count;
@@ -1682,6 +1706,8 @@ df11_status df11_decode_gemv(const df11_tensor *tensors, const df11_gemv *ops, i
     const uint64_t rows = p.n / g.cols;
     if (g.batch < 1 || g.batch > DF11_GEMV_MAX_BATCH) return DF11_ERR_INVALID;
     if (g.x_stride < g.cols || g.x_stride % 8 || g.y_stride < rows) return DF11_ERR_INVALID;
+    const uint32_t il = g.interleave ? g.interleave : 1u;
+    if (il > 32 || (il & (il - 1)) || rows % il) return DF11_ERR_INVALID;
     if (!aligned(g.x, 16) || !aligned(g.y, 4)) return DF11_ERR_ALIGN;
     df11_tensor v = t;
     v.out_bf16 = reinterpret_cast<uint16_t *>(16);  // not written; passes the output checks

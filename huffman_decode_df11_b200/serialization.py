@@ -10,8 +10,8 @@ Each compressed tensor `name` is stored as raw buffers:
   (U8);
 - `name.block_out_pos` and `name.luts` (U32).
 
-Its format parameters and original shape go in the header's `__metadata__` as JSON under
-`name.df11`. The header is padded with spaces so that the data start at a 16-byte boundary.
+Its format parameters, original shape and element order (rows interleaved per 16 columns; 1 for
+row-major) go in the header's `__metadata__` as JSON under `name.df11`. The header is padded with spaces so that the data start at a 16-byte boundary.
 Every buffer's length is a multiple of 16 (`block_out_pos` is zero-padded to one), so every buffer
 of a file starts 16-byte aligned, ready to be mapped.
 
@@ -73,7 +73,8 @@ def save(path: str, tensors: Mapping[str, Df11Host],
     offset = 0
     for name, h in tensors.items():
         params = {f: int(getattr(h.params, f)) for f in _PARAM_FIELDS}
-        meta[f"{name}.df11"] = json.dumps({"params": params, "shape": list(h.shape)})
+        meta[f"{name}.df11"] = json.dumps({"params": params, "shape": list(h.shape),
+                                           "interleave": int(getattr(h, "interleave", 1))})
         for suffix, dname, dt in _BUFFERS:
             a = np.ascontiguousarray(getattr(h, suffix), dtype=dt)
             if suffix == "block_out_pos" and a.nbytes % 16:
@@ -153,5 +154,6 @@ def load(path: str) -> Dict[str, Df11Host]:
                 f.seek(start + b)
                 a = np.frombuffer(f.read(e - b), dtype=dt)
                 arrays[suffix] = a[:need].copy()
-            out[name] = Df11Host(params=p, shape=tuple(info["shape"]), **arrays)
+            out[name] = Df11Host(params=p, shape=tuple(info["shape"]),
+                                 interleave=int(info.get("interleave", 1)), **arrays)
         return out

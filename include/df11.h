@@ -184,7 +184,13 @@ typedef struct df11_gemv {
   uint32_t y_stride;   /* elements between output rows: >= n/cols */
   int32_t accumulate;  /* 0: y = W x (the call clears y first, in stream order);
                           otherwise y += W x */
-  uint32_t pad;
+  uint32_t interleave; /* the tensor's element order: R rows interleaved per 16 columns
+                          (R = 1 or 0: row-major; else a power of two up to 32 that
+                          divides n/cols).  With R rows interleaved the compressed
+                          stream holds, for each block of R rows and each group of 16
+                          columns, the R rows' 16 elements one after another; lanes that
+                          share a column group then share activations, which makes
+                          batches above 1 cheaper (see df11_decode_gemv). */
 } df11_gemv;
 
 /*

@@ -26,7 +26,8 @@ bf16_to_f64                 hand-checked values (1, -2, the smallest subnormal,
                             back exactly
 gemv                        exact rational sums (fractions.Fraction) of tiny
                             products; one-hot activations return the decoded
-                            weight columns exactly
+                            weight columns exactly; an interleaved stream of
+                            a matrix gives the row-major stream's result
 ==========================  ==================================================
 
 No function is left "parity unpinned".
@@ -334,16 +335,31 @@ def bf16_to_f64(words) -> np.ndarray:
         return u.view(np.float32).astype(np.float64)
 
 
-def gemv(bitstream, code_lengths, sign_mantissa, n: int, cols: int, x) -> np.ndarray:
+def gemv(bitstream, code_lengths, sign_mantissa, n: int, cols: int, x,
+         interleave: int = 1) -> np.ndarray:
     """y = W x for the tensor W that the stream decodes to, taken as
-    (n / cols) x cols row-major (a weight applied right after its decode,
+    (n / cols) x cols (a weight applied right after its decode,
     "DFloat11无损压缩技术" (jsqmd.com) §2.2 item 3), and BF16 activations x
-    (batch x cols, or cols).  Float64 throughout: the decoded weights and the
-    activations widen exactly, and the product is one library matmul.
-    Returns float64 of shape (batch, n / cols)."""
+    (batch x cols, or cols).  The stream is row-major, or with `interleave`
+    = R > 1 holds, for each block of R rows and each group of 16 columns,
+    the R rows' 16 elements one after another (the library's option for its
+    fused product); the element of row r, column c is then at
+    ((r // R * (cols // 16) + c // 16) * R + r % R) * 16 + c % 16.
+    Float64 throughout: the decoded weights and the activations widen
+    exactly, and the product is one library matmul.  Returns float64 of
+    shape (batch, n / cols)."""
     if cols <= 0 or n % cols:
         raise ValueError("cols must divide n")
+    rows = n // cols
     w, end, _ = decode(bitstream, code_lengths, sign_mantissa, n)
-    W = bf16_to_f64(w).reshape(n // cols, cols)
+    if interleave > 1:
+        R = interleave
+        if rows % R or cols % 16:
+            raise ValueError("interleave needs rows a multiple of R and cols of 16")
+        r = np.arange(rows)[:, None]
+        c = np.arange(cols)[None, :]
+        pos = ((r // R * (cols // 16) + c // 16) * R + r % R) * 16 + c % 16
+        w = w[pos]
+    W = bf16_to_f64(w).reshape(rows, cols)
     X = bf16_to_f64(np.ascontiguousarray(x)).reshape(-1, cols)
     return X @ W.T

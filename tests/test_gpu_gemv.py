@@ -198,3 +198,43 @@ def test_more_than_one_launch_and_both_modes():
         cols = h.shape[1]
         _check(h, cols, x, y_acc, y0=y0.float().double().numpy())
         _check(h, cols, x, y_clr)
+
+
+@pytest.mark.parametrize("rows,cols,batch,R", [
+    (4096, 4096, 1, 8), (1024, 4096, 4, 8), (512, 12288, 8, 8), (64, 400, 2, 8), (32, 16, 3, 8),
+    (96, 1024, 2, 32), (40, 256, 1, 2)])
+def test_interleaved_rows(rows, cols, batch, R):
+    """Weights compressed with R rows interleaved per 16 columns: the plain
+    decode gives the interleaved order bit for bit, and the fused product
+    is within the fp32 bound of the oracle's product."""
+    w = _weights(rows, cols, 900 + rows + R)
+    h = df11.compress(workloads.as_numpy_u16(w), interleave=R)
+    assert h.interleave == R and h.shape == (rows, cols)
+    d = df11.to_device(h, "cuda")
+    out = df11.decode(d)
+    torch.cuda.synchronize()
+    want = df11.interleave_rows(workloads.as_numpy_u16(w), R)
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    x = _acts(batch, cols, rows + 7)
+    y = torch.empty(batch, rows, dtype=torch.float32, device="cuda")
+    err = df11.new_error_word()
+    df11.decode_gemv([d], [x.cuda().view(torch.bfloat16)], [y], err=err)
+    torch.cuda.synchronize()
+    df11.check_device_error(err)
+    xu = workloads.as_numpy_u16(x)
+    ref = oracle.gemv(h.bitstream, h.code_lengths, h.sign_mantissa, h.n, cols, xu, interleave=R)
+    W = np.abs(oracle.bf16_to_f64(workloads.as_numpy_u16(w))).reshape(rows, cols)
+    g = cols * U32 / (1 - cols * U32)
+    bound = g * (np.abs(oracle.bf16_to_f64(xu)).reshape(batch, cols) @ W.T)
+    got = y.double().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= bound), float(np.abs(got - ref).max())
+
+
+def test_interleaved_build_on_device_matches_host():
+    w = _weights(256, 1024, 77).cuda()
+    dh = df11.to_device(df11.compress(workloads.as_numpy_u16(w.cpu()), interleave=8), "cuda")
+    dd = df11.compress_on_device(w, interleave=8)
+    torch.cuda.synchronize()
+    assert dd.interleave == 8 and dd.shape == (256, 1024)
+    for f in ("bitstream", "gaps", "chunk_counts", "sign_mantissa"):
+        assert torch.equal(getattr(dd, f), getattr(dh, f)), f

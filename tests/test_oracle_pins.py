@@ -489,3 +489,25 @@ def test_gemv_one_hot_activations_return_weight_columns():
         x[j] = 0x3F80  # 1.0
         y = oracle.gemv(f.bitstream, f.code_lengths, f.sign_mantissa, f.n, cols, x)
         assert np.array_equal(y[0], W[:, j])  # column j, row by row: no transpose slip
+
+
+def test_gemv_interleaved_stream_equals_row_major():
+    """The same matrix encoded in the interleaved order (built here by
+    explicit index loops) gives the row-major result exactly."""
+    rng = np.random.default_rng(9)
+    rows, cols, R = 16, 48, 8
+    w = (np.float32(rng.normal(0, 0.05, rows * cols)).view(np.uint32) >> 16).astype(np.uint16)
+    W = w.reshape(rows, cols)
+    inter = np.zeros_like(w)
+    j = 0
+    for rb in range(rows // R):
+        for cg in range(cols // 16):
+            for r in range(R):
+                for k in range(16):
+                    inter[j] = W[rb * R + r, cg * 16 + k]
+                    j += 1
+    x = (np.float32(rng.normal(0, 1, 2 * cols)).view(np.uint32) >> 16).astype(np.uint16)
+    fa, fb = oracle.encode(w, 8, 128), oracle.encode(inter, 8, 128)
+    ya = oracle.gemv(fa.bitstream, fa.code_lengths, fa.sign_mantissa, fa.n, cols, x)
+    yb = oracle.gemv(fb.bitstream, fb.code_lengths, fb.sign_mantissa, fb.n, cols, x, interleave=R)
+    assert np.array_equal(ya, yb)

@@ -119,3 +119,13 @@ def test_loaded_tensors_decode_like_the_originals(tmp_path):
     out, end, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, h.n)
     assert end == h.params.total_bits
     assert np.array_equal(out, w)
+
+
+def test_interleave_survives_a_round_trip(tmp_path):
+    w = np.arange(64 * 32, dtype=np.uint16).reshape(64, 32) % 977
+    h = df11.compress(w, 8, 128, interleave=8)
+    path = str(tmp_path / "i.df11")
+    ser.save(path, {"w": h})
+    back = ser.load(path)["w"]
+    assert back.interleave == 8 and back.shape == (64, 32)
+    assert np.array_equal(back.bitstream, h.bitstream)
