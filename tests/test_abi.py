@@ -135,6 +135,31 @@ def test_device_builder_host_validation():
         df11.compress_on_device(df11.torch.zeros(4, dtype=df11.torch.int16))
 
 
+def test_batched_builder_host_validation():
+    """The batched builder phases reject bad arguments before any CUDA
+    call, and clear the handles they would return."""
+    L = df11.lib()
+    vp = ctypes.c_void_p
+    ptrs = (vp * 2)(FAKE, FAKE)
+    ns = (ctypes.c_uint64 * 2)(100, 200)
+    params = (df11.Params * 2)()
+    lens = (ctypes.c_uint8 * 512)()
+    handles = (vp * 2)(123, 456)
+    lp = ctypes.cast(lens, vp)
+    assert L.df11_gpu_build_begin_batched(ptrs, ns, 0, 24, 256, None, params, lp, handles) == 0
+    assert L.df11_gpu_build_begin_batched(ptrs, ns, -1, 24, 256, None, params, lp, handles) == 7
+    assert L.df11_gpu_build_begin_batched(None, ns, 2, 24, 256, None, params, lp, handles) == 1
+    assert handles[0] is None and handles[1] is None  # cleared on error
+    assert L.df11_gpu_build_begin_batched(ptrs, ns, 2, 6, 256, None, params, lp, handles) == 7
+    bad = (vp * 2)(FAKE, FAKE + 1)
+    assert L.df11_gpu_build_begin_batched(bad, ns, 2, 24, 256, None, params, lp, handles) == 2
+    big = (ctypes.c_uint64 * 2)(100, 1 << 32)
+    assert L.df11_gpu_build_begin_batched(ptrs, big, 2, 24, 256, None, params, lp, handles) == 6
+    assert L.df11_gpu_build_finish_batched(None, 2, ptrs, None, params, None) == 1
+    assert L.df11_gpu_build_finish_batched(handles, 0, ptrs, None, params, None) == 0
+    assert L.df11_gpu_build_finish_batched(handles, -1, ptrs, None, params, None) == 7
+
+
 def test_gemv_host_validation():
     """df11_decode_gemv rejects bad arguments before any CUDA call."""
     L = df11.lib()
