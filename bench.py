@@ -875,11 +875,13 @@ def measure_e2e(args, units, hosts, groups, device, world):
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     ev_in = {i: torch.cuda.Event() for i in idx}
     ev_dec = {i: torch.cuda.Event() for i in idx}
+    # smallest tensor first: the copy out, the slowest stage, starts as early as possible
+    order = sorted(idx, key=lambda i: hosts[i].n)
 
     def step():
         s_in.wait_stream(stream)   # the previous step's decodes are done with the inputs
         stream.wait_stream(s_out)  # and its copies out are done with the outputs
-        for i in idx:
+        for i in order:
             with torch.cuda.stream(s_in):
                 for k, t in pinned[i].items():
                     getattr(staged[i], k).view(torch.uint8).copy_(t, non_blocking=True)
