@@ -87,3 +87,36 @@ def test_builder_rejects_bad_parameters():
     for C, T in [(3, 256), (6, 256), (8, 100), (8, 2048), (0, 256), (32, 256), (68, 256)]:
         with pytest.raises(df11.Df11Error):
             df11.compress(w, C, T)
+
+
+# --- randomised: skewed exponent histograms, every valid chunk size ----------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@st.composite
+def _skewed_words(draw):
+    """BF16 words whose exponents follow a random skewed histogram over a
+    random subset of the 256 values (geometric weights give long codes),
+    with random sign and mantissa bits, in random order."""
+    k = draw(st.integers(1, 40))
+    exps = draw(st.lists(st.integers(0, 255), min_size=k, max_size=k, unique=True))
+    ratio = draw(st.sampled_from([1.0, 1.5, 2.0, 3.0]))
+    n = draw(st.integers(0, 30000))
+    seed = draw(st.integers(0, 2 ** 31 - 1))
+    rng = np.random.default_rng(seed)
+    p = ratio ** -np.arange(k, dtype=np.float64)
+    e = rng.choice(np.array(exps, dtype=np.uint32), size=n, p=p / p.sum())
+    sm = rng.integers(0, 256, size=n, dtype=np.uint32)
+    return (((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)).astype(np.uint16)
+
+
+@settings(max_examples=60, deadline=None)
+@given(_skewed_words(), st.sampled_from([4, 8, 12, 16, 20, 24, 28]),
+       st.sampled_from([128, 256, 512, 1024]))
+def test_random_histograms_every_chunk_size(w, C, T):
+    h = _compare(w, C, T)
+    if h.n:
+        out, end, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, h.n)
+        assert end == h.params.total_bits
+        assert np.array_equal(out, w)
