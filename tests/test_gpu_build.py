@@ -175,3 +175,33 @@ def test_batched_builds_equal_single_builds():
             assert np.array_equal(getattr(d, f).cpu().numpy().view(np.uint8), _host_bytes(h, f)), f
         if h.n:
             _decodes_to(d, w_np)
+
+
+# --- randomised: skewed exponent histograms, every valid chunk size ----------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@st.composite
+def _skewed_words(draw):
+    """BF16 words whose exponents follow a random geometric histogram over a
+    random subset of exponent values, random sign and mantissa bits."""
+    k = draw(st.integers(1, 40))
+    exps = draw(st.lists(st.integers(0, 255), min_size=k, max_size=k, unique=True))
+    ratio = draw(st.sampled_from([1.0, 1.5, 2.0, 3.0]))
+    n = draw(st.integers(0, 60000))
+    rng = np.random.default_rng(draw(st.integers(0, 2 ** 31 - 1)))
+    p = ratio ** -np.arange(k, dtype=np.float64)
+    e = rng.choice(np.array(exps, dtype=np.uint32), size=n, p=p / p.sum())
+    sm = rng.integers(0, 256, size=n, dtype=np.uint32)
+    return (((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)).astype(np.uint16)
+
+
+@settings(max_examples=25, deadline=None)
+@given(_skewed_words(), st.sampled_from([4, 8, 12, 16, 20, 24, 28]),
+       st.sampled_from([128, 256, 512, 1024]))
+def test_random_histograms_device_matches_host(w, C, T):
+    bits = torch.from_numpy(w.view(np.int16)).cuda()
+    d, h, w_np = _same_as_host(bits, C, T)
+    if h.n and df11.supported(C, T):
+        _decodes_to(d, w_np)
