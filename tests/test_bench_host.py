@@ -1,0 +1,87 @@
+"""Host-side pieces of bench.py that need no GPU: the clock summary taken
+from nvidia-smi samples, the DRAM-traffic record keyed on the kernel source,
+and the algorithmic byte count the roofline divides by."""
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import huffman_decode_df11_b200 as df11  # noqa: E402
+
+
+def _sampler(lines):
+    s = bench.ClockSampler(0)
+    s.lines = list(lines)
+    return s
+
+
+def _row(sm, mx=1965, hw="Not Active", hwt="Not Active", swt="Not Active", cap="Not Active"):
+    return f"0, {sm}, {mx}, 700.5, 0x0, {hw}, {hwt}, {swt}, {cap}"
+
+
+def test_clock_summary_median_and_reasons():
+    s = _sampler([_row(1965), _row(1950), _row(1900, cap="Active"), "garbage", "",
+                  "0, [N/A], 1965, 1, 0, a, b, c, d"])
+    out = s.summary()
+    assert out["sm_mhz"] == 1950 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3
+
+
+def test_clock_summary_flags_throttling_and_no_samples():
+    out = _sampler([_row(1500, hw="Active"), _row(1400, hwt="Active", swt="Active")]).summary()
+    assert out["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+    assert out["sm_mhz"] == 1450
+    empty = _sampler([]).summary()
+    assert empty["sm_mhz"] is None and empty["reasons"] == ["unsampled"]
+
+
+def test_traffic_record_follows_the_source_hash(tmp_path, monkeypatch):
+    src = tmp_path / "kernel.cu"
+    src.write_text("__global__ void k() {}\n")
+    h = bench.kernel_hash(str(src))
+    rec = tmp_path / "traffic.txt"
+    rec.write_text("# comment line\n"
+                   f"{h} block/c24/t256 591206912  capture.md\n"
+                   f"{h} build/c24/t256 1444705195\n"
+                   "0123456789abcdef block/c8/t256 1\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
+    assert bench.recorded_traffic("block/c24/t256", str(src)) == 591206912.0
+    assert bench.recorded_traffic("build/c24/t256", str(src)) == 1444705195.0
+    assert bench.recorded_traffic("block/c8/t256", str(src)) is None   # another source
+    assert bench.recorded_traffic("embedding/c24/t256", str(src)) is None
+    src.write_text("__global__ void k() { /* changed */ }\n")
+    assert bench.recorded_traffic("block/c24/t256", str(src)) is None  # stale once changed
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "absent.txt"))
+    assert bench.recorded_traffic("block/c24/t256", str(src)) is None
+
+
+@pytest.mark.parametrize("C,T,n", [(24, 256, 300_001), (8, 128, 70_000), (16, 512, 1)])
+def test_algorithmic_bytes_counts_every_buffer_the_decode_moves(C, T, n):
+    rng = np.random.default_rng(n)
+    w = (rng.normal(0, 0.02, n).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    h = df11.compress(w, C, T)
+    p = h.params
+    chunks = int(p.num_blocks) * T
+    # the stream up to its last bit, one sign/mantissa byte per element, the
+    # packed 5-bit gaps, one count per chunk, the block positions, the
+    # tables, the code lengths, and the BF16 output
+    want_in = (-(-int(p.total_bits) // 8) + n + -(-5 * chunks // 8) + chunks
+               + h.block_out_pos.nbytes + h.luts.nbytes + h.code_lengths.nbytes)
+    assert bench.algorithmic_bytes(h) == want_in + 2 * n
+    assert bench.algorithmic_bytes(h, counts=False) == want_in - chunks + 2 * n
+    # what is stored is the moved input plus paddings only
+    assert 0 <= h.compressed_bytes() - want_in < C * T + 64 + 16
+
+
+def test_measured_peak_reads_the_driver_file_or_falls_back(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6538.2}')
+    assert bench.measured_peak() == (6538.2, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").write_text("not json")
+    assert bench.measured_peak()[1] == "fallback"
