@@ -240,6 +240,48 @@ def barrier(world: int):
         dist.barrier()
 
 
+L2_BYTES = 126 * 2 ** 20  # B200 L2 cache
+FLUSH_BYTES = 2 * L2_BYTES
+
+
+def flush_wanted(mode: str, step_bytes: int) -> bool:
+    """Whether L2 is rewritten before every timed step: always ('on'), never
+    ('off'), or when one step's inputs and outputs fit in L2 ('auto')."""
+    if mode == "on":
+        return True
+    if mode == "off":
+        return False
+    return step_bytes < L2_BYTES
+
+
+def time_steps(step, steps: int, stream, new_event, flush=None) -> float:
+    """Mean device milliseconds of one step over `steps` steps, from events
+    recorded on `stream`.  Without `flush`, one event pair brackets all the
+    steps, so that launches run back to back.  With `flush` (a tensor larger
+    than L2), the tensor is rewritten before each step, which evicts the
+    previous step's data, and each step is timed by its own event pair."""
+    if steps < 1:
+        raise ValueError("time at least one step")
+    if flush is None:
+        a, b = new_event(), new_event()
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / steps
+    pairs = []
+    for s in range(steps):
+        flush.fill_(s + 1)
+        a, b = new_event(), new_event()
+        a.record(stream)
+        step()
+        b.record(stream)
+        pairs.append((a, b))
+    pairs[-1][1].synchronize()
+    return sum(a.elapsed_time(b) for a, b in pairs) / steps
+
+
 def prepare(config: str, seed: int, device: str, chunk_bytes: int = 24,
             threads_per_block: int = 256):
     """Compress every unit on the host; keep compressed tensors resident in
@@ -307,13 +349,15 @@ def run_b200(args, world, rank, local):
         step()
     torch.cuda.synchronize()
     launches_per_step = sum((len(g) + 15) // 16 for g in groups)
+    alg = [sum(algorithmic_bytes(hosts[i], counts) for i in g) for g in groups]
+    flush_used = flush_wanted(args.flush_l2, sum(alg))
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=device) if flush_used else None
     # per-launch events only in a separate pass after the timed region: an
     # event between two launches keeps the second from starting while the
     # first finishes (programmatic dependent launch)
     pg_steps = min(args.steps, 50)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in groups] for _ in range(pg_steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                       else local) as clocks:
         # keep the GPU busy (untimed) while the sampler starts, so that the
@@ -324,17 +368,15 @@ def run_b200(args, world, rank, local):
             torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
-        t0.record(stream)
-        for s in range(args.steps):
-            step()
-        t1.record(stream)
+        ms_local = time_steps(step, args.steps, stream,
+                              lambda: torch.cuda.Event(enable_timing=True), flush)
         torch.cuda.synchronize()
         barrier(world)
         for s in range(pg_steps):
             step(ev[s])
         torch.cuda.synchronize()
     df11.check_device_error(err)
-    ms_local = t0.elapsed_time(t1) / args.steps
+    del flush
     ms = max_over_ranks(ms_local, world)
     out_bytes_all = sum_over_ranks(2.0 * n_total, world)
     value = out_bytes_all / (ms * 1e-3) / 1e9
@@ -345,7 +387,6 @@ def run_b200(args, world, rank, local):
     # kernel runs, launch after launch
     per_group_ms = [statistics.mean(ev[s][gi][0].elapsed_time(ev[s][gi][1])
                                     for s in range(pg_steps)) for gi in range(len(groups))]
-    alg = [sum(algorithmic_bytes(hosts[i], counts) for i in g) for g in groups]
     achieved = sum(alg) / (ms_local * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     # the capture covers the chunk-count kernel; the page-layout kernel has none
@@ -375,8 +416,11 @@ def run_b200(args, world, rank, local):
                 "compressed_bytes": sum(h.compressed_bytes() for h in hosts),
                 "bits_per_weight": round(8.0 * sum(h.compressed_bytes() for h in hosts)
                                          / n_total, 3),
-                "l2": "inputs larger than L2 (no flush)" if sum(alg) > 126e6 else
-                      "inputs smaller than L2: numbers include L2 reuse",
+                "l2": (f"L2 flushed before every step ({FLUSH_BYTES >> 20} MiB written); "
+                       "each step timed alone by its own events") if flush_used else
+                      "inputs larger than L2 (no flush)" if sum(alg) >= L2_BYTES else
+                      "inputs smaller than L2, not flushed: numbers include L2 reuse",
+                "us_per_call": round(1e3 * ms / launches_per_step, 2),
                 "parallelism": f"replicas x{world} (no collective)",
                 "parity": "bit-exact vs original on every tensor before timing",
                 "chunk_counts": not args.no_counts,
@@ -1119,6 +1163,10 @@ def main(argv=None):
                     help="gemv workload: rows interleaved per 16 columns in the fused "
                          "path's compressed weights (1: row-major)")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--flush-l2", default="auto", choices=["auto", "on", "off"],
+                    help="rewrite a buffer twice the size of L2 before every timed decode "
+                         "step (auto: when one step's bytes fit in L2) and time each step "
+                         "alone")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-counts", action="store_true",

@@ -85,3 +85,56 @@ def test_measured_peak_reads_the_driver_file_or_falls_back(tmp_path, monkeypatch
     assert bench.measured_peak() == (6538.2, "measured")
     (tmp_path / "MEASURED_PEAKS.json").write_text("not json")
     assert bench.measured_peak()[1] == "fallback"
+
+
+class _FakeEvent:
+    """A CUDA event stand-in: records the position in a shared log, and its
+    'elapsed time' is the number of step calls between two records."""
+
+    def __init__(self, log):
+        self.log, self.at = log, None
+
+    def record(self, stream):
+        assert stream == "s"
+        self.log.append("rec")
+        self.at = self.log.count("step")
+
+    def synchronize(self):
+        self.log.append("sync")
+
+    def elapsed_time(self, other):
+        return float(other.at - self.at)
+
+
+class _FakeFlush:
+    def __init__(self, log):
+        self.log = log
+
+    def fill_(self, v):
+        self.log.append(f"flush{v}")
+
+
+def test_time_steps_back_to_back():
+    log = []
+    ms = bench.time_steps(lambda: log.append("step"), 4, "s", lambda: _FakeEvent(log))
+    assert ms == 1.0
+    assert log == ["rec", "step", "step", "step", "step", "rec", "sync"]
+
+
+def test_time_steps_flushes_before_every_step_and_times_steps_alone():
+    log = []
+    ms = bench.time_steps(lambda: log.append("step"), 3, "s", lambda: _FakeEvent(log),
+                          flush=_FakeFlush(log))
+    assert ms == 1.0
+    assert log == ["flush1", "rec", "step", "rec", "flush2", "rec", "step", "rec",
+                   "flush3", "rec", "step", "rec", "sync"]
+    with pytest.raises(ValueError):
+        bench.time_steps(lambda: None, 0, "s", lambda: _FakeEvent([]))
+
+
+def test_flush_rule():
+    assert bench.FLUSH_BYTES >= 2 * bench.L2_BYTES
+    assert bench.flush_wanted("auto", 3_500_000)             # 1024x1024: fits in L2
+    assert not bench.flush_wanted("auto", 646_000_000)       # the block: larger than L2
+    assert bench.flush_wanted("on", 646_000_000)
+    assert not bench.flush_wanted("off", 3_500_000)
