@@ -57,6 +57,7 @@ KERNEL_SRC = os.path.join(ROOT, "huffman_decode_df11_b200", "csrc", "df11_decode
 BUILD_SRC = os.path.join(ROOT, "huffman_decode_df11_b200", "csrc", "df11_gpu_build.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, the data-sheet figure
 
 
 # ---------------------------------------------------------------------------
@@ -406,6 +407,7 @@ def run_b200(args, world, rank, local):
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+            "elements_per_s": round(out_bytes_all / 2.0 / (ms * 1e-3), 1),
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u32",
@@ -429,6 +431,8 @@ def run_b200(args, world, rank, local):
                          "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "traffic": traffic, "peak_kind": peak_kind,
+                         "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "nominal_peak": NOMINAL_HBM_GBS,
                          "algorithmic_bytes_per_step": sum(alg)},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),
