@@ -106,6 +106,21 @@ def test_ragged_sizes(n, counts):
 
 
 @COUNTS
+@pytest.mark.parametrize("C", [16, 24])
+def test_ragged_sizes_around_warp_and_block_ranges(C, counts):
+    """Prefixes of one tensor ending one element before, at and after the
+    first block's and the first warp's element counts, at the wider chunks."""
+    base = workloads.as_numpy_u16(workloads.gaussian_bf16(200_000, 0.02, 31))
+    h = df11.compress(base, C, 256)
+    block_n = int(h.block_out_pos[1])
+    warp_n = int(h.chunk_counts[:32].sum())
+    sizes = {1, 33, warp_n - 1, warp_n, warp_n + 1, block_n - 1, block_n, block_n + 1,
+             2 * block_n + 1, 3 * block_n + warp_n}
+    for n in sorted(sizes):
+        _gpu_vs_oracle_full(base[:n], C=C, counts=counts)
+
+
+@COUNTS
 def test_every_bf16_pattern(counts):
     w = workloads.as_numpy_u16(workloads.all_bf16_patterns())
     _gpu_vs_oracle_full(w, counts=counts)
