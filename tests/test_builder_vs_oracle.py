@@ -33,7 +33,8 @@ def _compare(w, C, T, threads=4):
     return h
 
 
-@pytest.mark.parametrize("C,T", [(8, 256), (4, 256), (16, 256), (8, 128), (8, 512)])
+@pytest.mark.parametrize("C,T", [(8, 256), (4, 256), (16, 256), (24, 256), (28, 256),
+                                 (8, 128), (8, 512), (24, 1024)])
 def test_single_matrix(C, T):
     w = workloads.as_numpy_u16(workloads.single_matrix(0))
     _compare(w, C, T)
