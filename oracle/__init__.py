@@ -12,9 +12,11 @@ Functions and what pins them (tests/test_oracle_pins.py, tests/golden/):
 ==========================  ==================================================
 split / histogram           exact BF16 round trip over all 65,536 bit patterns
 huffman_lengths             brute-force optimum on small alphabets; Kraft
-                            equality; entropy bound H <= avg < H + 1
+                            equality; entropy bound H <= avg < H + 1; the
+                            tie order on hand-worked tied histograms
 package_merge_lengths       brute-force optimum of the length-limited problem;
-                            equal total cost to Huffman when the limit is slack
+                            equal total cost to Huffman when the limit is
+                            slack; leaf-first ties on hand-worked cases
 code_lengths                32-bit cap reached exactly on Fibonacci weights
 canonical_codes             RFC 1951 section 3.2.2 worked example; prefix-free
 build_luts                  every entry re-derived by brute-force parsing

@@ -121,3 +121,28 @@ def test_random_histograms_every_chunk_size(w, C, T):
         out, end, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, h.n)
         assert end == h.params.total_bits
         assert np.array_equal(out, w)
+
+
+def _tensor_with_exponent_counts(weights, base=120):
+    """BF16 words whose exponent histogram is `weights` (symbol s -> exponent
+    base + s), sign and mantissa varied, in a fixed shuffled order."""
+    words = []
+    for s, c in sorted((int(k), v) for k, v in weights.items()):
+        words += [((base + s) << 7) | ((7 * i + s) & 0x7F) | ((i & 1) << 15) for i in range(c)]
+    rng = np.random.default_rng(5)
+    return np.array(words, np.uint16)[rng.permutation(len(words))]
+
+
+def test_tie_breaks_match_hand_worked_golden(golden_dir):
+    """The host builder's Huffman tie order on the hand-worked golden cases
+    (tests/golden/huffman_ties.json): code lengths and the bytes of the
+    stream equal the golden's and the oracle's."""
+    import json
+    import os
+    fx = json.load(open(os.path.join(golden_dir, "huffman_ties.json")))
+    for case in fx["huffman"]:
+        w = _tensor_with_exponent_counts(case["weights"])
+        h = _compare(w, 8, 256)
+        for s, l in case["lengths"].items():
+            assert int(h.code_lengths[120 + int(s)]) == l, case["weights"]
+        assert int((h.code_lengths > 0).sum()) == len(case["lengths"])

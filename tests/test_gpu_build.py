@@ -205,3 +205,23 @@ def test_random_histograms_device_matches_host(w, C, T):
     d, h, w_np = _same_as_host(bits, C, T)
     if h.n and df11.supported(C, T):
         _decodes_to(d, w_np)
+
+
+def test_tie_breaks_match_hand_worked_golden(golden_dir):
+    """The device builder's code on the hand-worked tie cases
+    (tests/golden/huffman_ties.json): the golden's lengths, and the host
+    builder's bytes."""
+    import json
+    import os
+    fx = json.load(open(os.path.join(golden_dir, "huffman_ties.json")))
+    rng = np.random.default_rng(5)
+    for case in fx["huffman"]:
+        words = []
+        for s, c in sorted((int(k), v) for k, v in case["weights"].items()):
+            words += [((120 + s) << 7) | ((7 * i + s) & 0x7F) for i in range(c)]
+        w = np.array(words, np.uint16)[rng.permutation(len(words))]
+        d, h, w_np = _same_as_host(torch.from_numpy(w.view(np.int16)).cuda())
+        lens = d.code_lengths.cpu().numpy()
+        for s, l in case["lengths"].items():
+            assert int(lens[120 + int(s)]) == l, case["weights"]
+        _decodes_to(d, w_np)

@@ -192,6 +192,89 @@ def test_canonical_codes_are_prefix_free(workload_hists):
 
 
 # -------------------------------------------------------------------------
+# Tie-breaks of the code construction (hand-worked cases, tests/golden/
+# huffman_ties.json).  The pages are silent on ties; the format fixes them,
+# so that the encoded bytes are unique.
+
+def _ties(golden_dir):
+    return json.load(open(os.path.join(golden_dir, "huffman_ties.json")))
+
+
+def _hist_of(weights):
+    h = np.zeros(256, np.uint64)
+    for s, w in weights.items():
+        h[int(s)] = w
+    return h
+
+
+def test_huffman_ties_match_hand_worked_golden(golden_dir):
+    for case in _ties(golden_dir)["huffman"]:
+        h = _hist_of(case["weights"])
+        lens, longest = oracle.huffman_lengths(h)
+        want = {int(s): l for s, l in case["lengths"].items()}
+        assert {s: int(lens[s]) for s in want} == want, case["weights"]
+        assert int(lens.sum()) == sum(want.values())  # no other symbol coded
+        assert longest == max(want.values())
+        assert sum(int(h[s]) * l for s, l in want.items()) == case["cost_bits"]
+        # below the 32-bit cap the full construction is plain Huffman
+        full, _ = oracle.code_lengths(h)
+        assert np.array_equal(full, lens)
+        codes = oracle.canonical_codes(lens)
+        for s, bits in case["canonical"].items():
+            assert format(int(codes[int(s)]), f"0{want[int(s)]}b") == bits
+
+
+def test_package_merge_ties_match_hand_worked_golden(golden_dir):
+    for case in _ties(golden_dir)["package_merge"]:
+        h = _hist_of(case["weights"])
+        lens, longest = oracle.package_merge_lengths(h, case["max_len"])
+        want = {int(s): l for s, l in case["lengths"].items()}
+        assert {s: int(lens[s]) for s in want} == want, case["weights"]
+        assert int(lens.sum()) == sum(want.values())
+        assert sum(int(h[s]) * l for s, l in want.items()) == case["cost_bits"]
+
+
+def _huffman_by_rule(weights, key):
+    """Textbook Huffman in plain Python with a pluggable tie order (node =
+    (weight, smallest symbol, creation index, symbols)); only used to show
+    that the golden cases tell tie rules apart."""
+    nodes = [(w, s, i, [s]) for i, (s, w) in enumerate(sorted(weights.items()))]
+    depth = {s: 0 for s in weights}
+    made = len(nodes)
+    while len(nodes) > 1:
+        nodes.sort(key=key)
+        a, b = nodes[0], nodes[1]
+        for s in a[3] + b[3]:
+            depth[s] += 1
+        nodes = nodes[2:] + [(a[0] + b[0], min(a[1], b[1]), made, a[3] + b[3])]
+        made += 1
+    return depth
+
+
+def test_golden_ties_tell_tie_rules_apart(golden_dir):
+    """Each other plausible tie order fails at least one golden case, so a
+    swapped order in the oracle (or a builder) cannot pass the pins."""
+    cases = _ties(golden_dir)["huffman"]
+    rules = {"larger smallest-symbol first": lambda n: (n[0], -n[1]),
+             "newest node first": lambda n: (n[0], -n[2]),
+             "oldest node first": lambda n: (n[0], n[2])}
+    for name, key in rules.items():
+        differs = False
+        for case in cases:
+            w = {int(s): v for s, v in case["weights"].items()}
+            want = {int(s): l for s, l in case["lengths"].items()}
+            got = _huffman_by_rule(w, key)
+            assert sum(w[s] * got[s] for s in w) == case["cost_bits"]  # still optimal
+            differs |= got != want
+        assert differs, name
+    # the stated rule itself reproduces every case
+    for case in cases:
+        w = {int(s): v for s, v in case["weights"].items()}
+        assert _huffman_by_rule(w, lambda n: (n[0], n[1])) == \
+            {int(s): l for s, l in case["lengths"].items()}
+
+
+# -------------------------------------------------------------------------
 # Hand-written bitstreams
 
 def _golden_streams(golden_dir):
