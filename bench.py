@@ -6,11 +6,12 @@
 
 A step is one pass of the whole decode path over one workload: every tensor
 of it decoded from its resident compressed form into BF16 in HBM (one
-batched launch per 16 tensors).  The default workload is one Qwen3-8B-shaped
-transformer block (7 weights, 192,937,984 elements, one codebook each).
-Other workloads: single (1024x1024), adversarial (64M mix), fibonacci
-(32-bit codewords), embedding (151936x4096), stack (36 blocks + embedding +
-LM head, decoded block by block into one reused scratch buffer).
+batched launch per 16 tensors).  The default workload is the 36-layer
+Qwen3-8B-shaped stack (embedding, 36 blocks of 7 weights, LM head:
+8,190,427,136 elements, one codebook per tensor), decoded layer by layer
+into one reused scratch buffer on one stream.  Other workloads: single
+(1024x1024), block (one Qwen3-8B-shaped block), adversarial (64M mix),
+fibonacci (32-bit codewords), embedding (151936x4096).
 
 Inputs are seeded synthetic tensors; every step's output is checked
 bit-exact against the original tensor before any number is printed.
@@ -99,6 +100,16 @@ def block_groups(config: str, names):
         cur.append(i)
     groups.append(cur)
     return groups
+
+
+def workload_elements(config: str) -> int:
+    """Elements of a workload, from its shapes (no tensor is generated)."""
+    block = sum(r * c for _, r, c in workloads.BLOCK_SHAPES)
+    emb = workloads.VOCAB * workloads.HIDDEN
+    return {"single": 1 << 20, "block": block, "build": block, "gemv": block,
+            "adversarial": 64 << 20, "fibonacci": 14_930_351, "embedding": emb,
+            "stack": 2 * emb + workloads.LAYERS * block,
+            "offload": OFFLOAD_LAYERS * block}[config]
 
 
 def algorithmic_bytes(h, counts: bool = True) -> int:
@@ -284,39 +295,68 @@ def time_steps(step, steps: int, stream, new_event, flush=None) -> float:
 
 
 def prepare(config: str, seed: int, device: str, chunk_bytes: int = 24,
-            threads_per_block: int = 256):
-    """Compress every unit on the host; keep compressed tensors resident in
-    HBM.  Originals are regenerated from the seed when checked."""
+            threads_per_block: int = 256, host_build: bool = False):
+    """Compress every unit and keep the compressed tensors resident in HBM.
+    By default one decode group (a layer) at a time on the device
+    (compress_on_device_batched, byte-identical to the host builder);
+    host_build=True runs the host builder instead.  Originals are
+    regenerated from the seed when checked."""
     import huffman_decode_df11_b200 as df11
     units = workload_units(config, seed)
-    hosts, devs = [], []
-    for name, thunk in units:
-        bits = thunk(device)
-        h = df11.compress(bits, chunk_bytes=chunk_bytes, threads_per_block=threads_per_block)
-        hosts.append(h)
-        devs.append(df11.to_device(h, device))
-        del bits
-    return units, hosts, devs
+    groups = block_groups(config, [u[0] for u in units])
+    devs = [None] * len(units)
+    for g in groups:
+        if host_build:
+            for i in g:
+                h = df11.compress(units[i][1](device), chunk_bytes=chunk_bytes,
+                                  threads_per_block=threads_per_block)
+                devs[i] = df11.to_device(h, device)
+            continue
+        ws = [units[i][1](device) for i in g]
+        for i, d in zip(g, df11.compress_on_device_batched(ws, chunk_bytes, threads_per_block)):
+            devs[i] = d
+        del ws
+    torch.cuda.synchronize()
+    return units, groups, devs
+
+
+class LazyHosts:
+    """Host copies of device-resident compressed tensors, made on first use
+    (the CPU baseline and the end-to-end leg touch only a few of them)."""
+
+    def __init__(self, devs):
+        self._devs, self._cache = devs, {}
+
+    def __len__(self):
+        return len(self._devs)
+
+    def __getitem__(self, i):
+        if i not in self._cache:
+            import huffman_decode_df11_b200 as df11
+            self._cache[i] = df11.to_host(self._devs[i])
+        return self._cache[i]
+
+    def __iter__(self):
+        return (self[i] for i in range(len(self)))
 
 
 def run_b200(args, world, rank, local):
     import huffman_decode_df11_b200 as df11
     device = f"cuda:{local}"
     seed = args.seed + rank
-    units, hosts, devs = prepare(args.config, seed, device, args.chunk_bytes,
-                                 args.threads_per_block)
+    units, groups, devs = prepare(args.config, seed, device, args.chunk_bytes,
+                                  args.threads_per_block, args.host_build)
     names = [u[0] for u in units]
-    groups = block_groups(args.config, names)
-    n_total = sum(h.n for h in hosts)
+    n_total = sum(d.n for d in devs)
     # one reused scratch buffer sized for the largest group
-    group_elems = [sum(hosts[i].n for i in g) for g in groups]
+    group_elems = [sum(devs[i].n for i in g) for g in groups]
     scratch = torch.empty(max(group_elems), dtype=torch.bfloat16, device=device)
     outs_for = []
     for g in groups:
         off, outs = 0, []
         for i in g:
-            outs.append(scratch[off:off + hosts[i].n])
-            off += hosts[i].n
+            outs.append(scratch[off:off + devs[i].n])
+            off += devs[i].n
         outs_for.append(outs)
     err = df11.new_error_word(device)
     stream = torch.cuda.current_stream()
@@ -334,6 +374,25 @@ def run_b200(args, world, rank, local):
             if events is not None:
                 events[gi][1].record(stream)
 
+    # the decode-before-use pattern: after each layer's decode a small
+    # kernel that is not a decode reads the decoded weights (a sum over a
+    # slice of every tensor), so that no decode launch follows another
+    probe = torch.zeros(len(groups), dtype=torch.float32, device=device)
+    heads = [[o[: min(o.numel(), 1 << 16)] for o in outs] for outs in outs_for]
+
+    def consume(gi):
+        for h in heads[gi]:
+            probe[gi] += h.float().sum()
+
+    def step_consumed():
+        for gi, plan in enumerate(plans):
+            plan.run(err=err, stream=stream)
+            consume(gi)
+
+    def consumers_only():
+        for gi in range(len(plans)):
+            consume(gi)
+
     # parity: every group's output equals the original, bit for bit
     for gi, g in enumerate(groups):
         df11.decode_batched([devs[i] for i in g], outs_for[gi], err=err, stream=stream,
@@ -350,7 +409,7 @@ def run_b200(args, world, rank, local):
         step()
     torch.cuda.synchronize()
     launches_per_step = sum((len(g) + 15) // 16 for g in groups)
-    alg = [sum(algorithmic_bytes(hosts[i], counts) for i in g) for g in groups]
+    alg = [sum(algorithmic_bytes(devs[i], counts) for i in g) for g in groups]
     flush_used = flush_wanted(args.flush_l2, sum(alg))
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=device) if flush_used else None
     # per-launch events only in a separate pass after the timed region: an
@@ -359,6 +418,8 @@ def run_b200(args, world, rank, local):
     pg_steps = min(args.steps, 50)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in groups] for _ in range(pg_steps)]
+    cons_steps = max(3, min(args.steps, 50))
+    new_ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                       else local) as clocks:
         # keep the GPU busy (untimed) while the sampler starts, so that the
@@ -369,13 +430,19 @@ def run_b200(args, world, rank, local):
             torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
-        ms_local = time_steps(step, args.steps, stream,
-                              lambda: torch.cuda.Event(enable_timing=True), flush)
+        ms_local = time_steps(step, args.steps, stream, new_ev, flush)
         torch.cuda.synchronize()
         barrier(world)
         for s in range(pg_steps):
             step(ev[s])
         torch.cuda.synchronize()
+        if not flush_used:
+            step_consumed()
+            consumers_only()
+            torch.cuda.synchronize()
+            cons_ms = time_steps(step_consumed, cons_steps, stream, new_ev)
+            only_ms = time_steps(consumers_only, cons_steps, stream, new_ev)
+            torch.cuda.synchronize()
     df11.check_device_error(err)
     del flush
     ms = max_over_ranks(ms_local, world)
@@ -389,22 +456,37 @@ def run_b200(args, world, rank, local):
     per_group_ms = [statistics.mean(ev[s][gi][0].elapsed_time(ev[s][gi][1])
                                     for s in range(pg_steps)) for gi in range(len(groups))]
     achieved = sum(alg) / (ms_local * 1e-3) / 1e9
+    # each launch alone: no overlap with the launch before it
+    achieved_call = sum(alg) / (sum(per_group_ms) * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     # the capture covers the chunk-count kernel; the page-layout kernel has none
     traffic = (recorded_traffic(f"{args.config}/c{args.chunk_bytes}/t{args.threads_per_block}")
                if counts else None)
+    consumer = None
+    if not flush_used:
+        dec_ms = cons_ms - only_ms
+        consumer = {
+            "ms_per_step": round(cons_ms, 4), "consumers_only_ms": round(only_ms, 4),
+            "decode_ms": round(dec_ms, 4),
+            "frac": round(sum(alg) / (dec_ms * 1e-3) / 1e9 / peak, 4),
+            "what": "each layer's decode followed by a non-decode kernel reading its output "
+                    "(a sum over the first 64K elements of every tensor); decode_ms = "
+                    "ms_per_step - consumers_only_ms"}
 
+    hosts = LazyHosts(devs)
     # end to end through the public API: host (pinned) compressed tensors in,
     # host BF16 out, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(args, units, hosts, groups, device, world)
+        e2e = measure_e2e(args, units, hosts, groups, device, world,
+                          ns=[d.n for d in devs])
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(hosts, args.cpu_budget_s)
 
     if rank == 0:
+        compressed = sum(d.compressed_bytes() for d in devs)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT,
             "elements_per_s": round(out_bytes_all / 2.0 / (ms * 1e-3), 1),
@@ -414,10 +496,11 @@ def run_b200(args, world, rank, local):
             "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
             "config": {
                 "workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
-                "elements": n_total, "chunk_bytes": args.chunk_bytes, "threads_per_block": args.threads_per_block,
-                "compressed_bytes": sum(h.compressed_bytes() for h in hosts),
-                "bits_per_weight": round(8.0 * sum(h.compressed_bytes() for h in hosts)
-                                         / n_total, 3),
+                "elements": n_total, "chunk_bytes": args.chunk_bytes,
+                "threads_per_block": args.threads_per_block,
+                "compressed_bytes": compressed,
+                "bits_per_weight": round(8.0 * compressed / n_total, 3),
+                "builder": "host" if args.host_build else "device (byte-identical to host)",
                 "l2": (f"L2 flushed before every step ({FLUSH_BYTES >> 20} MiB written); "
                        "each step timed alone by its own events") if flush_used else
                       "inputs larger than L2 (no flush)" if sum(alg) >= L2_BYTES else
@@ -430,10 +513,17 @@ def run_b200(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
+                         "frac_what": "decode launches back to back; consecutive launches "
+                                      "overlap by programmatic dependent launch",
+                         "achieved_per_call": round(achieved_call, 1),
+                         "frac_per_call": round(achieved_call / peak, 4),
+                         "frac_per_call_what": "each launch timed alone by events on its "
+                                               "stream (no overlap with a neighbour)",
                          "traffic": traffic, "peak_kind": peak_kind,
                          "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                          "nominal_peak": NOMINAL_HBM_GBS,
                          "algorithmic_bytes_per_step": sum(alg)},
+            "decode_then_consumer": consumer,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),
             "e2e": e2e,
@@ -441,7 +531,12 @@ def run_b200(args, world, rank, local):
             "per_group_ms": [round(x, 4) for x in per_group_ms]
             if len(groups) <= 8 else {"min": round(min(per_group_ms), 4),
                                       "max": round(max(per_group_ms), 4),
-                                      "groups": len(groups)},
+                                      "mean": round(statistics.mean(per_group_ms), 4),
+                                      "sum": round(sum(per_group_ms), 4),
+                                      "groups": len(groups),
+                                      "names": [names[g[0]].split(".")[0] if len(g) == 1
+                                                else ".".join(names[g[0]].split(".")[:2])
+                                                for g in (groups[0], groups[-1])]},
         }
         print(json.dumps(line), flush=True)
 
@@ -889,15 +984,16 @@ def cpu_build_baseline(ws, budget_s: float):
             "kind": "oracle", "sample": what + " (single-threaded C encoder)"}
 
 
-def measure_e2e(args, units, hosts, groups, device, world):
+def measure_e2e(args, units, hosts, groups, device, world, ns=None):
     import huffman_decode_df11_b200 as df11
     # bounded host memory: the first groups up to ~2G elements
     keep, elems = [], 0
     for g in groups:
-        if keep and elems + sum(hosts[i].n for i in g) > 2_000_000_000:
+        g_n = sum(ns[i] if ns is not None else hosts[i].n for i in g)
+        if keep and elems + g_n > 2_000_000_000:
             break
         keep.append(g)
-        elems += sum(hosts[i].n for i in g)
+        elems += g_n
     sampled = len(keep) < len(groups)
     groups = keep
     idx = [i for g in groups for i in g]
@@ -1000,8 +1096,35 @@ def cpu_baseline(hosts, budget_s: float):
             "kind": "oracle", "sample": what + " (single-threaded bit-serial C decode)"}
 
 
+def _oracle_prefix_formats(units, elements: int, chunk_bytes: int, threads_per_block: int):
+    """The workload's tensors generated on the host and their leading
+    elements (up to `elements` in all, in order) encoded by the oracle's own
+    encoder: the bounded sample the reference arm decodes.  No library of
+    the GPU path is loaded.  Returns (formats, description).  `units` may
+    also give a row length per tensor, (name, thunk, cols), to encode whole
+    rows only."""
+    import oracle
+    fmts, left, names = [], elements, []
+    for unit in units:
+        name, thunk = unit[0], unit[1]
+        if left <= 0:
+            break
+        w = thunk("cpu")
+        take = int(min(w.numel(), left))
+        if len(unit) > 2:  # whole rows
+            take = min(w.numel(), -(-take // unit[2]) * unit[2])
+        fmts.append(oracle.encode(workloads.as_numpy_u16(w.reshape(-1)[:take]),
+                                  chunk_bytes, threads_per_block))
+        names.append(f"{name}[:{take}]")
+        left -= take
+        del w
+    return fmts, f"oracle-encoded leading elements of {', '.join(names)}"
+
+
 def run_reference(args, world, rank):
-    """The comparison arm: the CPU oracle, as it stands, on the host cores."""
+    """The comparison arm: the CPU oracle, as it stands, on the host cores.
+    Its input is encoded by the oracle itself, so this process loads no
+    library of the GPU path."""
     if rank != 0:
         return
     units = workload_units(args.config, args.seed)
@@ -1009,11 +1132,16 @@ def run_reference(args, world, rank):
         return run_reference_build(args, world, units)
     if args.config == "gemv":
         return run_reference_gemv(args, world, units)
-    import huffman_decode_df11_b200 as df11
-    hosts = [df11.compress(thunk("cpu"), chunk_bytes=args.chunk_bytes,
-                           threads_per_block=args.threads_per_block) for _, thunk in units]
-    n_total = sum(h.n for h in hosts)
+    n_total = workload_elements(args.config)
     budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
+    # a step decodes as many leading elements as fit its share of the budget
+    # (the bit-serial decoder runs at roughly 10 ns per element)
+    # the stack's sample is taken from its first layers (94% of its elements
+    # are in the 36 blocks), not from the 622M-element embedding, whose
+    # generation on the host would take longer than the sample itself
+    sample_units = units[1:-1] + [units[0], units[-1]] if args.config == "stack" else units
+    hosts, encoded = _oracle_prefix_formats(sample_units, int(budget / 8e-9) + 1,
+                                            args.chunk_bytes, args.threads_per_block)
     for _ in range(args.warmup):
         _oracle_sample(hosts, budget)
     tot_done, tot_s, what = 0, 0.0, ""
@@ -1030,9 +1158,10 @@ def run_reference(args, world, rank):
         "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
         "config": {"workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
                    "elements": n_total, "chunk_bytes": args.chunk_bytes, "threads_per_block": args.threads_per_block,
-                   "step": f"bounded sample of the workload, ~{budget:.1f} s of CPU work"},
+                   "step": f"bounded sample of the workload, ~{budget:.3f} s of CPU work"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": what + " per step (single-threaded bit-serial C decode)"},
+                         "sample": what + " per step (single-threaded bit-serial C decode); "
+                                   "input: " + encoded},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -1049,7 +1178,7 @@ def _oracle_gemv_sample(hosts, shapes, x_rows, budget_s: float):
     for h, (r, c), x in zip(hosts, shapes, x_rows):
         if t_used >= budget_s:
             break
-        rows = int(min(r, max(1, (budget_s - t_used) / 20e-9 / c)))
+        rows = int(min(r, h.n // c, max(1, (budget_s - t_used) / 20e-9 / c)))
         t = time.perf_counter()
         w, _, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, rows * c)
         W = oracle.bf16_to_f64(w).reshape(rows, c)
@@ -1063,14 +1192,18 @@ def _oracle_gemv_sample(hosts, shapes, x_rows, budget_s: float):
 def run_reference_gemv(args, world, units):
     """The comparison arm for the fused product: the oracle's decode and
     float64 product, as they stand, on bounded samples of the workload."""
-    import huffman_decode_df11_b200 as df11
     shapes = [(r, c) for _, r, c in workloads.BLOCK_SHAPES]
-    hosts = [df11.compress(thunk("cpu"), chunk_bytes=args.chunk_bytes,
-                           threads_per_block=args.threads_per_block) for _, thunk in units]
+    budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
+    # leading rows of the weights, encoded by the oracle itself (this process
+    # loads no library of the GPU path); the product runs at roughly 20 ns per
+    # weight
+    hosts, encoded = _oracle_prefix_formats(
+        [(n, t, c) for (n, t), (_, c) in zip(units, shapes)], int(budget / 15e-9) + 1,
+        args.chunk_bytes, args.threads_per_block)
+    shapes = shapes[: len(hosts)]
     xs = [workloads.as_numpy_u16(workloads.gaussian_bf16(args.batch * c, 1.0, 77 + i))
           for i, (_, c) in enumerate(shapes)]
-    n_total = sum(h.n for h in hosts)
-    budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
+    n_total = workload_elements(args.config)
     for _ in range(args.warmup):
         _oracle_gemv_sample(hosts, shapes, xs, budget)
     tot_done, tot_s, what = 0, 0.0, ""
@@ -1090,7 +1223,8 @@ def run_reference_gemv(args, world, units):
                    "threads_per_block": args.threads_per_block,
                    "step": f"bounded sample of the workload, ~{budget:.1f} s of CPU work"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": what + " per step (bit-serial C decode, float64 product)"},
+                         "sample": what + " per step (bit-serial C decode, float64 product); "
+                                   "input: " + encoded},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -1149,12 +1283,17 @@ WORKLOAD_NAMES = {
 }
 
 
+DEFAULT_STEPS = {"stack": 200, "build": 20, "gemv": 200, "offload": 40}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 200 for the stack, 2000 for one tensor "
+                         "or block, 20 for build, 200 for gemv, 40 for offload)")
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="block", choices=sorted(WORKLOAD_NAMES))
+    ap.add_argument("--config", default="stack", choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--chunk-bytes", type=int, default=24, choices=[4, 8, 16, 24],
@@ -1178,7 +1317,12 @@ def main(argv=None):
     ap.add_argument("--no-clock-window", action="store_true",
                     help="skip the busy untimed loop before the timed region "
                          "(for profiler runs)")
+    ap.add_argument("--host-build", action="store_true",
+                    help="compress the workload with the host builder instead of the "
+                         "device builder (same bytes)")
     args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS.get(args.config, 2000)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = setup_dist()

@@ -152,6 +152,8 @@ def lib():
     L.df11_decode_gemv.restype = ctypes.c_int
     L.df11_exponent_histogram.argtypes = [vp, u64, vp, vp]
     L.df11_exponent_histogram.restype = ctypes.c_int
+    L.df11_test_withhold_copies.argtypes = [ctypes.c_int, u32]
+    L.df11_test_withhold_copies.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -343,6 +345,23 @@ def to_device(h: Df11Host, device="cuda", decode_table: bool = True) -> Df11Devi
     if decode_table:
         d.decode_table = build_decode_table(d)
     return d
+
+
+def to_host(d: Df11Device) -> Df11Host:
+    """Copy a compressed tensor from device memory back into host arrays
+    (the inverse of to_device; e.g. to save a tensor built on the device).
+    Synchronises with the copies."""
+    def arr(t, dtype):
+        return t.cpu().numpy().view(dtype).copy()
+    cc = d.chunk_counts
+    return Df11Host(params=Params.from_buffer_copy(d.params),
+                    code_lengths=arr(d.code_lengths, np.uint8),
+                    bitstream=arr(d.bitstream, np.uint8), gaps=arr(d.gaps, np.uint8),
+                    block_out_pos=arr(d.block_out_pos, np.uint32),
+                    luts=arr(d.luts, np.uint32),
+                    sign_mantissa=arr(d.sign_mantissa, np.uint8),
+                    chunk_counts=arr(cc, np.uint8) if cc is not None else np.zeros(0, np.uint8),
+                    shape=d.shape, interleave=int(getattr(d, "interleave", 1)))
 
 
 class GpuBuildOut(ctypes.Structure):

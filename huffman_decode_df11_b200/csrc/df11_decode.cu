@@ -102,6 +102,9 @@ struct KBatch {
   uint32_t sub_words;    // deeper-table words kept in shared memory (0: global)
   uint32_t sm_bytes;     // sign/mantissa bytes per stage slot (warp-specialised kernel;
                          // 0: read from global memory)
+  uint32_t spin_limit;   // polls of every bounded wait (kSpinLimit unless a test lowers it)
+  uint32_t withhold;     // test hook: the producer issues no stage copy, so the
+                         // consumers' waits run out (df11_test_withhold_copies)
 };
 
 // ---- shared memory layout --------------------------------------------------
@@ -217,9 +220,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
       : "memory");
 }
 
-// Bounded wait for phase `parity` of an mbarrier; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+// Bounded wait for phase `parity` of an mbarrier: at most `limit` polls,
+// each suspending for up to about a microsecond; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n"
@@ -612,7 +617,7 @@ __global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_c
     }
     if (tid == 0 && b + ctas >= tk.num_blocks) pdl_launch_dependents();  // last block
     int bad = 0;
-    if (!mbar_wait(s ? bar1 : bar0, (k >> 1) & 1)) bad = DF11_DEV_ERR_TIMEOUT;
+    if (!mbar_wait(s ? bar1 : bar0, (k >> 1) & 1, kb.spin_limit)) bad = DF11_DEV_ERR_TIMEOUT;
     const uint4 m = meta[s];
     const uint32_t P0 = m.x, P1 = m.y, expected = P1 - P0;
     if (!m.z) {
@@ -1044,16 +1049,17 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
       mbar_arrive_expect_tx(tbar, DF11_DECODE_TABLE_BYTES);
       bulk_g2s(smem_addr(lens_s), tk.decode_table, DF11_DECODE_TABLE_BYTES, tbar);
     }
-    for (uint32_t b = first; b < tk.num_blocks && issued < kWsStages; b += ctas, ++issued)
-      ws_issue<T, C, SM>(tk, b, stages + issued * slot_bytes, smem_addr(&bars[issued]),
-                         kb.sm_bytes);
+    if (!kb.withhold)
+      for (uint32_t b = first; b < tk.num_blocks && issued < kWsStages; b += ctas, ++issued)
+        ws_issue<T, C, SM>(tk, b, stages + issued * slot_bytes, smem_addr(&bars[issued]),
+                           kb.sm_bytes);
   }
   const uint32_t *sub = tk.luts + 256;  // deeper tables: global memory
   for (uint32_t i = tid; i < CONSUMERS * kb.stage_bytes / 16; i += T + 32)
     reinterpret_cast<uint4 *>(regions)[i] = make_uint4(0, 0, 0, 0);
   bool tables_ok = true;
   if (have_table) {
-    tables_ok = mbar_wait(tbar, 0);
+    tables_ok = mbar_wait(tbar, 0, kb.spin_limit);
   } else {
     load_tables(tid, T + 32, tk.luts, tk.code_lengths, lut0_s, lens_s);
     __syncthreads();
@@ -1067,15 +1073,23 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
   if (warp == CONSUMERS) {  // producer
     if (lane == 0) {
       uint32_t k = issued;
-      for (uint32_t b = first + issued * ctas; b < tk.num_blocks; b += ctas, ++k) {
-        const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
-        if (!mbar_wait(smem_addr(&bars[kWsStages + s]), par ^ 1u)) {
-          report(kb.err, DF11_DEV_ERR_TIMEOUT);
-          break;
+      if (!kb.withhold) {
+        for (uint32_t b = first + issued * ctas; b < tk.num_blocks; b += ctas, ++k) {
+          const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
+          if (!mbar_wait(smem_addr(&bars[kWsStages + s]), par ^ 1u, kb.spin_limit)) {
+            report(kb.err, DF11_DEV_ERR_TIMEOUT);
+            break;
+          }
+          ws_issue<T, C, SM>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
         }
-        ws_issue<T, C, SM>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
       }
       pdl_launch_dependents();  // every block of this thread block is queued
+      // Stay until the last copy into each slot has landed, so that no copy
+      // is in flight into this thread block's shared memory when it exits,
+      // even when consumers gave up waiting (bounded as well).
+      for (uint32_t j = k > kWsStages ? k - kWsStages : 0; j < k; ++j)
+        if (!mbar_wait(smem_addr(&bars[j % kWsStages]), (j / kWsStages) & 1u, kb.spin_limit))
+          report(kb.err, DF11_DEV_ERR_TIMEOUT);
     }
     return;
   }
@@ -1091,7 +1105,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
   for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
     const uint32_t s = k % kWsStages, par = (k / kWsStages) & 1u;
     const uint8_t *slot = stages + s * slot_bytes;
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_addr(&bars[s]), par))) {
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_addr(&bars[s]), par, kb.spin_limit))) {
       if (lane == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
       return;  // whole warp
     }
@@ -1190,7 +1204,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
     }
     if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
     if (SM == kSmWarp && wsm_bytes) {
-      const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(wbar, wph & 1u));
+      const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(wbar, wph & 1u, kb.spin_limit));
       ++wph;
       if (!landed) {
         if (lane == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
@@ -1543,10 +1557,20 @@ size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t regio
          (size_t)sub_words * 4;
 }
 
+// Test hook (df11_test_withhold_copies): launches left to make with the
+// producer issuing no copies, and the wait limit they use.
+std::atomic<int> g_withhold_launches{0};
+std::atomic<uint32_t> g_withhold_spin_limit{kSpinLimit};
+
 df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaStream_t s,
                          bool ws, const df11_gemv *ops = nullptr) {
   KBatch kb{};
   kb.err = d_err;
+  kb.spin_limit = kSpinLimit;
+  if (ws && g_withhold_launches.load() > 0 && g_withhold_launches.fetch_sub(1) > 0) {
+    kb.withhold = 1;
+    kb.spin_limit = g_withhold_spin_limit.load();
+  }
   uint32_t blocks[DF11_MAX_BATCH];
   uint32_t max_elems = 0, max_chunk = 0, max_warp = 0, max_luts = 1, C = 0, T = 0;
   for (int i = 0; i < count; ++i) {
@@ -1764,6 +1788,13 @@ df11_status df11_build_decode_table(const uint32_t *luts, const uint8_t *code_le
   df11_table_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(luts, code_lengths, num_luts,
                                                            reinterpret_cast<uint4 *>(out));
   return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+df11_status df11_test_withhold_copies(int launches, uint32_t spin_limit) {
+  if (launches < 0 || spin_limit < 1 || spin_limit > kSpinLimit) return DF11_ERR_INVALID;
+  g_withhold_spin_limit.store(spin_limit);
+  g_withhold_launches.store(launches);
+  return DF11_OK;
 }
 
 size_t df11_shared_bytes(const df11_params *p) {

@@ -241,6 +241,19 @@ int df11_supported(uint32_t chunk_bytes, uint32_t threads_per_block);
 const char *df11_status_string(df11_status status);
 const char *df11_device_error_string(int32_t code);
 
+/* Testing hook for the decode's failure detection (no counterpart in the
+ * pages).  Every wait of the decode kernels is bounded: a thread block that
+ * has waited too long for its own copies reports DF11_DEV_ERR_TIMEOUT in
+ * d_err and stops, and the context stays usable.  After this call, the next
+ * `launches` decode launches of tensors with chunk counts are made with the
+ * producer issuing no stage copy, so that the consumers' waits run out after
+ * `spin_limit` polls (each suspends for up to about a microsecond; 1 ..
+ * 2^20, the default bound).  No copy is then in flight and nothing faults:
+ * the failure is a withheld message, injected from the host.  Returns
+ * DF11_ERR_INVALID for arguments out of range.  Process-wide; not for use
+ * alongside real decodes in other threads. */
+df11_status df11_test_withhold_copies(int launches, uint32_t spin_limit);
+
 /* ---------------------------------------------------------------------- */
 /* Host-side format builder ("compression"; offline, host memory only).   */
 
