@@ -34,7 +34,7 @@ DF11_DECODE_TABLE_BYTES = 17664
 STATUS = {
     0: "DF11_OK", 1: "DF11_ERR_NULL", 2: "DF11_ERR_ALIGN", 3: "DF11_ERR_FORMAT",
     4: "DF11_ERR_UNSUPPORTED", 5: "DF11_ERR_CUDA", 6: "DF11_ERR_TOO_LARGE",
-    7: "DF11_ERR_INVALID", 8: "DF11_ERR_NOMEM",
+    7: "DF11_ERR_INVALID", 8: "DF11_ERR_NOMEM", 9: "DF11_ERR_DEVICE",
 }
 DEV_ERRORS = {
     0: "DF11_DEV_OK", 1: "DF11_DEV_ERR_COUNT", 2: "DF11_DEV_ERR_OVERRUN",
@@ -389,9 +389,16 @@ def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24
     """compress_on_device for several tensors, with one stream
     synchronisation per phase for all of them
     (df11_gpu_build_begin_batched / _finish_batched)."""
-    count = len(ws)
-    if count == 0:
+    if len(ws) == 0:
         return []
+    with torch.cuda.device(ws[0].device):
+        return _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream,
+                                           decode_table, interleave)
+
+
+def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, decode_table,
+                                interleave):
+    count = len(ws)
     flats, shapes = [], []
     for w in ws:
         if not w.is_cuda:
@@ -457,27 +464,32 @@ def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24
 
 
 def exponent_histogram(w: torch.Tensor, stream=None) -> np.ndarray:
-    """Counts of the 256 exponent values of a BF16 tensor in device memory
-    (df11_exponent_histogram; allocates nothing on the device)."""
+    """Counts of the 256 exponent values of a contiguous BF16 tensor in
+    device memory (df11_exponent_histogram: allocates no device memory, for
+    callers that cannot; synchronises the stream)."""
     if not w.is_cuda:
         raise ValueError("exponent_histogram takes a CUDA tensor")
     if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
         raise TypeError(f"expected BF16 words (bfloat16, int16 or uint16), got {w.dtype}")
-    flat = w.contiguous().reshape(-1)
-    n = flat.numel()
+    if not w.is_contiguous():
+        # a contiguous copy would be a device allocation, which this call avoids
+        raise ValueError("exponent_histogram takes a contiguous tensor")
+    n = w.numel()
     hist = np.zeros(256, dtype=np.uint64)
-    _check(lib().df11_exponent_histogram(flat.data_ptr() if n else None, n,
-                                         hist.ctypes.data, _stream_handle(stream)),
-           "df11_exponent_histogram")
+    with torch.cuda.device(w.device):
+        _check(lib().df11_exponent_histogram(w.data_ptr() if n else None, n,
+                                             hist.ctypes.data, _stream_handle(stream)),
+               "df11_exponent_histogram")
     return hist
 
 
 def build_decode_table(d: Df11Device, stream=None) -> torch.Tensor:
     """The decode table of a device tensor (df11_build_decode_table)."""
     t = torch.empty(DF11_DECODE_TABLE_BYTES, dtype=torch.uint8, device=d.device)
-    _check(lib().df11_build_decode_table(d.luts.data_ptr(), d.code_lengths.data_ptr(),
-                                         int(d.params.num_luts), t.data_ptr(),
-                                         _stream_handle(stream)), "df11_build_decode_table")
+    with torch.cuda.device(d.device):
+        _check(lib().df11_build_decode_table(d.luts.data_ptr(), d.code_lengths.data_ptr(),
+                                             int(d.params.num_luts), t.data_ptr(),
+                                             _stream_handle(stream)), "df11_build_decode_table")
     return t
 
 
@@ -506,12 +518,13 @@ def decode(d: Df11Device, out: Optional[torch.Tensor] = None,
     if counts and d.chunk_counts is not None:
         return decode_batched([d], [out], err=err, stream=stream)[0]
     p = Params.from_buffer_copy(d.params)
-    _check(lib().df11_decode(
-        d.bitstream.data_ptr(), d.gaps.data_ptr(), d.block_out_pos.data_ptr(),
-        d.luts.data_ptr(), d.code_lengths.data_ptr(), d.sign_mantissa.data_ptr(),
-        out.data_ptr(), d.n, ctypes.byref(p),
-        err.data_ptr() if err is not None else None, _stream_handle(stream)),
-        "df11_decode")
+    with torch.cuda.device(d.device):
+        _check(lib().df11_decode(
+            d.bitstream.data_ptr(), d.gaps.data_ptr(), d.block_out_pos.data_ptr(),
+            d.luts.data_ptr(), d.code_lengths.data_ptr(), d.sign_mantissa.data_ptr(),
+            out.data_ptr(), d.n, ctypes.byref(p),
+            err.data_ptr() if err is not None else None, _stream_handle(stream)),
+            "df11_decode")
     return out
 
 
@@ -528,11 +541,24 @@ def decode_batched(ds: Sequence[Df11Device], outs: Sequence[torch.Tensor],
         raise ValueError("one output per tensor")
     for d, o in zip(ds, outs):
         _check_out(d, o)
-    arr = (TensorDesc * max(len(ds), 1))(*[d.desc(o, counts) for d, o in zip(ds, outs)])
-    _check(lib().df11_decode_batched(arr, len(ds),
-                                     err.data_ptr() if err is not None else None,
-                                     _stream_handle(stream)), "df11_decode_batched")
+    if not ds:
+        return outs
+    arr = (TensorDesc * len(ds))(*[d.desc(o, counts) for d, o in zip(ds, outs)])
+    with torch.cuda.device(_one_device(ds, outs)):
+        _check(lib().df11_decode_batched(arr, len(ds),
+                                         err.data_ptr() if err is not None else None,
+                                         _stream_handle(stream)), "df11_decode_batched")
     return outs
+
+
+def _one_device(ds, others=()):
+    """The one CUDA device of a call's tensors (the library's kernels run on
+    the current device and check that every buffer is its own)."""
+    dev = ds[0].device
+    for t in list(ds) + list(others):
+        if t.device != dev:
+            raise ValueError(f"tensors of one call on {dev} and {t.device}")
+    return dev
 
 
 class DecodePlan:
@@ -551,12 +577,16 @@ class DecodePlan:
         self._n = len(ds)
         self._arr = (TensorDesc * max(self._n, 1))(*[d.desc(o, counts) for d, o in zip(ds, outs)])
         self._lib = lib()
+        self._device = _one_device(ds, outs) if ds else None
 
     @property
     def outs(self):
         return self._keep[1]
 
     def run(self, err: Optional[torch.Tensor] = None, stream=None):
+        if self._device is not None and torch.cuda.current_device() != self._device.index:
+            with torch.cuda.device(self._device):
+                return self.run(err, stream)
         _check(self._lib.df11_decode_batched(self._arr, self._n,
                                              err.data_ptr() if err is not None else None,
                                              _stream_handle(stream)), "df11_decode_batched")
@@ -598,8 +628,10 @@ def decode_gemv(ds: Sequence["Df11Device"], xs: Sequence[torch.Tensor],
     for i, d in enumerate(ds):
         descs[i].out_bf16 = None
     ops = (GemvOp * n)(*[_gemv_op(d, x, y, accumulate) for d, x, y in zip(ds, xs, ys)])
-    _check(lib().df11_decode_gemv(descs, ops, n, err.data_ptr() if err is not None else None,
-                                  _stream_handle(stream)), "df11_decode_gemv")
+    with torch.cuda.device(_one_device(ds)):
+        _check(lib().df11_decode_gemv(descs, ops, n,
+                                      err.data_ptr() if err is not None else None,
+                                      _stream_handle(stream)), "df11_decode_gemv")
 
 
 def new_error_word(device="cuda") -> torch.Tensor:

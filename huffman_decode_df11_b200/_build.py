@@ -16,7 +16,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdf11.so")
 SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_gpu_build.cu"),
            os.path.join(CSRC, "df11_build.cpp")]
-HEADERS = [os.path.join(INCLUDE, "df11.h"), os.path.join(CSRC, "df11_codebook.h")]
+HEADERS = [os.path.join(INCLUDE, "df11.h"), os.path.join(CSRC, "df11_codebook.h"),
+           os.path.join(CSRC, "df11_device_check.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

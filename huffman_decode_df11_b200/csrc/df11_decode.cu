@@ -55,6 +55,7 @@
 #include <cstdint>
 
 #include "df11.h"
+#include "df11_device_check.h"
 
 namespace {
 
@@ -1653,6 +1654,22 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   return DF11_ERR_UNSUPPORTED;
 }
 
+// The buffers of a call's non-empty tensors must be memory of the current
+// device, where its kernels run (checked for every tensor of the call before
+// anything is queued): the stream, the sign/mantissa bytes and the output
+// (or the product's activations and results).
+df11_status check_devices(const df11_tensor *ts, int count, const df11_gemv *ops = nullptr) {
+  for (int i = 0; i < count; ++i) {
+    if (ts[i].params.n == 0) continue;
+    const void *ptrs[5] = {ts[i].bitstream, ts[i].sign_mantissa, ts[i].decode_table,
+                           ops ? (const void *)ops[i].x : (const void *)ts[i].out_bf16,
+                           ops ? (const void *)ops[i].y : nullptr};
+    const df11_status st = df11_internal::check_device_pointers(ptrs, 5);
+    if (st != DF11_OK) return st;
+  }
+  return DF11_OK;
+}
+
 // Tensors with chunk counts go to the warp-specialised kernel, the others to
 // the count-by-decoding kernel (one launch each, same stream).
 df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaStream_t s) {
@@ -1684,6 +1701,8 @@ df11_status df11_decode(const uint8_t *bitstream, const uint8_t *gaps,
                 out_bf16, nullptr, *params};
   df11_status st = validate(t);
   if (st != DF11_OK || n == 0) return st;
+  st = check_devices(&t, 1);
+  if (st != DF11_OK) return st;
   return launch_batch(&t, 1, d_err, (cudaStream_t)stream);
 }
 
@@ -1705,6 +1724,8 @@ df11_status df11_decode_batched(const df11_tensor *tensors, int count, int32_t *
       return DF11_ERR_INVALID;
     }
   }
+  const df11_status dst = check_devices(tensors, count);
+  if (dst != DF11_OK) return dst;
   for (int i = 0; i < count; i += DF11_MAX_BATCH) {
     const int c = count - i < DF11_MAX_BATCH ? count - i : DF11_MAX_BATCH;
     df11_status st = launch_batch(tensors + i, c, d_err, (cudaStream_t)stream);
@@ -1747,6 +1768,8 @@ df11_status df11_decode_gemv(const df11_tensor *tensors, const df11_gemv *ops, i
     }
   }
   if (C && !(T == 256 && (C == 8 || C == 16 || C == 24))) return DF11_ERR_UNSUPPORTED;
+  const df11_status dst = check_devices(tensors, count, ops);
+  if (dst != DF11_OK) return dst;
   // y = W x: clear the outputs first, in stream order, one launch per 16
   for (int i = 0; i < count; i += DF11_MAX_BATCH) {
     ClearArgs ca{};
@@ -1785,6 +1808,9 @@ df11_status df11_build_decode_table(const uint32_t *luts, const uint8_t *code_le
   if (!luts || !code_lengths || !out) return DF11_ERR_NULL;
   if (!aligned(luts, 16) || !aligned(out, 16)) return DF11_ERR_ALIGN;
   if (num_luts < 1 || num_luts >= (1u << 24)) return DF11_ERR_FORMAT;
+  const void *ptrs[3] = {luts, code_lengths, out};
+  const df11_status st = df11_internal::check_device_pointers(ptrs, 3);
+  if (st != DF11_OK) return st;
   df11_table_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(luts, code_lengths, num_luts,
                                                            reinterpret_cast<uint4 *>(out));
   return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
@@ -1825,6 +1851,7 @@ const char *df11_status_string(df11_status s) {
     case DF11_ERR_TOO_LARGE: return "size beyond the supported range";
     case DF11_ERR_INVALID: return "invalid argument";
     case DF11_ERR_NOMEM: return "host allocation failed";
+    case DF11_ERR_DEVICE: return "a device pointer is not memory of the current device";
   }
   return "unknown status";
 }

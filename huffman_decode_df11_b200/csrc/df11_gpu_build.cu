@@ -45,6 +45,7 @@
 #include <vector>
 
 #include "df11.h"
+#include "df11_device_check.h"
 #include "df11_codebook.h"
 
 namespace {
@@ -778,6 +779,11 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     const df11_status st = check_begin_args(d_bf16[i], n[i], C, T);
     if (st != DF11_OK) return st;
   }
+  for (int i = 0; i < count; ++i) {  // after every host-side check
+    const void *p = n[i] ? d_bf16[i] : nullptr;
+    const df11_status st = df11_internal::check_device_pointers(&p, 1);
+    if (st != DF11_OK) return st;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   std::vector<df11_gpu_build *> hs(count, nullptr);
   auto fail = [&](df11_status st) {
@@ -933,6 +939,13 @@ df11_status df11_gpu_build_finish_batched(df11_gpu_build *const *handles, int co
       st = DF11_ERR_ALIGN;
     }
   }
+  for (int i = 0; i < count && st == DF11_OK; ++i) {  // after every host-side check
+    const df11_gpu_build_out &o = outs[i];
+    const void *ptrs[8] = {o.bitstream, o.gaps, o.chunk_counts, o.block_out_pos,
+                           o.luts, o.code_lengths, o.sign_mantissa,
+                           handles[i]->n ? (const void *)d_bf16[i] : nullptr};
+    st = df11_internal::check_device_pointers(ptrs, 8);
+  }
   std::unique_lock<std::mutex> lock(g_staging.mu, std::defer_lock);
   size_t stage_bytes = 0;
   std::vector<size_t> off(count > 0 ? count : 0);
@@ -1036,37 +1049,70 @@ df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uin
 
 }  // extern "C"
 
-// ---- exponent histogram into a static device buffer ----------------------
+// ---- exponent histogram with no allocation --------------------------------
+// Some callers cannot allocate device memory: code running where the CUDA
+// allocator must not be entered (inside an allocator hook, or a pool that is
+// being resized), or a caller that has handed all device memory to its own
+// allocator and has none to spare.  For them df11_exponent_histogram runs
+// the builder's histogram kernel with its counters in this file-scope array
+// instead of scratch the builder takes from its memory pool.  Its size is
+// fixed: 256 64-bit counters (2 KB), held by every device that loads the
+// library until the process exits.  All calls on a device share it and it
+// keeps the last call's counts, so every call clears it first; two calls
+// whose work overlaps on the GPU would race on it, which the library
+// prevents within a process by taking one call at a time per device and
+// waiting for each call's counts to come back before the next starts.
+static __device__ __align__(256) unsigned long long g_exponent_hist[256];
+
 namespace {
-// The histogram entry point's device counters: a module global, so the call
-// needs no allocation.  One copy per device; calls are serialised.
-__device__ __align__(256) unsigned long long g_exponent_hist[256];
-std::mutex g_exponent_hist_mutex;
+struct HistDevice {
+  std::mutex mu;                       // one call at a time on this device's array
+  unsigned long long *addr = nullptr;  // device address of g_exponent_hist (set-up)
+};
+HistDevice g_hist_device[kMaxDevices];
 }  // namespace
 
 extern "C" df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t n,
                                                uint64_t hist[256], df11_stream_t stream) {
+  static_assert(sizeof(uint64_t) == sizeof(unsigned long long), "counter width");
   if (!hist || (n && !d_bf16)) return DF11_ERR_NULL;
   if (n >= (1ull << 32)) return DF11_ERR_TOO_LARGE;
   if ((uintptr_t)d_bf16 & 1) return DF11_ERR_ALIGN;
-  std::lock_guard<std::mutex> lock(g_exponent_hist_mutex);
-  void *sym = nullptr;
-  if (cudaGetSymbolAddress(&sym, g_exponent_hist) != cudaSuccess) return DF11_ERR_CUDA;
-  unsigned long long *d = static_cast<unsigned long long *>(sym);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DF11_ERR_INVALID;
+  if (n) {
+    const void *p = d_bf16;
+    const df11_status st = df11_internal::check_device_pointers(&p, 1);
+    if (st != DF11_OK) return st;
+  }
+  HistDevice &hd = g_hist_device[dev];
+  std::lock_guard<std::mutex> lock(hd.mu);
+  if (!hd.addr) {
+    // set-up, once per device, with that device current: in host code the
+    // array's name stands for a host-side shadow, not a device address
+    void *sym = nullptr;
+    if (cudaGetSymbolAddress(&sym, g_exponent_hist) != cudaSuccess || !sym) return DF11_ERR_CUDA;
+    hd.addr = static_cast<unsigned long long *>(sym);
+  }
   cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemsetAsync(d, 0, 256 * sizeof(unsigned long long), s) != cudaSuccess)
-    return DF11_ERR_CUDA;
+  if (cudaMemsetAsync(hd.addr, 0, sizeof(g_exponent_hist), s) != cudaSuccess) return DF11_ERR_CUDA;
   if (n) {
     const uint64_t tiles = (n + kPerCta - 1) / kPerCta, slots = resident(hist_kernel);
     const bool vec = ((uintptr_t)d_bf16 & 15) == 0;
-    hist_kernel<<<(unsigned)(tiles < slots ? tiles : slots), kThreads, 0, s>>>(d_bf16, n, vec, d,
-                                                                               nullptr);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(tiles < slots ? tiles : slots));
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = s;
+    unsigned long long *no_last = nullptr;
+    // the launch's own status (not an earlier error of the calling thread)
+    if (cudaLaunchKernelEx(&cfg, hist_kernel, d_bf16, n, vec, hd.addr, no_last) != cudaSuccess)
+      return DF11_ERR_CUDA;
   }
-  unsigned long long counts[256];
-  if (cudaGetLastError() != cudaSuccess ||
-      cudaMemcpyAsync(counts, d, sizeof(counts), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+  // straight into the caller's array (a DMA if the caller pinned it)
+  if (cudaMemcpyAsync(hist, hd.addr, sizeof(g_exponent_hist), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return DF11_ERR_CUDA;
-  for (int i = 0; i < 256; ++i) hist[i] = counts[i];
   return DF11_OK;
 }

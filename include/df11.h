@@ -75,7 +75,9 @@ typedef enum df11_status {
   DF11_ERR_CUDA = 5,        /* a CUDA runtime call failed */
   DF11_ERR_TOO_LARGE = 6,   /* n >= 2^32, or a batch over DF11_MAX_BATCH */
   DF11_ERR_INVALID = 7,     /* other invalid argument */
-  DF11_ERR_NOMEM = 8        /* host allocation failed (df11_build) */
+  DF11_ERR_NOMEM = 8,       /* host allocation failed (df11_build) */
+  DF11_ERR_DEVICE = 9       /* a device pointer is not memory of the current
+                               device (checked before anything is queued) */
 } df11_status;
 
 /* Values the GPU writes to *d_err.  A device word that is not 0 means the
@@ -340,17 +342,30 @@ df11_status df11_gpu_build_finish(df11_gpu_build *handle, const uint16_t *d_bf16
                                   df11_params *params, df11_stream_t stream);
 
 /*
- * Exponent histogram of n BF16 words in device memory: hist[e] (host array
- * of 256) = how many words have exponent field e (bits 7-14).  The paper has
- * no counterpart to this entry point: it is the builder's first step on its
- * own, for callers that want the exponent statistics (entropy, the size a
- * tensor will compress to) without building.  It allocates nothing: the
- * device counters are a static buffer of the library (one per device), so
- * concurrent calls are serialised inside the library.  Queues its work on
- * `stream` and synchronises it.  d_bf16 must be 2-byte aligned (16-byte
- * alignment lets the kernel load 8 words at a time).  Errors:
- * DF11_ERR_NULL, _TOO_LARGE (n >= 2^32), _ALIGN before any device work;
- * DF11_ERR_CUDA if a CUDA call fails.
+ * Exponent histogram of n BF16 words in device memory, with no allocation:
+ * hist[e] (host array of 256) = how many words have exponent field e (bits
+ * 7-14).  The paper has no counterpart to this entry point.  It is the
+ * builder's histogram kernel on its own, for callers that cannot allocate
+ * device memory -- code that runs where the CUDA allocator must not be
+ * entered (an allocator hook, a memory pool in the middle of a resize), or
+ * a program that has handed all device memory to its own allocator -- and
+ * still want the exponent statistics (entropy, the size a tensor will
+ * compress to).  It calls no cudaMalloc, cudaFree or other allocating
+ * routine: its counters are a fixed array of 256 64-bit counters (2 KB) in
+ * the library's device memory, one per device, held until the process
+ * exits.  The first call on a device looks up that array's device address
+ * (set-up, with the device current); make that first call before any
+ * stream capture.  All calls on a device share the array and it keeps the
+ * last call's counts, so every call clears it first; calls whose work
+ * overlapped on the GPU would race on it, so the library takes one call at
+ * a time per device and waits for each call's counts.  Queues its work on
+ * `stream` (of the current device) and synchronises it; the counts are
+ * copied straight into `hist` (pinned memory makes that a DMA).  d_bf16
+ * must be 2-byte aligned memory of the current device (16-byte alignment
+ * lets the kernel load 8 words at a time).  Errors: DF11_ERR_NULL,
+ * _TOO_LARGE (n >= 2^32: beyond the counters' and the kernel's index
+ * range), _ALIGN, _DEVICE (d_bf16 not memory of the current device) before
+ * any device work; DF11_ERR_CUDA if a CUDA call fails.
  */
 df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t n, uint64_t hist[256],
                                     df11_stream_t stream);

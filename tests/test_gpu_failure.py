@@ -79,3 +79,27 @@ def test_withheld_copies_in_the_middle_of_a_layer_loop(cuda):
     assert int(err.item()) == TIMEOUT
     for i in (0, 2):
         assert np.array_equal(got[i].view(torch.int16).cpu().numpy(), ws[i].numpy())
+
+
+@pytest.mark.gpu
+def test_buffers_that_are_not_device_memory_are_refused(cuda):
+    """A call whose buffers are not memory of the current device returns
+    DF11_ERR_DEVICE before anything is queued (a kernel would otherwise read
+    host or another GPU's memory)."""
+    import ctypes
+    ws, ds = _tensors(2)
+    outs = [df11.empty_output(d) for d in ds]
+    host_out = np.zeros(ds[1].n + 8, np.uint16)
+    descs = (df11.TensorDesc * 2)(ds[0].desc(outs[0]), ds[1].desc(outs[1]))
+    descs[1].out_bf16 = (host_out.ctypes.data + 15) // 16 * 16
+    err = df11.new_error_word()
+    outs[0].fill_(0)
+    st = df11.lib().df11_decode_batched(descs, 2, err.data_ptr(), None)
+    torch.cuda.synchronize()
+    assert st == 9  # DF11_ERR_DEVICE
+    assert int(err.item()) == 0
+    assert not outs[0].view(torch.int16).any()  # nothing was decoded
+    assert not host_out.any()
+    hist = np.zeros(256, np.uint64)
+    bad = torch.zeros(16, dtype=torch.int16).pin_memory()  # host memory
+    assert df11.lib().df11_exponent_histogram(bad.data_ptr(), 16, hist.ctypes.data, None) == 9
