@@ -1,20 +1,18 @@
 // df11_decode.cu -- DF11 decode on sm_100a (B200) and the C ABI around it.
 //
-// Two kernels, both with persistent thread blocks: every thread block is
-// assigned to one tensor of the launch (one wave, split by format blocks)
-// and walks that tensor's format blocks (T chunks of C bitstream bytes) with
-// a stride.  Both use a decode table in shared memory: table 0 of the format
-// and the code lengths with every exponent byte rotated right by one bit,
-// and a derived table of 2^11 entries, each holding up to five whole
-// codewords of the next 11 bits (built once per tensor by df11_table_kernel,
-// or by every thread block when none is passed; the page-layout kernel
-// derives its own with up to four, which its accumulator takes).
-// Deeper format tables (codewords longer than 8 bits) are read from global
-// memory.
+// One kernel, with persistent thread blocks: every thread block is assigned
+// to one tensor of the launch (one wave, split by format blocks) and walks
+// that tensor's format blocks (T chunks of C bitstream bytes) with a stride.
+// It uses a decode table in shared memory: table 0 of the format and the
+// code lengths with every exponent byte rotated right by one bit, and a
+// derived table of 2^11 entries, each holding up to five whole codewords of
+// the next 11 bits (built once per tensor by df11_table_kernel, or by every
+// thread block when none is passed).  Deeper format tables (codewords longer
+// than 8 bits) are read from global memory.
 //
-// df11_decode_ws_kernel, for tensors with chunk counts (the default path).
-// Warp-specialised: one producer warp and T/32 consumer warps per thread
-// block, no block-wide barrier per format block.
+// df11_decode_ws_kernel: warp-specialised, one producer warp and T/32
+// consumer warps per thread block, no block-wide barrier per format block.
+// With chunk counts (the default path):
 //   stage    the producer's lane 0 keeps two stage slots filled with bulk
 //            copies (cp.async.bulk, no multicast) of a block's bitstream
 //            slice, gap fields and chunk counts, and its sign/mantissa bytes
@@ -34,10 +32,12 @@
 //            and writes the two ragged 16-element groups one element per
 //            lane; then releases the slot.
 //
-// df11_decode_kernel, for the format as the pages state it (no chunk
-// counts): every thread decodes its chunk into a private slot, counting
-// ("locate"), a block-wide scan places the slots, they are compacted into a
-// block-wide exponent array, and the block writes its output range.
+// Without chunk counts (the format as the pages state it): each lane decodes
+// its chunk into its own column of the warp's column area, counting
+// ("locate"); the warps of the block post their totals and wait for each
+// other (one bounded mbarrier wait per block); each lane then moves its
+// bytes to their place in the warp's exponent region ("reconstruct"), and
+// the output runs as above.
 //
 // Why the rotation: with e' = e>>1 | (e&1)<<7, the high byte of a BF16 word
 // is (sm & 0x80) | (e' & 0x7F) and the low byte (e' & 0x80) | (sm & 0x7F), so
@@ -59,7 +59,6 @@
 
 namespace {
 
-constexpr int kSubTablesInSmem = 8;        // deeper tables kept in shared memory
 constexpr uint32_t kSpinLimit = 1u << 20;  // x ~1 us suspend hint: ~1 s
 constexpr uint32_t kSuspendHintNs = 1000;
 constexpr int kWideBits = 11;              // index bits of the derived table
@@ -99,28 +98,23 @@ struct KBatch {
   int count;
   uint32_t cta_end;      // total thread blocks
   uint32_t stage_bytes;  // bytes of the exponent array
-  uint32_t slot_words;   // 32-bit words of each thread's private slot
-  uint32_t sub_words;    // deeper-table words kept in shared memory (0: global)
   uint32_t sm_bytes;     // sign/mantissa bytes per stage slot (warp-specialised kernel;
                          // 0: read from global memory)
   uint32_t spin_limit;   // polls of every bounded wait (kSpinLimit unless a test lowers it)
   uint32_t withhold;     // test hook: the producer issues no stage copy, so the
                          // consumers' waits run out (df11_test_withhold_copies)
+  uint32_t col_bytes;    // without chunk counts: bytes of each warp's column area
+  uint32_t col_cap;      // without chunk counts: most bytes a column takes (max_chunk_elems)
 };
 
 // ---- shared memory layout --------------------------------------------------
-// [0,16)       2 mbarriers (one per stage slot)
-// [16,48)      2 x {P0, P1, ok, 0}: block positions of the block in each slot
-// [48,304)     2 x 32 ints of scan scratch (alternating between blocks)
+// [0,304)      mbarriers (full and empty per stage slot, per-warp copies, the
+//              decode table's copy, the page layout's counted barriers)
 // [304,560)    code lengths by rotated exponent
 // [560,1584)   table 0 (rotated)
 // [1584, ...)  wide table (2^WB x 8 bytes)
-// then         2 stage slots: bitstream (T*C+16), gaps (T*5/8+16)
-// then         exponent array (stage_bytes), private slots (slot_words*T*4),
-//              deeper tables (sub_words*4)
-constexpr uint32_t kOffMbar = 0;
-constexpr uint32_t kOffMeta = 16;
-constexpr uint32_t kOffScan = 48;
+// then         the stage slots, the warps' exponent regions, their
+//              sign/mantissa buffers and column areas (see the kernel)
 constexpr uint32_t kOffLens = 304;
 constexpr uint32_t kOffLut0 = 560;
 constexpr uint32_t kOffWide = 1584;
@@ -129,14 +123,6 @@ constexpr uint32_t kOffStages = kOffWide + kWideBytes;
 // a decode table (df11_build_decode_table) is the image of [kOffLens, kOffStages)
 static_assert(kOffStages - kOffLens == DF11_DECODE_TABLE_BYTES, "decode table layout");
 static_assert(kOffLut0 - kOffLens == 256 && kOffWide - kOffLut0 == 1024, "decode table layout");
-
-template <int T, int C>
-struct Layout {
-  static constexpr uint32_t bits_bytes = T * C + 16;
-  static constexpr uint32_t gaps_bytes = T * 5 / 8 + 16;
-  static constexpr uint32_t slot_bytes = bits_bytes + gaps_bytes;  // one slot
-  static_assert(bits_bytes % 16 == 0 && gaps_bytes % 16 == 0, "alignment");
-};
 
 __device__ __forceinline__ uint32_t rot8x3(uint32_t v) {
   // rotate each of the low three bytes right by one bit
@@ -349,55 +335,6 @@ __device__ __forceinline__ uint32_t window(const uint32_t (&w)[C / 4 + 1], uint3
   return __funnelshift_l(lo, hi, pos);
 }
 
-// Walk one thread's codewords [start, end) (bit positions relative to its
-// chunk's first bit) and append their exponents to its private slot: word j
-// at shared address slot + 4*T*j.  `pk` packs the bit position (bits 0-15)
-// with the number of bits waiting in the 64-bit accumulator a1:a0 (bits
-// 16-31, a multiple of 8).  The current word is stored after every lookup and the slot
-// address moves on when it is full, so no branch but the loop's and the rare
-// slow path's.  Returns the number of codewords; sets `bad` on inconsistent
-// data.
-template <int T, int C, bool MASKED>
-__device__ __forceinline__ uint32_t decode_chunk(const uint32_t (&w)[C / 4 + 1], int start,
-                                                 const int end, uint32_t wide,
-                                                 const uint32_t *__restrict__ lut0,
-                                                 const uint8_t *__restrict__ lens,
-                                                 const uint32_t *sub, uint32_t num_luts,
-                                                 uint32_t slot, uint32_t slot_words, int &bad) {
-  uint32_t a0 = 0, a1 = 0, pk = (uint32_t)start, sa = slot, words = 0;
-  const uint32_t sa_last = slot + (slot_words - 1) * (4u * T);
-  while ((int)(pk & 0xFFFFu) < end) {
-    const uint32_t win = window<C>(w, pk & 0xFFFFu);
-    uint2 e = lds64(wide + ((win >> (32 - kWideBits)) << 3));
-    if (e.y == 0 || (!MASKED && (int)(e.y & 0xFFFFu) > end - (int)(pk & 0xFFFFu))) {
-      // rare: a codeword longer than WB bits, or (unmasked streams) an
-      // entry running past the region's end: one codeword via the format's
-      // own tables
-      uint32_t sym, len;
-      if (!decode_one(win, lut0, lens, sub, num_luts, sym, len)) {
-        bad = DF11_DEV_ERR_TABLE;
-        return 0;
-      }
-      e = make_uint2(sym, len | (8u << 16));
-    }
-    const uint32_t sh = pk >> 16;
-    a0 |= e.x << sh;
-    a1 |= __funnelshift_l(e.x, 0u, sh);  // bytes pushed past the low word
-    pk += e.y;
-    sts32(sa, a0);
-    if (pk >= (32u << 16)) {  // the word is complete: move on
-      sa = min(sa + 4u * T, sa_last);
-      ++words;
-      a0 = a1;
-      a1 = 0;
-      pk -= 32u << 16;
-    }
-  }
-  if (pk >> 16) sts32(sa, a0);
-  if ((int)(pk & 0xFFFFu) != end) bad = DF11_DEV_ERR_OVERRUN;
-  return words * 4u + (pk >> 19);
-}
-
 // The same walk when the thread's output place is known before it decodes
 // (the format's chunk count): exponents go straight into the block's
 // (zeroed) exponent array from byte d on.  Every lookup ORs its up to five
@@ -501,6 +438,86 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t (&w)[C / 4 + 1
   return (pk >> 19) - d;
 }
 
+// The walk of the format as the pages state it (no chunk counts): a thread
+// learns where its output goes only once every warp of the block has
+// counted, so it decodes into its own column of the warp's column area
+// (its byte j at word (j/4)*32 + lane: the lanes' reductions never share a
+// bank) and counts.  The window moves as in decode_counted; the walk stops
+// at the chunk's end bit, or when `cap` bytes (the format's
+// max_chunk_elems) are written, beyond which the data are inconsistent.
+// Unmasked streams (every codeword within the derived table's index) check
+// each entry against the end.  Returns the number of codewords.
+template <int C, bool MASKED>
+__device__ __forceinline__ uint32_t decode_column(const uint32_t (&w)[C / 4 + 1], int start,
+                                                  const int end, uint32_t wide,
+                                                  const uint32_t *__restrict__ lut0,
+                                                  const uint8_t *__restrict__ lens,
+                                                  const uint32_t *sub, uint32_t num_luts,
+                                                  uint32_t col, uint32_t cap, int &bad) {
+  constexpr int NW = C / 4 + 1;
+  uint32_t s[NW];
+#pragma unroll
+  for (int j = 0; j < NW - 1; ++j) s[j] = __funnelshift_l(w[j + 1], w[j], (uint32_t)start);
+  s[NW - 1] = __funnelshift_l(0xFFFFFFFFu, w[NW - 1], (uint32_t)start);
+  uint32_t pk = (uint32_t)start;          // bit position | 8 * bytes written << 16
+  const uint32_t lim = (8u * cap) << 16;  // pk < lim: fewer than cap bytes written
+  while ((int)(pk & 0xFFFFu) < end && pk < lim) {
+    uint2 e = lds64(wide + ((s[0] >> (32 - kWideBits)) << 3));
+    if (e.y == 0 || (!MASKED && (int)(e.y & 0xFFFFu) > end - (int)(pk & 0xFFFFu))) {
+      // a codeword longer than the derived table's index, or (unmasked
+      // streams) an entry that runs past the end: one codeword through the
+      // format's own tables, the window moved by half its length here
+      uint32_t sym, len;
+      if (!decode_one(s[0], lut0, lens, sub, num_luts, sym, len)) {
+        bad = DF11_DEV_ERR_TABLE;
+        return 0;
+      }
+      const uint32_t half = len >> 1;
+#pragma unroll
+      for (int j = 0; j < NW - 1; ++j) s[j] = __funnelshift_l(s[j + 1], s[j], half);
+      s[NW - 1] = __funnelshift_l(0xFFFFFFFFu, s[NW - 1], half);
+      pk += half;
+      e = make_uint2(sym, (len - half) | (8u << 16));
+    }
+    const uint32_t sh = pk >> 16;
+    const uint32_t a = col + ((pk >> 21) << 7);
+    red_or32(a, __funnelshift_l(0u, e.x, sh));
+    red_or32(a + 128u, __funnelshift_l(e.x, e.y >> 24, sh));
+#pragma unroll
+    for (int j = 0; j < NW - 1; ++j) s[j] = __funnelshift_l(s[j + 1], s[j], e.y);
+    s[NW - 1] = __funnelshift_l(0xFFFFFFFFu, s[NW - 1], e.y);
+    pk += e.y & 0x00FFFFFFu;
+  }
+  const int pos = (int)(pk & 0xFFFFu);
+  if (pos != end) bad = pos < end ? DF11_DEV_ERR_COUNT : DF11_DEV_ERR_OVERRUN;
+  return pk >> 19;
+}
+
+// A lane's `cnt` exponent bytes, from its column (word k at col + 128k),
+// into the warp's element-order region from byte d on: whole words are
+// stored, the first and last (shared with the neighbouring lanes' ranges)
+// ORed into the zeroed region.  Column bytes past cnt are zero.  Each column
+// word is zeroed once read, for the next block.
+__device__ __forceinline__ void column_to_region(uint32_t col, uint32_t cnt, uint32_t region,
+                                                 uint32_t d) {
+  if (!cnt) return;
+  const uint32_t r8 = (d & 3u) * 8u;
+  const uint32_t words = ((d & 3u) + cnt + 3u) >> 2;  // destination words
+  const uint32_t held = (cnt + 3u) >> 2;              // column words with bytes
+  uint32_t prev = 0, dst = region + (d & ~3u);
+  for (uint32_t j = 0; j < words; ++j, dst += 4u) {
+    uint32_t cur = 0;
+    if (j < held) {
+      cur = lds32(col + 128u * j);
+      sts32(col + 128u * j, 0u);
+    }
+    const uint32_t v = __funnelshift_l(prev, cur, r8);  // bytes 4j - (d & 3) ..
+    if (j == 0 || j + 1 == words) red_or32(dst, v);
+    else sts32(dst, v);
+    prev = cur;
+  }
+}
+
 // four sign/mantissa bytes and four rotated exponents -> four BF16 words:
 // the four low bytes (E0 | mantissa) and the four high bytes (sign | E7..E1)
 // are two bitwise selects, then two byte permutes interleave them
@@ -517,257 +534,6 @@ __device__ __forceinline__ uint16_t fuse1(uint32_t sm, uint32_t er) {
 
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// Thread 0: queue the copies of block b into stage slot `stage` (or, for
-// inconsistent block positions, an empty completion flagged not ok) and an
-// L2 prefetch of its sign/mantissa bytes.
-template <int T, int C>
-__device__ __forceinline__ void issue_block(const KTensor &tk, uint32_t b, uint32_t P0,
-                                            uint32_t P1, uint8_t *stage, uint4 *meta,
-                                            uint32_t bar, uint32_t stage_bytes) {
-  using L = Layout<T, C>;
-  const uint32_t expected = P1 - P0;
-  const bool ok = P1 >= P0 && P1 <= tk.n && expected <= tk.max_block_elems &&
-                  expected + 32 <= stage_bytes;
-  *meta = make_uint4(P0, P1, ok ? 1u : 0u, 0u);
-  if (!ok) {
-    mbar_arrive_expect_tx(bar, 0);
-    return;
-  }
-  mbar_arrive_expect_tx(bar, L::bits_bytes + L::gaps_bytes);
-  bulk_g2s(smem_addr(stage), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, bar);
-  bulk_g2s(smem_addr(stage + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
-           bar);
-  const uint32_t sm_begin = P0 & ~15u;
-  const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
-  if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
-}
-
-template <int T, int C>
-__global__ void __launch_bounds__(T, 1536 / T) df11_decode_kernel(const __grid_constant__ KBatch kb) {
-  using L = Layout<T, C>;
-  constexpr int NW = C / 4 + 1;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + kOffMbar);
-  uint4 *meta = reinterpret_cast<uint4 *>(smem + kOffMeta);
-  int *scan = reinterpret_cast<int *>(smem + kOffScan);
-  uint8_t *lens_s = smem + kOffLens;
-  uint32_t *lut0_s = reinterpret_cast<uint32_t *>(smem + kOffLut0);
-  uint2 *wide_s = reinterpret_cast<uint2 *>(smem + kOffWide);
-  uint8_t *stages = smem + kOffStages;
-  uint8_t *ex_s = stages + 2 * L::slot_bytes;
-  uint32_t *slots = reinterpret_cast<uint32_t *>(ex_s + kb.stage_bytes);
-  uint32_t *sub_s = slots + kb.slot_words * T;
-
-  int ti = 0;
-  for (int i = 1; i < kb.count; ++i)
-    if (blockIdx.x >= kb.t[i].cta_begin) ti = i;
-  const KTensor &tk = kb.t[ti];
-  const uint32_t ctas = (ti + 1 < kb.count ? kb.t[ti + 1].cta_begin : kb.cta_end) - tk.cta_begin;
-  const uint32_t first = blockIdx.x - tk.cta_begin;
-  const int tid = threadIdx.x;
-  if (first >= tk.num_blocks) return;  // uniform: never issued anything
-  bool waited = false;  // for the previous grid (programmatic dependent launch)
-
-  const uint32_t bar0 = smem_addr(&mbar[0]), bar1 = smem_addr(&mbar[1]);
-  uint32_t nP0 = 0, nP1 = 0;  // thread 0: positions of the next block to issue
-  if (tid == 0) {
-    mbar_init(bar0, 1);
-    mbar_init(bar1, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    issue_block<T, C>(tk, first, tk.block_out_pos[first], tk.block_out_pos[first + 1], stages,
-                      &meta[0], bar0, kb.stage_bytes);
-    const uint32_t nb = first + ctas;
-    if (nb < tk.num_blocks) {
-      nP0 = tk.block_out_pos[nb];
-      nP1 = tk.block_out_pos[nb + 1];
-    }
-  }
-
-  // tables (once per thread block): table 0 and lengths rotated, deeper
-  // tables verbatim, then the derived wide table
-  load_tables(tid, T, tk.luts, tk.code_lengths, lut0_s, lens_s);
-  const uint32_t *sub = tk.luts + 256;
-  const uint32_t sub_words = (tk.num_luts - 1) * 256;
-  if (sub_words && sub_words <= kb.sub_words) {
-    for (uint32_t i = tid; i < sub_words; i += T) sub_s[i] = sub[i];
-    sub = sub_s;
-  }
-  for (uint32_t i = tid; i < kb.stage_bytes / 16; i += T)  // zeroed once; each
-    reinterpret_cast<uint4 *>(ex_s)[i] = make_uint4(0, 0, 0, 0);  // output re-zeroes
-  __syncthreads();
-  build_wide<T, 4>(wide_s, lut0_s, lens_s, sub, tk.num_luts);  // its accumulator takes 4
-  __syncthreads();
-
-  const int lane = tid & 31, warp = tid >> 5;
-  uint32_t k = 0;
-  for (uint32_t b = first; b < tk.num_blocks; b += ctas, ++k) {
-    const uint32_t s = k & 1;
-    const uint8_t *stage = stages + s * L::slot_bytes;
-    // queue the next block into the other slot (freed by the barrier that
-    // ended the previous iteration)
-    if (tid == 0 && b + ctas < tk.num_blocks) {
-      issue_block<T, C>(tk, b + ctas, nP0, nP1, stages + (s ^ 1) * L::slot_bytes, &meta[s ^ 1],
-                        s ? bar0 : bar1, kb.stage_bytes);
-      const uint32_t nb = b + 2 * ctas;
-      if (nb < tk.num_blocks) {
-        nP0 = tk.block_out_pos[nb];
-        nP1 = tk.block_out_pos[nb + 1];
-      }
-    }
-    if (tid == 0 && b + ctas >= tk.num_blocks) pdl_launch_dependents();  // last block
-    int bad = 0;
-    if (!mbar_wait(s ? bar1 : bar0, (k >> 1) & 1, kb.spin_limit)) bad = DF11_DEV_ERR_TIMEOUT;
-    const uint4 m = meta[s];
-    const uint32_t P0 = m.x, P1 = m.y, expected = P1 - P0;
-    if (!m.z) {
-      if (tid == 0) report(kb.err, DF11_DEV_ERR_CAPACITY);
-      __syncthreads();
-      continue;
-    }
-    const uint32_t head = P0 & 15u, span = head + expected;
-
-    const uint8_t *bits_s = stage;
-    const uint8_t *gaps_s = stage + L::bits_bytes;
-    // this thread's region, relative to its chunk's first bit: gaps of this
-    // chunk and the next, 10 bits at bit 5*tid of the big-endian gap words
-    const uint64_t chunk_bit = ((uint64_t)b * T + tid) * (uint64_t)(C * 8);
-    int start, end;
-    {
-      const uint32_t bit = 5u * (uint32_t)tid;
-      const uint32_t *g32 = reinterpret_cast<const uint32_t *>(gaps_s) + (bit >> 5);
-      const uint32_t v = __funnelshift_l(__byte_perm(g32[1], 0, 0x0123),
-                                         __byte_perm(g32[0], 0, 0x0123), bit);
-      start = (int)(v >> 27);
-      end = C * 8 + (int)((v >> 22) & 31u);
-    }
-    if (chunk_bit >= tk.total_bits) {
-      start = end = 0;
-    } else if ((uint64_t)end > tk.total_bits - chunk_bit) {
-      end = (int)(tk.total_bits - chunk_bit);
-    }
-    uint32_t w[NW];
-#pragma unroll
-    for (int j = 0; j < NW; ++j) {
-      w[j] = __byte_perm(*reinterpret_cast<const uint32_t *>(bits_s + tid * C + 4 * j), 0, 0x0123);
-      if (tk.masked)  // ones from bit `end` on
-        w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
-    }
-    const uint32_t ex_addr = smem_addr(ex_s);
-
-    // count by decoding into the private slot
-    uint32_t cnt = 0;
-    if (!bad) {
-      const uint32_t slot = smem_addr(slots + tid);
-      if (tk.masked)
-        cnt = decode_chunk<T, C, true>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
-                                       tk.num_luts, slot, kb.slot_words, bad);
-      else
-        cnt = decode_chunk<T, C, false>(w, start, end, smem_addr(wide_s), lut0_s, lens_s, sub,
-                                        tk.num_luts, slot, kb.slot_words, bad);
-    }
-    if (!bad && cnt > tk.max_chunk_elems) bad = DF11_DEV_ERR_CAPACITY;
-
-    // block exclusive scan of the counts: warp totals (bit 31: a thread of
-    // the warp found bad data) to shared memory, one barrier, then every
-    // warp adds up the totals of the warps before it
-    uint32_t incl = cnt;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-      if (lane >= d) incl += v;
-    }
-    const uint32_t warp_bad = __any_sync(0xFFFFFFFFu, bad != 0) ? 0x80000000u : 0u;
-    if (lane == 31) scan[(s << 5) + warp] = (int)(incl | warp_bad);
-    __syncthreads();
-    uint32_t before = 0, total = 0, any_bad = 0;
-#pragma unroll
-    for (int j = 0; j < T / 32; ++j) {
-      const uint32_t v = (uint32_t)scan[(s << 5) + j];
-      any_bad |= v;
-      before += j < warp ? (v & 0x7FFFFFFFu) : 0u;
-      total += v & 0x7FFFFFFFu;
-    }
-    const uint32_t excl = before + incl - cnt;
-    if ((any_bad >> 31) || total != expected) {
-      if (bad) report(kb.err, bad);
-      else if (tid == 0 && !(any_bad >> 31)) report(kb.err, DF11_DEV_ERR_COUNT);
-      continue;  // nothing was written to the exponent array yet
-    }
-
-    const uint32_t d = head + excl;  // my first byte in the exponent array
-    if (cnt) {
-      // compact: slot bytes [0, cnt) -> ex_s[d, d+cnt).  Destination word k
-      // holds slot bytes 4k-s .. 4k-s+3 (s = d & 3): a funnel shift of slot
-      // words k-1 and k.  The first and last words are shared with the
-      // neighbours and merged with OR into the zeroed array.
-      const uint32_t e_end = d + cnt;
-      const uint32_t last = ((e_end - 1) >> 2) - (d >> 2);
-      const uint32_t s8 = (d & 3u) * 8u, r = e_end & 3u;
-      const uint32_t mlast = r ? 0xFFFFFFFFu >> (32u - 8u * r) : 0xFFFFFFFFu;
-      const uint32_t sl = smem_addr(slots + tid);
-      const uint32_t dst = ex_addr + (d & ~3u);
-      uint32_t prev = lds32(sl);
-      if (last == 0) {
-        red_or32(dst, (prev << s8) & mlast);
-      } else {
-        red_or32(dst, prev << s8);
-        for (uint32_t j = 1; j < last; ++j) {  // slot word j <= cnt/4: inside the slot
-          const uint32_t cur = lds32(sl + j * (4u * T));
-          sts32(dst + 4u * j, __funnelshift_l(prev, cur, s8));
-          prev = cur;
-        }
-        const uint32_t cur = lds32(sl + last * (4u * T));
-        red_or32(dst + 4u * last, __funnelshift_l(prev, cur, s8) & mlast);
-      }
-    }
-    if (__syncthreads_or(bad)) {
-      if (bad) report(kb.err, bad);
-      // leave the exponent array zeroed for the next block
-      for (uint32_t i = tid; i < (span + 15u) >> 4; i += T)
-        reinterpret_cast<uint4 *>(ex_s)[i] = make_uint4(0, 0, 0, 0);
-      continue;
-    }
-
-    // output: fuse and store, 16 elements per thread per step; the ragged
-    // first and last groups one element per lane
-    if (!waited) {
-      pdl_wait();
-      waited = true;
-    }
-    {
-      const uint32_t sm_begin = P0 & ~15u;
-      uint16_t *out = tk.out + sm_begin;
-      const uint8_t *smg = tk.sign_mantissa + sm_begin;
-      const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
-      for (uint32_t g = g_begin + tid; g < g_end; g += T) {
-        const uint32_t i0 = g << 4;
-        const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(smg + i0));
-        uint4 *rp = reinterpret_cast<uint4 *>(ex_s + i0);
-        const uint4 rv = *rp;
-        *rp = make_uint4(0, 0, 0, 0);  // leave the array zeroed for the next block
-        const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
-        const uint2 dd = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
-        uint4 *o = reinterpret_cast<uint4 *>(out + i0);
-        o[0] = make_uint4(a.x, a.y, c.x, c.y);
-        o[1] = make_uint4(dd.x, dd.y, f.x, f.y);
-      }
-      if (warp == T / 32 - 1) {  // lanes 0-15: first group, 16-31: last group
-        const uint32_t gl = (span - 1) >> 4;
-        const bool first_partial = head != 0 || span < 16;
-        const bool last_partial = (span & 15u) != 0 && gl != 0;
-        const uint32_t i = lane < 16 ? (uint32_t)lane : (gl << 4) + (uint32_t)(lane - 16);
-        const bool mine = lane < 16 ? first_partial : last_partial;
-        if (mine && i >= head && i < span) out[i] = fuse1(smg[i], ex_s[i]);
-        if (mine) ex_s[i] = 0;
-      }
-    }
-    // No barrier here: the next block's decode writes only private slots,
-    // and the exponent array only after the next scan barrier, which every
-    // thread reaches after finishing this output; the stage slot refilled
-    // next was last read before this block's scan barrier.
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -884,7 +650,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-template <int T, int C, int SM>
+template <int T, int C, int SM, bool COUNTS>
 __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t *slot,
                                          uint32_t full, uint32_t sm_capacity) {
   using L = WsLayout<T, C>;
@@ -907,13 +673,14 @@ __device__ __forceinline__ void ws_issue(const KTensor &tk, uint32_t b, uint8_t 
   }
   const uint32_t sm_begin = P0 & ~15u;
   const uint32_t sm_bytes = ((P1 + 15u) & ~15u) - sm_begin;
-  mbar_arrive_expect_tx(full, L::bits_bytes + L::gaps_bytes + L::counts_bytes +
+  mbar_arrive_expect_tx(full, L::bits_bytes + L::gaps_bytes + (COUNTS ? L::counts_bytes : 0u) +
                                   (SM == kSmSlot ? sm_bytes : 0u));
   bulk_g2s(smem_addr(slot), tk.bitstream + (size_t)b * (T * C), L::bits_bytes, full);
   bulk_g2s(smem_addr(slot + L::bits_bytes), tk.gaps + (size_t)b * (T * 5 / 8), L::gaps_bytes,
            full);
-  bulk_g2s(smem_addr(slot + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
-           L::counts_bytes, full);
+  if (COUNTS)
+    bulk_g2s(smem_addr(slot + L::bits_bytes + L::gaps_bytes), tk.chunk_counts + (size_t)b * T,
+             L::counts_bytes, full);
   if (SM == kSmGlobal) {
     if (sm_bytes) bulk_prefetch_l2(tk.sign_mantissa + sm_begin, sm_bytes);
   } else if (SM == kSmSlot && sm_bytes) {
@@ -1001,7 +768,13 @@ __device__ __forceinline__ void gemv_groups(const KTensor &tk, int lane, uint32_
 // Register budget from the resident thread blocks the shared memory allows:
 // five at 8-byte chunks, at most four from 16 bytes on (more registers there
 // measured about 1% faster) and for the fused matrix-vector product.
-template <int T, int C, int SM, bool GEMV>
+//
+// COUNTS = false decodes the format as the pages state it (no chunk
+// counts): each lane decodes into its own column and counts, the warps of a
+// block exchange their totals (one bounded mbarrier wait per block), and
+// each lane then moves its bytes into the warp's element-order region, from
+// which the output runs as with counts.
+template <int T, int C, int SM, bool GEMV, bool COUNTS = true>
 __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
                                           : ((C >= 16 || GEMV) && T == 256 ? 4 : 1280 / T))
     df11_decode_ws_kernel(const __grid_constant__ KBatch kb) {
@@ -1018,6 +791,8 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
   uint8_t *regions = stages + kWsStages * slot_bytes;
   // kSmWarp: each warp's sign/mantissa buffer (region-sized) follows the regions
   uint8_t *warp_sm = regions + CONSUMERS * kb.stage_bytes;
+  // without counts: each warp's column area (kb.col_bytes) follows
+  uint8_t *columns = warp_sm + (SM == kSmWarp ? CONSUMERS * kb.stage_bytes : 0u);
 
   int ti = 0;
   for (int i = 1; i < kb.count; ++i)
@@ -1028,12 +803,14 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (first >= tk.num_blocks) return;
 
-  // barriers: full[S], empty[S], per-warp (kSmWarp), tables
+  // barriers: full[S], empty[S], per-warp (kSmWarp), tables, and without
+  // counts counted[S] (every consumer warp has posted its total)
   const uint32_t tbar = smem_addr(&bars[2 * kWsStages + 16]);
   if (tid == 0) {
     for (int i = 0; i < kWsStages; ++i) {
       mbar_init(smem_addr(&bars[i]), 1);
       mbar_init(smem_addr(&bars[kWsStages + i]), CONSUMERS);
+      if (!COUNTS) mbar_init(smem_addr(&bars[2 * kWsStages + 17 + i]), CONSUMERS);
     }
     if (SM == kSmWarp)
       for (int i = 0; i < CONSUMERS; ++i) mbar_init(smem_addr(&bars[2 * kWsStages + i]), 1);
@@ -1052,12 +829,15 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
     }
     if (!kb.withhold)
       for (uint32_t b = first; b < tk.num_blocks && issued < kWsStages; b += ctas, ++issued)
-        ws_issue<T, C, SM>(tk, b, stages + issued * slot_bytes, smem_addr(&bars[issued]),
-                           kb.sm_bytes);
+        ws_issue<T, C, SM, COUNTS>(tk, b, stages + issued * slot_bytes,
+                                   smem_addr(&bars[issued]), kb.sm_bytes);
   }
   const uint32_t *sub = tk.luts + 256;  // deeper tables: global memory
   for (uint32_t i = tid; i < CONSUMERS * kb.stage_bytes / 16; i += T + 32)
     reinterpret_cast<uint4 *>(regions)[i] = make_uint4(0, 0, 0, 0);
+  if (!COUNTS)
+    for (uint32_t i = tid; i < CONSUMERS * kb.col_bytes / 16; i += T + 32)
+      reinterpret_cast<uint4 *>(columns)[i] = make_uint4(0, 0, 0, 0);
   bool tables_ok = true;
   if (have_table) {
     tables_ok = mbar_wait(tbar, 0, kb.spin_limit);
@@ -1081,7 +861,8 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
             report(kb.err, DF11_DEV_ERR_TIMEOUT);
             break;
           }
-          ws_issue<T, C, SM>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]), kb.sm_bytes);
+          ws_issue<T, C, SM, COUNTS>(tk, b, stages + s * slot_bytes, smem_addr(&bars[s]),
+                                     kb.sm_bytes);
         }
       }
       pdl_launch_dependents();  // every block of this thread block is queued
@@ -1116,18 +897,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
     const uint32_t counts_sa = slot_sa + L::bits_bytes + L::gaps_bytes;
     const uint4 m = lds128(counts_sa + L::counts_bytes);
     const uint32_t P0 = m.x, P1 = m.y, expected = P1 - P0;
-    uint32_t lsum;
-    if (T == 128) {
-      lsum = __dp4a(lds32(counts_sa + 4u * lane), 0x01010101u, 0u);
-    } else if (T == 256) {
-      const uint2 v = lds64(counts_sa + 8u * lane);
-      lsum = __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u, 0u));
-    } else {
-      const uint4 v = lds128(counts_sa + 16u * lane);
-      lsum = __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u,
-                    __dp4a(v.z, 0x01010101u, __dp4a(v.w, 0x01010101u, 0u))));
-    }
-    const uint32_t cnt = lds8(counts_sa + tid);
+    const uint32_t release = smem_addr(&bars[kWsStages + s]);
     int start, end;
     {
       const uint32_t bit = 5u * (uint32_t)tid;
@@ -1141,19 +911,32 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
 #pragma unroll
     for (int j = 0; j < NW; ++j)
       w[j] = __byte_perm(lds32(slot_sa + (uint32_t)tid * C + 4u * j), 0, 0x0123);
-
-    const uint32_t before = __reduce_add_sync(0xFFFFFFFFu,
-                                              lane < warp * 32 / (T / 32) ? lsum : 0u);
-    const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, lsum);
-    const uint32_t release = smem_addr(&bars[kWsStages + s]);
-    if (!m.z || total != expected ||
-        __any_sync(0xFFFFFFFFu, cnt > tk.max_chunk_elems)) {
-      if (warp == 0 && lane == 0) report(kb.err, m.z ? (total != expected ? DF11_DEV_ERR_COUNT
-                                                                          : DF11_DEV_ERR_CAPACITY)
-                                                     : DF11_DEV_ERR_CAPACITY);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(release);
-      continue;
+    uint32_t cnt, before, incl, warp_total;
+    int bad = 0;
+    if constexpr (COUNTS) {
+      uint32_t lsum;
+      if (T == 128) {
+        lsum = __dp4a(lds32(counts_sa + 4u * lane), 0x01010101u, 0u);
+      } else if (T == 256) {
+        const uint2 v = lds64(counts_sa + 8u * lane);
+        lsum = __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u, 0u));
+      } else {
+        const uint4 v = lds128(counts_sa + 16u * lane);
+        lsum = __dp4a(v.x, 0x01010101u, __dp4a(v.y, 0x01010101u,
+                      __dp4a(v.z, 0x01010101u, __dp4a(v.w, 0x01010101u, 0u))));
+      }
+      cnt = lds8(counts_sa + tid);
+      before = __reduce_add_sync(0xFFFFFFFFu, lane < warp * 32 / (T / 32) ? lsum : 0u);
+      const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, lsum);
+      if (!m.z || total != expected ||
+          __any_sync(0xFFFFFFFFu, cnt > tk.max_chunk_elems)) {
+        if (warp == 0 && lane == 0)
+          report(kb.err, m.z ? (total != expected ? DF11_DEV_ERR_COUNT : DF11_DEV_ERR_CAPACITY)
+                             : DF11_DEV_ERR_CAPACITY);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(release);
+        continue;
+      }
     }
     if (m.w != 0xFFFFFFFFu) {  // the block that holds the end of the stream
       const uint32_t b0 = (uint32_t)tid * (C * 8);
@@ -1169,41 +952,91 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
           w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
       }
     }
-    uint32_t incl = cnt;
+    const uint32_t col = smem_addr(columns + warp * kb.col_bytes) + 4u * lane;  // !COUNTS
+    if constexpr (!COUNTS) {
+      // locate: decode into the lane's column, counting
+      cnt = 0;
+      if (m.z)
+        cnt = tk.masked ? decode_column<C, true>(w, start, end, wide, lut0_s, lens_s, sub,
+                                                 tk.num_luts, col, kb.col_cap, bad)
+                        : decode_column<C, false>(w, start, end, wide, lut0_s, lens_s, sub,
+                                                  tk.num_luts, col, kb.col_cap, bad);
+    }
+    incl = cnt;
 #pragma unroll
     for (int dd = 1; dd < 32; dd <<= 1) {
       const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, dd);
       if (lane >= dd) incl += v;
     }
-    const uint32_t warp_total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-    if (warp_total > tk.max_warp_elems) {  // would not fit the region (uniform)
-      if (lane == 0) report(kb.err, DF11_DEV_ERR_CAPACITY);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(release);
-      continue;
+    warp_total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if constexpr (!COUNTS) {
+      // scan across the block: every warp posts its total (bit 31: a lane
+      // found bad data) in the slot's unused chunk-count bytes, then waits
+      // (bounded) until all have
+      const bool warp_bad = __any_sync(0xFFFFFFFFu, bad != 0);
+      const uint32_t cbar = smem_addr(&bars[2 * kWsStages + 17 + s]);
+      if (lane == 0) {
+        sts32(counts_sa + 4u * warp, warp_total | (warp_bad ? 0x80000000u : 0u));
+        mbar_arrive(cbar);
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(cbar, par, kb.spin_limit))) {
+        if (lane == 0) report(kb.err, DF11_DEV_ERR_TIMEOUT);
+        return;  // whole warp
+      }
+      const uint32_t v = lane < CONSUMERS ? lds32(counts_sa + 4u * lane) : 0u;
+      const uint32_t any_bad = __reduce_or_sync(0xFFFFFFFFu, v) >> 31;
+      before = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? v & 0x7FFFFFFFu : 0u);
+      const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, v & 0x7FFFFFFFu);
+      const bool block_bad = !m.z || any_bad || total != expected;
+      if (block_bad || warp_total > tk.max_warp_elems) {
+        if (bad) {
+          report(kb.err, bad);  // the lane's own finding
+        } else if (lane == 0 && !any_bad) {
+          if (!block_bad)  // this warp's range would not fit its region
+            report(kb.err, DF11_DEV_ERR_CAPACITY);
+          else if (warp == 0)
+            report(kb.err, !m.z || total == expected ? DF11_DEV_ERR_CAPACITY : DF11_DEV_ERR_COUNT);
+        }
+        for (uint32_t j = 0; j < kb.col_bytes / 128u; ++j) sts32(col + 128u * j, 0u);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(release);
+        continue;
+      }
+    } else {
+      if (warp_total > tk.max_warp_elems) {  // would not fit the region (uniform)
+        if (lane == 0) report(kb.err, DF11_DEV_ERR_CAPACITY);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(release);
+        continue;
+      }
     }
     const uint32_t G0 = P0 + before;            // first element of this warp
     const uint32_t head = G0 & 15u, span = head + warp_total;
     const uint32_t d = head + incl - cnt;       // my first byte in the region
     // kSmWarp: the warp's sign/mantissa bytes, elements [G0 & ~15,
     // round16(G0 + warp_total)), inside the block's range, copied while it
-    // decodes; every path below waits for the copy before going on
+    // decodes (or, without counts, while it moves its bytes into place);
+    // every path below waits for the copy before going on
     const uint32_t wsm_bytes = SM == kSmWarp ? (span + 15u) & ~15u : 0u;
     if (SM == kSmWarp && wsm_bytes && lane == 0) {
       mbar_arrive_expect_tx(wbar, wsm_bytes);
       bulk_g2s(wsm, tk.sign_mantissa + (G0 & ~15u), wsm_bytes, wbar);
     }
-    int bad = 0;
-    uint32_t got;
-    if (tk.masked) {
-      got = decode_counted<C>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts, region, d,
-                              cnt, bad);
+    if constexpr (COUNTS) {
+      uint32_t got;
+      if (tk.masked) {
+        got = decode_counted<C>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts, region,
+                                d, cnt, bad);
+      } else {
+        const uint32_t limit = region + ((d + (cnt ? cnt : 1u) - 1u) & ~3u);
+        got = decode_direct<T, C, false>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts,
+                                         region, d, limit, bad);
+      }
+      if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
     } else {
-      const uint32_t limit = region + ((d + (cnt ? cnt : 1u) - 1u) & ~3u);
-      got = decode_direct<T, C, false>(w, start, end, wide, lut0_s, lens_s, sub, tk.num_luts,
-                                       region, d, limit, bad);
+      // reconstruct: the column's bytes to their place in element order
+      column_to_region(col, cnt, region, d);
     }
-    if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
     if (SM == kSmWarp && wsm_bytes) {
       const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(wbar, wph & 1u, kb.spin_limit));
       ++wph;
@@ -1212,7 +1045,7 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
         return;  // whole warp; the buffer may still be written
       }
     }
-    if (__any_sync(0xFFFFFFFFu, bad != 0)) {
+    if (COUNTS && __any_sync(0xFFFFFFFFu, bad != 0)) {
       if (bad) report(kb.err, bad);
       __syncwarp();
       // a counted walk over corrupt data may write up to 7 bytes past `span`
@@ -1333,19 +1166,6 @@ bool supported(uint32_t C, uint32_t T) {
 
 uint32_t stage_bytes_for(uint32_t max_block_elems) {
   return (max_block_elems + 32u + 15u) & ~15u;
-}
-
-uint32_t slot_words_for(uint32_t max_chunk_elems) { return (max_chunk_elems + 3u) / 4u + 1u; }
-
-// Must match the device layout: Layout<T, C>::slot_bytes per stage slot.
-size_t stage_slot_bytes(uint32_t C, uint32_t T) {
-  return (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16;
-}
-
-size_t shared_bytes(uint32_t C, uint32_t T, uint32_t stage, uint32_t slot_words,
-                    uint32_t sub_words) {
-  return (size_t)kOffStages + 2 * stage_slot_bytes(C, T) + stage +
-         (size_t)slot_words * T * 4 + (size_t)sub_words * 4;
 }
 
 bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -1494,34 +1314,22 @@ df11_status prepare(K kern, int threads, size_t smem, int instance, uint64_t &bu
   return DF11_OK;
 }
 
-template <int T, int C>
-df11_status launch(KBatch &kb, const uint32_t *blocks, size_t smem, cudaStream_t s,
-                   int instance) {
-  if (stage_slot_bytes(C, T) != Layout<T, C>::slot_bytes) return DF11_ERR_UNSUPPORTED;
-  auto kern = df11_decode_kernel<T, C>;
-  uint64_t budget = 0;
-  df11_status st = prepare(kern, T, smem, instance, budget);
-  if (st != DF11_OK) return st;
-  const uint32_t grid = split_grid(kb, blocks, budget);
-  return launch_pdl(kern, grid, T, smem, s, kb);
-}
-
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
-                       uint32_t sub_words, bool warp_sm);
+                       uint32_t columns, bool warp_sm);
 
 // Sign/mantissa bytes staged per block in the stage slot or per warp in the
 // warp's own buffer, whichever keeps more thread blocks resident (the slot
 // on a tie); read from global memory only when neither fits.  Measured: at
 // equal residency the slot beats the warp buffer, which beats global reads.
-template <int T, int C, bool GEMV = false>
+template <int T, int C, bool GEMV = false, bool COUNTS = true>
 df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
-  void (*kern[3])(KBatch) = {df11_decode_ws_kernel<T, C, kSmSlot, GEMV>,
-                             df11_decode_ws_kernel<T, C, kSmGlobal, GEMV>,
-                             df11_decode_ws_kernel<T, C, kSmWarp, GEMV>};
-  const size_t smem[3] = {ws_shared_bytes(C, T, sm_stage, kb.stage_bytes, kb.sub_words, false),
-                          ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, false),
-                          ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.sub_words, true)};
+  void (*kern[3])(KBatch) = {df11_decode_ws_kernel<T, C, kSmSlot, GEMV, COUNTS>,
+                             df11_decode_ws_kernel<T, C, kSmGlobal, GEMV, COUNTS>,
+                             df11_decode_ws_kernel<T, C, kSmWarp, GEMV, COUNTS>};
+  const size_t smem[3] = {ws_shared_bytes(C, T, sm_stage, kb.stage_bytes, kb.col_bytes, false),
+                          ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.col_bytes, false),
+                          ws_shared_bytes(C, T, 0, kb.stage_bytes, kb.col_bytes, true)};
   const int order[3] = {kSmSlot, kSmWarp, kSmGlobal};
   uint64_t best = 0;
   int pick = -1;
@@ -1551,11 +1359,19 @@ uint32_t region_bytes_for(uint32_t max_warp_elems) {
   return (15u + max_warp_elems + 8u + 15u) & ~15u;
 }
 
+// Without chunk counts, each warp's column area: the lane's byte j at word
+// (j/4)*32 + lane, for up to the bytes a walk may write (max_chunk_elems,
+// plus the four past it that its last lookup may reach, plus the word the
+// last lookup's bytes spill into).
+uint32_t column_bytes_for(uint32_t max_chunk_elems) {
+  return 128u * ((max_chunk_elems + 3u) / 4u + 1u);
+}
+
 size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t region,
-                       uint32_t sub_words, bool warp_sm) {
+                       uint32_t columns, bool warp_sm) {
   const size_t slot = (size_t)T * C + 16 + (size_t)T * 5 / 8 + 16 + T + 16 + sm_bytes;
-  return (size_t)kOffStages + kWsStages * slot + (size_t)(T / 32) * region * (warp_sm ? 2 : 1) +
-         (size_t)sub_words * 4;
+  return (size_t)kOffStages + kWsStages * slot +
+         (size_t)(T / 32) * ((size_t)region * (warp_sm ? 2 : 1) + columns);
 }
 
 // Test hook (df11_test_withhold_copies): launches left to make with the
@@ -1573,7 +1389,7 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     kb.spin_limit = g_withhold_spin_limit.load();
   }
   uint32_t blocks[DF11_MAX_BATCH];
-  uint32_t max_elems = 0, max_chunk = 0, max_warp = 0, max_luts = 1, C = 0, T = 0;
+  uint32_t max_elems = 0, max_chunk = 0, max_warp = 0, C = 0, T = 0;
   for (int i = 0; i < count; ++i) {
     const df11_params &p = ts[i].params;
     if (p.n == 0) continue;
@@ -1609,26 +1425,22 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     max_elems = max_elems > p.max_block_elems ? max_elems : p.max_block_elems;
     max_chunk = max_chunk > p.max_chunk_elems ? max_chunk : p.max_chunk_elems;
     max_warp = max_warp > p.max_warp_elems ? max_warp : p.max_warp_elems;
-    max_luts = max_luts > p.num_luts ? max_luts : p.num_luts;
     C = p.chunk_bytes;
     T = p.threads_per_block;
   }
   if (kb.count == 0) return DF11_OK;
-  kb.sub_words = (max_luts - 1) <= (uint32_t)kSubTablesInSmem ? (max_luts - 1) * 256 : 0;
+  kb.stage_bytes = region_bytes_for(max_warp);  // bytes of each warp's region
+  // deeper tables only serve codewords longer than the derived table's
+  // index (about one lookup in a thousand): they are read from global
+  // memory, and the shared memory goes to resident thread blocks
+  const uint32_t sm_stage = stage_bytes_for(max_elems);
+  if (ops) {
+    if (T == 256 && C == 8) return launch_ws<256, 8, true>(kb, blocks, sm_stage, s, 12);
+    if (T == 256 && C == 16) return launch_ws<256, 16, true>(kb, blocks, sm_stage, s, 13);
+    if (T == 256 && C == 24) return launch_ws<256, 24, true>(kb, blocks, sm_stage, s, 14);
+    return DF11_ERR_UNSUPPORTED;
+  }
   if (ws) {
-    kb.stage_bytes = region_bytes_for(max_warp);  // bytes of each warp's region
-    kb.slot_words = 0;
-    // deeper tables only serve codewords longer than the derived table's
-    // index (about one lookup in a thousand): read them from global memory
-    // and spend the shared memory on resident thread blocks
-    kb.sub_words = 0;
-    const uint32_t sm_stage = stage_bytes_for(max_elems);
-    if (ops) {
-      if (T == 256 && C == 8) return launch_ws<256, 8, true>(kb, blocks, sm_stage, s, 12);
-      if (T == 256 && C == 16) return launch_ws<256, 16, true>(kb, blocks, sm_stage, s, 13);
-      if (T == 256 && C == 24) return launch_ws<256, 24, true>(kb, blocks, sm_stage, s, 14);
-      return DF11_ERR_UNSUPPORTED;
-    }
     if (T == 256 && C == 8) return launch_ws<256, 8>(kb, blocks, sm_stage, s, 3);
     if (T == 256 && C == 4) return launch_ws<256, 4>(kb, blocks, sm_stage, s, 4);
     if (T == 256 && C == 16) return launch_ws<256, 16>(kb, blocks, sm_stage, s, 5);
@@ -1637,20 +1449,15 @@ df11_status launch_group(const df11_tensor *ts, int count, int32_t *d_err, cudaS
     if (T == 512 && C == 8) return launch_ws<512, 8>(kb, blocks, sm_stage, s, 7);
     return DF11_ERR_UNSUPPORTED;
   }
-  kb.stage_bytes = stage_bytes_for(max_elems);
-  kb.slot_words = slot_words_for(max_chunk);
-  size_t smem = shared_bytes(C, T, kb.stage_bytes, kb.slot_words, kb.sub_words);
-  if (smem > 227 * 1024 && kb.sub_words) {  // drop the deeper tables to global memory
-    kb.sub_words = 0;
-    smem = shared_bytes(C, T, kb.stage_bytes, kb.slot_words, 0);
-  }
-  if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
-  if (T == 256 && C == 8) return launch<256, 8>(kb, blocks, smem, s, 0);
-  if (T == 256 && C == 4) return launch<256, 4>(kb, blocks, smem, s, 1);
-  if (T == 256 && C == 16) return launch<256, 16>(kb, blocks, smem, s, 2);
-  if (T == 256 && C == 24) return launch<256, 24>(kb, blocks, smem, s, 5);
-  if (T == 128 && C == 8) return launch<128, 8>(kb, blocks, smem, s, 3);
-  if (T == 512 && C == 8) return launch<512, 8>(kb, blocks, smem, s, 4);
+  // the format as the pages state it: each lane decodes into its column
+  kb.col_cap = max_chunk;
+  kb.col_bytes = column_bytes_for(max_chunk);
+  if (T == 256 && C == 8) return launch_ws<256, 8, false, false>(kb, blocks, sm_stage, s, 15);
+  if (T == 256 && C == 4) return launch_ws<256, 4, false, false>(kb, blocks, sm_stage, s, 16);
+  if (T == 256 && C == 16) return launch_ws<256, 16, false, false>(kb, blocks, sm_stage, s, 17);
+  if (T == 256 && C == 24) return launch_ws<256, 24, false, false>(kb, blocks, sm_stage, s, 18);
+  if (T == 128 && C == 8) return launch_ws<128, 8, false, false>(kb, blocks, sm_stage, s, 19);
+  if (T == 512 && C == 8) return launch_ws<512, 8, false, false>(kb, blocks, sm_stage, s, 20);
   return DF11_ERR_UNSUPPORTED;
 }
 
@@ -1825,15 +1632,18 @@ df11_status df11_test_withhold_copies(int launches, uint32_t spin_limit) {
 
 size_t df11_shared_bytes(const df11_params *p) {
   if (!p || !supported(p->chunk_bytes, p->threads_per_block)) return 0;
-  const uint32_t subs =
-      p->num_luts - 1 <= (uint32_t)kSubTablesInSmem ? (p->num_luts - 1) * 256 : 0;
-  const size_t page = shared_bytes(p->chunk_bytes, p->threads_per_block,
-                                   stage_bytes_for(p->max_block_elems),
-                                   slot_words_for(p->max_chunk_elems), subs);
-  const size_t ws = ws_shared_bytes(p->chunk_bytes, p->threads_per_block,
-                                    stage_bytes_for(p->max_block_elems),
-                                    region_bytes_for(p->max_warp_elems), 0, false);
-  return page > ws ? page : ws;
+  const uint32_t C = p->chunk_bytes, T = p->threads_per_block;
+  const uint32_t region = region_bytes_for(p->max_warp_elems);
+  const uint32_t stage = stage_bytes_for(p->max_block_elems);
+  const uint32_t cols = column_bytes_for(p->max_chunk_elems);
+  size_t most = 0;  // over both layouts and the three sign/mantissa stagings
+  for (uint32_t c : {0u, cols}) {
+    const size_t v[3] = {ws_shared_bytes(C, T, stage, region, c, false),
+                         ws_shared_bytes(C, T, 0, region, c, false),
+                         ws_shared_bytes(C, T, 0, region, c, true)};
+    for (size_t x : v) most = x > most ? x : most;
+  }
+  return most;
 }
 
 int df11_supported(uint32_t chunk_bytes, uint32_t threads_per_block) {
