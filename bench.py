@@ -47,6 +47,8 @@ import workloads  # noqa: E402
 METRIC = ("decoded BF16 GB/s and % of HBM roofline (1×B200), "
           "bit-exact vs CPU oracle")
 UNIT = "GB/s"
+GEMM_METRIC = ("BF16-equivalent weight GB/s through the fused decode and tensor-core "
+               "matrix product (1×B200), within the fp32 sum bound of the exact product")
 GEMV_METRIC = ("BF16-equivalent weight GB/s through the fused decode and matrix-vector "
                "product (1×B200), within the fp32 sum bound of the exact product")
 BUILD_METRIC = ("compressed BF16 GB/s (device-side format builder, 1×B200), "
@@ -78,7 +80,7 @@ def workload_units(config: str, seed: int):
         return [("embed_151936x4096", lambda d: workloads.embedding(seed, d))]
     if config == "stack":
         return [(name, thunk) for name, _, thunk in workloads.stack_units(seed)]
-    if config in ("build", "gemv"):  # the block's tensors
+    if config in ("build", "gemv", "gemm"):  # the block's tensors
         return workload_units("block", seed)
     if config == "offload":  # the stack's first layers, without embedding and LM head
         return [(name, thunk) for name, _, thunk
@@ -106,7 +108,7 @@ def workload_elements(config: str) -> int:
     """Elements of a workload, from its shapes (no tensor is generated)."""
     block = sum(r * c for _, r, c in workloads.BLOCK_SHAPES)
     emb = workloads.VOCAB * workloads.HIDDEN
-    return {"single": 1 << 20, "block": block, "build": block, "gemv": block,
+    return {"single": 1 << 20, "block": block, "build": block, "gemv": block, "gemm": block,
             "adversarial": 64 << 20, "fibonacci": 14_930_351, "embedding": emb,
             "stack": 2 * emb + workloads.LAYERS * block,
             "offload": OFFLOAD_LAYERS * block}[config]
@@ -845,25 +847,30 @@ def run_gemv(args, world, rank, local):
     device = f"cuda:{local}"
     seed = args.seed + rank
     B = args.batch
-    if not 1 <= B <= 8:
-        raise SystemExit("--batch must be 1..8")
+    tc = args.config == "gemm"  # the tensor-core product (decode_gemm)
+    if not 1 <= B <= (128 if tc else 8):
+        raise SystemExit(f"--batch must be 1..{128 if tc else 8}")
+    # the fused path's format: decode_gemm takes 128 rows interleaved and
+    # 8-byte chunks; decode_gemv the --chunk-bytes and --interleave given
+    fc = args.chunk_bytes if not tc else (args.chunk_bytes if args.chunk_bytes in (8, 16) else 8)
+    fil = 128 if tc else args.interleave
     units = workload_units(args.config, seed)
     shapes = [(r, c) for _, r, c in workloads.BLOCK_SHAPES]
-    hosts, ds, ws_bf16, fused_ds = [], [], [], []
+    ds, ws_bf16, fused_ds = [], [], []
     for (name, thunk), shape in zip(units, shapes):
         bits = thunk(device)
-        h = df11.compress(bits, chunk_bytes=args.chunk_bytes,
-                          threads_per_block=args.threads_per_block)
-        h.shape = shape
-        hosts.append(h)
-        ds.append(df11.to_device(h, device))
-        if args.interleave != 1:  # the fused path's weights, in the interleaved order
-            hi = df11.compress(bits.view(shape), chunk_bytes=args.chunk_bytes,
-                               threads_per_block=args.threads_per_block,
-                               interleave=args.interleave)
-            fused_ds.append(df11.to_device(hi, device))
+        # the two-step path's weights: row-major, the decode's own format
+        d = df11.compress_on_device(bits, chunk_bytes=24 if tc else args.chunk_bytes,
+                                    threads_per_block=args.threads_per_block)
+        d.shape = shape
+        ds.append(d)
+        if fil != 1 or fc != args.chunk_bytes:  # the fused path's weights
+            fused_ds.append(df11.compress_on_device(bits.view(shape), chunk_bytes=fc,
+                                                    threads_per_block=args.threads_per_block,
+                                                    interleave=fil))
         ws_bf16.append(bits.view(shape).view(torch.bfloat16))
-    n_total = sum(h.n for h in hosts)
+    hosts = LazyHosts(ds)
+    n_total = sum(d.n for d in ds)
     g = torch.Generator(device=device)
     g.manual_seed(seed + 77)
     xs = [torch.randn(B, c, generator=g, device=device).to(torch.bfloat16) for _, c in shapes]
@@ -871,9 +878,10 @@ def run_gemv(args, world, rank, local):
     err = df11.new_error_word(device)
     stream = torch.cuda.current_stream()
 
-    fds = fused_ds if args.interleave != 1 else ds
+    fds = fused_ds if fused_ds else ds
+    product = df11.decode_gemm if tc else df11.decode_gemv
     # parity: within gamma_cols * |x||W|^T of the float64 product
-    df11.decode_gemv(fds, xs, ys, err=err)
+    product(fds, xs, ys, err=err)
     torch.cuda.synchronize()
     df11.check_device_error(err)
     for (name, _), (r, c), x, y, w in zip(units, shapes, xs, ys, ws_bf16):
@@ -885,11 +893,11 @@ def run_gemv(args, world, rank, local):
             raise SystemExit(f"gemv outside the fp32 bound on {name}")
         del W, ref, bound
 
-    scratch = torch.empty(max(h.n for h in hosts), dtype=torch.bfloat16, device=device)
+    scratch = torch.empty(max(d.n for d in ds), dtype=torch.bfloat16, device=device)
     plans = [df11.DecodePlan([d], [scratch[: d.n]]) for d in ds]
 
     def fused():
-        df11.decode_gemv(fds, xs, ys, err=err, stream=stream)
+        product(fds, xs, ys, err=err, stream=stream)
 
     ybs = [torch.empty(B, r, dtype=torch.bfloat16, device=device) for r, _ in shapes]
 
@@ -933,21 +941,21 @@ def run_gemv(args, world, rank, local):
         done, secs, what = _oracle_gemv_sample(hosts, shapes, x_host, args.cpu_budget_s)
         cpu = {"value": round(2.0 * done / secs / 1e9, 4), "unit": UNIT, "cores": 1,
                "kind": "oracle", "sample": what + " (bit-serial C decode, float64 product)"}
-    alg = sum(algorithmic_bytes(h) - 2 * h.n for h in hosts) + \
+    alg = sum(algorithmic_bytes(d) - 2 * d.n for d in fds) + \
         sum(x.numel() * 2 for x in xs) + sum(y.numel() * 4 for y in ys)
     achieved = alg / (ms_local * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     if rank == 0:
         line = {
-            "metric": GEMV_METRIC, "value": round(value, 2), "unit": UNIT,
+            "metric": GEMM_METRIC if tc else GEMV_METRIC, "value": round(value, 2), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32",
             "data": "synthetic (seeded; fp32 samples rounded to BF16 RNE)",
             "config": {
                 "workload": WORKLOAD_NAMES[args.config], "tensors": len(units),
-                "elements": n_total, "batch": B, "interleave": args.interleave,
-                "chunk_bytes": args.chunk_bytes,
+                "elements": n_total, "batch": B, "interleave": fil,
+                "chunk_bytes": fc, "two_step_chunk_bytes": 24 if tc else args.chunk_bytes,
                 "threads_per_block": args.threads_per_block,
                 "l2": "inputs larger than L2 (no flush)",
                 "parallelism": f"replicas x{world} (no collective)",
@@ -958,8 +966,10 @@ def run_gemv(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
                          "peak_kind": peak_kind, "algorithmic_bytes_per_step": alg,
-                         "kernel": "df11_decode_ws_kernel (fused product epilogue), one "
-                                   "launch per step for the seven weights"},
+                         "kernel": ("df11_decode_gemm_kernel (decode into shared memory, "
+                                    "tcgen05.mma into tensor memory)" if tc else
+                                    "df11_decode_ws_kernel (fused product epilogue)") +
+                                   ", one launch per step for the seven weights"},
             "decode_then_cublas": {"ms_per_step": round(ms_two, 4),
                                    "value": round(2.0 * n_total / (ms_two * 1e-3) / 1e9, 2)},
             "bf16_cublas": {"ms_per_step": round(ms_bf16, 4),
@@ -1143,7 +1153,7 @@ def run_reference(args, world, rank):
     units = workload_units(args.config, args.seed)
     if args.config == "build":
         return run_reference_build(args, world, units)
-    if args.config == "gemv":
+    if args.config in ("gemv", "gemm"):
         return run_reference_gemv(args, world, units)
     n_total = workload_elements(args.config)
     budget = args.cpu_budget_s / max(1, args.steps + args.warmup)
@@ -1226,7 +1236,8 @@ def run_reference_gemv(args, world, units):
         tot_s += s_
     value = 2.0 * tot_done / tot_s / 1e9
     line = {
-        "impl": "reference", "metric": GEMV_METRIC, "value": round(value, 4), "unit": UNIT,
+        "impl": "reference", "metric": GEMM_METRIC if args.config == "gemm" else GEMV_METRIC,
+        "value": round(value, 4), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u32+f64",
@@ -1288,6 +1299,8 @@ WORKLOAD_NAMES = {
     "stack": "36-layer Qwen3-8B-shaped stack + embedding + LM head, 8,190,427,136 elems",
     "gemv": "fused decode and matrix-vector product: Qwen3-8B-shaped block "
             "(q,k,v,o,gate,up,down), 192,937,984 weights, BF16 activations",
+    "gemm": "fused decode and tensor-core matrix product: Qwen3-8B-shaped block "
+            "(q,k,v,o,gate,up,down), 192,937,984 weights, BF16 activations",
     "build": "format builder on the GPU: Qwen3-8B-shaped block (q,k,v,o,gate,up,down) "
              "compressed from BF16 in HBM, 192,937,984 elems",
     "offload": f"{OFFLOAD_LAYERS} Qwen3-8B-shaped layers streamed from pinned host memory "
@@ -1296,7 +1309,7 @@ WORKLOAD_NAMES = {
 }
 
 
-DEFAULT_STEPS = {"stack": 200, "build": 20, "gemv": 200, "offload": 40}
+DEFAULT_STEPS = {"stack": 200, "build": 20, "gemv": 200, "gemm": 200, "offload": 40}
 
 
 def main(argv=None):
@@ -1349,7 +1362,7 @@ def main(argv=None):
                 run_offload(args, world, rank, local)
             elif args.config == "build":
                 run_build(args, world, rank, local)
-            elif args.config == "gemv":
+            elif args.config in ("gemv", "gemm"):
                 run_gemv(args, world, rank, local)
             else:
                 run_b200(args, world, rank, local)

@@ -150,6 +150,9 @@ def lib():
     L.df11_decode_gemv.argtypes = [ctypes.POINTER(TensorDesc), ctypes.POINTER(GemvOp),
                                    ctypes.c_int, vp, vp]
     L.df11_decode_gemv.restype = ctypes.c_int
+    L.df11_decode_gemm.argtypes = [ctypes.POINTER(TensorDesc), ctypes.POINTER(GemvOp),
+                                   ctypes.c_int, vp, vp]
+    L.df11_decode_gemm.restype = ctypes.c_int
     L.df11_exponent_histogram.argtypes = [vp, u64, vp, vp]
     L.df11_exponent_histogram.restype = ctypes.c_int
     L.df11_test_withhold_copies.argtypes = [ctypes.c_int, u32]
@@ -221,13 +224,14 @@ def _np_copy(ptr, count, dtype):
 
 def interleave_rows(w, rows_per_block: int):
     """The element order df11_gemv calls R rows interleaved (R =
-    rows_per_block): for each block of R rows and each group of 16 columns,
-    the R rows' 16 elements one after another.  Takes a 2-D array or tensor
-    (rows a multiple of R, columns of 16) and returns it flattened in that
-    order."""
+    rows_per_block, a power of two up to 128): for each block of R rows and
+    each group of 16 columns, the R rows' 16 elements one after another.
+    R = 128 makes every 2048 elements one 128 x 16 tile of the tensor-core
+    product (decode_gemm).  Takes a 2-D array or tensor (rows a multiple of
+    R, columns of 16) and returns it flattened in that order."""
     R = int(rows_per_block)
     rows, cols = w.shape
-    if R < 1 or R > 32 or R & (R - 1) or rows % R or cols % 16:
+    if R < 1 or R > 128 or R & (R - 1) or rows % R or cols % 16:
         raise ValueError(f"cannot interleave a {rows}x{cols} matrix by {R} rows")
     v = w.reshape(rows // R, R, cols // 16, 16)
     v = v.permute(0, 2, 1, 3) if isinstance(v, torch.Tensor) else v.transpose(0, 2, 1, 3)
@@ -632,6 +636,34 @@ def decode_gemv(ds: Sequence["Df11Device"], xs: Sequence[torch.Tensor],
         _check(lib().df11_decode_gemv(descs, ops, n,
                                       err.data_ptr() if err is not None else None,
                                       _stream_handle(stream)), "df11_decode_gemv")
+
+
+def decode_gemm(ds: Sequence["Df11Device"], xs: Sequence[torch.Tensor],
+                ys: Sequence[torch.Tensor], accumulate: bool = False,
+                err: Optional[torch.Tensor] = None, stream=None):
+    """y = W x (or y += W x) on the tensor cores for weights W (rows x cols)
+    compressed with interleave=128 (and chunk_bytes 8 or 16) and BF16
+    activations x (batch x cols, batch 1..128) into float32 y (batch x
+    rows), decoding W inside the product (df11_decode_gemm): the BF16
+    weights never reach memory.  One launch for up to 16 weights."""
+    if not (len(ds) == len(xs) == len(ys)):
+        raise ValueError("one x and one y per tensor")
+    n = len(ds)
+    if n == 0:
+        return
+    if n > DF11_MAX_BATCH:
+        raise ValueError(f"at most {DF11_MAX_BATCH} weights per call")
+    for d in ds:
+        if int(getattr(d, "interleave", 1)) != 128:
+            raise ValueError("decode_gemm needs weights compressed with interleave=128")
+    descs = (TensorDesc * n)(*[d.desc(torch.empty(0, device=d.device)) for d in ds])
+    for i in range(n):
+        descs[i].out_bf16 = None
+    ops = (GemvOp * n)(*[_gemv_op(d, x, y, accumulate) for d, x, y in zip(ds, xs, ys)])
+    with torch.cuda.device(_one_device(ds)):
+        _check(lib().df11_decode_gemm(descs, ops, n,
+                                      err.data_ptr() if err is not None else None,
+                                      _stream_handle(stream)), "df11_decode_gemm")
 
 
 def new_error_word(device="cuda") -> torch.Tensor:

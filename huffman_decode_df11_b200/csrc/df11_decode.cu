@@ -1082,6 +1082,9 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
       else
         gemv_groups<SM, DF11_GEMV_MAX_BATCH>(tk, lane, base, g_begin, g_end, sm, region, smg,
                                              cols, nb);
+      // every lane is done with the whole groups (it may have read one that
+      // a ragged lane zeroes next) before the ragged groups are touched
+      __syncwarp();
       if (span) {
         // the elements outside whole groups, one per lane: lanes 0-15 the
         // first group, 16-31 the last one when it is another group
@@ -1120,6 +1123,9 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
           o[1] = make_uint4(e2.x, e2.y, f.x, f.y);
         }
       }
+      // every lane is done with the whole groups (it may have read one that
+      // a ragged lane zeroes next) before the ragged groups are touched
+      __syncwarp();
       if (span) {
         // the elements outside whole groups [g_begin, g_end), one per lane:
         // lanes 0-15 take the first group, 16-31 the last one (the same group
@@ -1133,6 +1139,558 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(release);  // slot free for refill
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused decode and matrix product on the tensor cores (df11_decode_gemm):
+// y[b][r] (+)= sum_c W[r][c] x[b][c] for a batch of BF16 activation rows,
+// with W decoded inside the kernel and never written to memory.
+//
+// W is encoded with 128 rows interleaved per 16 columns (interleave 128), so
+// that the stream holds, per block of 128 rows and per 16-column group, a
+// 128 x 16 tile: the A operand of one tcgen05.mma of M = 128, K = 16.  The
+// work is cut into units of one row block and `kc` consecutive tiles; every
+// thread block takes a contiguous range of units.  Per unit:
+//   - the producer warp stages the format blocks that overlap the unit (as
+//     the decode kernel does; a block at a unit's edge is staged for each of
+//     the two units);
+//   - the consumer warps decode them as the decode kernel does (lanes whose
+//     codewords all lie outside the unit skip their walk) and write the
+//     unit's BF16 weights, 16 bytes at a time, into a ring of A tiles in
+//     shared memory, in the canonical K-major layout without swizzle (8-row
+//     x 16-byte core matrices; K halves 128 bytes apart, 8-row groups 256
+//     bytes apart); then they post the block (mbarrier);
+//   - one MMA warp loads the activation tile of every completed weight tile
+//     (N = batch rounded up to 16 rows x 16 columns, zero rows past the
+//     batch) into the same layout and issues tcgen05.mma into one of two
+//     fp32 accumulators in tensor memory (128 lanes x N columns), then
+//     commits to an mbarrier that the writers of the ring wait on before
+//     they overwrite tiles;
+//   - consecutive units of one row block (a segment) accumulate into one
+//     accumulator; consumer warps 0-3 (one per 32 tensor-memory lanes) move
+//     a finished segment's accumulator to registers (tcgen05.ld) and add it
+//     to y with fp32 atomics, while the next segment accumulates in the
+//     other one.
+// Every wait is bounded (DF11_DEV_ERR_TIMEOUT); no warp leaves early, so
+// the MMA warp frees the tensor memory after a final barrier in every case.
+constexpr int kGemmM = 128;                    // rows of a weight tile (MMA M)
+constexpr uint32_t kGemmTileBytes = 128u * 16u * 2u;  // one 128 x 16 BF16 tile
+
+struct GBatch {
+  KTensor t[DF11_MAX_BATCH];                  // decode fields, x, y, cols, batch, strides
+  uint32_t unit_begin[DF11_MAX_BATCH + 1];    // first unit of each tensor; [count] = all units
+  int32_t *err;
+  int count;
+  uint32_t ctas;         // thread blocks of the launch
+  uint32_t stage_bytes;  // bytes of each consumer warp's exponent region
+  uint32_t kc;           // tiles per unit (the last unit of a row block may have fewer)
+  uint32_t ring;         // A tile (and activation tile) slots
+  uint32_t n_mma;        // N of every MMA: the batch rounded up to 16
+  uint32_t tmem_cols;    // tensor-memory columns allocated (two accumulators)
+  uint32_t spin_limit;
+};
+
+// The unit's place: tensor, element range [u0, u1) of the stream, its row
+// block, its first 16-column group and its tiles.
+struct GUnit {
+  int ti;
+  uint32_t u0, u1, rb, cg0, tiles;
+};
+
+__device__ __forceinline__ GUnit gemm_unit(const GBatch &gb, uint32_t u) {
+  GUnit g;
+  g.ti = 0;
+  for (int i = 1; i < gb.count; ++i)
+    if (u >= gb.unit_begin[i]) g.ti = i;
+  const KTensor &tk = gb.t[g.ti];
+  const uint32_t tpr = tk.cols >> 4;                       // tiles per row block
+  const uint32_t upr = (tpr + gb.kc - 1) / gb.kc;          // units per row block
+  const uint32_t lu = u - gb.unit_begin[g.ti];
+  g.rb = lu / upr;
+  g.cg0 = (lu - g.rb * upr) * gb.kc;
+  g.tiles = min(gb.kc, tpr - g.cg0);
+  g.u0 = (g.rb * tpr + g.cg0) * 2048u;
+  g.u1 = g.u0 + g.tiles * 2048u;
+  return g;
+}
+
+// Format blocks overlapping [u0, u1): the last block starting at or before
+// u0 and the first block whose range reaches u1 (block_out_pos is the
+// positions' ascending table; a corrupt table gives some range inside
+// [0, num_blocks), which the per-block checks then flag).
+__device__ __forceinline__ void gemm_blocks(const KTensor &tk, uint32_t u0, uint32_t u1,
+                                            uint32_t &bf, uint32_t &bl) {
+  uint32_t lo = 0, hi = tk.num_blocks;  // bf: largest b with pos[b] <= u0
+  while (hi - lo > 1) {
+    const uint32_t mid = (lo + hi) >> 1;
+    if (__ldg(tk.block_out_pos + mid) <= u0) lo = mid;
+    else hi = mid;
+  }
+  bf = lo;
+  lo = bf;
+  hi = tk.num_blocks - 1;  // bl: smallest b >= bf with pos[b + 1] >= u1
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi) >> 1;
+    if (__ldg(tk.block_out_pos + mid + 1) >= u1) hi = mid;
+    else lo = mid + 1;
+  }
+  bl = lo;
+}
+
+// Byte offset of weight (r, c) of a 128 x 16 tile in the canonical K-major
+// layout without swizzle.
+__device__ __forceinline__ uint32_t umma_offset(uint32_t r, uint32_t c) {
+  return (r >> 3) * 256u + (c >> 3) * 128u + (r & 7u) * 16u + (c & 7u) * 2u;
+}
+
+// Shared-memory matrix descriptor: K-major, no swizzle, leading (K-half)
+// and stride (8-row group) byte offsets, version 1.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+template <int T, int C>
+__global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __grid_constant__ GBatch gb) {
+  static_assert(T == 256, "eight consumer warps, eight chunk counts per lane");
+  using L = WsLayout<T, C>;
+  constexpr int NW = C / 4 + 1;
+  constexpr int CONSUMERS = T / 32;
+  constexpr int PRODUCER = CONSUMERS, MMA = CONSUMERS + 1;
+  static_assert(CONSUMERS >= 4, "four consumer warps read the accumulator");
+  extern __shared__ __align__(1024) uint8_t gsmem[];
+  uint64_t *bars = reinterpret_cast<uint64_t *>(gsmem);
+  // barriers: full[2] 0-1, empty[2] 2-3, per-warp copies 4.., table, staged[2],
+  // mma_done[2], d_free[2]; the tensor-memory address after them
+  constexpr int kWarpBar = 4, kTableBar = 4 + CONSUMERS, kStaged = kTableBar + 1,
+                kMmaDone = kStaged + 2, kDFree = kMmaDone + 2, kBars = kDFree + 2;
+  static_assert(kBars * 8 + 8 <= (int)kOffLens, "barriers fit below the tables");
+  uint32_t *taddr_s = reinterpret_cast<uint32_t *>(gsmem + kBars * 8);
+  uint8_t *lens_s = gsmem + kOffLens;
+  uint32_t *lut0_s = reinterpret_cast<uint32_t *>(gsmem + kOffLut0);
+  uint2 *wide_s = reinterpret_cast<uint2 *>(gsmem + kOffWide);
+  uint8_t *stages = gsmem + kOffStages;
+  uint8_t *regions = stages + 2 * L::head_bytes;
+  uint8_t *warp_sm = regions + CONSUMERS * gb.stage_bytes;
+  const uint32_t ring_a = smem_addr(gsmem) +
+                          ((kOffStages + 2 * L::head_bytes + 2 * CONSUMERS * gb.stage_bytes + 1023u) &
+                           ~1023u);
+  const uint32_t x_tile_bytes = gb.n_mma * 32u;
+  const uint32_t ring_x = ring_a + gb.ring * kGemmTileBytes;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t ub = (uint32_t)(((uint64_t)blockIdx.x * gb.unit_begin[gb.count]) / gb.ctas);
+  const uint32_t ue = (uint32_t)(((uint64_t)(blockIdx.x + 1) * gb.unit_begin[gb.count]) / gb.ctas);
+  auto bar = [&](int i) { return smem_addr(&bars[i]); };
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(i), 1);
+      mbar_init(bar(2 + i), CONSUMERS);
+      mbar_init(bar(kStaged + i), CONSUMERS);
+      mbar_init(bar(kMmaDone + i), 1);
+      mbar_init(bar(kDFree + i), 4);
+    }
+    for (int i = 0; i < CONSUMERS; ++i) mbar_init(bar(kWarpBar + i), 1);
+    mbar_init(bar(kTableBar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == MMA) {  // tensor memory: two accumulators of n_mma columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(taddr_s)),
+                 "r"(gb.tmem_cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  for (uint32_t i = tid; i < CONSUMERS * gb.stage_bytes / 16; i += T + 64)
+    reinterpret_cast<uint4 *>(regions)[i] = make_uint4(0, 0, 0, 0);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *taddr_s;
+  int32_t *err = gb.err;
+  bool failed = false;  // this thread gave up on a wait: it skips to the end
+
+  // every tensor's decode table: fetched once per unit change of tensor
+  // (units of one thread block are contiguous, so rarely); here, by the
+  // producer before each unit of a new tensor, waited for by everyone
+  // through the table barrier's phase count
+  uint32_t k = 0;  // block instances so far (stage slot k & 1)
+
+  if (warp == PRODUCER) {
+    if (lane == 0) {
+      int cur_t = -1;
+      uint32_t tphase = 0;
+      for (uint32_t u = ub; u < ue && !failed; ++u) {
+        const GUnit g = gemm_unit(gb, u);
+        const KTensor &tk = gb.t[g.ti];
+        if (g.ti != cur_t) {
+          // the table is read by the consumers of the previous unit until
+          // they release its last block: wait for every slot to be free
+          for (uint32_t j = k > 2 ? k - 2 : 0; j < k && !failed; ++j)
+            failed = !mbar_wait(bar(2 + (j & 1)), (j >> 1) & 1u, gb.spin_limit);
+          if (failed) break;
+          mbar_arrive_expect_tx(bar(kTableBar), DF11_DECODE_TABLE_BYTES);
+          bulk_g2s(smem_addr(lens_s), tk.decode_table, DF11_DECODE_TABLE_BYTES, bar(kTableBar));
+          cur_t = g.ti;
+          ++tphase;
+        }
+        uint32_t bf, bl;
+        gemm_blocks(tk, g.u0, g.u1, bf, bl);
+        for (uint32_t b = bf; b <= bl; ++b, ++k) {
+          if (k >= 2 && !mbar_wait(bar(2 + (k & 1)), ((k >> 1) - 1) & 1u, gb.spin_limit)) {
+            failed = true;
+            break;
+          }
+          ws_issue<T, C, kSmWarp, true>(tk, b, stages + (k & 1) * L::head_bytes, bar(k & 1), 0);
+        }
+      }
+      if (failed) report(err, DF11_DEV_ERR_TIMEOUT);
+      pdl_launch_dependents();
+      // no copy of this thread block in flight when it ends
+      for (uint32_t j = k > 2 ? k - 2 : 0; j < k; ++j)
+        if (!mbar_wait(bar(j & 1), (j >> 1) & 1u, gb.spin_limit)) report(err, DF11_DEV_ERR_TIMEOUT);
+      if (tphase && !mbar_wait(bar(kTableBar), (tphase - 1) & 1u, gb.spin_limit))
+        report(err, DF11_DEV_ERR_TIMEOUT);
+    }
+  } else if (warp == MMA) {
+    // idesc: D fp32, A and B BF16, both K-major, N = n_mma, M = 128
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((gb.n_mma >> 3) << 17) |
+                           ((uint32_t)(kGemmM >> 4) << 24);
+    pdl_wait();  // the activations may come from the previous kernel
+    uint32_t t_run = 0;  // tiles of this thread block's units so far (ring position)
+    uint32_t seg = 0, seg_tiles = 0;  // segments so far (accumulator seg & 1), their tiles
+    int prev_ti = -1;
+    uint32_t prev_rb = 0;
+    for (uint32_t u = ub; u < ue && !failed; ++u) {
+      const GUnit g = gemm_unit(gb, u);
+      const KTensor &tk = gb.t[g.ti];
+      uint32_t bf, bl;
+      gemm_blocks(tk, g.u0, g.u1, bf, bl);
+      if (prev_ti >= 0 && (g.ti != prev_ti || g.rb != prev_rb)) {
+        ++seg;  // a new row block: the other accumulator
+        seg_tiles = 0;
+        // flushed two segments ago
+        if (seg >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar(kDFree + (seg & 1)),
+                                                            ((seg >> 1) - 1) & 1u, gb.spin_limit))) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+      }
+      prev_ti = g.ti;
+      prev_rb = g.rb;
+      const uint32_t d_tmem = tmem + (seg & 1) * gb.n_mma;
+      uint32_t done = 0;  // tiles of this unit issued
+      for (uint32_t b = bf; b <= bl; ++b, ++k) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(kStaged + (k & 1)), (k >> 1) & 1u,
+                                                gb.spin_limit))) {
+          failed = true;
+          break;
+        }
+        // the activation slots of this block's tiles held tiles of blocks
+        // up to the previous one: their products must be done
+        if (k >= 1 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar(kMmaDone + ((k - 1) & 1)),
+                                                          ((k - 1) >> 1) & 1u, gb.spin_limit))) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        uint32_t p1 = __ldg(tk.block_out_pos + b + 1);
+        p1 = min(max(p1, g.u0), g.u1);
+        const uint32_t ready = b == bl ? g.tiles : min((p1 - g.u0) >> 11, g.tiles);
+        for (; done < ready; ++done) {
+          // the activation tile of columns [16 cg, 16 cg + 16): K half h of
+          // row n at byte h * 16 * n_mma + 16 n; rows past the batch zero
+          const uint32_t slot = (t_run + done) % gb.ring;
+          const uint32_t xs = ring_x + slot * x_tile_bytes;
+          const uint32_t cg = g.cg0 + done;
+          for (uint32_t p = lane; p < 2u * gb.n_mma; p += 32) {
+            const uint32_t n = p >> 1, h = p & 1u;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (n < tk.batch)
+              v = __ldg(reinterpret_cast<const uint4 *>(tk.x + (size_t)n * tk.x_stride +
+                                                         16u * cg + 8u * h));
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xs + h * 16u * gb.n_mma +
+                                                                            16u * n),
+                         "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                         : "memory");
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            const uint64_t ad = umma_desc(ring_a + slot * kGemmTileBytes, 128u, 256u);
+            const uint64_t bd = umma_desc(xs, 16u * gb.n_mma, 128u);
+            const uint32_t acc = seg_tiles + done > 0 ? 1u : 0u;
+            asm volatile(
+                "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+                "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+                : "memory");
+          }
+          __syncwarp();
+        }
+        if (lane == 0)
+          asm volatile(
+              "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                  bar(kMmaDone + (k & 1)))
+              : "memory");
+        __syncwarp();
+      }
+      t_run += g.tiles;
+      seg_tiles += g.tiles;
+    }
+    if (failed && lane == 0) report(err, DF11_DEV_ERR_TIMEOUT);
+    // no product in flight when the tensor memory goes: its last commit
+    if (k >= 1 && !mbar_wait(bar(kMmaDone + ((k - 1) & 1)), ((k - 1) >> 1) & 1u, gb.spin_limit) &&
+        lane == 0)
+      report(err, DF11_DEV_ERR_TIMEOUT);
+  } else {
+    // ---- consumer warps ----
+    const uint32_t region = smem_addr(regions + warp * gb.stage_bytes);
+    uint8_t *region_p = regions + warp * gb.stage_bytes;
+    const uint32_t wide = smem_addr(wide_s);
+    const uint32_t wsm = smem_addr(warp_sm + warp * gb.stage_bytes);
+    const uint32_t wbar = bar(kWarpBar + warp);
+    uint32_t wph = 0, tphase = 0, t_run = 0, seg = 0;
+    int cur_t = -1;
+    bool waited = false;
+    int32_t flush_seg = -1;  // segment whose accumulator waits to be added to y (warps 0-3)
+    uint32_t flush_rb = 0, flush_k = 0, prev_rb = 0;
+    int flush_ti = 0, prev_ti = -1;
+    auto flush = [&]() {  // warps 0-3: accumulator of segment `flush_seg` into y
+      const KTensor &ft = gb.t[flush_ti];
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(kMmaDone + (flush_k & 1)), (flush_k >> 1) & 1u,
+                                              gb.spin_limit))) {
+        failed = true;
+        return;
+      }
+      tc_fence_after();
+      if (!waited) {
+        pdl_wait();  // y may still be cleared or read by the previous kernel
+        waited = true;
+      }
+      const uint32_t row = flush_rb * kGemmM + 32u * warp + lane;
+      const uint32_t base = tmem + ((32u * warp) << 16) + (flush_seg & 1) * gb.n_mma;
+      for (uint32_t c = 0; c < gb.n_mma; c += 8) {
+        uint32_t v[8];
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                       "=r"(v[6]), "=r"(v[7])
+                     : "r"(base + c)
+                     : "memory");
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (c + j < ft.batch) atomicAdd(ft.y + (size_t)(c + j) * ft.y_stride + row, __uint_as_float(v[j]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kDFree + (flush_seg & 1)));
+      flush_seg = -1;
+    };
+    for (uint32_t u = ub; u < ue && !failed; ++u) {
+      const GUnit g = gemm_unit(gb, u);
+      const KTensor &tk = gb.t[g.ti];
+      if (prev_ti >= 0 && (g.ti != prev_ti || g.rb != prev_rb)) {
+        // the previous segment is complete after its last block instance;
+        // warps 0-3 add it to y during this segment's first block
+        flush_seg = (int32_t)seg;
+        flush_rb = prev_rb;
+        flush_ti = prev_ti;
+        flush_k = k - 1;
+        ++seg;
+      }
+      prev_ti = g.ti;
+      prev_rb = g.rb;
+      if (g.ti != cur_t) {  // this tensor's decode table
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(kTableBar), tphase & 1u, gb.spin_limit))) {
+          failed = true;
+          break;
+        }
+        ++tphase;
+        cur_t = g.ti;
+      }
+      uint32_t bf, bl;
+      gemm_blocks(tk, g.u0, g.u1, bf, bl);
+      for (uint32_t b = bf; b <= bl && !failed; ++b, ++k) {
+        const uint32_t s = k & 1u, par = (k >> 1) & 1u;
+        const uint32_t slot_sa = smem_addr(stages + s * L::head_bytes);
+        const uint32_t release = bar(2 + s);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(s), par, gb.spin_limit))) {
+          failed = true;
+          break;
+        }
+        const uint32_t counts_sa = slot_sa + L::bits_bytes + L::gaps_bytes;
+        const uint4 m = lds128(counts_sa + L::counts_bytes);
+        const uint32_t P0 = m.x, P1 = m.y, expected = P1 - P0;
+        const uint2 cv = lds64(counts_sa + 8u * lane);  // T == 256: 8 counts per lane
+        const uint32_t lsum = __dp4a(cv.x, 0x01010101u, __dp4a(cv.y, 0x01010101u, 0u));
+        const uint32_t cnt = lds8(counts_sa + tid);
+        const uint32_t before = __reduce_add_sync(0xFFFFFFFFu,
+                                                  lane < warp * 32 / CONSUMERS ? lsum : 0u);
+        const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, lsum);
+        bool ok = m.z && total == expected && !__any_sync(0xFFFFFFFFu, cnt > tk.max_chunk_elems);
+        int start, end;
+        {
+          const uint32_t bit = 5u * (uint32_t)tid;
+          const uint32_t ga = slot_sa + L::bits_bytes + 4u * (bit >> 5);
+          const uint32_t v = __funnelshift_l(__byte_perm(lds32(ga + 4u), 0, 0x0123),
+                                             __byte_perm(lds32(ga), 0, 0x0123), bit);
+          start = (int)(v >> 27);
+          end = C * 8 + (int)((v >> 22) & 31u);
+        }
+        if (m.w != 0xFFFFFFFFu) {
+          const uint32_t b0 = (uint32_t)tid * (C * 8);
+          if (b0 >= m.w) start = end = 0;
+          else if ((uint32_t)end > m.w - b0) end = (int)(m.w - b0);
+        }
+        uint32_t w[NW];
+#pragma unroll
+        for (int j = 0; j < NW; ++j) {
+          w[j] = __byte_perm(lds32(slot_sa + (uint32_t)tid * C + 4u * j), 0, 0x0123);
+          if (tk.masked) w[j] |= __funnelshift_rc(0xFFFFFFFFu, 0u, (uint32_t)max(end - 32 * j, 0));
+        }
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int dd = 1; dd < 32; dd <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, dd);
+          if (lane >= dd) incl += v;
+        }
+        const uint32_t warp_total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        ok = ok && warp_total <= tk.max_warp_elems;
+        int bad = 0;
+        const uint32_t G0 = P0 + before;
+        const uint32_t head = G0 & 15u, span = head + warp_total;
+        const uint32_t d = head + incl - cnt;
+        const uint32_t wsm_bytes = ok ? (span + 15u) & ~15u : 0u;
+        if (wsm_bytes && lane == 0) {
+          mbar_arrive_expect_tx(wbar, wsm_bytes);
+          bulk_g2s(wsm, tk.sign_mantissa + (G0 & ~15u), wsm_bytes, wbar);
+        }
+        if (ok) {
+          // lanes whose codewords all lie outside the unit skip their walk
+          const uint32_t e0 = G0 + incl - cnt;
+          const bool inside = cnt && e0 < g.u1 && e0 + cnt > g.u0;
+          uint32_t got = cnt;
+          if (inside) {
+            if (tk.masked)
+              got = decode_counted<C>(w, start, end, wide, lut0_s, lens_s, tk.luts + 256,
+                                      tk.num_luts, region, d, cnt, bad);
+            else
+              got = decode_direct<T, C, false>(w, start, end, wide, lut0_s, lens_s, tk.luts + 256,
+                                               tk.num_luts, region, d,
+                                               region + ((d + cnt - 1u) & ~3u), bad);
+          }
+          if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
+        }
+        if (wsm_bytes) {
+          const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(wbar, wph & 1u, gb.spin_limit));
+          ++wph;
+          if (!landed) {
+            failed = true;
+            break;
+          }
+        }
+        if (!ok || __any_sync(0xFFFFFFFFu, bad != 0)) {
+          if (bad) report(err, bad);
+          else if (lane == 0 && warp == 0) report(err, m.z ? DF11_DEV_ERR_COUNT : DF11_DEV_ERR_CAPACITY);
+          ok = false;
+        }
+        // the ring's tiles that this block writes held tiles of blocks up
+        // to the previous one: their products must be done
+        if (k >= 1 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar(kMmaDone + ((k - 1) & 1)),
+                                                          ((k - 1) >> 1) & 1u, gb.spin_limit))) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        if (flush_seg >= 0 && warp < 4) flush();  // the previous segment's accumulator
+        if (failed) break;
+        __syncwarp();
+        const uint32_t base = G0 & ~15u;
+        if (ok) {
+          // whole 16-element groups inside the unit: row r of tile j, two
+          // 16-byte halves
+          const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
+          for (uint32_t gi = g_begin + lane; gi < g_end; gi += 32) {
+            const uint32_t q = base + 16u * gi;  // first element of the group
+            const uint32_t rv_a = region + 16u * gi;
+            if (q >= g.u0 && q < g.u1) {
+              const uint32_t e = q - g.u0, r = (e >> 4) & 127u;
+              const uint32_t dst = ring_a + ((t_run + (e >> 11)) % gb.ring) * kGemmTileBytes +
+                                   (r >> 3) * 256u + (r & 7u) * 16u;
+              const uint4 sv = lds128(wsm + 16u * gi);
+              const uint4 rv = lds128(rv_a);
+              const uint2 a = fuse4(sv.x, rv.x), c2 = fuse4(sv.y, rv.y);
+              const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(a.x),
+                           "r"(a.y), "r"(c2.x), "r"(c2.y)
+                           : "memory");
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 128u), "r"(e2.x),
+                           "r"(e2.y), "r"(f.x), "r"(f.y)
+                           : "memory");
+            }
+            sts128_zero(rv_a);
+          }
+          // every lane is done with the whole groups (it may have read one that
+          // a ragged lane zeroes next) before the ragged groups are touched
+          __syncwarp();
+          if (span) {  // the ragged first and last groups, one element per lane
+            const uint32_t i = ((uint32_t)lane & 15u) + (lane >> 4 ? ((span - 1) >> 4) << 4 : 0u);
+            const uint32_t q = base + i;
+            if (i >= head && i < span && (i < (g_begin << 4) || i >= (g_end << 4)) && q >= g.u0 &&
+                q < g.u1) {
+              const uint32_t e = q - g.u0;
+              const uint32_t dst = ring_a + ((t_run + (e >> 11)) % gb.ring) * kGemmTileBytes +
+                                   umma_offset((e >> 4) & 127u, e & 15u);
+              const uint16_t v = fuse1(lds8(wsm + i), lds8(region + i));
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst), "h"(v) : "memory");
+            }
+            sts8_zero(region + i);
+          }
+        } else {
+          for (uint32_t i = lane; i < (span + 8u + 15u) >> 4 && 16u * i < gb.stage_bytes; i += 32)
+            reinterpret_cast<uint4 *>(region_p)[i] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();  // the tiles are read by the tensor cores
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(kStaged + s));
+          mbar_arrive(release);
+        }
+      }
+      if (failed) break;
+      t_run += g.tiles;
+    }
+    if (!failed && prev_ti >= 0 && warp < 4) {  // the last segment
+      flush_seg = (int32_t)seg;
+      flush_rb = prev_rb;
+      flush_ti = prev_ti;
+      flush_k = k - 1;
+      flush();
+    }
+    if (failed && lane == 0) report(err, DF11_DEV_ERR_TIMEOUT);
+  }
+  // every warp is here before the tensor memory goes
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(gb.tmem_cols)
+                 : "memory");
   }
 }
 
@@ -1492,6 +2050,34 @@ df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaS
   return st;
 }
 
+// The fused product on tensor cores for up to DF11_MAX_BATCH tensors (one
+// launch): units of one row block and gemm_kc 16-column groups, spread over
+// one wave of thread blocks in contiguous ranges.
+constexpr uint32_t kGemmKc = 32;
+
+template <int C>
+df11_status launch_gemm(GBatch &gb, cudaStream_t s, int instance) {
+  constexpr int T = 256;
+  auto kern = df11_decode_gemm_kernel<T, C>;
+  using L = WsLayout<T, C>;
+  const size_t head = (kOffStages + 2 * L::head_bytes + 2 * (T / 32) * (size_t)gb.stage_bytes +
+                       1023) & ~(size_t)1023;
+  const size_t smem = head + (size_t)gb.ring * (kGemmTileBytes + 32u * gb.n_mma);
+  if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
+  uint64_t budget = 0;
+  const df11_status st = prepare(kern, T + 64, smem, instance, budget);
+  if (st != DF11_OK) return st;
+  // tensor memory: every resident thread block holds tmem_cols of 512 columns
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
+  const uint64_t sms = (uint64_t)device_info(dev).sms;
+  const uint64_t per_sm = budget / sms, tmem_fit = 512u / gb.tmem_cols;
+  budget = sms * (per_sm < tmem_fit ? per_sm : tmem_fit);
+  const uint32_t units = gb.unit_begin[gb.count];
+  gb.ctas = (uint32_t)(units < budget ? units : budget);
+  return launch_pdl(kern, gb.ctas, T + 64, smem, s, gb);
+}
+
 }  // namespace
 
 extern "C" {
@@ -1608,6 +2194,108 @@ df11_status df11_decode_gemv(const df11_tensor *tensors, const df11_gemv *ops, i
     if (st != DF11_OK) return st;
   }
   return DF11_OK;
+}
+
+df11_status df11_decode_gemm(const df11_tensor *tensors, const df11_gemv *ops, int count,
+                             int32_t *d_err, df11_stream_t stream) {
+  if (count < 0 || count > DF11_MAX_BATCH) return count < 0 ? DF11_ERR_INVALID : DF11_ERR_TOO_LARGE;
+  if (count == 0) return DF11_OK;
+  if (!tensors || !ops) return DF11_ERR_NULL;
+  if (d_err && !aligned(d_err, 4)) return DF11_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  GBatch gb{};
+  gb.err = d_err;
+  gb.spin_limit = kSpinLimit;
+  gb.kc = kGemmKc;
+  uint32_t C = 0, max_warp = 0, max_block = 0, max_batch = 0, units = 0;
+  df11_tensor ts[DF11_MAX_BATCH];
+  df11_gemv gs[DF11_MAX_BATCH];
+  int m = 0;
+  for (int i = 0; i < count; ++i) {
+    const df11_tensor &t = tensors[i];
+    const df11_gemv &g = ops[i];
+    const df11_params &p = t.params;
+    if (!g.y || (p.n && !g.x)) return DF11_ERR_NULL;
+    if (g.cols == 0 || g.cols % 16 || p.n % g.cols) return DF11_ERR_INVALID;
+    const uint64_t rows = p.n / g.cols;
+    if (rows % kGemmM || g.interleave != kGemmM) return DF11_ERR_INVALID;
+    if (g.batch < 1 || g.batch > DF11_GEMM_MAX_BATCH) return DF11_ERR_INVALID;
+    if (g.x_stride < g.cols || g.x_stride % 8 || g.y_stride < rows) return DF11_ERR_INVALID;
+    if (!aligned(g.x, 16) || !aligned(g.y, 4)) return DF11_ERR_ALIGN;
+    df11_tensor v = t;
+    v.out_bf16 = reinterpret_cast<uint16_t *>(16);  // not written; passes the output checks
+    const df11_status st = validate(v);
+    if (st != DF11_OK) return st;
+    if (p.n == 0) continue;
+    if (!t.chunk_counts || !t.decode_table) return DF11_ERR_UNSUPPORTED;
+    if (p.threads_per_block != 256 || (p.chunk_bytes != 8 && p.chunk_bytes != 16))
+      return DF11_ERR_UNSUPPORTED;
+    if (C && C != p.chunk_bytes) return DF11_ERR_INVALID;
+    C = p.chunk_bytes;
+    ts[m] = t;
+    gs[m] = g;
+    ++m;
+  }
+  if (m == 0) return DF11_OK;
+  {
+    const df11_status st = check_devices(ts, m, gs);
+    if (st != DF11_OK) return st;
+  }
+  for (int i = 0; i < m; ++i) {
+    const df11_params &p = ts[i].params;
+    KTensor &k = gb.t[i];
+    k.bitstream = ts[i].bitstream;
+    k.gaps = ts[i].gaps;
+    k.chunk_counts = ts[i].chunk_counts;
+    k.block_out_pos = ts[i].block_out_pos;
+    k.luts = ts[i].luts;
+    k.code_lengths = ts[i].code_lengths;
+    k.sign_mantissa = ts[i].sign_mantissa;
+    k.decode_table = ts[i].decode_table;
+    k.total_bits = p.total_bits;
+    k.n = (uint32_t)p.n;
+    k.num_blocks = p.num_blocks;
+    k.num_luts = p.num_luts;
+    k.max_block_elems = p.max_block_elems;
+    k.max_chunk_elems = p.max_chunk_elems;
+    k.max_warp_elems = p.max_warp_elems;
+    k.masked = p.max_len > (uint32_t)kWideBits ? 1u : 0u;
+    k.x = gs[i].x;
+    k.y = gs[i].y;
+    k.cols = gs[i].cols;
+    k.batch = gs[i].batch;
+    k.x_stride = gs[i].x_stride;
+    k.y_stride = gs[i].y_stride;
+    const uint32_t rows = (uint32_t)(p.n / gs[i].cols), tpr = gs[i].cols / 16;
+    gb.unit_begin[i] = units;
+    units += rows / kGemmM * ((tpr + kGemmKc - 1) / kGemmKc);
+    max_warp = max_warp > p.max_warp_elems ? max_warp : p.max_warp_elems;
+    max_block = max_block > p.max_block_elems ? max_block : p.max_block_elems;
+    max_batch = max_batch > gs[i].batch ? max_batch : gs[i].batch;
+  }
+  gb.count = m;
+  gb.unit_begin[m] = units;
+  gb.stage_bytes = region_bytes_for(max_warp);
+  // a block's elements touch at most ceil(max_block / 2048) + 1 tiles; one
+  // more slot so that a block never overwrites the tile it continues
+  gb.ring = (max_block + 2047u) / 2048u + 2u;
+  gb.n_mma = (max_batch + 15u) & ~15u;
+  gb.tmem_cols = 32;
+  while (gb.tmem_cols < 2 * gb.n_mma) gb.tmem_cols <<= 1;
+  // y = W x: clear the outputs first, in stream order
+  ClearArgs ca{};
+  for (int i = 0; i < m; ++i) {
+    if (gs[i].accumulate) continue;
+    ca.y[ca.count] = gs[i].y;
+    ca.rows[ca.count] = (uint32_t)(ts[i].params.n / gs[i].cols);
+    ca.batch[ca.count] = gs[i].batch;
+    ca.stride[ca.count] = gs[i].y_stride;
+    ++ca.count;
+  }
+  if (ca.count && launch_pdl(clear_rows_kernel, 148u, 256u, 0, s, ca) != DF11_OK)
+    return DF11_ERR_CUDA;
+  if (C == 8) return launch_gemm<8>(gb, s, 21);
+  return launch_gemm<16>(gb, s, 22);
 }
 
 df11_status df11_build_decode_table(const uint32_t *luts, const uint8_t *code_lengths,

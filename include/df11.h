@@ -216,6 +216,35 @@ typedef struct df11_gemv {
 df11_status df11_decode_gemv(const df11_tensor *tensors, const df11_gemv *ops, int count,
                              int32_t *d_err, df11_stream_t stream);
 
+/* Largest batch one df11_decode_gemm operation takes. */
+#define DF11_GEMM_MAX_BATCH 128
+
+/*
+ * The same product for batches of activation rows, on the tensor cores: for
+ * each tensor W (rows x cols) and its df11_gemv op, y[b][r] (+)= sum over c
+ * of W[r][c] * x[b][c], with W decoded inside the kernel into shared memory
+ * in 128 x 16 tiles that tcgen05.mma multiplies (BF16 operands, fp32
+ * accumulation in tensor memory); the decoded weights never reach global
+ * memory.  This is the pages' decode right before the matmul
+ * ("DFloat11无损压缩技术" (jsqmd.com) §2.2 item 3: the cost of decoding is
+ * spread over the batch, so the gap to BF16 shrinks as the batch grows;
+ * "DFloat11重新定义LLM无损压缩的技术边界" (ocdem.com) §3.2) for batches
+ * from 1 to DF11_GEMM_MAX_BATCH.
+ * Requirements beyond df11_decode_gemv's: the tensor encoded with 128 rows
+ * interleaved per 16 columns (interleave = 128, rows a multiple of 128),
+ * chunk counts and a decode table present, T = 256 and C = 8 or 16 (the
+ * tile ring and the accumulators must fit one thread block's shared and
+ * tensor memory), at most DF11_MAX_BATCH tensors per call, all of one C.
+ * The sums run in fp32 in an order that depends on the tiling and on
+ * scheduling (atomic adds per 128-row block and K range), within the usual
+ * bound for an fp32 sum of cols terms.  Same conventions as
+ * df11_decode_gemv otherwise.  DF11_ERR_UNSUPPORTED for a tensor without
+ * counts or table or of another chunk size; DF11_ERR_INVALID for a layout,
+ * batch or stride outside the rules.
+ */
+df11_status df11_decode_gemm(const df11_tensor *tensors, const df11_gemv *ops, int count,
+                             int32_t *d_err, df11_stream_t stream);
+
 /*
  * Derive, on the device, the decode table of one tensor from its luts and
  * code_lengths (device pointers, as in df11_tensor) into `out` (device,

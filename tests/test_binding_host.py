@@ -34,7 +34,7 @@ def test_interleave_order_matches_the_definition(rows, cols, R):
 
 
 @pytest.mark.parametrize("shape,R", [((12, 16), 8), ((16, 24), 8), ((16, 16), 3),
-                                     ((64, 16), 64)])
+                                     ((256, 16), 256)])
 def test_interleave_rejects_shapes_it_cannot_take(shape, R):
     with pytest.raises(ValueError):
         df11.interleave_rows(np.zeros(shape, np.uint16), R)
