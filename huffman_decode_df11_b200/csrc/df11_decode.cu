@@ -1150,28 +1150,27 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
 // W is encoded with 128 rows interleaved per 16 columns (interleave 128), so
 // that the stream holds, per block of 128 rows and per 16-column group, a
 // 128 x 16 tile: the A operand of one tcgen05.mma of M = 128, K = 16.  The
-// work is cut into units of one row block and `kc` consecutive tiles; every
-// thread block takes a contiguous range of units.  Per unit:
-//   - the producer warp stages the format blocks that overlap the unit (as
-//     the decode kernel does; a block at a unit's edge is staged for each of
-//     the two units);
+// work is cut into tiles: every thread block takes an equal, contiguous
+// range of the launch's tiles, in pieces of at most one row block.  Per
+// piece:
+//   - the producer warp stages the format blocks that overlap the piece (as
+//     the decode kernel does; a block at a piece's edge is staged for each
+//     of the two pieces);
 //   - the consumer warps decode them as the decode kernel does (lanes whose
-//     codewords all lie outside the unit skip their walk) and write the
-//     unit's BF16 weights, 16 bytes at a time, into a ring of A tiles in
+//     codewords all lie outside the piece skip their walk) and write the
+//     piece's BF16 weights, 16 bytes at a time, into a ring of A tiles in
 //     shared memory, in the canonical K-major layout without swizzle (8-row
 //     x 16-byte core matrices; K halves 128 bytes apart, 8-row groups 256
 //     bytes apart); then they post the block (mbarrier);
 //   - one MMA warp loads the activation tile of every completed weight tile
 //     (N = batch rounded up to 16 rows x 16 columns, zero rows past the
-//     batch) into the same layout and issues tcgen05.mma into one of two
-//     fp32 accumulators in tensor memory (128 lanes x N columns), then
-//     commits to an mbarrier that the writers of the ring wait on before
-//     they overwrite tiles;
-//   - consecutive units of one row block (a segment) accumulate into one
-//     accumulator; consumer warps 0-3 (one per 32 tensor-memory lanes) move
-//     a finished segment's accumulator to registers (tcgen05.ld) and add it
-//     to y with fp32 atomics, while the next segment accumulates in the
-//     other one.
+//     batch; fetched with cp.async one block ahead) into the same layout and
+//     issues tcgen05.mma into one of two fp32 accumulators in tensor memory
+//     (128 lanes x N columns), then commits to an mbarrier that the writers
+//     of the ring wait on before they overwrite tiles;
+//   - consumer warps 0-3 (one per 32 tensor-memory lanes) move a finished
+//     piece's accumulator to registers (tcgen05.ld) and add it to y with
+//     fp32 atomics, while the next piece accumulates in the other one.
 // Every wait is bounded (DF11_DEV_ERR_TIMEOUT); no warp leaves early, so
 // the MMA warp frees the tensor memory after a final barrier in every case.
 constexpr int kGemmM = 128;                    // rows of a weight tile (MMA M)
@@ -1179,38 +1178,38 @@ constexpr uint32_t kGemmTileBytes = 128u * 16u * 2u;  // one 128 x 16 BF16 tile
 
 struct GBatch {
   KTensor t[DF11_MAX_BATCH];                  // decode fields, x, y, cols, batch, strides
-  uint32_t unit_begin[DF11_MAX_BATCH + 1];    // first unit of each tensor; [count] = all units
+  uint32_t tile_begin[DF11_MAX_BATCH + 1];    // first tile of each tensor; [count] = all tiles
   int32_t *err;
   int count;
   uint32_t ctas;         // thread blocks of the launch
   uint32_t stage_bytes;  // bytes of each consumer warp's exponent region
-  uint32_t kc;           // tiles per unit (the last unit of a row block may have fewer)
   uint32_t ring;         // A tile (and activation tile) slots
   uint32_t n_mma;        // N of every MMA: the batch rounded up to 16
   uint32_t tmem_cols;    // tensor-memory columns allocated (two accumulators)
   uint32_t spin_limit;
 };
 
-// The unit's place: tensor, element range [u0, u1) of the stream, its row
-// block, its first 16-column group and its tiles.
+// A piece of a thread block's tile range: the tiles from global tile t on
+// that lie in one row block of one tensor (and below t_end): its tensor, its
+// element range [u0, u1) of that tensor's stream, its row block, its first
+// 16-column group and its tiles.
 struct GUnit {
   int ti;
   uint32_t u0, u1, rb, cg0, tiles;
 };
 
-__device__ __forceinline__ GUnit gemm_unit(const GBatch &gb, uint32_t u) {
+__device__ __forceinline__ GUnit gemm_piece(const GBatch &gb, uint32_t t, uint32_t t_end) {
   GUnit g;
   g.ti = 0;
   for (int i = 1; i < gb.count; ++i)
-    if (u >= gb.unit_begin[i]) g.ti = i;
+    if (t >= gb.tile_begin[i]) g.ti = i;
   const KTensor &tk = gb.t[g.ti];
-  const uint32_t tpr = tk.cols >> 4;                       // tiles per row block
-  const uint32_t upr = (tpr + gb.kc - 1) / gb.kc;          // units per row block
-  const uint32_t lu = u - gb.unit_begin[g.ti];
-  g.rb = lu / upr;
-  g.cg0 = (lu - g.rb * upr) * gb.kc;
-  g.tiles = min(gb.kc, tpr - g.cg0);
-  g.u0 = (g.rb * tpr + g.cg0) * 2048u;
+  const uint32_t tpr = tk.cols >> 4;  // tiles per row block
+  const uint32_t lt = t - gb.tile_begin[g.ti];
+  g.rb = lt / tpr;
+  g.cg0 = lt - g.rb * tpr;
+  g.tiles = min(tpr - g.cg0, t_end - t);
+  g.u0 = lt * 2048u;  // the tiles of a tensor follow one another in its stream
   g.u1 = g.u0 + g.tiles * 2048u;
   return g;
 }
@@ -1262,7 +1261,7 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 template <int T, int C>
-__global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __grid_constant__ GBatch gb) {
+__global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __grid_constant__ GBatch gb) {
   static_assert(T == 256, "eight consumer warps, eight chunk counts per lane");
   using L = WsLayout<T, C>;
   constexpr int NW = C / 4 + 1;
@@ -1290,8 +1289,9 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
   const uint32_t ring_x = ring_a + gb.ring * kGemmTileBytes;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t ub = (uint32_t)(((uint64_t)blockIdx.x * gb.unit_begin[gb.count]) / gb.ctas);
-  const uint32_t ue = (uint32_t)(((uint64_t)(blockIdx.x + 1) * gb.unit_begin[gb.count]) / gb.ctas);
+  // this thread block's tiles: an equal share of all tiles of the launch
+  const uint32_t ub = (uint32_t)(((uint64_t)blockIdx.x * gb.tile_begin[gb.count]) / gb.ctas);
+  const uint32_t ue = (uint32_t)(((uint64_t)(blockIdx.x + 1) * gb.tile_begin[gb.count]) / gb.ctas);
   auto bar = [&](int i) { return smem_addr(&bars[i]); };
 
   if (tid == 0) {
@@ -1315,6 +1315,8 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
   }
   for (uint32_t i = tid; i < CONSUMERS * gb.stage_bytes / 16; i += T + 64)
     reinterpret_cast<uint4 *>(regions)[i] = make_uint4(0, 0, 0, 0);
+  for (uint32_t i = tid; i < gb.ring * x_tile_bytes / 16; i += T + 64)  // activation rows past
+    sts128_zero(ring_x + 16u * i);                                    // the batch stay zero
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1322,21 +1324,21 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
   int32_t *err = gb.err;
   bool failed = false;  // this thread gave up on a wait: it skips to the end
 
-  // every tensor's decode table: fetched once per unit change of tensor
-  // (units of one thread block are contiguous, so rarely); here, by the
-  // producer before each unit of a new tensor, waited for by everyone
-  // through the table barrier's phase count
+  // a tensor's decode table: fetched by the producer before the first piece
+  // of each tensor in this thread block's range (a range is contiguous, so
+  // rarely), waited for by everyone through the table barrier's phases
   uint32_t k = 0;  // block instances so far (stage slot k & 1)
 
   if (warp == PRODUCER) {
     if (lane == 0) {
       int cur_t = -1;
       uint32_t tphase = 0;
-      for (uint32_t u = ub; u < ue && !failed; ++u) {
-        const GUnit g = gemm_unit(gb, u);
+      for (uint32_t u = ub; u < ue && !failed;) {
+        const GUnit g = gemm_piece(gb, u, ue);
+        u += g.tiles;
         const KTensor &tk = gb.t[g.ti];
         if (g.ti != cur_t) {
-          // the table is read by the consumers of the previous unit until
+          // the table is read by the consumers of the previous piece until
           // they release its last block: wait for every slot to be free
           for (uint32_t j = k > 2 ? k - 2 : 0; j < k && !failed; ++j)
             failed = !mbar_wait(bar(2 + (j & 1)), (j >> 1) & 1u, gb.spin_limit);
@@ -1369,12 +1371,27 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
     const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((gb.n_mma >> 3) << 17) |
                            ((uint32_t)(kGemmM >> 4) << 24);
     pdl_wait();  // the activations may come from the previous kernel
-    uint32_t t_run = 0;  // tiles of this thread block's units so far (ring position)
+    uint32_t t_run = 0;  // tiles of this thread block's pieces so far (ring position)
     uint32_t seg = 0, seg_tiles = 0;  // segments so far (accumulator seg & 1), their tiles
     int prev_ti = -1;
     uint32_t prev_rb = 0;
-    for (uint32_t u = ub; u < ue && !failed; ++u) {
-      const GUnit g = gemm_unit(gb, u);
+    // The activation tile of column group cg, rows below the batch (the
+    // rows past it stay zero from the start), into ring slot `slot`: K half
+    // h of row n at byte h * 16 * n_mma + 16 n, by 16-byte asynchronous
+    // copies that land while the consumers decode.
+    auto fetch_x = [&](const KTensor &tk, uint32_t cg, uint32_t slot) {
+      const uint32_t xs = ring_x + slot * x_tile_bytes;
+      for (uint32_t p = lane; p < 2u * tk.batch; p += 32) {
+        const uint32_t n = p >> 1, h = p & 1u;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xs + h * 16u * gb.n_mma +
+                                                                     16u * n),
+                     "l"(tk.x + (size_t)n * tk.x_stride + 16u * cg + 8u * h)
+                     : "memory");
+      }
+    };
+    for (uint32_t u = ub; u < ue && !failed;) {
+      const GUnit g = gemm_piece(gb, u, ue);
+      u += g.tiles;
       const KTensor &tk = gb.t[g.ti];
       uint32_t bf, bl;
       gemm_blocks(tk, g.u0, g.u1, bf, bl);
@@ -1392,46 +1409,36 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
       prev_ti = g.ti;
       prev_rb = g.rb;
       const uint32_t d_tmem = tmem + (seg & 1) * gb.n_mma;
-      uint32_t done = 0;  // tiles of this unit issued
+      // tiles of the piece complete once block b is decoded
+      auto ready_after = [&](uint32_t b) {
+        if (b >= bl) return g.tiles;
+        const uint32_t p1 = min(max(__ldg(tk.block_out_pos + b + 1), g.u0), g.u1);
+        return min((p1 - g.u0) >> 11, g.tiles);
+      };
+      // the first block's activation tiles (every earlier product is done:
+      // each block below waits for its own products before it goes on)
+      uint32_t done = 0, fetched = ready_after(bf);
+      for (uint32_t j = 0; j < fetched; ++j) fetch_x(tk, g.cg0 + j, (t_run + j) % gb.ring);
+      asm volatile("cp.async.commit_group;" ::: "memory");
       for (uint32_t b = bf; b <= bl; ++b, ++k) {
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(kStaged + (k & 1)), (k >> 1) & 1u,
                                                 gb.spin_limit))) {
           failed = true;
           break;
         }
-        // the activation slots of this block's tiles held tiles of blocks
-        // up to the previous one: their products must be done
-        if (k >= 1 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar(kMmaDone + ((k - 1) & 1)),
-                                                          ((k - 1) >> 1) & 1u, gb.spin_limit))) {
-          failed = true;
-          break;
-        }
         tc_fence_after();
-        uint32_t p1 = __ldg(tk.block_out_pos + b + 1);
-        p1 = min(max(p1, g.u0), g.u1);
-        const uint32_t ready = b == bl ? g.tiles : min((p1 - g.u0) >> 11, g.tiles);
-        for (; done < ready; ++done) {
-          // the activation tile of columns [16 cg, 16 cg + 16): K half h of
-          // row n at byte h * 16 * n_mma + 16 n; rows past the batch zero
-          const uint32_t slot = (t_run + done) % gb.ring;
-          const uint32_t xs = ring_x + slot * x_tile_bytes;
-          const uint32_t cg = g.cg0 + done;
-          for (uint32_t p = lane; p < 2u * gb.n_mma; p += 32) {
-            const uint32_t n = p >> 1, h = p & 1u;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (n < tk.batch)
-              v = __ldg(reinterpret_cast<const uint4 *>(tk.x + (size_t)n * tk.x_stride +
-                                                         16u * cg + 8u * h));
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xs + h * 16u * gb.n_mma +
-                                                                            16u * n),
-                         "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                         : "memory");
-          }
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) {
+        const uint32_t ready = ready_after(b);
+        for (uint32_t j = fetched; j < ready; ++j)  // not fetched ahead (inconsistent positions)
+          fetch_x(tk, g.cg0 + j, (t_run + j) % gb.ring);
+        fetched = fetched > ready ? fetched : ready;
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+        fence_proxy_async();  // the activation tiles are read by the tensor cores
+        __syncwarp();
+        if (lane == 0) {
+          for (; done < ready; ++done) {
+            const uint32_t slot = (t_run + done) % gb.ring;
             const uint64_t ad = umma_desc(ring_a + slot * kGemmTileBytes, 128u, 256u);
-            const uint64_t bd = umma_desc(xs, 16u * gb.n_mma, 128u);
+            const uint64_t bd = umma_desc(ring_x + slot * x_tile_bytes, 16u * gb.n_mma, 128u);
             const uint32_t acc = seg_tiles + done > 0 ? 1u : 0u;
             asm volatile(
                 "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -1439,18 +1446,31 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
                 "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
                 : "memory");
           }
-          __syncwarp();
-        }
-        if (lane == 0)
           asm volatile(
               "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                   bar(kMmaDone + (k & 1)))
               : "memory");
-        __syncwarp();
+        }
+        done = __shfl_sync(0xFFFFFFFFu, done, 0);
+        // these products done, their slots take the next block's activation
+        // tiles, which land while the consumers decode it
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(kMmaDone + (k & 1)), (k >> 1) & 1u,
+                                                gb.spin_limit))) {
+          failed = true;
+          ++k;  // this block's commit was made
+          break;
+        }
+        if (b < bl) {
+          const uint32_t next = ready_after(b + 1);
+          for (; fetched < next; ++fetched) fetch_x(tk, g.cg0 + fetched, (t_run + fetched) % gb.ring);
+          asm volatile("cp.async.commit_group;" ::: "memory");
+        }
       }
+      asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight past the piece
       t_run += g.tiles;
       seg_tiles += g.tiles;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (failed && lane == 0) report(err, DF11_DEV_ERR_TIMEOUT);
     // no product in flight when the tensor memory goes: its last commit
     if (k >= 1 && !mbar_wait(bar(kMmaDone + ((k - 1) & 1)), ((k - 1) >> 1) & 1u, gb.spin_limit) &&
@@ -1500,8 +1520,9 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
       if (lane == 0) mbar_arrive(bar(kDFree + (flush_seg & 1)));
       flush_seg = -1;
     };
-    for (uint32_t u = ub; u < ue && !failed; ++u) {
-      const GUnit g = gemm_unit(gb, u);
+    for (uint32_t u = ub; u < ue && !failed;) {
+      const GUnit g = gemm_piece(gb, u, ue);
+      u += g.tiles;
       const KTensor &tk = gb.t[g.ti];
       if (prev_ti >= 0 && (g.ti != prev_ti || g.rb != prev_rb)) {
         // the previous segment is complete after its last block instance;
@@ -1580,7 +1601,7 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
           bulk_g2s(wsm, tk.sign_mantissa + (G0 & ~15u), wsm_bytes, wbar);
         }
         if (ok) {
-          // lanes whose codewords all lie outside the unit skip their walk
+          // lanes whose codewords all lie outside the piece skip their walk
           const uint32_t e0 = G0 + incl - cnt;
           const bool inside = cnt && e0 < g.u1 && e0 + cnt > g.u0;
           uint32_t got = cnt;
@@ -1621,7 +1642,7 @@ __global__ void __launch_bounds__(T + 64, 2) df11_decode_gemm_kernel(const __gri
         __syncwarp();
         const uint32_t base = G0 & ~15u;
         if (ok) {
-          // whole 16-element groups inside the unit: row r of tile j, two
+          // whole 16-element groups inside the piece: row r of tile j, two
           // 16-byte halves
           const uint32_t g_begin = head ? 1u : 0u, g_end = span >> 4;
           for (uint32_t gi = g_begin + lane; gi < g_end; gi += 32) {
@@ -1754,13 +1775,15 @@ df11_status validate(const df11_tensor &t) {
   return DF11_OK;
 }
 
-// Per-device launch state, indexed by kernel instance: the page-layout
-// kernels use 0-5, the warp-specialised ones 3 * i + mode with i = 3-8
-// (decode) and 12-14 (fused matrix-vector product).
+// Per-device launch state, indexed by kernel instance: the warp-specialised
+// kernels use 3 * i + mode with i = 3-8 (decode with counts), 12-14 (fused
+// matrix-vector product) and 15-20 (decode without counts); the
+// tensor-core product 64-65.
+constexpr int kInstances = 80;
 struct DeviceInfo {
   int sms = 0;
-  std::atomic<size_t> configured[64];  // shared-memory limit set, per kernel instance
-  std::atomic<uint64_t> occupancy[64]; // last (smem << 8 | blocks per SM), per instance
+  std::atomic<size_t> configured[kInstances];  // shared-memory limit set, per kernel instance
+  std::atomic<uint64_t> occupancy[kInstances]; // last (smem << 8 | blocks per SM), per instance
 };
 
 DeviceInfo &device_info(int dev) {
@@ -1849,9 +1872,14 @@ df11_status prepare(K kern, int threads, size_t smem, int instance, uint64_t &bu
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
   DeviceInfo &di = device_info(dev);
+  if (instance < 0 || instance >= kInstances) return DF11_ERR_INVALID;
   if (smem > 48 * 1024 && di.configured[instance].load() < smem) {
+    // all of the unified L1 as shared memory: these kernels keep their
+    // working set there, and the occupancy query assumes this split
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+            cudaSuccess)
       return DF11_ERR_CUDA;
     di.configured[instance].store(smem);
   }
@@ -2051,9 +2079,8 @@ df11_status launch_batch(const df11_tensor *ts, int count, int32_t *d_err, cudaS
 }
 
 // The fused product on tensor cores for up to DF11_MAX_BATCH tensors (one
-// launch): units of one row block and gemm_kc 16-column groups, spread over
-// one wave of thread blocks in contiguous ranges.
-constexpr uint32_t kGemmKc = 32;
+// launch): the launch's tiles spread over one wave of thread blocks in
+// equal contiguous ranges.
 
 template <int C>
 df11_status launch_gemm(GBatch &gb, cudaStream_t s, int instance) {
@@ -2062,19 +2089,43 @@ df11_status launch_gemm(GBatch &gb, cudaStream_t s, int instance) {
   using L = WsLayout<T, C>;
   const size_t head = (kOffStages + 2 * L::head_bytes + 2 * (T / 32) * (size_t)gb.stage_bytes +
                        1023) & ~(size_t)1023;
-  const size_t smem = head + (size_t)gb.ring * (kGemmTileBytes + 32u * gb.n_mma);
+  size_t smem = head + (size_t)gb.ring * (kGemmTileBytes + 32u * gb.n_mma);
   if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
-  uint64_t budget = 0;
-  const df11_status st = prepare(kern, T + 64, smem, instance, budget);
-  if (st != DF11_OK) return st;
-  // tensor memory: every resident thread block holds tmem_cols of 512 columns
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
-  const uint64_t sms = (uint64_t)device_info(dev).sms;
-  const uint64_t per_sm = budget / sms, tmem_fit = 512u / gb.tmem_cols;
-  budget = sms * (per_sm < tmem_fit ? per_sm : tmem_fit);
-  const uint32_t units = gb.unit_begin[gb.count];
-  gb.ctas = (uint32_t)(units < budget ? units : budget);
+  // Resident thread blocks per SM, from the kernel's registers and shared
+  // memory and the SM's limits; and tensor memory: each resident block
+  // holds tmem_cols of the SM's 512 columns.  When tensor memory allows
+  // fewer blocks than the rest, the launch asks for more shared memory than
+  // it uses, so that no SM takes more blocks than its tensor memory holds
+  // (an allocation would otherwise wait for a neighbour to finish).
+  cudaFuncAttributes fa{};
+  int smem_sm = 0, regs_sm = 0, reserved = 0;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+          cudaSuccess)
+    return DF11_ERR_CUDA;
+  const uint64_t regs_block = (uint64_t)((fa.numRegs + 7) & ~7) * (T + 64);
+  uint64_t per_sm = (uint64_t)smem_sm / (smem + (size_t)reserved);
+  if (regs_block && (uint64_t)regs_sm / regs_block < per_sm) per_sm = (uint64_t)regs_sm / regs_block;
+  if (2048u / (T + 64) < per_sm) per_sm = 2048u / (T + 64);
+  const uint64_t tmem_fit = 512u / gb.tmem_cols;
+  if (tmem_fit < per_sm) {
+    per_sm = tmem_fit;
+    const size_t want = ((size_t)smem_sm / per_sm - (size_t)reserved) & ~(size_t)127;
+    if (want > smem) smem = want < 227 * 1024 ? want : 227 * 1024;
+  }
+  if (per_sm < 1) return DF11_ERR_TOO_LARGE;
+  uint64_t budget = 0;  // prepare() sets the kernel's shared-memory limit; its count is not used
+  const df11_status st = prepare(kern, T + 64, smem, instance, budget);
+  if (st != DF11_OK && st != DF11_ERR_TOO_LARGE) return st;
+  budget = (uint64_t)device_info(dev).sms * per_sm;
+  const uint32_t tiles = gb.tile_begin[gb.count];
+  gb.ctas = (uint32_t)(tiles < budget ? tiles : budget);
   return launch_pdl(kern, gb.ctas, T + 64, smem, s, gb);
 }
 
@@ -2206,8 +2257,7 @@ df11_status df11_decode_gemm(const df11_tensor *tensors, const df11_gemv *ops, i
   GBatch gb{};
   gb.err = d_err;
   gb.spin_limit = kSpinLimit;
-  gb.kc = kGemmKc;
-  uint32_t C = 0, max_warp = 0, max_block = 0, max_batch = 0, units = 0;
+  uint32_t C = 0, max_warp = 0, max_block = 0, max_batch = 0, tiles = 0;
   df11_tensor ts[DF11_MAX_BATCH];
   df11_gemv gs[DF11_MAX_BATCH];
   int m = 0;
@@ -2267,18 +2317,18 @@ df11_status df11_decode_gemm(const df11_tensor *tensors, const df11_gemv *ops, i
     k.x_stride = gs[i].x_stride;
     k.y_stride = gs[i].y_stride;
     const uint32_t rows = (uint32_t)(p.n / gs[i].cols), tpr = gs[i].cols / 16;
-    gb.unit_begin[i] = units;
-    units += rows / kGemmM * ((tpr + kGemmKc - 1) / kGemmKc);
+    gb.tile_begin[i] = tiles;
+    tiles += rows / kGemmM * tpr;
     max_warp = max_warp > p.max_warp_elems ? max_warp : p.max_warp_elems;
     max_block = max_block > p.max_block_elems ? max_block : p.max_block_elems;
     max_batch = max_batch > gs[i].batch ? max_batch : gs[i].batch;
   }
   gb.count = m;
-  gb.unit_begin[m] = units;
+  gb.tile_begin[m] = tiles;
   gb.stage_bytes = region_bytes_for(max_warp);
-  // a block's elements touch at most ceil(max_block / 2048) + 1 tiles; one
-  // more slot so that a block never overwrites the tile it continues
-  gb.ring = (max_block + 2047u) / 2048u + 2u;
+  // a block's elements touch at most ceil(max_block / 2048) + 1 tiles (one
+  // of them the tile the block before it began); the ring holds them
+  gb.ring = (max_block + 2047u) / 2048u + 1u;
   gb.n_mma = (max_batch + 15u) & ~15u;
   gb.tmem_cols = 32;
   while (gb.tmem_cols < 2 * gb.n_mma) gb.tmem_cols <<= 1;
@@ -2294,8 +2344,8 @@ df11_status df11_decode_gemm(const df11_tensor *tensors, const df11_gemv *ops, i
   }
   if (ca.count && launch_pdl(clear_rows_kernel, 148u, 256u, 0, s, ca) != DF11_OK)
     return DF11_ERR_CUDA;
-  if (C == 8) return launch_gemm<8>(gb, s, 21);
-  return launch_gemm<16>(gb, s, 22);
+  if (C == 8) return launch_gemm<8>(gb, s, 64);
+  return launch_gemm<16>(gb, s, 65);
 }
 
 df11_status df11_build_decode_table(const uint32_t *luts, const uint8_t *code_lengths,
