@@ -1261,7 +1261,7 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 template <int T, int C>
-__global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __grid_constant__ GBatch gb) {
+__global__ void __launch_bounds__(T + 64, 4) df11_decode_gemm_kernel(const __grid_constant__ GBatch gb) {
   static_assert(T == 256, "eight consumer warps, eight chunk counts per lane");
   using L = WsLayout<T, C>;
   constexpr int NW = C / 4 + 1;
@@ -1270,9 +1270,9 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
   static_assert(CONSUMERS >= 4, "four consumer warps read the accumulator");
   extern __shared__ __align__(1024) uint8_t gsmem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(gsmem);
-  // barriers: full[2] 0-1, empty[2] 2-3, per-warp copies 4.., table, staged[2],
-  // mma_done[2], d_free[2]; the tensor-memory address after them
-  constexpr int kWarpBar = 4, kTableBar = 4 + CONSUMERS, kStaged = kTableBar + 1,
+  // barriers: full[2] 0-1, empty[2] 2-3, table, staged[2], mma_done[2],
+  // d_free[2]; the tensor-memory address after them
+  constexpr int kTableBar = 4, kStaged = kTableBar + 1,
                 kMmaDone = kStaged + 2, kDFree = kMmaDone + 2, kBars = kDFree + 2;
   static_assert(kBars * 8 + 8 <= (int)kOffLens, "barriers fit below the tables");
   uint32_t *taddr_s = reinterpret_cast<uint32_t *>(gsmem + kBars * 8);
@@ -1281,9 +1281,8 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
   uint2 *wide_s = reinterpret_cast<uint2 *>(gsmem + kOffWide);
   uint8_t *stages = gsmem + kOffStages;
   uint8_t *regions = stages + 2 * L::head_bytes;
-  uint8_t *warp_sm = regions + CONSUMERS * gb.stage_bytes;
   const uint32_t ring_a = smem_addr(gsmem) +
-                          ((kOffStages + 2 * L::head_bytes + 2 * CONSUMERS * gb.stage_bytes + 1023u) &
+                          ((kOffStages + 2 * L::head_bytes + CONSUMERS * gb.stage_bytes + 1023u) &
                            ~1023u);
   const uint32_t x_tile_bytes = gb.n_mma * 32u;
   const uint32_t ring_x = ring_a + gb.ring * kGemmTileBytes;
@@ -1302,7 +1301,6 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
       mbar_init(bar(kMmaDone + i), 1);
       mbar_init(bar(kDFree + i), 4);
     }
-    for (int i = 0; i < CONSUMERS; ++i) mbar_init(bar(kWarpBar + i), 1);
     mbar_init(bar(kTableBar), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1355,7 +1353,8 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
             failed = true;
             break;
           }
-          ws_issue<T, C, kSmWarp, true>(tk, b, stages + (k & 1) * L::head_bytes, bar(k & 1), 0);
+          // the block's sign/mantissa bytes stay in global memory, prefetched to L2
+          ws_issue<T, C, kSmGlobal, true>(tk, b, stages + (k & 1) * L::head_bytes, bar(k & 1), 0);
         }
       }
       if (failed) report(err, DF11_DEV_ERR_TIMEOUT);
@@ -1481,9 +1480,7 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
     const uint32_t region = smem_addr(regions + warp * gb.stage_bytes);
     uint8_t *region_p = regions + warp * gb.stage_bytes;
     const uint32_t wide = smem_addr(wide_s);
-    const uint32_t wsm = smem_addr(warp_sm + warp * gb.stage_bytes);
-    const uint32_t wbar = bar(kWarpBar + warp);
-    uint32_t wph = 0, tphase = 0, t_run = 0, seg = 0;
+    uint32_t tphase = 0, t_run = 0, seg = 0;
     int cur_t = -1;
     bool waited = false;
     int32_t flush_seg = -1;  // segment whose accumulator waits to be added to y (warps 0-3)
@@ -1595,11 +1592,6 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
         const uint32_t G0 = P0 + before;
         const uint32_t head = G0 & 15u, span = head + warp_total;
         const uint32_t d = head + incl - cnt;
-        const uint32_t wsm_bytes = ok ? (span + 15u) & ~15u : 0u;
-        if (wsm_bytes && lane == 0) {
-          mbar_arrive_expect_tx(wbar, wsm_bytes);
-          bulk_g2s(wsm, tk.sign_mantissa + (G0 & ~15u), wsm_bytes, wbar);
-        }
         if (ok) {
           // lanes whose codewords all lie outside the piece skip their walk
           const uint32_t e0 = G0 + incl - cnt;
@@ -1615,14 +1607,6 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
                                                region + ((d + cnt - 1u) & ~3u), bad);
           }
           if (!bad && got != cnt) bad = DF11_DEV_ERR_COUNT;
-        }
-        if (wsm_bytes) {
-          const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(wbar, wph & 1u, gb.spin_limit));
-          ++wph;
-          if (!landed) {
-            failed = true;
-            break;
-          }
         }
         if (!ok || __any_sync(0xFFFFFFFFu, bad != 0)) {
           if (bad) report(err, bad);
@@ -1641,6 +1625,7 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
         if (failed) break;
         __syncwarp();
         const uint32_t base = G0 & ~15u;
+        const uint8_t *smg = tk.sign_mantissa + base;  // this warp's sign/mantissa bytes
         if (ok) {
           // whole 16-element groups inside the piece: row r of tile j, two
           // 16-byte halves
@@ -1652,7 +1637,7 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
               const uint32_t e = q - g.u0, r = (e >> 4) & 127u;
               const uint32_t dst = ring_a + ((t_run + (e >> 11)) % gb.ring) * kGemmTileBytes +
                                    (r >> 3) * 256u + (r & 7u) * 16u;
-              const uint4 sv = lds128(wsm + 16u * gi);
+              const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(smg) + gi);
               const uint4 rv = lds128(rv_a);
               const uint2 a = fuse4(sv.x, rv.x), c2 = fuse4(sv.y, rv.y);
               const uint2 e2 = fuse4(sv.z, rv.z), f = fuse4(sv.w, rv.w);
@@ -1676,7 +1661,7 @@ __global__ void __launch_bounds__(T + 64, 3) df11_decode_gemm_kernel(const __gri
               const uint32_t e = q - g.u0;
               const uint32_t dst = ring_a + ((t_run + (e >> 11)) % gb.ring) * kGemmTileBytes +
                                    umma_offset((e >> 4) & 127u, e & 15u);
-              const uint16_t v = fuse1(lds8(wsm + i), lds8(region + i));
+              const uint16_t v = fuse1(__ldg(smg + i), lds8(region + i));
               asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst), "h"(v) : "memory");
             }
             sts8_zero(region + i);
@@ -2087,7 +2072,7 @@ df11_status launch_gemm(GBatch &gb, cudaStream_t s, int instance) {
   constexpr int T = 256;
   auto kern = df11_decode_gemm_kernel<T, C>;
   using L = WsLayout<T, C>;
-  const size_t head = (kOffStages + 2 * L::head_bytes + 2 * (T / 32) * (size_t)gb.stage_bytes +
+  const size_t head = (kOffStages + 2 * L::head_bytes + (T / 32) * (size_t)gb.stage_bytes +
                        1023) & ~(size_t)1023;
   size_t smem = head + (size_t)gb.ring * (kGemmTileBytes + 32u * gb.n_mma);
   if (smem > 227 * 1024) return DF11_ERR_TOO_LARGE;
