@@ -105,6 +105,8 @@ struct KBatch {
                          // consumers' waits run out (df11_test_withhold_copies)
   uint32_t col_bytes;    // without chunk counts: bytes of each warp's column area
   uint32_t col_cap;      // without chunk counts: most bytes a column takes (max_chunk_elems)
+  uint32_t sub_bytes;    // room for a tensor's deeper tables in shared memory (0: read from
+                         // global memory); tensors whose tables do not fit read them there
 };
 
 // ---- shared memory layout --------------------------------------------------
@@ -793,6 +795,8 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
   uint8_t *warp_sm = regions + CONSUMERS * kb.stage_bytes;
   // without counts: each warp's column area (kb.col_bytes) follows
   uint8_t *columns = warp_sm + (SM == kSmWarp ? CONSUMERS * kb.stage_bytes : 0u);
+  // the tensor's deeper tables (codewords longer than 8 bits), when room was left
+  uint32_t *subs_s = reinterpret_cast<uint32_t *>(columns + CONSUMERS * kb.col_bytes);
 
   int ti = 0;
   for (int i = 1; i < kb.count; ++i)
@@ -821,18 +825,26 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
   // the producer queues the decode table and the first blocks before
   // anything else, so that they arrive while the tables are set up
   const bool have_table = tk.decode_table != nullptr;
+  // the tensor's deeper tables come into shared memory with its decode table
+  // when the launch left room for them
+  const uint32_t sub_bytes = have_table && tk.num_luts > 1 &&
+                                     (tk.num_luts - 1) * 1024u <= kb.sub_bytes
+                                 ? (tk.num_luts - 1) * 1024u
+                                 : 0u;
   uint32_t issued = 0;
   if (warp == CONSUMERS && lane == 0) {
     if (have_table) {
-      mbar_arrive_expect_tx(tbar, DF11_DECODE_TABLE_BYTES);
+      mbar_arrive_expect_tx(tbar, DF11_DECODE_TABLE_BYTES + sub_bytes);
       bulk_g2s(smem_addr(lens_s), tk.decode_table, DF11_DECODE_TABLE_BYTES, tbar);
+      if (sub_bytes) bulk_g2s(smem_addr(subs_s), tk.luts + 256, sub_bytes, tbar);
     }
     if (!kb.withhold)
       for (uint32_t b = first; b < tk.num_blocks && issued < kWsStages; b += ctas, ++issued)
         ws_issue<T, C, SM, COUNTS>(tk, b, stages + issued * slot_bytes,
                                    smem_addr(&bars[issued]), kb.sm_bytes);
   }
-  const uint32_t *sub = tk.luts + 256;  // deeper tables: global memory
+  // deeper tables: in shared memory when they came with the decode table
+  const uint32_t *sub = sub_bytes ? subs_s : tk.luts + 256;
   for (uint32_t i = tid; i < CONSUMERS * kb.stage_bytes / 16; i += T + 32)
     reinterpret_cast<uint4 *>(regions)[i] = make_uint4(0, 0, 0, 0);
   if (!COUNTS)
@@ -1768,7 +1780,8 @@ constexpr int kInstances = 80;
 struct DeviceInfo {
   int sms = 0;
   std::atomic<size_t> configured[kInstances];  // shared-memory limit set, per kernel instance
-  std::atomic<uint64_t> occupancy[kInstances]; // last (smem << 8 | blocks per SM), per instance
+  // (smem << 8 | blocks per SM) of the last two shared-memory sizes, per instance
+  std::atomic<uint64_t> occupancy[kInstances][2];
 };
 
 DeviceInfo &device_info(int dev) {
@@ -1871,14 +1884,18 @@ df11_status prepare(K kern, int threads, size_t smem, int instance, uint64_t &bu
   // occupancy queries cost microseconds of host time: one per instance and
   // shared-memory size (a layer-by-layer decode loop repeats the sizes)
   int per_sm = 0;
-  const uint64_t cached = di.occupancy[instance].load();
-  if (cached && (cached >> 8) == (uint64_t)smem) {
-    per_sm = (int)(cached & 0xFF);
+  const uint64_t c0 = di.occupancy[instance][0].load(), c1 = di.occupancy[instance][1].load();
+  if (c0 && (c0 >> 8) == (uint64_t)smem) {
+    per_sm = (int)(c0 & 0xFF);
+  } else if (c1 && (c1 >> 8) == (uint64_t)smem) {
+    per_sm = (int)(c1 & 0xFF);
   } else {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) !=
         cudaSuccess)
       return DF11_ERR_CUDA;
-    di.occupancy[instance].store(((uint64_t)smem << 8) | (uint64_t)(per_sm & 0xFF));
+    // keep the most recent size in slot 0, the one before in slot 1
+    di.occupancy[instance][1].store(c0);
+    di.occupancy[instance][0].store(((uint64_t)smem << 8) | (uint64_t)(per_sm & 0xFF));
   }
   if (per_sm < 1) return DF11_ERR_TOO_LARGE;
   budget = (uint64_t)di.sms * per_sm;
@@ -1895,6 +1912,10 @@ size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t regio
 template <int T, int C, bool GEMV = false, bool COUNTS = true>
 df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
+  uint32_t sub_need = 0;  // bytes of the largest set of deeper tables of the launch
+  for (int i = 0; i < kb.count; ++i)
+    if (kb.t[i].num_luts > 1 && (kb.t[i].num_luts - 1) * 1024u > sub_need)
+      sub_need = (kb.t[i].num_luts - 1) * 1024u;
   void (*kern[3])(KBatch) = {df11_decode_ws_kernel<T, C, kSmSlot, GEMV, COUNTS>,
                              df11_decode_ws_kernel<T, C, kSmGlobal, GEMV, COUNTS>,
                              df11_decode_ws_kernel<T, C, kSmWarp, GEMV, COUNTS>};
@@ -1917,8 +1938,32 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
   }
   if (pick < 0) return DF11_ERR_TOO_LARGE;
   kb.sm_bytes = pick == kSmSlot ? sm_stage : 0u;
+  // the deeper tables (read on codewords longer than the derived table's
+  // index) in shared memory too, when they fit in what the resident blocks
+  // leave of the SM's shared memory
+  size_t use = smem[pick];
+  kb.sub_bytes = 0;
+  if (sub_need && kb.col_bytes == 0) {
+    int dev = 0, smem_sm = 0, reserved = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+            cudaSuccess &&
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) ==
+            cudaSuccess) {
+      const uint64_t per_sm = best / (uint64_t)device_info(dev).sms;
+      if (per_sm && use + sub_need + (size_t)reserved <= (size_t)smem_sm / per_sm &&
+          use + sub_need <= 227 * 1024) {
+        uint64_t b2 = 0;
+        const df11_status st = prepare(kern[pick], T + 32, use + sub_need, 3 * instance + pick, b2);
+        if (st == DF11_OK && b2 == best) {
+          kb.sub_bytes = sub_need;
+          use += sub_need;
+        }
+      }
+    }
+  }
   const uint32_t grid = split_grid(kb, blocks, best);
-  return launch_pdl(kern[pick], grid, T + 32, smem[pick], s, kb);
+  return launch_pdl(kern[pick], grid, T + 32, use, s, kb);
 }
 
 // Per-warp exponent region of the warp-specialised kernel: the warp's head
