@@ -1177,7 +1177,8 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
 //   - one MMA warp loads the activation tile of every completed weight tile
 //     (N = batch rounded up to 16 rows x 16 columns, zero rows past the
 //     batch; fetched with cp.async one block ahead) into the same layout and
-//     issues tcgen05.mma into one of two fp32 accumulators in tensor memory
+//     issues tcgen05.mma into one of two (one at batches over 64) fp32
+//     accumulators in tensor memory
 //     (128 lanes x N columns), then commits to an mbarrier that the writers
 //     of the ring wait on before they overwrite tiles;
 //   - consumer warps 0-3 (one per 32 tensor-memory lanes) move a finished
@@ -1197,7 +1198,9 @@ struct GBatch {
   uint32_t stage_bytes;  // bytes of each consumer warp's exponent region
   uint32_t ring;         // A tile (and activation tile) slots
   uint32_t n_mma;        // N of every MMA: the batch rounded up to 16
-  uint32_t tmem_cols;    // tensor-memory columns allocated (two accumulators)
+  uint32_t tmem_cols;    // tensor-memory columns allocated (accs accumulators)
+  uint32_t accs;         // accumulators: 2 (a finished piece's is moved out while the
+                         // next accumulates) when they fit beside three others, else 1
   uint32_t spin_limit;
 };
 
@@ -1316,7 +1319,7 @@ __global__ void __launch_bounds__(T + 64, 4) df11_decode_gemm_kernel(const __gri
     mbar_init(bar(kTableBar), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == MMA) {  // tensor memory: two accumulators of n_mma columns
+  if (warp == MMA) {  // tensor memory: gb.accs accumulators of n_mma columns
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(taddr_s)),
                  "r"(gb.tmem_cols)
@@ -1383,7 +1386,7 @@ __global__ void __launch_bounds__(T + 64, 4) df11_decode_gemm_kernel(const __gri
                            ((uint32_t)(kGemmM >> 4) << 24);
     pdl_wait();  // the activations may come from the previous kernel
     uint32_t t_run = 0;  // tiles of this thread block's pieces so far (ring position)
-    uint32_t seg = 0, seg_tiles = 0;  // segments so far (accumulator seg & 1), their tiles
+    uint32_t seg = 0, seg_tiles = 0;  // pieces so far (accumulator seg % accs), their tiles
     int prev_ti = -1;
     uint32_t prev_rb = 0;
     // The activation tile of column group cg, rows below the batch (the
@@ -1410,8 +1413,10 @@ __global__ void __launch_bounds__(T + 64, 4) df11_decode_gemm_kernel(const __gri
         ++seg;  // a new row block: the other accumulator
         seg_tiles = 0;
         // flushed two segments ago
-        if (seg >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar(kDFree + (seg & 1)),
-                                                            ((seg >> 1) - 1) & 1u, gb.spin_limit))) {
+        // the accumulator it takes was emptied (the piece gb.accs before)
+        if (seg >= gb.accs &&
+            !__all_sync(0xFFFFFFFFu, mbar_wait(bar(kDFree + seg % gb.accs),
+                                                ((seg / gb.accs) - 1) & 1u, gb.spin_limit))) {
           failed = true;
           break;
         }
@@ -1419,7 +1424,7 @@ __global__ void __launch_bounds__(T + 64, 4) df11_decode_gemm_kernel(const __gri
       }
       prev_ti = g.ti;
       prev_rb = g.rb;
-      const uint32_t d_tmem = tmem + (seg & 1) * gb.n_mma;
+      const uint32_t d_tmem = tmem + (seg % gb.accs) * gb.n_mma;
       // tiles of the piece complete once block b is decoded
       auto ready_after = [&](uint32_t b) {
         if (b >= bl) return g.tiles;
@@ -1511,7 +1516,7 @@ __global__ void __launch_bounds__(T + 64, 4) df11_decode_gemm_kernel(const __gri
         waited = true;
       }
       const uint32_t row = flush_rb * kGemmM + 32u * warp + lane;
-      const uint32_t base = tmem + ((32u * warp) << 16) + (flush_seg & 1) * gb.n_mma;
+      const uint32_t base = tmem + ((32u * warp) << 16) + (flush_seg % gb.accs) * gb.n_mma;
       for (uint32_t c = 0; c < gb.n_mma; c += 8) {
         uint32_t v[8];
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -1526,7 +1531,7 @@ __global__ void __launch_bounds__(T + 64, 4) df11_decode_gemm_kernel(const __gri
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kDFree + (flush_seg & 1)));
+      if (lane == 0) mbar_arrive(bar(kDFree + flush_seg % gb.accs));
       flush_seg = -1;
     };
     for (uint32_t u = ub; u < ue && !failed;) {
@@ -2360,8 +2365,12 @@ df11_status df11_decode_gemm(const df11_tensor *tensors, const df11_gemv *ops, i
   // of them the tile the block before it began); the ring holds them
   gb.ring = (max_block + 2047u) / 2048u + 1u;
   gb.n_mma = (max_batch + 15u) & ~15u;
+  // two accumulators up to 128 columns (room for four resident blocks),
+  // one above: a thread block's range holds one or two pieces, so waiting
+  // for the one accumulator to be emptied costs little
+  gb.accs = 2 * gb.n_mma <= 128 ? 2u : 1u;
   gb.tmem_cols = 32;
-  while (gb.tmem_cols < 2 * gb.n_mma) gb.tmem_cols <<= 1;
+  while (gb.tmem_cols < gb.accs * gb.n_mma) gb.tmem_cols <<= 1;
   // y = W x: clear the outputs first, in stream order
   ClearArgs ca{};
   for (int i = 0; i < m; ++i) {
