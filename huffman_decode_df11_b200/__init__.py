@@ -300,13 +300,46 @@ class Df11Device:
     decode_table: Optional[torch.Tensor] = None  # df11_build_decode_table output
     interleave: int = 1  # rows interleaved per 16 columns in the stream (1: row-major)
 
+    @classmethod
+    def _in_block(cls, params: Params, block: torch.Tensor, spans: dict, shape: tuple,
+                  interleave: int) -> "Df11Device":
+        """A tensor whose buffers are byte ranges of one device allocation
+        (`spans`: name -> (offset, bytes, dtype)).  The tensor view of a
+        buffer is made when the buffer is first used; pointers for a decode
+        come straight from the allocation."""
+        d = cls.__new__(cls)
+        d.params, d.shape, d.interleave, d.decode_table = params, shape, interleave, None
+        d._block, d._spans = block, spans
+        off, nbytes, _ = spans["chunk_counts"]
+        d.chunk_counts = block[off:off + nbytes]  # a field with a default: made now
+        return d
+
+    def __getattr__(self, name):
+        # only reached for a buffer of a _in_block tensor not yet viewed
+        spans = self.__dict__.get("_spans")
+        if spans is None or name not in spans:
+            raise AttributeError(name)
+        off, nbytes, dtype = spans[name]
+        v = self.__dict__["_block"][off:off + nbytes]
+        if dtype is not None:
+            v = v.view(dtype)
+        self.__dict__[name] = v
+        return v
+
+    def _ptr(self, name: str) -> int:
+        spans = self.__dict__.get("_spans")
+        if spans is not None and name in spans and name not in self.__dict__:
+            return self.__dict__["_block"].data_ptr() + spans[name][0]
+        return getattr(self, name).data_ptr()
+
     @property
     def n(self) -> int:
         return int(self.params.n)
 
     @property
     def device(self):
-        return self.bitstream.device
+        b = self.__dict__.get("_block")
+        return b.device if b is not None else self.bitstream.device
 
     def compressed_bytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
@@ -317,10 +350,9 @@ class Df11Device:
     def desc(self, out: torch.Tensor, counts: bool = True) -> TensorDesc:
         cc = self.chunk_counts.data_ptr() if (counts and self.chunk_counts is not None) else None
         dt = self.decode_table.data_ptr() if self.decode_table is not None else None
-        return TensorDesc(self.bitstream.data_ptr(), self.gaps.data_ptr(), cc,
-                          self.block_out_pos.data_ptr(), self.luts.data_ptr(),
-                          self.code_lengths.data_ptr(), self.sign_mantissa.data_ptr(),
-                          out.data_ptr(), dt, self.params)
+        p = self._ptr
+        return TensorDesc(p("bitstream"), p("gaps"), cc, p("block_out_pos"), p("luts"),
+                          p("code_lengths"), p("sign_mantissa"), out.data_ptr(), dt, self.params)
 
 
 def _np_to(t: np.ndarray, device, pin: bool = False) -> torch.Tensor:
@@ -426,30 +458,24 @@ def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, deco
                                           params, ctypes.cast(lens, vp), handles),
            "df11_gpu_build_begin_batched")
     outs = (GpuBuildOut * count)()
-    views = []
     try:
         # every output buffer of the call in one allocation, each at a
         # 256-byte boundary (at least 16 bytes, so that no pointer is NULL)
         layout, total = [], 0
         for f, p in zip(flats, params):
-            chunks = int(p.num_blocks) * threads_per_block
-            sizes = (chunks * chunk_bytes + 16, chunks * 5 // 8 + 16, chunks + 16,
-                     4 * (int(p.num_blocks) + 1), 4 * int(p.num_luts) * 256, 256,
-                     (f.numel() + 15) // 16 * 16)
+            nb = int(p.num_blocks)
+            chunks = nb * threads_per_block
+            sizes = (chunks * chunk_bytes + 16, chunks * 5 // 8 + 16, chunks + 16, 4 * (nb + 1),
+                     1024 * int(p.num_luts), 256, (f.numel() + 15) // 16 * 16)
             offs = []
             for nbytes in sizes:
                 offs.append(total)
                 total += (max(nbytes, 16) + 255) & ~255
             layout.append((offs, sizes))
-        dev = flats[0].device
-        block = torch.empty(max(total, 256), dtype=torch.uint8, device=dev)
+        block = torch.empty(max(total, 256), dtype=torch.uint8, device=flats[0].device)
         base = block.data_ptr()
-        for i, (offs, sizes) in enumerate(layout):
+        for i, (offs, _) in enumerate(layout):
             outs[i] = GpuBuildOut(*[base + o for o in offs])
-            v = [block[o:o + nbytes] for o, nbytes in zip(offs, sizes)]
-            v[3] = v[3].view(torch.int32)
-            v[4] = v[4].view(torch.int32)
-            views.append(v)
     except BaseException:
         for hnd in handles:
             L.df11_gpu_build_free(hnd)
@@ -457,14 +483,21 @@ def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, deco
     _check(L.df11_gpu_build_finish_batched(handles, count, ptrs, outs, params, sh),
            "df11_gpu_build_finish_batched")
     out = []
-    for p, v, shape in zip(params, views, shapes):
-        d = Df11Device(params=Params.from_buffer_copy(p), bitstream=v[0], gaps=v[1],
-                       chunk_counts=v[2], block_out_pos=v[3], luts=v[4], code_lengths=v[5],
-                       sign_mantissa=v[6], shape=shape, interleave=int(interleave))
+    for p, (offs, sizes), shape in zip(params, layout, shapes):
+        spans = {name: (o, nbytes, dt) for name, o, nbytes, dt in
+                 zip(_GPU_BUILD_FIELDS, offs, sizes, _GPU_BUILD_DTYPES)}
+        d = Df11Device._in_block(Params.from_buffer_copy(p), block, spans, shape,
+                                 int(interleave))
         if decode_table:
             d.decode_table = build_decode_table(d, stream)
         out.append(d)
     return out
+
+
+# the order of df11_gpu_build_out, and the view each buffer gets
+_GPU_BUILD_FIELDS = ("bitstream", "gaps", "chunk_counts", "block_out_pos", "luts",
+                     "code_lengths", "sign_mantissa")
+_GPU_BUILD_DTYPES = (None, None, None, torch.int32, torch.int32, None, None)
 
 
 def exponent_histogram(w: torch.Tensor, stream=None) -> np.ndarray:
@@ -491,7 +524,7 @@ def build_decode_table(d: Df11Device, stream=None) -> torch.Tensor:
     """The decode table of a device tensor (df11_build_decode_table)."""
     t = torch.empty(DF11_DECODE_TABLE_BYTES, dtype=torch.uint8, device=d.device)
     with torch.cuda.device(d.device):
-        _check(lib().df11_build_decode_table(d.luts.data_ptr(), d.code_lengths.data_ptr(),
+        _check(lib().df11_build_decode_table(d._ptr("luts"), d._ptr("code_lengths"),
                                              int(d.params.num_luts), t.data_ptr(),
                                              _stream_handle(stream)), "df11_build_decode_table")
     return t

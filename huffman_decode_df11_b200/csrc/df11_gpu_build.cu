@@ -5,35 +5,36 @@
 // The pages compress offline on the host ("DFloat11无损压缩技术" (jsqmd.com)
 // §2.2 items 1-2 give the recipe; "DFloat11重新定义LLM无损压缩的技术边界"
 // (ocdem.com) §2.2 the lookup tables).  Here every step that touches the n
-// elements runs on the device; only the codebook, a function of 256 counts,
-// is computed on the host (df11_codebook.h, shared with the host builder).
-// The elements are cut into pack blocks of 2048 (8 per thread of a
-// 256-thread block); the kernels, in stream order:
-//   histogram  exponent counts, one pass: counters in registers for a
-//              window of 16 exponents around the mode of a first sample,
-//              summed over the warp now and then; shared counters for the
-//              rest;
-//   sums       the code-length total of every pack block.  Each thread
-//              block walks a contiguous range of pack blocks and keeps a
-//              running total, so it writes every pack block's first bit
-//              relative to its range, and the range's total;
-//   scan       the ranges' first bits (one thread block; at most a few
-//              thousand ranges) and the stream's total, which the host
-//              reads to size the outputs;
-//   prepare    chunk first elements preset to n, gaps and maxima cleared,
-//              the bitstream words two pack blocks share cleared;
-//   pack       persistent: per pack block, a block scan of the threads' bit
-//              counts, every codeword ORed into a shared-memory image of the
-//              block's words, the words written out coalesced (atomic OR
-//              for the first and last word when a neighbour owns part of
-//              it), the sign/mantissa bytes, and for every chunk and block
-//              whose first codeword start is one of the thread's elements
-//              the gap, first element and block position; the next pack
-//              block's words are loaded while this one is packed;
-//   finish     the chunks and blocks after the last codeword start, chunk
-//              counts from first-element differences, the gaps packed
-//              eight to five bytes, and the largest block, chunk and group
-//              of 32 chunks.
+// elements runs on the device.  The codebook, a function of 256 counts, is
+// computed on the host (df11_codebook.h, shared with the host builder), and
+// with it the stream's length, the sum over exponents of count x code
+// length, which sizes the outputs.  The device reads the elements twice,
+// in tiles of 16384:
+//   histogram  (phase 1) exponent counts per tile and in all: four-bit
+//              counters in registers for a window of 16 exponents around
+//              the mode of a first sample, spread into byte counters after
+//              every 8 elements and summed over the warp at the end of the
+//              tile; shared counters for exponents outside the window.
+//              Each tile's 256 counts are kept (16 bits each);
+//   tile bits  (phase 2) each tile's bit count, the dot product of its
+//              counts with the code lengths, and an exclusive scan of them:
+//              every tile's first bit, with no second pass over the
+//              elements and no wait between thread blocks;
+//   pack       one thread block per tile, in four steps of 4096 elements:
+//              a block scan of the code lengths, the codewords ORed into a
+//              shared-memory image of the step's words, written out
+//              coalesced (the word two steps share is carried to the next
+//              step; the first and last words of a tile, which it may share
+//              with its neighbours, go to a side array).  Also written: the
+//              sign/mantissa bytes, and for every chunk and block whose
+//              first codeword start is one of the tile's elements, its gap,
+//              first element and block position;
+//   finish     the shared words from the side array, chunk counts from
+//              first-element differences (n past the last codeword start),
+//              the gaps packed eight to five bytes, block positions past
+//              the last start, the paddings, the tables into the caller's
+//              buffers, and the largest block, chunk and group of 32
+//              chunks.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -52,7 +53,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kPerThread = 8;
-constexpr int kPerCta = kThreads * kPerThread;  // elements per pack block
+constexpr int kPerCta = kThreads * kPerThread;  // elements per histogram step of a block
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 __device__ __forceinline__ uint32_t exponent(uint32_t x) { return (x >> 7) & 0xFFu; }
@@ -71,9 +72,12 @@ __device__ __forceinline__ uint4 load8(const uint16_t *w, uint64_t n, uint64_t i
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int q) {
+  return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+}
+
 __device__ __forceinline__ uint32_t exponent_of(const uint4 &v, int k) {
-  const uint32_t u = (k >> 1) == 0 ? v.x : (k >> 1) == 1 ? v.y : (k >> 1) == 2 ? v.z : v.w;
-  return (u >> ((k & 1) ? 23 : 7)) & 0xFFu;
+  return (word_of(v, k >> 1) >> ((k & 1) ? 23 : 7)) & 0xFFu;
 }
 
 // how many of elements i0 .. i0+7 exist (0..8)
@@ -82,21 +86,22 @@ __device__ __forceinline__ uint32_t live_of(uint64_t i0, uint64_t n) {
 }
 
 // ---- histogram -----------------------------------------------------------
-// Per lane, 16 four-bit counters in one 64-bit register take the 8 elements
-// of a tile whose exponent falls in the warp's window (mode - 11 .. mode + 4);
-// after each tile they are spread into byte counters (four registers), and
-// those are summed over the warp into shared counters every 31 tiles
-// (at most 248 counts per byte).  Exponents outside the window go to the
-// shared counters at once.
-constexpr int kWindow = 16;
+// A tile is kTileSteps steps of 2048 elements (8 per thread of a 256-thread
+// block); a block takes tiles kGrid apart.  Per lane, 16 four-bit counters
+// in two registers (bins 0-7 and 8-15 of the warp's window, mode - 11 ..
+// mode + 4) take the 8 elements of a step; after each step they are spread
+// into byte counters (four registers), which are summed over the warp into
+// shared counters at the end of the tile (at most 64 counts per byte).
+// Exponents outside the window go to the shared counters at once.
 constexpr int kWindowBelow = 11;
-constexpr int kFlushTiles = 31;
+constexpr int kTileSteps = 8;
+constexpr uint32_t kTile = kTileSteps * kPerCta;  // elements per tile (16384)
 
 // byte j of counter register r holds window bin (r >> 1) * 8 + 2 j + (r & 1)
 __device__ __forceinline__ void flush_window(uint32_t (&c)[4], int lo, uint32_t *h, int lane) {
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    // two 16-bit sums per word: 32 lanes x 248 < 2^16
+    // two 16-bit sums per word: 32 lanes x 64 < 2^16
     const uint32_t even = __reduce_add_sync(0xFFFFFFFFu, c[r] & 0x00FF00FFu);
     const uint32_t odd = __reduce_add_sync(0xFFFFFFFFu, (c[r] >> 8) & 0x00FF00FFu);
     if (lane == 0) {
@@ -111,158 +116,170 @@ __device__ __forceinline__ void flush_window(uint32_t (&c)[4], int lo, uint32_t 
   }
 }
 
-__device__ __forceinline__ void count8(const uint4 &v, uint32_t live, int lo, uint32_t (&c)[4],
-                                       uint32_t *h) {
-  unsigned long long nib = 0;
+// One element whose exponent times 4 is e4: the window offset times 4 is
+// sh = e4 - lo4 (wrapping below the window), and 1 << sh lands in the
+// counter pair's low register for sh < 32, in the high one for 32 <= sh <
+// 64; the clamped funnel shifts give 0 elsewhere.
+__device__ __forceinline__ void count_one(uint32_t e4, uint32_t lo4, uint32_t &n_lo,
+                                          uint32_t &n_hi, uint32_t *h) {
+  const uint32_t sh = e4 - lo4;
+  n_lo += __funnelshift_lc(0u, 1u, sh);
+  n_hi += __funnelshift_lc(0u, 1u, sh - 32u);
+  if (sh >= 64u) atomicAdd(&h[e4 >> 2], 1u);
+}
+
+template <bool FULL>
+__device__ __forceinline__ void count8(const uint4 &v, uint32_t live, uint32_t lo4,
+                                       uint32_t (&c)[4], uint32_t *h) {
+  uint32_t n_lo = 0, n_hi = 0;
 #pragma unroll
-  for (int k = 0; k < kPerThread; ++k) {
-    if ((uint32_t)k < live) {
-      const uint32_t e = exponent_of(v, k);
-      const uint32_t d = (uint32_t)((int)e - lo);
-      if (d < (uint32_t)kWindow) nib += 1ull << (4 * d);
-      else atomicAdd(&h[e], 1u);
-    }
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t u = word_of(v, q);
+    if (FULL || (uint32_t)(2 * q) < live) count_one((u >> 5) & 0x3FCu, lo4, n_lo, n_hi, h);
+    if (FULL || (uint32_t)(2 * q + 1) < live) count_one((u >> 21) & 0x3FCu, lo4, n_lo, n_hi, h);
   }
-  const uint32_t n_lo = (uint32_t)nib, n_hi = (uint32_t)(nib >> 32);
   c[0] += n_lo & 0x0F0F0F0Fu;
   c[1] += (n_lo >> 4) & 0x0F0F0F0Fu;
   c[2] += n_hi & 0x0F0F0F0Fu;
   c[3] += (n_hi >> 4) & 0x0F0F0F0Fu;
 }
 
+// hist[e] += the count of exponent e (64-bit, device-wide); tile_hist, if
+// not null, gets each tile's 256 counts (16 bits; a tile has at most 16384
+// elements); *last, if not null, the last element (its codeword ends the
+// stream).
 __global__ void __launch_bounds__(kThreads) hist_kernel(const uint16_t *w, uint64_t n, bool vec,
                                                         unsigned long long *hist,
-                                                        unsigned long long *last) {
-  // the last element (its codeword ends the stream), for the builder
+                                                        unsigned long long *last,
+                                                        uint16_t *tile_hist) {
   if (last && blockIdx.x == 0 && threadIdx.x == 0 && n) *last = w[n - 1];
   __shared__ uint32_t h[kThreads / 32][256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int j = threadIdx.x; j < (kThreads / 32) * 256; j += kThreads) (&h[0][0])[j] = 0;
-  const uint64_t stride = (uint64_t)gridDim.x * kPerCta;
-  uint64_t base = (uint64_t)blockIdx.x * kPerCta;
-  const uint64_t me = (uint64_t)threadIdx.x * kPerThread;
-  uint4 next = load8(w, n, base + me, vec);
+  const uint32_t me = threadIdx.x * kPerThread;
   // the window: around the most frequent exponent among the warp's lanes'
-  // first elements
+  // first elements of the block's first tile
   int lo;
   {
-    const uint32_t key = base + me < n ? exponent(next.x & 0xFFFFu) : 256u;
+    const uint64_t i = (uint64_t)blockIdx.x * kTile + warp * (kTile / 8) + lane * kPerThread;
+    const uint32_t key = i < n ? exponent(w[i]) : 256u;
     const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
     const uint32_t best = __reduce_max_sync(0xFFFFFFFFu, ((uint32_t)__popc(peers) << 16) | key);
     lo = (int)(best & 0x1FFu) - kWindowBelow;
   }
+  const uint32_t lo4 = (uint32_t)(4 * lo);
   __syncthreads();
-  uint32_t c[4] = {0, 0, 0, 0};
-  int tiles = 0;
-  // `base` is the same for every thread of the block: whole warps iterate
-  for (; base < n; base += stride) {
-    const uint4 v = next;
-    if (base + stride < n) next = load8(w, n, base + stride + me, vec);
-    count8(v, live_of(base + me, n), lo, c, h[warp]);
-    if (++tiles == kFlushTiles) {
-      flush_window(c, lo, h[warp], lane);
-      tiles = 0;
+  uint32_t total = 0;  // exponent threadIdx.x over the block's tiles
+  for (uint64_t t0 = (uint64_t)blockIdx.x * kTile; t0 < n; t0 += (uint64_t)gridDim.x * kTile) {
+    uint32_t c[4] = {0, 0, 0, 0};
+    if (t0 + kTile <= n) {  // a whole tile: every load in flight at once
+      uint4 v[kTileSteps];
+#pragma unroll
+      for (int st = 0; st < kTileSteps; ++st) v[st] = load8(w, n, t0 + st * kPerCta + me, vec);
+#pragma unroll
+      for (int st = 0; st < kTileSteps; ++st) count8<true>(v[st], kPerThread, lo4, c, h[warp]);
+    } else {
+      for (int st = 0; st < kTileSteps; ++st) {
+        const uint64_t i = t0 + st * kPerCta + me;
+        count8<false>(load8(w, n, i, vec), live_of(i, n), lo4, c, h[warp]);
+      }
     }
+    flush_window(c, lo, h[warp], lane);
+    __syncthreads();
+    uint32_t v = 0;
+#pragma unroll
+    for (int j = 0; j < kThreads / 32; ++j) {
+      v += h[j][threadIdx.x];
+      h[j][threadIdx.x] = 0;
+    }
+    if (tile_hist) tile_hist[(t0 / kTile) * 256 + threadIdx.x] = (uint16_t)v;
+    total += v;
+    __syncthreads();
   }
-  flush_window(c, lo, h[warp], lane);
-  __syncthreads();
-  uint32_t s = 0;
-  for (int j = 0; j < kThreads / 32; ++j) s += h[j][threadIdx.x];
-  if (s) atomicAdd(&hist[threadIdx.x], (unsigned long long)s);
+  if (total) atomicAdd(&hist[threadIdx.x], (unsigned long long)total);
 }
 
-// ---- bit offsets ---------------------------------------------------------
-// The pack kernel works in units of 256 elements (one warp, 8 per lane).  A
-// sums thread block walks a contiguous range of units, 32 per iteration
-// (four per warp), and keeps a running total, so it writes each unit's first
-// bit relative to its range, and the range's total.
-constexpr int kUnit = 32 * kPerThread;        // elements per unit
-constexpr int kUnitWords = kUnit + 1;         // words a unit's codewords can touch
-constexpr int kUnitsPerWarp = 4;              // per iteration of the sums kernel
-constexpr int kUnitsPerIter = (kThreads / 32) * kUnitsPerWarp;
-static_assert(kUnitsPerIter == 32, "one warp scans an iteration's units");
+// ---- phase 2 jobs --------------------------------------------------------
+// Phase 2 of a batch runs as one launch per kernel over all its tensors;
+// each tensor is a job, described in device memory (copied there with the
+// code tables).  Tiles are numbered through the batch, job after job.
 
-struct Ranges {
-  uint64_t units;  // units of the tensor
-  uint64_t per;    // units per range (one range per sums thread block)
-  uint32_t *local; // first bit of each unit within its range
-  unsigned long long *range_start;  // first bit of each range; the total after the last
+// {codeword << 8 | length} for codes of up to 24 bits; 0x80 | length for
+// longer ones, whose codewords are in a second table
+constexpr uint32_t kLongCode = 0x80u;
+constexpr int kPackedCodeBits = 24;
+
+struct Job {
+  const uint16_t *w;  // the elements
+  uint64_t n;
+  uint32_t vec;       // w is 16-byte aligned
+  uint32_t longs;     // the code has codewords above 24 bits
+  uint64_t tiles, tile_base;  // tiles, and the first one's number in the batch
+  const uint16_t *tile_hist;  // phase 1: 256 counts per tile
+  uint32_t *tile_bits;
+  unsigned long long *tile_start;  // tiles + 1 (the total last)
+  uint32_t *edge;                  // per tile: its first and last word when shared
+  const uint32_t *tab;  // 256 packed entries, 256 codewords, the luts, 256 code lengths
+  // outputs
+  uint32_t *bs32;
+  uint8_t *sm, *gaps_packed, *counts, *code_lengths;
+  uint32_t *bpos, *luts;
+  // scratch: per chunk its first element and gap; the largest block, chunk
+  // and group of 32 chunks
+  uint32_t *first_elem;
+  uint8_t *gap;
+  unsigned int *maxima;
+  uint64_t chunks, total, last_start;
+  uint32_t num_blocks, luts_vec4;
+  uint32_t chunk_bits, block_bits;    // 8 C and 8 C T
+  uint32_t chunk_words, block_words;  // chunk_bits / 32, block_bits / 32
+  uint64_t chunk_magic, block_magic;  // ceil(2^64 / words) (words >= 2)
+  uint64_t fin_threads;               // threads of the finish kernel
+  uint8_t *zero[4];                   // byte ranges to clear: the paddings
+  uint32_t zero_bytes[4];
 };
 
-// units and ranges number below 2^24: 32-bit division
-__device__ __forceinline__ unsigned long long unit_start(const Ranges &r, uint64_t u) {
-  return r.range_start[(uint32_t)u / (uint32_t)r.per] + r.local[u];
+// floor(x / d) for x < 2^32 by a multiply-high with ceil(2^64 / d): the
+// error, below x / 2^64 < 2^-32, never crosses an integer (d < 2^32)
+__device__ __forceinline__ uint64_t div_words(uint32_t x, uint32_t d, uint64_t magic) {
+  return d == 1 ? x : __umul64hi((uint64_t)x, magic);
 }
 
-__global__ void __launch_bounds__(kThreads, 4) sums_kernel(const uint16_t *w, uint64_t n, bool vec,
-                                                           const uint2 *tab, const Ranges r,
-                                                           unsigned long long *range_total) {
-  __shared__ uint8_t len[256];
-  __shared__ uint32_t part[kUnitsPerIter];
-  len[threadIdx.x] = (uint8_t)tab[threadIdx.x].y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint64_t u_begin = (uint64_t)blockIdx.x * r.per;
-  const uint64_t u_end = u_begin + r.per < r.units ? u_begin + r.per : r.units;
-  const uint64_t me = (uint64_t)lane * kPerThread;
-  uint4 next[kUnitsPerWarp];
-#pragma unroll
-  for (int j = 0; j < kUnitsPerWarp; ++j) {
-    const uint64_t u = u_begin + warp * kUnitsPerWarp + j;
-    next[j] = u < u_end ? load8(w, n, u * kUnit + me, vec) : make_uint4(0, 0, 0, 0);
-  }
+// ---- tile bits -----------------------------------------------------------
+// Grid (x, job): one warp per tile, lane l takes exponents 8l .. 8l+7.
+__global__ void __launch_bounds__(256) tile_bits_kernel(const Job *jobs) {
+  const Job &J = jobs[blockIdx.y];
+  __shared__ uint32_t len_s[256];
+  len_s[threadIdx.x] = J.tab[threadIdx.x] & 0x3Fu;
   __syncthreads();
-  unsigned long long running = 0;  // warp 0: bits of the range so far (uniform)
-  for (uint64_t u0 = u_begin; u0 < u_end; u0 += kUnitsPerIter) {
-    uint4 v[kUnitsPerWarp];
+  const int lane = threadIdx.x & 31;
+  const uint64_t t = blockIdx.x * 8ull + (threadIdx.x >> 5);
+  if (t >= J.tiles) return;
+  const uint4 hv = reinterpret_cast<const uint4 *>(J.tile_hist + t * 256)[lane];
+  uint32_t sum = 0;
 #pragma unroll
-    for (int j = 0; j < kUnitsPerWarp; ++j) {
-      v[j] = next[j];
-      const uint64_t u = u0 + kUnitsPerIter + warp * kUnitsPerWarp + j;
-      if (u < u_end) next[j] = load8(w, n, u * kUnit + me, vec);
-    }
-#pragma unroll
-    for (int j = 0; j < kUnitsPerWarp; ++j) {
-      const uint64_t u = u0 + warp * kUnitsPerWarp + j;
-      const uint32_t live = u < u_end ? live_of(u * kUnit + me, n) : 0u;
-      uint32_t s = 0;
-#pragma unroll
-      for (int k = 0; k < kPerThread; ++k)
-        if ((uint32_t)k < live) s += len[exponent_of(v[j], k)];
-      s = __reduce_add_sync(0xFFFFFFFFu, s);
-      if (lane == 0) part[warp * kUnitsPerWarp + j] = s;
-    }
-    __syncthreads();
-    if (warp == 0) {  // the iteration's 32 units in order, one per lane
-      const uint32_t mine = part[lane];
-      uint32_t incl = mine;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += t;
-      }
-      const uint64_t u = u0 + lane;
-      if (u < u_end) r.local[u] = (uint32_t)(running + incl - mine);
-      running += __shfl_sync(0xFFFFFFFFu, incl, 31);
-    }
-    __syncthreads();  // part is rewritten next iteration
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t x = word_of(hv, q);
+    sum += (x & 0xFFFFu) * len_s[8 * lane + 2 * q] + (x >> 16) * len_s[8 * lane + 2 * q + 1];
   }
-  if (threadIdx.x == 0) range_total[blockIdx.x] = running;
+  sum = __reduce_add_sync(0xFFFFFFFFu, sum);  // at most 16384 x 32 bits
+  if (lane == 0) J.tile_bits[t] = sum;
 }
 
-// Exclusive scan of the range totals into the ranges' first bits, the total
-// at starts[count]; one thread block, each thread a contiguous run.
+// Exclusive scan of a job's tile bits into their first bits, the total at
+// tile_start[tiles]; one thread block per job, each thread a contiguous run.
 constexpr int kScanThreads = 1024;
 
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(const unsigned long long *totals,
-                                                            uint64_t count,
-                                                            unsigned long long *starts) {
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const Job *jobs) {
+  const Job &J = jobs[blockIdx.x];
   __shared__ unsigned long long warp_tot[kScanThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint64_t count = J.tiles;
   const uint64_t per = (count + kScanThreads - 1) / kScanThreads;
   const uint64_t b = threadIdx.x * per;
   const uint64_t e = b + per < count ? b + per : count;
   unsigned long long mine = 0;
-  for (uint64_t i = b; i < e; ++i) mine += totals[i];
+  for (uint64_t i = b; i < e; ++i) mine += J.tile_bits[i];
   unsigned long long incl = mine;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -274,338 +291,460 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const unsigned long 
   unsigned long long run = incl - mine;
   for (int j = 0; j < warp; ++j) run += warp_tot[j];
   for (uint64_t i = b; i < e; ++i) {
-    starts[i] = run;
-    run += totals[i];
+    J.tile_start[i] = run;
+    run += J.tile_bits[i];
   }
-  if (threadIdx.x == kScanThreads - 1) starts[count] = run;
-}
-
-// Before packing: first elements preset to n, gaps cleared, the bitstream
-// words that two units share cleared (they are ORed into), maxima cleared;
-// also the output paddings no kernel writes cleared, and the tables copied
-// from the device staging area into the caller's buffers.
-struct PrepareArgs {
-  uint32_t *first_elem;
-  uint8_t *gap;
-  uint64_t chunks;
-  uint32_t n;
-  Ranges r;
-  uint32_t *bs32;
-  unsigned int *maxima;
-  uint8_t *zero[4];        // byte ranges to clear
-  uint32_t zero_bytes[4];
-  const uint4 *luts_src;   // num_luts * 1 KB
-  uint4 *luts_dst;         // 16-byte aligned
-  uint32_t luts_vec4;      // 16-byte words of the tables
-  const uint8_t *lens_src;
-  uint8_t *lens_dst;       // 256 bytes, any alignment
-};
-
-__global__ void prepare_kernel(const PrepareArgs a) {
-  uint64_t all = a.chunks + 1 > a.r.units ? a.chunks + 1 : a.r.units;
-  all = all > a.luts_vec4 ? all : a.luts_vec4;
-  all = all > 256 ? all : 256;  // the code lengths, the paddings, the maxima
-  for (uint64_t i = blockIdx.x * 256ull + threadIdx.x; i < all; i += (uint64_t)gridDim.x * 256) {
-    if (i <= a.chunks) {
-      a.first_elem[i] = a.n;
-      a.gap[i] = 0;
-    }
-    if (i >= 1 && i < a.r.units) {
-      const unsigned long long st = unit_start(a.r, i);
-      if (st & 31u) a.bs32[st >> 5] = 0;
-    }
-    if (i < 3) a.maxima[i] = 0;
-    if (i < a.luts_vec4) a.luts_dst[i] = a.luts_src[i];
-    if (i < 256) a.lens_dst[i] = a.lens_src[i];
-  }
-  // paddings: each at most a block of the bitstream plus 16 bytes
-  for (int k = 0; k < 4; ++k)
-    for (uint32_t i = blockIdx.x * 256u + threadIdx.x; i < a.zero_bytes[k]; i += gridDim.x * 256u)
-      a.zero[k][i] = 0;
+  if (threadIdx.x == kScanThreads - 1) J.tile_start[count] = run;
 }
 
 // ---- pack ----------------------------------------------------------------
-struct PackArgs {
-  const uint16_t *w;
-  uint64_t n;
-  bool vec;             // w is 16-byte aligned
-  const uint2 *tab;     // {codeword, length} per exponent
-  Ranges r;
-  uint32_t *bs32;       // bitstream as 32-bit words
-  uint8_t *sm;          // 16-byte aligned
-  uint8_t *gap;         // one byte per chunk
-  uint32_t *first_elem; // chunks + 1, preset to n
-  uint32_t *bpos;
-  uint64_t chunks;
-  uint32_t num_blocks;
-  uint32_t chunk_bits, block_bits;  // 8 C and 8 C T
-  uint32_t chunk_words, block_words;  // chunk_bits / 32, block_bits / 32
-  uint64_t chunk_magic, block_magic;  // ceil(2^64 / words) (words >= 2)
-  uint32_t chunk_m32;                 // ceil(2^32 / chunk_bits): floor(x / chunk_bits)
-                                      // = umulhi(x, chunk_m32) for x < 2^16
-};
+// A thread block packs a tile in steps of 16 units of 256 elements; warp w
+// packs units w and w + 8 of a step, a unit being 8 consecutive elements
+// per lane.  Bits are counted relative to the step's origin, the first bit
+// of the word its first codeword begins in; a step spans at most 4096 x 32
+// bits plus the 31 before its start.
+constexpr int kUnit = 32 * kPerThread;           // elements per unit
+constexpr int kStepUnits = 2 * (kThreads / 32);  // units per step
+constexpr uint32_t kStep = kStepUnits * kUnit;   // elements per step (4096)
+constexpr int kStepsPerTile = kTile / kStep;
+constexpr int kStepWords = kStep + 2;            // words a step's codewords can touch
+static_assert(kTile % kStep == 0, "a tile is whole steps");
 
-// floor(x / d) for x < 2^32 by a multiply-high with ceil(2^64 / d): the
-// error, below x / 2^64 < 2^-32, never crosses an integer (d < 2^32)
-__device__ __forceinline__ uint64_t div_words(uint32_t x, uint32_t d, uint64_t magic) {
-  return d == 1 ? x : __umul64hi((uint64_t)x, magic);
+// the job whose tiles hold batch tile t (jobs in tile order)
+__device__ __forceinline__ int job_of(const Job *jobs, int count, uint64_t t) {
+  int lo = 0, hi = count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (jobs[mid].tile_base <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
 }
 
-__global__ void __launch_bounds__(kThreads) pack_kernel(const PackArgs a) {
-  __shared__ uint2 tab_s[256];
-  __shared__ uint32_t words_s[kThreads / 32][kUnitWords];
-  tab_s[threadIdx.x] = a.tab[threadIdx.x];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t *words = words_s[warp];
-  for (int j = lane; j < kUnitWords; j += 32) words[j] = 0;
-  const uint64_t me = (uint64_t)lane * kPerThread;
-  const uint64_t units = a.r.units;
-  const uint64_t stride = (uint64_t)gridDim.x * (kThreads / 32);
-  uint64_t u = (uint64_t)blockIdx.x * (kThreads / 32) + warp;
-  // unit u's words, first bit and previous element (lane 0)
-  uint4 nx = make_uint4(0, 0, 0, 0);
-  unsigned long long nstart = 0;
-  uint32_t nprev = 0;
-  if (u < units) {
-    nx = load8(a.w, a.n, u * kUnit + me, a.vec);
-    nstart = unit_start(a.r, u);
-    if (lane == 0 && u) nprev = a.w[u * kUnit - 1];
+// What a lane knows of its 8 elements of one unit.
+struct Seg {
+  uint4 v;           // the words
+  uint32_t tt[8];    // packed table entries (0 past n)
+  uint32_t live;     // elements that exist
+  uint32_t mine;     // their bits
+  bool longs;        // one of them has a codeword above 24 bits
+};
+
+// Table entries of the lane's elements (0 past n), their bits and, when the
+// code has them, whether one is above 24 bits.
+template <bool FULL, bool LONGS>
+__device__ __forceinline__ void seg_lengths(Seg &g, const uint32_t *tab_s) {
+  uint32_t mine = 0, any = 0;
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const uint32_t t = (FULL || (uint32_t)k < g.live) ? tab_s[exponent_of(g.v, k)] : 0u;
+    g.tt[k] = t;
+    mine += t & 0x3Fu;
+    if (LONGS) any |= t;
   }
-  __syncthreads();  // the table
-  for (; u < units; u += stride) {
-    const uint4 v = nx;
-    const unsigned long long start = nstart;
-    const uint32_t prev_word = nprev;
-    const uint64_t un = u + stride;
-    if (un < units) {
-      nx = load8(a.w, a.n, un * kUnit + me, a.vec);
-      nstart = unit_start(a.r, un);
-      if (lane == 0) nprev = a.w[un * kUnit - 1];
+  g.mine = mine;
+  g.longs = LONGS && (any & kLongCode) != 0;
+}
+
+// The lane's codewords, MSB first, ORed into the image from bit `rel` on:
+// up to 64 bits (the usual case) gathered in two registers and placed with
+// up to three ORs, longer runs word by word.
+__device__ __forceinline__ void seg_pack(const Seg &g, uint32_t rel, bool any_long,
+                                         const uint32_t *code_s, uint32_t *image) {
+  if (!g.mine) return;
+  uint32_t cw[kPerThread], ln[kPerThread];
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    ln[k] = g.tt[k] & 0x3Fu;
+    cw[k] = g.tt[k] >> 8;
+  }
+  if (any_long) {  // warp-uniform; rare
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k)
+      if (ln[k] > (uint32_t)kPackedCodeBits) cw[k] = code_s[exponent_of(g.v, k)];
+  }
+  const uint32_t o = rel & 31u, wk = rel >> 5;
+  if (g.mine <= 64) {
+    uint32_t hi = 0, lo = 0;
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {  // (hi:lo) = (hi:lo) << ln | cw, ln <= 32
+      hi = __funnelshift_lc(lo, hi, ln[k]);
+      lo = __funnelshift_lc(0u, lo, ln[k]) | cw[k];
     }
-    const uint64_t i0 = u * kUnit + me;
-    const uint32_t live = live_of(i0, a.n);
-    uint32_t e[kPerThread], l[kPerThread], cw[kPerThread];
-    uint32_t mine = 0, last = 0;
+    // left-align the `mine` bits: first bit at bit 63
+    const uint32_t s = 64u - g.mine;
+    uint32_t ah, al;
+    if (s >= 32) {
+      ah = lo << (s - 32);
+      al = 0;
+    } else {
+      ah = __funnelshift_l(lo, hi, s);
+      al = lo << s;
+    }
+    atomicOr(&image[wk], ah >> o);
+    if (o + g.mine > 32) atomicOr(&image[wk + 1], __funnelshift_r(al, ah, o));
+    if (o + g.mine > 64) atomicOr(&image[wk + 2], al << (32 - o));
+  } else {
+    // `cur` holds the pending bits left-aligned, `nb` of them
+    uint32_t w = wk, nb = o, cur = 0;
+    bool first = true;
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k) {
-      e[k] = exponent_of(v, k);
-      const uint2 t = tab_s[e[k]];
-      const bool in = (uint32_t)k < live;
-      l[k] = in ? t.y : 0u;
-      cw[k] = in ? t.x : 0u;
-      mine += l[k];
-      last = in ? l[k] : last;
+      if (ln[k]) {
+        const uint32_t tot = nb + ln[k];
+        if (tot >= 32) {
+          const uint32_t t = cur | (cw[k] >> (tot - 32));
+          if (first) atomicOr(&image[w], t);  // the previous lane may own its first bits
+          else image[w] = t;
+          first = false;
+          ++w;
+          nb = tot - 32;
+          cur = __funnelshift_lc(0u, cw[k], 32 - nb);  // 0 when nb == 0
+        } else {
+          cur |= cw[k] << (32 - tot);
+          nb = tot;
+        }
+      }
     }
-    uint32_t incl = mine;
+    if (nb) atomicOr(&image[w], cur);  // the last, partial word, which the next lane may share
+  }
+}
+
+// Sign/mantissa bytes of the lane's elements: bit 15 -> bit 7, bits 0-6
+// kept; two per word.
+__device__ __forceinline__ void seg_sign_mantissa(uint8_t *sm, const Seg &g, uint64_t i0) {
+  if (!g.live) return;
+  uint32_t sm2[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t t = word_of(g.v, q);
+    sm2[q] = (t & 0x007F007Fu) | ((t >> 8) & 0x00800080u);  // bytes 0 and 2
+  }
+  const uint2 smv = make_uint2(__byte_perm(sm2[0], sm2[1], 0x6420),
+                               __byte_perm(sm2[2], sm2[3], 0x6420));
+  if (g.live == kPerThread) {
+    *reinterpret_cast<uint2 *>(sm + i0) = smv;
+  } else {
+    for (uint32_t k = 0; k < g.live; ++k)
+      sm[i0 + k] = (uint8_t)((k < 4 ? smv.x : smv.y) >> (8 * (k & 3)));
+  }
+}
+
+// The element a boundary goes to: the first of the step whose codeword
+// starts at or after bit r (from the step's origin), and that start.  The
+// step's 512 lane segments of 8 elements, in element order, have their
+// first bits in seg_start and their words in seg_words: a binary search
+// finds the last segment that starts before r, a walk over its lengths the
+// element.  The caller guarantees that some element of the step starts at
+// or after r.
+__device__ __forceinline__ uint32_t boundary_element(int r, const int *seg_start,
+                                                     const uint4 *seg_words,
+                                                     const uint32_t *tab_s, int *start) {
+  int s = 0;
+#pragma unroll
+  for (int d = kStepUnits * 32 / 2; d; d >>= 1)
+    if (seg_start[s + d] < r) s += d;
+  int p = seg_start[s];
+  uint32_t k = 0;
+  if (p < r) {  // else s is 0 and the step's first element takes the boundary
+    const uint4 v = seg_words[s];
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      if (p < r) {
+        p += (int)(tab_s[exponent_of(v, j)] & 0x3Fu);
+        ++k;
+      }
+    }
+  }
+  *start = p;
+  return (uint32_t)s * kPerThread + k;  // k = 8: the next segment's first element
+}
+
+// Tiles are claimed one at a time from a counter, in batch order, so that
+// the blocks finish together.  A tile is packed in steps of 4096 elements,
+// each with its own image; two images alternate, so that the one a step
+// writes out is cleared during the next step, before the step after that
+// packs into it.  A step whose last word is partial (and not the tile's
+// last step) hands it to the next step, which ORs it into its first word.
+// The block keeps its job's descriptor and code tables in shared memory
+// and reloads them when a claimed tile belongs to another job.
+__global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int count,
+                                                        uint64_t all_tiles,
+                                                        unsigned long long *counter) {
+  __shared__ uint32_t tab_s[256];
+  __shared__ uint32_t code_s[256];
+  __shared__ uint32_t images[2][kStepWords];
+  __shared__ uint32_t unit_bits[kStepUnits];  // bits of each unit
+  __shared__ int seg_start[kStepUnits * 32];  // first bit of each lane segment
+  __shared__ uint4 seg_words[kStepUnits * 32];
+  __shared__ uint32_t carry[2];               // a step's partial last word
+  __shared__ uint32_t prev_len;               // codeword length of the element before the step
+  __shared__ unsigned long long claim;
+  __shared__ Job J;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) claim = atomicAdd(counter, 1ull);
+  for (int j = tid; j < 2 * kStepWords; j += kThreads) (&images[0][0])[j] = 0;
+  __syncthreads();
+  uint64_t g = claim;  // the tile, numbered through the batch
+  if (g >= all_tiles) return;
+  int job = job_of(jobs, count, g);
+  static_assert(sizeof(Job) % 8 == 0, "descriptor copied in 8-byte words");
+  for (int j = tid; j < (int)(sizeof(Job) / 8); j += kThreads)
+    reinterpret_cast<unsigned long long *>(&J)[j] =
+        reinterpret_cast<const unsigned long long *>(&jobs[job])[j];
+  __syncthreads();
+  tab_s[tid] = J.tab[tid];
+  code_s[tid] = J.tab[256 + tid];
+  uint64_t t = g - J.tile_base;  // the tile within its job
+  int q = 0;                     // the step within the tile
+  const uint32_t lane_off = (uint32_t)warp * kUnit + (uint32_t)lane * kPerThread;
+  // the step's words (units w and w + 8), and for thread 0 the element before
+  uint4 na, nb;
+  uint32_t nprev = 0;
+  {
+    const uint64_t i = t * kTile + lane_off;
+    na = load8(J.w, J.n, i, J.vec);
+    nb = load8(J.w, J.n, i + kStep / 2, J.vec);
+    if (tid == 0 && t) nprev = J.w[t * kTile - 1];
+  }
+  int cur = 0;
+  uint32_t stale = 0;  // words the other image holds from the step before
+  unsigned long long pos = J.tile_start[t];  // the step's first bit
+  __syncthreads();  // the tables
+  for (;;) {
+    uint32_t *image = images[cur];
+    const uint64_t step_first = t * kTile + (uint64_t)q * kStep;
+    Seg A, B;
+    A.v = na;
+    B.v = nb;
+    const uint32_t prev_word = nprev;
+    const uint64_t i_a = step_first + lane_off, i_b = i_a + kStep / 2;
+    A.live = live_of(i_a, J.n);
+    B.live = live_of(i_b, J.n);
+    if (step_first + kStep <= J.n) {  // uniform
+      if (J.longs) {
+        seg_lengths<true, true>(A, tab_s);
+        seg_lengths<true, true>(B, tab_s);
+      } else {
+        seg_lengths<true, false>(A, tab_s);
+        seg_lengths<true, false>(B, tab_s);
+      }
+    } else {
+      seg_lengths<false, true>(A, tab_s);
+      seg_lengths<false, true>(B, tab_s);
+    }
+    // both units' bits scanned over the warp at once, 16 bits each (a unit
+    // holds at most 8192)
+    const uint32_t both = A.mine | (B.mine << 16);
+    uint32_t incl = both;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-      if (lane >= d) incl += t;
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += y;
     }
-    const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-    // length of element i0 - 1's codeword: the previous lane's last, or
-    // for lane 0 the previous unit's last element (0 for element 0)
-    const uint32_t up = __shfl_up_sync(0xFFFFFFFFu, last, 1);
-    const uint32_t prev_len = lane ? up : (u ? tab_s[exponent(prev_word)].y : 0u);
-    // positions below are relative to `origin`, the first bit of the word
-    // this unit begins in
-    const unsigned long long origin = start & ~31ull;
-    const uint32_t lead = (uint32_t)(start & 31u);
-    const uint32_t rel = lead + incl - mine;  // this lane's first bit
-
-    // codewords, MSB first, ORed into the warp's image of the unit's words:
-    // up to 32 bits (the usual case) gathered in one register and placed
-    // with one or two ORs, up to 64 in two registers, longer runs word by word
-    __syncwarp();  // the previous unit's words are written out and cleared
-    if (mine && mine <= 32) {
-      uint32_t acc = 0;
+    const uint32_t excl = incl - both;
+    if (lane == 31) {
+      unit_bits[warp] = incl & 0xFFFFu;
+      unit_bits[warp + 8] = incl >> 16;
+    }
+    __syncthreads();
+    {
+      uint32_t *other = images[cur ^ 1];
+      for (uint32_t j = tid; j < stale; j += kThreads) other[j] = 0;
+    }
+    // every warp scans the 16 unit counts
+    const uint32_t ub = lane < kStepUnits ? unit_bits[lane] : 0u;
+    uint32_t ui = ub;
 #pragma unroll
-      for (int k = 0; k < kPerThread; ++k) acc = (acc << l[k]) | cw[k];
-      const uint32_t o = rel & 31u, wk = rel >> 5;
-      const uint32_t left = acc << (32 - mine);  // first bit at bit 31
-      atomicOr(&words[wk], left >> o);
-      if (o + mine > 32) atomicOr(&words[wk + 1], left << (32 - o));
-    } else if (mine) {
-      if (mine <= 64) {
-        unsigned long long acc = 0;
-#pragma unroll
-        for (int k = 0; k < kPerThread; ++k) acc = (acc << l[k]) | cw[k];
-        const uint32_t o = rel & 31u, wk = rel >> 5;
-        const unsigned long long left = acc << (64 - mine);
-        const uint32_t hi = (uint32_t)(left >> 32), lo = (uint32_t)left;
-        atomicOr(&words[wk], hi >> o);
-        atomicOr(&words[wk + 1], __funnelshift_r(lo, hi, o));
-        if (o + mine > 64) atomicOr(&words[wk + 2], __funnelshift_lc(0u, lo, 32 - o));
-      } else {
-        // `cur` holds the pending bits left-aligned, `nb` of them
-        uint32_t wk = rel >> 5, nb = rel & 31u, cur = 0;
-        bool first = true;
-#pragma unroll
-        for (int k = 0; k < kPerThread; ++k) {
-          if (l[k]) {
-            const uint32_t tot = nb + l[k];
-            if (tot >= 32) {
-              const uint32_t t = cur | (cw[k] >> (tot - 32));
-              if (first) atomicOr(&words[wk], t);  // the previous lane may own its first bits
-              else words[wk] = t;
-              first = false;
-              ++wk;
-              nb = tot - 32;
-              cur = __funnelshift_lc(0u, cw[k], 32 - nb);  // 0 when nb == 0
-            } else {
-              cur |= cw[k] << (32 - tot);
-              nb = tot;
-            }
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, ui, d);
+      if (lane >= d) ui += y;
+    }
+    const uint32_t bits = __shfl_sync(0xFFFFFFFFu, ui, 31);
+    const uint32_t off_a = __shfl_sync(0xFFFFFFFFu, ui - ub, warp);
+    const uint32_t off_b = __shfl_sync(0xFFFFFFFFu, ui - ub, warp + 8);
+    if (tid == 0) prev_len = step_first ? tab_s[exponent(prev_word)] & 0x3Fu : 0u;
+    const unsigned long long origin = pos & ~31ull;
+    const uint32_t lead = (uint32_t)(pos & 31u);
+    const uint32_t rel_a = lead + off_a + (excl & 0xFFFFu), rel_b = lead + off_b + (excl >> 16);
+    seg_pack(A, rel_a, J.longs && __any_sync(0xFFFFFFFFu, A.longs), code_s, image);
+    seg_pack(B, rel_b, J.longs && __any_sync(0xFFFFFFFFu, B.longs), code_s, image);
+    seg_start[warp * 32 + lane] = (int)rel_a;
+    seg_start[(warp + 8) * 32 + lane] = (int)rel_b;
+    seg_words[warp * 32 + lane] = A.v;
+    seg_words[(warp + 8) * 32 + lane] = B.v;
+    seg_sign_mantissa(J.sm, A, i_a);
+    seg_sign_mantissa(J.sm, B, i_b);
+    const bool last_step = q + 1 == kStepsPerTile || step_first + kStep >= J.n;
+    if (last_step && tid == 0) claim = atomicAdd(counter, 1ull);
+    __syncthreads();  // the image is complete; the step's starts and words are in place
+    // the next step: of this tile, or the next claimed tile
+    const uint64_t gn = last_step ? claim : g;
+    const int jn = !last_step ? job : gn < all_tiles ? job_of(jobs, count, gn) : job;
+    const uint64_t tn = !last_step ? t : gn - jobs[jn].tile_base;
+    const int qn = last_step ? 0 : q + 1;
+    if (gn < all_tiles) {  // in flight while this step is finished
+      const Job &N = jobs[jn];
+      const uint16_t *w = last_step ? N.w : J.w;
+      const uint64_t n = last_step ? N.n : J.n;
+      const bool vec = last_step ? N.vec != 0 : J.vec != 0;
+      const uint64_t first_n = tn * kTile + (uint64_t)qn * kStep;
+      const uint64_t i = first_n + lane_off;
+      na = load8(w, n, i, vec);
+      nb = load8(w, n, i + kStep / 2, vec);
+      if (tid == 0 && first_n) nprev = w[first_n - 1];
+    }
+    // the chunks and blocks whose first codeword start is in this step:
+    // those that begin after the start of the element before the step (any,
+    // for the first step of the tensor) and at or before the start of its
+    // last element; one thread each.  The first boundary after a start p is
+    // floor(p / chunk bits) + 1; bit offsets stay below 2^37, so p / 32
+    // fits 32 bits and floor(p / (32 m)) = floor(floor(p / 32) / m).
+    {
+      const uint64_t live_elems = J.n - step_first < kStep ? J.n - step_first : kStep;
+      const uint32_t e_last = (uint32_t)live_elems - 1;
+      const uint32_t last_len =
+          tab_s[exponent_of(seg_words[e_last / kPerThread], e_last % kPerThread)] & 0x3Fu;
+      const unsigned long long last_start = pos + bits - last_len;
+      const unsigned long long prev_start = pos - prev_len;
+      const uint32_t hi_w = (uint32_t)(last_start >> 5), lo_w = (uint32_t)(prev_start >> 5);
+      const uint64_t c_lo = step_first ? div_words(lo_w, J.chunk_words, J.chunk_magic) + 1 : 0;
+      const uint64_t c_hi = div_words(hi_w, J.chunk_words, J.chunk_magic);
+      const uint64_t q_lo = step_first ? div_words(lo_w, J.block_words, J.block_magic) + 1 : 0;
+      const uint64_t q_hi = div_words(hi_w, J.block_words, J.block_magic);
+      const uint64_t nc = c_hi + 1 - c_lo, nq = q_hi + 1 > q_lo ? q_hi + 1 - q_lo : 0;
+      // boundary b goes to lane b / 8 of warp b % 8, so that every warp
+      // takes its share of the searches' latency
+      const uint32_t me_b = (uint32_t)lane * (kThreads / 32) + (uint32_t)warp;
+      for (uint64_t b = me_b; b < nc + nq; b += kThreads) {
+        const bool chunk = b < nc;
+        const uint64_t idx = chunk ? c_lo + b : q_lo + (b - nc);
+        const unsigned long long at = idx * (chunk ? J.chunk_bits : J.block_bits);
+        const int r = (int)((long long)at - (long long)origin);
+        int start;
+        const uint32_t e = boundary_element(r, seg_start, seg_words, tab_s, &start);
+        const uint32_t elem = (uint32_t)step_first + e;
+        if (chunk) {
+          if (idx < J.chunks) {
+            J.gap[idx] = (uint8_t)(start - r);
+            J.first_elem[idx] = elem;
           }
+        } else if (idx < J.num_blocks) {
+          J.bpos[idx] = elem;
         }
-        if (nb) atomicOr(&words[wk], cur);  // the last, partial word, which the next lane may share
       }
     }
-    __syncwarp();
-    // words out, and cleared for the next unit: ORed where a neighbouring
-    // unit owns part of the word (cleared beforehand), stored otherwise
-    const uint64_t base = origin >> 5;
-    const uint32_t end_bits = lead + total;
+    // words out; the first word of a step after the first holds the
+    // previous step's partial last word too
+    const uint32_t end_bits = lead + bits;
     const uint32_t nwords = (end_bits + 31) >> 5;
-    const bool shared_last = (end_bits & 31u) && u + 1 < units;
-    for (uint32_t j = lane; j < nwords; j += 32) {
-      const uint32_t t = bswap32(words[j]);
-      words[j] = 0;
-      if ((j == 0 && lead) || (j == nwords - 1 && shared_last)) atomicOr(&a.bs32[base + j], t);
-      else a.bs32[base + j] = t;
-    }
-    // chunks and blocks whose first codeword start is one of these
-    // elements: those that begin after element i0 - 1's codeword start and
-    // at or before element i0 + live - 1's.  The first chunk (block) after
-    // that start is floor(start / chunk bits) + 1; bit offsets stay below
-    // 2^37, so offset / 32 fits 32 bits and floor(p / (32 m)) =
-    // floor(floor(p / 32) / m).  Blocks are skipped unless one begins
-    // inside this unit (warp-wide test, before any lane leaves).
-    const int p_last = (int)(rel + mine - last);
-    const uint32_t pw = (uint32_t)((origin + rel - prev_len) >> 5);  // element i0 - 1's start / 32
-    // chunk c_base begins o_c bits before `origin` (0 <= o_c < chunk bits)
-    const uint64_t c_base = div_words((uint32_t)(origin >> 5), a.chunk_words, a.chunk_magic);
-    const int o_c = (int)(origin - c_base * a.chunk_bits);
-    const uint32_t pw0 = __shfl_sync(0xFFFFFFFFu, pw, 0);
-    const int p_end = __shfl_sync(0xFFFFFFFFu, p_last, 31);
-    const uint64_t q0 = u ? div_words(pw0, a.block_words, a.block_magic) + 1 : 0;
-    const bool blocks_here = (long long)(q0 * a.block_bits) - (long long)origin <= p_end;
-    if (!live) continue;
-
-    // sign/mantissa bytes: bit 15 -> bit 7, bits 0-6 kept; two per word
-    uint32_t sm2[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t t = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
-      sm2[q] = (t & 0x007F007Fu) | ((t >> 8) & 0x00800080u);  // bytes 0 and 2
-    }
-    const uint2 smv = make_uint2(__byte_perm(sm2[0], sm2[1], 0x6420),
-                                 __byte_perm(sm2[2], sm2[3], 0x6420));
-    if (live == kPerThread) {
-      *reinterpret_cast<uint2 *>(a.sm + i0) = smv;
-    } else {
-      for (uint32_t k = 0; k < live; ++k)
-        a.sm[i0 + k] = (uint8_t)((k < 4 ? smv.x : smv.y) >> (8 * (k & 3)));
-    }
-
-    // the first chunk boundary after element i0 - 1's start; then, while
-    // it lies at or before this lane's last start, the first element
-    // starting at or after it (counted without branches) takes it
-    const uint32_t x = (uint32_t)((int)rel - (int)prev_len + o_c + (int)a.chunk_bits);
-    const uint32_t jc = i0 ? __umulhi(x, a.chunk_m32) : 0u;  // floor(x / chunk_bits)
-    int cb = (int)(jc * a.chunk_bits) - o_c;
-    if (cb <= p_last) {
-      uint64_t c = c_base + jc;
-      do {
-        uint32_t k = 0, bits = 0;
-        int pj = (int)rel;
-#pragma unroll
-        for (int j = 0; j < kPerThread; ++j) {
-          const bool before = l[j] && pj < cb;
-          k += before ? 1u : 0u;
-          bits += before ? l[j] : 0u;
-          pj += (int)l[j];
-        }
-        if (c < a.chunks) {
-          a.gap[c] = (uint8_t)((int)(rel + bits) - cb);
-          a.first_elem[c] = (uint32_t)(i0 + k);
-        }
-        ++c;
-        cb += (int)a.chunk_bits;
-      } while (cb <= p_last);
-    }
-    if (blocks_here) {  // the same for block boundaries (about one unit in 25)
-      uint64_t q = i0 ? div_words(pw, a.block_words, a.block_magic) + 1 : 0;
-      int qb = (int)((long long)(q * a.block_bits) - (long long)origin);
-      int pk = (int)rel;
-#pragma unroll
-      for (int k = 0; k < kPerThread; ++k) {
-        if (l[k]) {
-          for (; qb <= pk; qb += (int)a.block_bits, ++q)
-            if (q < a.num_blocks) a.bpos[q] = (uint32_t)(i0 + k);
-          pk += (int)l[k];
-        }
+    const bool end_partial = (end_bits & 31u) != 0;
+    const uint64_t base = origin >> 5;
+    for (uint32_t j = tid; j < nwords; j += kThreads) {
+      uint32_t val = image[j];
+      if (j == 0 && q && lead) val |= carry[cur ^ 1];
+      const bool head = j == 0 && q == 0 && lead, tail = j == nwords - 1 && end_partial;
+      if (tail && !last_step) {
+        carry[cur] = val;
+      } else {
+        if (head) J.edge[2 * t] = val;  // shared with the tile before
+        if (tail) J.edge[2 * t + 1] = val;  // shared with the tile after
+        if (!head && !tail) J.bs32[base + j] = bswap32(val);
       }
     }
+    if (gn >= all_tiles) break;  // uniform
+    if (jn != job) {  // another tensor: its descriptor and tables
+      __syncthreads();
+      for (int j = tid; j < (int)(sizeof(Job) / 8); j += kThreads)
+        reinterpret_cast<unsigned long long *>(&J)[j] =
+            reinterpret_cast<const unsigned long long *>(&jobs[jn])[j];
+      __syncthreads();
+      tab_s[tid] = J.tab[tid];
+      code_s[tid] = J.tab[256 + tid];
+      __syncthreads();
+      job = jn;
+    }
+    stale = nwords;
+    cur ^= 1;
+    pos = last_step ? J.tile_start[tn] : pos + bits;
+    g = gn;
+    t = tn;
+    q = qn;
   }
 }
 
 // ---- finish --------------------------------------------------------------
-struct FinishArgs {
-  const uint8_t *gap;
-  const uint32_t *first_elem;
-  uint8_t *gaps_packed;
-  uint8_t *counts;
-  uint32_t *bpos;
-  unsigned int *maxima;  // block, chunk, group of 32 chunks
-  uint64_t chunk_bits, chunks, block_bits, total, last_start;
-  uint32_t num_blocks, n;
-};
-
-// one thread per group of 8 chunks (5 packed gap bytes); chunks is a
-// multiple of 128
-__global__ void finish_chunks(const FinishArgs a) {
-  const uint64_t g = blockIdx.x * 256ull + threadIdx.x;
-  const uint64_t c0 = g * 8;
-  if (c0 >= a.chunks) return;
-  unsigned long long v = 0;
-  uint32_t mc = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint64_t c = c0 + j, cb = c * a.chunk_bits;
-    uint32_t gv = a.gap[c];
-    // a chunk that begins inside the last codeword: the distance to the end
-    if (a.n && cb > a.last_start && cb < a.total) gv = (uint32_t)(a.total - cb);
-    const uint32_t k = a.first_elem[c + 1] - a.first_elem[c];
-    a.counts[c] = (uint8_t)k;
-    mc = mc > k ? mc : k;
-    v = (v << 5) | gv;
-  }
-#pragma unroll
-  for (int j = 0; j < 5; ++j) a.gaps_packed[g * 5 + j] = (uint8_t)(v >> (32 - 8 * j));
-  atomicMax(&a.maxima[1], mc);
-  if (c0 % 32 == 0) {
-    const uint64_t e = c0 + 32 < a.chunks ? c0 + 32 : a.chunks;
-    atomicMax(&a.maxima[2], a.first_elem[e] - a.first_elem[c0]);
-  }
+// first element of chunk c: n for the chunks that begin after the last
+// codeword start (no element starts at or after them) and for the end entry
+__device__ __forceinline__ uint32_t chunk_first(const Job &J, uint64_t c) {
+  return c * J.chunk_bits > J.last_start ? (uint32_t)J.n : J.first_elem[c];
 }
 
 // entry b of block_out_pos as the format stores it: n for the blocks after
 // the last codeword start and for the end entry
-__device__ __forceinline__ uint32_t block_pos(const FinishArgs &a, uint64_t b) {
-  if (b >= a.num_blocks || (a.n && b * a.block_bits > a.last_start)) return a.n;
-  return a.bpos[b];
+__device__ __forceinline__ uint32_t block_pos(const Job &J, uint64_t b) {
+  if (b >= J.num_blocks || b * (uint64_t)J.block_bits > J.last_start) return (uint32_t)J.n;
+  return J.bpos[b];
 }
 
-// one thread per entry of block_out_pos.  Rewriting an entry with its
-// block_pos leaves its block_pos unchanged, so a neighbour may read it
-// before or after the rewrite.
-__global__ void finish_blocks(const FinishArgs a) {
-  const uint64_t b = blockIdx.x * 256ull + threadIdx.x;
-  if (b > a.num_blocks) return;
-  const uint32_t here = block_pos(a, b);
-  if (b < a.num_blocks) atomicMax(&a.maxima[0], block_pos(a, b + 1) - here);
-  a.bpos[b] = here;
+// Grid (x, job).  A job's threads in three ranges: one per group of 8 chunks
+// (5 packed gap bytes; chunks is a multiple of 128), one per entry of
+// block_out_pos, one per tile; then all of them over the paddings and
+// tables.  Rewriting an entry of block_out_pos with its block_pos leaves its
+// block_pos unchanged, so a neighbour may read it before or after the
+// rewrite.
+__global__ void finish_kernel(const Job *jobs) {
+  const Job &J = jobs[blockIdx.y];
+  const uint64_t i = blockIdx.x * 256ull + threadIdx.x;
+  const uint64_t groups = J.chunks / 8;
+  if (i < groups) {
+    const uint64_t c0 = i * 8;
+    unsigned long long v = 0;
+    uint32_t mc = 0;
+    const uint32_t f0 = chunk_first(J, c0);
+    uint32_t f = f0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint64_t c = c0 + j, cb = c * J.chunk_bits;
+      // a chunk that begins inside the last codeword: the distance to the end
+      const uint32_t gv =
+          cb > J.last_start ? (cb < J.total ? (uint32_t)(J.total - cb) : 0u) : J.gap[c];
+      const uint32_t fn = chunk_first(J, c + 1);
+      const uint32_t k = fn - f;
+      f = fn;
+      J.counts[c] = (uint8_t)k;
+      mc = mc > k ? mc : k;
+      v = (v << 5) | gv;
+    }
+#pragma unroll
+    for (int j = 0; j < 5; ++j) J.gaps_packed[i * 5 + j] = (uint8_t)(v >> (32 - 8 * j));
+    atomicMax(&J.maxima[1], mc);
+    if (c0 % 32 == 0) {
+      const uint64_t e = c0 + 32 < J.chunks ? c0 + 32 : J.chunks;
+      atomicMax(&J.maxima[2], chunk_first(J, e) - f0);
+    }
+  } else if (i - groups <= J.num_blocks) {
+    const uint64_t b = i - groups;
+    const uint32_t here = block_pos(J, b);
+    if (b < J.num_blocks) atomicMax(&J.maxima[0], block_pos(J, b + 1) - here);
+    J.bpos[b] = here;
+  } else if (i - groups - J.num_blocks - 1 < J.tiles) {
+    // the word a tile shares with the one before it, and the stream's last
+    // word when it is partial (unless that is the same word)
+    const uint64_t t = i - groups - J.num_blocks - 1;
+    const unsigned long long s = J.tile_start[t], e = J.tile_start[t + 1];
+    const bool head = (s & 31u) != 0;
+    if (head) J.bs32[s >> 5] = bswap32(J.edge[2 * (t - 1) + 1] | J.edge[2 * t]);
+    if (t + 1 == J.tiles && (e & 31u) && !(head && (s >> 5) == (e >> 5)))
+      J.bs32[e >> 5] = bswap32(J.edge[2 * t + 1]);
+  }
+  const uint64_t all = (uint64_t)gridDim.x * 256;
+  const uint4 *luts_src = reinterpret_cast<const uint4 *>(J.tab + 512);
+  for (uint64_t j = i; j < J.luts_vec4; j += all) reinterpret_cast<uint4 *>(J.luts)[j] = luts_src[j];
+  if (i < 256) J.code_lengths[i] = reinterpret_cast<const uint8_t *>(J.tab + 512 + 4 * J.luts_vec4)[i];
+  // paddings: each at most a block of the bitstream plus 16 bytes
+  for (int k = 0; k < 4; ++k)
+    for (uint64_t j = i; j < J.zero_bytes[k]; j += all) J.zero[k][j] = 0;
 }
 
 bool grid_for(uint64_t items, uint64_t per_cta, unsigned *grid) {
@@ -684,21 +823,22 @@ struct df11_gpu_build {
   uint32_t code[256];
   std::vector<uint32_t> luts;
   uint64_t total = 0, last_start = 0, num_blocks = 0, chunks = 0;
+  uint64_t tiles = 0;
   bool vec = false;
-  Ranges r{};
-  uint64_t ranges = 0;
-  // device scratch, phase 1: histogram, {codeword, length} per exponent,
-  // range totals and first bits, pack-block first bits within their range
   cudaStream_t stream = nullptr;  // the stream the scratch was allocated on
+  // device scratch, phase 1: histogram and last element, maxima (cleared
+  // there), each tile's counts
   void *scratch1 = nullptr;
-  unsigned long long *d_hist = nullptr, *d_range_total = nullptr;
-  uint2 *d_tab = nullptr;
-  // device scratch, phase 2: per-chunk first element and gap, the maxima
+  unsigned long long *d_hist = nullptr;
+  unsigned int *d_max = nullptr;  // block, chunk, group of 32 chunks
+  uint16_t *d_tile_hist = nullptr;
+  // device scratch, phase 2: per tile its bits, first bit and shared
+  // words, per chunk first element and gap
   void *scratch2 = nullptr;
-  uint32_t *d_first = nullptr;
-  unsigned int *d_max = nullptr;
+  uint32_t *d_tile_bits = nullptr;
+  unsigned long long *d_tile_start = nullptr;
+  uint32_t *d_edge = nullptr, *d_first = nullptr;
   uint8_t *d_gap = nullptr;
-  uint8_t *d_tables = nullptr;  // the luts, then the code lengths, for the prepare kernel
 };
 
 namespace {
@@ -738,13 +878,6 @@ struct Staging {
 };
 Staging g_staging;
 
-// what one tensor's phase 1 reads back and sends
-struct BeginSlot {
-  unsigned long long hist[257];  // the counts, then the last element
-  uint2 tab[256];
-  unsigned long long total;
-};
-
 df11_status check_begin_args(const uint16_t *d_bf16, uint64_t n, uint32_t C, uint32_t T) {
   if (n && !d_bf16) return DF11_ERR_NULL;
   if (C < 4 || C > 28 || C % 4) return DF11_ERR_INVALID;
@@ -753,6 +886,11 @@ df11_status check_begin_args(const uint16_t *d_bf16, uint64_t n, uint32_t C, uin
   if ((uintptr_t)d_bf16 & 1) return DF11_ERR_ALIGN;
   return DF11_OK;
 }
+
+// scratch layout of phase 1
+constexpr uint64_t kHistBytes = 257 * sizeof(unsigned long long);  // counts, last element
+constexpr uint64_t kMaxOffset = (kHistBytes + 255) & ~255ull;      // maxima
+constexpr uint64_t kTileHistOffset = kMaxOffset + 256;             // per-tile counts
 
 }  // namespace
 
@@ -793,9 +931,10 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     for (auto *h : hs) df11_gpu_build_free(h);
     return st;
   };
-  const uint64_t slots = resident(sums_kernel), hist_slots = resident(hist_kernel);
+  const uint64_t hist_slots = resident(hist_kernel);
   std::lock_guard<std::mutex> lock(g_staging.mu);
-  BeginSlot *stage = static_cast<BeginSlot *>(g_staging.get(sizeof(BeginSlot) * count));
+  auto *stage = static_cast<unsigned long long(*)[257]>(
+      g_staging.get(sizeof(unsigned long long[257]) * count));
   if (!stage) return DF11_ERR_NOMEM;
   // one event per tensor: its counts are back
   struct Events {
@@ -820,83 +959,56 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     h->T = T;
     h->vec = ((uintptr_t)d_bf16[i] & 15) == 0;
     h->stream = s;
-    // contiguous ranges of units, one per resident sums thread block.  A
-    // range's bits fit 32 bits: at most 2^24 units over at least
-    // min(units, SMs) ranges, at most 8192 bits per unit.
-    h->r.units = (h->n + kUnit - 1) / kUnit;
-    h->ranges = h->r.units < slots ? h->r.units : slots;
-    h->r.per = h->ranges ? (h->r.units + h->ranges - 1) / h->ranges : 1;
-    if (h->ranges) h->ranges = (h->r.units + h->r.per - 1) / h->r.per;
-    const uint64_t o_tab = round256(257 * sizeof(unsigned long long));
-    const uint64_t o_tot = o_tab + round256(256 * sizeof(uint2));
-    const uint64_t o_rs = o_tot + round256(h->ranges * sizeof(unsigned long long) + 8);
-    const uint64_t o_loc = o_rs + round256((h->ranges + 1) * sizeof(unsigned long long));
-    const uint64_t bytes1 = o_loc + round256(h->r.units * sizeof(uint32_t) + 4);
+    h->tiles = (h->n + kTile - 1) / kTile;
+    const uint64_t bytes1 = kTileHistOffset + round256(h->tiles * 512);
     if (scratch_alloc(&h->scratch1, bytes1, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
     char *base1 = static_cast<char *>(h->scratch1);
     h->d_hist = reinterpret_cast<unsigned long long *>(base1);
-    h->d_tab = reinterpret_cast<uint2 *>(base1 + o_tab);
-    h->d_range_total = reinterpret_cast<unsigned long long *>(base1 + o_tot);
-    h->r.range_start = reinterpret_cast<unsigned long long *>(base1 + o_rs);
-    h->r.local = reinterpret_cast<uint32_t *>(base1 + o_loc);
-    if (cudaMemsetAsync(h->d_hist, 0, 257 * sizeof(unsigned long long), s) != cudaSuccess)
+    h->d_max = reinterpret_cast<unsigned int *>(base1 + kMaxOffset);
+    h->d_tile_hist = reinterpret_cast<uint16_t *>(base1 + kTileHistOffset);
+    // the per-tile counts are written whole by the kernel
+    if (cudaMemsetAsync(h->scratch1, 0, kTileHistOffset, s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
     if (h->n) {
-      const uint64_t tiles = (h->n + kPerCta - 1) / kPerCta;
-      const unsigned grid = (unsigned)(tiles < hist_slots ? tiles : hist_slots);
-      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_hist, h->d_hist + 256);
+      const unsigned grid = (unsigned)(h->tiles < hist_slots ? h->tiles : hist_slots);
+      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_hist, h->d_hist + 256,
+                                            h->d_tile_hist);
       if (cudaGetLastError() != cudaSuccess) return fail(DF11_ERR_CUDA);
     }
-    if (cudaMemcpyAsync(stage[i].hist, h->d_hist, sizeof(stage[i].hist), cudaMemcpyDeviceToHost,
-                        s) != cudaSuccess ||
+    if (cudaMemcpyAsync(stage[i], h->d_hist, sizeof(stage[i]), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
         cudaEventRecord(events[i], s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
   }
 
   // codebooks (host: 256 symbols each), each as soon as its counts are
-  // back, while the device computes the previous tensors' bit offsets; then
-  // every unit's first bit and the totals
+  // back, while the device counts the later tensors; the stream's length
+  // is the sum of count x code length
   for (int i = 0; i < count; ++i) {
     df11_gpu_build *h = hs[i];
     if (cudaEventSynchronize(events[i]) != cudaSuccess) return fail(DF11_ERR_CUDA);
     uint64_t hist64[256];
-    for (int k = 0; k < 256; ++k) hist64[k] = stage[i].hist[k];
+    for (int k = 0; k < 256; ++k) hist64[k] = stage[i][k];
     h->longest = df11_internal::codebook(hist64, h->len, h->code, h->luts);
-    for (int k = 0; k < 256; ++k) stage[i].tab[k] = make_uint2(h->code[k], h->len[k]);
-    stage[i].total = 0;
-    if (cudaMemcpyAsync(h->d_tab, stage[i].tab, sizeof(stage[i].tab), cudaMemcpyHostToDevice,
-                        s) != cudaSuccess)
-      return fail(DF11_ERR_CUDA);
-    if (h->ranges) {
-      sums_kernel<<<(unsigned)h->ranges, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_tab,
-                                                           h->r, h->d_range_total);
-      scan_kernel<<<1, kScanThreads, 0, s>>>(h->d_range_total, h->ranges, h->r.range_start);
-      if (cudaGetLastError() != cudaSuccess ||
-          cudaMemcpyAsync(&stage[i].total, h->r.range_start + h->ranges,
-                          sizeof(stage[i].total), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return fail(DF11_ERR_CUDA);
-    }
-  }
-  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(DF11_ERR_CUDA);
-
-  for (int i = 0; i < count; ++i) {
-    df11_gpu_build *h = hs[i];
-    h->total = stage[i].total;
-    if (h->n) h->last_start = h->total - h->len[(stage[i].hist[256] >> 7) & 0xFF];
+    uint64_t total = 0;
+    for (int k = 0; k < 256; ++k) total += hist64[k] * h->len[k];
+    h->total = total;
+    if (h->n) h->last_start = h->total - h->len[(stage[i][256] >> 7) & 0xFF];
     const uint64_t block_bits = 8ull * C * T;
     h->num_blocks = (h->total + block_bits - 1) / block_bits;
     h->chunks = h->num_blocks * T;
-    const uint64_t o_max = round256((h->chunks + 1) * sizeof(uint32_t));
-    const uint64_t o_gap = o_max + 256;
-    const uint64_t o_tables = o_gap + round256(h->chunks + 1);
-    const uint64_t table_bytes = h->luts.size() * 4 + 256;
-    if (scratch_alloc(&h->scratch2, o_tables + round256(table_bytes), s) != cudaSuccess)
-      return fail(DF11_ERR_CUDA);
+    const uint64_t o_start = round256(h->tiles * 4);  // tile bits first
+    const uint64_t o_edge = o_start + round256((h->tiles + 1) * 8);
+    const uint64_t o_first = o_edge + round256(h->tiles * 8);
+    const uint64_t o_gap = o_first + round256((h->chunks + 1) * sizeof(uint32_t));
+    const uint64_t bytes2 = o_gap + round256(h->chunks + 1);
+    if (scratch_alloc(&h->scratch2, bytes2, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
     char *base2 = static_cast<char *>(h->scratch2);
-    h->d_first = reinterpret_cast<uint32_t *>(base2);
-    h->d_max = reinterpret_cast<unsigned int *>(base2 + o_max);
+    h->d_tile_bits = reinterpret_cast<uint32_t *>(base2);
+    h->d_tile_start = reinterpret_cast<unsigned long long *>(base2 + o_start);
+    h->d_edge = reinterpret_cast<uint32_t *>(base2 + o_edge);
+    h->d_first = reinterpret_cast<uint32_t *>(base2 + o_first);
     h->d_gap = reinterpret_cast<uint8_t *>(base2 + o_gap);
-    h->d_tables = reinterpret_cast<uint8_t *>(base2 + o_tables);
     fill_params(h, &params[i]);
     std::memcpy(code_lengths + 256 * (size_t)i, h->len, 256);
   }
@@ -946,89 +1058,134 @@ df11_status df11_gpu_build_finish_batched(df11_gpu_build *const *handles, int co
                            handles[i]->n ? (const void *)d_bf16[i] : nullptr};
     st = df11_internal::check_device_pointers(ptrs, 8);
   }
+  // One staging area and one device block for the whole call: the job
+  // descriptors, each job's tables (packed codes, codewords, luts, code
+  // lengths), the tile counter and the maxima (zeros on the way in, the
+  // results on the way out).
   std::unique_lock<std::mutex> lock(g_staging.mu, std::defer_lock);
-  size_t stage_bytes = 0;
-  std::vector<size_t> off(count > 0 ? count : 0);
-  if (st == DF11_OK) {
-    for (int i = 0; i < count; ++i) {
-      off[i] = stage_bytes;  // luts, code lengths, then the maxima read back
-      stage_bytes += (handles[i]->luts.size() * 4 + 256 + 16 + 15) & ~(size_t)15;
-    }
-    lock.lock();
-  }
-  uint8_t *stage = st == DF11_OK ? static_cast<uint8_t *>(g_staging.get(stage_bytes)) : nullptr;
-  if (st == DF11_OK && !stage) st = DF11_ERR_NOMEM;
+  std::vector<size_t> tab_off(count > 0 ? count : 0);
+  const size_t jobs_bytes = sizeof(Job) * (size_t)count;
+  size_t bytes = (jobs_bytes + 255) & ~(size_t)255;
   for (int i = 0; i < count && st == DF11_OK; ++i) {
-    df11_gpu_build *h = handles[i];
-    const df11_gpu_build_out &o = outs[i];
-    const uint64_t chunks = h->chunks, n = h->n;
-    const uint64_t bs_bytes = chunks * h->C + 16, gaps_bytes = chunks * 5 / 8 + 16;
-    const uint64_t sm_bytes = (n + 15) / 16 * 16;
-    const uint64_t bs_written = (h->total + 31) / 32 * 4;  // the units' words
-    const size_t lut_bytes = h->luts.size() * 4;
-    uint8_t *st_luts = stage + off[i], *st_lens = st_luts + lut_bytes;
-    std::memcpy(st_luts, h->luts.data(), lut_bytes);
-    std::memcpy(st_lens, h->len, 256);
-    if (cudaMemcpyAsync(h->d_tables, st_luts, lut_bytes + 256, cudaMemcpyHostToDevice, s) !=
-        cudaSuccess) {
-      st = DF11_ERR_CUDA;
-      break;
-    }
-    uint32_t *bs32 = reinterpret_cast<uint32_t *>(o.bitstream);
-    // every byte the kernels do not write: the padding after each buffer
-    PrepareArgs pr{h->d_first, h->d_gap, chunks, (uint32_t)n, h->r, bs32, h->d_max,
-                   {o.bitstream + bs_written, o.gaps + chunks * 5 / 8, o.chunk_counts + chunks,
-                    o.sign_mantissa + n},
-                   {(uint32_t)(bs_bytes - bs_written), (uint32_t)(gaps_bytes - chunks * 5 / 8), 16u,
-                    (uint32_t)(sm_bytes - n)},
-                   reinterpret_cast<const uint4 *>(h->d_tables), reinterpret_cast<uint4 *>(o.luts),
-                   (uint32_t)(lut_bytes / 16), h->d_tables + lut_bytes, o.code_lengths};
-    prepare_kernel<<<148 * 4, 256, 0, s>>>(pr);
-    const uint32_t chunk_bits = 8 * h->C, block_bits = 8 * h->C * h->T;
-    const uint32_t chunk_words = h->C / 4, block_words = h->C / 4 * h->T;
-    const PackArgs pa{d_bf16[i], n, h->vec, h->d_tab, h->r, bs32, o.sign_mantissa, h->d_gap,
-                      h->d_first, o.block_out_pos, chunks, (uint32_t)h->num_blocks,
-                      chunk_bits, block_bits, chunk_words, block_words,
-                      chunk_words > 1 ? UINT64_MAX / chunk_words + 1 : 0,
-                      block_words > 1 ? UINT64_MAX / block_words + 1 : 0,
-                      (uint32_t)(((1ull << 32) + chunk_bits - 1) / chunk_bits)};
-    if (h->r.units) {
-      const uint64_t want = resident(pack_kernel), ctas = (h->r.units + 7) / 8;
-      const unsigned grid = (unsigned)(ctas < want ? ctas : want);
-      pack_kernel<<<grid, kThreads, 0, s>>>(pa);
-    }
-    const FinishArgs fa{h->d_gap, h->d_first, o.gaps, o.chunk_counts, o.block_out_pos,
-                        h->d_max, 8ull * h->C, chunks, 8ull * h->C * h->T, h->total,
-                        h->last_start, (uint32_t)h->num_blocks, (uint32_t)n};
-    unsigned grid;
-    if (chunks) {
-      if (!grid_for(chunks / 8, 256, &grid)) {
-        st = DF11_ERR_TOO_LARGE;
-        break;
+    tab_off[i] = bytes;
+    bytes += (512 * 4 + handles[i]->luts.size() * 4 + 256 + 255) & ~(size_t)255;
+  }
+  const size_t ctl_off = bytes;  // counter, then 3 maxima per job
+  bytes += 8 + 12 * (size_t)count;
+  if (st == DF11_OK) lock.lock();
+  uint8_t *stage = st == DF11_OK ? static_cast<uint8_t *>(g_staging.get(bytes)) : nullptr;
+  if (st == DF11_OK && !stage) st = DF11_ERR_NOMEM;
+  void *blk = nullptr;
+  if (st == DF11_OK && scratch_alloc(&blk, bytes, s) != cudaSuccess) {
+    blk = nullptr;
+    st = DF11_ERR_CUDA;
+  }
+  uint8_t *dev = static_cast<uint8_t *>(blk);
+  uint64_t all_tiles = 0, max_tiles = 0, max_fin = 0;
+  if (st == DF11_OK) {
+    Job *jobs = reinterpret_cast<Job *>(stage);
+    std::memset(stage + ctl_off, 0, 8 + 12 * (size_t)count);
+    for (int i = 0; i < count; ++i) {
+      df11_gpu_build *h = handles[i];
+      const df11_gpu_build_out &o = outs[i];
+      const uint64_t chunks = h->chunks, n = h->n;
+      const uint64_t bs_bytes = chunks * h->C + 16, gaps_bytes = chunks * 5 / 8 + 16;
+      const uint64_t sm_bytes = (n + 15) / 16 * 16;
+      const uint64_t bs_written = (h->total + 31) / 32 * 4;  // the stream's words
+      const size_t lut_bytes = h->luts.size() * 4;
+      uint32_t *st_tab = reinterpret_cast<uint32_t *>(stage + tab_off[i]);
+      for (int e = 0; e < 256; ++e) {
+        const uint32_t l = h->len[e];
+        st_tab[e] = l <= (uint32_t)kPackedCodeBits ? (h->code[e] << 8) | l : kLongCode | l;
+        st_tab[256 + e] = h->code[e];
       }
-      finish_chunks<<<grid, 256, 0, s>>>(fa);
+      std::memcpy(st_tab + 512, h->luts.data(), lut_bytes);
+      std::memcpy(reinterpret_cast<uint8_t *>(st_tab + 512) + lut_bytes, h->len, 256);
+      Job &J = jobs[i];
+      std::memset(&J, 0, sizeof(J));
+      J.w = d_bf16[i];
+      J.n = n;
+      J.vec = h->vec;
+      J.longs = h->longest > kPackedCodeBits;
+      J.tiles = h->tiles;
+      J.tile_base = all_tiles;
+      J.tile_hist = h->d_tile_hist;
+      J.tile_bits = h->d_tile_bits;
+      J.tile_start = h->d_tile_start;
+      J.edge = h->d_edge;
+      J.tab = reinterpret_cast<const uint32_t *>(dev + tab_off[i]);
+      J.bs32 = reinterpret_cast<uint32_t *>(o.bitstream);
+      J.sm = o.sign_mantissa;
+      J.gaps_packed = o.gaps;
+      J.counts = o.chunk_counts;
+      J.code_lengths = o.code_lengths;
+      J.bpos = o.block_out_pos;
+      J.luts = o.luts;
+      J.first_elem = h->d_first;
+      J.gap = h->d_gap;
+      J.maxima = reinterpret_cast<unsigned int *>(dev + ctl_off + 8) + 3 * i;
+      J.chunks = chunks;
+      J.total = h->total;
+      J.last_start = h->last_start;
+      J.num_blocks = (uint32_t)h->num_blocks;
+      J.luts_vec4 = (uint32_t)(lut_bytes / 16);
+      J.chunk_bits = 8 * h->C;
+      J.block_bits = 8 * h->C * h->T;
+      J.chunk_words = h->C / 4;
+      J.block_words = h->C / 4 * h->T;
+      J.chunk_magic = J.chunk_words > 1 ? UINT64_MAX / J.chunk_words + 1 : 0;
+      J.block_magic = J.block_words > 1 ? UINT64_MAX / J.block_words + 1 : 0;
+      // every byte no kernel writes otherwise: the padding after each buffer
+      J.zero[0] = o.bitstream + bs_written;
+      J.zero[1] = o.gaps + chunks * 5 / 8;
+      J.zero[2] = o.chunk_counts + chunks;
+      J.zero[3] = o.sign_mantissa + n;
+      J.zero_bytes[0] = (uint32_t)(bs_bytes - bs_written);
+      J.zero_bytes[1] = (uint32_t)(gaps_bytes - chunks * 5 / 8);
+      J.zero_bytes[2] = 16u;
+      J.zero_bytes[3] = (uint32_t)(sm_bytes - n);
+      J.fin_threads = chunks / 8 + h->num_blocks + 1 + h->tiles;
+      all_tiles += h->tiles;
+      max_tiles = h->tiles > max_tiles ? h->tiles : max_tiles;
+      max_fin = J.fin_threads > max_fin ? J.fin_threads : max_fin;
     }
-    grid_for(h->num_blocks + 1, 256, &grid);
-    finish_blocks<<<grid, 256, 0, s>>>(fa);
-    if (cudaGetLastError() != cudaSuccess ||
-        cudaMemcpyAsync(st_lens + 256, h->d_max, 3 * sizeof(unsigned int), cudaMemcpyDeviceToHost,
-                        s) != cudaSuccess) {
+    if (cudaMemcpyAsync(dev, stage, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
       st = DF11_ERR_CUDA;
-      break;
+  }
+  if (st == DF11_OK) {
+    const Job *jobs = reinterpret_cast<const Job *>(dev);
+    unsigned long long *counter = reinterpret_cast<unsigned long long *>(dev + ctl_off);
+    unsigned fin_x;
+    if (count > 65535 || !grid_for(max_fin, 256, &fin_x)) st = DF11_ERR_TOO_LARGE;
+    if (st == DF11_OK && all_tiles) {
+      // each tile's first bit, then the tiles packed
+      tile_bits_kernel<<<dim3((unsigned)((max_tiles + 7) / 8), (unsigned)count), 256, 0, s>>>(
+          jobs);
+      scan_kernel<<<(unsigned)count, kScanThreads, 0, s>>>(jobs);
+      const uint64_t slots = resident(pack_kernel);
+      pack_kernel<<<(unsigned)(all_tiles < slots ? all_tiles : slots), kThreads, 0, s>>>(
+          jobs, count, all_tiles, counter);
+    }
+    if (st == DF11_OK) {
+      finish_kernel<<<dim3(fin_x, (unsigned)count), 256, 0, s>>>(jobs);
+      if (cudaGetLastError() != cudaSuccess ||
+          cudaMemcpyAsync(stage + ctl_off + 8, dev + ctl_off + 8, 12 * (size_t)count,
+                          cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        st = DF11_ERR_CUDA;
     }
   }
   if (st == DF11_OK && cudaStreamSynchronize(s) != cudaSuccess) st = DF11_ERR_CUDA;
   for (int i = 0; i < count && st == DF11_OK; ++i) {
-    const df11_gpu_build *h = handles[i];
     unsigned int mx[3];
-    std::memcpy(mx, stage + off[i] + h->luts.size() * 4 + 256, sizeof(mx));
-    fill_params(h, &params[i]);
+    std::memcpy(mx, stage + ctl_off + 8 + 12 * (size_t)i, sizeof(mx));
+    fill_params(handles[i], &params[i]);
     params[i].max_block_elems = mx[0];
     params[i].max_chunk_elems = mx[1];
     params[i].max_warp_elems = mx[2];
   }
   if (st != DF11_OK) cudaStreamSynchronize(s);  // the staging buffer is read until then
   if (lock.owns_lock()) lock.unlock();
+  if (blk) cudaFreeAsync(blk, s);
   for (int i = 0; i < count; ++i) {
     if (!handles[i]) continue;
     handles[i]->stream = s;  // frees follow this call's work
@@ -1048,7 +1205,6 @@ df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uin
 }
 
 }  // extern "C"
-
 // ---- exponent histogram with no allocation --------------------------------
 // Some callers cannot allocate device memory: code running where the CUDA
 // allocator must not be entered (inside an allocator hook, or a pool that is
@@ -1098,15 +1254,17 @@ extern "C" df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t 
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(hd.addr, 0, sizeof(g_exponent_hist), s) != cudaSuccess) return DF11_ERR_CUDA;
   if (n) {
-    const uint64_t tiles = (n + kPerCta - 1) / kPerCta, slots = resident(hist_kernel);
+    const uint64_t tiles = (n + kTile - 1) / kTile, slots = resident(hist_kernel);
     const bool vec = ((uintptr_t)d_bf16 & 15) == 0;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(tiles < slots ? tiles : slots));
     cfg.blockDim = dim3(kThreads);
     cfg.stream = s;
     unsigned long long *no_last = nullptr;
+    uint16_t *no_tiles = nullptr;
     // the launch's own status (not an earlier error of the calling thread)
-    if (cudaLaunchKernelEx(&cfg, hist_kernel, d_bf16, n, vec, hd.addr, no_last) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, hist_kernel, d_bf16, n, vec, hd.addr, no_last, no_tiles) !=
+        cudaSuccess)
       return DF11_ERR_CUDA;
   }
   // straight into the caller's array (a DMA if the caller pinned it)

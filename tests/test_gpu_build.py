@@ -62,7 +62,12 @@ def _decodes_to(d, w_np):
     assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), w_np)
 
 
-@pytest.mark.parametrize("n", [0, 1, 2, 7, 8, 9, 2047, 2048, 2049, 3 * 2048 + 77, 1_000_003])
+# around the histogram's steps (2048) and the pack tiles (4096 elements, 16
+# units of 256); 1,000,003 and 5,000,011 span hundreds of tiles, so that the
+# look-back reads past 32 predecessors
+@pytest.mark.parametrize("n", [0, 1, 2, 7, 8, 9, 255, 256, 257, 2047, 2048, 2049,
+                               3 * 2048 + 77, 4095, 4096, 4097, 3 * 4096 + 1,
+                               37 * 4096 + 2049, 1_000_003, 5_000_011])
 def test_gaussian_sizes(n):
     bits = workloads.gaussian_bf16(n, 0.02, 500 + n, device="cuda")
     d, h, w = _same_as_host(bits)
