@@ -460,6 +460,38 @@ __device__ __forceinline__ uint32_t boundary_element(int r, const int *seg_start
   return (uint32_t)s * kPerThread + k;  // k = 8: the next segment's first element
 }
 
+// The chunks and blocks whose first codeword start is in a step: those
+// that begin after the start of the element before the step (any, for the
+// first step of the tensor) and at or before the start of its last
+// element.  The first boundary after a start p is floor(p / chunk bits) +
+// 1; bit offsets stay below 2^37, so p / 32 fits 32 bits and floor(p / (32
+// m)) = floor(floor(p / 32) / m).  r0 and rq0 are the first chunk and block
+// boundary from the step's origin.
+struct StepRanges {
+  unsigned long long c_lo, q_lo;
+  uint32_t nc, nq;
+  int r0, rq0;
+};
+
+__device__ __forceinline__ StepRanges step_ranges(const Job &J, unsigned long long origin,
+                                                  uint32_t lead, uint32_t bits,
+                                                  uint32_t prev_len, uint32_t last_len,
+                                                  bool tensor_first) {
+  const unsigned long long pos = origin + lead;
+  const uint32_t hi_w = (uint32_t)((pos + bits - last_len) >> 5);
+  const uint32_t lo_w = (uint32_t)((pos - prev_len) >> 5);
+  StepRanges r;
+  r.c_lo = tensor_first ? 0 : div_words(lo_w, J.chunk_words, J.chunk_magic) + 1;
+  r.q_lo = tensor_first ? 0 : div_words(lo_w, J.block_words, J.block_magic) + 1;
+  const unsigned long long c_hi = div_words(hi_w, J.chunk_words, J.chunk_magic);
+  const unsigned long long q_hi = div_words(hi_w, J.block_words, J.block_magic);
+  r.nc = (uint32_t)(c_hi + 1 - r.c_lo);
+  r.nq = q_hi + 1 > r.q_lo ? (uint32_t)(q_hi + 1 - r.q_lo) : 0u;
+  r.r0 = (int)((long long)(r.c_lo * J.chunk_bits) - (long long)origin);
+  r.rq0 = (int)((long long)(r.q_lo * J.block_bits) - (long long)origin);
+  return r;
+}
+
 // Tiles are claimed one at a time from a counter, in batch order, so that
 // the blocks finish together.  A tile is packed in steps of 4096 elements,
 // each with its own image; two images alternate, so that the one a step
@@ -479,6 +511,7 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
   __shared__ uint4 seg_words[kStepUnits * 32];
   __shared__ uint32_t carry[2];               // a step's partial last word
   __shared__ uint32_t prev_len;               // codeword length of the element before the step
+  __shared__ StepRanges ranges;               // of a whole step, from its last thread
   __shared__ unsigned long long claim;
   __shared__ Job J;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -505,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
     const uint64_t i = t * kTile + lane_off;
     na = load8(J.w, J.n, i, J.vec);
     nb = load8(J.w, J.n, i + kStep / 2, J.vec);
-    if (tid == 0 && t) nprev = J.w[t * kTile - 1];
+    if (tid == kThreads - 1 && t) nprev = J.w[t * kTile - 1];
   }
   int cur = 0;
   uint32_t stale = 0;  // words the other image holds from the step before
@@ -521,7 +554,8 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
     const uint64_t i_a = step_first + lane_off, i_b = i_a + kStep / 2;
     A.live = live_of(i_a, J.n);
     B.live = live_of(i_b, J.n);
-    if (step_first + kStep <= J.n) {  // uniform
+    const bool whole = step_first + kStep <= J.n;  // uniform
+    if (whole) {
       if (J.longs) {
         seg_lengths<true, true>(A, tab_s);
         seg_lengths<true, true>(B, tab_s);
@@ -563,9 +597,16 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
     const uint32_t bits = __shfl_sync(0xFFFFFFFFu, ui, 31);
     const uint32_t off_a = __shfl_sync(0xFFFFFFFFu, ui - ub, warp);
     const uint32_t off_b = __shfl_sync(0xFFFFFFFFu, ui - ub, warp + 8);
-    if (tid == 0) prev_len = step_first ? tab_s[exponent(prev_word)] & 0x3Fu : 0u;
     const unsigned long long origin = pos & ~31ull;
     const uint32_t lead = (uint32_t)(pos & 31u);
+    if (tid == kThreads - 1) {
+      // the element before the step; for a whole step this thread's last
+      // element is the step's last
+      const uint32_t pl = step_first ? tab_s[exponent(prev_word)] & 0x3Fu : 0u;
+      prev_len = pl;
+      if (whole) ranges = step_ranges(J, origin, lead, bits, pl, B.tt[kPerThread - 1] & 0x3Fu,
+                                      step_first == 0);
+    }
     const uint32_t rel_a = lead + off_a + (excl & 0xFFFFu), rel_b = lead + off_b + (excl >> 16);
     seg_pack(A, rel_a, J.longs && __any_sync(0xFFFFFFFFu, A.longs), code_s, image);
     seg_pack(B, rel_b, J.longs && __any_sync(0xFFFFFFFFu, B.longs), code_s, image);
@@ -592,45 +633,36 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
       const uint64_t i = first_n + lane_off;
       na = load8(w, n, i, vec);
       nb = load8(w, n, i + kStep / 2, vec);
-      if (tid == 0 && first_n) nprev = w[first_n - 1];
+      if (tid == kThreads - 1 && first_n) nprev = w[first_n - 1];
     }
-    // the chunks and blocks whose first codeword start is in this step:
-    // those that begin after the start of the element before the step (any,
-    // for the first step of the tensor) and at or before the start of its
-    // last element; one thread each.  The first boundary after a start p is
-    // floor(p / chunk bits) + 1; bit offsets stay below 2^37, so p / 32
-    // fits 32 bits and floor(p / (32 m)) = floor(floor(p / 32) / m).
+    // the chunks and blocks whose first codeword start is in this step, one
+    // thread each (a step that ends the tensor works out its ranges here)
     {
-      const uint64_t live_elems = J.n - step_first < kStep ? J.n - step_first : kStep;
-      const uint32_t e_last = (uint32_t)live_elems - 1;
-      const uint32_t last_len =
-          tab_s[exponent_of(seg_words[e_last / kPerThread], e_last % kPerThread)] & 0x3Fu;
-      const unsigned long long last_start = pos + bits - last_len;
-      const unsigned long long prev_start = pos - prev_len;
-      const uint32_t hi_w = (uint32_t)(last_start >> 5), lo_w = (uint32_t)(prev_start >> 5);
-      const uint64_t c_lo = step_first ? div_words(lo_w, J.chunk_words, J.chunk_magic) + 1 : 0;
-      const uint64_t c_hi = div_words(hi_w, J.chunk_words, J.chunk_magic);
-      const uint64_t q_lo = step_first ? div_words(lo_w, J.block_words, J.block_magic) + 1 : 0;
-      const uint64_t q_hi = div_words(hi_w, J.block_words, J.block_magic);
-      const uint64_t nc = c_hi + 1 - c_lo, nq = q_hi + 1 > q_lo ? q_hi + 1 - q_lo : 0;
-      // boundary b goes to lane b / 8 of warp b % 8, so that every warp
-      // takes its share of the searches' latency
-      const uint32_t me_b = (uint32_t)lane * (kThreads / 32) + (uint32_t)warp;
-      for (uint64_t b = me_b; b < nc + nq; b += kThreads) {
-        const bool chunk = b < nc;
-        const uint64_t idx = chunk ? c_lo + b : q_lo + (b - nc);
-        const unsigned long long at = idx * (chunk ? J.chunk_bits : J.block_bits);
-        const int r = (int)((long long)at - (long long)origin);
+      StepRanges rg;
+      if (whole) {
+        rg = ranges;
+      } else {
+        const uint32_t e_last = (uint32_t)(J.n - step_first) - 1;
+        const uint32_t last_len =
+            tab_s[exponent_of(seg_words[e_last / kPerThread], e_last % kPerThread)] & 0x3Fu;
+        rg = step_ranges(J, origin, lead, bits, prev_len, last_len, step_first == 0);
+      }
+      for (uint32_t b = tid; b < rg.nc + rg.nq; b += kThreads) {
+        const bool chunk = b < rg.nc;
+        const int r = chunk ? rg.r0 + (int)(b * J.chunk_bits)
+                            : rg.rq0 + (int)((b - rg.nc) * J.block_bits);
         int start;
         const uint32_t e = boundary_element(r, seg_start, seg_words, tab_s, &start);
         const uint32_t elem = (uint32_t)step_first + e;
         if (chunk) {
+          const uint64_t idx = rg.c_lo + b;
           if (idx < J.chunks) {
             J.gap[idx] = (uint8_t)(start - r);
             J.first_elem[idx] = elem;
           }
-        } else if (idx < J.num_blocks) {
-          J.bpos[idx] = elem;
+        } else {
+          const uint64_t idx = rg.q_lo + (b - rg.nc);
+          if (idx < J.num_blocks) J.bpos[idx] = elem;
         }
       }
     }
