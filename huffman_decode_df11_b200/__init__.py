@@ -301,35 +301,34 @@ class Df11Device:
     interleave: int = 1  # rows interleaved per 16 columns in the stream (1: row-major)
 
     @classmethod
-    def _in_block(cls, params: Params, block: torch.Tensor, spans: dict, shape: tuple,
-                  interleave: int) -> "Df11Device":
+    def _in_block(cls, params: Params, block: torch.Tensor, offs: tuple, sizes: tuple,
+                  shape: tuple, interleave: int) -> "Df11Device":
         """A tensor whose buffers are byte ranges of one device allocation
-        (`spans`: name -> (offset, bytes, dtype)).  The tensor view of a
+        (offsets and sizes in the order of _BUFFERS).  The tensor view of a
         buffer is made when the buffer is first used; pointers for a decode
         come straight from the allocation."""
         d = cls.__new__(cls)
-        d.params, d.shape, d.interleave, d.decode_table = params, shape, interleave, None
-        d._block, d._spans = block, spans
-        off, nbytes, _ = spans["chunk_counts"]
-        d.chunk_counts = block[off:off + nbytes]  # a field with a default: made now
+        d.__dict__.update(params=params, shape=shape, interleave=interleave, decode_table=None,
+                          _block=block, _offs=offs, _sizes=sizes)
         return d
 
     def __getattr__(self, name):
         # only reached for a buffer of a _in_block tensor not yet viewed
-        spans = self.__dict__.get("_spans")
-        if spans is None or name not in spans:
+        dd = self.__dict__
+        i = _BUFFER_INDEX.get(name)
+        if i is None or "_offs" not in dd:
             raise AttributeError(name)
-        off, nbytes, dtype = spans[name]
-        v = self.__dict__["_block"][off:off + nbytes]
-        if dtype is not None:
-            v = v.view(dtype)
-        self.__dict__[name] = v
+        off = dd["_offs"][i]
+        v = dd["_block"][off:off + dd["_sizes"][i]]
+        if _BUFFERS[i][1] is not None:
+            v = v.view(_BUFFERS[i][1])
+        dd[name] = v
         return v
 
     def _ptr(self, name: str) -> int:
-        spans = self.__dict__.get("_spans")
-        if spans is not None and name in spans and name not in self.__dict__:
-            return self.__dict__["_block"].data_ptr() + spans[name][0]
+        dd = self.__dict__
+        if "_offs" in dd and name not in dd:
+            return dd["_block"].data_ptr() + dd["_offs"][_BUFFER_INDEX[name]]
         return getattr(self, name).data_ptr()
 
     @property
@@ -348,11 +347,24 @@ class Df11Device:
                    + ((self.chunk_counts,) if self.chunk_counts is not None else ()))
 
     def desc(self, out: torch.Tensor, counts: bool = True) -> TensorDesc:
-        cc = self.chunk_counts.data_ptr() if (counts and self.chunk_counts is not None) else None
+        cc = (self._ptr("chunk_counts") if counts and ("_offs" in self.__dict__
+                                                        or self.chunk_counts is not None)
+              else None)
         dt = self.decode_table.data_ptr() if self.decode_table is not None else None
         p = self._ptr
         return TensorDesc(p("bitstream"), p("gaps"), cc, p("block_out_pos"), p("luts"),
                           p("code_lengths"), p("sign_mantissa"), out.data_ptr(), dt, self.params)
+
+
+# the buffers of a device tensor in the order of df11_gpu_build_out, with the
+# view each gets (None: bytes)
+_BUFFERS = (("bitstream", None), ("gaps", None), ("chunk_counts", None),
+            ("block_out_pos", torch.int32), ("luts", torch.int32), ("code_lengths", None),
+            ("sign_mantissa", None))
+_BUFFER_INDEX = {name: i for i, (name, _) in enumerate(_BUFFERS)}
+# a tensor built by _in_block has no chunk_counts attribute until first use;
+# the default stays in the constructor
+del Df11Device.chunk_counts
 
 
 def _np_to(t: np.ndarray, device, pin: bool = False) -> torch.Tensor:
@@ -449,33 +461,33 @@ def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, deco
     L = lib()
     sh = _stream_handle(stream)
     vp = ctypes.c_void_p
-    ptrs = (vp * count)(*[f.data_ptr() if f.numel() else None for f in flats])
-    ns = (ctypes.c_uint64 * count)(*[f.numel() for f in flats])
+    nums = [f.numel() for f in flats]
+    ptrs = (vp * count)(*[f.data_ptr() if k else None for f, k in zip(flats, nums)])
+    ns = (ctypes.c_uint64 * count)(*nums)
     params = (Params * count)()
     lens = (ctypes.c_uint8 * (256 * count))()
     handles = (vp * count)()
     _check(L.df11_gpu_build_begin_batched(ptrs, ns, count, chunk_bytes, threads_per_block, sh,
                                           params, ctypes.cast(lens, vp), handles),
            "df11_gpu_build_begin_batched")
-    outs = (GpuBuildOut * count)()
     try:
         # every output buffer of the call in one allocation, each at a
-        # 256-byte boundary (at least 16 bytes, so that no pointer is NULL)
+        # 256-byte boundary (at least 16 bytes, so that no pointer is NULL),
+        # in the order of df11_gpu_build_out
         layout, total = [], 0
-        for f, p in zip(flats, params):
-            nb = int(p.num_blocks)
+        for k, p in zip(nums, params):
+            nb = p.num_blocks
             chunks = nb * threads_per_block
-            sizes = (chunks * chunk_bytes + 16, chunks * 5 // 8 + 16, chunks + 16, 4 * (nb + 1),
-                     1024 * int(p.num_luts), 256, (f.numel() + 15) // 16 * 16)
+            sizes = (chunks * chunk_bytes + 16, chunks * 5 // 8 + 16, chunks + 16, 4 * nb + 4,
+                     1024 * p.num_luts, 256, (k + 15) & ~15)
             offs = []
             for nbytes in sizes:
                 offs.append(total)
-                total += (max(nbytes, 16) + 255) & ~255
-            layout.append((offs, sizes))
+                total += ((nbytes if nbytes > 16 else 16) + 255) & ~255
+            layout.append((tuple(offs), sizes))
         block = torch.empty(max(total, 256), dtype=torch.uint8, device=flats[0].device)
         base = block.data_ptr()
-        for i, (offs, _) in enumerate(layout):
-            outs[i] = GpuBuildOut(*[base + o for o in offs])
+        outs = (vp * (7 * count))(*[base + o for offs, _ in layout for o in offs])
     except BaseException:
         for hnd in handles:
             L.df11_gpu_build_free(hnd)
@@ -483,21 +495,12 @@ def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, deco
     _check(L.df11_gpu_build_finish_batched(handles, count, ptrs, outs, params, sh),
            "df11_gpu_build_finish_batched")
     out = []
-    for p, (offs, sizes), shape in zip(params, layout, shapes):
-        spans = {name: (o, nbytes, dt) for name, o, nbytes, dt in
-                 zip(_GPU_BUILD_FIELDS, offs, sizes, _GPU_BUILD_DTYPES)}
-        d = Df11Device._in_block(Params.from_buffer_copy(p), block, spans, shape,
-                                 int(interleave))
+    for i, ((offs, sizes), shape) in enumerate(zip(layout, shapes)):
+        d = Df11Device._in_block(params[i], block, offs, sizes, shape, int(interleave))
         if decode_table:
             d.decode_table = build_decode_table(d, stream)
         out.append(d)
     return out
-
-
-# the order of df11_gpu_build_out, and the view each buffer gets
-_GPU_BUILD_FIELDS = ("bitstream", "gaps", "chunk_counts", "block_out_pos", "luts",
-                     "code_lengths", "sign_mantissa")
-_GPU_BUILD_DTYPES = (None, None, None, torch.int32, torch.int32, None, None)
 
 
 def exponent_histogram(w: torch.Tensor, stream=None) -> np.ndarray:

@@ -858,11 +858,8 @@ struct df11_gpu_build {
   uint64_t tiles = 0;
   bool vec = false;
   cudaStream_t stream = nullptr;  // the stream the scratch was allocated on
-  // device scratch, phase 1: histogram and last element, maxima (cleared
-  // there), each tile's counts
+  // device scratch, phase 1: each tile's counts
   void *scratch1 = nullptr;
-  unsigned long long *d_hist = nullptr;
-  unsigned int *d_max = nullptr;  // block, chunk, group of 32 chunks
   uint16_t *d_tile_hist = nullptr;
   // device scratch, phase 2: per tile its bits, first bit and shared
   // words, per chunk first element and gap
@@ -919,10 +916,22 @@ df11_status check_begin_args(const uint16_t *d_bf16, uint64_t n, uint32_t C, uin
   return DF11_OK;
 }
 
-// scratch layout of phase 1
-constexpr uint64_t kHistBytes = 257 * sizeof(unsigned long long);  // counts, last element
-constexpr uint64_t kMaxOffset = (kHistBytes + 255) & ~255ull;      // maxima
-constexpr uint64_t kTileHistOffset = kMaxOffset + 256;             // per-tile counts
+// phase 1's counts and last element of one tensor, in a block for the call
+constexpr uint64_t kHistBytes = (257 * sizeof(unsigned long long) + 255) & ~255ull;
+
+// A stream per device for phase 1's copies of the counts, so that they do
+// not queue between the histogram kernels on the caller's stream (created
+// once, non-blocking, kept for the process).
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
 
 }  // namespace
 
@@ -955,11 +964,16 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     if (st != DF11_OK) return st;
   }
   cudaStream_t s = (cudaStream_t)stream;
+  cudaStream_t side = side_stream();
+  if (!side) return DF11_ERR_CUDA;
   std::vector<df11_gpu_build *> hs(count, nullptr);
+  void *hblk = nullptr;  // the call's counts
   auto fail = [&](df11_status st) {
     // copies into the staging buffer may still be queued: let them land
     // before the buffer is released to another call
     cudaStreamSynchronize(s);
+    cudaStreamSynchronize(side);
+    if (hblk) cudaFreeAsync(hblk, s);
     for (auto *h : hs) df11_gpu_build_free(h);
     return st;
   };
@@ -968,7 +982,8 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
   auto *stage = static_cast<unsigned long long(*)[257]>(
       g_staging.get(sizeof(unsigned long long[257]) * count));
   if (!stage) return DF11_ERR_NOMEM;
-  // one event per tensor: its counts are back
+  // per tensor: its kernel is done (caller's stream), its counts are back
+  // (side stream)
   struct Events {
     std::vector<cudaEvent_t> e;
     ~Events() {
@@ -976,11 +991,15 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
         if (x) cudaEventDestroy(x);
     }
   } ev;
-  ev.e.assign(count, nullptr);
-  for (int i = 0; i < count; ++i)
-    if (cudaEventCreateWithFlags(&ev.e[i], cudaEventDisableTiming) != cudaSuccess)
-      return DF11_ERR_CUDA;
-  const std::vector<cudaEvent_t> &events = ev.e;
+  ev.e.assign(2 * (size_t)count, nullptr);
+  for (auto &x : ev.e)
+    if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) return DF11_ERR_CUDA;
+  cudaEvent_t *done = ev.e.data(), *back = ev.e.data() + count;
+  if (scratch_alloc(&hblk, kHistBytes * count, s) != cudaSuccess) {
+    hblk = nullptr;
+    return fail(DF11_ERR_CUDA);
+  }
+  if (cudaMemsetAsync(hblk, 0, kHistBytes * count, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
 
   // histograms, and each tensor's last element (its codeword ends the stream)
   for (int i = 0; i < count; ++i) {
@@ -992,24 +1011,23 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     h->vec = ((uintptr_t)d_bf16[i] & 15) == 0;
     h->stream = s;
     h->tiles = (h->n + kTile - 1) / kTile;
-    const uint64_t bytes1 = kTileHistOffset + round256(h->tiles * 512);
-    if (scratch_alloc(&h->scratch1, bytes1, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
-    char *base1 = static_cast<char *>(h->scratch1);
-    h->d_hist = reinterpret_cast<unsigned long long *>(base1);
-    h->d_max = reinterpret_cast<unsigned int *>(base1 + kMaxOffset);
-    h->d_tile_hist = reinterpret_cast<uint16_t *>(base1 + kTileHistOffset);
     // the per-tile counts are written whole by the kernel
-    if (cudaMemsetAsync(h->scratch1, 0, kTileHistOffset, s) != cudaSuccess)
+    if (scratch_alloc(&h->scratch1, round256(h->tiles * 512) + 256, s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
+    h->d_tile_hist = static_cast<uint16_t *>(h->scratch1);
+    unsigned long long *hist =
+        reinterpret_cast<unsigned long long *>(static_cast<char *>(hblk) + kHistBytes * i);
     if (h->n) {
       const unsigned grid = (unsigned)(h->tiles < hist_slots ? h->tiles : hist_slots);
-      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, h->d_hist, h->d_hist + 256,
+      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, hist, hist + 256,
                                             h->d_tile_hist);
       if (cudaGetLastError() != cudaSuccess) return fail(DF11_ERR_CUDA);
     }
-    if (cudaMemcpyAsync(stage[i], h->d_hist, sizeof(stage[i]), cudaMemcpyDeviceToHost, s) !=
+    if (cudaEventRecord(done[i], s) != cudaSuccess ||
+        cudaStreamWaitEvent(side, done[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(stage[i], hist, sizeof(stage[i]), cudaMemcpyDeviceToHost, side) !=
             cudaSuccess ||
-        cudaEventRecord(events[i], s) != cudaSuccess)
+        cudaEventRecord(back[i], side) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
   }
 
@@ -1018,7 +1036,7 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
   // is the sum of count x code length
   for (int i = 0; i < count; ++i) {
     df11_gpu_build *h = hs[i];
-    if (cudaEventSynchronize(events[i]) != cudaSuccess) return fail(DF11_ERR_CUDA);
+    if (cudaEventSynchronize(back[i]) != cudaSuccess) return fail(DF11_ERR_CUDA);
     uint64_t hist64[256];
     for (int k = 0; k < 256; ++k) hist64[k] = stage[i][k];
     h->longest = df11_internal::codebook(hist64, h->len, h->code, h->luts);
@@ -1044,6 +1062,7 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     fill_params(h, &params[i]);
     std::memcpy(code_lengths + 256 * (size_t)i, h->len, 256);
   }
+  cudaFreeAsync(hblk, s);  // every copy of it is done
   for (int i = 0; i < count; ++i) handles[i] = hs[i];
   return DF11_OK;
 }

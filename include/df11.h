@@ -333,8 +333,8 @@ typedef struct df11_gpu_build df11_gpu_build;
  * Phase 1.  d_bf16: n BF16 words in device memory (2-byte aligned; 16-byte
  * alignment lets the kernels load 8 words at a time and must then hold in
  * phase 2 too).  Same chunk_bytes / threads_per_block rules as df11_build.
- * Computes the histogram and the code, synchronises `stream`, and on
- * success fills *params (n, total_bits, chunk_bytes, threads_per_block,
+ * Computes the histogram and the code, waits for the counts (everything
+ * queued on `stream` before them has then run), and on success fills *params (n, total_bits, chunk_bytes, threads_per_block,
  * num_blocks, num_luts, max_len; the max_* counts are filled by phase 2),
  * code_lengths (host, 256 bytes) and *handle, which holds device scratch
  * until phase 2 or df11_gpu_build_free.  The scratch comes from a memory
