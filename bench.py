@@ -712,11 +712,12 @@ def _same_bytes(d, h) -> bool:
 def run_build(args, world, rank, local):
     """The format builder on the device: every tensor of the workload
     compressed from BF16 already in HBM (df11_gpu_build_begin_batched /
-    _finish_batched via compress_on_device_batched, one call per step).  Parity: byte-identical buffers and parameters to
-    the host builder, and a decode back to the original words, before any
-    timing.  A step builds every tensor once; the counts and the stream
-    lengths are read back to the host (three synchronisations per step, in
-    the timed region)."""
+    _finish_batched via compress_on_device_batched, one call per step).
+    Parity: byte-identical buffers and parameters to the host builder, and a
+    decode back to the original words, before any timing.  A step builds
+    every tensor once: the counts come back to the host for the codebooks,
+    and the largest block, chunk and warp counts at the end (two round trips
+    per step, in the timed region)."""
     import huffman_decode_df11_b200 as df11
     device = f"cuda:{local}"
     seed = args.seed + rank

@@ -80,6 +80,13 @@ __device__ __forceinline__ uint32_t exponent_of(const uint4 &v, int k) {
   return (word_of(v, k >> 1) >> ((k & 1) ? 23 : 7)) & 0xFFu;
 }
 
+// entry e of a 256-entry table of 32-bit words, e the exponent of element k:
+// the exponent field times 4 is the byte offset
+__device__ __forceinline__ uint32_t entry_of(const uint32_t *table, const uint4 &v, int k) {
+  const uint32_t off = (word_of(v, k >> 1) >> ((k & 1) ? 21 : 5)) & 0x3FCu;
+  return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(table) + off);
+}
+
 // how many of elements i0 .. i0+7 exist (0..8)
 __device__ __forceinline__ uint32_t live_of(uint64_t i0, uint64_t n) {
   return i0 >= n ? 0u : (n - i0 >= (uint64_t)kPerThread ? (uint32_t)kPerThread : (uint32_t)(n - i0));
@@ -337,7 +344,7 @@ __device__ __forceinline__ void seg_lengths(Seg &g, const uint32_t *tab_s) {
   uint32_t mine = 0, any = 0;
 #pragma unroll
   for (int k = 0; k < kPerThread; ++k) {
-    const uint32_t t = (FULL || (uint32_t)k < g.live) ? tab_s[exponent_of(g.v, k)] : 0u;
+    const uint32_t t = (FULL || (uint32_t)k < g.live) ? entry_of(tab_s, g.v, k) : 0u;
     g.tt[k] = t;
     mine += t & 0x3Fu;
     if (LONGS) any |= t;
@@ -361,7 +368,7 @@ __device__ __forceinline__ void seg_pack(const Seg &g, uint32_t rel, bool any_lo
   if (any_long) {  // warp-uniform; rare
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k)
-      if (ln[k] > (uint32_t)kPackedCodeBits) cw[k] = code_s[exponent_of(g.v, k)];
+      if (ln[k] > (uint32_t)kPackedCodeBits) cw[k] = entry_of(code_s, g.v, k);
   }
   const uint32_t o = rel & 31u, wk = rel >> 5;
   if (g.mine <= 64) {
@@ -451,7 +458,7 @@ __device__ __forceinline__ uint32_t boundary_element(int r, const int *seg_start
 #pragma unroll
     for (int j = 0; j < kPerThread; ++j) {
       if (p < r) {
-        p += (int)(tab_s[exponent_of(v, j)] & 0x3Fu);
+        p += (int)(entry_of(tab_s, v, j) & 0x3Fu);
         ++k;
       }
     }
@@ -546,15 +553,18 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
   __syncthreads();  // the tables
   for (;;) {
     uint32_t *image = images[cur];
-    const uint64_t step_first = t * kTile + (uint64_t)q * kStep;
+    // element indices fit 32 bits (n < 2^32); a lane's index may wrap only
+    // in the step that ends the tensor, where such a lane has no elements
+    const uint32_t step_first = (uint32_t)(t * kTile) + (uint32_t)q * kStep;
+    const uint32_t n = (uint32_t)J.n;
     Seg A, B;
     A.v = na;
     B.v = nb;
     const uint32_t prev_word = nprev;
-    const uint64_t i_a = step_first + lane_off, i_b = i_a + kStep / 2;
-    A.live = live_of(i_a, J.n);
-    B.live = live_of(i_b, J.n);
-    const bool whole = step_first + kStep <= J.n;  // uniform
+    const uint32_t i_a = step_first + lane_off, i_b = i_a + kStep / 2;
+    const bool whole = n - step_first >= kStep;  // uniform
+    A.live = whole ? kPerThread : live_of((uint64_t)step_first + lane_off, n);
+    B.live = whole ? kPerThread : live_of((uint64_t)step_first + lane_off + kStep / 2, n);
     if (whole) {
       if (J.longs) {
         seg_lengths<true, true>(A, tab_s);
@@ -616,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
     seg_words[(warp + 8) * 32 + lane] = B.v;
     seg_sign_mantissa(J.sm, A, i_a);
     seg_sign_mantissa(J.sm, B, i_b);
-    const bool last_step = q + 1 == kStepsPerTile || step_first + kStep >= J.n;
+    const bool last_step = q + 1 == kStepsPerTile || n - step_first <= kStep;
     if (last_step && tid == 0) claim = atomicAdd(counter, 1ull);
     __syncthreads();  // the image is complete; the step's starts and words are in place
     // the next step: of this tile, or the next claimed tile
@@ -642,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
       if (whole) {
         rg = ranges;
       } else {
-        const uint32_t e_last = (uint32_t)(J.n - step_first) - 1;
+        const uint32_t e_last = n - step_first - 1;
         const uint32_t last_len =
             tab_s[exponent_of(seg_words[e_last / kPerThread], e_last % kPerThread)] & 0x3Fu;
         rg = step_ranges(J, origin, lead, bits, prev_len, last_len, step_first == 0);
