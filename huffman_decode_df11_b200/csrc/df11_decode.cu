@@ -1912,8 +1912,9 @@ size_t ws_shared_bytes(uint32_t C, uint32_t T, uint32_t sm_bytes, uint32_t regio
 
 // Sign/mantissa bytes staged per block in the stage slot or per warp in the
 // warp's own buffer, whichever keeps more thread blocks resident (the slot
-// on a tie); read from global memory only when neither fits.  Measured: at
-// equal residency the slot beats the warp buffer, which beats global reads.
+// on a tie); read from global memory (L2) only when neither fits, or, without
+// chunk counts, when that keeps more blocks resident.  Measured: at equal
+// residency the slot beats the warp buffer, which beats global reads.
 template <int T, int C, bool GEMV = false, bool COUNTS = true>
 df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cudaStream_t s,
                       int instance) {
@@ -1931,7 +1932,11 @@ df11_status launch_ws(KBatch &kb, const uint32_t *blocks, uint32_t sm_stage, cud
   uint64_t best = 0;
   int pick = -1;
   for (int m : order) {
-    if (m == kSmGlobal && pick >= 0) break;
+    // with chunk counts, global reads only when nothing else fits (measured
+    // slower at C = 24 even with a fourth resident block); without counts
+    // also when they keep more blocks resident (the column areas leave room
+    // for two blocks per SM with staged bytes, three without)
+    if (m == kSmGlobal && pick >= 0 && COUNTS) break;
     if (smem[m] > 227 * 1024) continue;
     uint64_t budget = 0;
     const df11_status st = prepare(kern[m], T + 32, smem[m], 3 * instance + m, budget);
