@@ -126,24 +126,33 @@ __device__ __forceinline__ void flush_window(uint32_t (&c)[4], int lo, uint32_t 
 // One element whose exponent times 4 is e4: the window offset times 4 is
 // sh = e4 - lo4 (wrapping below the window), and 1 << sh lands in the
 // counter pair's low register for sh < 32, in the high one for 32 <= sh <
-// 64; the clamped funnel shifts give 0 elsewhere.
+// 64; the clamped funnel shifts give 0 elsewhere.  `oow` collects the
+// offsets: at least 64 once an element lies outside the window.
 __device__ __forceinline__ void count_one(uint32_t e4, uint32_t lo4, uint32_t &n_lo,
-                                          uint32_t &n_hi, uint32_t *h) {
+                                          uint32_t &n_hi, uint32_t &oow) {
   const uint32_t sh = e4 - lo4;
   n_lo += __funnelshift_lc(0u, 1u, sh);
   n_hi += __funnelshift_lc(0u, 1u, sh - 32u);
-  if (sh >= 64u) atomicAdd(&h[e4 >> 2], 1u);
+  oow |= sh;
 }
 
 template <bool FULL>
 __device__ __forceinline__ void count8(const uint4 &v, uint32_t live, uint32_t lo4,
                                        uint32_t (&c)[4], uint32_t *h) {
-  uint32_t n_lo = 0, n_hi = 0;
+  uint32_t n_lo = 0, n_hi = 0, oow = 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const uint32_t u = word_of(v, q);
-    if (FULL || (uint32_t)(2 * q) < live) count_one((u >> 5) & 0x3FCu, lo4, n_lo, n_hi, h);
-    if (FULL || (uint32_t)(2 * q + 1) < live) count_one((u >> 21) & 0x3FCu, lo4, n_lo, n_hi, h);
+    if (FULL || (uint32_t)(2 * q) < live) count_one((u >> 5) & 0x3FCu, lo4, n_lo, n_hi, oow);
+    if (FULL || (uint32_t)(2 * q + 1) < live)
+      count_one((u >> 21) & 0x3FCu, lo4, n_lo, n_hi, oow);
+  }
+  if (oow >= 64u) {  // rare: an exponent outside the window goes to the shared counters
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const uint32_t e4 = (word_of(v, k >> 1) >> ((k & 1) ? 21 : 5)) & 0x3FCu;
+      if ((FULL || (uint32_t)k < live) && e4 - lo4 >= 64u) atomicAdd(&h[e4 >> 2], 1u);
+    }
   }
   c[0] += n_lo & 0x0F0F0F0Fu;
   c[1] += (n_lo >> 4) & 0x0F0F0F0Fu;
@@ -682,17 +691,27 @@ __global__ void __launch_bounds__(kThreads, 3) pack_kernel(const Job *jobs, int 
     const uint32_t nwords = (end_bits + 31) >> 5;
     const bool end_partial = (end_bits & 31u) != 0;
     const uint64_t base = origin >> 5;
-    for (uint32_t j = tid; j < nwords; j += kThreads) {
-      uint32_t val = image[j];
-      if (j == 0 && q && lead) val |= carry[cur ^ 1];
-      const bool head = j == 0 && q == 0 && lead, tail = j == nwords - 1 && end_partial;
-      if (tail && !last_step) {
-        carry[cur] = val;
-      } else {
-        if (head) J.edge[2 * t] = val;  // shared with the tile before
-        if (tail) J.edge[2 * t + 1] = val;  // shared with the tile after
-        if (!head && !tail) J.bs32[base + j] = bswap32(val);
+    // the step's first and last words, which it may share, by the first
+    // and last thread; the rest stored plainly
+    const uint32_t last_w = nwords - 1;
+    if (tid == 0 || tid == kThreads - 1) {
+      const uint32_t j = tid == 0 ? 0u : last_w;
+      if (tid == 0 || last_w != 0) {  // one word: thread 0 takes it
+        uint32_t val = image[j];
+        if (j == 0 && q && lead) val |= carry[cur ^ 1];
+        const bool head = j == 0 && q == 0 && lead, tail = j == last_w && end_partial;
+        if (tail && !last_step) {
+          carry[cur] = val;
+        } else {
+          if (head) J.edge[2 * t] = val;  // shared with the tile before
+          if (tail) J.edge[2 * t + 1] = val;  // shared with the tile after
+          if (!head && !tail) J.bs32[base + j] = bswap32(val);
+        }
       }
+    }
+    {
+      uint32_t *dst = J.bs32 + base;
+      for (uint32_t j = tid + 1; j < last_w; j += kThreads) dst[j] = bswap32(image[j]);
     }
     if (gn >= all_tiles) break;  // uniform
     if (jn != job) {  // another tensor: its descriptor and tables
