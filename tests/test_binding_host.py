@@ -49,3 +49,49 @@ def test_host_builder_interleave_encodes_the_interleaved_order():
     words, end, _ = oracle.decode(h.bitstream, h.code_lengths, h.sign_mantissa, h.n)
     assert end == h.params.total_bits
     assert np.array_equal(words, _loop_order(W, 8))
+
+
+def test_device_tensor_in_one_block_views_and_pointers():
+    """A device-built tensor keeps its buffers as byte ranges of one
+    allocation (Df11Device._in_block): every buffer read as an attribute is
+    that range, with the view the format gives it, and the pointers a decode
+    takes come straight from the allocation, before and after a view is
+    made.  Checked on a host tensor standing in for the allocation."""
+    block = torch.arange(8192, dtype=torch.int32).view(torch.uint8)[:8192]
+    offs = (0, 256, 512, 768, 1024, 2048, 2304)
+    sizes = (40, 21, 32, 12, 1024, 256, 16)
+    d = df11.Df11Device._in_block(df11.Params(), block, offs, sizes, (4, 4), 1)
+    base = block.data_ptr()
+    names = ("bitstream", "gaps", "chunk_counts", "block_out_pos", "luts", "code_lengths",
+             "sign_mantissa")
+    # pointers before any view exists
+    for name, o in zip(names, offs):
+        assert d._ptr(name) == base + o
+    for name, o, nb in zip(names, offs, sizes):
+        v = getattr(d, name)
+        want = block[o:o + nb]
+        if name in ("block_out_pos", "luts"):
+            assert v.dtype == torch.int32 and v.numel() == nb // 4
+            want = want.view(torch.int32)
+        else:
+            assert v.dtype == torch.uint8 and v.numel() == nb
+        assert v.data_ptr() == base + o
+        assert torch.equal(v, want)
+        assert d._ptr(name) == base + o  # and after
+    assert d.device == block.device and d.shape == (4, 4) and d.decode_table is None
+    desc = d.desc(torch.empty(16, dtype=torch.bfloat16))
+    assert desc.bitstream == base and desc.chunk_counts == base + offs[2]
+    assert desc.sign_mantissa == base + offs[6]
+    with pytest.raises(AttributeError):
+        d.not_a_buffer
+
+
+def test_device_tensor_built_the_usual_way_keeps_its_defaults():
+    """The constructor still defaults chunk_counts to None (its class
+    attribute is gone, so that a tensor in one block can make it lazily)."""
+    t = torch.zeros(64, dtype=torch.uint8)
+    d = df11.Df11Device(params=df11.Params(), bitstream=t, gaps=t, block_out_pos=t, luts=t,
+                        code_lengths=t, sign_mantissa=t)
+    assert d.chunk_counts is None and d.interleave == 1 and d.shape == ()
+    desc = d.desc(torch.empty(16, dtype=torch.bfloat16))
+    assert not desc.chunk_counts
