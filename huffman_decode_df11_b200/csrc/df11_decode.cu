@@ -1025,6 +1025,15 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
     const uint32_t G0 = P0 + before;            // first element of this warp
     const uint32_t head = G0 & 15u, span = head + warp_total;
     const uint32_t d = head + incl - cnt;       // my first byte in the region
+    // kSmGlobal: the sign/mantissa bytes of the lane's first whole group of
+    // the output, loaded now so that they arrive from L2 during the walk (or
+    // the move into the region) instead of stalling the output
+    uint4 sv_first = make_uint4(0, 0, 0, 0);
+    if (SM == kSmGlobal && !GEMV) {
+      const uint32_t g0 = (head ? 1u : 0u) + (uint32_t)lane;
+      if (g0 < (span >> 4))
+        sv_first = __ldg(reinterpret_cast<const uint4 *>(tk.sign_mantissa + (G0 & ~15u)) + g0);
+    }
     // kSmWarp: the warp's sign/mantissa bytes, elements [G0 & ~15,
     // round16(G0 + warp_total)), inside the block's range, copied while it
     // decodes (or, without counts, while it moves its bytes into place);
@@ -1125,8 +1134,15 @@ __global__ void __launch_bounds__(T + 32, (T + 32) <= 160 ? 8
         uint32_t sa_sm = sm + 16u * g, sa_rg = region + 16u * g;
         uint4 *o = reinterpret_cast<uint4 *>(out) + 2u * g;
         const uint4 *sp = reinterpret_cast<const uint4 *>(smg) + g;
+        uint4 sv_next = sv_first;  // kSmGlobal: one group ahead
         for (; g < g_end; g += 32, sa_sm += 512u, sa_rg += 512u, o += 64, sp += 32) {
-          const uint4 sv = SM == kSmGlobal ? __ldg(sp) : lds128(sa_sm);
+          uint4 sv;
+          if (SM == kSmGlobal) {
+            sv = sv_next;
+            if (g + 32 < g_end) sv_next = __ldg(sp + 32);
+          } else {
+            sv = lds128(sa_sm);
+          }
           const uint4 rv = lds128(sa_rg);
           sts128_zero(sa_rg);  // leave the region zeroed for the next block
           const uint2 a = fuse4(sv.x, rv.x), c = fuse4(sv.y, rv.y);
