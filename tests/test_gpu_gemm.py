@@ -180,3 +180,32 @@ def test_gemm_flags_corrupt_tables_and_stays_usable():
     torch.cuda.synchronize()
     df11.check_device_error(err)
     _check(h, w, x.view(torch.int16).cpu(), y)
+
+
+def test_gemm_block_shapes_full_size_in_one_call():
+    """The bench's launch: the seven weights of a Qwen3-8B-shaped block
+    (192,937,984 elements), compressed on the device at C = 8 with 128 rows
+    interleaved, times 32 activation rows, in one call; every output within
+    the fp32 sum bound of the float64 product of the original weights (the
+    decode is lossless, so the original weights are the exact reference;
+    computed on the device, one weight at a time)."""
+    shapes = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (12288, 4096),
+              (12288, 4096), (4096, 12288)]
+    batch = 32
+    ws = [workloads.gaussian_bf16(r * c, 1.0 / np.sqrt(c), 700 + i, device="cuda").view(r, c)
+          for i, (r, c) in enumerate(shapes)]
+    ds = df11.compress_on_device_batched(ws, 8, 256, decode_table=True, interleave=R)
+    xs = [workloads.gaussian_bf16(batch * c, 1.0, 800 + i, device="cuda").view(batch, c)
+          for i, (_, c) in enumerate(shapes)]
+    ys = [torch.full((batch, r), 5.0, dtype=torch.float32, device="cuda") for r, _ in shapes]
+    err = df11.new_error_word()
+    df11.decode_gemm(ds, [x.view(torch.bfloat16) for x in xs], ys, err=err)
+    torch.cuda.synchronize()
+    df11.check_device_error(err)
+    for w, x, y, (r, c) in zip(ws, xs, ys, shapes):
+        W = w.view(torch.bfloat16).double()
+        X = x.view(torch.bfloat16).double()
+        ref = X @ W.T
+        bound = _gamma(c) * (X.abs() @ W.abs().T)
+        assert bool(torch.all((y.double() - ref).abs() <= bound)), (r, c)
+        del W, X, ref, bound
