@@ -145,6 +145,8 @@ def lib():
     L.df11_gpu_build_begin_batched.restype = ctypes.c_int
     L.df11_gpu_build_finish_batched.argtypes = [vp, ctypes.c_int, vp, vp, vp, vp]
     L.df11_gpu_build_finish_batched.restype = ctypes.c_int
+    L.df11_gpu_build_layout.argtypes = [vp, ctypes.c_int, vp, vp]
+    L.df11_gpu_build_layout.restype = u64
     L.df11_gpu_build_free.argtypes = [vp]
     L.df11_gpu_build_free.restype = None
     L.df11_decode_gemv.argtypes = [ctypes.POINTER(TensorDesc), ctypes.POINTER(GemvOp),
@@ -447,17 +449,22 @@ def compress_on_device_batched(ws: Sequence[torch.Tensor], chunk_bytes: int = 24
 def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, decode_table,
                                 interleave):
     count = len(ws)
+    # the words as flat contiguous tensors (the interleaved copy, or the
+    # tensor itself: only its address and size go to the library)
     flats, shapes = [], []
+    dev = ws[0].get_device()
     for w in ws:
         if not w.is_cuda:
             raise ValueError("compress_on_device takes CUDA tensors; use compress() for host data")
-        if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        if w.dtype not in _WORD_DTYPES:
             raise TypeError(f"expected BF16 words (bfloat16, int16 or uint16), got {w.dtype}")
-        if w.device != ws[0].device:
+        if w.get_device() != dev:
             raise ValueError("all tensors of one batched build must be on one device")
         shapes.append(tuple(w.shape))
-        flats.append(interleave_rows(w, interleave).contiguous() if interleave != 1
-                     else w.contiguous().reshape(-1))
+        if interleave != 1:
+            flats.append(interleave_rows(w, interleave).contiguous())
+        else:
+            flats.append(w if w.is_contiguous() else w.contiguous())
     L = lib()
     sh = _stream_handle(stream)
     vp = ctypes.c_void_p
@@ -471,23 +478,13 @@ def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, deco
                                           params, ctypes.cast(lens, vp), handles),
            "df11_gpu_build_begin_batched")
     try:
-        # every output buffer of the call in one allocation, each at a
-        # 256-byte boundary (at least 16 bytes, so that no pointer is NULL),
-        # in the order of df11_gpu_build_out
-        layout, total = [], 0
-        for k, p in zip(nums, params):
-            nb = p.num_blocks
-            chunks = nb * threads_per_block
-            sizes = (chunks * chunk_bytes + 16, chunks * 5 // 8 + 16, chunks + 16, 4 * nb + 4,
-                     1024 * p.num_luts, 256, (k + 15) & ~15)
-            offs = []
-            for nbytes in sizes:
-                offs.append(total)
-                total += ((nbytes if nbytes > 16 else 16) + 255) & ~255
-            layout.append((tuple(offs), sizes))
+        # every output buffer of the call in one allocation (df11_gpu_build_layout)
+        offs = (ctypes.c_uint64 * (7 * count))()
+        sizes = (ctypes.c_uint64 * (7 * count))()
+        total = L.df11_gpu_build_layout(params, count, offs, sizes)
         block = torch.empty(max(total, 256), dtype=torch.uint8, device=flats[0].device)
-        base = block.data_ptr()
-        outs = (vp * (7 * count))(*[base + o for offs, _ in layout for o in offs])
+        addr = np.frombuffer(offs, dtype=np.uint64) + np.uint64(block.data_ptr())
+        outs = (vp * (7 * count)).from_buffer(addr)
     except BaseException:
         for hnd in handles:
             L.df11_gpu_build_free(hnd)
@@ -495,8 +492,10 @@ def _compress_on_device_batched(ws, chunk_bytes, threads_per_block, stream, deco
     _check(L.df11_gpu_build_finish_batched(handles, count, ptrs, outs, params, sh),
            "df11_gpu_build_finish_batched")
     out = []
-    for i, ((offs, sizes), shape) in enumerate(zip(layout, shapes)):
-        d = Df11Device._in_block(params[i], block, offs, sizes, shape, int(interleave))
+    il = int(interleave)
+    for i, shape in enumerate(shapes):
+        d = Df11Device._in_block(params[i], block, offs[7 * i:7 * i + 7],
+                                 sizes[7 * i:7 * i + 7], shape, il)
         if decode_table:
             d.decode_table = build_decode_table(d, stream)
         out.append(d)
@@ -531,6 +530,9 @@ def build_decode_table(d: Df11Device, stream=None) -> torch.Tensor:
                                              int(d.params.num_luts), t.data_ptr(),
                                              _stream_handle(stream)), "df11_build_decode_table")
     return t
+
+
+_WORD_DTYPES = (torch.bfloat16, torch.int16, torch.uint16)
 
 
 def _stream_handle(stream) -> Optional[int]:

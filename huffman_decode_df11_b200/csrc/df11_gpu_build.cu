@@ -10,12 +10,13 @@
 // with it the stream's length, the sum over exponents of count x code
 // length, which sizes the outputs.  The device reads the elements twice,
 // in tiles of 16384:
-//   histogram  (phase 1) exponent counts per tile and in all: four-bit
-//              counters in registers for a window of 16 exponents around
-//              the mode of a first sample, spread into byte counters after
-//              every 8 elements and summed over the warp at the end of the
-//              tile; shared counters for exponents outside the window.
-//              Each tile's 256 counts are kept (16 bits each);
+//   histogram  (phase 1) exponent counts per tile and in all, for up to 32
+//              tensors a launch: four-bit counters in registers for a
+//              window of 16 exponents around the mode of a first sample,
+//              spread into byte counters after every 8 elements and summed
+//              over the warp at the end of the tile; shared counters for
+//              exponents outside the window.  Each tile's 256 counts are
+//              kept (16 bits each);
 //   tile bits  (phase 2) each tile's bit count, the dot product of its
 //              counts with the code lengths, and an exclusive scan of them:
 //              every tile's first bit, with no second pass over the
@@ -93,34 +94,65 @@ __device__ __forceinline__ uint32_t live_of(uint64_t i0, uint64_t n) {
 }
 
 // ---- histogram -----------------------------------------------------------
-// A tile is kTileSteps steps of 2048 elements (8 per thread of a 256-thread
-// block); a block takes tiles kGrid apart.  Per lane, 16 four-bit counters
-// in two registers (bins 0-7 and 8-15 of the warp's window, mode - 11 ..
-// mode + 4) take the 8 elements of a step; after each step they are spread
-// into byte counters (four registers), which are summed over the warp into
-// shared counters at the end of the tile (at most 64 counts per byte).
-// Exponents outside the window go to the shared counters at once.
+// One launch counts the exponents of a batch of tensors (jobs): their tiles
+// are numbered job after job, and block b takes tiles b, b + gridDim.x, and
+// so on.  A tile
+// is kTileSteps steps of 2048 elements (8 per thread of a 256-thread
+// block), loaded in two halves so that one half is in flight while the
+// other is counted: the tile's second half during the count of its first,
+// the next tile's first half during the count of its second.  Per lane, 16
+// four-bit counters in two registers (bins 0-7 and 8-15 of the warp's
+// window, mode - 11 .. mode + 4, the mode taken over the first elements of
+// the warp's lanes in the tile) take the 8 elements of a step; after each
+// step they are spread into byte counters (four registers), which are
+// summed over the warp at the end of the tile and added to the block's
+// shared counters, one bin per lane (at most 64 counts per byte).
+// Exponents outside the window go to the shared counters at once.  The
+// shared counters alternate between two arrays from tile to tile, so that
+// one barrier per tile separates a tile's adds from the reads of the tile
+// before.
 constexpr int kWindowBelow = 11;
 constexpr int kTileSteps = 8;
+constexpr int kHalfSteps = kTileSteps / 2;
 constexpr uint32_t kTile = kTileSteps * kPerCta;  // elements per tile (16384)
+constexpr int kHistJobs = 32;                     // jobs per histogram launch
 
-// byte j of counter register r holds window bin (r >> 1) * 8 + 2 j + (r & 1)
+struct HistJob {
+  const uint16_t *w;
+  uint64_t n;
+  uint64_t tile_base;        // its first tile's number in the launch
+  unsigned long long *hist;  // 256 counts, added to
+  unsigned long long *last;  // its last element (its codeword ends the stream), or null
+  uint16_t *tile_hist;       // 256 counts per tile (16 bits: at most 16384), or null
+  uint32_t vec;              // w is 16-byte aligned
+};
+
+struct HistBatch {
+  HistJob job[kHistJobs];
+  int count;
+  uint64_t tiles;  // of all its jobs
+};
+
+// The window's byte counters summed over the warp and added to the shared
+// counters h, lane b (0-15) taking window bin b.  Byte j of counter
+// register r holds bin (r >> 1) * 8 + 2 j + (r & 1): bin b is byte
+// (b & 7) >> 1 of register (b >> 3) * 2 + (b & 1).
 __device__ __forceinline__ void flush_window(uint32_t (&c)[4], int lo, uint32_t *h, int lane) {
+  uint32_t even[4], odd[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    // two 16-bit sums per word: 32 lanes x 64 < 2^16
-    const uint32_t even = __reduce_add_sync(0xFFFFFFFFu, c[r] & 0x00FF00FFu);
-    const uint32_t odd = __reduce_add_sync(0xFFFFFFFFu, (c[r] >> 8) & 0x00FF00FFu);
-    if (lane == 0) {
-      const uint32_t v[4] = {even & 0xFFFFu, odd & 0xFFFFu, even >> 16, odd >> 16};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int e = lo + (r >> 1) * 8 + 2 * j + (r & 1);
-        if (v[j] && e >= 0 && e < 256) atomicAdd(&h[e], v[j]);
-      }
-    }
+    // two 16-bit sums per word (bytes 0 and 2, or 1 and 3): 32 lanes x 64 < 2^16
+    even[r] = __reduce_add_sync(0xFFFFFFFFu, c[r] & 0x00FF00FFu);
+    odd[r] = __reduce_add_sync(0xFFFFFFFFu, (c[r] >> 8) & 0x00FF00FFu);
     c[r] = 0;
   }
+  const int b = lane & 15;
+  const int r = ((b >> 3) << 1) | (b & 1), j = (b & 7) >> 1;
+  const uint32_t ev = r == 0 ? even[0] : r == 1 ? even[1] : r == 2 ? even[2] : even[3];
+  const uint32_t od = r == 0 ? odd[0] : r == 1 ? odd[1] : r == 2 ? odd[2] : odd[3];
+  const uint32_t v = (((j & 1) ? od : ev) >> ((j & 2) ? 16 : 0)) & 0xFFFFu;
+  const int e = lo + b;
+  if (lane < 16 && v && e >= 0 && e < 256) atomicAdd(&h[e], v);
 }
 
 // One element whose exponent times 4 is e4: the window offset times 4 is
@@ -160,59 +192,85 @@ __device__ __forceinline__ void count8(const uint4 &v, uint32_t live, uint32_t l
   c[3] += (n_hi >> 4) & 0x0F0F0F0Fu;
 }
 
-// hist[e] += the count of exponent e (64-bit, device-wide); tile_hist, if
-// not null, gets each tile's 256 counts (16 bits; a tile has at most 16384
-// elements); *last, if not null, the last element (its codeword ends the
-// stream).
-__global__ void __launch_bounds__(kThreads) hist_kernel(const uint16_t *w, uint64_t n, bool vec,
-                                                        unsigned long long *hist,
-                                                        unsigned long long *last,
-                                                        uint16_t *tile_hist) {
-  if (last && blockIdx.x == 0 && threadIdx.x == 0 && n) *last = w[n - 1];
-  __shared__ uint32_t h[kThreads / 32][256];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int j = threadIdx.x; j < (kThreads / 32) * 256; j += kThreads) (&h[0][0])[j] = 0;
+// Steps s0 .. s0 + kHalfSteps - 1 of the tile at element t0 of a job
+__device__ __forceinline__ void load_half(uint4 (&v)[kHalfSteps], const HistJob &J, uint64_t t0,
+                                          int s0, uint32_t me) {
+#pragma unroll
+  for (int st = 0; st < kHalfSteps; ++st)
+    v[st] = load8(J.w, J.n, t0 + (uint64_t)(s0 + st) * kPerCta + me, J.vec != 0);
+}
+
+__device__ __forceinline__ void count_half(const uint4 (&v)[kHalfSteps], bool full, uint64_t t0,
+                                           int s0, uint64_t n, uint32_t me, uint32_t lo4,
+                                           uint32_t (&c)[4], uint32_t *h) {
+  if (full) {
+#pragma unroll
+    for (int st = 0; st < kHalfSteps; ++st) count8<true>(v[st], kPerThread, lo4, c, h);
+  } else {
+#pragma unroll
+    for (int st = 0; st < kHalfSteps; ++st)
+      count8<false>(v[st], live_of(t0 + (uint64_t)(s0 + st) * kPerCta + me, n), lo4, c, h);
+  }
+}
+
+// Per job: hist[e] += the count of exponent e (64-bit, device-wide);
+// tile_hist, if not null, each tile's 256 counts; last, if not null, the
+// last element.
+__global__ void __launch_bounds__(kThreads, 4) hist_kernel(const __grid_constant__ HistBatch hb) {
+  __shared__ uint32_t h[2][256];
+  static_assert(kThreads == 256, "a thread per exponent value");
+  const int lane = threadIdx.x & 31;
   const uint32_t me = threadIdx.x * kPerThread;
-  // the window: around the most frequent exponent among the warp's lanes'
-  // first elements of the block's first tile
-  int lo;
-  {
-    const uint64_t i = (uint64_t)blockIdx.x * kTile + warp * (kTile / 8) + lane * kPerThread;
-    const uint32_t key = i < n ? exponent(w[i]) : 256u;
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
-    const uint32_t best = __reduce_max_sync(0xFFFFFFFFu, ((uint32_t)__popc(peers) << 16) | key);
-    lo = (int)(best & 0x1FFu) - kWindowBelow;
+  if (blockIdx.x == 0 && threadIdx.x < (unsigned)hb.count) {
+    const HistJob &J = hb.job[threadIdx.x];
+    if (J.last && J.n) *J.last = J.w[J.n - 1];
   }
-  const uint32_t lo4 = (uint32_t)(4 * lo);
+  h[0][threadIdx.x] = 0;
+  h[1][threadIdx.x] = 0;
   __syncthreads();
-  uint32_t total = 0;  // exponent threadIdx.x over the block's tiles
-  for (uint64_t t0 = (uint64_t)blockIdx.x * kTile; t0 < n; t0 += (uint64_t)gridDim.x * kTile) {
+  uint64_t t = blockIdx.x;  // the grid has at most as many blocks as tiles
+  int ji = 0;
+  while (ji + 1 < hb.count && t >= hb.job[ji + 1].tile_base) ++ji;
+  uint4 va[kHalfSteps], vb[kHalfSteps];
+  load_half(va, hb.job[ji], (t - hb.job[ji].tile_base) * kTile, 0, me);
+  uint32_t total = 0;  // exponent threadIdx.x over the block's tiles of job ji
+  for (int p = 0;; p ^= 1) {
+    const HistJob &J = hb.job[ji];
+    const uint64_t t0 = (t - J.tile_base) * kTile;
+    const bool full = t0 + kTile <= J.n;
+    load_half(vb, J, t0, kHalfSteps, me);
+    const uint64_t tn = t + gridDim.x;
+    int jn = ji;
+    while (jn + 1 < hb.count && tn >= hb.job[jn + 1].tile_base) ++jn;
+    // the window: around the most frequent exponent among the lanes' first
+    // elements (256 for a lane past the end: no exponent)
+    int lo;
+    {
+      const uint32_t key = t0 + me < J.n ? exponent(va[0].x) : 256u;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
+      const uint32_t best = __reduce_max_sync(0xFFFFFFFFu, ((uint32_t)__popc(peers) << 16) | key);
+      lo = (int)(best & 0x1FFu) - kWindowBelow;
+    }
+    const uint32_t lo4 = (uint32_t)(4 * lo);
+    uint32_t *hp = h[p];
     uint32_t c[4] = {0, 0, 0, 0};
-    if (t0 + kTile <= n) {  // a whole tile: every load in flight at once
-      uint4 v[kTileSteps];
-#pragma unroll
-      for (int st = 0; st < kTileSteps; ++st) v[st] = load8(w, n, t0 + st * kPerCta + me, vec);
-#pragma unroll
-      for (int st = 0; st < kTileSteps; ++st) count8<true>(v[st], kPerThread, lo4, c, h[warp]);
-    } else {
-      for (int st = 0; st < kTileSteps; ++st) {
-        const uint64_t i = t0 + st * kPerCta + me;
-        count8<false>(load8(w, n, i, vec), live_of(i, n), lo4, c, h[warp]);
-      }
-    }
-    flush_window(c, lo, h[warp], lane);
+    count_half(va, full, t0, 0, J.n, me, lo4, c, hp);
+    if (tn < hb.tiles) load_half(va, hb.job[jn], (tn - hb.job[jn].tile_base) * kTile, 0, me);
+    count_half(vb, full, t0, kHalfSteps, J.n, me, lo4, c, hp);
+    flush_window(c, lo, hp, lane);
     __syncthreads();
-    uint32_t v = 0;
-#pragma unroll
-    for (int j = 0; j < kThreads / 32; ++j) {
-      v += h[j][threadIdx.x];
-      h[j][threadIdx.x] = 0;
-    }
-    if (tile_hist) tile_hist[(t0 / kTile) * 256 + threadIdx.x] = (uint16_t)v;
+    const uint32_t v = hp[threadIdx.x];
+    hp[threadIdx.x] = 0;
+    if (J.tile_hist) J.tile_hist[(t - J.tile_base) * 256 + threadIdx.x] = (uint16_t)v;
     total += v;
-    __syncthreads();
+    if (tn >= hb.tiles || jn != ji) {
+      if (total) atomicAdd(&J.hist[threadIdx.x], (unsigned long long)total);
+      total = 0;
+    }
+    if (tn >= hb.tiles) break;
+    t = tn;
+    ji = jn;
   }
-  if (total) atomicAdd(&hist[threadIdx.x], (unsigned long long)total);
 }
 
 // ---- phase 2 jobs --------------------------------------------------------
@@ -945,8 +1003,9 @@ df11_status check_begin_args(const uint16_t *d_bf16, uint64_t n, uint32_t C, uin
   return DF11_OK;
 }
 
-// phase 1's counts and last element of one tensor, in a block for the call
-constexpr uint64_t kHistBytes = (257 * sizeof(unsigned long long) + 255) & ~255ull;
+// phase 1's counts and last element of one tensor, one after another for
+// the call's tensors (as in the host staging array)
+constexpr uint64_t kHistWords = 257;
 
 // A stream per device for phase 1's copies of the counts, so that they do
 // not queue between the histogram kernels on the caller's stream (created
@@ -1008,29 +1067,9 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
   };
   const uint64_t hist_slots = resident(hist_kernel);
   std::lock_guard<std::mutex> lock(g_staging.mu);
-  auto *stage = static_cast<unsigned long long(*)[257]>(
-      g_staging.get(sizeof(unsigned long long[257]) * count));
+  auto *stage = static_cast<unsigned long long(*)[kHistWords]>(
+      g_staging.get(sizeof(unsigned long long[kHistWords]) * count));
   if (!stage) return DF11_ERR_NOMEM;
-  // per tensor: its kernel is done (caller's stream), its counts are back
-  // (side stream)
-  struct Events {
-    std::vector<cudaEvent_t> e;
-    ~Events() {
-      for (cudaEvent_t x : e)
-        if (x) cudaEventDestroy(x);
-    }
-  } ev;
-  ev.e.assign(2 * (size_t)count, nullptr);
-  for (auto &x : ev.e)
-    if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) return DF11_ERR_CUDA;
-  cudaEvent_t *done = ev.e.data(), *back = ev.e.data() + count;
-  if (scratch_alloc(&hblk, kHistBytes * count, s) != cudaSuccess) {
-    hblk = nullptr;
-    return fail(DF11_ERR_CUDA);
-  }
-  if (cudaMemsetAsync(hblk, 0, kHistBytes * count, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
-
-  // histograms, and each tensor's last element (its codeword ends the stream)
   for (int i = 0; i < count; ++i) {
     df11_gpu_build *h = hs[i] = new (std::nothrow) df11_gpu_build();
     if (!h) return fail(DF11_ERR_NOMEM);
@@ -1040,32 +1079,90 @@ df11_status df11_gpu_build_begin_batched(const uint16_t *const *d_bf16, const ui
     h->vec = ((uintptr_t)d_bf16[i] & 15) == 0;
     h->stream = s;
     h->tiles = (h->n + kTile - 1) / kTile;
+  }
+  // The launches: the jobs in order, at most kHistJobs per launch, and the
+  // shortest run of last jobs that holds a quarter of the tiles in a launch
+  // of its own, so that the codebooks of the jobs before it are computed
+  // while it runs.
+  uint64_t all_tiles = 0;
+  for (int i = 0; i < count; ++i) all_tiles += hs[i]->tiles;
+  int tail = count - 1;
+  uint64_t tail_tiles = hs[tail]->tiles;
+  while (tail > 0 && count - tail < kHistJobs && 4 * tail_tiles < all_tiles)
+    tail_tiles += hs[--tail]->tiles;
+  std::vector<int> cut;  // launch k takes jobs cut[k] .. cut[k + 1] - 1
+  for (int i = 0; i < tail; i += kHistJobs) cut.push_back(i);
+  cut.push_back(tail);
+  cut.push_back(count);
+  const int launches = (int)cut.size() - 1;
+  // per launch: its kernel is done (caller's stream), its counts are back
+  // (side stream)
+  struct Events {
+    std::vector<cudaEvent_t> e;
+    ~Events() {
+      for (cudaEvent_t x : e)
+        if (x) cudaEventDestroy(x);
+    }
+  } ev;
+  ev.e.assign(2 * (size_t)launches, nullptr);
+  for (auto &x : ev.e)
+    if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess)
+      return fail(DF11_ERR_CUDA);
+  cudaEvent_t *done = ev.e.data(), *back = ev.e.data() + launches;
+  const size_t hist_bytes = sizeof(unsigned long long) * kHistWords * count;
+  if (scratch_alloc(&hblk, hist_bytes, s) != cudaSuccess) {
+    hblk = nullptr;
+    return fail(DF11_ERR_CUDA);
+  }
+  if (cudaMemsetAsync(hblk, 0, hist_bytes, s) != cudaSuccess) return fail(DF11_ERR_CUDA);
+  unsigned long long *hist = static_cast<unsigned long long *>(hblk);
+  for (int i = 0; i < count; ++i) {
+    df11_gpu_build *h = hs[i];
     // the per-tile counts are written whole by the kernel
     if (scratch_alloc(&h->scratch1, round256(h->tiles * 512) + 256, s) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
     h->d_tile_hist = static_cast<uint16_t *>(h->scratch1);
-    unsigned long long *hist =
-        reinterpret_cast<unsigned long long *>(static_cast<char *>(hblk) + kHistBytes * i);
-    if (h->n) {
-      const unsigned grid = (unsigned)(h->tiles < hist_slots ? h->tiles : hist_slots);
-      hist_kernel<<<grid, kThreads, 0, s>>>(d_bf16[i], h->n, h->vec, hist, hist + 256,
-                                            h->d_tile_hist);
+  }
+  // histograms, and each tensor's last element (its codeword ends the stream)
+  for (int k = 0; k < launches; ++k) {
+    HistBatch hb;
+    std::memset(&hb, 0, sizeof(hb));
+    hb.count = cut[k + 1] - cut[k];
+    for (int j = 0; j < hb.count; ++j) {
+      const int i = cut[k] + j;
+      HistJob &J = hb.job[j];
+      J.w = d_bf16[i];
+      J.n = hs[i]->n;
+      J.tile_base = hb.tiles;
+      J.hist = hist + kHistWords * i;
+      J.last = hist + kHistWords * i + 256;
+      J.tile_hist = hs[i]->d_tile_hist;
+      J.vec = hs[i]->vec;
+      hb.tiles += hs[i]->tiles;
+    }
+    if (hb.tiles) {
+      const unsigned grid = (unsigned)(hb.tiles < hist_slots ? hb.tiles : hist_slots);
+      hist_kernel<<<grid, kThreads, 0, s>>>(hb);
       if (cudaGetLastError() != cudaSuccess) return fail(DF11_ERR_CUDA);
     }
-    if (cudaEventRecord(done[i], s) != cudaSuccess ||
-        cudaStreamWaitEvent(side, done[i], 0) != cudaSuccess ||
-        cudaMemcpyAsync(stage[i], hist, sizeof(stage[i]), cudaMemcpyDeviceToHost, side) !=
+    if (cudaEventRecord(done[k], s) != cudaSuccess ||
+        cudaStreamWaitEvent(side, done[k], 0) != cudaSuccess ||
+        cudaMemcpyAsync(stage[cut[k]], hist + kHistWords * cut[k],
+                        sizeof(stage[0]) * hb.count, cudaMemcpyDeviceToHost, side) !=
             cudaSuccess ||
-        cudaEventRecord(back[i], side) != cudaSuccess)
+        cudaEventRecord(back[k], side) != cudaSuccess)
       return fail(DF11_ERR_CUDA);
   }
 
-  // codebooks (host: 256 symbols each), each as soon as its counts are
-  // back, while the device counts the later tensors; the stream's length
-  // is the sum of count x code length
-  for (int i = 0; i < count; ++i) {
+  // codebooks (host: 256 symbols each), each as soon as its launch's
+  // counts are back, while the device counts the later tensors; the
+  // stream's length is the sum of count x code length
+  for (int i = 0, k = 0; i < count; ++i) {
     df11_gpu_build *h = hs[i];
-    if (cudaEventSynchronize(back[i]) != cudaSuccess) return fail(DF11_ERR_CUDA);
+    if (i == cut[k]) {
+      if (cudaEventSynchronize(back[k]) != cudaSuccess) return fail(DF11_ERR_CUDA);
+      ++k;
+    }
     uint64_t hist64[256];
     for (int k = 0; k < 256; ++k) hist64[k] = stage[i][k];
     h->longest = df11_internal::codebook(hist64, h->len, h->code, h->luts);
@@ -1254,24 +1351,46 @@ df11_status df11_gpu_build_finish_batched(df11_gpu_build *const *handles, int co
         st = DF11_ERR_CUDA;
     }
   }
-  if (st == DF11_OK && cudaStreamSynchronize(s) != cudaSuccess) st = DF11_ERR_CUDA;
+  // the parameters' host-side fields, while the handles exist
+  for (int i = 0; i < count && st == DF11_OK; ++i) fill_params(handles[i], &params[i]);
+  // the scratch is freed in stream order after this call's work; the frees
+  // are queued before the wait, so that their host time overlaps the kernels
+  if (blk) cudaFreeAsync(blk, s);
+  for (int i = 0; i < count; ++i) {
+    if (!handles[i]) continue;
+    handles[i]->stream = s;
+    df11_gpu_build_free(handles[i]);
+  }
+  // the maxima come back (the staging buffer is read until then in any case)
+  if (cudaStreamSynchronize(s) != cudaSuccess && st == DF11_OK) st = DF11_ERR_CUDA;
   for (int i = 0; i < count && st == DF11_OK; ++i) {
     unsigned int mx[3];
     std::memcpy(mx, stage + ctl_off + 8 + 12 * (size_t)i, sizeof(mx));
-    fill_params(handles[i], &params[i]);
     params[i].max_block_elems = mx[0];
     params[i].max_chunk_elems = mx[1];
     params[i].max_warp_elems = mx[2];
   }
-  if (st != DF11_OK) cudaStreamSynchronize(s);  // the staging buffer is read until then
   if (lock.owns_lock()) lock.unlock();
-  if (blk) cudaFreeAsync(blk, s);
-  for (int i = 0; i < count; ++i) {
-    if (!handles[i]) continue;
-    handles[i]->stream = s;  // frees follow this call's work
-    df11_gpu_build_free(handles[i]);
-  }
   return st;
+}
+
+uint64_t df11_gpu_build_layout(const df11_params *params, int count, uint64_t *offsets,
+                               uint64_t *sizes) {
+  if (!params || count < 0) return 0;
+  uint64_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    const df11_params &p = params[i];
+    const uint64_t chunks = (uint64_t)p.num_blocks * p.threads_per_block;
+    const uint64_t sz[7] = {chunks * p.chunk_bytes + 16, chunks * 5 / 8 + 16, chunks + 16,
+                            4ull * p.num_blocks + 4,     1024ull * p.num_luts, 256,
+                            (p.n + 15) / 16 * 16};
+    for (int j = 0; j < 7; ++j) {
+      if (offsets) offsets[7 * (size_t)i + j] = total;
+      if (sizes) sizes[7 * (size_t)i + j] = sz[j];
+      total += round256(sz[j] > 16 ? sz[j] : 16);
+    }
+  }
+  return total;
 }
 
 df11_status df11_gpu_build_finish(df11_gpu_build *h, const uint16_t *d_bf16, uint8_t *bitstream,
@@ -1335,17 +1454,20 @@ extern "C" df11_status df11_exponent_histogram(const uint16_t *d_bf16, uint64_t 
   if (cudaMemsetAsync(hd.addr, 0, sizeof(g_exponent_hist), s) != cudaSuccess) return DF11_ERR_CUDA;
   if (n) {
     const uint64_t tiles = (n + kTile - 1) / kTile, slots = resident(hist_kernel);
-    const bool vec = ((uintptr_t)d_bf16 & 15) == 0;
+    HistBatch hb;
+    std::memset(&hb, 0, sizeof(hb));
+    hb.count = 1;
+    hb.tiles = tiles;
+    hb.job[0].w = d_bf16;
+    hb.job[0].n = n;
+    hb.job[0].hist = hd.addr;  // no last element, no per-tile counts
+    hb.job[0].vec = ((uintptr_t)d_bf16 & 15) == 0;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(tiles < slots ? tiles : slots));
     cfg.blockDim = dim3(kThreads);
     cfg.stream = s;
-    unsigned long long *no_last = nullptr;
-    uint16_t *no_tiles = nullptr;
     // the launch's own status (not an earlier error of the calling thread)
-    if (cudaLaunchKernelEx(&cfg, hist_kernel, d_bf16, n, vec, hd.addr, no_last, no_tiles) !=
-        cudaSuccess)
-      return DF11_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, hist_kernel, hb) != cudaSuccess) return DF11_ERR_CUDA;
   }
   // straight into the caller's array (a DMA if the caller pinned it)
   if (cudaMemcpyAsync(hist, hd.addr, sizeof(g_exponent_hist), cudaMemcpyDeviceToHost, s) !=

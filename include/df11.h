@@ -414,9 +414,11 @@ typedef struct df11_gpu_build_out {
 /*
  * Both phases for `count` tensors at once (d_bf16[i], n[i]; params and
  * handles arrays of count, code_lengths count*256 bytes, all host arrays).
- * Phase 1 waits for each tensor's counts as they arrive (computing its
- * code while the device works on the later tensors) and synchronises the
- * stream once; phase 2 synchronises it once.  Same conventions as the
+ * Phase 1 counts up to 32 tensors per launch, the last quarter of the
+ * elements (the shortest run of last tensors that holds it) in a launch of
+ * its own, and waits for each launch's counts as they arrive (computing
+ * their codes while the device works on the later tensors); phase 2
+ * synchronises the stream once.  Same conventions as the
  * single-tensor calls; on an error in phase 1 no handle is returned (all
  * NULL), and phase 2 releases every handle in all cases.  The
  * single-tensor calls are these with count 1.
@@ -430,6 +432,19 @@ df11_status df11_gpu_build_finish_batched(df11_gpu_build *const *handles, int co
                                           const uint16_t *const *d_bf16,
                                           const df11_gpu_build_out *outs, df11_params *params,
                                           df11_stream_t stream);
+
+/*
+ * Where the phase-2 outputs of `count` tensors go in one device allocation
+ * (params as phase 1 filled them): tensor after tensor, each tensor's seven
+ * buffers in the order of df11_gpu_build_out with the sizes listed at
+ * df11_gpu_build_begin, every buffer at a 256-byte offset and given at
+ * least 16 bytes.  Writes buffer j of tensor i's byte offset to
+ * offsets[7 i + j] and its size to sizes[7 i + j] (either array may be
+ * NULL) and returns the allocation's size in bytes; 0 for a NULL params or
+ * a negative count.  Host only: touches no device.
+ */
+uint64_t df11_gpu_build_layout(const df11_params *params, int count, uint64_t *offsets,
+                               uint64_t *sizes);
 
 /* Release a phase-1 handle without running phase 2 (NULL is a no-op); its
  * scratch is freed in order on the stream phase 1 ran on, which must still

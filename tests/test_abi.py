@@ -135,6 +135,35 @@ def test_device_builder_host_validation():
         df11.compress_on_device(df11.torch.zeros(4, dtype=df11.torch.int16))
 
 
+def test_build_layout_places_every_buffer():
+    """df11_gpu_build_layout (host only): the seven buffers of each tensor
+    with the sizes the header lists, at 256-byte offsets in order, none
+    overlapping, none below 16 bytes, and the total covering the last."""
+    L = df11.lib()
+    ps = [_params(n=1000, num_blocks=1, num_luts=1),
+          _params(n=0, num_blocks=0, num_luts=1, chunk_bytes=24, threads_per_block=512),
+          _params(n=123_457, num_blocks=37, num_luts=4, chunk_bytes=12, threads_per_block=128)]
+    arr = (df11.Params * len(ps))(*ps)
+    offs = (ctypes.c_uint64 * (7 * len(ps)))()
+    sizes = (ctypes.c_uint64 * (7 * len(ps)))()
+    total = L.df11_gpu_build_layout(arr, len(ps), offs, sizes)
+    end = 0
+    for i, p in enumerate(ps):
+        chunks = p.num_blocks * p.threads_per_block
+        want = [chunks * p.chunk_bytes + 16, chunks * 5 // 8 + 16, chunks + 16,
+                4 * (p.num_blocks + 1), 4 * 256 * p.num_luts, 256, -(-p.n // 16) * 16]
+        for j, w in enumerate(want):
+            o, sz = offs[7 * i + j], sizes[7 * i + j]
+            assert sz == w
+            assert o % 256 == 0 and o >= end
+            end = o + max(sz, 16)
+    assert end <= total < end + 256
+    assert L.df11_gpu_build_layout(arr, len(ps), None, None) == total
+    assert L.df11_gpu_build_layout(arr, 0, None, None) == 0
+    assert L.df11_gpu_build_layout(None, 3, None, None) == 0
+    assert L.df11_gpu_build_layout(arr, -1, None, None) == 0
+
+
 def test_batched_builder_host_validation():
     """The batched builder phases reject bad arguments before any CUDA
     call, and clear the handles they would return."""

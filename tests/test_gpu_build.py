@@ -182,6 +182,40 @@ def test_batched_builds_equal_single_builds():
             _decodes_to(d, w_np)
 
 
+def test_many_tensors_in_one_call():
+    """Forty tensors in one call, more than one histogram launch takes (32),
+    with more tiles (16384 elements) than the histogram grid has blocks, so
+    that blocks cross from one tensor to the next: sizes from empty to two
+    million elements, some views that start off a 16-byte boundary, and
+    tensors of other exponent spreads.  Each must equal the host builder's
+    output byte for byte."""
+    rng = np.random.default_rng(7)
+    bits = []
+    for i in range(40):
+        kind = i % 5
+        if kind == 0:
+            n = int(rng.integers(0, 3))
+        elif kind == 1:
+            n = int(rng.integers(1, 20000))
+        else:
+            n = int(rng.integers(200_000, 2_000_000))
+        std = float(rng.choice([0.02, 0.5, 3.0]))
+        w = workloads.gaussian_bf16(n + 5, std, 100 + i, device="cuda")
+        bits.append(w[5:] if i % 3 == 0 else w[:n])
+    tiles = sum((b.numel() + 16383) // 16384 for b in bits)
+    assert tiles > 148 * 4  # more tiles than the histogram grid's blocks
+    ds = df11.compress_on_device_batched(bits, 24, 256)
+    torch.cuda.synchronize()
+    for b, d in zip(bits, ds):
+        w_np = workloads.as_numpy_u16(b.cpu())
+        h = df11.compress(w_np, 24, 256)
+        for f, _ in df11.Params._fields_:
+            assert getattr(d.params, f) == getattr(h.params, f), f
+        for f in _BUFFERS:
+            assert np.array_equal(getattr(d, f).cpu().numpy().view(np.uint8), _host_bytes(h, f)), f
+    _decodes_to(ds[2], workloads.as_numpy_u16(bits[2].cpu()))
+
+
 # --- randomised: skewed exponent histograms, every valid chunk size ----------
 
 from hypothesis import given, settings, strategies as st  # noqa: E402
