@@ -138,3 +138,27 @@ def test_flush_rule():
     assert not bench.flush_wanted("auto", 646_000_000)       # the block: larger than L2
     assert bench.flush_wanted("on", 646_000_000)
     assert not bench.flush_wanted("off", 3_500_000)
+
+
+def test_build_hist_launches_follows_the_builder_rule():
+    """bench.build_hist_launches (the launch count the build line claims):
+    tensors in order, at most 32 per histogram launch, the shortest run of
+    last tensors holding a quarter of the tiles in a launch of its own, and
+    no kernel for a launch of empty tensors."""
+    t = bench.BUILD_TILE
+    block = [4096 * 4096, 1024 * 4096, 1024 * 4096, 4096 * 4096] + [12288 * 4096] * 3
+    assert bench.build_hist_launches(block) == 2      # six tensors, then the last
+    assert bench.build_hist_launches([]) == 0
+    assert bench.build_hist_launches([0, 0, 0]) == 0  # nothing to count
+    assert bench.build_hist_launches([1]) == 1
+    assert bench.build_hist_launches([t] * 4) == 2    # the last tile is a quarter
+    assert bench.build_hist_launches([t] * 8) == 2    # the last two
+    # forty equal tensors: the last ten in their own launch, thirty before
+    assert bench.build_hist_launches([10 * t] * 40) == 2
+    # a hundred: the last 25 in their own launch, the 75 before in three
+    assert bench.build_hist_launches([t] * 100) == 4
+    # at most 32 in the last launch: 32 of 200, the 168 before in six
+    assert bench.build_hist_launches([t] * 200) == 7
+    # a first launch of empty tensors runs no kernel
+    assert bench.build_hist_launches([0, 0, 0, t]) == 1
+    assert bench.build_hist_launches([0] * 5 + [t] * 20) == 2
